@@ -1,0 +1,480 @@
+#!/usr/bin/env python3
+"""Benchmark of the SIGE sparse-conv hot path on B200.
+
+Workload (one step = one pass of the whole hot path over one edit): the
+DDPM-style residual block at 256x256, C=128, bf16 storage / fp32 accumulation,
+with a ~1.2% edit made of 1-3 seeded discs:
+    mask   : difference mask of x_orig vs x_edit -> 8x8 tile list (dilate 1)
+    conv1  : gather(GN1 + SiLU) -> 3x3 conv -> scatter(+bias) into cached y1
+    conv2  : gather(GN2 + SiLU) -> 3x3 conv -> scatter(+bias +x_edit) into cached out
+The caches (y1 and out of the original image, GroupNorm statistics of the
+original) are computed once beforehand by the same library's dense conv, as
+the engine pre-computes the original activations.
+
+Timing: each call is captured in its own CUDA graph; every step starts with a
+256 MiB write that flushes the 126 MB L2, then CUDA events on the launching
+stream bracket the three replays.  W warm-up steps, then exactly K timed
+steps, barrier + synchronize on both sides, max over ranks.  More GPUs run
+independent replicas (one edit each, no collective).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {sige,reference}]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-conv layer latency (us) & % of roofline at 1.2% edit area vs dense conv"
+WORKLOAD = "DDPM res block 256x256 C=128 bf16, GN(32)+SiLU -> conv3x3 -> GN+SiLU -> conv3x3 + residual, 8x8 tiles, 1.2% edit"
+H = W = 256
+C = 128
+BLOCK = 8
+THRESH = 1e-3
+FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {**FALLBACK_PEAKS, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def src_sha(relpath):
+    with open(os.path.join(ROOT, relpath), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, when it was taken
+    on the current source of that kernel; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel)
+    if not d:
+        return None
+    try:
+        if src_sha(d["source"]) != d["source_sha"]:
+            return None
+    except OSError:
+        return None
+    return float(d["bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed loop runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in out.strip().splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------------ workload
+
+def make_workload(seed, dev):
+    import spatially_sparse_incremental_b200 as sige
+    from spatially_sparse_incremental_b200 import inputs
+    blk = inputs.make_cfg3(seed, H=H, W=W, C=C, area=0.012, block=BLOCK)
+    d = {k: getattr(blk, k).to(dev) for k in ("x_orig", "x_edit", "w1", "b1", "w2", "b2", "g1", "be1", "g2", "be2")}
+    cd = sige.conv_desc(3, 1, 1, C, C, BLOCK)
+    cap = (H // BLOCK) * (W // BLOCK)
+    # cache of the original image (computed once, untimed)
+    gs1, gh1 = sige.sige_groupnorm_affine(d["x_orig"], 32, d["g1"], d["be1"])
+    y1 = sige.sige_dense_conv(d["x_orig"], d["w1"], d["b1"], cd, gn_scale=gs1, gn_shift=gh1, silu=True)
+    gs2, gh2 = sige.sige_groupnorm_affine(y1, 32, d["g2"], d["be2"])
+    out = sige.sige_dense_conv(y1, d["w2"], d["b2"], cd, gn_scale=gs2, gn_shift=gh2, silu=True, residual=d["x_orig"])
+    idx = torch.zeros((cap, 2), dtype=torch.int32, device=dev)
+    cnt = torch.zeros(1, dtype=torch.int32, device=dev)
+    mask_ws = sige.zeros_workspace(sige.sige_reduce_mask_workspace_bytes(sige.tensor_desc(d["x_orig"]),
+                                                                         [(H, W, BLOCK, cap)]), dev)
+    conv_ws = sige.zeros_workspace(sige.sige_conv_workspace_bytes(cd, 1, cap, H, W), dev)
+    d.update(cd=cd, cap=cap, gs1=gs1, gh1=gh1, gs2=gs2, gh2=gh2, y1=y1, out=out, idx=idx, cnt=cnt,
+             mask_ws=mask_ws, conv_ws=conv_ws, blk=blk)
+    return d
+
+
+def step_calls(d, stream=None):
+    """The three hot-path calls of one step, as closures (for graph capture)."""
+    import spatially_sparse_incremental_b200 as sige
+
+    def mask():
+        sige.sige_reduce_mask(d["x_orig"], d["x_edit"], THRESH, [(H, W, BLOCK, d["cap"])], 1, idx=d["idx"],
+                              counts=d["cnt"], workspace=d["mask_ws"], stream=stream)
+
+    def conv1():
+        sige.sige_conv_fused(d["x_edit"], d["w1"], d["b1"], d["cd"], d["idx"], d["cnt"], d["cap"], d["y1"],
+                             d["gs1"], d["gh1"], silu=True, workspace=d["conv_ws"], stream=stream)
+
+    def conv2():
+        sige.sige_conv_fused(d["y1"], d["w2"], d["b2"], d["cd"], d["idx"], d["cnt"], d["cap"], d["out"],
+                             d["gs2"], d["gh2"], silu=True, residual=d["x_edit"], workspace=d["conv_ws"],
+                             stream=stream)
+    return {"mask": mask, "conv1": conv1, "conv2": conv2}
+
+
+def dense_calls(d, stream=None):
+    import spatially_sparse_incremental_b200 as sige
+    y1d = torch.empty_like(d["y1"])
+    outd = torch.empty_like(d["out"])
+
+    def dense1():
+        sige.sige_dense_conv(d["x_edit"], d["w1"], d["b1"], d["cd"], y=y1d, gn_scale=d["gs1"], gn_shift=d["gh1"],
+                             silu=True, workspace=d["conv_ws"], stream=stream)
+
+    def dense2():
+        sige.sige_dense_conv(y1d, d["w2"], d["b2"], d["cd"], y=outd, gn_scale=d["gs2"], gn_shift=d["gh2"],
+                             silu=True, residual=d["x_edit"], workspace=d["conv_ws"], stream=stream)
+    return {"dense1": dense1, "dense2": dense2}
+
+
+def capture(fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def timed_graph_steps(graphs, flush, steps, stream):
+    """Per step: L2 flush, then events around each graph replay.  Returns per-
+    call lists of durations (ms) and the per-step totals."""
+    names = list(graphs)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for k in range(steps):
+            flush.zero_()
+            ev[k][0].record(stream)
+            for i, nm in enumerate(names):
+                graphs[nm].replay()
+                ev[k][i + 1].record(stream)
+    stream.synchronize()
+    per = {nm: [ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps)] for i, nm in enumerate(names)}
+    tot = [ev[k][0].elapsed_time(ev[k][-1]) for k in range(steps)]
+    return per, tot
+
+
+# ------------------------------------------------------------------ roofline
+
+def conv_work(n_tiles, residual):
+    """Algorithmic FLOPs and bytes of one fused sparse conv launch on this workload."""
+    macs = n_tiles * BLOCK * BLOCK * C * C * 9
+    bin_ = BLOCK + 2
+    gather = n_tiles * bin_ * bin_ * C * 2
+    scatter = n_tiles * BLOCK * BLOCK * C * 2 * (2 if residual else 1)
+    weights = C * 9 * C * 2 + C * 4
+    return 2 * macs, gather + scatter + weights
+
+
+def mask_work(n_tiles):
+    return 2 * H * W * C * 2 + n_tiles * 8 + 4
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline only)
+
+def oracle_band_steps(seed, nbands, min_seconds, max_steps, threads, exact=False):
+    """Time the CPU oracle on a bounded sample: each sample is one horizontal
+    band (H/nbands rows, full width) of the workload, run as its own image:
+    pixel mask + tile list, then both sparse convs of the res block on the
+    band's tiles.  Returns (seconds per full step, samples, seconds)."""
+    import oracle
+    from spatially_sparse_incremental_b200 import inputs
+    oracle.set_threads(threads)
+    blk = inputs.make_cfg3(seed, H=H, W=W, C=C, area=0.012, block=BLOCK)
+    g1 = oracle.gn_affine(blk.x_orig, 32, blk.g1, blk.be1)
+    g2 = oracle.gn_affine(blk.x_orig, 32, blk.g2, blk.be2)   # stand-in statistics (timing only)
+    rows = H // nbands
+    gen = torch.Generator().manual_seed(seed)
+    y1c = torch.randn(1, rows, W, C, generator=gen).to(torch.bfloat16)
+    outc = torch.randn(1, rows, W, C, generator=gen).to(torch.bfloat16)
+    times = []
+    t_start = time.perf_counter()
+    k = 0
+    while k < max_steps and (exact or time.perf_counter() - t_start < min_seconds or k < nbands):
+        r0 = (k % nbands) * rows
+        xo = blk.x_orig[:, r0:r0 + rows].contiguous()
+        xe = blk.x_edit[:, r0:r0 + rows].contiguous()
+        t0 = time.perf_counter()
+        idx = oracle.reduce_mask(xo, xe, THRESH, [(rows, W, BLOCK)], 1)[0]
+        y1 = oracle.sparse_conv(xe, blk.w1, blk.b1, idx, y1c, block=BLOCK, gn=g1, silu=True)
+        oracle.sparse_conv(y1, blk.w2, blk.b2, idx, outc, block=BLOCK, gn=g2, silu=True, residual=xe)
+        times.append(time.perf_counter() - t0)
+        k += 1
+    return float(np.mean(times)) * nbands, k, time.perf_counter() - t_start
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ arms
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    cores = host_cores()
+    nbands = 32
+    # warm-up samples, then exactly K samples (each one band of the workload)
+    oracle_band_steps(args.seed, nbands, 0.0, args.warmup, cores, exact=True)
+    per_step_s, n, secs = oracle_band_steps(args.seed, nbands, 0.0, args.steps, cores, exact=True)
+    us = per_step_s * 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us, "unit": "us", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "H": H, "W": W, "C": C, "block": BLOCK, "edit_area": 0.012},
+        "cpu_baseline": {"value": us, "unit": "us", "cores": cores, "kind": "oracle",
+                         "sample": f"each step = one {H // nbands}-row band of the 256x256 image run as its own "
+                                   f"image (mask + tile list + both sparse convs); value scaled x{nbands} to a full "
+                                   f"step; {n} samples in {secs:.1f} s"},
+        "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_sige(args):
+    import spatially_sparse_incremental_b200 as sige
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if ws > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+
+    d = make_workload(args.seed + rank, dev)
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device=dev)
+    calls = step_calls(d, stream)
+    # eager warm-up of every call once (also counts kernels per call)
+    with torch.cuda.stream(stream):
+        launches = {}
+        for nm, fn in calls.items():
+            before = sige.sige_launch_count()
+            fn()
+            launches[nm] = sige.sige_launch_count() - before
+    stream.synchronize()
+    n_tiles = int(d["cnt"].item())
+    graphs = {nm: capture(fn, stream) for nm, fn in calls.items()}
+    dgraphs = {nm: capture(fn, stream) for nm, fn in dense_calls(d, stream).items()}
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream.synchronize()
+
+    # warm-up steps
+    timed_graph_steps(graphs, flush, args.warmup, stream)
+
+    def barrier():
+        if ws > 1:
+            torch.distributed.barrier()
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index)
+    per, tot = timed_graph_steps(graphs, flush, args.steps, stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    step_ms = float(np.mean(tot))
+    kern_ms = {nm: float(np.mean(v)) for nm, v in per.items()}
+    if ws > 1:
+        t = torch.tensor([step_ms] + [kern_ms[k] for k in kern_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        step_ms = float(t[0])
+        kern_ms = {k: float(t[i + 1]) for i, k in enumerate(kern_ms)}
+
+    # dense comparison (same launch mode, L2 flushed)
+    dper, dtot = timed_graph_steps(dgraphs, flush, max(10, min(args.steps, 50)), stream)
+    dense_ms = {nm: float(np.mean(v)) for nm, v in dper.items()}
+
+    # end to end through the public API: pinned host input, host output
+    host_in = d["x_edit"].cpu().pin_memory()
+    host_out = torch.empty(d["out"].shape, dtype=d["out"].dtype).pin_memory()
+    dev_in = torch.empty_like(d["x_edit"])
+    d_e2e = dict(d, x_edit=dev_in)
+    ecalls = step_calls(d_e2e, stream)
+    e2e_times = []
+    for k in range(args.warmup + args.e2e_steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            e0.record(stream)
+            dev_in.copy_(host_in, non_blocking=True)
+            for fn in ecalls.values():
+                fn()
+            host_out.copy_(d["out"], non_blocking=True)
+            e1.record(stream)
+        stream.synchronize()
+        if k >= args.warmup:
+            e2e_times.append(e0.elapsed_time(e1))
+    e2e_ms = float(np.mean(e2e_times))
+    if ws > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+
+    # roofline of the dominant kernel
+    work = {"mask": ("hbm", None, mask_work(n_tiles)),
+            "conv1": (None,) + conv_work(n_tiles, False),
+            "conv2": (None,) + conv_work(n_tiles, True)}
+    dom = max(kern_ms, key=kern_ms.get)
+    kernel_name = {"mask": "k_mask_reduce", "conv1": "conv", "conv2": "conv"}[dom]
+    if dom == "mask":
+        nbytes = work["mask"][2]
+        ach = nbytes / (kern_ms[dom] * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "traffic": ncu_traffic("k_mask_reduce"),
+                "kernel": kernel_name, "algorithmic_bytes": nbytes,
+                "peak_source": f"{peaks['source']} hbm_gbs"}
+    else:
+        _, flops, nbytes = work[dom]
+        t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+        t_bw = nbytes / (peaks["hbm_gbs"] * 1e9)
+        if t_tc >= t_bw:
+            ach = flops / (kern_ms[dom] * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": ach / peaks["bf16_tflops"], "peak_source": f"{peaks['source']} bf16_tflops (burst)"}
+        else:
+            ach = nbytes / (kern_ms[dom] * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": ach / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} hbm_gbs"}
+        roof.update(traffic=ncu_traffic("k_conv_tc" if sige.sige_conv_path(d["cd"], torch.bfloat16) == 1
+                                        else "k_conv_simt"), kernel=kernel_name,
+                    algorithmic_bytes=nbytes, algorithmic_flops=flops)
+    # step roofline: every call at its own bound
+    t_roof = mask_work(n_tiles) / (peaks["hbm_gbs"] * 1e9)
+    for res in (False, True):
+        f, b = conv_work(n_tiles, res)
+        t_roof += max(f / (peaks["bf16_tflops"] * 1e12), b / (peaks["hbm_gbs"] * 1e9))
+    sparse_conv_ms = kern_ms["conv1"] + kern_ms["conv2"]
+    dense_conv_ms = dense_ms["dense1"] + dense_ms["dense2"]
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cores = host_cores()
+        per_step_s, n, secs = oracle_band_steps(args.seed, 32, args.cpu_seconds, 100000, cores)
+        cpu = {"value": per_step_s * 1e6, "unit": "us", "cores": cores, "kind": "oracle",
+               "sample": f"{n} samples, each one 8-row band (1/32) of the 256x256 workload run as its own image "
+                         f"(mask + tile list + both sparse convs), scaled x32 to a full step; {secs:.1f} s of CPU work"}
+
+    line = {
+        "metric": METRIC, "value": step_ms * 1e3, "unit": "us", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "H": H, "W": W, "C": C, "block": BLOCK, "edit_area": 0.012,
+                   "active_tiles": n_tiles, "tile_fraction": n_tiles / d["cap"],
+                   "l2": "flushed (256 MiB write) before every step", "launch": "one CUDA graph per call",
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+        "breakdown_us": {k: v * 1e3 for k, v in kern_ms.items()},
+        "dense_conv_us": dense_conv_ms * 1e3, "sparse_conv_us": sparse_conv_ms * 1e3,
+        "speedup_vs_dense_conv": dense_conv_ms / sparse_conv_ms,
+        "step_roofline_frac": t_roof / (step_ms * 1e-3),
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_ms * 1e3, "unit": "us", "h2d_bytes_per_step": host_in.numel() * host_in.element_size(),
+                "d2h_bytes_per_step": host_out.numel() * host_out.element_size(),
+                "api": "sige_reduce_mask + 2x sige_conv_fused, eager, pinned host buffers"},
+        "gpu_launches": sum(launches.values()) * args.steps,
+        "clocks": clocks,
+        "conv_path": "tcgen05" if sige.sige_conv_path(d["cd"], torch.bfloat16) == 1 else "cuda-core",
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for g in list(graphs.values()) + list(dgraphs.values()):
+        del g
+    graphs.clear()
+    dgraphs.clear()
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["sige", "reference"], default="sige")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_sige(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

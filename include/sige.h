@@ -1,0 +1,220 @@
+/*
+ * sige.h -- C ABI of the B200 spatially sparse incremental convolution.
+ *
+ * The method (SIGE, "Efficient Spatially Sparse Inference for Conditional
+ * GANs and Diffusion Models"): the activations of the original image are
+ * computed once and cached; for an edited image the engine compares the
+ * original and edited inputs to get a difference mask (mer.dev notes on SIGE,
+ * section 3 "Method"), downsamples that mask to each scale, dilates it and
+ * selects tiles (section 3.2 "Sparse Engine SIGE"), reduces it to active-block
+ * indices, gathers the active blocks with their halo from the edited
+ * activation, stacks them on the batch axis, runs the layer F_l on the stack
+ * and scatters the output blocks back into the cached F_l(A_original)
+ * (SIGE project page, "Overview").
+ *
+ * Conventions for every call
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no device memory and keeps no state between calls.
+ *   - Every call is asynchronous on `stream` (NULL = legacy default stream),
+ *     launches exactly one kernel, and returns after enqueueing it.  Only
+ *     sige_get_error() synchronises.
+ *   - Host-side checks run before any launch: invalid arguments return
+ *     SIGE_ERR_INVALID_ARG, shapes the kernels do not cover return
+ *     SIGE_ERR_UNSUPPORTED, a failed launch returns SIGE_ERR_CUDA.  Nothing
+ *     is enqueued in those cases.
+ *   - Errors found on the device (an index list longer than its capacity, a
+ *     bounded wait that expired) never trap: the kernel records the first one
+ *     in the 256-byte header at the start of the call's workspace and finishes
+ *     without touching memory it cannot vouch for.  sige_get_error() reads and
+ *     clears that record.
+ *   - Activations are NHWC.  Conv weights are [C_out][k][k][C_in] (KRSC) in
+ *     the activation dtype.  Biases and GroupNorm scale/shift are float32.
+ *   - Tile lists are int32 pairs (h0, w0): the output-pixel origin of each
+ *     active b x b tile, in row-major tile order.  Counts live on the device,
+ *     so no call needs the host to know how many tiles are active.
+ */
+#ifndef SIGE_H
+#define SIGE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle as cudaStream_t. */
+typedef struct CUstream_st *sige_stream_t;
+
+typedef enum {
+    SIGE_OK = 0,
+    SIGE_ERR_INVALID_ARG = -1,   /* NULL pointer, bad size, inconsistent descriptors */
+    SIGE_ERR_UNSUPPORTED = -2,   /* valid but not covered by the kernels (dtype, layout, C % 8) */
+    SIGE_ERR_CUDA = -3,          /* no device, launch or runtime failure */
+    SIGE_ERR_CAPACITY = -4,      /* device: more active tiles than the list capacity */
+    SIGE_ERR_TIMEOUT = -5,       /* device: a bounded wait expired */
+    SIGE_ERR_WORKSPACE = -6      /* workspace missing or smaller than required */
+} sige_status;
+
+typedef enum { SIGE_U8 = 0, SIGE_F32 = 1, SIGE_BF16 = 2 } sige_dtype;
+typedef enum { SIGE_NHWC = 0, SIGE_NCHW = 1 } sige_layout;
+
+/* A dense activation tensor.  `layout` NCHW is accepted only by
+ * sige_reduce_mask (images such as 3 x H x W uint8). */
+typedef struct {
+    int32_t n, h, w, c;
+    int32_t dtype;   /* sige_dtype */
+    int32_t layout;  /* sige_layout */
+} sige_tensor_desc;
+
+/* One convolution layer F_l.  Output size Ho = (H + 2 pad - kernel)/stride + 1.
+ * `block` is the output tile edge b; each gathered input block is
+ * b_in = (b - 1) * stride + kernel pixels wide, so neighbouring blocks of a
+ * 3x3 stride-1 conv overlap by 2 pixels (SIGE project page, "Overview"). */
+typedef struct {
+    int32_t kernel, stride, pad;
+    int32_t c_in, c_out;
+    int32_t block;
+} sige_conv_desc;
+
+/* One scale of the mask reduction: the grid (h, w) the mask is downsampled
+ * to, the tile edge at that scale and the capacity (pairs) of its list. */
+typedef struct {
+    int32_t h, w, block, capacity;
+} sige_scale_desc;
+
+#define SIGE_MAX_SCALES 8
+#define SIGE_WORKSPACE_HEADER_BYTES 256
+
+/* ------------------------------------------------------------------ calls */
+
+/* (1) Difference mask -> per-scale active-tile lists.
+ * mer.dev notes on SIGE, section 3 "Method" (difference mask between the
+ * original and edited inputs) and section 3.2 "Sparse Engine SIGE" (downsample
+ * to several scales, dilate, select tiles); SIGE project page, "Overview"
+ * (reduce the mask to active block indices).
+ *
+ * Pixel (y, x) is edited when, for some batch item, max_c |a_edit - a_orig| >
+ * threshold, the difference taken in float32.  For scale s the mask is
+ * OR-downsampled to (scales[s].h, scales[s].w) (in->h, in->w must be integer
+ * multiples of them), dilated by `dilate` tiles of scales[s].block pixels,
+ * cut into block x block tiles anchored at (0, 0) and clipped at the border;
+ * every tile holding a set pixel is listed.
+ *   a_orig, a_edit : device, `in` shape/dtype/layout (u8, f32 or bf16; NHWC or NCHW)
+ *   idx            : device int32 pairs; scale s's list starts at pair offset
+ *                    sum_{t<s} scales[t].capacity, row-major tile order
+ *   counts         : device int32[n_scales], the number of active tiles (may
+ *                    exceed the capacity: then only `capacity` pairs are written
+ *                    and the device error SIGE_ERR_CAPACITY is recorded)
+ *   workspace      : device, >= sige_reduce_mask_workspace_bytes(), zero-filled
+ *                    before its first use; each call leaves it zero-filled
+ *                    apart from a recorded device error.  One workspace per
+ *                    stream: calls sharing one must not overlap on the GPU. */
+size_t sige_reduce_mask_workspace_bytes(const sige_tensor_desc *in, int32_t n_scales,
+                                        const sige_scale_desc *scales);
+int sige_reduce_mask(const void *a_orig, const void *a_edit, const sige_tensor_desc *in,
+                     float threshold, int32_t dilate, int32_t n_scales,
+                     const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
+                     void *workspace, size_t workspace_bytes, sige_stream_t stream);
+
+/* (2) Gather the active blocks, with halo, from the edited activation and
+ * stack them on the batch axis (SIGE project page, "Overview").
+ *   blocks[t][n][hh][ww][c] = T(x[n][h0*s - p + hh][w0*s - p + ww][c]),
+ *   hh, ww < b_in, zero outside the image (the conv's zero padding), with
+ *   T(v) = v, or v*gn_scale[n][c] + gn_shift[n][c] when gn_scale != NULL,
+ *   followed by SiLU v/(1+exp(-v)) when silu != 0; computed in float32 and
+ *   stored in x's dtype.
+ *   x        : device, NHWC f32 or bf16, xd->c == cd->c_in, C % 8 == 0 for bf16, % 4 for f32
+ *   idx/count: the list of one scale from sige_reduce_mask; min(*count, capacity) tiles
+ *   gn_scale, gn_shift : device float32 [N][C_in] or both NULL
+ *   blocks   : device, [capacity][N][b_in][b_in][C_in] in x's dtype; entries
+ *              past the count are left untouched. */
+int sige_gather(const void *x, const sige_tensor_desc *xd, const sige_conv_desc *cd,
+                const int32_t *idx, const int32_t *count, int32_t capacity,
+                const float *gn_scale, const float *gn_shift, int32_t silu, void *blocks,
+                sige_stream_t stream);
+
+/* (3) Run the layer F_l on the stacked blocks: a valid convolution of each
+ * block, no bias (SIGE project page, "Overview").
+ *   out[t][n][i][j][o] = sum_{r,c,ci} W[o][r][c][ci] * blocks[t][n][i*s+r][j*s+c][ci]
+ *   blocks     : device, [capacity][batch][b_in][b_in][C_in] in `dtype` (f32 or bf16)
+ *   weight     : device, [C_out][k][k][C_in] in `dtype`
+ *   out_blocks : device float32 [capacity][batch][b][b][C_out]
+ *   workspace  : device, >= sige_conv_workspace_bytes(), zero-filled before
+ *                first use and left zero-filled (split-K partial sums).
+ * bf16 runs on the tensor cores (bf16 operands, float32 accumulation);
+ * f32 runs on the CUDA cores in float32. */
+int sige_sparse_conv(const void *blocks, const sige_conv_desc *cd, int32_t dtype, int32_t batch,
+                     const void *weight, const int32_t *count, int32_t capacity, float *out_blocks,
+                     void *workspace, size_t workspace_bytes, sige_stream_t stream);
+
+/* (4) Scatter the output blocks into the cached output, in place (SIGE
+ * project page, "Overview": scatter back into F_l(A_original)).
+ *   y[n][h0+i][w0+j][o] = round(out[t][n][i][j][o] + bias[o] + residual[n][h0+i][w0+j][o])
+ * for every in-image pixel of the listed tiles, rounded once to y's dtype
+ * (ties to even).  Every other byte of y is left untouched.
+ *   bias     : device float32 [C_out] or NULL
+ *   residual : device, same shape/dtype as y, or NULL
+ *   y        : device NHWC f32 or bf16 holding F_l(A_original) on entry */
+int sige_scatter(const float *out_blocks, const sige_conv_desc *cd, const int32_t *idx,
+                 const int32_t *count, int32_t capacity, const float *bias, const void *residual,
+                 void *y, const sige_tensor_desc *yd, sige_stream_t stream);
+
+/* (5) Gather (+GroupNorm affine +SiLU), conv and scatter (+bias +residual) of
+ * one layer in a single launch; the result equals (2) -> (3) -> (4) without
+ * the stacked blocks or output blocks ever reaching memory.  Arguments as in
+ * those calls. */
+int sige_conv_fused(const void *x, const sige_tensor_desc *xd, const void *weight,
+                    const float *bias, const sige_conv_desc *cd, const int32_t *idx,
+                    const int32_t *count, int32_t capacity, const float *gn_scale,
+                    const float *gn_shift, int32_t silu, const void *residual, void *y,
+                    const sige_tensor_desc *yd, void *workspace, size_t workspace_bytes,
+                    sige_stream_t stream);
+
+/* The same layer on every tile of the output: the dense conv that fills the
+ * cache F_l(A_original) and the dense baseline the sparse path is compared
+ * with.  y is fully written. */
+int sige_dense_conv(const void *x, const sige_tensor_desc *xd, const void *weight,
+                    const float *bias, const sige_conv_desc *cd, const float *gn_scale,
+                    const float *gn_shift, int32_t silu, const void *residual, void *y,
+                    const sige_tensor_desc *yd, void *workspace, size_t workspace_bytes,
+                    sige_stream_t stream);
+
+/* GroupNorm of the cached ORIGINAL activation folded into a per-channel
+ * affine: scale[n][c] = gamma[c]/sqrt(var + eps), shift[n][c] = beta[c] -
+ * mean*scale, mean and biased variance over H, W and the C/groups channels of
+ * each group.  Computed once with the cache; the pages mention no
+ * normalisation, and taking the statistics from the original keeps every op
+ * of the sparse layer local.
+ *   x : device NHWC f32 or bf16;  gamma, beta : device float32 [C];
+ *   scale, shift : device float32 [N][C] */
+int sige_groupnorm_affine(const void *x, const sige_tensor_desc *xd, int32_t groups,
+                          const float *gamma, const float *beta, float eps, float *scale,
+                          float *shift, sige_stream_t stream);
+
+/* ------------------------------------------------------------ utilities */
+
+/* Workspace bytes for sige_sparse_conv / sige_conv_fused / sige_dense_conv
+ * with this layer, batch and list capacity (capacity is ignored for the dense
+ * call, which uses the full tile grid of an output of `out_h` x `out_w`). */
+size_t sige_conv_workspace_bytes(const sige_conv_desc *cd, int32_t batch, int32_t capacity,
+                                 int32_t out_h, int32_t out_w);
+
+/* Synchronise `stream`, return the first device error recorded in the
+ * workspace header (SIGE_OK if none) and clear it. */
+int sige_get_error(void *workspace, sige_stream_t stream);
+
+/* Which conv kernel a call with this layer and dtype runs: 1 = tcgen05 tensor
+ * cores, 0 = CUDA cores; negative = a sige_status for an unsupported layer. */
+int sige_conv_path(const sige_conv_desc *cd, int32_t dtype);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t sige_launch_count(void);
+
+const char *sige_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SIGE_H */

@@ -1,0 +1,251 @@
+"""Python binding of libsige (the C ABI in include/sige.h).
+
+Argument marshalling only: every step of the sparse layer runs in the CUDA
+kernels of ``libsige.so``; torch supplies device memory and streams.  The
+functions carry the ABI's names and raise ``SigeError`` on any non-OK status.
+There is no fallback: if the library is missing, importing a call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsige.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_CAPACITY, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5, -6
+U8, F32, BF16 = 0, 1, 2
+NHWC, NCHW = 0, 1
+WORKSPACE_HEADER = 256
+MAX_SCALES = 8
+
+_DT = {torch.uint8: U8, torch.float32: F32, torch.bfloat16: BF16}
+
+
+class SigeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+class TensorDesc(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int32), ("h", ctypes.c_int32), ("w", ctypes.c_int32), ("c", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("layout", ctypes.c_int32)]
+
+
+class ConvDesc(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int32), ("stride", ctypes.c_int32), ("pad", ctypes.c_int32),
+                ("c_in", ctypes.c_int32), ("c_out", ctypes.c_int32), ("block", ctypes.c_int32)]
+
+
+class ScaleDesc(ctypes.Structure):
+    _fields_ = [("h", ctypes.c_int32), ("w", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("capacity", ctypes.c_int32)]
+
+
+# Every symbol include/sige.h declares, with its ctypes signature.
+_vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+_TD, _CD, _SD = ctypes.POINTER(TensorDesc), ctypes.POINTER(ConvDesc), ctypes.POINTER(ScaleDesc)
+SIGNATURES = {
+    "sige_reduce_mask_workspace_bytes": (_sz, [_TD, _i32, _SD]),
+    "sige_reduce_mask": (_i32, [_vp, _vp, _TD, _f32, _i32, _i32, _SD, _vp, _vp, _vp, _sz, _vp]),
+    "sige_gather": (_i32, [_vp, _TD, _CD, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _vp]),
+    "sige_sparse_conv": (_i32, [_vp, _CD, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _sz, _vp]),
+    "sige_scatter": (_i32, [_vp, _CD, _vp, _vp, _i32, _vp, _vp, _vp, _TD, _vp]),
+    "sige_conv_fused": (_i32, [_vp, _TD, _vp, _vp, _CD, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _vp, _TD,
+                               _vp, _sz, _vp]),
+    "sige_dense_conv": (_i32, [_vp, _TD, _vp, _vp, _CD, _vp, _vp, _i32, _vp, _vp, _TD, _vp, _sz, _vp]),
+    "sige_groupnorm_affine": (_i32, [_vp, _TD, _i32, _vp, _vp, _f32, _vp, _vp, _vp]),
+    "sige_conv_workspace_bytes": (_sz, [_CD, _i32, _i32, _i32, _i32]),
+    "sige_get_error": (_i32, [_vp, _vp]),
+    "sige_conv_path": (_i32, [_CD, _i32]),
+    "sige_launch_count": (ctypes.c_uint64, []),
+    "sige_status_string": (ctypes.c_char_p, [_i32]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsige.so (built by ``__graft_entry__.build()``); raise if absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run __graft_entry__.build() first")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().sige_status_string(int(status)).decode()
+    except Exception:  # library missing
+        return "status"
+
+
+def _check(st: int, what: str):
+    if st != OK:
+        raise SigeError(st, what)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def tensor_desc(t: torch.Tensor, layout: int = NHWC) -> TensorDesc:
+    if t.dim() != 4:
+        raise ValueError("expected a 4-d tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    if layout == NHWC:
+        n, h, w, c = t.shape
+    else:
+        n, c, h, w = t.shape
+    return TensorDesc(n, h, w, c, _DT[t.dtype], layout)
+
+
+def conv_desc(kernel, stride, pad, c_in, c_out, block) -> ConvDesc:
+    return ConvDesc(kernel, stride, pad, c_in, c_out, block)
+
+
+def zeros_workspace(nbytes: int, device) -> torch.Tensor:
+    """A zero-filled device workspace (16-byte aligned, as torch allocations are)."""
+    return torch.zeros(max(int(nbytes), WORKSPACE_HEADER), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------ calls
+
+def sige_reduce_mask_workspace_bytes(desc: TensorDesc, scales) -> int:
+    arr = (ScaleDesc * len(scales))(*[ScaleDesc(*s) for s in scales])
+    return int(lib().sige_reduce_mask_workspace_bytes(ctypes.byref(desc), len(scales), arr))
+
+
+def sige_reduce_mask(a_orig, a_edit, threshold, scales, dilate=1, layout=NHWC, idx=None, counts=None,
+                     workspace=None, stream=None):
+    """Difference mask -> per-scale active-tile lists.  ``scales`` is a list of
+    (h, w, block, capacity).  Returns (idx [sum(capacity), 2] int32, counts
+    [n_scales] int32, workspace); all on the device, nothing synchronised."""
+    desc = tensor_desc(a_orig, layout)
+    arr = (ScaleDesc * len(scales))(*[ScaleDesc(*s) for s in scales])
+    dev = a_orig.device
+    if idx is None:
+        idx = torch.empty((max(1, sum(s[3] for s in scales)), 2), dtype=torch.int32, device=dev)
+    if counts is None:
+        counts = torch.empty(len(scales), dtype=torch.int32, device=dev)
+    need = int(lib().sige_reduce_mask_workspace_bytes(ctypes.byref(desc), len(scales), arr))
+    if workspace is None:
+        workspace = zeros_workspace(need, dev)
+    st = lib().sige_reduce_mask(_ptr(a_orig), _ptr(a_edit), ctypes.byref(desc), float(threshold), int(dilate),
+                                len(scales), arr, _ptr(idx), _ptr(counts), _ptr(workspace),
+                                workspace.numel(), _stream(stream))
+    _check(st, "sige_reduce_mask")
+    return idx, counts, workspace
+
+
+def sige_gather(x, cd: ConvDesc, idx, count, capacity, gn_scale=None, gn_shift=None, silu=False,
+                blocks=None, stream=None):
+    xd = tensor_desc(x)
+    bin_ = (cd.block - 1) * cd.stride + cd.kernel
+    if blocks is None:
+        blocks = torch.empty((max(capacity, 1), x.shape[0], bin_, bin_, cd.c_in), dtype=x.dtype, device=x.device)
+    st = lib().sige_gather(_ptr(x), ctypes.byref(xd), ctypes.byref(cd), _ptr(idx), _ptr(count), int(capacity),
+                           _ptr(gn_scale), _ptr(gn_shift), int(bool(silu)), _ptr(blocks), _stream(stream))
+    _check(st, "sige_gather")
+    return blocks
+
+
+def sige_sparse_conv(blocks, cd: ConvDesc, weight, count, capacity, batch=1, out_blocks=None, workspace=None,
+                     stream=None):
+    if out_blocks is None:
+        out_blocks = torch.empty((max(capacity, 1), batch, cd.block, cd.block, cd.c_out), dtype=torch.float32,
+                                 device=blocks.device)
+    if workspace is None:
+        workspace = zeros_workspace(sige_conv_workspace_bytes(cd, batch, capacity, 0, 0), blocks.device)
+    st = lib().sige_sparse_conv(_ptr(blocks), ctypes.byref(cd), _DT[blocks.dtype], int(batch), _ptr(weight),
+                                _ptr(count), int(capacity), _ptr(out_blocks), _ptr(workspace), workspace.numel(),
+                                _stream(stream))
+    _check(st, "sige_sparse_conv")
+    return out_blocks
+
+
+def sige_scatter(out_blocks, cd: ConvDesc, idx, count, capacity, y, bias=None, residual=None, stream=None):
+    yd = tensor_desc(y)
+    st = lib().sige_scatter(_ptr(out_blocks), ctypes.byref(cd), _ptr(idx), _ptr(count), int(capacity),
+                            _ptr(bias), _ptr(residual), _ptr(y), ctypes.byref(yd), _stream(stream))
+    _check(st, "sige_scatter")
+    return y
+
+
+def sige_conv_fused(x, weight, bias, cd: ConvDesc, idx, count, capacity, y, gn_scale=None, gn_shift=None,
+                    silu=False, residual=None, workspace=None, stream=None):
+    xd, yd = tensor_desc(x), tensor_desc(y)
+    if workspace is None:
+        workspace = zeros_workspace(sige_conv_workspace_bytes(cd, x.shape[0], capacity, 0, 0), x.device)
+    st = lib().sige_conv_fused(_ptr(x), ctypes.byref(xd), _ptr(weight), _ptr(bias), ctypes.byref(cd), _ptr(idx),
+                               _ptr(count), int(capacity), _ptr(gn_scale), _ptr(gn_shift), int(bool(silu)),
+                               _ptr(residual), _ptr(y), ctypes.byref(yd), _ptr(workspace), workspace.numel(),
+                               _stream(stream))
+    _check(st, "sige_conv_fused")
+    return y
+
+
+def sige_dense_conv(x, weight, bias, cd: ConvDesc, y=None, gn_scale=None, gn_shift=None, silu=False,
+                    residual=None, workspace=None, stream=None):
+    N, H, W, _ = x.shape
+    Ho = (H + 2 * cd.pad - cd.kernel) // cd.stride + 1
+    Wo = (W + 2 * cd.pad - cd.kernel) // cd.stride + 1
+    if y is None:
+        y = torch.empty((N, Ho, Wo, cd.c_out), dtype=x.dtype, device=x.device)
+    xd, yd = tensor_desc(x), tensor_desc(y)
+    if workspace is None:
+        workspace = zeros_workspace(sige_conv_workspace_bytes(cd, N, 0, Ho, Wo), x.device)
+    st = lib().sige_dense_conv(_ptr(x), ctypes.byref(xd), _ptr(weight), _ptr(bias), ctypes.byref(cd),
+                               _ptr(gn_scale), _ptr(gn_shift), int(bool(silu)), _ptr(residual), _ptr(y),
+                               ctypes.byref(yd), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "sige_dense_conv")
+    return y
+
+
+def sige_groupnorm_affine(x, groups, gamma, beta, eps=1e-5, scale=None, shift=None, stream=None):
+    xd = tensor_desc(x)
+    if scale is None:
+        scale = torch.empty((x.shape[0], x.shape[3]), dtype=torch.float32, device=x.device)
+    if shift is None:
+        shift = torch.empty_like(scale)
+    st = lib().sige_groupnorm_affine(_ptr(x), ctypes.byref(xd), int(groups), _ptr(gamma), _ptr(beta), float(eps),
+                                     _ptr(scale), _ptr(shift), _stream(stream))
+    _check(st, "sige_groupnorm_affine")
+    return scale, shift
+
+
+def sige_conv_workspace_bytes(cd: ConvDesc, batch: int, capacity: int, out_h: int, out_w: int) -> int:
+    return int(lib().sige_conv_workspace_bytes(ctypes.byref(cd), int(batch), int(capacity), int(out_h), int(out_w)))
+
+
+def sige_get_error(workspace, stream=None) -> int:
+    return int(lib().sige_get_error(_ptr(workspace), _stream(stream)))
+
+
+def sige_conv_path(cd: ConvDesc, dtype: torch.dtype) -> int:
+    return int(lib().sige_conv_path(ctypes.byref(cd), _DT[dtype]))
+
+
+def sige_launch_count() -> int:
+    return int(lib().sige_launch_count())

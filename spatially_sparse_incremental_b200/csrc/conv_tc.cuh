@@ -1,0 +1,12 @@
+// Tensor-core (tcgen05) conv kernel: interface used by the ABI layer.
+#pragma once
+
+#include "conv_common.cuh"
+
+namespace sige {
+
+bool tc_supported(const sige_conv_desc *cd, int dtype);
+size_t tc_workspace_bytes(const sige_conv_desc *cd, int batch, int ntiles);
+int launch_conv_tc(const ConvParams &p, cudaStream_t stream);
+
+} // namespace sige

@@ -1,0 +1,256 @@
+// Gather of halo'd active blocks and scatter of output blocks into the cached
+// output (SIGE project page, "Overview": gather the active blocks from the
+// edited activation, stack them along the batch axis, and scatter the output
+// blocks back into F_l(A_original)).  Plus the GroupNorm statistics of the
+// cached original activation, folded into a per-channel affine.
+#include <algorithm>
+
+#include "sige_internal.cuh"
+#include "transform.cuh"
+
+namespace sige {
+
+// ------------------------------------------------------------------ gather
+
+struct GatherParams {
+    const uint8_t *x;
+    int32_t N, H, W, C, dtype;
+    int32_t s, pad, bin;
+    const int32_t *idx;
+    const int32_t *count;
+    int32_t cap;
+    const float *gsc, *gsh;
+    int32_t silu;
+    uint8_t *blocks;
+    int32_t vpp;  // 16-byte vectors per pixel
+};
+
+__global__ void __launch_bounds__(256) k_gather(const __grid_constant__ GatherParams p)
+{
+    const int64_t ntile = min(__ldg(p.count), p.cap);
+    const int64_t per_tile = (int64_t)p.N * p.bin * p.bin * p.vpp;
+    const int64_t total = ntile * per_tile;
+    const int esz = p.dtype == SIGE_BF16 ? 2 : 4;
+    const int epv = 16 / esz;
+    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
+         v += (int64_t)gridDim.x * blockDim.x) {
+        const int cv = (int)(v % p.vpp);
+        int64_t pix = v / p.vpp;
+        const int ww = (int)(pix % p.bin);
+        pix /= p.bin;
+        const int hh = (int)(pix % p.bin);
+        pix /= p.bin;
+        const int n = (int)(pix % p.N);
+        const int t = (int)(pix / p.N);
+        const int2 o = __ldg(reinterpret_cast<const int2 *>(p.idx) + t);
+        const int y = o.x * p.s - p.pad + hh, x = o.y * p.s - p.pad + ww;
+        uint4 out = make_uint4(0, 0, 0, 0);
+        if (y >= 0 && y < p.H && x >= 0 && x < p.W) {
+            const uint4 in = ld_nc16(p.x + ((((int64_t)n * p.H + y) * p.W + x) * p.C) * esz + cv * 16);
+            const int c0 = cv * epv;
+            out = transform16(in, p.dtype, p.gsc ? p.gsc + (int64_t)n * p.C + c0 : nullptr,
+                              p.gsc ? p.gsh + (int64_t)n * p.C + c0 : nullptr, p.silu);
+        }
+        reinterpret_cast<uint4 *>(p.blocks)[v] = out;
+    }
+}
+
+// ------------------------------------------------------------------ scatter
+
+struct ScatterParams {
+    const float *out;
+    int32_t N, Ho, Wo, Co, dtype, b;
+    const int32_t *idx;
+    const int32_t *count;
+    int32_t cap;
+    const float *bias;
+    const uint8_t *residual;
+    uint8_t *y;
+};
+
+__global__ void __launch_bounds__(256) k_scatter(const __grid_constant__ ScatterParams p)
+{
+    const int64_t ntile = min(__ldg(p.count), p.cap);
+    const int c4n = p.Co / 4;
+    const int64_t total = ntile * p.N * p.b * p.b * c4n;
+    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
+         v += (int64_t)gridDim.x * blockDim.x) {
+        const int c4 = (int)(v % c4n);
+        int64_t pix = v / c4n;
+        const int j = (int)(pix % p.b);
+        pix /= p.b;
+        const int i = (int)(pix % p.b);
+        pix /= p.b;
+        const int n = (int)(pix % p.N);
+        const int t = (int)(pix / p.N);
+        const int2 o = __ldg(reinterpret_cast<const int2 *>(p.idx) + t);
+        const int yo = o.x + i, xo = o.y + j;
+        if (yo >= p.Ho || xo >= p.Wo)
+            continue;
+        float4 a = __ldg(reinterpret_cast<const float4 *>(p.out) + v);
+        const int c = c4 * 4;
+        const int64_t e = (((int64_t)n * p.Ho + yo) * p.Wo + xo) * p.Co + c;
+        store_out4(p.y, e, p.dtype, a, p.bias ? p.bias + c : nullptr, p.residual);
+    }
+}
+
+// ------------------------------------------------------------------ GroupNorm affine
+
+struct GnParams {
+    const uint8_t *x;
+    int32_t N, HW, C, dtype, groups;
+    const float *gamma, *beta;
+    float eps;
+    float *scale, *shift;
+};
+
+__device__ __forceinline__ double block_sum_d(double v, double *sh)
+{
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0)
+        sh[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        v = lane < (int)(blockDim.x >> 5) ? sh[lane] : 0.0;
+        for (int o = 16; o > 0; o >>= 1)
+            v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        if (lane == 0)
+            sh[32] = v;
+    }
+    __syncthreads();
+    double r = sh[32];
+    __syncthreads();
+    return r;
+}
+
+__device__ __forceinline__ float gn_elem(const GnParams &p, int64_t i)
+{
+    if (p.dtype == SIGE_BF16)
+        return __uint_as_float((uint32_t)(reinterpret_cast<const uint16_t *>(p.x)[i]) << 16);
+    return reinterpret_cast<const float *>(p.x)[i];
+}
+
+// One CTA per (n, group): two passes in double, fixed reduction order.
+__global__ void __launch_bounds__(1024) k_gn_affine(const __grid_constant__ GnParams p)
+{
+    __shared__ double sh[33];
+    const int n = blockIdx.x / p.groups, g = blockIdx.x % p.groups;
+    const int cg = p.C / p.groups;
+    const int64_t cnt = (int64_t)p.HW * cg;
+    const int64_t base = (int64_t)n * p.HW * p.C + (int64_t)g * cg;
+    double s = 0.0;
+    for (int64_t k = threadIdx.x; k < cnt; k += blockDim.x)
+        s += gn_elem(p, base + (k / cg) * p.C + (k % cg));
+    const double mean = block_sum_d(s, sh) / (double)cnt;
+    double v = 0.0;
+    for (int64_t k = threadIdx.x; k < cnt; k += blockDim.x) {
+        double d = gn_elem(p, base + (k / cg) * p.C + (k % cg)) - mean;
+        v += d * d;
+    }
+    const double var = block_sum_d(v, sh) / (double)cnt;
+    for (int c = threadIdx.x; c < cg; c += blockDim.x) {
+        const int ch = g * cg + c;
+        const double sc = (double)p.gamma[ch] / sqrt(var + (double)p.eps);
+        p.scale[(int64_t)n * p.C + ch] = (float)sc;
+        p.shift[(int64_t)n * p.C + ch] = (float)((double)p.beta[ch] - mean * sc);
+    }
+}
+
+static int grid_for(int64_t work, int threads)
+{
+    int64_t g = (work + threads - 1) / threads;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(g, (int64_t)device_sm_count() * 8));
+}
+
+} // namespace sige
+
+using namespace sige;
+
+static bool conv_desc_ok(const sige_conv_desc *cd)
+{
+    return cd && cd->kernel >= 1 && cd->stride >= 1 && cd->pad >= 0 && cd->pad < cd->kernel &&
+           cd->c_in >= 1 && cd->c_out >= 1 && cd->block >= 1 && cd->block <= 64;
+}
+
+extern "C" int sige_gather(const void *x, const sige_tensor_desc *xd, const sige_conv_desc *cd,
+                           const int32_t *idx, const int32_t *count, int32_t capacity,
+                           const float *gn_scale, const float *gn_shift, int32_t silu, void *blocks,
+                           sige_stream_t stream)
+{
+    if (!x || !xd || !idx || !count || !blocks || capacity < 0 || !conv_desc_ok(cd))
+        return SIGE_ERR_INVALID_ARG;
+    if ((gn_scale == nullptr) != (gn_shift == nullptr))
+        return SIGE_ERR_INVALID_ARG;
+    if (xd->n < 1 || xd->h < 1 || xd->w < 1 || xd->c != cd->c_in)
+        return SIGE_ERR_INVALID_ARG;
+    if (xd->layout != SIGE_NHWC || (xd->dtype != SIGE_F32 && xd->dtype != SIGE_BF16))
+        return SIGE_ERR_UNSUPPORTED;
+    const int esz = xd->dtype == SIGE_BF16 ? 2 : 4;
+    if ((xd->c * esz) % 16 || (reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(blocks) & 15))
+        return SIGE_ERR_UNSUPPORTED;
+    if (capacity == 0)
+        return SIGE_OK;
+    GatherParams p{};
+    p.x = static_cast<const uint8_t *>(x);
+    p.N = xd->n; p.H = xd->h; p.W = xd->w; p.C = xd->c; p.dtype = xd->dtype;
+    p.s = cd->stride; p.pad = cd->pad;
+    p.bin = (cd->block - 1) * cd->stride + cd->kernel;
+    p.idx = idx; p.count = count; p.cap = capacity;
+    p.gsc = gn_scale; p.gsh = gn_shift; p.silu = silu ? 1 : 0;
+    p.blocks = static_cast<uint8_t *>(blocks);
+    p.vpp = xd->c * esz / 16;
+    const int64_t work = (int64_t)capacity * p.N * p.bin * p.bin * p.vpp;
+    k_gather<<<grid_for(work, 256), 256, 0, (cudaStream_t)stream>>>(p);
+    count_launch();
+    return launch_check();
+}
+
+extern "C" int sige_scatter(const float *out_blocks, const sige_conv_desc *cd, const int32_t *idx,
+                            const int32_t *count, int32_t capacity, const float *bias,
+                            const void *residual, void *y, const sige_tensor_desc *yd,
+                            sige_stream_t stream)
+{
+    if (!out_blocks || !idx || !count || !y || !yd || capacity < 0 || !conv_desc_ok(cd))
+        return SIGE_ERR_INVALID_ARG;
+    if (yd->c != cd->c_out || yd->n < 1 || yd->h < 1 || yd->w < 1)
+        return SIGE_ERR_INVALID_ARG;
+    if (yd->layout != SIGE_NHWC || (yd->dtype != SIGE_F32 && yd->dtype != SIGE_BF16) || cd->c_out % 4)
+        return SIGE_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(out_blocks) & 15) || (reinterpret_cast<uintptr_t>(y) & 15) ||
+        (reinterpret_cast<uintptr_t>(residual) & 15))
+        return SIGE_ERR_UNSUPPORTED;
+    if (capacity == 0)
+        return SIGE_OK;
+    ScatterParams p{};
+    p.out = out_blocks;
+    p.N = yd->n; p.Ho = yd->h; p.Wo = yd->w; p.Co = yd->c; p.dtype = yd->dtype; p.b = cd->block;
+    p.idx = idx; p.count = count; p.cap = capacity;
+    p.bias = bias;
+    p.residual = static_cast<const uint8_t *>(residual);
+    p.y = static_cast<uint8_t *>(y);
+    const int64_t work = (int64_t)capacity * p.N * p.b * p.b * (p.Co / 4);
+    k_scatter<<<grid_for(work, 256), 256, 0, (cudaStream_t)stream>>>(p);
+    count_launch();
+    return launch_check();
+}
+
+extern "C" int sige_groupnorm_affine(const void *x, const sige_tensor_desc *xd, int32_t groups,
+                                     const float *gamma, const float *beta, float eps, float *scale,
+                                     float *shift, sige_stream_t stream)
+{
+    if (!x || !xd || !gamma || !beta || !scale || !shift || groups < 1 || !(eps >= 0.0f))
+        return SIGE_ERR_INVALID_ARG;
+    if (xd->n < 1 || xd->h < 1 || xd->w < 1 || xd->c < 1 || xd->c % groups)
+        return SIGE_ERR_INVALID_ARG;
+    if (xd->layout != SIGE_NHWC || (xd->dtype != SIGE_F32 && xd->dtype != SIGE_BF16))
+        return SIGE_ERR_UNSUPPORTED;
+    GnParams p{};
+    p.x = static_cast<const uint8_t *>(x);
+    p.N = xd->n; p.HW = xd->h * xd->w; p.C = xd->c; p.dtype = xd->dtype; p.groups = groups;
+    p.gamma = gamma; p.beta = beta; p.eps = eps; p.scale = scale; p.shift = shift;
+    k_gn_affine<<<xd->n * groups, 1024, 0, (cudaStream_t)stream>>>(p);
+    count_launch();
+    return launch_check();
+}

@@ -1,0 +1,227 @@
+// C ABI entry points for the conv calls, host-side validation and utilities.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+
+#include "conv_common.cuh"
+#include "conv_tc.cuh"
+
+namespace sige {
+
+static std::atomic<uint64_t> g_launches{0};
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+int launch_check()
+{
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SIGE_OK : SIGE_ERR_CUDA;
+}
+
+int device_sm_count()
+{
+    static int cache[64] = {0};
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64)
+        return kNumSMs;
+    if (!cache[d]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0)
+            n = kNumSMs;
+        cache[d] = n;
+    }
+    return cache[d];
+}
+
+static int esize(int dtype) { return dtype == SIGE_BF16 ? 2 : dtype == SIGE_F32 ? 4 : 1; }
+
+static int check_layer(const sige_conv_desc *cd, int dtype)
+{
+    if (!cd || cd->kernel < 1 || cd->stride < 1 || cd->pad < 0 || cd->pad >= cd->kernel ||
+        cd->c_in < 1 || cd->c_out < 1 || cd->block < 1 || cd->block > 64)
+        return SIGE_ERR_INVALID_ARG;
+    if (dtype != SIGE_F32 && dtype != SIGE_BF16)
+        return SIGE_ERR_UNSUPPORTED;
+    const int bin = (cd->block - 1) * cd->stride + cd->kernel;
+    if (bin * bin > 12288)
+        return SIGE_ERR_UNSUPPORTED;
+    return SIGE_OK;
+}
+
+// 1 = tensor-core kernel, 0 = CUDA-core kernel.
+static int choose_path(const sige_conv_desc *cd, int dtype)
+{
+    return tc_supported(cd, dtype) ? 1 : 0;
+}
+
+static size_t ws_need(const sige_conv_desc *cd, int batch, int ntiles)
+{
+    return kWsHeader + tc_workspace_bytes(cd, batch, ntiles);
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+static int run_conv(ConvParams &p, const sige_conv_desc *cd, void *ws, size_t ws_bytes, cudaStream_t st)
+{
+    p.k = cd->kernel; p.s = cd->stride; p.pad = cd->pad; p.b = cd->block;
+    p.bin = (cd->block - 1) * cd->stride + cd->kernel;
+    p.Cin = cd->c_in; p.Cout = cd->c_out;
+    p.ws = static_cast<uint8_t *>(ws);
+    p.ws_bytes = ws_bytes;
+    const int ntiles = p.dense ? p.tiles_total : p.cap;
+    if (!ws || ws_bytes < ws_need(cd, p.N, ntiles) || !aligned16(ws))
+        return SIGE_ERR_WORKSPACE;
+    if (ntiles == 0)
+        return SIGE_OK;
+    if (choose_path(cd, p.dtype) == 1)
+        return launch_conv_tc(p, st);
+    return launch_conv_simt(p, st);
+}
+
+} // namespace sige
+
+using namespace sige;
+
+extern "C" size_t sige_conv_workspace_bytes(const sige_conv_desc *cd, int32_t batch, int32_t capacity,
+                                            int32_t out_h, int32_t out_w)
+{
+    if (!cd || cd->block < 1 || batch < 1 || capacity < 0)
+        return 0;
+    const int64_t dense_tiles = (int64_t)((out_h + cd->block - 1) / cd->block) * ((out_w + cd->block - 1) / cd->block);
+    const int64_t nt = std::max<int64_t>(capacity, dense_tiles);
+    return ws_need(cd, batch, (int)std::min<int64_t>(nt, INT32_MAX));
+}
+
+extern "C" int sige_conv_path(const sige_conv_desc *cd, int32_t dtype)
+{
+    const int st = check_layer(cd, dtype);
+    if (st != SIGE_OK)
+        return st;
+    return choose_path(cd, dtype);
+}
+
+extern "C" int sige_sparse_conv(const void *blocks, const sige_conv_desc *cd, int32_t dtype, int32_t batch,
+                                const void *weight, const int32_t *count, int32_t capacity,
+                                float *out_blocks, void *workspace, size_t workspace_bytes,
+                                sige_stream_t stream)
+{
+    if (!blocks || !weight || !count || !out_blocks || batch < 1 || capacity < 0)
+        return SIGE_ERR_INVALID_ARG;
+    const int st = check_layer(cd, dtype);
+    if (st != SIGE_OK)
+        return st;
+    if (!aligned16(blocks) || !aligned16(weight) || !aligned16(out_blocks))
+        return SIGE_ERR_UNSUPPORTED;
+    ConvParams p{};
+    p.src = static_cast<const uint8_t *>(blocks);
+    p.N = batch; p.dtype = dtype;
+    p.count = count; p.cap = capacity;
+    p.w = static_cast<const uint8_t *>(weight);
+    p.out_blocks = out_blocks;
+    p.from_image = 0; p.to_y = 0;
+    return run_conv(p, cd, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+static int fused_common(ConvParams &p, const void *x, const sige_tensor_desc *xd, const void *weight,
+                        const float *bias, const sige_conv_desc *cd, const float *gn_scale,
+                        const float *gn_shift, int32_t silu, const void *residual, void *y,
+                        const sige_tensor_desc *yd)
+{
+    if (!x || !xd || !weight || !y || !yd)
+        return SIGE_ERR_INVALID_ARG;
+    if ((gn_scale == nullptr) != (gn_shift == nullptr))
+        return SIGE_ERR_INVALID_ARG;
+    const int st = check_layer(cd, xd->dtype);
+    if (st != SIGE_OK)
+        return st;
+    if (xd->layout != SIGE_NHWC || yd->layout != SIGE_NHWC || yd->dtype != xd->dtype)
+        return SIGE_ERR_UNSUPPORTED;
+    if (xd->n < 1 || xd->h < 1 || xd->w < 1 || xd->c != cd->c_in)
+        return SIGE_ERR_INVALID_ARG;
+    const int Ho = (xd->h + 2 * cd->pad - cd->kernel) / cd->stride + 1;
+    const int Wo = (xd->w + 2 * cd->pad - cd->kernel) / cd->stride + 1;
+    if (Ho < 1 || Wo < 1 || yd->n != xd->n || yd->h != Ho || yd->w != Wo || yd->c != cd->c_out)
+        return SIGE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(weight) || !aligned16(y) || !aligned16(residual) ||
+        !aligned16(bias) || !aligned16(gn_scale) || !aligned16(gn_shift))
+        return SIGE_ERR_UNSUPPORTED;
+    p.src = static_cast<const uint8_t *>(x);
+    p.N = xd->n; p.H = xd->h; p.W = xd->w; p.dtype = xd->dtype;
+    p.gsc = gn_scale; p.gsh = gn_shift; p.silu = silu ? 1 : 0;
+    p.w = static_cast<const uint8_t *>(weight);
+    p.bias = bias;
+    p.residual = static_cast<const uint8_t *>(residual);
+    p.y = static_cast<uint8_t *>(y);
+    p.Ho = Ho; p.Wo = Wo;
+    p.from_image = 1; p.to_y = 1;
+    (void)esize;
+    return SIGE_OK;
+}
+
+extern "C" int sige_conv_fused(const void *x, const sige_tensor_desc *xd, const void *weight,
+                               const float *bias, const sige_conv_desc *cd, const int32_t *idx,
+                               const int32_t *count, int32_t capacity, const float *gn_scale,
+                               const float *gn_shift, int32_t silu, const void *residual, void *y,
+                               const sige_tensor_desc *yd, void *workspace, size_t workspace_bytes,
+                               sige_stream_t stream)
+{
+    if (!idx || !count || capacity < 0)
+        return SIGE_ERR_INVALID_ARG;
+    ConvParams p{};
+    int st = fused_common(p, x, xd, weight, bias, cd, gn_scale, gn_shift, silu, residual, y, yd);
+    if (st != SIGE_OK)
+        return st;
+    if (reinterpret_cast<uintptr_t>(idx) & 7)
+        return SIGE_ERR_INVALID_ARG;
+    p.idx = idx; p.count = count; p.cap = capacity; p.dense = 0;
+    return run_conv(p, cd, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+extern "C" int sige_dense_conv(const void *x, const sige_tensor_desc *xd, const void *weight,
+                               const float *bias, const sige_conv_desc *cd, const float *gn_scale,
+                               const float *gn_shift, int32_t silu, const void *residual, void *y,
+                               const sige_tensor_desc *yd, void *workspace, size_t workspace_bytes,
+                               sige_stream_t stream)
+{
+    ConvParams p{};
+    int st = fused_common(p, x, xd, weight, bias, cd, gn_scale, gn_shift, silu, residual, y, yd);
+    if (st != SIGE_OK)
+        return st;
+    p.dense = 1;
+    p.tiles_w = (p.Wo + cd->block - 1) / cd->block;
+    p.tiles_total = ((p.Ho + cd->block - 1) / cd->block) * p.tiles_w;
+    p.cap = p.tiles_total;
+    return run_conv(p, cd, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+extern "C" int sige_get_error(void *workspace, sige_stream_t stream)
+{
+    if (!workspace)
+        return SIGE_ERR_INVALID_ARG;
+    int32_t h[2] = {0, 0};
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(h, workspace, sizeof h, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return SIGE_ERR_CUDA;
+    if (h[0] != 0) {
+        if (cudaMemsetAsync(workspace, 0, sizeof h, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+            return SIGE_ERR_CUDA;
+    }
+    return h[0];
+}
+
+extern "C" uint64_t sige_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+extern "C" const char *sige_status_string(int32_t status)
+{
+    switch (status) {
+    case SIGE_OK: return "ok";
+    case SIGE_ERR_INVALID_ARG: return "invalid argument";
+    case SIGE_ERR_UNSUPPORTED: return "unsupported shape, dtype or layout";
+    case SIGE_ERR_CUDA: return "CUDA error";
+    case SIGE_ERR_CAPACITY: return "more active tiles than the list capacity";
+    case SIGE_ERR_TIMEOUT: return "bounded wait expired on the device";
+    case SIGE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    default: return "unknown status";
+    }
+}

@@ -1,0 +1,62 @@
+// Internal definitions shared by the CUDA sources of libsige.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sige.h"
+
+namespace sige {
+
+constexpr int kNumSMs = 148;            // B200
+constexpr int kMaxScales = SIGE_MAX_SCALES;
+constexpr size_t kWsHeader = SIGE_WORKSPACE_HEADER_BYTES;
+
+// Workspace header (first 256 bytes of every workspace).
+struct WsHeader {
+    int32_t error;        // first device error (a sige_status), 0 = none
+    int32_t detail;       // call-specific detail of that error
+    uint32_t arrive;      // "last CTA" arrival counter (self-resetting)
+    uint32_t pad[61];
+};
+static_assert(sizeof(WsHeader) == kWsHeader, "header size");
+
+__device__ __forceinline__ void record_error(WsHeader *h, int32_t code, int32_t detail)
+{
+    if (atomicCAS(&h->error, 0, code) == 0)
+        atomicExch(&h->detail, detail);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Two floats -> packed bf16x2 (round to nearest even), low half = a.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float silu_f(float v) { return v / (1.0f + __expf(-v)); }
+
+// 16-byte loads/stores.
+__device__ __forceinline__ uint4 ld_stream16(const void *p)
+{
+    uint4 r;
+    asm volatile("ld.global.cs.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+__device__ __forceinline__ uint4 ld_nc16(const void *p)
+{
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+// Host-side helpers (sige_api.cu)
+int launch_check();           // SIGE_OK or SIGE_ERR_CUDA after a launch
+void count_launch();
+int device_sm_count();
+
+} // namespace sige

@@ -1,0 +1,140 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports
+every symbol include/sige.h declares with the signature the binding uses, and
+rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import spatially_sparse_incremental_b200 as sige
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sige.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    import __graft_entry__
+    __graft_entry__.build_library()
+    return sige.lib()
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_ ]*?\**\s*\b(sige_[a-z_]+)\s*\(", txt, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_calls():
+    names = _declared()
+    for call in ("sige_reduce_mask", "sige_gather", "sige_sparse_conv", "sige_scatter", "sige_conv_fused"):
+        assert call in names
+
+
+def test_every_declared_symbol_is_exported_and_bound(L):
+    names = _declared()
+    assert set(names) == set(sige.SIGNATURES), set(names) ^ set(sige.SIGNATURES)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for st in (0, -1, -2, -3, -4, -5, -6):
+        s = sige.status_string(st)
+        assert s and s != "unknown status"
+    assert sige.status_string(-99) == "unknown status"
+
+
+def _scales(*s):
+    return (sige.ScaleDesc * len(s))(*[sige.ScaleDesc(*q) for q in s])
+
+
+def test_reduce_mask_validation(L):
+    d = sige.TensorDesc(1, 256, 256, 3, sige.U8, sige.NCHW)
+    sc = _scales((256, 256, 8, 1024), (128, 128, 4, 1024), (64, 64, 4, 256), (32, 32, 2, 256))
+    need = L.sige_reduce_mask_workspace_bytes(ctypes.byref(d), 4, sc)
+    # header + one 16-byte-padded flag byte per tile per scale
+    assert need == 256 + 1024 + 1024 + 256 + 256
+    fake = ctypes.c_void_p(0x1000)
+    ws = ctypes.c_void_p(0x2000)
+    args = lambda **kw: dict(dict(a=fake, b=fake, d=ctypes.byref(d), thr=0.0, dil=1, ns=4, sc=sc,
+                                  idx=fake, cnt=fake, ws=ws, wsb=need, st=None), **kw)
+
+    def call(**kw):
+        a = args(**kw)
+        return L.sige_reduce_mask(a["a"], a["b"], a["d"], a["thr"], a["dil"], a["ns"], a["sc"], a["idx"],
+                                  a["cnt"], a["ws"], a["wsb"], a["st"])
+    assert call(a=None) == sige.ERR_INVALID_ARG
+    assert call(idx=None) == sige.ERR_INVALID_ARG
+    assert call(thr=-1.0) == sige.ERR_INVALID_ARG
+    assert call(thr=float("nan")) == sige.ERR_INVALID_ARG
+    assert call(dil=-1) == sige.ERR_INVALID_ARG
+    assert call(ns=0) == sige.ERR_INVALID_ARG
+    assert call(ns=9) == sige.ERR_INVALID_ARG
+    assert call(wsb=need - 1) == sige.ERR_WORKSPACE
+    assert call(ws=None) == sige.ERR_WORKSPACE
+    bad = _scales((100, 100, 8, 16))          # 256 is not a multiple of 100
+    assert call(ns=1, sc=bad) == sige.ERR_INVALID_ARG
+    d16 = sige.TensorDesc(1, 16, 16, 3, 7, sige.NHWC)
+    assert call(d=ctypes.byref(d16)) == sige.ERR_UNSUPPORTED
+
+
+def test_conv_validation(L):
+    cd = sige.ConvDesc(3, 1, 1, 128, 128, 8)
+    xd = sige.TensorDesc(1, 64, 64, 128, sige.BF16, sige.NHWC)
+    yd = sige.TensorDesc(1, 64, 64, 128, sige.BF16, sige.NHWC)
+    fake = ctypes.c_void_p(0x1000)
+    ws = ctypes.c_void_p(0x2000)
+    wsb = L.sige_conv_workspace_bytes(ctypes.byref(cd), 1, 64, 64, 64)
+    assert wsb >= 256
+
+    def fused(**kw):
+        a = dict(x=fake, xd=ctypes.byref(xd), w=fake, b=None, cd=ctypes.byref(cd), idx=fake, cnt=fake, cap=64,
+                 gs=None, gh=None, silu=0, res=None, y=fake, yd=ctypes.byref(yd), ws=ws, wsb=wsb, st=None)
+        a.update(kw)
+        return L.sige_conv_fused(*a.values())
+    assert fused(x=None) == sige.ERR_INVALID_ARG
+    assert fused(cap=-1) == sige.ERR_INVALID_ARG
+    assert fused(gs=fake) == sige.ERR_INVALID_ARG               # scale without shift
+    ydb = sige.TensorDesc(1, 63, 64, 128, sige.BF16, sige.NHWC)
+    assert fused(yd=ctypes.byref(ydb)) == sige.ERR_INVALID_ARG  # wrong output size
+    ydf = sige.TensorDesc(1, 64, 64, 128, sige.F32, sige.NHWC)
+    assert fused(yd=ctypes.byref(ydf)) == sige.ERR_UNSUPPORTED  # dtype mismatch
+    assert fused(ws=None) == sige.ERR_WORKSPACE
+    assert fused(wsb=10) == sige.ERR_WORKSPACE
+    bad = sige.ConvDesc(3, 1, 3, 128, 128, 8)                   # pad >= kernel
+    assert fused(cd=ctypes.byref(bad)) == sige.ERR_INVALID_ARG
+    assert fused(x=ctypes.c_void_p(0x1001)) == sige.ERR_UNSUPPORTED  # misaligned
+
+
+def test_conv_path_selection(L):
+    assert sige.sige_conv_path(sige.ConvDesc(3, 1, 1, 64, 64, 4), __import__("torch").float32) == 0
+    assert sige.sige_conv_path(sige.ConvDesc(3, 1, 3, 64, 64, 4), __import__("torch").float32) == sige.ERR_INVALID_ARG
+
+
+def test_gather_scatter_validation(L):
+    cd = sige.ConvDesc(3, 1, 1, 64, 64, 4)
+    fake = ctypes.c_void_p(0x1000)
+    xd = sige.TensorDesc(1, 16, 16, 64, sige.F32, sige.NHWC)
+    assert L.sige_gather(None, ctypes.byref(xd), ctypes.byref(cd), fake, fake, 4, None, None, 0, fake, None) \
+        == sige.ERR_INVALID_ARG
+    xd3 = sige.TensorDesc(1, 16, 16, 3, sige.F32, sige.NHWC)      # C != c_in
+    assert L.sige_gather(fake, ctypes.byref(xd3), ctypes.byref(cd), fake, fake, 4, None, None, 0, fake, None) \
+        == sige.ERR_INVALID_ARG
+    yd = sige.TensorDesc(1, 16, 16, 64, sige.U8, sige.NHWC)
+    assert L.sige_scatter(fake, ctypes.byref(cd), fake, fake, 4, None, None, fake, ctypes.byref(yd), None) \
+        == sige.ERR_UNSUPPORTED
+    # zero capacity is a no-op that launches nothing
+    n0 = sige.sige_launch_count()
+    yd2 = sige.TensorDesc(1, 16, 16, 64, sige.F32, sige.NHWC)
+    assert L.sige_scatter(fake, ctypes.byref(cd), fake, fake, 0, None, None, fake, ctypes.byref(yd2), None) == sige.OK
+    assert sige.sige_launch_count() == n0
+
+
+def test_groupnorm_validation(L):
+    fake = ctypes.c_void_p(0x1000)
+    xd = sige.TensorDesc(1, 8, 8, 30, sige.F32, sige.NHWC)        # 30 channels, 32 groups
+    assert L.sige_groupnorm_affine(fake, ctypes.byref(xd), 32, fake, fake, 1e-5, fake, fake, None) \
+        == sige.ERR_INVALID_ARG

@@ -1,0 +1,130 @@
+"""GPU mask reduction vs the oracle: bit-exact tile lists and counts.
+
+mer.dev notes on SIGE, section 3.2 "Sparse Engine SIGE" (downsample, dilate,
+select tiles); SIGE project page, "Overview" (active block indices)."""
+import numpy as np
+import pytest
+import torch
+
+import spatially_sparse_incremental_b200 as sige
+from spatially_sparse_incremental_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _gpu_lists(a, b, thr, scales, dilate=1, layout=sige.NHWC, workspace=None):
+    idx, cnt, ws = sige.sige_reduce_mask(a.to(DEV), b.to(DEV), thr, scales, dilate, layout, workspace=workspace)
+    torch.cuda.synchronize()
+    cnt = cnt.cpu().numpy()
+    idx = idx.cpu().numpy()
+    out, off = [], 0
+    for s, (h, w, blk, cap) in enumerate(scales):
+        out.append(idx[off:off + min(cnt[s], cap)])
+        off += cap
+    return out, cnt, ws
+
+
+def _full_caps(scales):
+    return [(h, w, b, -(-h // b) * -(-w // b)) for (h, w, b) in scales]
+
+
+def test_cfg2_images_100_seeds(orc):
+    scales = inputs.CFG2_SCALES
+    for seed in range(100):
+        o, e, _ = inputs.make_cfg2(seed)
+        ref = orc.reduce_mask(o, e, 0.0, scales, 1, orc.NCHW)
+        got, cnt, _ = _gpu_lists(o, e, 0.0, _full_caps(scales), 1, sige.NCHW)
+        for s in range(len(scales)):
+            assert cnt[s] == len(ref[s]), (seed, s)
+            assert np.array_equal(got[s], ref[s]), (seed, s)
+
+
+def test_cfg1_f32_nhwc(orc):
+    for seed in range(10):
+        L = inputs.make_cfg1(seed)
+        sc = [(64, 64, 4)]
+        ref = orc.reduce_mask(L.x_orig, L.x_edit, 1e-3, sc, 1)
+        got, _, _ = _gpu_lists(L.x_orig, L.x_edit, 1e-3, _full_caps(sc))
+        assert np.array_equal(got[0], ref[0])
+
+
+def test_cfg3_bf16_activations(orc):
+    for seed in range(3):
+        blk = inputs.make_cfg3(seed)
+        sc = [(256, 256, 8), (128, 128, 4), (64, 64, 2)]
+        ref = orc.reduce_mask(blk.x_orig, blk.x_edit, 1e-3, sc, 1)
+        got, _, _ = _gpu_lists(blk.x_orig, blk.x_edit, 1e-3, _full_caps(sc))
+        for s in range(len(sc)):
+            assert np.array_equal(got[s], ref[s]), (seed, s)
+
+
+def test_random_small_cases(orc):
+    # covers the scalar path (C*esize not a multiple of 16, odd widths), both
+    # layouts, batch > 1, several scales, dilation 0..2, ragged tile grids.
+    rng = np.random.default_rng(7)
+    for case in range(150):
+        dtype = [torch.uint8, torch.float32, torch.bfloat16][case % 3]
+        layout = sige.NHWC if rng.random() < 0.5 else sige.NCHW
+        N = int(rng.integers(1, 3))
+        f = int(rng.choice([1, 2, 4]))
+        Hs, Ws = int(rng.integers(1, 12)), int(rng.integers(1, 12))
+        H, W = Hs * f, Ws * f
+        C = int(rng.choice([1, 3, 8, 16, 64]))
+        if dtype == torch.uint8:
+            a = torch.from_numpy(rng.integers(0, 256, size=(N, H, W, C)).astype(np.uint8))
+        else:
+            a = torch.from_numpy(rng.normal(size=(N, H, W, C)).astype(np.float32)).to(dtype)
+        b = a.clone()
+        m = rng.random((N, H, W)) < rng.choice([0.0, 0.02, 0.1, 1.0])
+        if dtype == torch.uint8:
+            b[torch.from_numpy(m)] = b[torch.from_numpy(m)] ^ 1
+        else:
+            b[torch.from_numpy(m)] = b[torch.from_numpy(m)] + 1.0
+        if layout == sige.NCHW:
+            a, b = a.permute(0, 3, 1, 2).contiguous(), b.permute(0, 3, 1, 2).contiguous()
+        thr = 0.0 if dtype == torch.uint8 else 1e-3
+        sc = [(H, W, int(rng.integers(1, 5)))]
+        if f > 1:
+            sc.append((Hs, Ws, int(rng.integers(1, 4))))
+        D = int(rng.integers(0, 3))
+        ref = orc.reduce_mask(a, b, thr, sc, D, orc.NHWC if layout == sige.NHWC else orc.NCHW)
+        got, _, _ = _gpu_lists(a, b, thr, _full_caps(sc), D, layout)
+        for s in range(len(sc)):
+            assert np.array_equal(got[s], ref[s]), (case, s)
+
+
+def test_empty_and_full_masks():
+    x = torch.randn(1, 64, 64, 32)
+    got, cnt, _ = _gpu_lists(x, x.clone(), 1e-3, [(64, 64, 8, 64)])
+    assert cnt[0] == 0 and len(got[0]) == 0
+    got, cnt, _ = _gpu_lists(x, x + 1, 1e-3, [(64, 64, 8, 64), (32, 32, 4, 64)])
+    want = np.array([(i, j) for i in range(0, 64, 8) for j in range(0, 64, 8)], np.int32)
+    assert cnt[0] == 64 and np.array_equal(got[0], want)
+    want2 = np.array([(i, j) for i in range(0, 32, 4) for j in range(0, 32, 4)], np.int32)
+    assert np.array_equal(got[1], want2)
+
+
+def test_capacity_overflow_reports_and_truncates(orc):
+    x = torch.randn(1, 64, 64, 16)
+    y = x + 1
+    ref = orc.reduce_mask(x, y, 1e-3, [(64, 64, 4)], 1)[0]
+    got, cnt, ws = _gpu_lists(x, y, 1e-3, [(64, 64, 4, 100)])
+    assert cnt[0] == 256
+    assert np.array_equal(got[0], ref[:100])
+    assert sige.sige_get_error(ws) == sige.ERR_CAPACITY
+    assert sige.sige_get_error(ws) == sige.OK                # cleared
+    # the workspace is reusable and left zero-filled past its header
+    got, cnt, ws = _gpu_lists(x, y, 1e-3, [(64, 64, 4, 256)], workspace=ws)
+    assert cnt[0] == 256 and sige.sige_get_error(ws) == sige.OK
+    assert int(ws[256:].sum().item()) == 0
+
+
+def test_workspace_reuse_across_calls(orc):
+    ws = None
+    for seed in range(5):
+        o, e, _ = inputs.make_cfg2(seed)
+        ref = orc.reduce_mask(o, e, 0.0, inputs.CFG2_SCALES, 1, orc.NCHW)
+        got, _, ws = _gpu_lists(o, e, 0.0, _full_caps(inputs.CFG2_SCALES), 1, sige.NCHW, workspace=ws)
+        for s in range(4):
+            assert np.array_equal(got[s], ref[s])

@@ -33,8 +33,9 @@ __global__ void __launch_bounds__(kSimtThreads) k_conv_simt(const __grid_constan
         const int cog = u % ncog;
         const int tn = u / ncog;
         const int n = tn % p.N, t = tn / p.N;
-        int h0, w0;
-        tile_origin(p, t, h0, w0);
+        int h0 = 0, w0 = 0;
+        if (p.from_image || p.to_y)   // stacked blocks carry no tile list
+            tile_origin(p, t, h0, w0);
         const int o = cog * p.cob + ol;
         float acc[kSimtMaxQ];
 #pragma unroll

@@ -18,6 +18,8 @@
 //     block-wide prefix sum, write the (h0, w0) list and the count, then clear
 //     the flags and the arrival counter so the workspace is ready for the next
 //     call.
+#include <algorithm>
+
 #include "sige_internal.cuh"
 
 namespace sige {
@@ -50,8 +52,8 @@ struct MaskParams {
     int32_t epv;         // elements per vector
 };
 
-constexpr int kMaskThreads = 512;
-constexpr int kMaskUnroll = 4;
+constexpr int kMaskThreads = 256;
+constexpr int kMaskUnroll = 8;
 constexpr int kFlagSmem = 16384;
 
 __device__ __forceinline__ float elem_as_float(uint32_t word, int k, int dtype)
@@ -92,11 +94,14 @@ __device__ __forceinline__ uint32_t diff_bits16(uint4 a, uint4 b, int dtype, flo
     return bits;
 }
 
-__device__ __forceinline__ void mark(const MaskParams &p, int y, int x)
+// The scale table is indexed with a runtime scale number; kernel parameters
+// read that way go through generic loads, so every CTA first copies the table
+// into shared memory.
+__device__ __forceinline__ void mark(const ScaleParams *sc, int n_scales, uint8_t *flags, int y, int x)
 {
-    for (int s = 0; s < p.n_scales; ++s) {
-        const ScaleParams &q = p.sc[s];
-        p.flags[q.flag_off + (y / q.tile_h) * q.tw + (x / q.tile_w)] = 1;
+    for (int s = 0; s < n_scales; ++s) {
+        const ScaleParams q = sc[s];
+        flags[q.flag_off + (y / q.tile_h) * q.tw + (x / q.tile_w)] = 1;
     }
 }
 
@@ -109,30 +114,38 @@ __device__ __forceinline__ float scalar_elem(const uint8_t *base, int64_t i, int
     return reinterpret_cast<const float *>(base)[i];
 }
 
-__device__ void phase1(const MaskParams &p)
+__device__ __forceinline__ bool phase1(const MaskParams &p, const ScaleParams *sc)
 {
+    bool wrote = false;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t HW = (int64_t)p.H * p.W;
-    for (int64_t v0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v0 < p.nwork;
+    const int n_scales = p.n_scales, mode = p.mode, dtype = p.dtype, W = p.W, H = p.H, C = p.C;
+    const int vpp = p.vpp, epv = p.epv, layout = p.layout;
+    const float thr = p.thr;
+    const int64_t nwork = p.nwork;
+    const uint8_t *a = p.a, *b = p.b;
+    uint8_t *flags = p.flags;
+    for (int64_t v0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v0 < nwork;
          v0 += stride * kMaskUnroll) {
-        if (p.mode == 2) {
+        if (mode == 2) {
 #pragma unroll
             for (int u = 0; u < kMaskUnroll; ++u) {
                 int64_t i = v0 + u * stride;
-                if (i >= p.nwork)
+                if (i >= nwork)
                     break;
-                float d = fabsf(scalar_elem(p.b, i, p.dtype) - scalar_elem(p.a, i, p.dtype));
-                if (d > p.thr) {
+                float d = fabsf(scalar_elem(b, i, dtype) - scalar_elem(a, i, dtype));
+                if (d > thr) {
+                    wrote = true;
                     int y, x;
-                    if (p.layout == SIGE_NHWC) {
-                        int64_t pix = i / p.C;
-                        y = (int)((pix % HW) / p.W);
-                        x = (int)(pix % p.W);
+                    if (layout == SIGE_NHWC) {
+                        int64_t pix = i / C;
+                        y = (int)((pix % HW) / W);
+                        x = (int)(pix % W);
                     } else {
-                        y = (int)((i / p.W) % p.H);
-                        x = (int)(i % p.W);
+                        y = (int)((i / W) % H);
+                        x = (int)(i % W);
                     }
-                    mark(p, y, x);
+                    mark(sc, n_scales, flags, y, x);
                 }
             }
             continue;
@@ -141,110 +154,133 @@ __device__ void phase1(const MaskParams &p)
 #pragma unroll
         for (int u = 0; u < kMaskUnroll; ++u) {
             int64_t v = v0 + u * stride;
-            if (v < p.nwork) {
-                av[u] = ld_stream16(p.a + v * 16);
-                bv[u] = ld_stream16(p.b + v * 16);
+            if (v < nwork) {
+                av[u] = ld_stream16(a + v * 16);
+                bv[u] = ld_stream16(b + v * 16);
             }
         }
 #pragma unroll
         for (int u = 0; u < kMaskUnroll; ++u) {
             int64_t v = v0 + u * stride;
-            if (v >= p.nwork)
+            if (v >= nwork)
                 break;
-            uint32_t bits = diff_bits16(av[u], bv[u], p.dtype, p.thr);
+            uint32_t bits = diff_bits16(av[u], bv[u], dtype, thr);
             if (!bits)
                 continue;
-            if (p.mode == 0) {
-                int64_t pix = v / p.vpp;
-                mark(p, (int)((pix % HW) / p.W), (int)(pix % p.W));
+            wrote = true;
+            if (mode == 0) {
+                int64_t pix = v / vpp;
+                mark(sc, n_scales, flags, (int)((pix % HW) / W), (int)(pix % W));
             } else {
-                int64_t e0 = v * p.epv;
-                int y = (int)((e0 / p.W) % p.H);
-                int x0 = (int)(e0 % p.W);
+                int64_t e0 = v * epv;
+                int y = (int)((e0 / W) % H);
+                int x0 = (int)(e0 % W);
                 while (bits) {
                     int k = __ffs(bits) - 1;
                     bits &= bits - 1;
-                    mark(p, y, x0 + k);
+                    mark(sc, n_scales, flags, y, x0 + k);
                 }
             }
         }
     }
+    return wrote;
 }
 
-// Block-wide exclusive prefix sum of one bit per thread; returns the offset of
-// this thread and writes the block total to *total (all threads).
-__device__ __forceinline__ int block_scan_bit(int bit, int *warp_sums, int *total)
+// Block-wide exclusive prefix sum of one int per thread; *total gets the sum.
+__device__ __forceinline__ int block_scan(int v, int *warp_sums, int *total)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    uint32_t ballot = __ballot_sync(0xFFFFFFFFu, bit);
-    int in_warp = __popc(ballot & ((1u << lane) - 1u));
-    if (lane == 0)
-        warp_sums[warp] = __popc(ballot);
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o)
+            incl += t;
+    }
+    if (lane == 31)
+        warp_sums[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        int v = lane < nw ? warp_sums[lane] : 0;
-        int incl = v;
+        const int w = lane < nw ? warp_sums[lane] : 0;
+        int wi = w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            const int t = __shfl_up_sync(0xFFFFFFFFu, wi, o);
             if (lane >= o)
-                incl += t;
+                wi += t;
         }
         if (lane < nw)
-            warp_sums[lane] = incl - v;
+            warp_sums[lane] = wi - w;
         if (lane == 31)
-            warp_sums[32] = incl;
+            warp_sums[32] = wi;
     }
     __syncthreads();
-    int off = warp_sums[warp] + in_warp;
+    const int off = warp_sums[warp] + incl - v;
     *total = warp_sums[32];
     __syncthreads();
     return off;
 }
 
-__device__ void phase2(const MaskParams &p)
+constexpr int kTilesPerThread = 4;
+
+__device__ __forceinline__ void phase2(const MaskParams &p, const ScaleParams *sc)
 {
     __shared__ uint8_t sflag[kFlagSmem];
     __shared__ int warp_sums[33];
-    for (int s = 0; s < p.n_scales; ++s) {
-        const ScaleParams &q = p.sc[s];
+    const int n_scales = p.n_scales, dilate = p.dilate;
+    for (int s = 0; s < n_scales; ++s) {
+        const ScaleParams q = sc[s];
         const int nt = q.th * q.tw;
         const uint8_t *g = p.flags + q.flag_off;
         const bool in_smem = nt <= kFlagSmem;
         if (in_smem) {
-            for (int t = threadIdx.x * 4; t < nt; t += blockDim.x * 4) {
-                // flag_off is 16-byte aligned, so 4-byte reads stay in bounds of
-                // the 16-byte-padded flag area
-                uint32_t w = __ldcg(reinterpret_cast<const unsigned int *>(g + t));
-                for (int k = 0; k < 4 && t + k < nt; ++k)
-                    sflag[t + k] = (uint8_t)((w >> (8 * k)) & 0xFF);
+            // flag_off is 16-byte aligned and the flag area is padded to 16
+            // bytes, so these 16-byte reads stay inside it
+            for (int t = threadIdx.x * 16; t < nt; t += blockDim.x * 16) {
+                const uint4 w = __ldcg(reinterpret_cast<const uint4 *>(g + t));
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    if (t + k < nt)
+                        sflag[t + k] = (uint8_t)((ws[k >> 2] >> (8 * (k & 3))) & 0xFF);
             }
             __syncthreads();
         }
         int base = 0;
-        for (int t0 = 0; t0 < nt; t0 += blockDim.x) {
-            const int t = t0 + threadIdx.x;
-            int act = 0, i = 0, j = 0;
-            if (t < nt) {
-                i = t / q.tw;
-                j = t - i * q.tw;
-                const int i0 = max(0, i - p.dilate), i1 = min(q.th - 1, i + p.dilate);
-                const int j0 = max(0, j - p.dilate), j1 = min(q.tw - 1, j + p.dilate);
+        const int chunk = blockDim.x * kTilesPerThread;
+        for (int t0 = 0; t0 < nt; t0 += chunk) {
+            const int tb = t0 + threadIdx.x * kTilesPerThread;
+            uint32_t bits = 0;
+#pragma unroll
+            for (int k = 0; k < kTilesPerThread; ++k) {
+                const int t = tb + k;
+                if (t >= nt)
+                    break;
+                const int i = t / q.tw, j = t - i * q.tw;
+                const int i0 = max(0, i - dilate), i1 = min(q.th - 1, i + dilate);
+                const int j0 = max(0, j - dilate), j1 = min(q.tw - 1, j + dilate);
+                int act = 0;
                 for (int ii = i0; ii <= i1 && !act; ++ii)
                     for (int jj = j0; jj <= j1; ++jj) {
-                        uint8_t f = in_smem ? sflag[ii * q.tw + jj] : __ldcg(g + ii * q.tw + jj);
+                        const uint8_t f = in_smem ? sflag[ii * q.tw + jj] : __ldcg(g + ii * q.tw + jj);
                         if (f) {
                             act = 1;
                             break;
                         }
                     }
+                bits |= (uint32_t)act << k;
             }
             int chunk_total;
-            const int off = block_scan_bit(act, warp_sums, &chunk_total);
-            const int pos = base + off;
-            if (act && pos < q.capacity) {
-                int2 v = make_int2(i * q.block, j * q.block);
-                reinterpret_cast<int2 *>(p.idx)[q.idx_off + pos] = v;
+            int pos = base + block_scan(__popc(bits), warp_sums, &chunk_total);
+            while (bits) {
+                const int k = __ffs(bits) - 1;
+                bits &= bits - 1;
+                if (pos < q.capacity) {
+                    const int t = tb + k;
+                    const int i = t / q.tw, j = t - i * q.tw;
+                    reinterpret_cast<int2 *>(p.idx)[q.idx_off + pos] = make_int2(i * q.block, j * q.block);
+                }
+                ++pos;
             }
             base += chunk_total;
         }
@@ -256,7 +292,7 @@ __device__ void phase2(const MaskParams &p)
         __syncthreads();
     }
     // leave the workspace zero-filled for the next call
-    uint4 z = make_uint4(0, 0, 0, 0);
+    const uint4 z = make_uint4(0, 0, 0, 0);
     for (int k = threadIdx.x; k < p.flag_bytes / 16; k += blockDim.x)
         reinterpret_cast<uint4 *>(p.flags)[k] = z;
     if (threadIdx.x == 0)
@@ -265,8 +301,12 @@ __device__ void phase2(const MaskParams &p)
 
 __global__ void __launch_bounds__(kMaskThreads) k_mask_reduce(const __grid_constant__ MaskParams p)
 {
-    phase1(p);
-    __threadfence();
+    __shared__ ScaleParams s_sc[kMaxScales];
+    if (threadIdx.x < kMaxScales)
+        s_sc[threadIdx.x] = p.sc[threadIdx.x];
+    __syncthreads();
+    if (phase1(p, s_sc))
+        __threadfence();   // flags stored by this thread are visible before the arrival below
     __syncthreads();
     __shared__ int is_last;
     if (threadIdx.x == 0) {
@@ -277,7 +317,7 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask_reduce(const __grid_const
     if (!is_last)
         return;
     __threadfence();
-    phase2(p);
+    phase2(p, s_sc);
 }
 
 // ------------------------------------------------------------------ host
@@ -388,8 +428,19 @@ extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const si
         p.mode = 2;
         p.nwork = nelem;
     }
+    static int occ[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64)
+        dev = 0;
+    if (!occ[dev]) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_mask_reduce, kMaskThreads, 0) != cudaSuccess || n < 1)
+            n = 1;
+        occ[dev] = n;
+    }
     int64_t per_cta = (int64_t)kMaskThreads * kMaskUnroll;
-    int grid = (int)std::min<int64_t>((p.nwork + per_cta - 1) / per_cta, (int64_t)device_sm_count() * 4);
+    int grid = (int)std::min<int64_t>((p.nwork + per_cta - 1) / per_cta, (int64_t)device_sm_count() * occ[dev]);
     grid = std::max(grid, 1);
     k_mask_reduce<<<grid, kMaskThreads, 0, (cudaStream_t)stream>>>(p);
     count_launch();

@@ -38,7 +38,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__device__ __forceinline__ float silu_f(float v) { return v / (1.0f + __expf(-v)); }
+// SiLU v * sigmoid(v) = v / (1 + e^-v); __fdividef returns 0 once the
+// denominator overflows, which is the limit of SiLU for v -> -inf.
+__device__ __forceinline__ float silu_f(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
 
 // 16-byte loads/stores.
 __device__ __forceinline__ uint4 ld_stream16(const void *p)

@@ -41,6 +41,29 @@ __device__ __forceinline__ uint4 transform16(uint4 in, int dtype, const float *s
     return out;
 }
 
+// transform16 for 8 bf16 channels whose affine parameters are in registers.
+__device__ __forceinline__ uint4 transform16_bf16_reg(uint4 in, const float (&sc)[8], const float (&sh)[8],
+                                                      bool affine, int silu)
+{
+    uint4 out;
+    uint32_t *o = reinterpret_cast<uint32_t *>(&out);
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(&in);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float a = bf16_lo(w[q]), b = bf16_hi(w[q]);
+        if (affine) {
+            a = __fmaf_rn(a, sc[2 * q], sh[2 * q]);
+            b = __fmaf_rn(b, sc[2 * q + 1], sh[2 * q + 1]);
+        }
+        if (silu) {
+            a = silu_f(a);
+            b = silu_f(b);
+        }
+        o[q] = pack_bf16x2(a, b);
+    }
+    return out;
+}
+
 __device__ __forceinline__ float load_elem(const uint8_t *base, int64_t e, int dtype)
 {
     if (dtype == SIGE_BF16)

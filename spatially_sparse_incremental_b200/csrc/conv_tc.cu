@@ -46,12 +46,14 @@
 
 namespace sige {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 320;              // warp 0 TMA, warp 1 MMA, warps 2-9 halo + epilogue
+constexpr int kProd = 256;                    // halo / epilogue threads
 constexpr uint32_t kAStageBytes = 128 * 64 * 2;
 constexpr int kMaxSplit = 32;
 constexpr long long kWaitCycles = 1ll << 31;   // ~1.1 s at 1.9 GHz
 constexpr int kSmemLimit = 232448;             // 227 KB opt-in per CTA
-constexpr int kSmemFloor = 120 * 1024;         // keeps one CTA (and one TMEM owner) per SM
+constexpr int kMaxSA = 16;                     // weight stages at most
+constexpr uint32_t kCtrlBytes = 4096;          // barriers, flags, tile origins
 
 // Flat argument block.  The kernel copies it into a local at entry: fields of
 // a kernel parameter read through a reference (non-inlined helpers, or after an
@@ -79,10 +81,12 @@ struct TcArgs {
     int32_t taps, kci;        // k*k, C_in / 64
     int32_t MT;               // output-channel tiles of 128
     int32_t T_max;            // ROW: tiles per unit; POS: slots (multiple of 16)
-    int32_t SA, SB;           // pipeline stages
-    uint32_t b_off, bar_off, stage_b;
+    int32_t SB;               // halo stages (the weight stage count is set per launch from the unit size)
+    uint32_t per_slot;        // bytes of one tile (ROW) or slot (POS) per halo stage
+    uint32_t smem_bytes;      // dynamic shared memory of the launch
     int32_t ncols;            // tensor-memory columns allocated (power of 2)
     int32_t num_sms;
+    int32_t halo_tma;         // 1: ROW-mode halo rows come by TMA (tmx), 0: per-thread cp.async
 };
 
 __device__ __forceinline__ void tile_origin_a(const TcArgs &a, int t, int &h0, int &w0)
@@ -158,6 +162,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1, int c2,
+                                            int c3, int c4)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+        : "memory");
+}
+
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -229,7 +242,9 @@ __device__ __forceinline__ Sched make_sched(const TcArgs &p, int G)
         s.T = min(p.T_max, ((want + 15) / 16) * 16);
     s.TB = (G + s.T - 1) / s.T;
     const int KC = p.taps * p.kci;
-    s.S = max(1, min(p.num_sms / max(1, s.TB * p.MT), min(KC, kMaxSplit)));
+    // split K only where each split keeps a long K loop: below that the extra
+    // round trip of the partial sums costs more than the shorter loop saves
+    s.S = max(1, min(p.num_sms / max(1, s.TB * p.MT), min(KC / 12, kMaxSplit)));
     s.units = s.TB * p.MT * s.S;
     return s;
 }
@@ -251,6 +266,31 @@ __device__ __forceinline__ Unit decode_unit(const TcArgs &p, const Sched &s, int
     return r;
 }
 
+// ------------------------------------------------------------------ shared-memory carve-up
+//
+//   [0, 1024)        mbarriers and control words
+//   [1024, 3072)     tile origins of the current unit (256 x int2)
+//   [4096, ...)      weight stages, 16 KB each, as many as fit (<= 16)
+//   [.., end)        SB halo stages of T slots each; reused as the epilogue's
+//                    staging buffer once the unit's MMAs are complete
+
+struct Carve {
+    uint32_t a_base;    // byte offset of weight stage 0
+    uint32_t b_base;    // byte offset of halo stage 0
+    uint32_t stage_b;   // bytes per halo stage
+    int SA;             // weight stages
+};
+
+__device__ __forceinline__ Carve carve(const TcArgs &p, int T)
+{
+    Carve c;
+    c.stage_b = (uint32_t)T * p.per_slot;
+    c.b_base = (p.smem_bytes - 1024 - p.SB * c.stage_b) & ~15u;
+    c.a_base = kCtrlBytes;
+    c.SA = min(kMaxSA, (int)((c.b_base - c.a_base) / kAStageBytes));
+    return c;
+}
+
 // ------------------------------------------------------------------ B staging
 
 // Byte offset of (tile slot, halo row, halo col, 16-byte channel group) in a B stage.
@@ -263,27 +303,69 @@ __device__ __forceinline__ uint32_t b_offset(const TcArgs &p, int slots, int slo
     return (uint32_t)((((hh * bin + ww) * 8 + kc) * slots + slot) * 16);
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+// Source of one 16-byte halo chunk, or nullptr where the conv's zero padding
+// (or a tile past the list) applies.
+__device__ __forceinline__ const uint8_t *halo_src(const TcArgs &c, const int2 *s_orig, int T, int tb, int G, int slot,
+                                                   int hh, int ww, int pix, int ch)
+{
+    const int g = tb * T + slot;
+    if (g >= G)
+        return nullptr;
+    if (!c.from_image)
+        return c.src + (((int64_t)g * c.bin * c.bin + pix) * c.Cin + ch) * 2;
+    const int2 o = s_orig[slot];
+    const int y = o.x * c.s - c.pad + hh, x = o.y * c.s - c.pad + ww;
+    if (y < 0 || y >= c.H || x < 0 || x >= c.W)
+        return nullptr;
+    return c.src + ((((int64_t)(g % c.N) * c.H + y) * c.W + x) * c.Cin + ch) * 2;
+}
+
 // Fill one B stage: 64 input channels (chunk q) of the halo of every tile of
-// the unit, transformed and zero-padded, in the core-matrix layout.
-__device__ __forceinline__ void fill_b(const TcArgs &p, const Sched &s, int tb, int q, int G, uint8_t *stage, int et,
+// the unit, in the core-matrix layout.  Every chunk is one 16-byte cp.async
+// (zero-filled for padding), all in flight at once; then the GroupNorm affine
+// and SiLU are applied in place.  Thread et always handles channel group
+// kc = et & 7 and pixels (et >> 3) + (kProd / 8) k, walked incrementally.
+__device__ __forceinline__ void fill_b(const TcArgs &c, int T, int tb, int q, int G, uint8_t *stage, int et,
                                        const int2 *s_orig)
 {
-    const TcArgs &c = p;
-    const int bin2 = c.bin * c.bin;
-    const int slots = s.T;
-    const int n_ent = slots * bin2 * 8;
-    const bool affine = c.gsc != nullptr;
-    const bool xform = affine || c.silu;
-    // entries e = et + 128 k all share the 16-byte channel group kc = et & 7,
-    // so a thread needs the affine parameters of 8 channels only
+    const int bin = c.bin, bin2 = bin * bin;
     const int kc = et & 7;
     const int ch = q * 64 + kc * 8;
+    const uint32_t sbase = smem_u32(stage);
+    const int lin0 = et >> 3;
+    const int slot0 = lin0 / bin2, pix0 = lin0 - slot0 * bin2;
+    const int hh0 = pix0 / bin, ww0 = pix0 - hh0 * bin;
+    {
+        int slot = slot0, hh = hh0, ww = ww0;
+#pragma unroll 1
+        while (slot < T) {
+            const uint8_t *src = halo_src(c, s_orig, T, tb, G, slot, hh, ww, hh * bin + ww, ch);
+            cp_async16(sbase + b_offset(c, T, slot, hh, ww, kc), src ? src : c.src, src ? 16u : 0u);
+            ww += kProd / 8;
+            while (ww >= bin) {
+                ww -= bin;
+                if (++hh == bin) {
+                    hh = 0;
+                    ++slot;
+                }
+            }
+        }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (c.gsc == nullptr && !c.silu)
+        return;
     float gsc[8], gsh[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
         gsc[k] = 1.0f;
         gsh[k] = 0.0f;
     }
+    const bool affine = c.gsc != nullptr;
     if (affine && c.N == 1) {
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -291,180 +373,180 @@ __device__ __forceinline__ void fill_b(const TcArgs &p, const Sched &s, int tb, 
             gsh[k] = __ldg(c.gsh + ch + k);
         }
     }
-    constexpr int U = 8;
-    for (int e0 = et; e0 < n_ent; e0 += 128 * U) {
-        uint4 v[U];
-        uint32_t dst[U];
-        int gsel[U];
-        bool inb[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int e = e0 + u * 128;
-            inb[u] = false;
-            v[u] = make_uint4(0, 0, 0, 0);
-            dst[u] = 0xFFFFFFFFu;
-            gsel[u] = 0;
-            if (e >= n_ent)
-                continue;
-            const int pix = (e >> 3) % bin2;
-            const int slot = (e >> 3) / bin2;
-            const int hh = pix / c.bin, ww = pix % c.bin;
-            dst[u] = b_offset(p, slots, slot, hh, ww, kc);
-            const int g = tb * s.T + slot;
-            gsel[u] = g;
-            if (g >= G)
-                continue;
-            const uint8_t *src;
-            if (c.from_image) {
-                const int2 o = s_orig[slot];
-                const int y = o.x * c.s - c.pad + hh, x = o.y * c.s - c.pad + ww;
-                if (y < 0 || y >= c.H || x < 0 || x >= c.W)
-                    continue;
-                const int n = g % c.N;
-                src = c.src + ((((int64_t)n * c.H + y) * c.W + x) * c.Cin + ch) * 2;
+    int slot = slot0, hh = hh0, ww = ww0;
+#pragma unroll 1
+    while (slot < T) {
+        if (halo_src(c, s_orig, T, tb, G, slot, hh, ww, hh * bin + ww, ch)) {
+            uint4 *d = reinterpret_cast<uint4 *>(stage + b_offset(c, T, slot, hh, ww, kc));
+            if (affine && c.N > 1) {
+                const int n = (tb * T + slot) % c.N;
+                *d = transform16(*d, SIGE_BF16, c.gsc + (int64_t)n * c.Cin + ch, c.gsh + (int64_t)n * c.Cin + ch,
+                                 c.silu);
             } else {
-                src = c.src + (((int64_t)g * bin2 + pix) * c.Cin + ch) * 2;
+                *d = transform16_bf16_reg(*d, gsc, gsh, affine, c.silu);
             }
-            v[u] = ld_nc16(src);
-            inb[u] = true;
         }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            if (dst[u] == 0xFFFFFFFFu)
-                continue;
-            uint4 w = v[u];
-            if (inb[u] && xform) {
-                if (affine && c.N > 1) {
-                    const int n = gsel[u] % c.N;
-                    w = transform16(w, SIGE_BF16, c.gsc + (int64_t)n * c.Cin + ch, c.gsh + (int64_t)n * c.Cin + ch,
-                                    c.silu);
-                } else {
-                    w = transform16_bf16_reg(w, gsc, gsh, affine, c.silu);
-                }
+        ww += kProd / 8;
+        while (ww >= bin) {
+            ww -= bin;
+            if (++hh == bin) {
+                hh = 0;
+                ++slot;
             }
-            *reinterpret_cast<uint4 *>(stage + dst[u]) = w;
+        }
+    }
+}
+
+// In-place GroupNorm affine + SiLU of a B stage whose raw halo arrived by TMA
+// (zero-filled outside the image); padding entries are left at zero.
+__device__ __forceinline__ void transform_b(const TcArgs &c, int T, int tb, int q, int G, uint8_t *stage, int et,
+                                            const int2 *s_orig)
+{
+    if (c.gsc == nullptr && !c.silu)
+        return;
+    const int bin = c.bin, bin2 = bin * bin;
+    const int kc = et & 7;
+    const int ch = q * 64 + kc * 8;
+    const bool affine = c.gsc != nullptr;
+    float gsc[8], gsh[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        gsc[k] = affine && c.N == 1 ? __ldg(c.gsc + ch + k) : 1.0f;
+        gsh[k] = affine && c.N == 1 ? __ldg(c.gsh + ch + k) : 0.0f;
+    }
+    const int lin0 = et >> 3;
+    int slot = lin0 / bin2, pix = lin0 - slot * bin2;
+    int hh = pix / bin, ww = pix - hh * bin;
+#pragma unroll 1
+    while (slot < T) {
+        if (halo_src(c, s_orig, T, tb, G, slot, hh, ww, hh * bin + ww, ch)) {
+            uint4 *d = reinterpret_cast<uint4 *>(stage + b_offset(c, T, slot, hh, ww, kc));
+            if (affine && c.N > 1) {
+                const int n = (tb * T + slot) % c.N;
+                *d = transform16(*d, SIGE_BF16, c.gsc + (int64_t)n * c.Cin + ch, c.gsh + (int64_t)n * c.Cin + ch,
+                                 c.silu);
+            } else {
+                *d = transform16_bf16_reg(*d, gsc, gsh, affine, c.silu);
+            }
+        }
+        ww += kProd / 8;
+        while (ww >= bin) {
+            ww -= bin;
+            if (++hh == bin) {
+                hh = 0;
+                ++slot;
+            }
         }
     }
 }
 
 // ------------------------------------------------------------------ epilogue
 
-// Write 16 consecutive accumulator columns (pixels) of one output channel.
-// Addresses are computed first and every load (residual) is issued before the
-// first store, so the 16 loads are in flight together.
-__device__ __forceinline__ void emit16(const TcArgs &p, const Sched &s, const int2 *s_orig, int tb, int c0,
-                                       int co, float bias_c, const float (&v)[16], int G)
+__device__ __forceinline__ int unit_cols(const TcArgs &p, int T)
 {
-    const TcArgs &c = p;
-    int64_t e[16];
-    bool ok[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const int col = c0 + k;
-        int slot, i, j;
-        if (p.mode == 0) {
-            slot = col >> 6;
-            i = (col >> 3) & 7;
-            j = col & 7;
-        } else {
-            const int pos = col / s.T;
-            slot = col - pos * s.T;
-            i = pos / c.b;
-            j = pos - i * c.b;
-        }
-        const int g = tb * s.T + slot;
-        ok[k] = g < G && co < c.Cout;
-        e[k] = 0;
-        if (ok[k]) {
-            if (c.to_y) {
-                const int2 o = s_orig[slot];
-                const int yo = o.x + i, xo = o.y + j;
-                ok[k] = yo < c.Ho && xo < c.Wo;
-                e[k] = (((int64_t)(g % c.N) * c.Ho + yo) * c.Wo + xo) * c.Cout + co;
-            } else {
-                e[k] = (((int64_t)g * c.b + i) * c.b + j) * c.Cout + co;
-            }
-        }
-    }
-    if (c.to_y) {
-        float r[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            r[k] = 0.0f;
-            if (ok[k] && c.residual) {
-                if (c.dtype == SIGE_BF16)
-                    r[k] = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(c.residual) + e[k]) << 16);
-                else
-                    r[k] = __ldg(reinterpret_cast<const float *>(c.residual) + e[k]);
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            if (!ok[k])
-                continue;
-            const float y = (v[k] + bias_c) + r[k];
-            if (c.dtype == SIGE_BF16)
-                reinterpret_cast<__nv_bfloat16 *>(c.y)[e[k]] = __float2bfloat16_rn(y);
-            else
-                reinterpret_cast<float *>(c.y)[e[k]] = y;
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-            if (ok[k])
-                c.out_blocks[e[k]] = v[k];
-    }
+    return p.mode == 0 ? T * 64 : p.b * p.b * T;
 }
 
-__device__ __forceinline__ int unit_cols(const TcArgs &p, const Sched &s)
+// Pixel of accumulator column `col`: returns the flat element index of its
+// first channel `co0` in the destination, or -1 when the column is not a
+// pixel to write (past the list, outside the image).
+__device__ __forceinline__ int64_t col_target(const TcArgs &c, const int2 *s_orig, int T, int tb, int G, int col,
+                                              int co0)
 {
-    return p.mode == 0 ? s.T * 64 : p.b * p.b * s.T;
+    int slot, i, j;
+    if (c.mode == 0) {
+        slot = col >> 6;
+        i = (col >> 3) & 7;
+        j = col & 7;
+    } else {
+        const int pos = col / T;
+        slot = col - pos * T;
+        i = pos / c.b;
+        j = pos - i * c.b;
+    }
+    const int g = tb * T + slot;
+    if (g >= G)
+        return -1;
+    if (c.to_y) {
+        const int2 o = s_orig[slot];
+        const int yo = o.x + i, xo = o.y + j;
+        if (yo >= c.Ho || xo >= c.Wo)
+            return -1;
+        return (((int64_t)(g % c.N) * c.Ho + yo) * c.Wo + xo) * c.Cout + co0;
+    }
+    return (((int64_t)g * c.b + i) * c.b + j) * c.Cout + co0;
+}
+
+// Write 8 (bf16) or 4 (float32) consecutive channels of one pixel: bias,
+// residual (already loaded: rw), one rounding, one 16-byte store.
+__device__ __forceinline__ void store_vec(const TcArgs &c, int64_t e, const float *v, const float *bias8, uint4 rw)
+{
+    if (!c.to_y) {
+        *reinterpret_cast<float4 *>(c.out_blocks + e) = make_float4(v[0], v[1], v[2], v[3]);
+        return;
+    }
+    if (c.dtype == SIGE_BF16) {
+        const float r[8] = {bf16_lo(rw.x), bf16_hi(rw.x), bf16_lo(rw.y), bf16_hi(rw.y),
+                            bf16_lo(rw.z), bf16_hi(rw.z), bf16_lo(rw.w), bf16_hi(rw.w)};
+        uint4 o;
+        o.x = pack_bf16x2((v[0] + bias8[0]) + r[0], (v[1] + bias8[1]) + r[1]);
+        o.y = pack_bf16x2((v[2] + bias8[2]) + r[2], (v[3] + bias8[3]) + r[3]);
+        o.z = pack_bf16x2((v[4] + bias8[4]) + r[4], (v[5] + bias8[5]) + r[5]);
+        o.w = pack_bf16x2((v[6] + bias8[6]) + r[6], (v[7] + bias8[7]) + r[7]);
+        *reinterpret_cast<uint4 *>(c.y + e * 2) = o;
+    }
 }
 
 // ------------------------------------------------------------------ kernel
 
 __global__ void __launch_bounds__(kTcThreads, 1)
-    k_conv_tc(const __grid_constant__ TcArgs args, const __grid_constant__ CUtensorMap tmw)
+    k_conv_tc(const __grid_constant__ TcArgs args, const __grid_constant__ CUtensorMap tmw,
+              const __grid_constant__ CUtensorMap tmx)
 {
     const TcArgs p = args;   // registers, see TcArgs
+    const TcArgs &c = p;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw_addr + 1023) & ~1023u) - raw_addr);
     const uint32_t sbase = smem_u32(smem);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.bar_off);
-    const uint32_t bar0 = smem_u32(bars);
+    const uint32_t bar0 = sbase;
     auto a_full = [&](int i) { return bar0 + 8u * i; };
-    auto a_empty = [&](int i) { return bar0 + 8u * (p.SA + i); };
-    auto b_full = [&](int i) { return bar0 + 8u * (2 * p.SA + i); };
-    auto b_empty = [&](int i) { return bar0 + 8u * (2 * p.SA + p.SB + i); };
-    const uint32_t acc_full = bar0 + 8u * (2 * p.SA + 2 * p.SB);
+    auto a_empty = [&](int i) { return bar0 + 8u * (kMaxSA + i); };
+    auto b_full = [&](int i) { return bar0 + 8u * (2 * kMaxSA + i); };
+    auto b_empty = [&](int i) { return bar0 + 8u * (2 * kMaxSA + 2 + i); };
+    const uint32_t acc_full = bar0 + 8u * (2 * kMaxSA + 4);
     const uint32_t acc_empty = acc_full + 8u;
     const uint32_t drain = acc_full + 16u;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * p.SA + 2 * p.SB + 3);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    auto b_load = [&](int i) { return acc_full + 24u + 8u * i; };   // halo TMA arrivals
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 512);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 516);
     volatile int *bcast = abort_flag + 1;
     volatile int *group_ok = abort_flag + 2;
-    int2 *s_orig = reinterpret_cast<int2 *>(smem + p.bar_off + 1024);   // tile origins of the current unit
+    int2 *s_orig = reinterpret_cast<int2 *>(smem + 1024);
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < p.SA; ++i) {
+        for (int i = 0; i < kMaxSA; ++i) {
             mbar_init(a_full(i), 1);
             mbar_init(a_empty(i), 1);
         }
         for (int i = 0; i < p.SB; ++i) {
-            mbar_init(b_full(i), 128);
+            mbar_init(b_full(i), kProd);
             mbar_init(b_empty(i), 1);
+            mbar_init(b_load(i), 1);
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 128);
+        mbar_init(acc_empty, kProd);
         mbar_init(drain, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0 && lane == 0)
+    if (warp == 0 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmw)) : "memory");
+        if (args.halo_tma)
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmx)) : "memory");
+    }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(p.ncols));
@@ -475,44 +557,74 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    const TcArgs &c = p;
     const int ntile = c.dense ? c.tiles_total : min(__ldg(c.count), c.cap);
     const int G = ntile * c.N;
     const Sched sc = make_sched(p, G);
+    const Carve cv = carve(p, sc.T);
 
     if (warp == 0) {
         // ---------------- weight producer (TMA)
         if (lane == 0) {
-            uint32_t it = 0;
+            // stage index and phase advance incrementally: a runtime division
+            // per k-chunk costs more than the TMA issue itself
+            int s = 0;
+            uint32_t ph = 1, issued = 0;
             bool ok = true;
+#pragma unroll 1
             for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, sc, u);
+                int q = un.kb / p.taps, tap = un.kb - q * p.taps;
+                const int y0 = un.mt * 128;
+#pragma unroll 1
                 for (int kc = un.kb; kc < un.ke; ++kc) {
-                    const int s = it % p.SA;
-                    if (!mbar_wait(a_empty(s), ((it / p.SA) & 1) ^ 1, abort_flag, hdr, 1)) {
+                    if (!mbar_wait(a_empty(s), ph, abort_flag, hdr, 1)) {
                         ok = false;
                         break;
                     }
-                    const int q = kc / p.taps, tap = kc - q * p.taps;
                     mbar_expect_tx(a_full(s), kAStageBytes);
-                    tma_load_2d(sbase + s * kAStageBytes, &tmw, a_full(s), tap * c.Cin + q * 64, un.mt * 128);
-                    ++it;
+                    tma_load_2d(sbase + cv.a_base + s * kAStageBytes, &tmw, a_full(s), tap * c.Cin + q * 64, y0);
+                    ++issued;
+                    if (++s == cv.SA) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                    if (++tap == p.taps) {
+                        tap = 0;
+                        ++q;
+                    }
                 }
             }
-            // drain: every issued load must land before the CTA may exit
-            for (uint32_t k = (it > (uint32_t)p.SA ? it - p.SA : 0); k < it; ++k) {
-                const int s = k % p.SA;
+            // every issued load must land before the CTA may exit: wait for the
+            // last use of each stage
+#pragma unroll 1
+            for (uint32_t k = 0; k < (uint32_t)cv.SA && k < issued; ++k) {
+                // the use of stage st waited on a_empty with parity w, so its
+                // a_full completion has parity w ^ 1; w is ph for stages used
+                // in the current round and ph ^ 1 for those before the wrap
+                int st = s - 1 - (int)k;
+                uint32_t full_par = ph ^ 1;
+                if (st < 0) {
+                    st += cv.SA;
+                    full_par ^= 1;
+                }
                 const long long t0 = clock64();
-                while (!mbar_try(a_full(s), (k / p.SA) & 1) && clock64() - t0 < kWaitCycles) {
+                while (!mbar_try(a_full(st), full_par) && clock64() - t0 < kWaitCycles) {
                 }
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer
         if (lane == 0) {
-            uint32_t ait = 0, bit = 0, uit = 0;
+            int sa = 0, sb = 0;
+            uint32_t pa = 0, pb = 0, uit = 0, ait = 0;
             bool ok = true;
             const int bin = c.bin;
+            const int n_mma = p.mode == 0 ? 64 : sc.T;
+            const uint32_t idesc = idesc_bf16(n_mma);
+            const uint32_t sk = p.mode == 0 ? (uint32_t)bin * 16 : (uint32_t)sc.T * 16;   // LBO
+            const uint32_t sh = 8 * sk;      // ROW: halo row stride; POS: halo pixel stride
+            const uint64_t tile_step = (uint64_t)((bin * sh) >> 4);
+#pragma unroll 1
             for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, sc, u);
                 if (uit > 0 && !mbar_wait(acc_empty, (uit - 1) & 1, abort_flag, hdr, 2)) {
@@ -520,54 +632,75 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                const int n_mma = p.mode == 0 ? 64 : sc.T;
-                const uint32_t idesc = idesc_bf16(n_mma);
-                const uint32_t sk = p.mode == 0 ? (uint32_t)bin * 16 : (uint32_t)sc.T * 16;   // LBO
-                int sb = 0;
+                int q = un.kb / p.taps, tap = un.kb - q * p.taps;
+                int r = tap / c.k, cc = tap - r * c.k;
+#pragma unroll 1
                 for (int kc = un.kb; kc < un.ke; ++kc) {
-                    const int q = kc / p.taps, tap = kc - q * p.taps;
                     if (kc == un.kb || tap == 0) {
-                        sb = bit % p.SB;
-                        if (!mbar_wait(b_full(sb), (bit / p.SB) & 1, abort_flag, hdr, 3)) {
+                        if (!mbar_wait(b_full(sb), pb, abort_flag, hdr, 3)) {
                             ok = false;
                             break;
                         }
                     }
-                    const int sa = ait % p.SA;
-                    if (!mbar_wait(a_full(sa), (ait / p.SA) & 1, abort_flag, hdr, 4)) {
+                    if (!mbar_wait(a_full(sa), pa, abort_flag, hdr, 4)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int r = tap / c.k, cc = tap - r * c.k;
-                    const uint32_t a_base = sbase + sa * kAStageBytes;
-                    const uint32_t b_base = sbase + p.b_off + sb * p.stage_b;
-                    const bool first = (kc == un.kb);
+                    const uint32_t a_base = sbase + cv.a_base + sa * kAStageBytes;
+                    const uint32_t b_base = sbase + cv.b_base + sb * cv.stage_b;
+                    const uint32_t acc0 = (kc == un.kb) ? 0u : 1u;
+                    // descriptors differ only in their start address field
+                    // (address >> 4, low bits), so offsets are added directly
+                    const uint64_t ad0 = desc_sw128(a_base);
+                    if (p.mode == 0) {
+                        const uint64_t bd0 = desc_plain(b_base + r * sh + cc * 16, sk, sh);
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t ad = desc_sw128(a_base + ks * 32);
-                        const uint32_t acc = (first && ks == 0) ? 0u : 1u;
-                        if (p.mode == 0) {
-                            const uint32_t sh = 8 * sk;  // halo row stride
-                            for (int t = 0; t < sc.T; ++t) {
-                                const uint32_t bs = b_base + t * bin * sh + r * sh + cc * 16 + 2 * ks * sk;
-                                tc_mma(tmem + t * 64, ad, desc_plain(bs, sk, sh), idesc, acc);
-                            }
-                        } else {
-                            const uint32_t sp = 8 * sk;  // halo pixel stride
-                            for (int pos = 0; pos < c.b * c.b; ++pos) {
-                                const int i = pos / c.b, j = pos - i * c.b;
-                                const uint32_t bs =
-                                    b_base + ((i * c.s + r) * bin + (j * c.s + cc)) * sp + 2 * ks * sk;
-                                tc_mma(tmem + pos * sc.T, ad, desc_plain(bs, sk, 128), idesc, acc);
+                        for (int ks = 0; ks < 4; ++ks) {
+                            const uint64_t bk = bd0 + (uint64_t)((2 * ks * sk) >> 4);
+#pragma unroll 1
+                            for (int t = 0; t < sc.T; ++t)
+                                tc_mma(tmem + t * 64, ad0 + (uint64_t)(2 * ks), bk + t * tile_step, idesc,
+                                       ks == 0 ? acc0 : 1u);
+                        }
+                    } else {
+                        const uint64_t bd0 = desc_plain(b_base + (r * bin + cc) * sh, sk, 128);
+                        const uint64_t step_i = (uint64_t)((c.s * bin * sh) >> 4), step_j = (uint64_t)((c.s * sh) >> 4);
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+                            uint64_t bi = bd0 + (uint64_t)((2 * ks * sk) >> 4);
+                            uint32_t col = 0;
+#pragma unroll 1
+                            for (int i = 0; i < c.b; ++i, bi += step_i) {
+                                uint64_t bj = bi;
+#pragma unroll 1
+                                for (int j = 0; j < c.b; ++j, bj += step_j, col += sc.T)
+                                    tc_mma(tmem + col, ad0 + (uint64_t)(2 * ks), bj, idesc, ks == 0 ? acc0 : 1u);
                             }
                         }
                     }
                     tc_commit(a_empty(sa));
                     ++ait;
-                    if (kc == un.ke - 1 || tap == p.taps - 1) {
+                    if (++sa == cv.SA) {
+                        sa = 0;
+                        pa ^= 1;
+                    }
+                    const bool last_of_q = (kc == un.ke - 1) || (tap == p.taps - 1);
+                    if (last_of_q) {
                         tc_commit(b_empty(sb));
-                        ++bit;
+                        if (++sb == p.SB) {
+                            sb = 0;
+                            pb ^= 1;
+                        }
+                    }
+                    if (++cc == c.k) {
+                        cc = 0;
+                        ++r;
+                    }
+                    if (++tap == p.taps) {
+                        tap = 0;
+                        r = 0;
+                        ++q;
                     }
                 }
                 if (!ok)
@@ -584,34 +717,44 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
         }
     } else {
-        // ---------------- halo producers + epilogue (warps 2..5)
+        // ---------------- halo producers + epilogue (warps 2..9)
         const int et = threadIdx.x - 64;
         const int sub = warp & 3;           // tensor-memory subpartition of this warp
+        const int half = et >= 128 ? 1 : 0; // two warps per subpartition split the columns
         const int row = sub * 32 + lane;    // accumulator lane = output channel in the tile
         // One thread waits (bounded) and the group learns the outcome through a
         // named barrier, so that all 128 threads always take the same branch.
         auto group_wait = [&](uint32_t bar, uint32_t parity, int where) -> bool {
             if (et == 0)
                 *group_ok = mbar_wait(bar, parity, abort_flag, hdr, where) ? 1 : 0;
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, 256;" ::: "memory");
             const bool r = *group_ok != 0;
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, 256;" ::: "memory");
             return r;
         };
+        // output vectors: 8 bf16 channels (16 per 128-channel column) or 4 floats (32)
+        const int vpc = (c.to_y && c.dtype == SIGE_BF16) ? 16 : 32;
+        const int cpv = 128 / vpc;          // channels per vector
+        const int cg = et % vpc;            // this thread's vector within a column (fixed)
+        float * const stage_d = reinterpret_cast<float *>(smem + cv.b_base);
+        const int stage_cols = min(512, (int)((p.SB * cv.stage_b) / 512) & ~15);
         uint32_t bit = 0, uit = 0;
         bool ok = true;
+#pragma unroll 1
         for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
             const Unit un = decode_unit(p, sc, u);
             // the previous unit's epilogue may still be reading the origins
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            for (int slot = et; slot < sc.T; slot += 128) {
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+#pragma unroll 1
+            for (int slot = et; slot < sc.T; slot += kProd) {
                 const int g = un.tb * sc.T + slot;
                 int h0 = 0, w0 = 0;
                 if (g < G && (c.from_image || c.to_y))
                     tile_origin_a(c, g / c.N, h0, w0);
                 s_orig[slot] = make_int2(h0, w0);
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+#pragma unroll 1
             for (int kc = un.kb; kc < un.ke; ++kc) {
                 const int q = kc / p.taps, tap = kc - q * p.taps;
                 if (kc == un.kb || tap == 0) {
@@ -620,7 +763,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         ok = false;
                         break;
                     }
-                    fill_b(p, sc, un.tb, q, G, smem + p.b_off + sb * p.stage_b, et, s_orig);
+                    uint8_t *stage = smem + cv.b_base + sb * cv.stage_b;
+                    if (p.halo_tma) {
+                        // one TMA per (tile, halo row): [kc][ww][8 channels], zero outside the image
+                        if (et == 0) {
+                            const uint32_t bl = b_load(sb);
+                            mbar_expect_tx(bl, (uint32_t)(sc.T * c.bin) * c.bin * 128u);
+                            const uint32_t st = smem_u32(stage);
+#pragma unroll 1
+                            for (int slot = 0; slot < sc.T; ++slot) {
+                                const int g = un.tb * sc.T + slot;
+                                const int gg = g < G ? g : G - 1;   // past the list: any valid tile, unused
+                                const int2 o = s_orig[slot];
+                                const int x1 = c.from_image ? o.y * c.s - c.pad : 0;
+                                const int y0 = c.from_image ? o.x * c.s - c.pad : 0;
+                                const int n = c.from_image ? gg % c.N : gg;
+#pragma unroll 1
+                                for (int hh = 0; hh < c.bin; ++hh)
+                                    tma_load_5d(st + b_offset(c, sc.T, slot, hh, 0, 0), &tmx, bl, 0, x1, q * 8,
+                                                y0 + hh, n);
+                            }
+                        }
+                        if (!group_wait(b_load(sb), (bit / p.SB) & 1, 7)) {
+                            ok = false;
+                            break;
+                        }
+                        transform_b(c, sc.T, un.tb, q, G, stage, et, s_orig);
+                    } else {
+                        fill_b(c, sc.T, un.tb, q, G, stage, et, s_orig);
+                    }
                     fence_async_smem();
                     mbar_arrive(b_full(sb));
                     ++bit;
@@ -628,25 +799,75 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             if (!ok)
                 break;
+            // bias of this thread's output channels (fixed across the unit)
+            const int co0 = un.mt * 128 + cg * cpv;
+            float bias8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (c.bias && co0 < c.Cout) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    if (k < cpv)
+                        bias8[k] = __ldg(c.bias + co0 + k);
+            }
             if (!group_wait(acc_full, uit & 1, 6)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const int co = un.mt * 128 + row;
-            const float bias_c = (c.bias && co < c.Cout) ? __ldg(c.bias + co) : 0.0f;
-            const int ncols = unit_cols(p, sc);
+            const int ncols = unit_cols(p, sc.T);
             const uint32_t tbase = tmem + ((uint32_t)(sub * 32) << 16);
+            const bool write_ok = co0 < c.Cout;
             if (sc.S == 1) {
-                for (int c0 = 0; c0 < ncols; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tbase + c0, v);
-                    emit16(p, sc, s_orig, un.tb, c0, co, bias_c, v, G);
+                // accumulator -> shared staging (column-major, 128 floats per
+                // column) -> 16-byte vectors per pixel
+#pragma unroll 1
+                for (int c0 = 0; c0 < ncols; c0 += stage_cols) {
+                    const int cc_n = min(stage_cols, ncols - c0);
+#pragma unroll 1
+                    for (int k0 = 16 * half; k0 < cc_n; k0 += 32) {
+                        float v[16];
+                        tmem_ld16(tbase + c0 + k0, v);
+#pragma unroll
+                        for (int k = 0; k < 16; ++k)
+                            stage_d[(k0 + k) * 128 + row] = v[k];
+                    }
+                    asm volatile("bar.sync 1, 256;" ::: "memory");
+#pragma unroll 1
+                    for (int it0 = et; it0 < cc_n * vpc; it0 += 4 * kProd) {
+                        // four items per thread: addresses and residual loads first
+                        int64_t e[4];
+                        uint4 rr[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int it = it0 + k * kProd;
+                            e[k] = (it < cc_n * vpc && write_ok)
+                                       ? col_target(c, s_orig, sc.T, un.tb, G, c0 + it / vpc, co0) : -1;
+                            rr[k] = make_uint4(0, 0, 0, 0);
+                            if (e[k] >= 0 && c.residual && c.to_y)
+                                rr[k] = __ldg(reinterpret_cast<const uint4 *>(c.residual + e[k] * (c.dtype == SIGE_BF16 ? 2 : 4)));
+                        }
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            if (e[k] < 0)
+                                continue;
+                            const int col = (it0 + k * kProd) / vpc;
+                            float v[8];
+                            const float4 *src = reinterpret_cast<const float4 *>(stage_d + col * 128 + cg * cpv);
+                            const float4 lo = src[0];
+                            v[0] = lo.x; v[1] = lo.y; v[2] = lo.z; v[3] = lo.w;
+                            if (cpv == 8) {
+                                const float4 hi = src[1];
+                                v[4] = hi.x; v[5] = hi.y; v[6] = hi.z; v[7] = hi.w;
+                            }
+                            store_vec(c, e[k], v, bias8, rr[k]);
+                        }
+                    }
+                    asm volatile("bar.sync 1, 256;" ::: "memory");
                 }
             } else {
                 const int group = un.tb * p.MT + un.mt;
                 float *slab = p.partials + (size_t)(group * sc.S + un.split) * p.ncols * 128;
-                for (int c0 = 0; c0 < ncols; c0 += 16) {
+#pragma unroll 1
+                for (int c0 = 16 * half; c0 < ncols; c0 += 32) {
                     float v[16];
                     tmem_ld16(tbase + c0, v);
 #pragma unroll
@@ -654,7 +875,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         slab[(size_t)(c0 + k) * 128 + row] = v[k];
                 }
                 __threadfence();
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                asm volatile("bar.sync 1, 256;" ::: "memory");
                 if (et == 0) {
                     const unsigned prev = atomicAdd(p.counters + group, 1u);
                     const int last = prev == (unsigned)(sc.S - 1);
@@ -662,28 +883,51 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         p.counters[group] = 0;
                     *bcast = last;
                 }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                asm volatile("bar.sync 1, 256;" ::: "memory");
                 if (*bcast) {
                     __threadfence();
                     const float *base = p.partials + (size_t)group * sc.S * p.ncols * 128;
-                    for (int c0 = 0; c0 < ncols; c0 += 16) {
-                        float acc[16];
+#pragma unroll 1
+                    for (int it0 = et; it0 < ncols * vpc; it0 += 4 * kProd) {
+                        int64_t e[4];
+                        uint4 rr[4];
+                        float v[4][8];
 #pragma unroll
-                        for (int k = 0; k < 16; ++k)
-                            acc[k] = 0.0f;
-                        for (int s2 = 0; s2 < sc.S; ++s2) {   // fixed order: deterministic sum
-                            float t[16];
+                        for (int k = 0; k < 4; ++k) {
+                            const int it = it0 + k * kProd;
+                            e[k] = (it < ncols * vpc && write_ok)
+                                       ? col_target(c, s_orig, sc.T, un.tb, G, it / vpc, co0) : -1;
+                            rr[k] = make_uint4(0, 0, 0, 0);
+                            if (e[k] >= 0 && c.residual && c.to_y)
+                                rr[k] = __ldg(reinterpret_cast<const uint4 *>(c.residual + e[k] * (c.dtype == SIGE_BF16 ? 2 : 4)));
 #pragma unroll
-                            for (int k = 0; k < 16; ++k)
-                                t[k] = __ldcg(base + ((size_t)s2 * p.ncols + c0 + k) * 128 + row);
-#pragma unroll
-                            for (int k = 0; k < 16; ++k)
-                                acc[k] += t[k];
+                            for (int m = 0; m < 8; ++m)
+                                v[k][m] = 0.0f;
                         }
-                        emit16(p, sc, s_orig, un.tb, c0, co, bias_c, acc, G);
+#pragma unroll 1
+                        for (int s2 = 0; s2 < sc.S; ++s2) {   // fixed order: deterministic sum
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                if (e[k] < 0)
+                                    continue;
+                                const int col = (it0 + k * kProd) / vpc;
+                                const float4 *src = reinterpret_cast<const float4 *>(
+                                    base + ((size_t)s2 * p.ncols + col) * 128 + cg * cpv);
+                                const float4 lo = __ldcg(src);
+                                v[k][0] += lo.x; v[k][1] += lo.y; v[k][2] += lo.z; v[k][3] += lo.w;
+                                if (cpv == 8) {
+                                    const float4 hi = __ldcg(src + 1);
+                                    v[k][4] += hi.x; v[k][5] += hi.y; v[k][6] += hi.z; v[k][7] += hi.w;
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            if (e[k] >= 0)
+                                store_vec(c, e[k], v[k], bias8, rr[k]);
                     }
                 }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                asm volatile("bar.sync 1, 256;" ::: "memory");
             }
             tc_fence_before();
             mbar_arrive(acc_empty);
@@ -717,8 +961,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode()
 }
 
 struct TcPlan {
-    int mode, T_max, SA, SB, ncols;
-    uint32_t stage_b, b_off, bar_off, smem;
+    int mode, T_max, SB, ncols;
+    uint32_t per_slot;
 };
 
 static int pow2_at_least(int v)
@@ -730,39 +974,35 @@ static int pow2_at_least(int v)
 }
 
 // Shared memory / tensor memory plan for a layer; false if it does not fit.
+// The launch always takes the full 227 KB; T_max is the most tiles (slots) a
+// unit may hold with at least two weight stages beside SB halo stages.
 static bool plan_layer(const sige_conv_desc *cd, TcPlan &pl)
 {
     const int b = cd->block, s = cd->stride, k = cd->kernel;
     const int bin = (b - 1) * s + k;
-    const uint32_t per_slot = (uint32_t)bin * bin * 128;  // one tile, 64 channels
+    pl.per_slot = (uint32_t)bin * bin * 128;  // one tile, 64 channels
     pl.mode = (b == 8 && s == 1) ? 0 : 1;
-    const uint32_t bar_bytes = 1024 + 256 * 8;   // barriers and flags, then tile origins
-    for (int SA : {4, 2}) {
-        const uint32_t a_bytes = SA * kAStageBytes;
-        const int budget = kSmemLimit - 1024 /*alignment slack*/ - (int)a_bytes - (int)bar_bytes;
-        for (int SB : {2, 1}) {
-            int tmax;
-            if (pl.mode == 0) {
-                tmax = std::min(8, budget / (int)(SB * per_slot));      // 64 TMEM columns per tile
-            } else {
-                const int by_tmem = (512 / (b * b)) / 16 * 16;
-                const int by_smem = (budget / (int)(SB * per_slot)) / 16 * 16;
-                tmax = std::min({256, by_tmem, by_smem});
-                if (tmax < 16)
-                    tmax = 0;
-            }
-            if (tmax >= 1) {
-                pl.T_max = tmax;
-                pl.SA = SA;
-                pl.SB = SB;
-                pl.stage_b = (uint32_t)tmax * per_slot;
-                pl.b_off = a_bytes;
-                pl.bar_off = (pl.b_off + SB * pl.stage_b + 15) & ~15u;
-                pl.smem = std::max<uint32_t>(pl.bar_off + bar_bytes + 1024, kSmemFloor);
-                const int cols = pl.mode == 0 ? tmax * 64 : b * b * tmax;
-                pl.ncols = pow2_at_least(cols);
-                return pl.ncols <= 512 && pl.smem <= (uint32_t)kSmemLimit;
-            }
+    const int budget = kSmemLimit - 1024 /*alignment*/ - (int)kCtrlBytes - 2 * (int)kAStageBytes - 1024;
+    for (int SB : {2, 1}) {
+        int tmax;
+        if (pl.mode == 0) {
+            tmax = std::min(8, budget / (int)(SB * pl.per_slot));      // 64 TMEM columns per tile
+        } else {
+            const int by_tmem = (512 / (b * b)) / 16 * 16;
+            const int by_smem = (budget / (int)(SB * pl.per_slot)) / 16 * 16;
+            tmax = std::min({256, by_tmem, by_smem});
+            if (tmax < 16)
+                tmax = 0;
+        }
+        // the epilogue stages at least 16 accumulator columns (8 KB) in the
+        // halo stages of the smallest unit (1 tile, or 16 slots)
+        const uint32_t min_stage = SB * pl.per_slot * (pl.mode == 0 ? 1u : 16u);
+        if (tmax >= 1 && min_stage >= 16u * 512u) {
+            pl.T_max = tmax;
+            pl.SB = SB;
+            const int cols = pl.mode == 0 ? tmax * 64 : b * b * tmax;
+            pl.ncols = pow2_at_least(cols);
+            return pl.ncols <= 512;
         }
     }
     return false;
@@ -770,7 +1010,7 @@ static bool plan_layer(const sige_conv_desc *cd, TcPlan &pl)
 
 bool tc_supported(const sige_conv_desc *cd, int dtype)
 {
-    if (!cd || dtype != SIGE_BF16 || cd->c_in % 64 || cd->c_in < 64 || cd->c_out < 1)
+    if (!cd || dtype != SIGE_BF16 || cd->c_in % 64 || cd->c_in < 64 || cd->c_out < 8 || cd->c_out % 8)
         return false;
     if ((long long)cd->kernel * cd->kernel * cd->c_in >= (1ll << 31))
         return false;
@@ -811,7 +1051,34 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
     if (r != CUDA_SUCCESS)
         return SIGE_ERR_CUDA;
 
+    // ROW mode: one TMA per (tile, halo row) from a 5-d view of the source
+    // [n][y][x][c/8][8] (image) or [g][hh][ww][c/8][8] (stacked blocks),
+    // box (8 channels, b_in pixels, 8 channel groups), zero outside.
+    CUtensorMap xmap = map;
+    int halo_tma = 0;
+    if (pl.mode == 0) {
+        const cuuint64_t C = (cuuint64_t)cp.Cin;
+        cuuint64_t xd[5], xs[4];
+        if (cp.from_image) {
+            xd[0] = 8; xd[1] = (cuuint64_t)cp.W; xd[2] = C / 8; xd[3] = (cuuint64_t)cp.H; xd[4] = (cuuint64_t)cp.N;
+            xs[0] = C * 2; xs[1] = 16; xs[2] = (cuuint64_t)cp.W * C * 2; xs[3] = (cuuint64_t)cp.H * cp.W * C * 2;
+        } else {
+            const cuuint64_t bin = (cuuint64_t)cp.bin;
+            xd[0] = 8; xd[1] = bin; xd[2] = C / 8; xd[3] = bin; xd[4] = (cuuint64_t)std::max(1, cp.cap) * cp.N;
+            xs[0] = C * 2; xs[1] = 16; xs[2] = bin * C * 2; xs[3] = bin * bin * C * 2;
+        }
+        cuuint32_t xbox[5] = {8, (cuuint32_t)cp.bin, 8, 1, 1};
+        cuuint32_t xes[5] = {1, 1, 1, 1, 1};
+        if (encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<uint8_t *>(cp.src), xd, xs, xbox, xes,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+            halo_tma = 1;
+        else
+            xmap = map;
+    }
+
     TcArgs p{};
+    p.halo_tma = halo_tma;
     p.src = cp.src; p.idx = cp.idx; p.count = cp.count; p.gsc = cp.gsc; p.gsh = cp.gsh; p.bias = cp.bias;
     p.residual = cp.residual; p.y = cp.y; p.out_blocks = cp.out_blocks; p.ws = cp.ws;
     p.N = cp.N; p.H = cp.H; p.W = cp.W; p.Cin = cp.Cin; p.Cout = cp.Cout; p.dtype = cp.dtype;
@@ -823,11 +1090,9 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
     p.kci = cp.Cin / 64;
     p.MT = (cp.Cout + 127) / 128;
     p.T_max = pl.T_max;
-    p.SA = pl.SA;
     p.SB = pl.SB;
-    p.b_off = pl.b_off;
-    p.bar_off = pl.bar_off;
-    p.stage_b = pl.stage_b;
+    p.per_slot = pl.per_slot;
+    p.smem_bytes = kSmemLimit - 1024;   // usable after aligning the base to 1024
     p.ncols = pl.ncols;
     p.num_sms = device_sm_count();
     uint8_t *ws = cp.ws + kWsHeader;
@@ -842,7 +1107,7 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
             return SIGE_ERR_CUDA;
         smem_set[dev] = 1;
     }
-    k_conv_tc<<<p.num_sms, kTcThreads, pl.smem, stream>>>(p, map);
+    k_conv_tc<<<p.num_sms, kTcThreads, kSmemLimit, stream>>>(p, map, xmap);
     count_launch();
     return launch_check();
 }

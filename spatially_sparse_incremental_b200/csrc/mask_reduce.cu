@@ -54,7 +54,6 @@ struct MaskParams {
 
 constexpr int kMaskThreads = 256;
 constexpr int kMaskUnroll = 8;
-constexpr int kFlagSmem = 16384;
 
 __device__ __forceinline__ float elem_as_float(uint32_t word, int k, int dtype)
 {
@@ -114,73 +113,92 @@ __device__ __forceinline__ float scalar_elem(const uint8_t *base, int64_t i, int
     return reinterpret_cast<const float *>(base)[i];
 }
 
-__device__ __forceinline__ bool phase1(const MaskParams &p, const ScaleParams *sc)
+// Exact test of the vectors whose bytes differ (rare: only edited pixels), kept
+// out of line so that the streaming loop stays a few dozen instructions.
+// The vectors are read again here (a few percent of them at most) so that the
+// streaming loop keeps its loads in registers.
+__device__ __noinline__ void mark_vectors(const MaskParams &p, const ScaleParams *sc, int64_t v0, int64_t stride,
+                                          uint32_t neq)
+{
+    const int64_t HW = (int64_t)p.H * p.W;
+    while (neq) {
+        const int u = __ffs(neq) - 1;
+        neq &= neq - 1;
+        const int64_t v = v0 + u * stride;
+        uint32_t bits = diff_bits16(ld_nc16(p.a + v * 16), ld_nc16(p.b + v * 16), p.dtype, p.thr);
+        if (!bits)
+            continue;
+        if (p.mode == 0) {
+            const int64_t pix = v / p.vpp;
+            mark(sc, p.n_scales, p.flags, (int)((pix % HW) / p.W), (int)(pix % p.W));
+        } else {
+            const int64_t e0 = v * p.epv;
+            const int y = (int)((e0 / p.W) % p.H);
+            const int x0 = (int)(e0 % p.W);
+            while (bits) {
+                const int k = __ffs(bits) - 1;
+                bits &= bits - 1;
+                mark(sc, p.n_scales, p.flags, y, x0 + k);
+            }
+        }
+    }
+}
+
+__device__ __noinline__ bool scalar_pass(const MaskParams &p, const ScaleParams *sc)
 {
     bool wrote = false;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t HW = (int64_t)p.H * p.W;
-    const int n_scales = p.n_scales, mode = p.mode, dtype = p.dtype, W = p.W, H = p.H, C = p.C;
-    const int vpp = p.vpp, epv = p.epv, layout = p.layout;
-    const float thr = p.thr;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.nwork; i += stride) {
+        const float d = fabsf(scalar_elem(p.b, i, p.dtype) - scalar_elem(p.a, i, p.dtype));
+        if (d > p.thr) {
+            wrote = true;
+            int y, x;
+            if (p.layout == SIGE_NHWC) {
+                const int64_t pix = i / p.C;
+                y = (int)((pix % HW) / p.W);
+                x = (int)(pix % p.W);
+            } else {
+                y = (int)((i / p.W) % p.H);
+                x = (int)(i % p.W);
+            }
+            mark(sc, p.n_scales, p.flags, y, x);
+        }
+    }
+    return wrote;
+}
+
+// Stream both inputs once.  Bitwise-equal 16-byte vectors cannot differ by
+// more than a non-negative threshold, so the hot loop only compares raw bits;
+// vectors whose bytes differ get the exact float32 test in mark_vectors.
+__device__ __forceinline__ bool phase1(const MaskParams &p, const ScaleParams *sc)
+{
+    if (p.mode == 2)
+        return scalar_pass(p, sc);
+    bool wrote = false;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t nwork = p.nwork;
     const uint8_t *a = p.a, *b = p.b;
-    uint8_t *flags = p.flags;
-    for (int64_t v0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v0 < nwork;
-         v0 += stride * kMaskUnroll) {
-        if (mode == 2) {
-#pragma unroll
-            for (int u = 0; u < kMaskUnroll; ++u) {
-                int64_t i = v0 + u * stride;
-                if (i >= nwork)
-                    break;
-                float d = fabsf(scalar_elem(b, i, dtype) - scalar_elem(a, i, dtype));
-                if (d > thr) {
-                    wrote = true;
-                    int y, x;
-                    if (layout == SIGE_NHWC) {
-                        int64_t pix = i / C;
-                        y = (int)((pix % HW) / W);
-                        x = (int)(pix % W);
-                    } else {
-                        y = (int)((i / W) % H);
-                        x = (int)(i % W);
-                    }
-                    mark(sc, n_scales, flags, y, x);
-                }
-            }
-            continue;
-        }
+    for (int64_t v0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v0 < nwork; v0 += stride * kMaskUnroll) {
         uint4 av[kMaskUnroll], bv[kMaskUnroll];
 #pragma unroll
         for (int u = 0; u < kMaskUnroll; ++u) {
-            int64_t v = v0 + u * stride;
+            const int64_t v = v0 + u * stride;
+            av[u] = make_uint4(0, 0, 0, 0);
+            bv[u] = av[u];
             if (v < nwork) {
                 av[u] = ld_stream16(a + v * 16);
                 bv[u] = ld_stream16(b + v * 16);
             }
         }
+        uint32_t neq = 0;
 #pragma unroll
-        for (int u = 0; u < kMaskUnroll; ++u) {
-            int64_t v = v0 + u * stride;
-            if (v >= nwork)
-                break;
-            uint32_t bits = diff_bits16(av[u], bv[u], dtype, thr);
-            if (!bits)
-                continue;
+        for (int u = 0; u < kMaskUnroll; ++u)
+            neq |= (uint32_t)(((av[u].x ^ bv[u].x) | (av[u].y ^ bv[u].y) | (av[u].z ^ bv[u].z) |
+                               (av[u].w ^ bv[u].w)) != 0) << u;
+        if (neq) {
             wrote = true;
-            if (mode == 0) {
-                int64_t pix = v / vpp;
-                mark(sc, n_scales, flags, (int)((pix % HW) / W), (int)(pix % W));
-            } else {
-                int64_t e0 = v * epv;
-                int y = (int)((e0 / W) % H);
-                int x0 = (int)(e0 % W);
-                while (bits) {
-                    int k = __ffs(bits) - 1;
-                    bits &= bits - 1;
-                    mark(sc, n_scales, flags, y, x0 + k);
-                }
-            }
+            mark_vectors(p, sc, v0, stride, neq);
         }
     }
     return wrote;
@@ -221,68 +239,110 @@ __device__ __forceinline__ int block_scan(int v, int *warp_sums, int *total)
     return off;
 }
 
-constexpr int kTilesPerThread = 4;
+// Phase 2 works on bit rows: word (i, w) holds the flags of tiles
+// (i, 32w .. 32w+31).  Dilation by D tiles is then an OR of the D rows above and
+// below followed by shifts of +-1..D bits (with carries from the neighbouring
+// words), and the row-major compaction is a prefix sum of popcounts.
+constexpr int kMaxWords = 4096;          // bit words per scale held in shared memory (131072 tiles)
 
-__device__ __forceinline__ void phase2(const MaskParams &p, const ScaleParams *sc)
+__device__ __forceinline__ uint32_t row_word(const uint32_t *bits, int wpr, int th, int i, int w, int D)
 {
-    __shared__ uint8_t sflag[kFlagSmem];
+    uint32_t v = 0;
+    const int i0 = max(0, i - D), i1 = min(th - 1, i + D);
+#pragma unroll 1
+    for (int ii = i0; ii <= i1; ++ii)
+        v |= bits[ii * wpr + w];
+    return v;
+}
+
+__device__ __noinline__ void phase2(const MaskParams &p, const ScaleParams *sc)
+{
+    __shared__ __align__(16) uint32_t sbits[kMaxWords];    // raw tile bits
+    __shared__ __align__(16) uint32_t sdil[kMaxWords];     // dilated tile bits
     __shared__ int warp_sums[33];
-    const int n_scales = p.n_scales, dilate = p.dilate;
+    const int n_scales = p.n_scales, D = p.dilate;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+#pragma unroll 1
     for (int s = 0; s < n_scales; ++s) {
         const ScaleParams q = sc[s];
-        const int nt = q.th * q.tw;
+        const int wpr = (q.tw + 31) >> 5;
+        const int nw = q.th * wpr;
         const uint8_t *g = p.flags + q.flag_off;
-        const bool in_smem = nt <= kFlagSmem;
-        if (in_smem) {
-            // flag_off is 16-byte aligned and the flag area is padded to 16
-            // bytes, so these 16-byte reads stay inside it
-            for (int t = threadIdx.x * 16; t < nt; t += blockDim.x * 16) {
-                const uint4 w = __ldcg(reinterpret_cast<const uint4 *>(g + t));
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    if (t + k < nt)
-                        sflag[t + k] = (uint8_t)((ws[k >> 2] >> (8 * (k & 3))) & 0xFF);
+        int base = 0;
+        if (nw <= kMaxWords && D < 32) {
+            // flag bytes -> bit words (one ballot per word)
+#pragma unroll 1
+            for (int wi = warp; wi < nw; wi += nwarps) {
+                const int i = wi / wpr, j = (wi - i * wpr) * 32 + lane;
+                const int f = j < q.tw ? __ldcg(g + i * q.tw + j) : 0;
+                const uint32_t word = __ballot_sync(0xFFFFFFFFu, f != 0);
+                if (lane == 0)
+                    sbits[wi] = word;
             }
             __syncthreads();
-        }
-        int base = 0;
-        const int chunk = blockDim.x * kTilesPerThread;
-        for (int t0 = 0; t0 < nt; t0 += chunk) {
-            const int tb = t0 + threadIdx.x * kTilesPerThread;
-            uint32_t bits = 0;
-#pragma unroll
-            for (int k = 0; k < kTilesPerThread; ++k) {
-                const int t = tb + k;
-                if (t >= nt)
-                    break;
-                const int i = t / q.tw, j = t - i * q.tw;
-                const int i0 = max(0, i - dilate), i1 = min(q.th - 1, i + dilate);
-                const int j0 = max(0, j - dilate), j1 = min(q.tw - 1, j + dilate);
-                int act = 0;
-                for (int ii = i0; ii <= i1 && !act; ++ii)
-                    for (int jj = j0; jj <= j1; ++jj) {
-                        const uint8_t f = in_smem ? sflag[ii * q.tw + jj] : __ldcg(g + ii * q.tw + jj);
-                        if (f) {
-                            act = 1;
-                            break;
-                        }
-                    }
-                bits |= (uint32_t)act << k;
+            // dilation: vertical OR, then horizontal shifts with carries
+            const uint32_t last_mask = (q.tw & 31) ? ((1u << (q.tw & 31)) - 1u) : 0xFFFFFFFFu;
+#pragma unroll 1
+            for (int wi = threadIdx.x; wi < nw; wi += blockDim.x) {
+                const int i = wi / wpr, w = wi - i * wpr;
+                const uint32_t v = row_word(sbits, wpr, q.th, i, w, D);
+                const uint32_t prev = w > 0 ? row_word(sbits, wpr, q.th, i, w - 1, D) : 0u;
+                const uint32_t next = w + 1 < wpr ? row_word(sbits, wpr, q.th, i, w + 1, D) : 0u;
+                uint32_t h = v;
+#pragma unroll 1
+                for (int d = 1; d <= D; ++d)
+                    h |= (v << d) | (v >> d) | (prev >> (32 - d)) | (next << (32 - d));
+                sdil[wi] = (w == wpr - 1) ? (h & last_mask) : h;
             }
-            int chunk_total;
-            int pos = base + block_scan(__popc(bits), warp_sums, &chunk_total);
-            while (bits) {
-                const int k = __ffs(bits) - 1;
-                bits &= bits - 1;
-                if (pos < q.capacity) {
-                    const int t = tb + k;
+            __syncthreads();
+            // compaction: each thread takes a contiguous run of words
+            const int per = (nw + blockDim.x - 1) / blockDim.x;
+            const int w0 = min(nw, (int)threadIdx.x * per), w1 = min(nw, w0 + per);
+            int cnt = 0;
+#pragma unroll 1
+            for (int wi = w0; wi < w1; ++wi)
+                cnt += __popc(sdil[wi]);
+            int total;
+            int pos = block_scan(cnt, warp_sums, &total);
+#pragma unroll 1
+            for (int wi = w0; wi < w1; ++wi) {
+                uint32_t m = sdil[wi];
+                const int i = wi / wpr, jb = (wi - i * wpr) * 32;
+                while (m) {
+                    const int k = __ffs(m) - 1;
+                    m &= m - 1;
+                    if (pos < q.capacity)
+                        reinterpret_cast<int2 *>(p.idx)[q.idx_off + pos] = make_int2(i * q.block, (jb + k) * q.block);
+                    ++pos;
+                }
+            }
+            base = total;
+        } else {
+            // very large grids: byte flags straight from global memory
+            const int nt = q.th * q.tw;
+            const int chunk = blockDim.x;
+#pragma unroll 1
+            for (int t0 = 0; t0 < nt; t0 += chunk) {
+                const int t = t0 + threadIdx.x;
+                int act = 0;
+                if (t < nt) {
+                    const int i = t / q.tw, j = t - i * q.tw;
+                    const int i0 = max(0, i - D), i1 = min(q.th - 1, i + D);
+                    const int j0 = max(0, j - D), j1 = min(q.tw - 1, j + D);
+#pragma unroll 1
+                    for (int ii = i0; ii <= i1 && !act; ++ii)
+#pragma unroll 1
+                        for (int jj = j0; jj <= j1 && !act; ++jj)
+                            act = __ldcg(g + ii * q.tw + jj) != 0;
+                }
+                int chunk_total;
+                const int pos = base + block_scan(act, warp_sums, &chunk_total);
+                if (act && pos < q.capacity) {
                     const int i = t / q.tw, j = t - i * q.tw;
                     reinterpret_cast<int2 *>(p.idx)[q.idx_off + pos] = make_int2(i * q.block, j * q.block);
                 }
-                ++pos;
+                base += chunk_total;
             }
-            base += chunk_total;
         }
         if (threadIdx.x == 0) {
             p.counts[s] = base;
@@ -293,6 +353,7 @@ __device__ __forceinline__ void phase2(const MaskParams &p, const ScaleParams *s
     }
     // leave the workspace zero-filled for the next call
     const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll 1
     for (int k = threadIdx.x; k < p.flag_bytes / 16; k += blockDim.x)
         reinterpret_cast<uint4 *>(p.flags)[k] = z;
     if (threadIdx.x == 0)

@@ -128,3 +128,20 @@ def test_workspace_reuse_across_calls(orc):
         got, _, ws = _gpu_lists(o, e, 0.0, _full_caps(inputs.CFG2_SCALES), 1, sige.NCHW, workspace=ws)
         for s in range(4):
             assert np.array_equal(got[s], ref[s])
+
+
+def test_wide_grids_multiword_rows(orc):
+    # tile rows wider than 32 tiles span several bit words: dilation must
+    # carry across word boundaries (and stay inside the last, partial word)
+    rng = np.random.default_rng(11)
+    for (H, W, b, D) in [(64, 300, 1, 1), (40, 520, 2, 2), (16, 1000, 1, 5), (48, 96, 1, 1), (8, 2048, 1, 33)]:
+        a = torch.from_numpy(rng.normal(size=(1, H, W, 8)).astype(np.float32))
+        e = a.clone()
+        m = rng.random((H, W)) < 0.01
+        m[:, 31] = rng.random(H) < 0.3        # flags right at word boundaries
+        m[:, 32] |= rng.random(H) < 0.3
+        e[0, torch.from_numpy(m)] += 1.0
+        sc = [(H, W, b)]
+        ref = orc.reduce_mask(a, e, 1e-3, sc, D)
+        got, cnt, _ = _gpu_lists(a, e, 1e-3, _full_caps(sc), D)
+        assert cnt[0] == len(ref[0]) and np.array_equal(got[0], ref[0]), (H, W, b, D)

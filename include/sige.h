@@ -117,6 +117,30 @@ int sige_reduce_mask(const void *a_orig, const void *a_edit, const sige_tensor_d
                      const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
                      void *workspace, size_t workspace_bytes, sige_stream_t stream);
 
+/* (1b) sige_reduce_mask without a caller workspace.  There is no counterpart
+ * in the paper: this is a convenience for callers that cannot allocate device
+ * memory for a workspace (a process that reserves all device memory up front,
+ * a plugin interface without an allocator, a binding that only forwards the
+ * tensors it was given).  The scratch lives in a 64 KB array inside the
+ * library, one per GPU, held until the process exits:
+ *   - requests needing more than that (256-byte header + one flag byte per
+ *     tile, 16-byte padded per scale) return SIGE_ERR_WORKSPACE, nothing
+ *     enqueued;
+ *   - the first call on a device looks the array's address up (once, with
+ *     that device current), so make that first call before any stream
+ *     capture;
+ *   - each call clears the part of the array it uses with an asynchronous
+ *     memset on `stream`, then runs the same kernel as sige_reduce_mask;
+ *   - all calls share the array: calls that overlap on the GPU (other
+ *     streams, other threads) race and must be serialised by the caller;
+ *   - a list longer than its capacity shows as counts[s] > capacity (there
+ *     is no workspace header to read with sige_get_error).
+ * Other arguments as in sige_reduce_mask. */
+int sige_reduce_mask_static(const void *a_orig, const void *a_edit, const sige_tensor_desc *in,
+                            float threshold, int32_t dilate, int32_t n_scales,
+                            const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
+                            sige_stream_t stream);
+
 /* (2) Gather the active blocks, with halo, from the edited activation and
  * stack them on the batch axis (SIGE project page, "Overview").
  *   blocks[t][n][hh][ww][c] = T(x[n][h0*s - p + hh][w0*s - p + ww][c]),

@@ -51,6 +51,7 @@ _TD, _CD, _SD = ctypes.POINTER(TensorDesc), ctypes.POINTER(ConvDesc), ctypes.POI
 SIGNATURES = {
     "sige_reduce_mask_workspace_bytes": (_sz, [_TD, _i32, _SD]),
     "sige_reduce_mask": (_i32, [_vp, _vp, _TD, _f32, _i32, _i32, _SD, _vp, _vp, _vp, _sz, _vp]),
+    "sige_reduce_mask_static": (_i32, [_vp, _vp, _TD, _f32, _i32, _i32, _SD, _vp, _vp, _vp]),
     "sige_gather": (_i32, [_vp, _TD, _CD, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _vp]),
     "sige_sparse_conv": (_i32, [_vp, _CD, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _sz, _vp]),
     "sige_scatter": (_i32, [_vp, _CD, _vp, _vp, _i32, _vp, _vp, _vp, _TD, _vp]),
@@ -157,6 +158,24 @@ def sige_reduce_mask(a_orig, a_edit, threshold, scales, dilate=1, layout=NHWC, i
                                 workspace.numel(), _stream(stream))
     _check(st, "sige_reduce_mask")
     return idx, counts, workspace
+
+
+def sige_reduce_mask_static(a_orig, a_edit, threshold, scales, dilate=1, layout=NHWC, idx=None, counts=None,
+                            stream=None):
+    """sige_reduce_mask for callers that cannot allocate a workspace: the
+    library's built-in 64 KB scratch is used instead (calls on one device must
+    not overlap).  Returns (idx, counts)."""
+    desc = tensor_desc(a_orig, layout)
+    arr = (ScaleDesc * len(scales))(*[ScaleDesc(*s) for s in scales])
+    dev = a_orig.device
+    if idx is None:
+        idx = torch.empty((max(1, sum(s[3] for s in scales)), 2), dtype=torch.int32, device=dev)
+    if counts is None:
+        counts = torch.empty(len(scales), dtype=torch.int32, device=dev)
+    st = lib().sige_reduce_mask_static(_ptr(a_orig), _ptr(a_edit), ctypes.byref(desc), float(threshold),
+                                       int(dilate), len(scales), arr, _ptr(idx), _ptr(counts), _stream(stream))
+    _check(st, "sige_reduce_mask_static")
+    return idx, counts
 
 
 def sige_gather(x, cd: ConvDesc, idx, count, capacity, gn_scale=None, gn_shift=None, silu=False,

@@ -19,6 +19,7 @@
 //     the flags and the arrival counter so the workspace is ready for the next
 //     call.
 #include <algorithm>
+#include <mutex>
 
 #include "sige_internal.cuh"
 
@@ -506,4 +507,67 @@ extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const si
     k_mask_reduce<<<grid, kMaskThreads, 0, (cudaStream_t)stream>>>(p);
     count_launch();
     return launch_check();
+}
+
+// ------------------------------------------------------------------ variant without a workspace
+//
+// The same reduction for callers that cannot hand the library a device
+// workspace: processes that reserve all device memory up front and allow no
+// further allocation, plugin interfaces that expose no allocator, or bindings
+// that only forward the tensors they were given.  Its scratch (the header and
+// the per-scale tile flags) lives in this file-scope array instead.  Every
+// GPU that loads the library holds the array until the process exits, and
+// every call on a device shares it.
+
+namespace sige {
+
+constexpr size_t kStaticScratchBytes = 64 * 1024;
+static __device__ __align__(256) uint8_t g_mask_scratch[kStaticScratchBytes];
+
+// The array's name is only a host-side stand-in; its device address is looked
+// up once per device, with that device current.
+static void *static_scratch_address(int &status)
+{
+    static std::mutex mu;
+    static void *addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        status = SIGE_ERR_CUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_mask_scratch) != cudaSuccess || !p) {
+            status = SIGE_ERR_CUDA;
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    status = SIGE_OK;
+    return addr[dev];
+}
+
+} // namespace sige
+
+extern "C" int sige_reduce_mask_static(const void *a_orig, const void *a_edit, const sige_tensor_desc *in,
+                                       float threshold, int32_t dilate, int32_t n_scales,
+                                       const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
+                                       sige_stream_t stream)
+{
+    if (!in || !scales_ok(in, n_scales, scales))
+        return SIGE_ERR_INVALID_ARG;
+    const size_t need = kWsHeader + flag_bytes_of(n_scales, scales);
+    if (need > kStaticScratchBytes)
+        return SIGE_ERR_WORKSPACE;   // more tiles than the built-in scratch holds
+    int st = SIGE_OK;
+    void *scratch = static_scratch_address(st);
+    if (!scratch)
+        return st;
+    // the kernel needs its flags and arrival counter at zero on entry; an
+    // earlier call that failed part-way could have left them otherwise
+    if (cudaMemsetAsync(scratch, 0, need, (cudaStream_t)stream) != cudaSuccess)
+        return SIGE_ERR_CUDA;
+    return sige_reduce_mask(a_orig, a_edit, in, threshold, dilate, n_scales, scales, idx, counts, scratch, need,
+                            stream);
 }

@@ -130,6 +130,7 @@ int launch_conv_simt(ConvParams p, cudaStream_t stream)
     const int ncog = (p.Cout + p.cob - 1) / p.cob;
     const int64_t max_units = (int64_t)(p.dense ? p.tiles_total : p.cap) * p.N * ncog;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(max_units, (int64_t)device_sm_count() * 8));
+    prefer_max_shared(k_conv_simt);
     k_conv_simt<<<grid, kSimtThreads, smem, stream>>>(p);
     count_launch();
     return launch_check();

@@ -244,7 +244,7 @@ __device__ __forceinline__ Sched make_sched(const TcArgs &p, int G)
     const int KC = p.taps * p.kci;
     // split K only where each split keeps a long K loop: below that the extra
     // round trip of the partial sums costs more than the shorter loop saves
-    s.S = max(1, min(p.num_sms / max(1, s.TB * p.MT), min(KC / 12, kMaxSplit)));
+    s.S = max(1, min(p.num_sms / max(1, s.TB * p.MT), min(KC / 8, kMaxSplit)));
     s.units = s.TB * p.MT * s.S;
     return s;
 }
@@ -614,16 +614,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer
+        // One thread issues every MMA, so this loop is kept to the bare chain:
+        // per k-chunk one barrier test, the MMAs and a commit.  The B
+        // descriptor is built once per halo stage and moves by constant
+        // offsets from tap to tap; the A descriptor moves by one stage.
         if (lane == 0) {
             int sa = 0, sb = 0;
             uint32_t pa = 0, pb = 0, uit = 0, ait = 0;
             bool ok = true;
-            const int bin = c.bin;
-            const int n_mma = p.mode == 0 ? 64 : sc.T;
+            const int bin = c.bin, k = c.k, taps = p.taps, nT = sc.T, bb = c.b;
+            const int n_mma = p.mode == 0 ? 64 : nT;
             const uint32_t idesc = idesc_bf16(n_mma);
-            const uint32_t sk = p.mode == 0 ? (uint32_t)bin * 16 : (uint32_t)sc.T * 16;   // LBO
+            const uint32_t sk = p.mode == 0 ? (uint32_t)bin * 16 : (uint32_t)nT * 16;   // LBO
             const uint32_t sh = 8 * sk;      // ROW: halo row stride; POS: halo pixel stride
-            const uint64_t tile_step = (uint64_t)((bin * sh) >> 4);
+            // descriptor start-address steps (address >> 4)
+            const uint64_t d_tile = (uint64_t)((bin * sh) >> 4);      // ROW: next tile
+            const uint64_t d_ks = (uint64_t)((2 * sk) >> 4);          // next 16 channels
+            const uint64_t d_col = p.mode == 0 ? 1u : (uint64_t)(sh >> 4);                 // tap column + 1
+            const uint64_t d_row = p.mode == 0 ? (uint64_t)(sh >> 4) : (uint64_t)((bin * sh) >> 4);  // tap row + 1
+            const uint64_t d_i = (uint64_t)((c.s * bin * sh) >> 4), d_j = (uint64_t)((c.s * sh) >> 4);  // POS
+            const uint64_t a_desc0 = desc_sw128(sbase + cv.a_base);
+            uint64_t a_cur = a_desc0;
 #pragma unroll 1
             for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, sc, u);
@@ -632,76 +643,74 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                int q = un.kb / p.taps, tap = un.kb - q * p.taps;
-                int r = tap / c.k, cc = tap - r * c.k;
+                int tap = un.kb % taps;
+                uint32_t acc0 = 0;
 #pragma unroll 1
-                for (int kc = un.kb; kc < un.ke; ++kc) {
-                    if (kc == un.kb || tap == 0) {
-                        if (!mbar_wait(b_full(sb), pb, abort_flag, hdr, 3)) {
-                            ok = false;
-                            break;
-                        }
-                    }
-                    if (!mbar_wait(a_full(sa), pa, abort_flag, hdr, 4)) {
+                for (int kc = un.kb; kc < un.ke && ok;) {
+                    // one halo stage: taps [tap, tap_end) of one 64-channel chunk
+                    if (!mbar_wait(b_full(sb), pb, abort_flag, hdr, 3)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    const uint32_t a_base = sbase + cv.a_base + sa * kAStageBytes;
-                    const uint32_t b_base = sbase + cv.b_base + sb * cv.stage_b;
-                    const uint32_t acc0 = (kc == un.kb) ? 0u : 1u;
-                    // descriptors differ only in their start address field
-                    // (address >> 4, low bits), so offsets are added directly
-                    const uint64_t ad0 = desc_sw128(a_base);
-                    if (p.mode == 0) {
-                        const uint64_t bd0 = desc_plain(b_base + r * sh + cc * 16, sk, sh);
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks) {
-                            const uint64_t bk = bd0 + (uint64_t)((2 * ks * sk) >> 4);
+                    const int tap_end = min(taps, tap + (un.ke - kc));
+                    const uint64_t b_stage = p.mode == 0
+                        ? desc_plain(sbase + cv.b_base + sb * cv.stage_b, sk, sh)
+                        : desc_plain(sbase + cv.b_base + sb * cv.stage_b, sk, 128);
+                    int r = tap / k, cc = tap - r * k;
+                    uint64_t b_tap = b_stage + (uint64_t)r * d_row + (uint64_t)cc * d_col;
 #pragma unroll 1
-                            for (int t = 0; t < sc.T; ++t)
-                                tc_mma(tmem + t * 64, ad0 + (uint64_t)(2 * ks), bk + t * tile_step, idesc,
-                                       ks == 0 ? acc0 : 1u);
+                    for (; tap < tap_end; ++tap, ++kc) {
+                        if (!mbar_wait(a_full(sa), pa, abort_flag, hdr, 4)) {
+                            ok = false;
+                            break;
                         }
-                    } else {
-                        const uint64_t bd0 = desc_plain(b_base + (r * bin + cc) * sh, sk, 128);
-                        const uint64_t step_i = (uint64_t)((c.s * bin * sh) >> 4), step_j = (uint64_t)((c.s * sh) >> 4);
+                        tc_fence_after();
+                        if (p.mode == 0) {
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks) {
-                            uint64_t bi = bd0 + (uint64_t)((2 * ks * sk) >> 4);
-                            uint32_t col = 0;
+                            for (int ks = 0; ks < 4; ++ks) {
+                                uint64_t bt = b_tap + ks * d_ks;
 #pragma unroll 1
-                            for (int i = 0; i < c.b; ++i, bi += step_i) {
-                                uint64_t bj = bi;
+                                for (int t = 0; t < nT; ++t, bt += d_tile)
+                                    tc_mma(tmem + t * 64, a_cur + 2 * ks, bt, idesc, ks ? 1u : acc0);
+                            }
+                        } else {
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks) {
+                                uint64_t bi = b_tap + ks * d_ks;
+                                uint32_t col = 0;
 #pragma unroll 1
-                                for (int j = 0; j < c.b; ++j, bj += step_j, col += sc.T)
-                                    tc_mma(tmem + col, ad0 + (uint64_t)(2 * ks), bj, idesc, ks == 0 ? acc0 : 1u);
+                                for (int i = 0; i < bb; ++i, bi += d_i) {
+                                    uint64_t bj = bi;
+#pragma unroll 1
+                                    for (int j = 0; j < bb; ++j, bj += d_j, col += nT)
+                                        tc_mma(tmem + col, a_cur + 2 * ks, bj, idesc, ks ? 1u : acc0);
+                                }
                             }
                         }
-                    }
-                    tc_commit(a_empty(sa));
-                    ++ait;
-                    if (++sa == cv.SA) {
-                        sa = 0;
-                        pa ^= 1;
-                    }
-                    const bool last_of_q = (kc == un.ke - 1) || (tap == p.taps - 1);
-                    if (last_of_q) {
-                        tc_commit(b_empty(sb));
-                        if (++sb == p.SB) {
-                            sb = 0;
-                            pb ^= 1;
+                        acc0 = 1;
+                        tc_commit(a_empty(sa));
+                        ++ait;
+                        if (++sa == cv.SA) {
+                            sa = 0;
+                            pa ^= 1;
+                            a_cur = a_desc0;
+                        } else {
+                            a_cur += kAStageBytes >> 4;
                         }
+                        if (++cc == k) {
+                            cc = 0;
+                            b_tap += d_row - (uint64_t)k * d_col;
+                        }
+                        b_tap += d_col;
                     }
-                    if (++cc == c.k) {
-                        cc = 0;
-                        ++r;
+                    if (!ok)
+                        break;
+                    tc_commit(b_empty(sb));
+                    if (++sb == p.SB) {
+                        sb = 0;
+                        pb ^= 1;
                     }
-                    if (++tap == p.taps) {
-                        tap = 0;
-                        r = 0;
-                        ++q;
-                    }
+                    tap = 0;
                 }
                 if (!ok)
                     break;

@@ -202,6 +202,7 @@ extern "C" int sige_gather(const void *x, const sige_tensor_desc *xd, const sige
     p.blocks = static_cast<uint8_t *>(blocks);
     p.vpp = xd->c * esz / 16;
     const int64_t work = (int64_t)capacity * p.N * p.bin * p.bin * p.vpp;
+    prefer_max_shared(k_gather);
     k_gather<<<grid_for(work, 256), 256, 0, (cudaStream_t)stream>>>(p);
     count_launch();
     return launch_check();
@@ -231,6 +232,7 @@ extern "C" int sige_scatter(const float *out_blocks, const sige_conv_desc *cd, c
     p.residual = static_cast<const uint8_t *>(residual);
     p.y = static_cast<uint8_t *>(y);
     const int64_t work = (int64_t)capacity * p.N * p.b * p.b * (p.Co / 4);
+    prefer_max_shared(k_scatter);
     k_scatter<<<grid_for(work, 256), 256, 0, (cudaStream_t)stream>>>(p);
     count_launch();
     return launch_check();
@@ -250,6 +252,7 @@ extern "C" int sige_groupnorm_affine(const void *x, const sige_tensor_desc *xd, 
     p.x = static_cast<const uint8_t *>(x);
     p.N = xd->n; p.HW = xd->h * xd->w; p.C = xd->c; p.dtype = xd->dtype; p.groups = groups;
     p.gamma = gamma; p.beta = beta; p.eps = eps; p.scale = scale; p.shift = shift;
+    prefer_max_shared(k_gn_affine);
     k_gn_affine<<<xd->n * groups, 1024, 0, (cudaStream_t)stream>>>(p);
     count_launch();
     return launch_check();

@@ -271,11 +271,22 @@ __device__ __noinline__ void phase2(const MaskParams &p, const ScaleParams *sc)
         const uint8_t *g = p.flags + q.flag_off;
         int base = 0;
         if (nw <= kMaxWords && D < 32) {
-            // flag bytes -> bit words (one ballot per word)
+            // flag bytes -> shared memory in one round of 16-byte loads (the
+            // flag area of a scale is 16-byte aligned and padded), then one
+            // ballot per bit word
+            const int nt = q.th * q.tw;
+            uint8_t *sflag = reinterpret_cast<uint8_t *>(sdil);   // free until the dilation pass
+            if (nt <= (int)sizeof(sdil)) {
+#pragma unroll 1
+                for (int t = threadIdx.x * 16; t < nt; t += blockDim.x * 16)
+                    *reinterpret_cast<uint4 *>(sflag + t) = __ldcg(reinterpret_cast<const uint4 *>(g + t));
+                __syncthreads();
+            }
+            const bool in_smem = nt <= (int)sizeof(sdil);
 #pragma unroll 1
             for (int wi = warp; wi < nw; wi += nwarps) {
                 const int i = wi / wpr, j = (wi - i * wpr) * 32 + lane;
-                const int f = j < q.tw ? __ldcg(g + i * q.tw + j) : 0;
+                const int f = j < q.tw ? (in_smem ? sflag[i * q.tw + j] : __ldcg(g + i * q.tw + j)) : 0;
                 const uint32_t word = __ballot_sync(0xFFFFFFFFu, f != 0);
                 if (lane == 0)
                     sbits[wi] = word;
@@ -504,6 +515,7 @@ extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const si
     int64_t per_cta = (int64_t)kMaskThreads * kMaskUnroll;
     int grid = (int)std::min<int64_t>((p.nwork + per_cta - 1) / per_cta, (int64_t)device_sm_count() * occ[dev]);
     grid = std::max(grid, 1);
+    prefer_max_shared(k_mask_reduce);
     k_mask_reduce<<<grid, kMaskThreads, 0, (cudaStream_t)stream>>>(p);
     count_launch();
     return launch_check();

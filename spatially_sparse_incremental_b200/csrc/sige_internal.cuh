@@ -58,6 +58,20 @@ __device__ __forceinline__ uint4 ld_nc16(const void *p)
 
 // Host-side helpers (sige_api.cu)
 int launch_check();           // SIGE_OK or SIGE_ERR_CUDA after a launch
+// Every kernel of the library asks for the largest shared-memory carveout, the
+// configuration the tensor-core conv needs: consecutive launches then run
+// without reconfiguring the SM's L1 / shared-memory split in between.
+template <typename K>
+inline void prefer_max_shared(K kernel)
+{
+    static int done[64] = {0};
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64 || done[d])
+        return;
+    cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    cudaGetLastError();   // a refused preference is not an error of the call
+    done[d] = 1;
+}
 void count_launch();
 int device_sm_count();
 

@@ -342,13 +342,18 @@ def run_sige(args):
             launches[nm] = sige.sige_launch_count() - before
     stream.synchronize()
     n_tiles = int(d["cnt"].item())
+
+    def whole_step():
+        for fn in calls.values():
+            fn()
+    step_graph = {"step": capture(whole_step, stream)}
     graphs = {nm: capture(fn, stream) for nm, fn in calls.items()}
     dgraphs = {nm: capture(fn, stream) for nm, fn in dense_calls(d, stream).items()}
     flush = L2Flush(dev)
     stream.synchronize()
 
     # warm-up steps
-    timed_graph_steps(graphs, flush, args.warmup, stream)
+    timed_graph_steps(step_graph, flush, args.warmup, stream)
 
     def barrier():
         if ws > 1:
@@ -356,11 +361,15 @@ def run_sige(args):
     barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(dev.index)
-    per, tot = timed_graph_steps(graphs, flush, args.steps, stream)
+    _, tot = timed_graph_steps(step_graph, flush, args.steps, stream)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
     step_ms = float(np.mean(tot))
+    # per-call breakdown: each call in a graph of its own (so each number also
+    # carries one graph launch), same L2 flush before every step
+    timed_graph_steps(graphs, flush, args.warmup, stream)
+    per, _ = timed_graph_steps(graphs, flush, args.steps, stream)
     kern_ms = {nm: float(np.mean(v)) for nm, v in per.items()}
     if ws > 1:
         t = torch.tensor([step_ms] + [kern_ms[k] for k in kern_ms], dtype=torch.float64, device=dev)
@@ -448,7 +457,7 @@ def run_sige(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "H": H, "W": W, "C": C, "block": BLOCK, "edit_area": 0.012,
                    "active_tiles": n_tiles, "tile_fraction": n_tiles / d["cap"],
-                   "l2": "cold: 256 MiB write then 256 MiB read (clean lines) before every step, untimed", "launch": "one CUDA graph per call",
+                   "l2": "cold: 256 MiB write then 256 MiB read (clean lines) before every step, untimed", "launch": "one CUDA graph per step (mask + conv1 + conv2); breakdown_us from one graph per call",
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
         "breakdown_us": {k: v * 1e3 for k, v in kern_ms.items()},
         "dense_conv_us": dense_conv_ms * 1e3, "sparse_conv_us": sparse_conv_ms * 1e3,
@@ -465,9 +474,10 @@ def run_sige(args):
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    for g in list(graphs.values()) + list(dgraphs.values()):
+    for g in list(graphs.values()) + list(dgraphs.values()) + list(step_graph.values()):
         del g
     graphs.clear()
+    step_graph.clear()
     dgraphs.clear()
     if ws > 1:
         torch.distributed.barrier()

@@ -109,7 +109,11 @@ typedef struct {
  *   workspace      : device, >= sige_reduce_mask_workspace_bytes(), zero-filled
  *                    before its first use; each call leaves it zero-filled
  *                    apart from a recorded device error.  One workspace per
- *                    stream: calls sharing one must not overlap on the GPU. */
+ *                    stream: calls sharing one must not overlap on the GPU.
+ * One CTA of the launch waits (bounded, about 4 s) for the others to finish
+ * comparing; past the bound the device error SIGE_ERR_TIMEOUT is recorded, no
+ * list or count is written, and the workspace must be zero-filled again
+ * before its next use. */
 size_t sige_reduce_mask_workspace_bytes(const sige_tensor_desc *in, int32_t n_scales,
                                         const sige_scale_desc *scales);
 int sige_reduce_mask(const void *a_orig, const void *a_edit, const sige_tensor_desc *in,

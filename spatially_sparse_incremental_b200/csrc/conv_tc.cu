@@ -556,6 +556,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // everything above touches only this CTA's own resources; the tile list,
+    // the activations and the output may come from the kernel before
+    pdl_trigger();
+    pdl_wait();
 
     const int ntile = c.dense ? c.tiles_total : min(__ldg(c.count), c.cap);
     const int G = ntile * c.N;
@@ -1116,8 +1120,10 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
             return SIGE_ERR_CUDA;
         smem_set[dev] = 1;
     }
-    k_conv_tc<<<p.num_sms, kTcThreads, kSmemLimit, stream>>>(p, map, xmap);
+    const cudaError_t e = launch_pdl(k_conv_tc, dim3(p.num_sms), dim3(kTcThreads), kSmemLimit, stream, p, map, xmap);
     count_launch();
+    if (e != cudaSuccess)
+        return SIGE_ERR_CUDA;
     return launch_check();
 }
 

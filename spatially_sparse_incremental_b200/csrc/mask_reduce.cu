@@ -12,12 +12,19 @@
 //     scale, the tile its pixel falls in.  Downsampling by an integer factor f
 //     followed by b x b tiles is the same as tiles of b*f input pixels, so the
 //     OR-downsample and the tile OR collapse into one flag store per scale.
-//   phase 2 (the last CTA to arrive): per scale, dilate the tile flags by
-//     `dilate` tiles (equal to dilating the scale's mask by dilate*b pixels
-//     before tiling), compact the active tiles in row-major order with a
-//     block-wide prefix sum, write the (h0, w0) list and the count, then clear
-//     the flags and the arrival counter so the workspace is ready for the next
-//     call.
+//   phase 2 (CTA 0, which takes no part in phase 1): per scale, dilate the
+//     tile flags by `dilate` tiles (equal to dilating the scale's mask by
+//     dilate*b pixels before tiling), compact the active tiles in row-major
+//     order with a block-wide prefix sum, write the (h0, w0) list and the
+//     count, then clear the flags and the arrival counter so the workspace is
+//     ready for the next call.
+//
+// Phase 2 runs once per call on one CTA, so its cost is latency: each of its
+// instructions is fetched cold.  CTA 0 therefore runs it once without storing
+// anything while the other CTAs stream the inputs, which leaves its code in
+// this SM's instruction cache, then waits (bounded) for the last arrival and
+// runs it for real.  CTA 0 is the only CTA that waits on others, and the
+// others wait on nothing, so any scheduling order of the CTAs completes.
 #include <algorithm>
 #include <mutex>
 
@@ -32,6 +39,7 @@ struct ScaleParams {
     int32_t capacity;        // pairs
     int32_t flag_off;        // byte offset of this scale's flags
     int32_t idx_off;         // pair offset of this scale's list
+    int32_t log_h, log_w;    // log2 of tile_h / tile_w when powers of two, else -1
 };
 
 struct MaskParams {
@@ -51,6 +59,8 @@ struct MaskParams {
     int32_t mode;        // 0 = NHWC 16-byte vectors, 1 = NCHW 16-byte vectors, 2 = scalar
     int32_t vpp;         // mode 0: vectors per pixel
     int32_t epv;         // elements per vector
+    int32_t pow2;        // vpp, H and W are powers of two: index math by shifts
+    int32_t log_vpp, log_w, log_epv;
 };
 
 constexpr int kMaskThreads = 256;
@@ -94,14 +104,17 @@ __device__ __forceinline__ uint32_t diff_bits16(uint4 a, uint4 b, int dtype, flo
     return bits;
 }
 
-// The scale table is indexed with a runtime scale number; kernel parameters
-// read that way go through generic loads, so every CTA first copies the table
-// into shared memory.
+// Kernel parameters read through a pointer or with a runtime index go through
+// generic loads, which cost about a global-memory round trip each.  Every CTA
+// therefore copies the parameter block into shared memory once, and the
+// out-of-line functions below read that copy.
 __device__ __forceinline__ void mark(const ScaleParams *sc, int n_scales, uint8_t *flags, int y, int x)
 {
     for (int s = 0; s < n_scales; ++s) {
         const ScaleParams q = sc[s];
-        flags[q.flag_off + (y / q.tile_h) * q.tw + (x / q.tile_w)] = 1;
+        const int ty = q.log_h >= 0 ? y >> q.log_h : y / q.tile_h;
+        const int tx = q.log_w >= 0 ? x >> q.log_w : x / q.tile_w;
+        flags[q.flag_off + ty * q.tw + tx] = 1;
     }
 }
 
@@ -114,43 +127,37 @@ __device__ __forceinline__ float scalar_elem(const uint8_t *base, int64_t i, int
     return reinterpret_cast<const float *>(base)[i];
 }
 
-// Exact test of the vectors whose bytes differ (rare: only edited pixels), kept
-// out of line so that the streaming loop stays a few dozen instructions.
-// The vectors are read again here (a few percent of them at most) so that the
-// streaming loop keeps its loads in registers.
-__device__ __noinline__ void mark_vectors(const MaskParams &p, const ScaleParams *sc, int64_t v0, int64_t stride,
-                                          uint32_t neq)
+// Mark the tiles of the elements set in `bits` (the exact test of vector v);
+// out of line, since only vectors inside the edit reach it.
+__device__ __noinline__ void mark_bits(const MaskParams &p, const ScaleParams *sc, int64_t v, uint32_t bits)
 {
-    const int64_t HW = (int64_t)p.H * p.W;
-    while (neq) {
-        const int u = __ffs(neq) - 1;
-        neq &= neq - 1;
-        const int64_t v = v0 + u * stride;
-        uint32_t bits = diff_bits16(ld_nc16(p.a + v * 16), ld_nc16(p.b + v * 16), p.dtype, p.thr);
-        if (!bits)
-            continue;
-        if (p.mode == 0) {
+    if (p.mode == 0) {
+        if (p.pow2) {
+            const int64_t pix = v >> p.log_vpp;
+            mark(sc, p.n_scales, p.flags, (int)(pix >> p.log_w) & (p.H - 1), (int)pix & (p.W - 1));
+        } else {
+            const int64_t HW = (int64_t)p.H * p.W;
             const int64_t pix = v / p.vpp;
             mark(sc, p.n_scales, p.flags, (int)((pix % HW) / p.W), (int)(pix % p.W));
-        } else {
-            const int64_t e0 = v * p.epv;
-            const int y = (int)((e0 / p.W) % p.H);
-            const int x0 = (int)(e0 % p.W);
-            while (bits) {
-                const int k = __ffs(bits) - 1;
-                bits &= bits - 1;
-                mark(sc, p.n_scales, p.flags, y, x0 + k);
-            }
+        }
+    } else {
+        const int64_t e0 = v * p.epv;
+        const int y = p.pow2 ? (int)(e0 >> p.log_w) & (p.H - 1) : (int)((e0 / p.W) % p.H);
+        const int x0 = p.pow2 ? (int)e0 & (p.W - 1) : (int)(e0 % p.W);
+        while (bits) {
+            const int k = __ffs(bits) - 1;
+            bits &= bits - 1;
+            mark(sc, p.n_scales, p.flags, y, x0 + k);
         }
     }
 }
 
-__device__ __noinline__ bool scalar_pass(const MaskParams &p, const ScaleParams *sc)
+__device__ __noinline__ bool scalar_pass(const MaskParams &p, const ScaleParams *sc, int worker, int nworkers)
 {
     bool wrote = false;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t stride = (int64_t)nworkers * blockDim.x;
     const int64_t HW = (int64_t)p.H * p.W;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.nwork; i += stride) {
+    for (int64_t i = (int64_t)worker * blockDim.x + threadIdx.x; i < p.nwork; i += stride) {
         const float d = fabsf(scalar_elem(p.b, i, p.dtype) - scalar_elem(p.a, i, p.dtype));
         if (d > p.thr) {
             wrote = true;
@@ -171,16 +178,17 @@ __device__ __noinline__ bool scalar_pass(const MaskParams &p, const ScaleParams 
 
 // Stream both inputs once.  Bitwise-equal 16-byte vectors cannot differ by
 // more than a non-negative threshold, so the hot loop only compares raw bits;
-// vectors whose bytes differ get the exact float32 test in mark_vectors.
-__device__ __forceinline__ bool phase1(const MaskParams &p, const ScaleParams *sc)
+// vectors whose bytes differ get the exact float32 test on the values already
+// in registers (the unrolled loop keeps every index a constant).
+__device__ __forceinline__ bool phase1(const MaskParams &p, const MaskParams &sp, int worker, int nworkers)
 {
     if (p.mode == 2)
-        return scalar_pass(p, sc);
+        return scalar_pass(sp, sp.sc, worker, nworkers);
     bool wrote = false;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t stride = (int64_t)nworkers * blockDim.x;
     const int64_t nwork = p.nwork;
     const uint8_t *a = p.a, *b = p.b;
-    for (int64_t v0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v0 < nwork; v0 += stride * kMaskUnroll) {
+    for (int64_t v0 = (int64_t)worker * blockDim.x + threadIdx.x; v0 < nwork; v0 += stride * kMaskUnroll) {
         uint4 av[kMaskUnroll], bv[kMaskUnroll];
 #pragma unroll
         for (int u = 0; u < kMaskUnroll; ++u) {
@@ -199,7 +207,14 @@ __device__ __forceinline__ bool phase1(const MaskParams &p, const ScaleParams *s
                                (av[u].w ^ bv[u].w)) != 0) << u;
         if (neq) {
             wrote = true;
-            mark_vectors(p, sc, v0, stride, neq);
+#pragma unroll
+            for (int u = 0; u < kMaskUnroll; ++u) {
+                if (neq & (1u << u)) {
+                    const uint32_t bits = diff_bits16(av[u], bv[u], p.dtype, p.thr);
+                    if (bits)
+                        mark_bits(sp, sp.sc, v0 + u * stride, bits);
+                }
+            }
         }
     }
     return wrote;
@@ -256,11 +271,111 @@ __device__ __forceinline__ uint32_t row_word(const uint32_t *bits, int wpr, int 
     return v;
 }
 
-__device__ __noinline__ void phase2(const MaskParams &p, const ScaleParams *sc)
+// Tile grids of at most 32 x 32 (every grid of the SIGE workloads): one warp
+// per scale, lane i holding tile row i as a bit word.  The scale's flags (at
+// most 1 KB) come into shared memory with two 16-byte loads per lane (many
+// small loads per thread do not overlap well); dilation is shuffles and
+// shifts, the row-major prefix sum a warp scan, so no block barrier is on the
+// path.
+__device__ __forceinline__ void scale_small(const MaskParams &p, const ScaleParams &qs, int s, bool commit,
+                                            uint8_t *stage)
+{
+    const ScaleParams q = qs;   // registers: stores below must not force re-reads
+    const int lane = threadIdx.x & 31, D = p.dilate;
+    const int nb = (q.th * q.tw + 15) & ~15;
+    const uint4 *g = reinterpret_cast<const uint4 *>(p.flags + q.flag_off);
+    uint4 *st = reinterpret_cast<uint4 *>(stage);
+    const uint4 g0 = lane * 16 < nb ? __ldcg(g + lane) : make_uint4(0, 0, 0, 0);
+    const uint4 g1 = (lane + 32) * 16 < nb ? __ldcg(g + lane + 32) : make_uint4(0, 0, 0, 0);
+    st[lane] = g0;
+    st[lane + 32] = g1;
+    __syncwarp();
+    // lane i assembles tile row i: bit j = flag (i, j)
+    uint32_t mine = 0;
+    if (lane < q.th) {
+        const uint8_t *row = stage + lane * q.tw;
+        if ((q.tw & 3) == 0) {
+            uint32_t w[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                w[k] = 4 * k < q.tw ? *reinterpret_cast<const uint32_t *>(row + 4 * k) : 0u;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    mine |= (uint32_t)(((w[k] >> (8 * b)) & 0xFFu) != 0) << (4 * k + b);
+        } else {
+#pragma unroll 4
+            for (int j = 0; j < q.tw; ++j)
+                mine |= (uint32_t)(row[j] != 0) << j;
+        }
+    }
+    uint32_t v = mine;
+#pragma unroll 1
+    for (int d = 1; d <= D; ++d) {
+        const uint32_t up = __shfl_up_sync(0xFFFFFFFFu, mine, d);
+        const uint32_t dn = __shfl_down_sync(0xFFFFFFFFu, mine, d);
+        if (lane >= d)
+            v |= up;
+        if (lane + d < 32)
+            v |= dn;
+    }
+    uint32_t h = v;
+#pragma unroll 1
+    for (int d = 1; d <= D; ++d)
+        h |= (v << d) | (v >> d);
+    h &= q.tw == 32 ? 0xFFFFFFFFu : ((1u << q.tw) - 1u);
+    if (lane >= q.th)
+        h = 0;
+    const int c = __popc(h);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o)
+            incl += t;
+    }
+    const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    if (!commit)
+        return;
+    int pos = incl - c;
+    int2 *out = reinterpret_cast<int2 *>(p.idx) + q.idx_off;
+    while (h) {
+        const int k = __ffs(h) - 1;
+        h &= h - 1;
+        if (pos < q.capacity)
+            out[pos] = make_int2(lane * q.block, k * q.block);
+        ++pos;
+    }
+    if (lane == 0) {
+        p.counts[s] = total;
+        if (total > q.capacity)
+            record_error(p.hdr, SIGE_ERR_CAPACITY, s);
+    }
+    // leave this scale's flags zero-filled for the next call
+#pragma unroll 1
+    for (int o = lane * 16; o < nb; o += 32 * 16)
+        *reinterpret_cast<uint4 *>(p.flags + q.flag_off + o) = make_uint4(0, 0, 0, 0);
+}
+
+// commit = false: the same work with every global store left out (the warm-up
+// pass of CTA 0, which may read flags that other CTAs are still writing).
+__device__ __noinline__ void phase2(const MaskParams &p, const ScaleParams *sc, bool commit)
 {
     __shared__ __align__(16) uint32_t sbits[kMaxWords];    // raw tile bits
     __shared__ __align__(16) uint32_t sdil[kMaxWords];     // dilated tile bits
     __shared__ int warp_sums[33];
+    bool small = p.dilate < 32;
+    for (int s = 0; s < p.n_scales; ++s)
+        small = small && sc[s].th <= 32 && sc[s].tw <= 32;
+    if (small) {
+        const int warp = threadIdx.x >> 5;
+        if (warp < p.n_scales)
+            scale_small(p, sc[warp], warp, commit, reinterpret_cast<uint8_t *>(sdil) + warp * 1024);
+        if (commit && threadIdx.x == 0)
+            p.hdr->arrive = 0;
+        return;
+    }
     const int n_scales = p.n_scales, D = p.dilate;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
 #pragma unroll 1
@@ -323,7 +438,7 @@ __device__ __noinline__ void phase2(const MaskParams &p, const ScaleParams *sc)
                 while (m) {
                     const int k = __ffs(m) - 1;
                     m &= m - 1;
-                    if (pos < q.capacity)
+                    if (commit && pos < q.capacity)
                         reinterpret_cast<int2 *>(p.idx)[q.idx_off + pos] = make_int2(i * q.block, (jb + k) * q.block);
                     ++pos;
                 }
@@ -349,20 +464,22 @@ __device__ __noinline__ void phase2(const MaskParams &p, const ScaleParams *sc)
                 }
                 int chunk_total;
                 const int pos = base + block_scan(act, warp_sums, &chunk_total);
-                if (act && pos < q.capacity) {
+                if (commit && act && pos < q.capacity) {
                     const int i = t / q.tw, j = t - i * q.tw;
                     reinterpret_cast<int2 *>(p.idx)[q.idx_off + pos] = make_int2(i * q.block, j * q.block);
                 }
                 base += chunk_total;
             }
         }
-        if (threadIdx.x == 0) {
+        if (commit && threadIdx.x == 0) {
             p.counts[s] = base;
             if (base > q.capacity)
                 record_error(p.hdr, SIGE_ERR_CAPACITY, s);
         }
         __syncthreads();
     }
+    if (!commit)
+        return;
     // leave the workspace zero-filled for the next call
     const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll 1
@@ -372,30 +489,68 @@ __device__ __noinline__ void phase2(const MaskParams &p, const ScaleParams *sc)
         p.hdr->arrive = 0;
 }
 
+// Bound of CTA 0's wait for the streaming CTAs (about 4 s at 2 GHz); past it
+// the call records SIGE_ERR_TIMEOUT and leaves its workspace as it is.
+constexpr long long kMaskWaitCycles = 1ll << 33;
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *ptr)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
 __global__ void __launch_bounds__(kMaskThreads) k_mask_reduce(const __grid_constant__ MaskParams p)
 {
-    __shared__ ScaleParams s_sc[kMaxScales];
-    if (threadIdx.x < kMaxScales)
-        s_sc[threadIdx.x] = p.sc[threadIdx.x];
+    __shared__ MaskParams s_p;
+    __shared__ int s_go;
+    if (threadIdx.x == 0)
+        s_p = p;
+    pdl_trigger();
+    pdl_wait();   // the inputs, lists and workspace may come from the kernel before
     __syncthreads();
-    if (phase1(p, s_sc))
+    const ScaleParams *s_sc = s_p.sc;
+    if (blockIdx.x == 0) {
+        phase2(s_p, s_sc, false);
+        if (threadIdx.x == 0) {
+            const uint32_t want = gridDim.x - 1;
+            const long long t0 = clock64();
+            int go = 1;
+            while (ld_acquire_u32(&p.hdr->arrive) != want) {
+                if (clock64() - t0 > kMaskWaitCycles) {
+                    record_error(p.hdr, SIGE_ERR_TIMEOUT, -1);
+                    go = 0;
+                    break;
+                }
+                __nanosleep(32);
+            }
+            s_go = go;
+        }
+        __syncthreads();
+        if (s_go)
+            phase2(s_p, s_sc, true);
+        return;
+    }
+    if (phase1(p, s_p, blockIdx.x - 1, gridDim.x - 1))
         __threadfence();   // flags stored by this thread are visible before the arrival below
     __syncthreads();
-    __shared__ int is_last;
-    if (threadIdx.x == 0) {
-        unsigned prev = atomicAdd(&p.hdr->arrive, 1u);
-        is_last = (prev == gridDim.x - 1);
-    }
-    __syncthreads();
-    if (!is_last)
-        return;
-    __threadfence();
-    phase2(p, s_sc);
+    if (threadIdx.x == 0)
+        atomicAdd(&p.hdr->arrive, 1u);
 }
 
 // ------------------------------------------------------------------ host
 
 static size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
+
+static int32_t log2_exact(int64_t v)
+{
+    if (v < 1 || (v & (v - 1)))
+        return -1;
+    int32_t l = 0;
+    while ((int64_t)1 << l < v)
+        ++l;
+    return l;
+}
 
 static bool scales_ok(const sige_tensor_desc *in, int32_t n_scales, const sige_scale_desc *scales)
 {
@@ -477,6 +632,8 @@ extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const si
         o.capacity = q.capacity;
         o.flag_off = foff;
         o.idx_off = ioff;
+        o.log_h = log2_exact(o.tile_h);
+        o.log_w = log2_exact(o.tile_w);
         foff += (int32_t)align16((size_t)o.th * o.tw);
         ioff += q.capacity;
     }
@@ -501,6 +658,10 @@ extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const si
         p.mode = 2;
         p.nwork = nelem;
     }
+    p.log_vpp = p.mode == 0 ? log2_exact(p.vpp) : 0;
+    p.log_w = log2_exact(in->w);
+    p.log_epv = log2_exact(p.epv);
+    p.pow2 = p.log_vpp >= 0 && p.log_w >= 0 && log2_exact(in->h) >= 0;
     static int occ[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -512,12 +673,15 @@ extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const si
             n = 1;
         occ[dev] = n;
     }
+    // CTA 0 reduces; the others stream the inputs
     int64_t per_cta = (int64_t)kMaskThreads * kMaskUnroll;
-    int grid = (int)std::min<int64_t>((p.nwork + per_cta - 1) / per_cta, (int64_t)device_sm_count() * occ[dev]);
-    grid = std::max(grid, 1);
+    int grid = 1 + (int)std::min<int64_t>((p.nwork + per_cta - 1) / per_cta,
+                                          std::max<int64_t>(1, (int64_t)device_sm_count() * occ[dev] - 1));
     prefer_max_shared(k_mask_reduce);
-    k_mask_reduce<<<grid, kMaskThreads, 0, (cudaStream_t)stream>>>(p);
+    const cudaError_t e = launch_pdl(k_mask_reduce, dim3(grid), dim3(kMaskThreads), 0, (cudaStream_t)stream, p);
     count_launch();
+    if (e != cudaSuccess)
+        return SIGE_ERR_CUDA;
     return launch_check();
 }
 

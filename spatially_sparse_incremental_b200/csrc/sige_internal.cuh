@@ -1,6 +1,7 @@
 // Internal definitions shared by the CUDA sources of libsige.
 #pragma once
 
+#include <utility>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -74,5 +75,32 @@ inline void prefer_max_shared(K kernel)
 }
 void count_launch();
 int device_sm_count();
+
+// Programmatic dependent launch.  A kernel launched this way may start while
+// the kernel before it in the stream is still running: its CTAs take SMs as
+// that kernel's CTAs leave.  It must call pdl_wait() before it touches any
+// memory the previous kernel may write (pdl_wait returns once that kernel has
+// completed and its writes are visible), and it calls pdl_trigger() to let the
+// kernel after it start early in the same way.  Both are no-ops for a kernel
+// launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... P, typename... A>
+inline cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              A &&...args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
 
 } // namespace sige

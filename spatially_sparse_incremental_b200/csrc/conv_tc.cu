@@ -190,6 +190,48 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
         : "memory");
 }
 
+// Warp-wide forms.  The whole converged warp calls them with identical
+// arguments and one lane, chosen by elect.sync, issues the instruction.  The
+// issuing loops then stay warp-uniform (their exits depend only on votes), so
+// the compiler keeps descriptors, coordinates and stage counters in uniform
+// registers, which is what the tensor-core and TMA instructions read.
+__device__ __forceinline__ void tc_mma_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n .reg .pred p, e;\n .reg .b32 l;\n elect.sync l|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_commit_w(uint32_t bar)
+{
+    asm volatile(
+        "{\n .reg .pred e;\n .reg .b32 l;\n elect.sync l|e, 0xffffffff;\n"
+        " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(bar)
+        : "memory");
+}
+
+// expect_tx on `bar` and the 2-D tile load that completes it, from one lane
+__device__ __forceinline__ void tma_load_2d_w(uint32_t dst, const CUtensorMap *map, uint32_t bar, uint32_t bytes, int x,
+                                              int y)
+{
+    asm volatile(
+        "{\n .reg .pred e;\n .reg .b32 l;\n elect.sync l|e, 0xffffffff;\n"
+        " @e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%2], %3;\n"
+        " @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%4, %5}], [%2];\n}\n"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(bytes), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Bounded wait by every lane of a warp; the outcome is the same in all lanes.
+__device__ __forceinline__ bool mbar_wait_w(uint32_t bar, uint32_t parity, volatile int *abort_flag, WsHeader *hdr,
+                                            int where)
+{
+    return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag, hdr, where));
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
 {
     uint32_t r[16];
@@ -567,62 +609,61 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const Carve cv = carve(p, sc.T);
 
     if (warp == 0) {
-        // ---------------- weight producer (TMA)
-        if (lane == 0) {
-            // stage index and phase advance incrementally: a runtime division
-            // per k-chunk costs more than the TMA issue itself
-            int s = 0;
-            uint32_t ph = 1, issued = 0;
-            bool ok = true;
+        // ---------------- weight producer (TMA), whole warp, one issuing lane
+        // stage index and phase advance incrementally: a runtime division per
+        // k-chunk costs more than the TMA issue itself
+        int s = 0;
+        uint32_t ph = 1, issued = 0;
+        bool ok = true;
 #pragma unroll 1
-            for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
-                const Unit un = decode_unit(p, sc, u);
-                int q = un.kb / p.taps, tap = un.kb - q * p.taps;
-                const int y0 = un.mt * 128;
+        for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
+            const Unit un = decode_unit(p, sc, u);
+            int q = un.kb / p.taps, tap = un.kb - q * p.taps;
+            const int y0 = un.mt * 128;
 #pragma unroll 1
-                for (int kc = un.kb; kc < un.ke; ++kc) {
-                    if (!mbar_wait(a_empty(s), ph, abort_flag, hdr, 1)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_expect_tx(a_full(s), kAStageBytes);
-                    tma_load_2d(sbase + cv.a_base + s * kAStageBytes, &tmw, a_full(s), tap * c.Cin + q * 64, y0);
-                    ++issued;
-                    if (++s == cv.SA) {
-                        s = 0;
-                        ph ^= 1;
-                    }
-                    if (++tap == p.taps) {
-                        tap = 0;
-                        ++q;
-                    }
+            for (int kc = un.kb; kc < un.ke; ++kc) {
+                if (!mbar_wait_w(a_empty(s), ph, abort_flag, hdr, 1)) {
+                    ok = false;
+                    break;
                 }
-            }
-            // every issued load must land before the CTA may exit: wait for the
-            // last use of each stage
-#pragma unroll 1
-            for (uint32_t k = 0; k < (uint32_t)cv.SA && k < issued; ++k) {
-                // the use of stage st waited on a_empty with parity w, so its
-                // a_full completion has parity w ^ 1; w is ph for stages used
-                // in the current round and ph ^ 1 for those before the wrap
-                int st = s - 1 - (int)k;
-                uint32_t full_par = ph ^ 1;
-                if (st < 0) {
-                    st += cv.SA;
-                    full_par ^= 1;
+                tma_load_2d_w(sbase + cv.a_base + s * kAStageBytes, &tmw, a_full(s), kAStageBytes,
+                              tap * c.Cin + q * 64, y0);
+                ++issued;
+                if (++s == cv.SA) {
+                    s = 0;
+                    ph ^= 1;
                 }
-                const long long t0 = clock64();
-                while (!mbar_try(a_full(st), full_par) && clock64() - t0 < kWaitCycles) {
+                if (++tap == p.taps) {
+                    tap = 0;
+                    ++q;
                 }
             }
         }
+        // every issued load must land before the CTA may exit: wait for the
+        // last use of each stage
+#pragma unroll 1
+        for (uint32_t k = 0; k < (uint32_t)cv.SA && k < issued; ++k) {
+            // the use of stage st waited on a_empty with parity w, so its
+            // a_full completion has parity w ^ 1; w is ph for stages used in
+            // the current round and ph ^ 1 for those before the wrap
+            int st = s - 1 - (int)k;
+            uint32_t full_par = ph ^ 1;
+            if (st < 0) {
+                st += cv.SA;
+                full_par ^= 1;
+            }
+            const long long t0 = clock64();
+            while (!mbar_try(a_full(st), full_par) && clock64() - t0 < kWaitCycles) {
+            }
+        }
+        __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer
-        // One thread issues every MMA, so this loop is kept to the bare chain:
-        // per k-chunk one barrier test, the MMAs and a commit.  The B
+        // ---------------- MMA issuer: the whole warp runs the loop, one lane issues
+        // The issue is a single serial chain, so this loop is kept to the bare
+        // minimum: per k-chunk one barrier test, the MMAs and a commit.  The B
         // descriptor is built once per halo stage and moves by constant
         // offsets from tap to tap; the A descriptor moves by one stage.
-        if (lane == 0) {
+        {
             int sa = 0, sb = 0;
             uint32_t pa = 0, pb = 0, uit = 0, ait = 0;
             bool ok = true;
@@ -642,7 +683,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll 1
             for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, sc, u);
-                if (uit > 0 && !mbar_wait(acc_empty, (uit - 1) & 1, abort_flag, hdr, 2)) {
+                if (uit > 0 && !mbar_wait_w(acc_empty, (uit - 1) & 1, abort_flag, hdr, 2)) {
                     ok = false;
                     break;
                 }
@@ -652,7 +693,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll 1
                 for (int kc = un.kb; kc < un.ke && ok;) {
                     // one halo stage: taps [tap, tap_end) of one 64-channel chunk
-                    if (!mbar_wait(b_full(sb), pb, abort_flag, hdr, 3)) {
+                    if (!mbar_wait_w(b_full(sb), pb, abort_flag, hdr, 3)) {
                         ok = false;
                         break;
                     }
@@ -664,18 +705,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     uint64_t b_tap = b_stage + (uint64_t)r * d_row + (uint64_t)cc * d_col;
 #pragma unroll 1
                     for (; tap < tap_end; ++tap, ++kc) {
-                        if (!mbar_wait(a_full(sa), pa, abort_flag, hdr, 4)) {
+                        if (!mbar_wait_w(a_full(sa), pa, abort_flag, hdr, 4)) {
                             ok = false;
                             break;
                         }
-                        tc_fence_after();
                         if (p.mode == 0) {
 #pragma unroll
                             for (int ks = 0; ks < 4; ++ks) {
                                 uint64_t bt = b_tap + ks * d_ks;
 #pragma unroll 1
                                 for (int t = 0; t < nT; ++t, bt += d_tile)
-                                    tc_mma(tmem + t * 64, a_cur + 2 * ks, bt, idesc, ks ? 1u : acc0);
+                                    tc_mma_w(tmem + t * 64, a_cur + 2 * ks, bt, idesc, ks ? 1u : acc0);
                             }
                         } else {
 #pragma unroll
@@ -687,12 +727,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                     uint64_t bj = bi;
 #pragma unroll 1
                                     for (int j = 0; j < bb; ++j, bj += d_j, col += nT)
-                                        tc_mma(tmem + col, a_cur + 2 * ks, bj, idesc, ks ? 1u : acc0);
+                                        tc_mma_w(tmem + col, a_cur + 2 * ks, bj, idesc, ks ? 1u : acc0);
                                 }
                             }
                         }
                         acc0 = 1;
-                        tc_commit(a_empty(sa));
+                        tc_commit_w(a_empty(sa));
                         ++ait;
                         if (++sa == cv.SA) {
                             sa = 0;
@@ -709,7 +749,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                     if (!ok)
                         break;
-                    tc_commit(b_empty(sb));
+                    tc_commit_w(b_empty(sb));
                     if (++sb == p.SB) {
                         sb = 0;
                         pb ^= 1;
@@ -718,16 +758,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 if (!ok)
                     break;
-                tc_commit(acc_full);
+                tc_commit_w(acc_full);
                 ++uit;
             }
             // every MMA issued by this thread must finish before tensor memory is freed
             if (ait > 0) {
-                tc_commit(drain);
+                tc_commit_w(drain);
                 const long long t0 = clock64();
                 while (!mbar_try(drain, 0) && clock64() - t0 < kWaitCycles) {
                 }
             }
+            __syncwarp();
         }
     } else {
         // ---------------- halo producers + epilogue (warps 2..9)

@@ -60,14 +60,17 @@ def load_peaks():
     return {**FALLBACK_PEAKS, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def src_sha(relpath):
-    with open(os.path.join(ROOT, relpath), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def src_sha(relpaths):
+    h = hashlib.sha256()
+    for rp in relpaths:
+        with open(os.path.join(ROOT, rp), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, when it was taken
-    on the current source of that kernel; else None."""
+    """DRAM bytes (read + write) per launch from the committed ncu summary, when
+    it was taken on the current sources of that kernel; else None."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
@@ -76,9 +79,9 @@ def ncu_traffic(kernel):
     if not d:
         return None
     try:
-        if src_sha(d["source"]) != d["source_sha"]:
+        if src_sha(d["sources"]) != d["source_sha"]:
             return None
-    except OSError:
+    except (OSError, KeyError):
         return None
     return float(d["bytes_per_launch"])
 

@@ -137,6 +137,18 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(vals, device):
+    """Element-wise maximum of a list of floats over all ranks of the default
+    process group (identity with one rank).  Every rank must call it with the
+    same number of values, in the same order of calls."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 # ------------------------------------------------------------------ workload
 
 def make_workload(seed, dev):
@@ -374,11 +386,9 @@ def run_sige(args):
     timed_graph_steps(graphs, flush, args.warmup, stream)
     per, _ = timed_graph_steps(graphs, flush, args.steps, stream)
     kern_ms = {nm: float(np.mean(v)) for nm, v in per.items()}
-    if ws > 1:
-        t = torch.tensor([step_ms] + [kern_ms[k] for k in kern_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        step_ms = float(t[0])
-        kern_ms = {k: float(t[i + 1]) for i, k in enumerate(kern_ms)}
+    red = max_over_ranks([step_ms] + [kern_ms[k] for k in kern_ms], dev)
+    step_ms = red[0]
+    kern_ms = {k: red[i + 1] for i, k in enumerate(kern_ms)}
 
     # dense comparison (same launch mode, L2 flushed)
     dper, dtot = timed_graph_steps(dgraphs, flush, max(10, min(args.steps, 50)), stream)
@@ -405,10 +415,7 @@ def run_sige(args):
         if k >= args.warmup:
             e2e_times.append(e0.elapsed_time(e1))
     e2e_ms = float(np.mean(e2e_times))
-    if ws > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    e2e_ms = max_over_ranks([e2e_ms], dev)[0]
 
     # roofline of the dominant kernel
     work = {"mask": ("hbm", None, mask_work(n_tiles)),

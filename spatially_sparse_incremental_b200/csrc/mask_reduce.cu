@@ -7,9 +7,12 @@
 // active block indices.
 //
 // Layout of the work:
-//   phase 1 (all CTAs, HBM-bound): stream both inputs once with 16-byte
-//     loads; an element whose |edit - orig| > threshold marks, at every
-//     scale, the tile its pixel falls in.  Downsampling by an integer factor f
+//   phase 1 (every CTA but CTA 0, HBM-bound): stream both inputs once.  The
+//     inputs are cut into chunks (up to 16 KB of each input); a CTA takes
+//     every (number of streaming CTAs)-th chunk and keeps six of them in
+//     flight with bulk asynchronous copies into shared memory, so nearly the
+//     whole input is requested at once.  An element whose |edit - orig| >
+//     threshold marks, at every scale, the tile its pixel falls in.  Downsampling by an integer factor f
 //     followed by b x b tiles is the same as tiles of b*f input pixels, so the
 //     OR-downsample and the tile OR collapse into one flag store per scale.
 //   phase 2 (CTA 0, which takes no part in phase 1): per scale, dilate the
@@ -42,7 +45,7 @@ struct ScaleParams {
     int32_t log_h, log_w;    // log2 of tile_h / tile_w when powers of two, else -1
 };
 
-struct MaskParams {
+struct __align__(16) MaskParams {
     const uint8_t *a;  // original
     const uint8_t *b;  // edited
     int32_t N, H, W, C, dtype, layout;
@@ -61,10 +64,27 @@ struct MaskParams {
     int32_t epv;         // elements per vector
     int32_t pow2;        // vpp, H and W are powers of two: index math by shifts
     int32_t log_vpp, log_w, log_epv;
+    int32_t chunk;       // modes 0, 1: vectors per chunk of each input (multiple of 256)
+    int32_t chunks_base, chunks_rem;   // chunks per streaming CTA: base, +1 for the first rem
 };
 
+// Copy the parameter block into shared memory, one 16-byte piece per lane of
+// warp 0: a single round of loads, whose latency the streaming CTAs overlap
+// with their first copies in flight.
+__device__ __forceinline__ void copy_params(MaskParams *dst, const MaskParams &src)
+{
+    constexpr int kPieces = (int)(sizeof(MaskParams) / 16);
+    static_assert(sizeof(MaskParams) % 16 == 0, "parameter block is copied in 16-byte pieces");
+    const int lane = threadIdx.x & 31;
+    static_assert(kPieces <= 64, "two pieces per lane at most");
+    if (lane < kPieces)
+        reinterpret_cast<uint4 *>(dst)[lane] = reinterpret_cast<const uint4 *>(&src)[lane];
+    if (lane + 32 < kPieces)
+        reinterpret_cast<uint4 *>(dst)[lane + 32] = reinterpret_cast<const uint4 *>(&src)[lane + 32];
+}
+
 constexpr int kMaskThreads = 256;
-constexpr int kMaskUnroll = 8;
+constexpr int kScalarPerThread = 8;   // mode 2: elements per thread of the grid size
 
 __device__ __forceinline__ float elem_as_float(uint32_t word, int k, int dtype)
 {
@@ -176,46 +196,119 @@ __device__ __noinline__ bool scalar_pass(const MaskParams &p, const ScaleParams 
     return wrote;
 }
 
-// Stream both inputs once.  Bitwise-equal 16-byte vectors cannot differ by
-// more than a non-negative threshold, so the hot loop only compares raw bits;
-// vectors whose bytes differ get the exact float32 test on the values already
-// in registers (the unrolled loop keeps every index a constant).
-__device__ __forceinline__ bool phase1(const MaskParams &p, const MaskParams &sp, int worker, int nworkers)
+constexpr int kMaskStages = 7;          // chunks in flight per streaming CTA
+constexpr int kMaskChunkMax = 1024;     // vectors (16 KB) per chunk and input
+constexpr size_t kMaskStreamSmem = (size_t)kMaskStages * 2 * kMaskChunkMax * 16;   // 224 KB
+constexpr long long kMaskCopyWait = 1ll << 31;   // bound of one chunk wait (about 1 s)
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
 {
-    if (p.mode == 2)
-        return scalar_pass(sp, sp.sc, worker, nworkers);
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ bool mbar_try_parity(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n .reg .pred q;\n mbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\n selp.u32 %0, 1, 0, q;\n}\n"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
+{
+    if (mbar_try_parity(bar, parity))
+        return true;
+    const long long t0 = clock64();
+    while (!mbar_try_parity(bar, parity))
+        if (clock64() - t0 > kMaskCopyWait)
+            return false;
+    return true;
+}
+
+// Chunk i of this CTA (global chunk worker + i * nworkers) of both inputs into
+// stage i % kMaskStages; one thread issues it.
+__device__ __forceinline__ void issue_chunk(const MaskParams &p, uint8_t *stages, uint64_t *full, int worker,
+                                            int nworkers, int64_t i)
+{
+    const int64_t c = worker + i * nworkers;
+    const int64_t v0 = c * p.chunk;
+    const uint32_t bytes = (uint32_t)(min((int64_t)p.chunk, p.nwork - v0) * 16);
+    const int st = (int)(i % kMaskStages);
+    uint8_t *da = stages + (size_t)st * 2 * kMaskChunkMax * 16;
+    uint8_t *db = da + (size_t)kMaskChunkMax * 16;
+    const uint32_t bar = smem_addr(&full[st]);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * bytes) : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(da)),
+                 "l"(p.a + v0 * 16), "r"(bytes), "r"(bar)
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(db)),
+                 "l"(p.b + v0 * 16), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ int64_t chunks_of(const MaskParams &p, int worker, int nworkers)
+{
+    return p.chunks_base + (worker < p.chunks_rem ? 1 : 0);
+}
+
+// The first copies of a streaming CTA (one thread; barriers initialised).
+__device__ __forceinline__ void issue_first_chunks(const MaskParams &p, uint8_t *stages, uint64_t *full, int worker,
+                                                   int nworkers)
+{
+    const int64_t mine = chunks_of(p, worker, nworkers);
+    for (int64_t i = 0; i < min(mine, (int64_t)kMaskStages); ++i)
+        issue_chunk(p, stages, full, worker, nworkers, i);
+}
+
+// Stream this CTA's chunks through the stage ring and compare them.  The first
+// kMaskStages chunks were issued by issue_first_chunks.
+// Bitwise-equal 16-byte vectors cannot differ by more than a non-negative
+// threshold, so only vectors whose bytes differ get the exact float32 test.  Returns
+// whether this thread stored a flag; *ok turns false if a copy never landed
+// (then every copy still in flight has been waited for, boundedly).
+__device__ __forceinline__ bool phase1_bulk(const MaskParams &p, const MaskParams &sp, uint8_t *stages,
+                                            uint64_t *full, int worker, int nworkers, bool *ok)
+{
+    const int64_t mine = chunks_of(p, worker, nworkers);
     bool wrote = false;
-    const int64_t stride = (int64_t)nworkers * blockDim.x;
-    const int64_t nwork = p.nwork;
-    const uint8_t *a = p.a, *b = p.b;
-    for (int64_t v0 = (int64_t)worker * blockDim.x + threadIdx.x; v0 < nwork; v0 += stride * kMaskUnroll) {
-        uint4 av[kMaskUnroll], bv[kMaskUnroll];
-#pragma unroll
-        for (int u = 0; u < kMaskUnroll; ++u) {
-            const int64_t v = v0 + u * stride;
-            av[u] = make_uint4(0, 0, 0, 0);
-            bv[u] = av[u];
-            if (v < nwork) {
-                av[u] = ld_stream16(a + v * 16);
-                bv[u] = ld_stream16(b + v * 16);
-            }
-        }
-        uint32_t neq = 0;
-#pragma unroll
-        for (int u = 0; u < kMaskUnroll; ++u)
-            neq |= (uint32_t)(((av[u].x ^ bv[u].x) | (av[u].y ^ bv[u].y) | (av[u].z ^ bv[u].z) |
-                               (av[u].w ^ bv[u].w)) != 0) << u;
-        if (neq) {
-            wrote = true;
-#pragma unroll
-            for (int u = 0; u < kMaskUnroll; ++u) {
-                if (neq & (1u << u)) {
-                    const uint32_t bits = diff_bits16(av[u], bv[u], p.dtype, p.thr);
-                    if (bits)
-                        mark_bits(sp, sp.sc, v0 + u * stride, bits);
+    *ok = true;
+    int64_t i = 0;
+    for (; i < mine; ++i) {
+        const int st = (int)(i % kMaskStages);
+        const bool landed = mbar_wait_bounded(smem_addr(&full[st]), (uint32_t)((i / kMaskStages) & 1));
+        if (landed) {
+            const int64_t v0 = (worker + i * nworkers) * (int64_t)p.chunk;
+            const int nv = (int)min((int64_t)p.chunk, p.nwork - v0);
+            const uint4 *sa = reinterpret_cast<const uint4 *>(stages + (size_t)st * 2 * kMaskChunkMax * 16);
+            const uint4 *sb = sa + kMaskChunkMax;
+#pragma unroll 4
+            for (int j = threadIdx.x; j < nv; j += blockDim.x) {
+                const uint4 a = sa[j], b = sb[j];
+                if ((a.x ^ b.x) | (a.y ^ b.y) | (a.z ^ b.z) | (a.w ^ b.w)) {
+                    const uint32_t bits = diff_bits16(a, b, p.dtype, p.thr);
+                    if (bits) {
+                        mark_bits(sp, sp.sc, v0 + j, bits);
+                        wrote = true;
+                    }
                 }
             }
         }
+        // every thread is done with the stage before it is refilled
+        if (!__syncthreads_and(landed)) {
+            *ok = false;
+            break;
+        }
+        if (threadIdx.x == 0 && i + kMaskStages < mine)
+            issue_chunk(p, stages, full, worker, nworkers, i + kMaskStages);
+    }
+    if (!*ok && threadIdx.x == 0) {
+        // no copy may still be writing this CTA's shared memory when it exits
+        for (int64_t k = i; k < min(mine, i + kMaskStages); ++k)
+            mbar_wait_bounded(smem_addr(&full[k % kMaskStages]), (uint32_t)((k / kMaskStages) & 1));
     }
     return wrote;
 }
@@ -360,10 +453,11 @@ __device__ __forceinline__ void scale_small(const MaskParams &p, const ScalePara
 
 // commit = false: the same work with every global store left out (the warm-up
 // pass of CTA 0, which may read flags that other CTAs are still writing).
-__device__ __noinline__ void phase2(const MaskParams &p, const ScaleParams *sc, bool commit)
+// sbits, sdil: kMaxWords words each of shared memory (CTA 0 streams nothing, so
+// its dynamic shared memory is free for them).
+__device__ __noinline__ void phase2(const MaskParams &p, const ScaleParams *sc, bool commit, uint32_t *sbits,
+                                   uint32_t *sdil)
 {
-    __shared__ __align__(16) uint32_t sbits[kMaxWords];    // raw tile bits
-    __shared__ __align__(16) uint32_t sdil[kMaxWords];     // dilated tile bits
     __shared__ int warp_sums[33];
     bool small = p.dilate < 32;
     for (int s = 0; s < p.n_scales; ++s)
@@ -391,13 +485,13 @@ __device__ __noinline__ void phase2(const MaskParams &p, const ScaleParams *sc, 
             // ballot per bit word
             const int nt = q.th * q.tw;
             uint8_t *sflag = reinterpret_cast<uint8_t *>(sdil);   // free until the dilation pass
-            if (nt <= (int)sizeof(sdil)) {
+            if (nt <= (int)(kMaxWords * sizeof(uint32_t))) {
 #pragma unroll 1
                 for (int t = threadIdx.x * 16; t < nt; t += blockDim.x * 16)
                     *reinterpret_cast<uint4 *>(sflag + t) = __ldcg(reinterpret_cast<const uint4 *>(g + t));
                 __syncthreads();
             }
-            const bool in_smem = nt <= (int)sizeof(sdil);
+            const bool in_smem = nt <= (int)(kMaxWords * sizeof(uint32_t));
 #pragma unroll 1
             for (int wi = warp; wi < nw; wi += nwarps) {
                 const int i = wi / wpr, j = (wi - i * wpr) * 32 + lane;
@@ -502,16 +596,27 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *ptr)
 
 __global__ void __launch_bounds__(kMaskThreads) k_mask_reduce(const __grid_constant__ MaskParams p)
 {
+    extern __shared__ __align__(128) uint8_t dyn[];
     __shared__ MaskParams s_p;
+    __shared__ __align__(8) uint64_t full[kMaskStages];
     __shared__ int s_go;
-    if (threadIdx.x == 0)
-        s_p = p;
     pdl_trigger();
     pdl_wait();   // the inputs, lists and workspace may come from the kernel before
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kMaskStages; ++i)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&full[i])));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (blockIdx.x != 0 && p.mode != 2)
+            issue_first_chunks(p, dyn, full, blockIdx.x - 1, gridDim.x - 1);
+    }
+    if (threadIdx.x < 32)
+        copy_params(&s_p, p);
     __syncthreads();
     const ScaleParams *s_sc = s_p.sc;
     if (blockIdx.x == 0) {
-        phase2(s_p, s_sc, false);
+        uint32_t *sbits = reinterpret_cast<uint32_t *>(dyn);
+        uint32_t *sdil = sbits + kMaxWords;
+        phase2(s_p, s_sc, false, sbits, sdil);
         if (threadIdx.x == 0) {
             const uint32_t want = gridDim.x - 1;
             const long long t0 = clock64();
@@ -528,14 +633,24 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask_reduce(const __grid_const
         }
         __syncthreads();
         if (s_go)
-            phase2(s_p, s_sc, true);
+            phase2(s_p, s_sc, true, sbits, sdil);
         return;
     }
-    if (phase1(p, s_p, blockIdx.x - 1, gridDim.x - 1))
-        __threadfence();   // flags stored by this thread are visible before the arrival below
-    __syncthreads();
-    if (threadIdx.x == 0)
+    bool wrote, ok = true;
+    if (p.mode == 2)
+        wrote = scalar_pass(s_p, s_sc, blockIdx.x - 1, gridDim.x - 1);
+    else
+        wrote = phase1_bulk(p, s_p, dyn, full, blockIdx.x - 1, gridDim.x - 1, &ok);
+    if (!ok && threadIdx.x == 0)
+        record_error(p.hdr, SIGE_ERR_TIMEOUT, -2);
+    // The barrier orders every thread's flag stores before thread 0's fence,
+    // and the fence (cumulative) makes them visible before the arrival.
+    const bool any = __syncthreads_or(wrote);
+    if (threadIdx.x == 0) {
+        if (any)
+            __threadfence();
         atomicAdd(&p.hdr->arrive, 1u);
+    }
 }
 
 // ------------------------------------------------------------------ host
@@ -662,23 +777,35 @@ extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const si
     p.log_w = log2_exact(in->w);
     p.log_epv = log2_exact(p.epv);
     p.pow2 = p.log_vpp >= 0 && p.log_w >= 0 && log2_exact(in->h) >= 0;
-    static int occ[64] = {0};
+    // CTA 0 reduces; the others stream the inputs, one per SM
+    const int workers_max = std::max(1, device_sm_count() - 1);
+    int grid;
+    size_t smem;
+    if (p.mode == 2) {
+        grid = 1 + (int)std::min<int64_t>((p.nwork + kMaskThreads * kScalarPerThread - 1) / (kMaskThreads * kScalarPerThread), workers_max);
+        smem = 2 * kMaxWords * sizeof(uint32_t);
+    } else {
+        // chunks of 256..1024 vectors, about four per streaming CTA
+        int64_t chunk = (p.nwork / ((int64_t)workers_max * 4) + 255) / 256 * 256;
+        chunk = std::max<int64_t>(256, std::min<int64_t>(kMaskChunkMax, chunk));
+        p.chunk = (int32_t)chunk;
+        const int64_t nchunks = (p.nwork + chunk - 1) / chunk;
+        grid = 1 + (int)std::min<int64_t>(nchunks, workers_max);
+        p.chunks_base = (int32_t)(nchunks / (grid - 1));
+        p.chunks_rem = (int32_t)(nchunks % (grid - 1));
+        smem = std::max(kMaskStreamSmem, 2 * kMaxWords * sizeof(uint32_t));
+    }
+    static int attr_done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64)
-        dev = 0;
-    if (!occ[dev]) {
-        int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_mask_reduce, kMaskThreads, 0) != cudaSuccess || n < 1)
-            n = 1;
-        occ[dev] = n;
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(k_mask_reduce, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaskStreamSmem) !=
+            cudaSuccess)
+            return SIGE_ERR_CUDA;
+        attr_done[dev] = 1;
     }
-    // CTA 0 reduces; the others stream the inputs
-    int64_t per_cta = (int64_t)kMaskThreads * kMaskUnroll;
-    int grid = 1 + (int)std::min<int64_t>((p.nwork + per_cta - 1) / per_cta,
-                                          std::max<int64_t>(1, (int64_t)device_sm_count() * occ[dev] - 1));
     prefer_max_shared(k_mask_reduce);
-    const cudaError_t e = launch_pdl(k_mask_reduce, dim3(grid), dim3(kMaskThreads), 0, (cudaStream_t)stream, p);
+    const cudaError_t e = launch_pdl(k_mask_reduce, dim3(grid), dim3(kMaskThreads), smem, (cudaStream_t)stream, p);
     count_launch();
     if (e != cudaSuccess)
         return SIGE_ERR_CUDA;

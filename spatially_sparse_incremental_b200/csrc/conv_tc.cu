@@ -54,6 +54,7 @@ constexpr long long kWaitCycles = 1ll << 31;   // ~1.1 s at 1.9 GHz
 constexpr int kSmemLimit = 232448;             // 227 KB opt-in per CTA
 constexpr int kMaxSA = 16;                     // weight stages at most
 constexpr uint32_t kCtrlBytes = 4096;          // barriers, flags, tile origins
+constexpr uint32_t kRedBytes = 64 * 128 * 4;   // split-K partial of one unit received from the cluster peer
 
 // Flat argument block.  The kernel copies it into a local at entry: fields of
 // a kernel parameter read through a reference (non-inlined helpers, or after an
@@ -87,6 +88,8 @@ struct TcArgs {
     int32_t ncols;            // tensor-memory columns allocated (power of 2)
     int32_t num_sms;
     int32_t halo_tma;         // 1: ROW-mode halo rows come by TMA (tmx), 0: per-thread cp.async
+    int32_t pair;             // 1: launched in clusters of two CTAs; a 2-way K split of a unit
+                              // of <= 64 columns is summed through the peer's shared memory
 };
 
 __device__ __forceinline__ void tile_origin_a(const TcArgs &a, int t, int &h0, int &w0)
@@ -189,6 +192,67 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+
+// Cluster helpers (pair launches).
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_peer(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void st_peer_f32(uint32_t addr, float v)
+{
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+// Arrive on an mbarrier of the peer; orders this thread's (and, through a
+// preceding CTA barrier, the CTA's) earlier writes before the arrival.
+__device__ __forceinline__ void mbar_arrive_peer(uint32_t addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                                  WsHeader *hdr, int where)
+{
+    if (mbar_try_cluster(bar, parity))
+        return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_cluster(bar, parity))
+            return true;
+        if (*abort_flag)
+            return false;
+        if (clock64() - t0 > kWaitCycles) {
+            *abort_flag = 1;
+            record_error(hdr, SIGE_ERR_TIMEOUT, where);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 // Warp-wide forms.  The whole converged warp calls them with identical
 // arguments and one lane, chosen by elect.sync, issues the instruction.  The
@@ -302,9 +366,9 @@ __device__ __forceinline__ Unit decode_unit(const TcArgs &p, const Sched &s, int
     const int tm = u / s.S;
     r.mt = tm % p.MT;
     r.tb = tm / p.MT;
-    const int KC = p.taps * p.kci;
-    r.kb = (int)((long long)r.split * KC / s.S);
-    r.ke = (int)((long long)(r.split + 1) * KC / s.S);
+    const int KC = p.taps * p.kci;   // small: 32-bit products
+    r.kb = r.split * KC / s.S;
+    r.ke = (r.split + 1) * KC / s.S;
     return r;
 }
 
@@ -313,13 +377,23 @@ __device__ __forceinline__ Unit decode_unit(const TcArgs &p, const Sched &s, int
 //   [0, 1024)        mbarriers and control words
 //   [1024, 3072)     tile origins of the current unit (256 x int2)
 //   [4096, ...)      weight stages, 16 KB each, as many as fit (<= 16)
-//   [.., end)        SB halo stages of T slots each; reused as the epilogue's
+//   [.., b_base)     pair launches only: the 32 KB receive buffer of the split-K
+//                    partial sent by the cluster peer
+//   [b_base, end)    SB halo stages of T slots each; reused as the epilogue's
 //                    staging buffer once the unit's MMAs are complete
+
+// Accumulator columns of a unit of T tiles (ROW) or T slots (POS).
+__device__ __forceinline__ int unit_cols(const TcArgs &p, int T)
+{
+    return p.mode == 0 ? T * 64 : p.b * p.b * T;
+}
 
 struct Carve {
     uint32_t a_base;    // byte offset of weight stage 0
     uint32_t b_base;    // byte offset of halo stage 0
     uint32_t stage_b;   // bytes per halo stage
+    uint32_t red_base;  // receive buffer of the peer's partial (kRedBytes), when red
+    bool red;           // pair launch, unit of <= 64 columns, and two weight stages still fit
     int SA;             // weight stages
 };
 
@@ -329,7 +403,16 @@ __device__ __forceinline__ Carve carve(const TcArgs &p, int T)
     c.stage_b = (uint32_t)T * p.per_slot;
     c.b_base = (p.smem_bytes - 1024 - p.SB * c.stage_b) & ~15u;
     c.a_base = kCtrlBytes;
-    c.SA = min(kMaxSA, (int)((c.b_base - c.a_base) / kAStageBytes));
+    c.red_base = c.b_base;
+    c.red = false;
+    if (p.pair && unit_cols(p, T) * 512 <= (int)kRedBytes && c.b_base >= kRedBytes + 1024) {
+        const uint32_t rb = (c.b_base - kRedBytes) & ~1023u;
+        if (rb >= c.a_base + 2 * kAStageBytes) {
+            c.red_base = rb;
+            c.red = true;
+        }
+    }
+    c.SA = min(kMaxSA, (int)((c.red_base - c.a_base) / kAStageBytes));
     return c;
 }
 
@@ -439,10 +522,24 @@ __device__ __forceinline__ void fill_b(const TcArgs &c, int T, int tb, int q, in
     }
 }
 
+// GroupNorm scale / shift of this thread's 8 channels of chunk q (batch 1);
+// loaded before the halo wait so that their latency overlaps the copy.
+__device__ __forceinline__ void load_gn8(const TcArgs &c, int q, int et, float (&gsc)[8], float (&gsh)[8])
+{
+    const int ch = q * 64 + (et & 7) * 8;
+    const bool affine = c.gsc != nullptr && c.N == 1;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        gsc[k] = affine ? __ldg(c.gsc + ch + k) : 1.0f;
+        gsh[k] = affine ? __ldg(c.gsh + ch + k) : 0.0f;
+    }
+}
+
 // In-place GroupNorm affine + SiLU of a B stage whose raw halo arrived by TMA
-// (zero-filled outside the image); padding entries are left at zero.
+// (zero-filled outside the image); padding entries are left at zero.  gsc /
+// gsh come from load_gn8 (batch 1; larger batches read theirs per tile).
 __device__ __forceinline__ void transform_b(const TcArgs &c, int T, int tb, int q, int G, uint8_t *stage, int et,
-                                            const int2 *s_orig)
+                                            const int2 *s_orig, const float (&gsc)[8], const float (&gsh)[8])
 {
     if (c.gsc == nullptr && !c.silu)
         return;
@@ -450,12 +547,6 @@ __device__ __forceinline__ void transform_b(const TcArgs &c, int T, int tb, int 
     const int kc = et & 7;
     const int ch = q * 64 + kc * 8;
     const bool affine = c.gsc != nullptr;
-    float gsc[8], gsh[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        gsc[k] = affine && c.N == 1 ? __ldg(c.gsc + ch + k) : 1.0f;
-        gsh[k] = affine && c.N == 1 ? __ldg(c.gsh + ch + k) : 0.0f;
-    }
     const int lin0 = et >> 3;
     int slot = lin0 / bin2, pix = lin0 - slot * bin2;
     int hh = pix / bin, ww = pix - hh * bin;
@@ -484,10 +575,6 @@ __device__ __forceinline__ void transform_b(const TcArgs &c, int T, int tb, int 
 
 // ------------------------------------------------------------------ epilogue
 
-__device__ __forceinline__ int unit_cols(const TcArgs &p, int T)
-{
-    return p.mode == 0 ? T * 64 : p.b * p.b * T;
-}
 
 // Pixel of accumulator column `col`: returns the flat element index of its
 // first channel `co0` in the destination, or -1 when the column is not a
@@ -560,6 +647,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t acc_empty = acc_full + 8u;
     const uint32_t drain = acc_full + 16u;
     auto b_load = [&](int i) { return acc_full + 24u + 8u * i; };   // halo TMA arrivals
+    const uint32_t red_full = acc_full + 40u;   // pair launches, rank 0: the peer's partial has arrived
+    const uint32_t red_free = acc_full + 48u;   // pair launches, rank 1: the peer has consumed it
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 512);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 516);
     volatile int *bcast = abort_flag + 1;
@@ -581,6 +670,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kProd);
         mbar_init(drain, 1);
+        mbar_init(red_full, 1);
+        mbar_init(red_free, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -598,10 +689,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // the barriers of both CTAs of a pair are initialised before either side's
+    // first remote access (each waits on this cluster barrier before it)
+    bool cwaited = false;
+    if (p.pair)
+        cluster_arrive();
     // everything above touches only this CTA's own resources; the tile list,
     // the activations and the output may come from the kernel before
     pdl_trigger();
     pdl_wait();
+    if (threadIdx.x == 64 && !c.dense) {
+        // the tile origins this CTA reads first, for K split in 1 or 2
+        const int32_t *i0 = c.idx + 2 * min(c.cap - 1, (int)blockIdx.x);
+        const int32_t *i1 = c.idx + 2 * min(c.cap - 1, (int)blockIdx.x / 2);
+        if (c.cap > 0) {
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(i0));
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(i1));
+        }
+    }
 
     const int ntile = c.dense ? c.tiles_total : min(__ldg(c.count), c.cap);
     const int G = ntile * c.N;
@@ -786,6 +891,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             asm volatile("bar.sync 1, 256;" ::: "memory");
             return r;
         };
+        // the same on a barrier that a cluster peer completes (acquire at cluster scope)
+        auto group_wait_c = [&](uint32_t bar, uint32_t parity, int where) -> bool {
+            if (et == 0)
+                *group_ok = mbar_wait_cluster(bar, parity, abort_flag, hdr, where) ? 1 : 0;
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            const bool r = *group_ok != 0;
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            return r;
+        };
+        uint32_t pit = 0;   // pair units done (phase of red_full / red_free)
         // output vectors: 8 bf16 channels (16 per 128-channel column) or 4 floats (32)
         const int vpc = (c.to_y && c.dtype == SIGE_BF16) ? 16 : 32;
         const int cpv = 128 / vpc;          // channels per vector
@@ -838,11 +953,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                                 y0 + hh, n);
                             }
                         }
+                        float gsc[8], gsh[8];
+                        load_gn8(c, q, et, gsc, gsh);
                         if (!group_wait(b_load(sb), (bit / p.SB) & 1, 7)) {
                             ok = false;
                             break;
                         }
-                        transform_b(c, sc.T, un.tb, q, G, stage, et, s_orig);
+                        transform_b(c, sc.T, un.tb, q, G, stage, et, s_orig, gsc, gsh);
                     } else {
                         fill_b(c, sc.T, un.tb, q, G, stage, et, s_orig);
                     }
@@ -862,15 +979,111 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     if (k < cpv)
                         bias8[k] = __ldg(c.bias + co0 + k);
             }
+            const int ncols = unit_cols(p, sc.T);
+            const bool write_ok = co0 < c.Cout;
+            // 2-way K split summed through the cluster peer's shared memory:
+            // rank 1 sends its partial, rank 0 adds it and writes the output
+            const bool pair = cv.red && sc.S == 2;
+            const uint32_t rank = pair ? cluster_rank() : 0u;
+            // rank 0 (or an unsplit unit of one batch of items): the residual of
+            // this thread's items is read while the MMAs run
+            const bool pre = (pair ? rank == 0 : sc.S == 1 && ncols <= stage_cols) && ncols * vpc <= 4 * kProd &&
+                             c.residual && c.to_y;
+            int64_t e_pre[4];
+            uint4 rr_pre[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int it = et + k * kProd;
+                e_pre[k] = (it < ncols * vpc && write_ok) ? col_target(c, s_orig, sc.T, un.tb, G, it / vpc, co0) : -1;
+                rr_pre[k] = make_uint4(0, 0, 0, 0);
+                if (pre && e_pre[k] >= 0)
+                    rr_pre[k] = __ldg(reinterpret_cast<const uint4 *>(c.residual + e_pre[k] * (c.dtype == SIGE_BF16 ? 2 : 4)));
+            }
+            if (pair && !cwaited) {
+                cluster_wait();
+                cwaited = true;
+            }
+            if (pair && rank == 1 && pit > 0 && !group_wait_c(red_free, (pit - 1) & 1, 8)) {
+                ok = false;
+                break;
+            }
             if (!group_wait(acc_full, uit & 1, 6)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const int ncols = unit_cols(p, sc.T);
             const uint32_t tbase = tmem + ((uint32_t)(sub * 32) << 16);
-            const bool write_ok = co0 < c.Cout;
-            if (sc.S == 1) {
+            if (pair && rank == 1) {
+                // partial -> rank 0's receive buffer, [column][128 channels] floats
+                const uint32_t rbuf = map_peer(sbase + cv.red_base, 0);
+#pragma unroll 1
+                for (int c0 = 16 * half; c0 < ncols; c0 += 32) {
+                    float v[16];
+                    tmem_ld16(tbase + c0, v);
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        st_peer_f32(rbuf + (uint32_t)(((c0 + k) * 128 + row) * 4), v[k]);
+                }
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+                if (et == 0)
+                    mbar_arrive_peer(map_peer(red_full, 0));
+                ++pit;
+            } else if (pair) {
+                float *red = reinterpret_cast<float *>(smem + cv.red_base);
+                if (!group_wait_c(red_full, pit & 1, 9)) {
+                    ok = false;
+                    break;
+                }
+                // own partial added in place (two terms: the order does not change the sum)
+#pragma unroll 1
+                for (int c0 = 16 * half; c0 < ncols; c0 += 32) {
+                    float v[16];
+                    tmem_ld16(tbase + c0, v);
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        red[(c0 + k) * 128 + row] += v[k];
+                }
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+#pragma unroll 1
+                for (int it0 = et; it0 < ncols * vpc; it0 += 4 * kProd) {
+                    int64_t e[4];
+                    uint4 rr[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int it = it0 + k * kProd;
+                        if (it0 == et) {
+                            e[k] = e_pre[k];
+                            rr[k] = rr_pre[k];
+                        } else {
+                            e[k] = (it < ncols * vpc && write_ok) ? col_target(c, s_orig, sc.T, un.tb, G, it / vpc, co0)
+                                                                  : -1;
+                            rr[k] = make_uint4(0, 0, 0, 0);
+                        }
+                        if (e[k] >= 0 && c.residual && c.to_y && !(pre && it0 == et))
+                            rr[k] = __ldg(reinterpret_cast<const uint4 *>(c.residual + e[k] * (c.dtype == SIGE_BF16 ? 2 : 4)));
+                    }
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        if (e[k] < 0)
+                            continue;
+                        const int col = (it0 + k * kProd) / vpc;
+                        float v[8];
+                        const float4 *src = reinterpret_cast<const float4 *>(red + col * 128 + cg * cpv);
+                        const float4 lo = src[0];
+                        v[0] = lo.x; v[1] = lo.y; v[2] = lo.z; v[3] = lo.w;
+                        if (cpv == 8) {
+                            const float4 hi = src[1];
+                            v[4] = hi.x; v[5] = hi.y; v[6] = hi.z; v[7] = hi.w;
+                        }
+                        store_vec(c, e[k], v, bias8, rr[k]);
+                    }
+                }
+                // the buffer is free for the peer's next partial
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+                if (et == 0)
+                    mbar_arrive_peer(map_peer(red_free, 1));
+                ++pit;
+            } else if (sc.S == 1) {
                 // accumulator -> shared staging (column-major, 128 floats per
                 // column) -> 16-byte vectors per pixel
 #pragma unroll 1
@@ -893,6 +1106,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const int it = it0 + k * kProd;
+                            if (pre) {   // one chunk, one batch: read before the accumulator wait
+                                e[k] = e_pre[k];
+                                rr[k] = rr_pre[k];
+                                continue;
+                            }
                             e[k] = (it < cc_n * vpc && write_ok)
                                        ? col_target(c, s_orig, sc.T, un.tb, G, c0 + it / vpc, co0) : -1;
                             rr[k] = make_uint4(0, 0, 0, 0);
@@ -987,8 +1205,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_arrive(acc_empty);
             ++uit;
         }
+        // rank 1 stays until rank 0 has signalled its last use of the pair
+        // (that arrival writes this CTA's shared memory)
+        if (p.pair && pit > 0 && cluster_rank() == 1)
+            group_wait_c(red_free, (pit - 1) & 1, 10);
     }
 
+    if (p.pair && !cwaited)
+        cluster_wait();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1154,14 +1378,57 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
     p.partials = reinterpret_cast<float *>(ws + ((p.num_sms * 4 + 255) / 256) * 256);
 
     static int smem_set[64] = {0};
+    static int pair_clusters[64] = {0};   // co-resident clusters of two, -1: none
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !smem_set[dev]) {
+    if (dev < 0 || dev >= 64)
+        dev = 0;
+    if (!smem_set[dev]) {
         if (cudaFuncSetAttribute(k_conv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
             return SIGE_ERR_CUDA;
         smem_set[dev] = 1;
     }
-    const cudaError_t e = launch_pdl(k_conv_tc, dim3(p.num_sms), dim3(kTcThreads), kSmemLimit, stream, p, map, xmap);
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = kSmemLimit;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    if (!pair_clusters[dev]) {
+        int n = 0;
+        cfg.gridDim = dim3(2 * ((p.num_sms + 1) / 2));
+        cfg.numAttrs = 2;
+        if (cudaOccupancyMaxActiveClusters(&n, k_conv_tc, &cfg) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = -1;
+        }
+        pair_clusters[dev] = n;
+    }
+    // clusters of two CTAs (a 2-way K split then sums through the peer's
+    // shared memory), as many as are co-resident; otherwise one CTA per SM
+    cudaError_t e = cudaErrorUnknown;
+    if (pair_clusters[dev] > 0) {
+        p.pair = 1;
+        p.num_sms = 2 * std::min(pair_clusters[dev], p.num_sms / 2);
+        cfg.gridDim = dim3(p.num_sms);
+        cfg.numAttrs = 2;
+        e = cudaLaunchKernelEx(&cfg, k_conv_tc, p, map, xmap);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            pair_clusters[dev] = -1;
+        }
+    }
+    if (e != cudaSuccess) {
+        p.pair = 0;
+        p.num_sms = device_sm_count();
+        e = launch_pdl(k_conv_tc, dim3(p.num_sms), dim3(kTcThreads), kSmemLimit, stream, p, map, xmap);
+    }
     count_launch();
     if (e != cudaSuccess)
         return SIGE_ERR_CUDA;

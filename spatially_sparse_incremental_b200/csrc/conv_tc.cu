@@ -137,12 +137,11 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait: false when the limit expired or another role gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag, WsHeader *hdr,
-                                          int where)
+// Bounded wait: false when the limit expired or another role gave up.  The
+// polling loop is out of line so that the callers' loops stay compact.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag, WsHeader *hdr,
+                                            int where)
 {
-    if (mbar_try(bar, parity))
-        return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try(bar, parity))
@@ -155,6 +154,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag, WsHeader *hdr,
+                                          int where)
+{
+    return mbar_try(bar, parity) || mbar_wait_slow(bar, parity, abort_flag, hdr, where);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y)
@@ -232,11 +237,9 @@ __device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                                  WsHeader *hdr, int where)
+__device__ __noinline__ bool mbar_wait_cluster_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                                    WsHeader *hdr, int where)
 {
-    if (mbar_try_cluster(bar, parity))
-        return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_cluster(bar, parity))
@@ -251,7 +254,15 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
     }
 }
 
-__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                                  WsHeader *hdr, int where)
+{
+    return mbar_try_cluster(bar, parity) || mbar_wait_cluster_slow(bar, parity, abort_flag, hdr, where);
+}
+
+// Relaxed: what the peer must see (the mbarrier initialisation) is released by
+// the initialising thread's fence.mbarrier_init before it arrives.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 // Warp-wide forms.  The whole converged warp calls them with identical
@@ -274,6 +285,25 @@ __device__ __forceinline__ void tc_commit_w(uint32_t bar)
     asm volatile(
         "{\n .reg .pred e;\n .reg .b32 l;\n elect.sync l|e, 0xffffffff;\n"
         " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(bar)
+        : "memory");
+}
+
+// The four K=16 steps of one 64-channel k-chunk (A advances 32 bytes per step,
+// B by b_step) and the commit of the chunk's stage, from one elected lane.
+__device__ __forceinline__ void tc_mma4_commit_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint64_t b_step,
+                                                 uint32_t idesc, uint32_t accumulate, uint32_t bar)
+{
+    asm volatile(
+        "{\n .reg .pred p, e, t;\n .reg .b32 l;\n .reg .b64 a1, a2, a3, b1, b2, b3;\n"
+        " elect.sync l|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n setp.eq.b32 t, 0, 0;\n"
+        " add.s64 a1, %1, 2;\n add.s64 a2, %1, 4;\n add.s64 a3, %1, 6;\n"
+        " add.s64 b1, %2, %5;\n add.s64 b2, b1, %5;\n add.s64 b3, b2, %5;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, t;\n"
+        " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "l"(b_step), "r"(bar)
         : "memory");
 }
 
@@ -808,6 +838,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         : desc_plain(sbase + cv.b_base + sb * cv.stage_b, sk, 128);
                     int r = tap / k, cc = tap - r * k;
                     uint64_t b_tap = b_stage + (uint64_t)r * d_row + (uint64_t)cc * d_col;
+                    if (p.mode == 0 && nT == 1) {
+                        // one tile per unit: the whole k-chunk is one issue block
+#pragma unroll 1
+                        for (; tap < tap_end; ++tap, ++kc) {
+                            if (!mbar_wait_w(a_full(sa), pa, abort_flag, hdr, 4)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_mma4_commit_w(tmem, a_cur, b_tap, d_ks, idesc, acc0, a_empty(sa));
+                            acc0 = 1;
+                            ++ait;
+                            if (++sa == cv.SA) {
+                                sa = 0;
+                                pa ^= 1;
+                                a_cur = a_desc0;
+                            } else {
+                                a_cur += kAStageBytes >> 4;
+                            }
+                            if (++cc == k) {
+                                cc = 0;
+                                b_tap += d_row - (uint64_t)k * d_col;
+                            }
+                            b_tap += d_col;
+                        }
+                    } else {
 #pragma unroll 1
                     for (; tap < tap_end; ++tap, ++kc) {
                         if (!mbar_wait_w(a_full(sa), pa, abort_flag, hdr, 4)) {
@@ -851,6 +906,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             b_tap += d_row - (uint64_t)k * d_col;
                         }
                         b_tap += d_col;
+                    }
                     }
                     if (!ok)
                         break;

@@ -151,10 +151,10 @@ def max_over_ranks(vals, device):
 
 # ------------------------------------------------------------------ workload
 
-def make_workload(seed, dev):
+def make_workload(seed, dev, area=0.012):
     import spatially_sparse_incremental_b200 as sige
     from spatially_sparse_incremental_b200 import inputs
-    blk = inputs.make_cfg3(seed, H=H, W=W, C=C, area=0.012, block=BLOCK)
+    blk = inputs.make_cfg3(seed, H=H, W=W, C=C, area=area, block=BLOCK)
     d = {k: getattr(blk, k).to(dev) for k in ("x_orig", "x_edit", "w1", "b1", "w2", "b2", "g1", "be1", "g2", "be2")}
     cd = sige.conv_desc(3, 1, 1, C, C, BLOCK)
     cap = (H // BLOCK) * (W // BLOCK)
@@ -246,6 +246,125 @@ def timed_graph_steps(graphs, flush, steps, stream):
     per = {nm: [ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps)] for i, nm in enumerate(names)}
     tot = [ev[k][0].elapsed_time(ev[k][-1]) for k in range(steps)]
     return per, tot
+
+
+def time_graph(g, flush, reps, stream, warm=False):
+    """Device time (ms) of each replay of graph g, L2 flushed before each
+    replay unless warm."""
+    times = []
+    with torch.cuda.stream(stream):
+        for k in range(reps + 3):
+            if not warm:
+                flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            if k >= 3:
+                times.append((e0, e1))
+    stream.synchronize()
+    return [a.elapsed_time(b) for a, b in times]
+
+
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # FMA lanes x 2 x max SM clock
+
+
+def layer_roofline(macs, nbytes, dtype_bits, peaks, us):
+    """Roofline time of one sparse layer and the fraction reached: tensor (bf16)
+    or FP32 ALU for the arithmetic, measured HBM copy bandwidth for the bytes."""
+    if dtype_bits == 32:
+        t_c, bound_c = 2 * macs / (FP32_ALU_TFLOPS * 1e12), "alu"
+    else:
+        t_c, bound_c = 2 * macs / (peaks["bf16_tflops"] * 1e12), "tensor"
+    t_b = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t = max(t_c, t_b)
+    return {"bound": bound_c if t_c >= t_b else "hbm", "roof_us": t * 1e6, "frac": t / (us * 1e-6)}
+
+
+def measure_extras(dev, flush, stream, peaks, seed, step_graph):
+    """Measurement rows beyond the headline step: warm-L2 step, the edit-area
+    sweep with a linear fit of step latency on active tiles, and one sparse vs
+    dense layer per shape of the other workloads (fp32 64x64x64, the SD-latent
+    and GauGAN-shaped layers) at 1.2% edit."""
+    import spatially_sparse_incremental_b200 as sige
+    from spatially_sparse_incremental_b200 import inputs
+    out = {}
+    warm = time_graph(step_graph, flush, 50, stream, warm=True)
+    out["warm_l2_step_us"] = float(np.median(warm)) * 1e3
+
+    sweep = []
+    for area in (0.005, 0.012, 0.05, 0.10, 0.20):
+        d = make_workload(seed, dev, area=area)
+        torch.cuda.synchronize()   # the workload is built on the default stream
+        calls = step_calls(d, stream)
+        with torch.cuda.stream(stream):
+            calls["mask"]()
+        stream.synchronize()
+        tiles = int(d["cnt"].item())
+
+        def whole():
+            for fn in calls.values():
+                fn()
+        g = capture(whole, stream)
+        t = time_graph(g, flush, 40, stream)
+        sweep.append({"area": area, "active_tiles": tiles, "step_us": float(np.median(t)) * 1e3,
+                      "p90_us": float(np.percentile(t, 90)) * 1e3})
+        del g, d
+    x = np.array([r["active_tiles"] for r in sweep], dtype=np.float64)
+    y = np.array([r["step_us"] for r in sweep], dtype=np.float64)
+    A = np.vstack([x, np.ones_like(x)]).T
+    (slope, icpt), *_ = np.linalg.lstsq(A, y, rcond=None)
+    pred = A @ np.array([slope, icpt])
+    r2 = 1.0 - float(((y - pred) ** 2).sum()) / max(1e-30, float(((y - y.mean()) ** 2).sum()))
+    out["area_sweep"] = {"rows": sweep, "fit": {"slope_us_per_tile": float(slope), "intercept_us": float(icpt),
+                                                "r2": r2}}
+
+    layers = [("fp32 64x64 C64 3x3 b4", inputs.make_cfg1(seed), 32)]
+    for i, (h, w, c, b) in enumerate(inputs.CFG4_LAYERS):
+        layers.append((f"SD latent {h}x{w} C{c} 3x3 b{b}", inputs.make_cfg4_layer(seed, i), 16))
+    for i, (h, w, ci, co, k, st, b) in enumerate(inputs.CFG5_LAYERS):
+        layers.append((f"GauGAN {h}x{w} {ci}->{co} {k}x{k} s{st} b{b}", inputs.make_cfg5_layer(seed, i), 16))
+    rows = []
+    for name, L, bits in layers:
+        try:
+            rows.append(dict(name=name, **layer_timing(L, bits, dev, flush, stream, peaks)))
+        except Exception as e:   # a failing row is reported, not fatal to the headline line
+            rows.append({"name": name, "error": str(e)[:200]})
+    out["layers"] = rows
+    return out
+
+
+def layer_timing(L, bits, dev, flush, stream, peaks):
+    import spatially_sparse_incremental_b200 as sige
+    xo, xe = L.x_orig.to(dev), L.x_edit.to(dev)
+    wt, bias = L.weight.to(dev), L.bias.to(dev)
+    N, Hi, Wi, ci = xo.shape
+    co, k, st, b = wt.shape[0], L.kernel, L.stride, L.block
+    cd = sige.conv_desc(k, st, L.pad, ci, co, b)
+    y0 = sige.sige_dense_conv(xo, wt, bias, cd)
+    Ho, Wo = y0.shape[1], y0.shape[2]
+    cap = -(-Ho // b) * -(-Wo // b)
+    thr = L.meta.get("threshold", 1e-3) if L.meta else 1e-3
+    idx, cnt, _ = sige.sige_reduce_mask(xo, xe, thr, [(Ho, Wo, b, cap)], 1)
+    torch.cuda.synchronize()
+    tiles = int(cnt.item())
+    y = y0.clone()
+    ws = sige.zeros_workspace(sige.sige_conv_workspace_bytes(cd, N, cap, Ho, Wo), dev)
+    yd = torch.empty_like(y0)
+    g_sp = capture(lambda: sige.sige_conv_fused(xe, wt, bias, cd, idx, cnt, cap, y, workspace=ws, stream=stream),
+                   stream)
+    g_de = capture(lambda: sige.sige_dense_conv(xe, wt, bias, cd, y=yd, workspace=ws, stream=stream), stream)
+    t_sp = float(np.median(time_graph(g_sp, flush, 30, stream))) * 1e3
+    t_de = float(np.median(time_graph(g_de, flush, 30, stream))) * 1e3
+    esz = bits // 8
+    bin_ = (b - 1) * st + k
+    macs = tiles * b * b * ci * co * k * k
+    nbytes = tiles * (bin_ * bin_ * ci + b * b * co) * esz + co * k * k * ci * esz + co * 4
+    roof = layer_roofline(macs, nbytes, bits, peaks, t_sp)
+    del g_sp, g_de
+    return {"active_tiles": tiles, "tiles_total": cap, "sparse_us": t_sp, "dense_us": t_de,
+            "speedup": t_de / t_sp, "path": "tcgen05" if sige.sige_conv_path(cd, L.x_orig.dtype) == 1 else "cuda-core",
+            "roofline": roof}
 
 
 # ------------------------------------------------------------------ roofline
@@ -453,6 +572,10 @@ def run_sige(args):
     sparse_conv_ms = kern_ms["conv1"] + kern_ms["conv2"]
     dense_conv_ms = dense_ms["dense1"] + dense_ms["dense2"]
 
+    extras = None
+    if not args.no_extras:
+        extras = measure_extras(dev, flush, stream, peaks, args.seed + rank, step_graph["step"])
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cores = host_cores()
@@ -469,6 +592,7 @@ def run_sige(args):
                    "active_tiles": n_tiles, "tile_fraction": n_tiles / d["cap"],
                    "l2": "cold: 256 MiB write then 256 MiB read (clean lines) before every step, untimed", "launch": "one CUDA graph per step (mask + conv1 + conv2); breakdown_us from one graph per call",
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+        "step_p50_us": float(np.median(tot)) * 1e3, "step_p90_us": float(np.percentile(tot, 90)) * 1e3,
         "breakdown_us": {k: v * 1e3 for k, v in kern_ms.items()},
         "dense_conv_us": dense_conv_ms * 1e3, "sparse_conv_us": sparse_conv_ms * 1e3,
         "speedup_vs_dense_conv": dense_conv_ms / sparse_conv_ms,
@@ -482,6 +606,8 @@ def run_sige(args):
         "clocks": clocks,
         "conv_path": "tcgen05" if sige.sige_conv_path(d["cd"], torch.bfloat16) == 1 else "cuda-core",
     }
+    if extras is not None:
+        line.update(extras)
     if rank == 0:
         print(json.dumps(line), flush=True)
     for g in list(graphs.values()) + list(dgraphs.values()) + list(step_graph.values()):
@@ -505,6 +631,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the area sweep, warm-L2 step and per-layer rows")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

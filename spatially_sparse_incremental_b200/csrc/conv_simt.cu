@@ -2,10 +2,11 @@
 // layers, and for bf16 layers the tensor-core kernel does not cover.
 //
 // One CTA works on one (tile, batch item, group of output channels) unit at a
-// time.  It stages the tile's halo'd input block in shared memory (from the
-// stacked blocks, or straight from the image with zero padding and the
-// GroupNorm affine + SiLU applied on the way in), then each thread accumulates
-// one output channel for a few of the tile's pixels.  The epilogue either
+// time.  Per chunk of input channels it stages the tile's halo'd input block
+// (from the stacked blocks, or straight from the image with zero padding and
+// the GroupNorm affine + SiLU applied on the way in) and the chunk of the
+// group's weights in shared memory, then each thread accumulates one output
+// channel for a few of the tile's pixels.  The epilogue either
 // writes float32 output blocks or scatters bias + residual + one rounding into
 // the cached output.
 #include <algorithm>
@@ -18,16 +19,54 @@ namespace sige {
 constexpr int kSimtThreads = 256;
 constexpr int kSimtMaxQ = 16;
 constexpr int kSimtSmemFloats = 12288;  // 48 KB
+constexpr int kStageBatch = 8;           // loads in flight per thread while staging
+
+// Read-only element load (input activations and weights are never written here).
+__device__ __forceinline__ float ldg_elem(const uint8_t *base, int64_t e, int dtype)
+{
+    if (dtype == SIGE_BF16)
+        return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(base) + e) << 16);
+    return __ldg(reinterpret_cast<const float *>(base) + e);
+}
+
+// acc[q] += sum over taps and the chunk's channels of w * x, for the NQ pixels
+// of this thread (NQ a compile-time count so no lane issues idle FMAs).
+template <int NQ>
+__device__ __forceinline__ void accumulate(float (&acc)[kSimtMaxQ], const int (&pix0)[kSimtMaxQ], const float *sm,
+                                           const float *sw, int wst, int ol, int cc, int k, int bin)
+{
+#pragma unroll 1
+    for (int r = 0; r < k; ++r)
+#pragma unroll 1
+        for (int c = 0; c < k; ++c) {
+            const float *wrow = sw + (r * k + c) * cc * wst + ol;
+            const float *xs[NQ];
+#pragma unroll
+            for (int q = 0; q < NQ; ++q)
+                xs[q] = sm + (pix0[q] + r * bin + c) * cc;
+#pragma unroll 4
+            for (int ci = 0; ci < cc; ++ci) {
+                const float wv = wrow[ci * wst];
+#pragma unroll
+                for (int q = 0; q < NQ; ++q)
+                    acc[q] = fmaf(wv, xs[q][ci], acc[q]);
+            }
+        }
+}
 
 __global__ void __launch_bounds__(kSimtThreads) k_conv_simt(const __grid_constant__ ConvParams p)
 {
     extern __shared__ float sm[];
+    float *sw = sm + p.bin * p.bin * p.ci_chunk;   // weights [tap][ci][cob + 1]
+    const int wst = p.cob + 1;
+    const int taps = p.k * p.k;
     const int ntiles = p.dense ? p.tiles_total : min(__ldg(p.count), p.cap);
     const int ncog = (p.Cout + p.cob - 1) / p.cob;
     const int units = ntiles * p.N * ncog;
     const int npx = p.b * p.b;
     const int ol = threadIdx.x % p.cob, pgi = threadIdx.x / p.cob;
-    const int esz = p.dtype == SIGE_BF16 ? 2 : 4;
+    const int nq = pgi < npx ? (npx - pgi + p.pg - 1) / p.pg : 0;   // this thread's pixels
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
     const bool xform = p.gsc != nullptr || p.silu;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
         const int cog = u % ncog;
@@ -38,52 +77,123 @@ __global__ void __launch_bounds__(kSimtThreads) k_conv_simt(const __grid_constan
             tile_origin(p, t, h0, w0);
         const int o = cog * p.cob + ol;
         float acc[kSimtMaxQ];
+        int pix0[kSimtMaxQ];   // halo pixel of output pixel q at tap (0, 0)
 #pragma unroll
-        for (int q = 0; q < kSimtMaxQ; ++q)
+        for (int q = 0; q < kSimtMaxQ; ++q) {
             acc[q] = 0.0f;
+            const int pp = min(pgi + p.pg * q, npx - 1);
+            pix0[q] = (pp / p.b) * p.s * p.bin + (pp % p.b) * p.s;
+        }
         for (int ci0 = 0; ci0 < p.Cin; ci0 += p.ci_chunk) {
             const int cc = min(p.ci_chunk, p.Cin - ci0);
             __syncthreads();
-            for (int e = threadIdx.x; e < p.bin * p.bin * cc; e += blockDim.x) {
-                const int pix = e / cc, ci = e % cc;
-                const int hh = pix / p.bin, ww = pix % p.bin;
-                float v = 0.0f;
-                if (p.from_image) {
-                    const int y = h0 * p.s - p.pad + hh, x = w0 * p.s - p.pad + ww;
-                    if (y >= 0 && y < p.H && x >= 0 && x < p.W) {
-                        v = load_elem(p.src, (((int64_t)n * p.H + y) * p.W + x) * p.Cin + ci0 + ci, p.dtype);
-                        if (xform) {
-                            v = transform1(v, p.gsc ? p.gsc + (int64_t)n * p.Cin : nullptr,
-                                           p.gsc ? p.gsh + (int64_t)n * p.Cin : nullptr, ci0 + ci, p.silu);
-                            if (p.dtype == SIGE_BF16)
-                                v = __bfloat162float(__float2bfloat16_rn(v));
+            // Staging: a warp takes a row (one halo pixel, or one (output
+            // channel, tap) of the weights) and its lanes the row's channels, so
+            // the index arithmetic is per row; each lane issues up to
+            // kStageBatch loads before it stores them.
+            const int npix = p.bin * p.bin;
+#pragma unroll 1
+            for (int r0 = warp; r0 < npix; r0 += nwarp * kStageBatch) {
+                float v[kStageBatch];
+#pragma unroll
+                for (int k = 0; k < kStageBatch; ++k) {
+                    v[k] = 0.0f;
+                    const int pix = r0 + k * nwarp;
+                    if (pix >= npix || lane >= cc)
+                        continue;
+                    const int hh = pix / p.bin, ww = pix - hh * p.bin;
+                    if (p.from_image) {
+                        const int y = h0 * p.s - p.pad + hh, x = w0 * p.s - p.pad + ww;
+                        if (y >= 0 && y < p.H && x >= 0 && x < p.W) {
+                            float xv = ldg_elem(p.src, (((int64_t)n * p.H + y) * p.W + x) * p.Cin + ci0 + lane, p.dtype);
+                            if (xform) {   // padding stays zero
+                                xv = transform1(xv, p.gsc ? p.gsc + (int64_t)n * p.Cin : nullptr,
+                                                p.gsc ? p.gsh + (int64_t)n * p.Cin : nullptr, ci0 + lane, p.silu);
+                                if (p.dtype == SIGE_BF16)
+                                    xv = __bfloat162float(__float2bfloat16_rn(xv));
+                            }
+                            v[k] = xv;
                         }
+                    } else {
+                        v[k] = ldg_elem(p.src, (((int64_t)t * p.N + n) * npix + pix) * p.Cin + ci0 + lane, p.dtype);
                     }
-                } else {
-                    v = load_elem(p.src, (((int64_t)t * p.N + n) * p.bin * p.bin + pix) * p.Cin + ci0 + ci, p.dtype);
                 }
-                sm[pix * cc + ci] = v;
+#pragma unroll
+                for (int k = 0; k < kStageBatch; ++k) {
+                    const int pix = r0 + k * nwarp;
+                    if (pix < npix && lane < cc)
+                        sm[pix * cc + lane] = v[k];
+                }
+            }
+            // chunks of more than 32 channels: the remaining lanes' share
+#pragma unroll 1
+            for (int e = 32; e < cc; e += 32)
+#pragma unroll 1
+                for (int pix = warp; pix < npix; pix += nwarp) {
+                    const int ci = e + lane;
+                    if (ci >= cc)
+                        continue;
+                    const int hh = pix / p.bin, ww = pix - hh * p.bin;
+                    float xv = 0.0f;
+                    if (p.from_image) {
+                        const int y = h0 * p.s - p.pad + hh, x = w0 * p.s - p.pad + ww;
+                        if (y >= 0 && y < p.H && x >= 0 && x < p.W) {
+                            xv = ldg_elem(p.src, (((int64_t)n * p.H + y) * p.W + x) * p.Cin + ci0 + ci, p.dtype);
+                            if (xform) {
+                                xv = transform1(xv, p.gsc ? p.gsc + (int64_t)n * p.Cin : nullptr,
+                                                p.gsc ? p.gsh + (int64_t)n * p.Cin : nullptr, ci0 + ci, p.silu);
+                                if (p.dtype == SIGE_BF16)
+                                    xv = __bfloat162float(__float2bfloat16_rn(xv));
+                            }
+                        }
+                    } else {
+                        xv = ldg_elem(p.src, (((int64_t)t * p.N + n) * npix + pix) * p.Cin + ci0 + ci, p.dtype);
+                    }
+                    sm[pix * cc + ci] = xv;
+                }
+            // weights of this channel group and chunk: row (output channel, tap)
+            // is contiguous over input channels in [C_out][k][k][C_in]
+            const int nrow = p.cob * taps;
+#pragma unroll 1
+            for (int r0 = warp; r0 < nrow; r0 += nwarp * kStageBatch) {
+#pragma unroll 1
+                for (int e = 0; e < cc; e += 32) {
+                    const int ci = e + lane;
+                    float v[kStageBatch];
+#pragma unroll
+                    for (int k = 0; k < kStageBatch; ++k) {
+                        v[k] = 0.0f;
+                        const int row = r0 + k * nwarp;
+                        if (row >= nrow || ci >= cc)
+                            continue;
+                        const int ol2 = row / taps, tap = row - ol2 * taps;
+                        const int o2 = cog * p.cob + ol2;
+                        if (o2 < p.Cout)
+                            v[k] = ldg_elem(p.w, ((int64_t)o2 * taps + tap) * p.Cin + ci0 + ci, p.dtype);
+                    }
+#pragma unroll
+                    for (int k = 0; k < kStageBatch; ++k) {
+                        const int row = r0 + k * nwarp;
+                        if (row >= nrow || ci >= cc)
+                            continue;
+                        const int ol2 = row / taps, tap = row - ol2 * taps;
+                        sw[(tap * cc + ci) * wst + ol2] = v[k];
+                    }
+                }
             }
             __syncthreads();
             if (o < p.Cout) {
-                for (int r = 0; r < p.k; ++r)
-                    for (int c = 0; c < p.k; ++c) {
-                        const int64_t wrow = (((int64_t)o * p.k + r) * p.k + c) * p.Cin + ci0;
-                        for (int ci = 0; ci < cc; ++ci) {
-                            const float wv = load_elem(p.w, wrow + ci, p.dtype);
-#pragma unroll
-                            for (int q = 0; q < kSimtMaxQ; ++q) {
-                                const int pp = pgi + p.pg * q;
-                                if (pp < npx) {
-                                    const int i = pp / p.b, j = pp % p.b;
-                                    acc[q] = fmaf(wv, sm[((i * p.s + r) * p.bin + j * p.s + c) * cc + ci], acc[q]);
-                                }
-                            }
-                        }
-                    }
+                // a power of two at least nq: the extra accumulators read a valid
+                // (clamped) pixel and are never stored
+                switch (nq <= 1 ? 1 : nq <= 2 ? 2 : nq <= 4 ? 4 : nq <= 8 ? 8 : 16) {
+                case 16: accumulate<16>(acc, pix0, sm, sw, wst, ol, cc, p.k, p.bin); break;
+                case 8: accumulate<8>(acc, pix0, sm, sw, wst, ol, cc, p.k, p.bin); break;
+                case 4: accumulate<4>(acc, pix0, sm, sw, wst, ol, cc, p.k, p.bin); break;
+                case 2: accumulate<2>(acc, pix0, sm, sw, wst, ol, cc, p.k, p.bin); break;
+                default: accumulate<1>(acc, pix0, sm, sw, wst, ol, cc, p.k, p.bin); break;
+                }
             }
         }
-        (void)esz;
         if (o < p.Cout) {
 #pragma unroll
             for (int q = 0; q < kSimtMaxQ; ++q) {
@@ -121,10 +231,12 @@ int launch_conv_simt(ConvParams p, cudaStream_t stream)
     p.pg = pg;
     p.cob = kSimtThreads / pg;
     const int bin2 = p.bin * p.bin;
-    p.ci_chunk = std::min(p.Cin, std::max(1, kSimtSmemFloats / bin2));
+    // per input channel of a chunk: its halo block and the group's weights
+    const int per_ci = bin2 + p.k * p.k * (p.cob + 1);
+    p.ci_chunk = std::min(p.Cin, kSimtSmemFloats / per_ci);
     if (p.ci_chunk < 1)
         return SIGE_ERR_UNSUPPORTED;
-    const size_t smem = (size_t)bin2 * p.ci_chunk * sizeof(float);
+    const size_t smem = (size_t)per_ci * p.ci_chunk * sizeof(float);
     if (smem > 48 * 1024)
         return SIGE_ERR_UNSUPPORTED;
     const int ncog = (p.Cout + p.cob - 1) / p.cob;

@@ -965,13 +965,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int stage_cols = min(512, (int)((p.SB * cv.stage_b) / 512) & ~15);
         uint32_t bit = 0, uit = 0;
         bool ok = true;
+        // one TMA per tile: the whole halo [hh][kc][ww][8 channels], zero outside
+        // the image (issued by thread et 0 once the origins are in s_orig)
+        auto issue_halo = [&](int sb, int q, int tb) {
+            const uint32_t bl = b_load(sb);
+            mbar_expect_tx(bl, (uint32_t)(sc.T * c.bin) * c.bin * 128u);
+            const uint32_t st = smem_u32(smem + cv.b_base + sb * cv.stage_b);
+#pragma unroll 1
+            for (int slot = 0; slot < sc.T; ++slot) {
+                const int g = tb * sc.T + slot;
+                const int gg = g < G ? g : G - 1;   // past the list: any valid tile, unused
+                const int2 o = s_orig[slot];
+                const int x1 = c.from_image ? o.y * c.s - c.pad : 0;
+                const int y0 = c.from_image ? o.x * c.s - c.pad : 0;
+                const int n = c.from_image ? gg % c.N : gg;
+                tma_load_5d(st + b_offset(c, sc.T, slot, 0, 0, 0), &tmx, bl, 0, x1, q * 8, y0, n);
+            }
+        };
 #pragma unroll 1
         for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
             const Unit un = decode_unit(p, sc, u);
+            // First unit of one tile: thread et 0 reads the origin and starts the
+            // halo copy at once (its stage has never been used, so it is free).
+            const bool early = uit == 0 && p.halo_tma && sc.T == 1;
+            if (early && et == 0) {
+                int h0 = 0, w0 = 0;
+                if (un.tb < G && (c.from_image || c.to_y))
+                    tile_origin_a(c, un.tb / c.N, h0, w0);
+                s_orig[0] = make_int2(h0, w0);
+                issue_halo(bit % p.SB, un.kb / p.taps, un.tb);
+            }
             // the previous unit's epilogue may still be reading the origins
             asm volatile("bar.sync 1, 256;" ::: "memory");
 #pragma unroll 1
-            for (int slot = et; slot < sc.T; slot += kProd) {
+            for (int slot = et; slot < sc.T && !early; slot += kProd) {
                 const int g = un.tb * sc.T + slot;
                 int h0 = 0, w0 = 0;
                 if (g < G && (c.from_image || c.to_y))
@@ -984,31 +1011,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int q = kc / p.taps, tap = kc - q * p.taps;
                 if (kc == un.kb || tap == 0) {
                     const int sb = bit % p.SB;
-                    if (!group_wait(b_empty(sb), ((bit / p.SB) & 1) ^ 1, 5)) {
+                    const bool issued = early && kc == un.kb;
+                    if (!issued && !group_wait(b_empty(sb), ((bit / p.SB) & 1) ^ 1, 5)) {
                         ok = false;
                         break;
                     }
                     uint8_t *stage = smem + cv.b_base + sb * cv.stage_b;
                     if (p.halo_tma) {
-                        // one TMA per (tile, halo row): [kc][ww][8 channels], zero outside the image
-                        if (et == 0) {
-                            const uint32_t bl = b_load(sb);
-                            mbar_expect_tx(bl, (uint32_t)(sc.T * c.bin) * c.bin * 128u);
-                            const uint32_t st = smem_u32(stage);
-#pragma unroll 1
-                            for (int slot = 0; slot < sc.T; ++slot) {
-                                const int g = un.tb * sc.T + slot;
-                                const int gg = g < G ? g : G - 1;   // past the list: any valid tile, unused
-                                const int2 o = s_orig[slot];
-                                const int x1 = c.from_image ? o.y * c.s - c.pad : 0;
-                                const int y0 = c.from_image ? o.x * c.s - c.pad : 0;
-                                const int n = c.from_image ? gg % c.N : gg;
-#pragma unroll 1
-                                for (int hh = 0; hh < c.bin; ++hh)
-                                    tma_load_5d(st + b_offset(c, sc.T, slot, hh, 0, 0), &tmx, bl, 0, x1, q * 8,
-                                                y0 + hh, n);
-                            }
-                        }
+                        if (et == 0 && !issued)
+                            issue_halo(sb, q, un.tb);
                         float gsc[8], gsh[8];
                         load_gn8(c, q, et, gsc, gsh);
                         if (!group_wait(b_load(sb), (bit / p.SB) & 1, 7)) {
@@ -1385,9 +1396,9 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
     if (r != CUDA_SUCCESS)
         return SIGE_ERR_CUDA;
 
-    // ROW mode: one TMA per (tile, halo row) from a 5-d view of the source
+    // ROW mode: one TMA per tile from a 5-d view of the source
     // [n][y][x][c/8][8] (image) or [g][hh][ww][c/8][8] (stacked blocks),
-    // box (8 channels, b_in pixels, 8 channel groups), zero outside.
+    // box (8 channels, b_in pixels, 8 channel groups, b_in rows), zero outside.
     CUtensorMap xmap = map;
     int halo_tma = 0;
     if (pl.mode == 0) {
@@ -1401,7 +1412,7 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
             xd[0] = 8; xd[1] = bin; xd[2] = C / 8; xd[3] = bin; xd[4] = (cuuint64_t)std::max(1, cp.cap) * cp.N;
             xs[0] = C * 2; xs[1] = 16; xs[2] = bin * C * 2; xs[3] = bin * bin * C * 2;
         }
-        cuuint32_t xbox[5] = {8, (cuuint32_t)cp.bin, 8, 1, 1};
+        cuuint32_t xbox[5] = {8, (cuuint32_t)cp.bin, 8, (cuuint32_t)cp.bin, 1};
         cuuint32_t xes[5] = {1, 1, 1, 1, 1};
         if (encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<uint8_t *>(cp.src), xd, xs, xbox, xes,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,

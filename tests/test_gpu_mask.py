@@ -145,3 +145,14 @@ def test_wide_grids_multiword_rows(orc):
         ref = orc.reduce_mask(a, e, 1e-3, sc, D)
         got, cnt, _ = _gpu_lists(a, e, 1e-3, _full_caps(sc), D)
         assert cnt[0] == len(ref[0]) and np.array_equal(got[0], ref[0]), (H, W, b, D)
+
+
+@pytest.mark.parametrize("area", [0.10, 0.20, 0.30, 0.50])
+def test_cfg3_large_edits(orc, area):
+    # large edits: many chunks hold nothing but differing vectors
+    blk = inputs.make_cfg3(0, H=256, W=256, C=128, area=area, block=8)
+    sc = [(256, 256, 8)]
+    ref = orc.reduce_mask(blk.x_orig, blk.x_edit, 1e-3, sc, 1)
+    got, cnt, ws = _gpu_lists(blk.x_orig, blk.x_edit, 1e-3, _full_caps(sc))
+    assert sige.sige_get_error(ws) == sige.OK
+    assert cnt[0] == len(ref[0]) and np.array_equal(got[0], ref[0])

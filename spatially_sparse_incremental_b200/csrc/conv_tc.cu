@@ -78,7 +78,7 @@ struct TcArgs {
     int32_t cap, dense, tiles_w, tiles_total;
     int32_t silu, from_image, to_y;
     // schedule / shared-memory plan
-    int32_t mode;             // 0 = ROW, 1 = POS
+    int32_t mode;             // 0 = ROW, 1 = POS, 2 = POS with 8 slots and one MMA per output row
     int32_t taps, kci;        // k*k, C_in / 64
     int32_t MT;               // output-channel tiles of 128
     int32_t T_max;            // ROW: tiles per unit; POS: slots (multiple of 16)
@@ -374,6 +374,8 @@ __device__ __forceinline__ Sched make_sched(const TcArgs &p, int G)
     const int want = max(1, (G * p.MT + p.num_sms - 1) / p.num_sms);
     if (p.mode == 0)
         s.T = min(p.T_max, want);
+    else if (p.mode == 2)
+        s.T = 8;
     else
         s.T = min(p.T_max, ((want + 15) / 16) * 16);
     s.TB = (G + s.T - 1) / s.T;
@@ -803,7 +805,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             uint32_t pa = 0, pb = 0, uit = 0, ait = 0;
             bool ok = true;
             const int bin = c.bin, k = c.k, taps = p.taps, nT = sc.T, bb = c.b;
-            const int n_mma = p.mode == 0 ? 64 : nT;
+            // ROW: a tile's 64 pixels; POS: the unit's slots at one pixel; mode 2:
+            // the 8 slots at each of an output row's b pixels (8 b rows of N)
+            const int n_mma = p.mode == 0 ? 64 : p.mode == 2 ? 8 * bb : nT;
             const uint32_t idesc = idesc_bf16(n_mma);
             const uint32_t sk = p.mode == 0 ? (uint32_t)bin * 16 : (uint32_t)nT * 16;   // LBO
             const uint32_t sh = 8 * sk;      // ROW: halo row stride; POS: halo pixel stride
@@ -833,9 +837,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         break;
                     }
                     const int tap_end = min(taps, tap + (un.ke - kc));
+                    // N-groups of 8 rows: ROW, 8 halo pixels of a row (next group one
+                    // halo row on); POS, 8 slots (next group 8 slots on); mode 2,
+                    // the 8 slots at one pixel (next group the next output pixel,
+                    // s halo pixels on)
                     const uint64_t b_stage = p.mode == 0
                         ? desc_plain(sbase + cv.b_base + sb * cv.stage_b, sk, sh)
-                        : desc_plain(sbase + cv.b_base + sb * cv.stage_b, sk, 128);
+                        : p.mode == 2 ? desc_plain(sbase + cv.b_base + sb * cv.stage_b, sk, (uint32_t)c.s * sh)
+                                      : desc_plain(sbase + cv.b_base + sb * cv.stage_b, sk, 128);
                     int r = tap / k, cc = tap - r * k;
                     uint64_t b_tap = b_stage + (uint64_t)r * d_row + (uint64_t)cc * d_col;
                     if (p.mode == 0 && nT == 1) {
@@ -876,6 +885,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll 1
                                 for (int t = 0; t < nT; ++t, bt += d_tile)
                                     tc_mma_w(tmem + t * 64, a_cur + 2 * ks, bt, idesc, ks ? 1u : acc0);
+                            }
+                        } else if (p.mode == 2) {
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks) {
+                                uint64_t bi = b_tap + ks * d_ks;
+#pragma unroll 1
+                                for (int i = 0; i < bb; ++i, bi += d_i)
+                                    tc_mma_w(tmem + (uint32_t)(i * bb * 8), a_cur + 2 * ks, bi, idesc, ks ? 1u : acc0);
                             }
                         } else {
 #pragma unroll
@@ -1326,12 +1343,16 @@ static bool plan_layer(const sige_conv_desc *cd, TcPlan &pl)
     const int b = cd->block, s = cd->stride, k = cd->kernel;
     const int bin = (b - 1) * s + k;
     pl.per_slot = (uint32_t)bin * bin * 128;  // one tile, 64 channels
-    pl.mode = (b == 8 && s == 1) ? 0 : 1;
+    // ROW for 8x8 tiles at stride 1; mode 2 where an output row of 8 slots is a
+    // legal MMA width (8 b a multiple of 16); POS otherwise
+    pl.mode = (b == 8 && s == 1) ? 0 : (b % 2 == 0 && 8 * b <= 256) ? 2 : 1;
     const int budget = kSmemLimit - 1024 /*alignment*/ - (int)kCtrlBytes - 2 * (int)kAStageBytes - 1024;
     for (int SB : {2, 1}) {
         int tmax;
         if (pl.mode == 0) {
             tmax = std::min(8, budget / (int)(SB * pl.per_slot));      // 64 TMEM columns per tile
+        } else if (pl.mode == 2) {
+            tmax = (8 * SB * (int)pl.per_slot <= budget && b * b * 8 <= 512) ? 8 : 0;
         } else {
             const int by_tmem = (512 / (b * b)) / 16 * 16;
             const int by_smem = (budget / (int)(SB * pl.per_slot)) / 16 * 16;
@@ -1341,7 +1362,7 @@ static bool plan_layer(const sige_conv_desc *cd, TcPlan &pl)
         }
         // the epilogue stages at least 16 accumulator columns (8 KB) in the
         // halo stages of the smallest unit (1 tile, or 16 slots)
-        const uint32_t min_stage = SB * pl.per_slot * (pl.mode == 0 ? 1u : 16u);
+        const uint32_t min_stage = SB * pl.per_slot * (pl.mode == 0 ? 1u : pl.mode == 2 ? 8u : 16u);
         if (tmax >= 1 && min_stage >= 16u * 512u) {
             pl.T_max = tmax;
             pl.SB = SB;

@@ -220,6 +220,24 @@ int sige_groupnorm_affine(const void *x, const sige_tensor_desc *xd, int32_t gro
                           const float *gamma, const float *beta, float eps, float *scale,
                           float *shift, sige_stream_t stream);
 
+/* (7) Restore listed tiles from a source tensor, for sequential edits.
+ * SIGE project page, "Overview", updates the cached F_l(A_original) in place
+ * with the edited tiles; an interactive session applies edit after edit.  Each
+ * edit's tile list comes from the mask against the ORIGINAL input, so it covers
+ * every region that still differs; the tiles of the previous edit must first
+ * be put back to their original values (a region the user reverted would
+ * otherwise keep stale values).  This copies, for every in-image pixel of the
+ * listed tiles,
+ *   dst[n][h0+i][w0+j][:] = src[n][h0+i][w0+j][:]     (i, j < block)
+ * where src holds the original cache (untouched) and dst the working cache.
+ *   src, dst : device, NHWC, the same shape and dtype (u8, f32 or bf16), not
+ *              overlapping
+ *   idx      : device int32 (h0, w0) pairs; count : device int32, the number
+ *              of valid pairs (only the first min(count, capacity) are used)
+ * Every other byte of dst is left untouched.  Asynchronous on `stream`. */
+int sige_restore_tiles(const void *src, void *dst, const sige_tensor_desc *d, int32_t block,
+                       const int32_t *idx, const int32_t *count, int32_t capacity, sige_stream_t stream);
+
 /* ------------------------------------------------------------ utilities */
 
 /* Workspace bytes for sige_sparse_conv / sige_conv_fused / sige_dense_conv

@@ -256,3 +256,19 @@ def block_conv(blocks: np.ndarray, w: torch.Tensor, k=3, stride=1, block=4) -> n
     out = np.zeros((nb, block, block, Cout), dtype=np.float64)
     lib().oracle_block_conv(_p(blocks), nb, Cin, _p(w), _dtype_code(w), Cout, k, stride, block, _p(out))
     return out
+
+
+def restore_tiles(src: torch.Tensor, dst: torch.Tensor, block: int, idx: np.ndarray) -> torch.Tensor:
+    """Sequential edits (SIGE project page, "Overview": the cache of F_l(A_original)
+    is updated in place): the tiles (h0, w0) of ``idx`` are put back from ``src``
+    into a copy of ``dst``, clipped at the border; every other element keeps
+    dst's value.  A plain copy, written out pixel by pixel."""
+    out = dst.clone()
+    N, H, W, _ = dst.shape
+    for h0, w0 in np.asarray(idx, dtype=np.int64).reshape(-1, 2):
+        for i in range(block):
+            for j in range(block):
+                y, x = int(h0) + i, int(w0) + j
+                if y < H and x < W:
+                    out[:, y, x, :] = src[:, y, x, :]
+    return out

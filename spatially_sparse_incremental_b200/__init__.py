@@ -59,6 +59,7 @@ SIGNATURES = {
                                _vp, _sz, _vp]),
     "sige_dense_conv": (_i32, [_vp, _TD, _vp, _vp, _CD, _vp, _vp, _i32, _vp, _vp, _TD, _vp, _sz, _vp]),
     "sige_groupnorm_affine": (_i32, [_vp, _TD, _i32, _vp, _vp, _f32, _vp, _vp, _vp]),
+    "sige_restore_tiles": (_i32, [_vp, _vp, _TD, _i32, _vp, _vp, _i32, _vp]),
     "sige_conv_workspace_bytes": (_sz, [_CD, _i32, _i32, _i32, _i32]),
     "sige_get_error": (_i32, [_vp, _vp]),
     "sige_conv_path": (_i32, [_CD, _i32]),
@@ -252,6 +253,18 @@ def sige_groupnorm_affine(x, groups, gamma, beta, eps=1e-5, scale=None, shift=No
                                      _ptr(scale), _ptr(shift), _stream(stream))
     _check(st, "sige_groupnorm_affine")
     return scale, shift
+
+
+def sige_restore_tiles(src, dst, block, idx, count, capacity, stream=None):
+    """dst[n, h0+i, w0+j, :] = src[n, h0+i, w0+j, :] for the listed tiles (in-image
+    pixels, i, j < block); every other element of dst is left as it is."""
+    if src.shape != dst.shape or src.dtype != dst.dtype:
+        raise ValueError("src and dst must have the same shape and dtype")
+    d = tensor_desc(dst)
+    st = lib().sige_restore_tiles(_ptr(src), _ptr(dst), ctypes.byref(d), int(block), _ptr(idx), _ptr(count),
+                                  int(capacity), _stream(stream))
+    _check(st, "sige_restore_tiles")
+    return dst
 
 
 def sige_conv_workspace_bytes(cd: ConvDesc, batch: int, capacity: int, out_h: int, out_w: int) -> int:

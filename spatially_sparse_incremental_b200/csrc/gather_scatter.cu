@@ -158,6 +158,47 @@ __global__ void __launch_bounds__(1024) k_gn_affine(const __grid_constant__ GnPa
     }
 }
 
+// Tile restore for sequential edits: dst[n][h0+i][w0+j][:] = src[...] for the
+// in-image pixels of every listed tile.  One thread per 16-byte vector of a
+// tile row (NHWC: a tile row is b * C contiguous elements), or per element when
+// rows are not made of whole vectors.
+struct RestoreParams {
+    const uint8_t *src;
+    uint8_t *dst;
+    int32_t N, H, W, row_bytes;  // row_bytes = C * element size
+    int32_t b, vec;              // vec: 1 = 16-byte vectors, 0 = bytes
+    const int32_t *idx, *count;
+    int32_t cap;
+};
+
+__global__ void __launch_bounds__(256) k_restore(const __grid_constant__ RestoreParams p)
+{
+    const int ntiles = min(__ldg(p.count), p.cap);
+    const int unit = p.vec ? 16 : 1;
+    const int per_px = p.row_bytes / unit;          // units per pixel
+    const int64_t per_tile = (int64_t)p.N * p.b * p.b * per_px;
+    const int64_t total = per_tile * ntiles;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+        const int t = (int)(e / per_tile);
+        int64_t r = e - (int64_t)t * per_tile;
+        const int v = (int)(r % per_px);
+        r /= per_px;
+        const int j = (int)(r % p.b);
+        r /= p.b;
+        const int i = (int)(r % p.b);
+        const int n = (int)(r / p.b);
+        const int2 o = __ldg(reinterpret_cast<const int2 *>(p.idx) + t);
+        const int y = o.x + i, x = o.y + j;
+        if (y >= p.H || x >= p.W)
+            continue;
+        const int64_t off = (((int64_t)n * p.H + y) * p.W + x) * p.row_bytes + (int64_t)v * unit;
+        if (p.vec)
+            *reinterpret_cast<uint4 *>(p.dst + off) = __ldg(reinterpret_cast<const uint4 *>(p.src + off));
+        else
+            p.dst[off] = __ldg(p.src + off);
+    }
+}
+
 static int grid_for(int64_t work, int threads)
 {
     int64_t g = (work + threads - 1) / threads;
@@ -254,6 +295,33 @@ extern "C" int sige_groupnorm_affine(const void *x, const sige_tensor_desc *xd, 
     p.gamma = gamma; p.beta = beta; p.eps = eps; p.scale = scale; p.shift = shift;
     prefer_max_shared(k_gn_affine);
     k_gn_affine<<<xd->n * groups, 1024, 0, (cudaStream_t)stream>>>(p);
+    count_launch();
+    return launch_check();
+}
+
+extern "C" int sige_restore_tiles(const void *src, void *dst, const sige_tensor_desc *d, int32_t block,
+                                  const int32_t *idx, const int32_t *count, int32_t capacity, sige_stream_t stream)
+{
+    if (!src || !dst || !d || !idx || !count || capacity < 0 || block < 1)
+        return SIGE_ERR_INVALID_ARG;
+    if (d->n < 1 || d->h < 1 || d->w < 1 || d->c < 1)
+        return SIGE_ERR_INVALID_ARG;
+    if (d->layout != SIGE_NHWC || (d->dtype != SIGE_U8 && d->dtype != SIGE_F32 && d->dtype != SIGE_BF16))
+        return SIGE_ERR_UNSUPPORTED;
+    if (capacity == 0)
+        return SIGE_OK;
+    const int esz = d->dtype == SIGE_U8 ? 1 : d->dtype == SIGE_BF16 ? 2 : 4;
+    RestoreParams p{};
+    p.src = static_cast<const uint8_t *>(src);
+    p.dst = static_cast<uint8_t *>(dst);
+    p.N = d->n; p.H = d->h; p.W = d->w;
+    p.row_bytes = d->c * esz;
+    p.b = block;
+    p.vec = (p.row_bytes % 16 == 0 && ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) == 0)
+                ? 1 : 0;
+    p.idx = idx; p.count = count; p.cap = capacity;
+    const int64_t work = (int64_t)capacity * p.N * block * block * (p.row_bytes / (p.vec ? 16 : 1));
+    k_restore<<<grid_for(work, 256), 256, 0, (cudaStream_t)stream>>>(p);
     count_launch();
     return launch_check();
 }

@@ -456,3 +456,18 @@ def test_gather_stride2_definition(orc):
     for t, (h0, w0) in enumerate(idx):
         hi, wi = min(h0 + 4, ref.shape[1]), min(w0 + 4, ref.shape[2])
         assert np.allclose(out[t, :hi - h0, :wi - w0], ref[0, h0:hi, w0:wi], rtol=0, atol=1e-12)
+
+
+def test_restore_tiles_copies_listed_regions_only(orc):
+    # hand-checkable: a 5x5 image, 2x2 tiles at (0, 0) and the clipped corner (4, 4)
+    src = torch.arange(2 * 5 * 5 * 3, dtype=torch.float32).reshape(2, 5, 5, 3)
+    dst = -torch.ones_like(src)
+    got = orc.restore_tiles(src, dst, 2, np.array([[0, 0], [4, 4]], np.int32))
+    want = dst.clone()
+    for (y, x) in [(0, 0), (0, 1), (1, 0), (1, 1), (4, 4)]:
+        want[:, y, x, :] = src[:, y, x, :]
+    assert torch.equal(got, want)
+    assert int((got != dst).sum()) == 2 * 5 * 3   # exactly 5 pixels x 2 batch x 3 channels changed
+    # an empty list leaves dst as it is; restoring src onto itself is the identity
+    assert torch.equal(orc.restore_tiles(src, dst, 2, np.zeros((0, 2), np.int32)), dst)
+    assert torch.equal(orc.restore_tiles(src, src, 3, np.array([[0, 3]], np.int32)), src)

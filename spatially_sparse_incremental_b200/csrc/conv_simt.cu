@@ -10,6 +10,7 @@
 // writes float32 output blocks or scatters bias + residual + one rounding into
 // the cached output.
 #include <algorithm>
+#include <atomic>
 
 #include "conv_common.cuh"
 #include "transform.cuh"
@@ -443,13 +444,13 @@ static int launch_conv_simt16(ConvParams p, cudaStream_t stream)
     if (p.ci_chunk < 1)
         return SIGE_ERR_UNSUPPORTED;
     const size_t smem = (size_t)kS16SmemFloats * sizeof(float);
-    static int attr_done[64] = {0};
+    static std::atomic<int> attr_done[64];
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if (dev >= 0 && dev < 64 && !attr_done[dev].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(k_conv_simt16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
             return SIGE_ERR_CUDA;
-        attr_done[dev] = 1;
+        attr_done[dev].store(1, std::memory_order_release);
     }
     const int ncog = (p.Cout + kS16Cout - 1) / kS16Cout;
     const int64_t max_units = (int64_t)(p.dense ? p.tiles_total : p.cap) * p.N * ncog;

@@ -39,6 +39,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "conv_tc.cuh"
@@ -1465,16 +1466,18 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
     p.counters = reinterpret_cast<uint32_t *>(ws);
     p.partials = reinterpret_cast<float *>(ws + ((p.num_sms * 4 + 255) / 256) * 256);
 
-    static int smem_set[64] = {0};
-    static int pair_clusters[64] = {0};   // co-resident clusters of two, -1: none
+    // per device: attribute set, co-resident clusters of two (0 = not yet
+    // known, -1 = none); concurrent first calls compute the same values
+    static std::atomic<int> smem_set[64];
+    static std::atomic<int> pair_clusters[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64)
         dev = 0;
-    if (!smem_set[dev]) {
+    if (!smem_set[dev].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(k_conv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
             return SIGE_ERR_CUDA;
-        smem_set[dev] = 1;
+        smem_set[dev].store(1, std::memory_order_release);
     }
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1488,7 +1491,7 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
     cfg.dynamicSmemBytes = kSmemLimit;
     cfg.stream = stream;
     cfg.attrs = attr;
-    if (!pair_clusters[dev]) {
+    if (!pair_clusters[dev].load(std::memory_order_acquire)) {
         int n = 0;
         cfg.gridDim = dim3(2 * ((p.num_sms + 1) / 2));
         cfg.numAttrs = 2;
@@ -1496,20 +1499,21 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
             cudaGetLastError();
             n = -1;
         }
-        pair_clusters[dev] = n;
+        pair_clusters[dev].store(n, std::memory_order_release);
     }
     // clusters of two CTAs (a 2-way K split then sums through the peer's
     // shared memory), as many as are co-resident; otherwise one CTA per SM
     cudaError_t e = cudaErrorUnknown;
-    if (pair_clusters[dev] > 0) {
+    const int clusters = pair_clusters[dev].load(std::memory_order_acquire);
+    if (clusters > 0) {
         p.pair = 1;
-        p.num_sms = 2 * std::min(pair_clusters[dev], p.num_sms / 2);
+        p.num_sms = 2 * std::min(clusters, p.num_sms / 2);
         cfg.gridDim = dim3(p.num_sms);
         cfg.numAttrs = 2;
         e = cudaLaunchKernelEx(&cfg, k_conv_tc, p, map, xmap);
         if (e != cudaSuccess) {
             cudaGetLastError();
-            pair_clusters[dev] = -1;
+            pair_clusters[dev].store(-1, std::memory_order_release);
         }
     }
     if (e != cudaSuccess) {

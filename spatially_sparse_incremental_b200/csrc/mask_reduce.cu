@@ -29,6 +29,7 @@
 // runs it for real.  CTA 0 is the only CTA that waits on others, and the
 // others wait on nothing, so any scheduling order of the CTAs completes.
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "sige_internal.cuh"
@@ -795,14 +796,14 @@ extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const si
         p.chunks_rem = (int32_t)(nchunks % (grid - 1));
         smem = std::max(kMaskStreamSmem, 2 * kMaxWords * sizeof(uint32_t));
     }
-    static int attr_done[64] = {0};
+    static std::atomic<int> attr_done[64];
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if (dev >= 0 && dev < 64 && !attr_done[dev].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(k_mask_reduce, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaskStreamSmem) !=
             cudaSuccess)
             return SIGE_ERR_CUDA;
-        attr_done[dev] = 1;
+        attr_done[dev].store(1, std::memory_order_release);
     }
     prefer_max_shared(k_mask_reduce);
     const cudaError_t e = launch_pdl(k_mask_reduce, dim3(grid), dim3(kMaskThreads), smem, (cudaStream_t)stream, p);

@@ -20,17 +20,17 @@ int launch_check()
 
 int device_sm_count()
 {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64];   // per device, 0 = not yet queried
     int d = 0;
     if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64)
         return kNumSMs;
-    if (!cache[d]) {
-        int n = 0;
+    int n = cache[d].load(std::memory_order_relaxed);
+    if (!n) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0)
             n = kNumSMs;
-        cache[d] = n;
+        cache[d].store(n, std::memory_order_relaxed);
     }
-    return cache[d];
+    return n;
 }
 
 static int esize(int dtype) { return dtype == SIGE_BF16 ? 2 : dtype == SIGE_F32 ? 4 : 1; }

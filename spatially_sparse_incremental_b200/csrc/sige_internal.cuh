@@ -1,6 +1,7 @@
 // Internal definitions shared by the CUDA sources of libsige.
 #pragma once
 
+#include <atomic>
 #include <utility>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -65,13 +66,13 @@ int launch_check();           // SIGE_OK or SIGE_ERR_CUDA after a launch
 template <typename K>
 inline void prefer_max_shared(K kernel)
 {
-    static int done[64] = {0};
+    static std::atomic<int> done[64];   // per device; concurrent first calls both set the same attribute
     int d = 0;
-    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64 || done[d])
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64 || done[d].load(std::memory_order_acquire))
         return;
     cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
     cudaGetLastError();   // a refused preference is not an error of the call
-    done[d] = 1;
+    done[d].store(1, std::memory_order_release);
 }
 void count_launch();
 int device_sm_count();

@@ -319,6 +319,29 @@ def measure_extras(dev, flush, stream, peaks, seed, step_graph):
     out["area_sweep"] = {"rows": sweep, "fit": {"slope_us_per_tile": float(slope), "intercept_us": float(icpt),
                                                 "r2": r2}}
 
+    # the same step with the tile list from a 2-pixel dilation (exact for two
+    # chained 3x3 convs) instead of one tile
+    d = make_workload(seed, dev)
+    torch.cuda.synchronize()
+    calls = step_calls(d, stream)
+
+    def mask_px():
+        sige.sige_reduce_mask_px(d["x_orig"], d["x_edit"], THRESH, [(H, W, BLOCK, d["cap"])], 2, idx=d["idx"],
+                                 counts=d["cnt"], workspace=d["mask_ws"], stream=stream)
+    with torch.cuda.stream(stream):
+        mask_px()
+    stream.synchronize()
+    tiles_px = int(d["cnt"].item())
+
+    def whole_px():
+        mask_px()
+        calls["conv1"]()
+        calls["conv2"]()
+    g = capture(whole_px, stream)
+    t = time_graph(g, flush, 40, stream)
+    out["pixel_dilation_step"] = {"radius_px": 2, "active_tiles": tiles_px, "step_us": float(np.median(t)) * 1e3}
+    del g, d
+
     layers = [("fp32 64x64 C64 3x3 b4", inputs.make_cfg1(seed), 32)]
     for i, (h, w, c, b) in enumerate(inputs.CFG4_LAYERS):
         layers.append((f"SD latent {h}x{w} C{c} 3x3 b{b}", inputs.make_cfg4_layer(seed, i), 16))

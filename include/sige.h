@@ -121,6 +121,21 @@ int sige_reduce_mask(const void *a_orig, const void *a_edit, const sige_tensor_d
                      const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
                      void *workspace, size_t workspace_bytes, sige_stream_t stream);
 
+/* (1c) sige_reduce_mask with the dilation in pixels instead of tiles.
+ * mer.dev notes on SIGE, section 3.2 "Sparse Engine SIGE": the mask is dilated
+ * before the tiles are selected; the dilation only has to cover the layers'
+ * receptive-field growth.  Per scale the OR-downsampled mask is dilated by a
+ * square of `radius` pixels at that scale (clipped at the border) and every
+ * b x b tile holding a set pixel is listed; no tile dilation follows.  With
+ * radius = the layers' total halo (1 for one 3x3 conv, 2 for two chained ones)
+ * the sparse result still equals the dense one of the edited input, on fewer
+ * tiles than a one-tile dilation.  Arguments, layout, workspace and errors as
+ * sige_reduce_mask; radius >= 0 (0: tiles of the raw downsampled mask). */
+int sige_reduce_mask_px(const void *a_orig, const void *a_edit, const sige_tensor_desc *in,
+                        float threshold, int32_t radius, int32_t n_scales,
+                        const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
+                        void *workspace, size_t workspace_bytes, sige_stream_t stream);
+
 /* (1b) sige_reduce_mask without a caller workspace.  There is no counterpart
  * in the paper: this is a convenience for callers that cannot allocate device
  * memory for a workspace (a process that reserves all device memory up front,

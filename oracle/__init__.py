@@ -151,6 +151,19 @@ def reduce_mask(a_orig, a_edit, threshold, scales, dilate_tiles=1, layout=NHWC):
     return [reduce_scale(m, Hs, Ws, b, dilate_tiles) for (Hs, Ws, b) in scales]
 
 
+def reduce_mask_px(a_orig, a_edit, threshold, scales, radius=1, layout=NHWC):
+    """Pixel-level dilation (mer.dev notes, section 3.2: dilate, then select
+    tiles): per scale, OR-downsample the pixel mask, dilate it by a square of
+    ``radius`` pixels at that scale, then list the b x b tiles holding a set
+    pixel (no tile dilation)."""
+    m = pixel_mask(a_orig, a_edit, threshold, layout)
+    out = []
+    for (Hs, Ws, b) in scales:
+        md = dilate(downsample(m, Hs, Ws), radius)
+        out.append(reduce_scale(md, Hs, Ws, b, 0))
+    return out
+
+
 def gn_affine(x: torch.Tensor, groups: int, gamma: torch.Tensor, beta: torch.Tensor, eps: float = 1e-5):
     """Per-(n, channel) scale and shift (float64 [N, C]) folding GroupNorm of ``x``."""
     x = _c(x)

@@ -51,6 +51,7 @@ _TD, _CD, _SD = ctypes.POINTER(TensorDesc), ctypes.POINTER(ConvDesc), ctypes.POI
 SIGNATURES = {
     "sige_reduce_mask_workspace_bytes": (_sz, [_TD, _i32, _SD]),
     "sige_reduce_mask": (_i32, [_vp, _vp, _TD, _f32, _i32, _i32, _SD, _vp, _vp, _vp, _sz, _vp]),
+    "sige_reduce_mask_px": (_i32, [_vp, _vp, _TD, _f32, _i32, _i32, _SD, _vp, _vp, _vp, _sz, _vp]),
     "sige_reduce_mask_static": (_i32, [_vp, _vp, _TD, _f32, _i32, _i32, _SD, _vp, _vp, _vp]),
     "sige_gather": (_i32, [_vp, _TD, _CD, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _vp]),
     "sige_sparse_conv": (_i32, [_vp, _CD, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _sz, _vp]),
@@ -158,6 +159,27 @@ def sige_reduce_mask(a_orig, a_edit, threshold, scales, dilate=1, layout=NHWC, i
                                 len(scales), arr, _ptr(idx), _ptr(counts), _ptr(workspace),
                                 workspace.numel(), _stream(stream))
     _check(st, "sige_reduce_mask")
+    return idx, counts, workspace
+
+
+def sige_reduce_mask_px(a_orig, a_edit, threshold, scales, radius=1, layout=NHWC, idx=None, counts=None,
+                        workspace=None, stream=None):
+    """As sige_reduce_mask, with the mask dilated by ``radius`` pixels at each
+    scale before tiling (no tile dilation)."""
+    desc = tensor_desc(a_orig, layout)
+    arr = (ScaleDesc * len(scales))(*[ScaleDesc(*s) for s in scales])
+    dev = a_orig.device
+    if idx is None:
+        idx = torch.empty((max(1, sum(s[3] for s in scales)), 2), dtype=torch.int32, device=dev)
+    if counts is None:
+        counts = torch.empty(len(scales), dtype=torch.int32, device=dev)
+    need = int(lib().sige_reduce_mask_workspace_bytes(ctypes.byref(desc), len(scales), arr))
+    if workspace is None:
+        workspace = zeros_workspace(need, dev)
+    st = lib().sige_reduce_mask_px(_ptr(a_orig), _ptr(a_edit), ctypes.byref(desc), float(threshold), int(radius),
+                                   len(scales), arr, _ptr(idx), _ptr(counts), _ptr(workspace),
+                                   workspace.numel(), _stream(stream))
+    _check(st, "sige_reduce_mask_px")
     return idx, counts, workspace
 
 

@@ -44,6 +44,8 @@ struct ScaleParams {
     int32_t flag_off;        // byte offset of this scale's flags
     int32_t idx_off;         // pair offset of this scale's list
     int32_t log_h, log_w;    // log2 of tile_h / tile_w when powers of two, else -1
+    int32_t fy, fx;          // downsample factors (input pixels per scale pixel)
+    int32_t hs, ws;          // the scale's grid
 };
 
 struct __align__(16) MaskParams {
@@ -67,6 +69,7 @@ struct __align__(16) MaskParams {
     int32_t log_vpp, log_w, log_epv;
     int32_t chunk;       // modes 0, 1: vectors per chunk of each input (multiple of 256)
     int32_t chunks_base, chunks_rem;   // chunks per streaming CTA: base, +1 for the first rem
+    int32_t radius;      // pixel dilation at each scale before tiling (0: none)
 };
 
 // Copy the parameter block into shared memory, one 16-byte piece per lane of
@@ -129,13 +132,24 @@ __device__ __forceinline__ uint32_t diff_bits16(uint4 a, uint4 b, int dtype, flo
 // generic loads, which cost about a global-memory round trip each.  Every CTA
 // therefore copies the parameter block into shared memory once, and the
 // out-of-line functions below read that copy.
-__device__ __forceinline__ void mark(const ScaleParams *sc, int n_scales, uint8_t *flags, int y, int x)
+__device__ __forceinline__ void mark(const ScaleParams *sc, int n_scales, uint8_t *flags, int y, int x, int R)
 {
     for (int s = 0; s < n_scales; ++s) {
         const ScaleParams q = sc[s];
-        const int ty = q.log_h >= 0 ? y >> q.log_h : y / q.tile_h;
-        const int tx = q.log_w >= 0 ? x >> q.log_w : x / q.tile_w;
-        flags[q.flag_off + ty * q.tw + tx] = 1;
+        if (R == 0) {
+            const int ty = q.log_h >= 0 ? y >> q.log_h : y / q.tile_h;
+            const int tx = q.log_w >= 0 ? x >> q.log_w : x / q.tile_w;
+            flags[q.flag_off + ty * q.tw + tx] = 1;
+            continue;
+        }
+        // pixel dilation: every tile the (2R+1)^2 square around the pixel's
+        // scale position touches (clipped at the border)
+        const int Y = y / q.fy, X = x / q.fx;
+        const int t0 = max(0, Y - R) / q.block, t1 = min(q.hs - 1, Y + R) / q.block;
+        const int u0 = max(0, X - R) / q.block, u1 = min(q.ws - 1, X + R) / q.block;
+        for (int ty = t0; ty <= t1; ++ty)
+            for (int tx = u0; tx <= u1; ++tx)
+                flags[q.flag_off + ty * q.tw + tx] = 1;
     }
 }
 
@@ -155,11 +169,11 @@ __device__ __noinline__ void mark_bits(const MaskParams &p, const ScaleParams *s
     if (p.mode == 0) {
         if (p.pow2) {
             const int64_t pix = v >> p.log_vpp;
-            mark(sc, p.n_scales, p.flags, (int)(pix >> p.log_w) & (p.H - 1), (int)pix & (p.W - 1));
+            mark(sc, p.n_scales, p.flags, (int)(pix >> p.log_w) & (p.H - 1), (int)pix & (p.W - 1), p.radius);
         } else {
             const int64_t HW = (int64_t)p.H * p.W;
             const int64_t pix = v / p.vpp;
-            mark(sc, p.n_scales, p.flags, (int)((pix % HW) / p.W), (int)(pix % p.W));
+            mark(sc, p.n_scales, p.flags, (int)((pix % HW) / p.W), (int)(pix % p.W), p.radius);
         }
     } else {
         const int64_t e0 = v * p.epv;
@@ -168,7 +182,7 @@ __device__ __noinline__ void mark_bits(const MaskParams &p, const ScaleParams *s
         while (bits) {
             const int k = __ffs(bits) - 1;
             bits &= bits - 1;
-            mark(sc, p.n_scales, p.flags, y, x0 + k);
+            mark(sc, p.n_scales, p.flags, y, x0 + k, p.radius);
         }
     }
 }
@@ -191,7 +205,7 @@ __device__ __noinline__ bool scalar_pass(const MaskParams &p, const ScaleParams 
                 y = (int)((i / p.W) % p.H);
                 x = (int)(i % p.W);
             }
-            mark(sc, p.n_scales, p.flags, y, x);
+            mark(sc, p.n_scales, p.flags, y, x, p.radius);
         }
     }
     return wrote;
@@ -705,10 +719,10 @@ extern "C" size_t sige_reduce_mask_workspace_bytes(const sige_tensor_desc *in, i
     return kWsHeader + flag_bytes_of(n_scales, scales);
 }
 
-extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const sige_tensor_desc *in,
-                                float threshold, int32_t dilate, int32_t n_scales,
-                                const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
-                                void *workspace, size_t workspace_bytes, sige_stream_t stream)
+static int reduce_mask_impl(const void *a_orig, const void *a_edit, const sige_tensor_desc *in, float threshold,
+                            int32_t dilate, int32_t radius, int32_t n_scales, const sige_scale_desc *scales,
+                            int32_t *idx, int32_t *counts, void *workspace, size_t workspace_bytes,
+                            sige_stream_t stream)
 {
     if (!a_orig || !a_edit || !in || !idx || !counts)
         return SIGE_ERR_INVALID_ARG;
@@ -718,7 +732,7 @@ extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const si
         return SIGE_ERR_UNSUPPORTED;
     if (in->layout != SIGE_NHWC && in->layout != SIGE_NCHW)
         return SIGE_ERR_UNSUPPORTED;
-    if (!(threshold >= 0.0f) || threshold != threshold || dilate < 0)
+    if (!(threshold >= 0.0f) || threshold != threshold || dilate < 0 || radius < 0)
         return SIGE_ERR_INVALID_ARG;
     if (!scales_ok(in, n_scales, scales))
         return SIGE_ERR_INVALID_ARG;
@@ -735,6 +749,7 @@ extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const si
     p.dtype = in->dtype; p.layout = in->layout;
     p.thr = threshold;
     p.dilate = dilate;
+    p.radius = radius;
     p.n_scales = n_scales;
     int32_t foff = 0, ioff = 0;
     for (int s = 0; s < n_scales; ++s) {
@@ -750,6 +765,10 @@ extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const si
         o.idx_off = ioff;
         o.log_h = log2_exact(o.tile_h);
         o.log_w = log2_exact(o.tile_w);
+        o.fy = in->h / q.h;
+        o.fx = in->w / q.w;
+        o.hs = q.h;
+        o.ws = q.w;
         foff += (int32_t)align16((size_t)o.th * o.tw);
         ioff += q.capacity;
     }
@@ -811,6 +830,24 @@ extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const si
     if (e != cudaSuccess)
         return SIGE_ERR_CUDA;
     return launch_check();
+}
+
+extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const sige_tensor_desc *in,
+                                float threshold, int32_t dilate, int32_t n_scales,
+                                const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
+                                void *workspace, size_t workspace_bytes, sige_stream_t stream)
+{
+    return reduce_mask_impl(a_orig, a_edit, in, threshold, dilate, 0, n_scales, scales, idx, counts, workspace,
+                            workspace_bytes, stream);
+}
+
+extern "C" int sige_reduce_mask_px(const void *a_orig, const void *a_edit, const sige_tensor_desc *in,
+                                   float threshold, int32_t radius, int32_t n_scales,
+                                   const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
+                                   void *workspace, size_t workspace_bytes, sige_stream_t stream)
+{
+    return reduce_mask_impl(a_orig, a_edit, in, threshold, 0, radius, n_scales, scales, idx, counts, workspace,
+                            workspace_bytes, stream);
 }
 
 // ------------------------------------------------------------------ variant without a workspace

@@ -156,3 +156,45 @@ def test_cfg3_large_edits(orc, area):
     got, cnt, ws = _gpu_lists(blk.x_orig, blk.x_edit, 1e-3, _full_caps(sc))
     assert sige.sige_get_error(ws) == sige.OK
     assert cnt[0] == len(ref[0]) and np.array_equal(got[0], ref[0])
+
+
+def test_pixel_dilation_random_cases(orc):
+    rng = np.random.default_rng(21)
+    for case in range(80):
+        dtype = [torch.uint8, torch.float32, torch.bfloat16][case % 3]
+        layout = sige.NHWC if rng.random() < 0.6 else sige.NCHW
+        f = int(rng.choice([1, 2, 4]))
+        Hs, Ws = int(rng.integers(2, 20)), int(rng.integers(2, 20))
+        H, W, C = Hs * f, Ws * f, int(rng.choice([3, 8, 16, 64]))
+        if dtype == torch.uint8:
+            a = torch.from_numpy(rng.integers(0, 256, size=(1, H, W, C)).astype(np.uint8))
+        else:
+            a = torch.from_numpy(rng.normal(size=(1, H, W, C)).astype(np.float32)).to(dtype)
+        b = a.clone()
+        m = rng.random((1, H, W)) < rng.choice([0.01, 0.05, 0.3])
+        b[torch.from_numpy(m)] = (b[torch.from_numpy(m)] ^ 1) if dtype == torch.uint8 else b[torch.from_numpy(m)] + 1.0
+        if layout == sige.NCHW:
+            a, b = a.permute(0, 3, 1, 2).contiguous(), b.permute(0, 3, 1, 2).contiguous()
+        thr = 0.0 if dtype == torch.uint8 else 1e-3
+        sc = [(H, W, int(rng.integers(1, 6))), (Hs, Ws, int(rng.integers(1, 4)))]
+        R = int(rng.integers(0, 4))
+        ref = orc.reduce_mask_px(a, b, thr, sc, R, orc.NHWC if layout == sige.NHWC else orc.NCHW)
+        caps = _full_caps(sc)
+        idx, cnt, _ = sige.sige_reduce_mask_px(a.to(DEV), b.to(DEV), thr, caps, R, layout)
+        torch.cuda.synchronize()
+        cnt, idx, off = cnt.cpu().numpy(), idx.cpu().numpy(), 0
+        for s, (h, w, blk, cap) in enumerate(caps):
+            assert cnt[s] == len(ref[s]) and np.array_equal(idx[off:off + cnt[s]], ref[s]), (case, s, R)
+            off += cap
+
+
+def test_pixel_dilation_cfg3(orc):
+    blk = inputs.make_cfg3(0, H=256, W=256, C=128, area=0.012)
+    sc = [(256, 256, 8)]
+    for R in (1, 2):
+        ref = orc.reduce_mask_px(blk.x_orig, blk.x_edit, 1e-3, sc, R)[0]
+        idx, cnt, ws = sige.sige_reduce_mask_px(blk.x_orig.to(DEV), blk.x_edit.to(DEV), 1e-3, _full_caps(sc), R)
+        torch.cuda.synchronize()
+        n = int(cnt[0].item())
+        assert n == len(ref) and np.array_equal(idx[:n].cpu().numpy(), ref)
+        assert sige.sige_get_error(ws) == sige.OK

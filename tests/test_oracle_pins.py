@@ -471,3 +471,75 @@ def test_restore_tiles_copies_listed_regions_only(orc):
     # an empty list leaves dst as it is; restoring src onto itself is the identity
     assert torch.equal(orc.restore_tiles(src, dst, 2, np.zeros((0, 2), np.int32)), dst)
     assert torch.equal(orc.restore_tiles(src, src, 3, np.array([[0, 3]], np.int32)), src)
+
+
+# ------------------------------------------------------------------ pixel-level dilation
+
+def _px_tiles_brute(m, Hs, Ws, b, R):
+    # a tile is active iff some set pixel of the downsampled mask lies within
+    # Chebyshev distance R of one of the tile's pixels (independent of dilate())
+    H, W = m.shape
+    fy, fx = H // Hs, W // Ws
+    ms = m.reshape(Hs, fy, Ws, fx).max(axis=(1, 3))
+    ys, xs = np.nonzero(ms)
+    out = []
+    for i in range(0, Hs, b):
+        for j in range(0, Ws, b):
+            y1, x1 = min(i + b, Hs) - 1, min(j + b, Ws) - 1
+            dy = np.maximum(0, np.maximum(i - ys, ys - y1))
+            dx = np.maximum(0, np.maximum(j - xs, xs - x1))
+            if len(ys) and (np.maximum(dy, dx) <= R).any():
+                out.append((i, j))
+    return np.array(out, np.int32).reshape(-1, 2)
+
+
+@pytest.mark.parametrize("R", [0, 1, 2, 5])
+def test_pixel_dilation_lists_brute_force(orc, R):
+    rng = np.random.default_rng(100 + R)
+    for case in range(60):
+        H, W = int(rng.integers(2, 20)) * 2, int(rng.integers(2, 20)) * 2
+        a = torch.from_numpy(rng.normal(size=(1, H, W, 4)).astype(np.float32))
+        e = a.clone()
+        m = rng.random((H, W)) < rng.choice([0.01, 0.05, 0.2])
+        e[0, torch.from_numpy(m)] += 1.0
+        for (Hs, Ws, b) in [(H, W, int(rng.integers(1, 6))), (H // 2, W // 2, int(rng.integers(1, 4)))]:
+            got = orc.reduce_mask_px(a, e, 1e-3, [(Hs, Ws, b)], R)[0]
+            want = _px_tiles_brute(m.astype(np.uint8), Hs, Ws, b, R)
+            assert np.array_equal(got, want), (case, Hs, Ws, b, R)
+
+
+def test_pixel_dilation_between_raw_and_tile_dilation(orc):
+    L = inputs.make_conv_case(41, 64, 64, 8, 8, block=4, area=0.03)
+    sc = [(64, 64, 4)]
+    raw = {tuple(t) for t in orc.reduce_mask_px(L.x_orig, L.x_edit, 1e-3, sc, 0)[0]}
+    px = {tuple(t) for t in orc.reduce_mask_px(L.x_orig, L.x_edit, 1e-3, sc, 1)[0]}
+    tile = {tuple(t) for t in orc.reduce_mask(L.x_orig, L.x_edit, 1e-3, sc, 1)[0]}
+    assert raw <= px <= tile and len(px) < len(tile)
+
+
+@pytest.mark.parametrize("b,k", [(4, 3), (8, 3), (2, 3), (4, 1)])
+def test_single_layer_exact_with_pixel_dilation(orc, b, k):
+    # dilating by the conv's halo (k // 2 pixels) is enough for the sparse
+    # layer to equal the dense layer of the edited input at every pixel
+    pad = k // 2
+    L = inputs.make_conv_case(13 + b, 32, 32, 8, 8, kernel=k, stride=1, pad=pad, block=b, area=0.03)
+    yc = orc.dense_conv(L.x_orig, L.weight, L.bias, k, 1, pad)
+    ye = orc.dense_conv(L.x_edit, L.weight, L.bias, k, 1, pad)
+    idx = orc.reduce_mask_px(L.x_orig, L.x_edit, 1e-3, [(32, 32, b)], pad)[0]
+    ys = orc.sparse_conv(L.x_edit, L.weight, L.bias, idx, yc, k, 1, pad, b)
+    assert torch.equal(ys, ye)
+
+
+def test_resblock_exact_with_two_pixel_dilation(orc):
+    # two chained 3x3 convs move the change by 2 pixels; with that dilation the
+    # sparse block equals the dense block of the edited input (cached GN stats)
+    blk = inputs.make_cfg3(3, H=32, W=32, C=64, area=0.03)
+    gn1 = orc.gn_affine(blk.x_orig, 32, blk.g1, blk.be1)
+    y1o = orc.dense_conv(blk.x_orig, blk.w1, blk.b1, gn=gn1, silu=True)
+    gn2 = orc.gn_affine(y1o, 32, blk.g2, blk.be2)
+    y1o, outo = orc.resblock_dense(blk.x_orig, blk, gn1, gn2)
+    y1e, oute = orc.resblock_dense(blk.x_edit, blk, gn1, gn2)
+    idx = orc.reduce_mask_px(blk.x_orig, blk.x_edit, 1e-3, [(32, 32, blk.block)], 2)[0]
+    assert 0 < len(idx) < 16
+    y1s, outs = orc.resblock_sparse(blk.x_edit, blk, idx, y1o, outo, gn1, gn2)
+    assert torch.equal(outs, oute)

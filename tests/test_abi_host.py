@@ -138,3 +138,34 @@ def test_groupnorm_validation(L):
     xd = sige.TensorDesc(1, 8, 8, 30, sige.F32, sige.NHWC)        # 30 channels, 32 groups
     assert L.sige_groupnorm_affine(fake, ctypes.byref(xd), 32, fake, fake, 1e-5, fake, fake, None) \
         == sige.ERR_INVALID_ARG
+
+
+def test_reduce_mask_px_validation(L):
+    d = sige.TensorDesc(1, 64, 64, 8, sige.F32, sige.NHWC)
+    sc = _scales((64, 64, 8, 64))
+    need = L.sige_reduce_mask_workspace_bytes(ctypes.byref(d), 1, sc)
+    fake, ws = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000)
+
+    def call(radius=1, a=fake, wsb=need, thr=1e-3):
+        return L.sige_reduce_mask_px(a, fake, ctypes.byref(d), thr, radius, 1, sc, fake, fake, ws, wsb, None)
+    assert call(radius=-1) == sige.ERR_INVALID_ARG
+    assert call(a=None) == sige.ERR_INVALID_ARG
+    assert call(thr=float("nan")) == sige.ERR_INVALID_ARG
+    assert call(wsb=need - 1) == sige.ERR_WORKSPACE
+
+
+def test_restore_tiles_validation(L):
+    d = sige.TensorDesc(1, 32, 32, 16, sige.BF16, sige.NHWC)
+    fake = ctypes.c_void_p(0x1000)
+
+    def call(src=fake, dst=fake, desc=ctypes.byref(d), block=8, idx=fake, cnt=fake, cap=16):
+        return L.sige_restore_tiles(src, dst, desc, block, idx, cnt, cap, None)
+    assert call(src=None) == sige.ERR_INVALID_ARG
+    assert call(dst=None) == sige.ERR_INVALID_ARG
+    assert call(idx=None) == sige.ERR_INVALID_ARG
+    assert call(block=0) == sige.ERR_INVALID_ARG
+    assert call(cap=-1) == sige.ERR_INVALID_ARG
+    assert call(cap=0) == sige.OK                      # nothing to restore, no launch
+    dn = sige.TensorDesc(1, 32, 32, 16, sige.BF16, sige.NCHW)
+    assert call(desc=ctypes.byref(dn)) == sige.ERR_UNSUPPORTED
+    assert call(desc=None) == sige.ERR_INVALID_ARG

@@ -3,6 +3,7 @@
 // edited activation, stack them along the batch axis, and scatter the output
 // blocks back into F_l(A_original)).  Plus the GroupNorm statistics of the
 // cached original activation, folded into a per-channel affine.
+#include <atomic>
 #include <algorithm>
 
 #include "sige_internal.cuh"
@@ -199,6 +200,145 @@ __global__ void __launch_bounds__(256) k_restore(const __grid_constant__ Restore
     }
 }
 
+// GroupNorm statistics of one image on a cluster of kGnCluster CTAs.  Each CTA
+// streams a contiguous range of pixels with 16-byte loads; a thread keeps, for
+// the channels of its vector column, the sums of (x - K_c) and (x - K_c)^2 in
+// double, with K_c the image's first pixel (the shift keeps the one-pass
+// variance exact to double rounding).  Partial sums meet in shared memory in
+// a fixed order, rank 0 adds the ranks' partials through distributed shared
+// memory (rank order) and turns each group's sums into scale / shift.
+constexpr int kGnCluster = 8;
+constexpr int kGnThreads = 512;
+constexpr int kGnBatch = 8;      // independent 16-byte loads in flight per thread
+
+__device__ __forceinline__ float gn_vec_elem(uint4 v, int k, int dtype)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    if (dtype == SIGE_BF16)
+        return (k & 1) ? bf16_hi(w[k >> 1]) : bf16_lo(w[k >> 1]);
+    return __uint_as_float(w[k]);
+}
+
+__global__ void __cluster_dims__(kGnCluster, 1, 1) __launch_bounds__(kGnThreads)
+    k_gn_stats_cluster(const __grid_constant__ GnParams p)
+{
+    extern __shared__ __align__(16) double gsm[];
+    const int C = p.C, esz = p.dtype == SIGE_BF16 ? 2 : 4, epv = 16 / esz;
+    const int vpp = C / epv;                       // vectors per pixel
+    const int rows = kGnThreads / vpp;             // pixels per pass
+    double *part = gsm;                            // [C][2] this CTA's sums
+    double *red = gsm + 2 * C;                     // [rows][C][2]
+    uint32_t rank;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+    const int n = blockIdx.x / kGnCluster;
+    const int t = threadIdx.x, v = t % vpp, r0 = t / vpp;
+    const uint8_t *img = p.x + (size_t)n * p.HW * C * esz;
+    const int64_t p0 = (int64_t)p.HW * rank / kGnCluster, p1 = (int64_t)p.HW * (rank + 1) / kGnCluster;
+    double s1[8], s2[8];
+    float K[8];
+    const uint4 k4 = __ldg(reinterpret_cast<const uint4 *>(img) + v);   // pixel 0 of the image
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        s1[k] = 0.0;
+        s2[k] = 0.0;
+        K[k] = k < epv ? gn_vec_elem(k4, k, p.dtype) : 0.0f;
+    }
+    if (r0 < rows) {
+#pragma unroll 1
+        for (int64_t px0 = p0 + r0; px0 < p1; px0 += (int64_t)rows * kGnBatch) {
+            uint4 x4[kGnBatch];
+#pragma unroll
+            for (int u = 0; u < kGnBatch; ++u) {
+                const int64_t px = px0 + (int64_t)u * rows;
+                x4[u] = px < p1 ? __ldg(reinterpret_cast<const uint4 *>(img + (size_t)px * C * esz) + v) : k4;
+            }
+#pragma unroll
+            for (int u = 0; u < kGnBatch; ++u)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    if (k >= epv)
+                        break;
+                    // past the range: the shift itself, which adds nothing
+                    const double d = (double)gn_vec_elem(x4[u], k, p.dtype) - (double)K[k];
+                    s1[k] += d;
+                    s2[k] = fma(d, d, s2[k]);
+                }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (k < epv) {
+                red[((size_t)r0 * C + v * epv + k) * 2] = s1[k];
+                red[((size_t)r0 * C + v * epv + k) * 2 + 1] = s2[k];
+            }
+    }
+    __syncthreads();
+    for (int c = t; c < C; c += kGnThreads) {      // fixed row order
+        double a = 0.0, b = 0.0;
+        for (int rr = 0; rr < rows; ++rr) {
+            a += red[((size_t)rr * C + c) * 2];
+            b += red[((size_t)rr * C + c) * 2 + 1];
+        }
+        part[2 * c] = a;
+        part[2 * c + 1] = b;
+    }
+    // every rank's partials are complete before rank 0 reads them
+    asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    if (rank == 0) {
+        const uint32_t local = static_cast<uint32_t>(__cvta_generic_to_shared(part));
+        const int cg = C / p.groups;
+        uint32_t remote[kGnCluster];
+#pragma unroll
+        for (int q = 0; q < kGnCluster; ++q)
+            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote[q]) : "r"(local), "r"(q));
+        for (int g = t; g < p.groups; g += kGnThreads) {
+            // channel sums over the ranks in rank order; two passes over the
+            // group's channels: the mean, then the centred second moment
+            const double cnt = (double)p.HW * cg;
+            double sx = 0.0;
+            for (int j = 0; j < cg; ++j) {
+                const int c = g * cg + j;
+                double a = 0.0;
+#pragma unroll
+                for (int q = 0; q < kGnCluster; ++q) {
+                    double e;
+                    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(e) : "r"(remote[q] + (uint32_t)(c * 16)));
+                    a += e;
+                }
+                const double Kc = (double)gn_vec_elem(__ldg(reinterpret_cast<const uint4 *>(img) + c / epv),
+                                                      c % epv, p.dtype);
+                sx += a + (double)p.HW * Kc;
+            }
+            const double mean = sx / cnt;
+            double sxx = 0.0;
+            for (int j = 0; j < cg; ++j) {
+                const int c = g * cg + j;
+                double a = 0.0, bb = 0.0;
+#pragma unroll
+                for (int q = 0; q < kGnCluster; ++q) {
+                    double e, f;
+                    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(e) : "r"(remote[q] + (uint32_t)(c * 16)));
+                    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(f) : "r"(remote[q] + (uint32_t)(c * 16 + 8)));
+                    a += e;
+                    bb += f;
+                }
+                const double Kc = (double)gn_vec_elem(__ldg(reinterpret_cast<const uint4 *>(img) + c / epv),
+                                                      c % epv, p.dtype);
+                const double dk = Kc - mean;
+                sxx += bb + 2.0 * dk * a + (double)p.HW * dk * dk;
+            }
+            const double var = sxx / cnt;
+            for (int j = 0; j < cg; ++j) {
+                const int c = g * cg + j;
+                const double sc = (double)p.gamma[c] / sqrt(var + (double)p.eps);
+                p.scale[(int64_t)n * C + c] = (float)sc;
+                p.shift[(int64_t)n * C + c] = (float)((double)p.beta[c] - mean * sc);
+            }
+        }
+    }
+    // rank 0 has read every rank's shared memory before any CTA leaves
+    asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 static int grid_for(int64_t work, int threads)
 {
     int64_t g = (work + threads - 1) / threads;
@@ -293,6 +433,33 @@ extern "C" int sige_groupnorm_affine(const void *x, const sige_tensor_desc *xd, 
     p.x = static_cast<const uint8_t *>(x);
     p.N = xd->n; p.HW = xd->h * xd->w; p.C = xd->c; p.dtype = xd->dtype; p.groups = groups;
     p.gamma = gamma; p.beta = beta; p.eps = eps; p.scale = scale; p.shift = shift;
+    // cluster path: whole 16-byte vectors per pixel, at most 256 of them, at
+    // most 64 channels per group, 16-byte aligned input
+    const int esz = xd->dtype == SIGE_BF16 ? 2 : 4;
+    const int vpp = (xd->c * esz) % 16 == 0 ? xd->c * esz / 16 : 0;
+    if (vpp >= 1 && vpp <= kGnThreads && xd->c / groups <= 64 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
+        const int rows = kGnThreads / vpp;
+        const size_t smem = (size_t)(2 * xd->c + (size_t)rows * xd->c * 2) * sizeof(double);
+        static std::atomic<int> attr_done[64];
+        int dev = 0;
+        cudaGetDevice(&dev);
+        bool ok = smem <= 200 * 1024;
+        if (ok && dev >= 0 && dev < 64 && !attr_done[dev].load(std::memory_order_acquire)) {
+            ok = cudaFuncSetAttribute(k_gn_stats_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      200 * 1024) == cudaSuccess;
+            if (ok)
+                attr_done[dev].store(1, std::memory_order_release);
+            else
+                cudaGetLastError();
+        }
+        if (ok) {
+            k_gn_stats_cluster<<<xd->n * kGnCluster, kGnThreads, smem, (cudaStream_t)stream>>>(p);
+            if (cudaGetLastError() == cudaSuccess) {
+                count_launch();
+                return SIGE_OK;
+            }
+        }
+    }
     prefer_max_shared(k_gn_affine);
     k_gn_affine<<<xd->n * groups, 1024, 0, (cudaStream_t)stream>>>(p);
     count_launch();

@@ -1,14 +1,17 @@
 // Layer F_l on the CUDA cores (float32 arithmetic): the path for float32
 // layers, and for bf16 layers the tensor-core kernel does not cover.
 //
-// One CTA works on one (tile, batch item, group of output channels) unit at a
-// time.  Per chunk of input channels it stages the tile's halo'd input block
-// (from the stacked blocks, or straight from the image with zero padding and
-// the GroupNorm affine + SiLU applied on the way in) and the chunk of the
-// group's weights in shared memory, then each thread accumulates one output
-// channel for a few of the tile's pixels.  The epilogue either
-// writes float32 output blocks or scatters bias + residual + one rounding into
-// the cached output.
+// Tiles of at most 16 pixels (b <= 4) run k_conv_simt16: a unit of 64 output
+// channels x 16 pixel slots, 4 K groups of 64 threads each holding a
+// 4-channel x 4-pixel block of accumulators, weights and halo staged per
+// input-channel chunk in shared memory (float32: asynchronous 4-byte copies),
+// the K groups summed in a fixed order at the end.  Larger tiles run
+// k_conv_simt: one CTA per (tile, batch item, group of output channels), each
+// thread one output channel for up to 16 of the tile's pixels.  Both stage the
+// halo from the stacked blocks, or straight from the image with zero padding
+// and the GroupNorm affine + SiLU applied on the way in, and end by writing
+// float32 output blocks or scattering bias + residual + one rounding into the
+// cached output.
 #include <algorithm>
 #include <atomic>
 

@@ -16,25 +16,35 @@
 //     address: the halo is read from global memory once per 64 channels and
 //     reused by all k*k taps inside shared memory;
 //   * D lives in tensor memory: lane = output channel, column = pixel.
-// Two B layouts:
+// Three B layouts:
 //   ROW (b = 8, stride 1): an N-group of 8 rows is one output row of a tile,
 //     i.e. 8 consecutive halo pixels; one MMA per (tile, tap, 16 channels),
 //     N = 64 (the tile's 8 x 8 pixels).
-//   POS (any other b, stride, kernel): an N-group of 8 rows is 8 tiles at the
-//     same halo position; one MMA per (output position (i, j), tap, 16
-//     channels), N = the number of tiles of the unit (16..256).
+//   Row-batched POS (even b otherwise): units of 8 tiles stored
+//     [halo row][halo col][channel group][slot]; an N-group of 8 rows is the 8
+//     tiles at one halo pixel, the next N-group the next output pixel of the
+//     row (s halo columns on), so one MMA covers an output row of all 8 tiles,
+//     N = 8 b.
+//   POS (odd b): an N-group of 8 rows is 8 tiles at the same halo position;
+//     one MMA per (output position (i, j), tap, 16 channels), N = the number
+//     of tiles of the unit (16..256).
 // The producers apply the GroupNorm affine + SiLU (and the zero padding
 // outside the image) while moving the halo into shared memory; the epilogue
 // adds bias and residual and rounds once into the cached output, or writes
 // float32 output blocks.  When the active tiles are too few to fill the GPU,
-// the K loop is split over several CTAs; the last CTA to finish a tile group
-// sums the partial accumulators in a fixed order (deterministic) and runs the
-// epilogue.
+// the K loop is split over several CTAs.  The kernel is launched in clusters
+// of two CTAs: a 2-way split of a unit of at most 64 columns is summed through
+// the peer's shared memory (rank 1 sends its partial to rank 0, which adds its
+// own and runs the epilogue); other splits end with the last CTA of a tile
+// group summing the partials from global memory in a fixed order
+// (deterministic either way).
 //
-// Warp roles (192 threads): warp 0 issues the weight TMA, warp 1 allocates
-// tensor memory and one thread issues the MMAs, warps 2-5 stage the halo and
-// run the epilogue.  Every mbarrier wait is bounded; on expiry the kernel
-// records SIGE_ERR_TIMEOUT in the workspace header and unwinds.
+// Warp roles (320 threads): warp 0 issues the weight TMA, warp 1 allocates
+// tensor memory and issues the MMAs, warps 2-9 stage the halo and run the
+// epilogue.  Warps 0 and 1 run warp-uniform loops and one lane, chosen by
+// elect.sync, issues each TMA / MMA / commit.  Every mbarrier wait is bounded;
+// on expiry the kernel records SIGE_ERR_TIMEOUT in the workspace header and
+// unwinds.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

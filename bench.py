@@ -87,34 +87,80 @@ def ncu_traffic(kernel):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled while the timed loop runs."""
+    """nvidia-smi clocks / throttle reasons sampled while the timed loop runs.
+
+    A reader thread stamps every sample with its arrival time.  `begin()` waits
+    for the first sample (nvidia-smi takes a moment to start) and marks the
+    start of the timed region, `stop()` marks its end and summarises the
+    samples taken inside it.  A timed region shorter than the sampling period
+    may hold none; then the last sample before it and the first after it
+    (which bracket it) are reported, and `window` says so."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 50
 
-    def __init__(self, device_index):
-        self.proc = None
+    def __init__(self, device_index, cmd=None):
+        import threading
+        self.proc, self.lines, self.t0 = None, [], None
+        self.lock = threading.Lock()
         try:
-            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
-            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "50"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            if cmd is None:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+                cmd = ["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                       "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            with self.lock:
+                self.lines.append((time.perf_counter(), ln))
+
+    def _wait_lines(self, n, timeout):
+        end = time.perf_counter() + timeout
+        while time.perf_counter() < end:
+            with self.lock:
+                if len(self.lines) >= n:
+                    return
+            time.sleep(0.005)
+
+    def begin(self):
+        if self.proc is not None:
+            self._wait_lines(1, 10.0)
+        self.t0 = time.perf_counter()
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        t1 = time.perf_counter()
+        with self.lock:
+            n_at_end = len(self.lines)
+        self._wait_lines(n_at_end + 1, 1.0)        # one sample after the region
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-            out = ""
+        self.reader.join(timeout=5)
+        with self.lock:
+            lines = list(self.lines)
+        t0 = self.t0 if self.t0 is not None else t1
+        inside = [ln for t, ln in lines if t0 <= t <= t1]
+        window = "inside the timed region"
+        if not inside:
+            before = [ln for t, ln in lines if t < t0][-1:]
+            after = [ln for t, ln in lines if t > t1][:1]
+            inside = before + after
+            window = "timed region shorter than the sampling period: the samples just before and after it"
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in out.strip().splitlines():
+        for ln in inside:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 8:
                 continue
@@ -127,7 +173,7 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(nm)
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "window": window}
 
 
 def dist_env():
@@ -515,9 +561,10 @@ def run_sige(args):
     def barrier():
         if ws > 1:
             torch.distributed.barrier()
+    sampler = ClockSampler(dev.index)
+    sampler.begin()
     barrier()
     torch.cuda.synchronize()
-    sampler = ClockSampler(dev.index)
     _, tot = timed_graph_steps(step_graph, flush, args.steps, stream)
     torch.cuda.synchronize()
     barrier()

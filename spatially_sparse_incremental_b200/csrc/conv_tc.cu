@@ -99,8 +99,11 @@ struct TcArgs {
     int32_t ncols;            // tensor-memory columns allocated (power of 2)
     int32_t num_sms;
     int32_t halo_tma;         // 1: ROW-mode halo rows come by TMA (tmx), 0: per-thread cp.async
-    int32_t pair;             // 1: launched in clusters of two CTAs; a 2-way K split of a unit
-                              // of <= 64 columns is summed through the peer's shared memory
+    int32_t pair;             // 1: launched in clusters (of csize CTAs)
+    int32_t csize;            // CTAs per cluster (1: no clusters).  csize 2: a 2-way K split of
+                              // a unit of <= 64 columns is summed through the peer's shared
+                              // memory; other splits that divide csize reduce-scatter within
+                              // the cluster; the rest go through global memory
 };
 
 __device__ __forceinline__ void tile_origin_a(const TcArgs &a, int t, int &h0, int &w0)
@@ -199,17 +202,7 @@ __device__ __forceinline__ void tc_commit(uint32_t bar)
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate)
-{
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Cluster helpers (pair launches).
+// Cluster helpers (cluster launches).
 __device__ __forceinline__ uint32_t cluster_rank()
 {
     uint32_t r;
@@ -230,11 +223,23 @@ __device__ __forceinline__ void st_peer_f32(uint32_t addr, float v)
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
+__device__ __forceinline__ void st_peer_f32x4(uint32_t addr, float a, float b, float c, float d)
+{
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
 // Arrive on an mbarrier of the peer; orders this thread's (and, through a
 // preceding CTA barrier, the CTA's) earlier writes before the arrival.
 __device__ __forceinline__ void mbar_arrive_peer(uint32_t addr)
 {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
+// The same with an arrival count.
+__device__ __forceinline__ void mbar_arrive_peer_n(uint32_t addr, uint32_t n)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(addr), "r"(n) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity)
@@ -281,16 +286,6 @@ __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.w
 // issuing loops then stay warp-uniform (their exits depend only on votes), so
 // the compiler keeps descriptors, coordinates and stage counters in uniform
 // registers, which is what the tensor-core and TMA instructions read.
-__device__ __forceinline__ void tc_mma_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t accumulate)
-{
-    asm volatile(
-        "{\n .reg .pred p, e;\n .reg .b32 l;\n elect.sync l|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 __device__ __forceinline__ void tc_commit_w(uint32_t bar)
 {
     asm volatile(
@@ -315,6 +310,24 @@ __device__ __forceinline__ void tc_mma4_commit_w(uint32_t d_tmem, uint64_t a_des
         " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, t;\n"
         " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n}\n" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "l"(b_step), "r"(bar)
+        : "memory");
+}
+
+// The four K=16 steps of one 64-channel k-chunk into one accumulator block,
+// from one elected lane (no commit).
+__device__ __forceinline__ void tc_mma4_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint64_t b_step,
+                                          uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n .reg .pred p, e, t;\n .reg .b32 l;\n .reg .b64 a1, a2, a3, b1, b2, b3;\n"
+        " elect.sync l|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n setp.eq.b32 t, 0, 0;\n"
+        " add.s64 a1, %1, 2;\n add.s64 a2, %1, 4;\n add.s64 a3, %1, 6;\n"
+        " add.s64 b1, %2, %5;\n add.s64 b2, b1, %5;\n add.s64 b3, b2, %5;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, t;\n}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "l"(b_step)
         : "memory");
 }
 
@@ -379,23 +392,36 @@ struct Sched {
     int units;
 };
 
-__device__ __forceinline__ Sched make_sched(const TcArgs &p, int G)
+// Units of work for G tiles: tile groups of T tiles (slots) x output-channel
+// tiles x K splits.  In clusters of csize >= 4 the split is a power of two that
+// divides csize, so that all splits of a tile group sit in one cluster.
+__host__ __device__ inline Sched make_sched_for(int mode, int T_max, int MT, int KC, int num_sms, int csize, int G)
 {
     Sched s;
-    const int want = max(1, (G * p.MT + p.num_sms - 1) / p.num_sms);
-    if (p.mode == 0)
-        s.T = min(p.T_max, want);
-    else if (p.mode == 2)
+    const int want = max(1, (G * MT + num_sms - 1) / num_sms);
+    if (mode == 0)
+        s.T = min(T_max, want);
+    else if (mode == 2)
         s.T = 8;
     else
-        s.T = min(p.T_max, ((want + 15) / 16) * 16);
+        s.T = min(T_max, ((want + 15) / 16) * 16);
     s.TB = (G + s.T - 1) / s.T;
-    const int KC = p.taps * p.kci;
     // split K only where each split keeps a long K loop: below that the extra
     // round trip of the partial sums costs more than the shorter loop saves
-    s.S = max(1, min(p.num_sms / max(1, s.TB * p.MT), min(KC / 8, kMaxSplit)));
-    s.units = s.TB * p.MT * s.S;
+    s.S = max(1, min(num_sms / max(1, s.TB * MT), min(KC / 8, kMaxSplit)));
+    if (csize >= 4) {
+        int q = 1;
+        while (2 * q <= min(s.S, csize))
+            q *= 2;
+        s.S = q;
+    }
+    s.units = s.TB * MT * s.S;
     return s;
+}
+
+__device__ __forceinline__ Sched make_sched(const TcArgs &p, int G)
+{
+    return make_sched_for(p.mode, p.T_max, p.MT, p.taps * p.kci, p.num_sms, p.csize, G);
 }
 
 struct Unit {
@@ -436,7 +462,7 @@ struct Carve {
     uint32_t b_base;    // byte offset of halo stage 0
     uint32_t stage_b;   // bytes per halo stage
     uint32_t red_base;  // receive buffer of the peer's partial (kRedBytes), when red
-    bool red;           // pair launch, unit of <= 64 columns, and two weight stages still fit
+    bool red;           // clusters of two, unit of <= 64 columns, and two weight stages still fit
     int SA;             // weight stages
 };
 
@@ -448,7 +474,7 @@ __device__ __forceinline__ Carve carve(const TcArgs &p, int T)
     c.a_base = kCtrlBytes;
     c.red_base = c.b_base;
     c.red = false;
-    if (p.pair && unit_cols(p, T) * 512 <= (int)kRedBytes && c.b_base >= kRedBytes + 1024) {
+    if (p.csize == 2 && unit_cols(p, T) * 512 <= (int)kRedBytes && c.b_base >= kRedBytes + 1024) {
         const uint32_t rb = (c.b_base - kRedBytes) & ~1023u;
         if (rb >= c.a_base + 2 * kAStageBytes) {
             c.red_base = rb;
@@ -562,6 +588,45 @@ __device__ __forceinline__ void fill_b(const TcArgs &c, int T, int tb, int q, in
                 ++slot;
             }
         }
+    }
+}
+
+// Fill one B stage of the slot layouts (POS and row-batched POS), whose bytes
+// run [halo pixel][channel group][slot]: 16-byte chunk `lin` of the stage sits
+// at byte 16 lin, so thread et copies chunks et, et + 256, ...  A warp then
+// writes 512 contiguous bytes of shared memory (no bank conflicts) and reads
+// 64 contiguous bytes from each of 8 tiles.  Then the GroupNorm affine and
+// SiLU are applied in place, in the same order.
+__device__ __forceinline__ void fill_b_slots(const TcArgs &c, int T, int tb, int q, int G, uint8_t *stage, int et,
+                                             const int2 *s_orig)
+{
+    const int bin = c.bin;
+    const int total = bin * bin * 8 * T;
+    const uint32_t sbase = smem_u32(stage);
+#pragma unroll 1
+    for (int lin = et; lin < total; lin += kProd) {
+        const int slot = lin % T, r = lin / T;
+        const int kc = r & 7, pix = r >> 3;
+        const int hh = pix / bin, ww = pix - hh * bin;
+        const uint8_t *src = halo_src(c, s_orig, T, tb, G, slot, hh, ww, pix, q * 64 + kc * 8);
+        cp_async16(sbase + (uint32_t)lin * 16u, src ? src : c.src, src ? 16u : 0u);
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (c.gsc == nullptr && !c.silu)
+        return;
+    const bool affine = c.gsc != nullptr;
+#pragma unroll 1
+    for (int lin = et; lin < total; lin += kProd) {
+        const int slot = lin % T, r = lin / T;
+        const int kc = r & 7, pix = r >> 3;
+        const int hh = pix / bin, ww = pix - hh * bin;
+        const int ch = q * 64 + kc * 8;
+        if (!halo_src(c, s_orig, T, tb, G, slot, hh, ww, pix, ch))
+            continue;   // zero padding stays zero
+        uint4 *d = reinterpret_cast<uint4 *>(stage + (size_t)lin * 16);
+        const int n = affine ? (tb * T + slot) % c.N : 0;
+        *d = transform16(*d, SIGE_BF16, affine ? c.gsc + (int64_t)n * c.Cin + ch : nullptr,
+                         affine ? c.gsh + (int64_t)n * c.Cin + ch : nullptr, c.silu);
     }
 }
 
@@ -692,6 +757,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     auto b_load = [&](int i) { return acc_full + 24u + 8u * i; };   // halo TMA arrivals
     const uint32_t red_full = acc_full + 40u;   // pair launches, rank 0: the peer's partial has arrived
     const uint32_t red_free = acc_full + 48u;   // pair launches, rank 1: the peer has consumed it
+    const uint32_t rs_ready = acc_full + 56u;   // reduce-scatter: every member of the group may be written
+    const uint32_t rs_full = acc_full + 64u;    // reduce-scatter: every member's slice for this CTA has landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 512);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 516);
     volatile int *bcast = abort_flag + 1;
@@ -715,6 +782,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_init(drain, 1);
         mbar_init(red_full, 1);
         mbar_init(red_free, 1);
+        // reduce-scatter: each of the S members arrives with weight csize / S
+        mbar_init(rs_ready, max(1, p.csize));
+        mbar_init(rs_full, max(1, p.csize));
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -889,34 +959,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             ok = false;
                             break;
                         }
+                        // each accumulator block takes its four K steps in one
+                        // issue block (per block the order is ks = 0..3)
                         if (p.mode == 0) {
-#pragma unroll
-                            for (int ks = 0; ks < 4; ++ks) {
-                                uint64_t bt = b_tap + ks * d_ks;
+                            uint64_t bt = b_tap;
 #pragma unroll 1
-                                for (int t = 0; t < nT; ++t, bt += d_tile)
-                                    tc_mma_w(tmem + t * 64, a_cur + 2 * ks, bt, idesc, ks ? 1u : acc0);
-                            }
+                            for (int t = 0; t < nT; ++t, bt += d_tile)
+                                tc_mma4_w(tmem + t * 64, a_cur, bt, d_ks, idesc, acc0);
                         } else if (p.mode == 2) {
-#pragma unroll
-                            for (int ks = 0; ks < 4; ++ks) {
-                                uint64_t bi = b_tap + ks * d_ks;
+                            uint64_t bi = b_tap;
+                            uint32_t col = 0;
 #pragma unroll 1
-                                for (int i = 0; i < bb; ++i, bi += d_i)
-                                    tc_mma_w(tmem + (uint32_t)(i * bb * 8), a_cur + 2 * ks, bi, idesc, ks ? 1u : acc0);
-                            }
+                            for (int i = 0; i < bb; ++i, bi += d_i, col += (uint32_t)(bb * 8))
+                                tc_mma4_w(tmem + col, a_cur, bi, d_ks, idesc, acc0);
                         } else {
-#pragma unroll
-                            for (int ks = 0; ks < 4; ++ks) {
-                                uint64_t bi = b_tap + ks * d_ks;
-                                uint32_t col = 0;
+                            uint64_t bi = b_tap;
+                            uint32_t col = 0;
 #pragma unroll 1
-                                for (int i = 0; i < bb; ++i, bi += d_i) {
-                                    uint64_t bj = bi;
+                            for (int i = 0; i < bb; ++i, bi += d_i) {
+                                uint64_t bj = bi;
 #pragma unroll 1
-                                    for (int j = 0; j < bb; ++j, bj += d_j, col += nT)
-                                        tc_mma_w(tmem + col, a_cur + 2 * ks, bj, idesc, ks ? 1u : acc0);
-                                }
+                                for (int j = 0; j < bb; ++j, bj += d_j, col += nT)
+                                    tc_mma4_w(tmem + col, a_cur, bj, d_ks, idesc, acc0);
                             }
                         }
                         acc0 = 1;
@@ -985,6 +1049,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             return r;
         };
         uint32_t pit = 0;   // pair units done (phase of red_full / red_free)
+        uint32_t rsit = 0;  // reduce-scatter units done (phase of rs_ready / rs_full)
         // output vectors: 8 bf16 channels (16 per 128-channel column) or 4 floats (32)
         const int vpc = (c.to_y && c.dtype == SIGE_BF16) ? 16 : 32;
         const int cpv = 128 / vpc;          // channels per vector
@@ -1056,7 +1121,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         }
                         transform_b(c, sc.T, un.tb, q, G, stage, et, s_orig, gsc, gsh);
                     } else {
-                        fill_b(c, sc.T, un.tb, q, G, stage, et, s_orig);
+                        if (p.mode == 0)
+                            fill_b(c, sc.T, un.tb, q, G, stage, et, s_orig);
+                        else
+                            fill_b_slots(c, sc.T, un.tb, q, G, stage, et, s_orig);
                     }
                     fence_async_smem();
                     mbar_arrive(b_full(sb));
@@ -1080,6 +1148,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // rank 1 sends its partial, rank 0 adds it and writes the output
             const bool pair = cv.red && sc.S == 2;
             const uint32_t rank = pair ? cluster_rank() : 0u;
+            // other K splits that divide the cluster: reduce-scatter among the
+            // S CTAs of the tile group (consecutive ranks of one cluster), the
+            // slices staged in the halo stages, which are free by then
+            const bool rs = !pair && sc.S >= 2 && p.csize >= 2 && p.csize % sc.S == 0 && (ncols / sc.S) % 4 == 0 &&
+                            (uint32_t)ncols * 512u <= (uint32_t)p.SB * cv.stage_b;
             // rank 0 (or an unsplit unit of one batch of items): the residual of
             // this thread's items is read while the MMAs run
             const bool pre = (pair ? rank == 0 : sc.S == 1 && ncols <= stage_cols) && ncols * vpc <= 4 * kProd &&
@@ -1094,7 +1167,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (pre && e_pre[k] >= 0)
                     rr_pre[k] = __ldg(reinterpret_cast<const uint4 *>(c.residual + e_pre[k] * (c.dtype == SIGE_BF16 ? 2 : 4)));
             }
-            if (pair && !cwaited) {
+            if ((pair || rs) && !cwaited) {
                 cluster_wait();
                 cwaited = true;
             }
@@ -1178,6 +1251,96 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (et == 0)
                     mbar_arrive_peer(map_peer(red_free, 1));
                 ++pit;
+            } else if (rs) {
+                // Every member sends column slice q of its partial to member q,
+                // into q's halo stages laid out [member][128 channels][w (+4)]
+                // floats (16-byte remote stores of 4 columns); each member sums
+                // its slice in member order and writes it.
+                const uint32_t S = (uint32_t)sc.S;
+                const uint32_t crank = cluster_rank();
+                const uint32_t me = crank % S, g0 = crank - me;
+                const uint32_t share = (uint32_t)p.csize / S;
+                const int w = ncols / (int)S;
+                // row stride: 4 floats of padding when they fit keep the
+                // 16-byte accesses of a warp free of bank conflicts
+                const int rsw = (uint32_t)(ncols + 4 * (int)S) * 512u <= (uint32_t)p.SB * cv.stage_b ? w + 4 : w;
+                const uint32_t rb = sbase + cv.b_base;
+                float *slab = reinterpret_cast<float *>(smem + cv.b_base);
+                // this CTA's MMAs are complete: its halo stages may be written
+                if (et == 0) {
+#pragma unroll 1
+                    for (uint32_t q = 0; q < S; ++q)
+                        mbar_arrive_peer_n(map_peer(rs_ready, g0 + q), share);
+                }
+                if (!group_wait_c(rs_ready, rsit & 1, 11)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t my_row = rb + (uint32_t)(((int)me * 128 + row) * rsw * 4);
+#pragma unroll 1
+                for (int c0 = 16 * half; c0 < ncols; c0 += 32) {
+                    float v[16];
+                    tmem_ld16(tbase + c0, v);
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const int col = c0 + 4 * k4;
+                        const int q = col / w, off = col - q * w;   // w % 4 == 0: 4 columns, one owner
+                        st_peer_f32x4(map_peer(my_row + (uint32_t)off * 4u, g0 + (uint32_t)q), v[4 * k4],
+                                      v[4 * k4 + 1], v[4 * k4 + 2], v[4 * k4 + 3]);
+                    }
+                }
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+                if (et == 0) {
+#pragma unroll 1
+                    for (uint32_t q = 0; q < S; ++q)
+                        mbar_arrive_peer_n(map_peer(rs_full, g0 + q), share);
+                }
+                if (!group_wait_c(rs_full, rsit & 1, 12)) {
+                    ok = false;
+                    break;
+                }
+                // fixed member order: the sum does not depend on arrival order
+#pragma unroll 1
+                for (int j = 4 * half; j < w; j += 8) {
+                    float4 *d = reinterpret_cast<float4 *>(slab + row * rsw + j);
+                    float4 acc = *d;
+#pragma unroll 1
+                    for (uint32_t s2 = 1; s2 < S; ++s2) {
+                        const float4 t = *reinterpret_cast<const float4 *>(slab + ((int)s2 * 128 + row) * rsw + j);
+                        acc.x += t.x;
+                        acc.y += t.y;
+                        acc.z += t.z;
+                        acc.w += t.w;
+                    }
+                    *d = acc;
+                }
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+#pragma unroll 1
+                for (int it0 = et; it0 < w * vpc; it0 += 4 * kProd) {
+                    int64_t e[4];
+                    uint4 rr[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int it = it0 + k * kProd;
+                        e[k] = (it < w * vpc && write_ok)
+                                   ? col_target(c, s_orig, sc.T, un.tb, G, (int)me * w + it / vpc, co0) : -1;
+                        rr[k] = make_uint4(0, 0, 0, 0);
+                        if (e[k] >= 0 && c.residual && c.to_y)
+                            rr[k] = __ldg(reinterpret_cast<const uint4 *>(c.residual + e[k] * (c.dtype == SIGE_BF16 ? 2 : 4)));
+                    }
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        if (e[k] < 0)
+                            continue;
+                        const int col = (it0 + k * kProd) / vpc;
+                        float v[8];
+#pragma unroll
+                        for (int m = 0; m < 8; ++m)
+                            v[m] = m < cpv ? slab[(cg * cpv + m) * rsw + col] : 0.0f;
+                        store_vec(c, e[k], v, bias8, rr[k]);
+                    }
+                }
+                ++rsit;
             } else if (sc.S == 1) {
                 // accumulator -> shared staging (column-major, 128 floats per
                 // column) -> 16-byte vectors per pixel
@@ -1476,10 +1639,20 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
     p.counters = reinterpret_cast<uint32_t *>(ws);
     p.partials = reinterpret_cast<float *>(ws + ((p.num_sms * 4 + 255) / 256) * 256);
 
-    // per device: attribute set, co-resident clusters of two (0 = not yet
-    // known, -1 = none); concurrent first calls compute the same values
+    // Cluster size: 4 where the K split may reach 4 (so that it can
+    // reduce-scatter within the cluster), else 2.  The split is decided on the
+    // device from the tile count; the bound below is its value for one tile
+    // (the largest), or the exact value for a dense launch.
+    const int KC = p.taps * p.kci;
+    const int G_hint = cp.dense ? cp.tiles_total * cp.N : 1;
+    const Sched s_hint = make_sched_for(p.mode, p.T_max, p.MT, KC, p.num_sms, 1, std::max(1, G_hint));
+    const int want_c = s_hint.S >= 4 ? 4 : 2;
+
+    // per device: attribute set, co-resident clusters of 2 and of 4 CTAs (0 =
+    // not yet known, -1 = none); concurrent first calls compute the same values
     static std::atomic<int> smem_set[64];
     static std::atomic<int> pair_clusters[64];
+    static std::atomic<int> quad_clusters[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64)
@@ -1501,33 +1674,45 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
     cfg.dynamicSmemBytes = kSmemLimit;
     cfg.stream = stream;
     cfg.attrs = attr;
-    if (!pair_clusters[dev].load(std::memory_order_acquire)) {
-        int n = 0;
-        cfg.gridDim = dim3(2 * ((p.num_sms + 1) / 2));
-        cfg.numAttrs = 2;
-        if (cudaOccupancyMaxActiveClusters(&n, k_conv_tc, &cfg) != cudaSuccess || n < 1) {
-            cudaGetLastError();
-            n = -1;
+    auto clusters_of = [&](int csz, std::atomic<int> &slot) {
+        if (!slot.load(std::memory_order_acquire)) {
+            int n = 0;
+            attr[1].val.clusterDim.x = csz;
+            cfg.gridDim = dim3(csz * ((p.num_sms + csz - 1) / csz));
+            cfg.numAttrs = 2;
+            if (cudaOccupancyMaxActiveClusters(&n, k_conv_tc, &cfg) != cudaSuccess || n < 1) {
+                cudaGetLastError();
+                n = -1;
+            }
+            slot.store(n, std::memory_order_release);
         }
-        pair_clusters[dev].store(n, std::memory_order_release);
-    }
-    // clusters of two CTAs (a 2-way K split then sums through the peer's
-    // shared memory), as many as are co-resident; otherwise one CTA per SM
+        return slot.load(std::memory_order_acquire);
+    };
+    // clusters of csize CTAs, as many as are co-resident; otherwise one CTA per SM
     cudaError_t e = cudaErrorUnknown;
-    const int clusters = pair_clusters[dev].load(std::memory_order_acquire);
-    if (clusters > 0) {
+    const int sms = p.num_sms;
+    for (int csz : {want_c, 2}) {
+        if (csz == 4 && want_c != 4)
+            continue;
+        const int clusters = clusters_of(csz, csz == 4 ? quad_clusters[dev] : pair_clusters[dev]);
+        if (clusters <= 0)
+            continue;
         p.pair = 1;
-        p.num_sms = 2 * std::min(clusters, p.num_sms / 2);
+        p.csize = csz;
+        p.num_sms = csz * std::min(clusters, sms / csz);
+        attr[1].val.clusterDim.x = csz;
         cfg.gridDim = dim3(p.num_sms);
         cfg.numAttrs = 2;
         e = cudaLaunchKernelEx(&cfg, k_conv_tc, p, map, xmap);
-        if (e != cudaSuccess) {
-            cudaGetLastError();
-            pair_clusters[dev].store(-1, std::memory_order_release);
-        }
+        if (e == cudaSuccess)
+            break;
+        cudaGetLastError();
+        (csz == 4 ? quad_clusters[dev] : pair_clusters[dev]).store(-1, std::memory_order_release);
+        p.num_sms = sms;
     }
     if (e != cudaSuccess) {
         p.pair = 0;
+        p.csize = 1;
         p.num_sms = device_sm_count();
         e = launch_pdl(k_conv_tc, dim3(p.num_sms), dim3(kTcThreads), kSmemLimit, stream, p, map, xmap);
     }

@@ -240,6 +240,16 @@ def test_fused_cfg5_all_ones_equals_dense(orc, layer):
     assert_close(y.cpu(), ref, torch.bfloat16)
 
 
+@pytest.mark.parametrize("block,stride,N", [(4, 1, 1), (4, 1, 2), (2, 1, 2), (3, 1, 1), (4, 2, 1)])
+def test_fused_gn_slot_layouts(orc, block, stride, N):
+    # GroupNorm affine + SiLU applied while the halo is staged in the slot
+    # layouts (row-batched POS for even b, POS otherwise), batch 1 and 2,
+    # with a residual; K = 9 x 256 is long enough to be split
+    L = inputs.make_conv_case(40 + block + N, 36, 28, 256, 128, dtype=torch.bfloat16, block=block,
+                              stride=stride, area=0.08, gn=True, N=N)
+    _fused_vs_oracle(orc, L, _tiles(orc, L), residual=True)
+
+
 def test_fused_ragged_edges_and_batch(orc):
     L = inputs.make_conv_case(25, 30, 26, 64, 64, dtype=torch.bfloat16, block=8, area=0.1, gn=True, N=2)
     _fused_vs_oracle(orc, L, _tiles(orc, L), residual=True)

@@ -269,6 +269,29 @@ int sige_get_error(void *workspace, sige_stream_t stream);
  * cores, 0 = CUDA cores; negative = a sige_status for an unsupported layer. */
 int sige_conv_path(const sige_conv_desc *cd, int32_t dtype);
 
+/* Work decomposition of the tensor-core conv kernel for a bf16 layer, computed
+ * on the host (no device work, no GPU needed): the same functions the kernel
+ * runs at launch.  The active tiles are split into tile groups of T tiles
+ * (slots), one unit per (tile group, 128 output channels, K split); a unit's S
+ * K-splits are summed through a cluster peer (pair), by a reduce-scatter among
+ * the S CTAs of one cluster, or through global memory (SIGE tile-based sparse
+ * convolution, "Sparse Engine SIGE"; the split is this implementation's).
+ *   tiles   : active tiles times batch (G), >= 0
+ *   grid    : CTAs of the launch, a multiple of `cluster`
+ *   cluster : CTAs per cluster (1 = no clusters)
+ *   out     : host int32[n_out], filled with (missing entries 0):
+ *             [0] B layout (0 ROW, 1 POS, 2 row-batched POS), [1] T, [2] tile
+ *             groups, [3] K splits S, [4] units, [5] split sum (0 none, 1 pair,
+ *             2 cluster reduce-scatter, 3 global), [6] accumulator columns of a
+ *             unit, [7] weight stages, [8] halo stage bytes, [9] bytes the
+ *             reduce-scatter stages (unpadded), [10] output-channel tiles,
+ *             [11] 64-channel k-chunks, [12] cluster size a sparse launch asks
+ *             for, [13] byte offset of the halo stages, [14] usable shared bytes
+ * Returns SIGE_ERR_UNSUPPORTED for layers the tensor-core kernel does not run,
+ * SIGE_ERR_INVALID_ARG for bad sizes. */
+int sige_conv_schedule(const sige_conv_desc *cd, int32_t tiles, int32_t grid, int32_t cluster,
+                       int32_t *out, int32_t n_out);
+
 /* Number of kernels this library has launched in this process. */
 uint64_t sige_launch_count(void);
 

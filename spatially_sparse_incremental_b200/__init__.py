@@ -64,6 +64,7 @@ SIGNATURES = {
     "sige_conv_workspace_bytes": (_sz, [_CD, _i32, _i32, _i32, _i32]),
     "sige_get_error": (_i32, [_vp, _vp]),
     "sige_conv_path": (_i32, [_CD, _i32]),
+    "sige_conv_schedule": (_i32, [_CD, _i32, _i32, _i32, _vp, _i32]),
     "sige_launch_count": (ctypes.c_uint64, []),
     "sige_status_string": (ctypes.c_char_p, [_i32]),
 }
@@ -299,6 +300,21 @@ def sige_get_error(workspace, stream=None) -> int:
 
 def sige_conv_path(cd: ConvDesc, dtype: torch.dtype) -> int:
     return int(lib().sige_conv_path(ctypes.byref(cd), _DT[dtype]))
+
+
+SCHEDULE_FIELDS = ("layout", "T", "tile_groups", "splits", "units", "split_sum", "unit_cols", "weight_stages",
+                   "halo_bytes", "reduce_scatter_bytes", "cout_tiles", "k_chunks", "cluster_for_sparse",
+                   "halo_offset", "smem_bytes")
+
+
+def sige_conv_schedule(cd: ConvDesc, tiles: int, grid: int, cluster: int) -> dict:
+    """Work decomposition of the tensor-core conv for ``tiles`` active tiles
+    (times batch) on a launch of ``grid`` CTAs in clusters of ``cluster``;
+    host-only.  Keys are SCHEDULE_FIELDS."""
+    out = (ctypes.c_int32 * len(SCHEDULE_FIELDS))()
+    _check(lib().sige_conv_schedule(ctypes.byref(cd), int(tiles), int(grid), int(cluster),
+                                    ctypes.cast(out, ctypes.c_void_p), len(SCHEDULE_FIELDS)), "sige_conv_schedule")
+    return dict(zip(SCHEDULE_FIELDS, (int(v) for v in out)))
 
 
 def sige_launch_count() -> int:

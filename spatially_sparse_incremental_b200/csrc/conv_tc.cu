@@ -452,7 +452,7 @@ __device__ __forceinline__ Unit decode_unit(const TcArgs &p, const Sched &s, int
 //                    staging buffer once the unit's MMAs are complete
 
 // Accumulator columns of a unit of T tiles (ROW) or T slots (POS).
-__device__ __forceinline__ int unit_cols(const TcArgs &p, int T)
+__host__ __device__ inline int unit_cols(const TcArgs &p, int T)
 {
     return p.mode == 0 ? T * 64 : p.b * p.b * T;
 }
@@ -466,7 +466,7 @@ struct Carve {
     int SA;             // weight stages
 };
 
-__device__ __forceinline__ Carve carve(const TcArgs &p, int T)
+__host__ __device__ inline Carve carve(const TcArgs &p, int T)
 {
     Carve c;
     c.stage_b = (uint32_t)T * p.per_slot;
@@ -483,6 +483,25 @@ __device__ __forceinline__ Carve carve(const TcArgs &p, int T)
     }
     c.SA = min(kMaxSA, (int)((c.red_base - c.a_base) / kAStageBytes));
     return c;
+}
+
+// How the K splits of a unit are summed (the same for every CTA of a launch).
+enum : int { kSplitNone = 0, kSplitPair = 1, kSplitCluster = 2, kSplitGlobal = 3 };
+
+__host__ __device__ inline int split_kind(const TcArgs &p, const Sched &sc, const Carve &cv)
+{
+    const int ncols = unit_cols(p, sc.T);
+    if (sc.S == 1)
+        return kSplitNone;
+    // 2-way split through the cluster peer's receive buffer
+    if (cv.red && sc.S == 2)
+        return kSplitPair;
+    // reduce-scatter among the S CTAs of the tile group (consecutive ranks of
+    // one cluster), the slices staged in the halo stages, which are free by then
+    if (p.csize >= 2 && p.csize % sc.S == 0 && (ncols / sc.S) % 4 == 0 &&
+        (uint32_t)ncols * 512u <= (uint32_t)p.SB * cv.stage_b)
+        return kSplitCluster;
+    return kSplitGlobal;
 }
 
 // ------------------------------------------------------------------ B staging
@@ -1146,13 +1165,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const bool write_ok = co0 < c.Cout;
             // 2-way K split summed through the cluster peer's shared memory:
             // rank 1 sends its partial, rank 0 adds it and writes the output
-            const bool pair = cv.red && sc.S == 2;
+            const int skind = split_kind(p, sc, cv);
+            const bool pair = skind == kSplitPair;
             const uint32_t rank = pair ? cluster_rank() : 0u;
-            // other K splits that divide the cluster: reduce-scatter among the
-            // S CTAs of the tile group (consecutive ranks of one cluster), the
-            // slices staged in the halo stages, which are free by then
-            const bool rs = !pair && sc.S >= 2 && p.csize >= 2 && p.csize % sc.S == 0 && (ncols / sc.S) % 4 == 0 &&
-                            (uint32_t)ncols * 512u <= (uint32_t)p.SB * cv.stage_b;
+            const bool rs = skind == kSplitCluster;
             // rank 0 (or an unsplit unit of one batch of items): the residual of
             // this thread's items is read while the MMAs run
             const bool pre = (pair ? rank == 0 : sc.S == 1 && ncols <= stage_cols) && ncols * vpc <= 4 * kProd &&
@@ -1558,6 +1574,57 @@ bool tc_supported(const sige_conv_desc *cd, int dtype)
     return plan_layer(cd, pl);
 }
 
+// Schedule fields of the argument block that depend only on the layer and
+// its plan (the launch adds the buffers and the grid).
+static void plan_args(const sige_conv_desc *cd, const TcPlan &pl, TcArgs &p)
+{
+    p.k = cd->kernel;
+    p.s = cd->stride;
+    p.b = cd->block;
+    p.bin = (cd->block - 1) * cd->stride + cd->kernel;
+    p.mode = pl.mode;
+    p.taps = cd->kernel * cd->kernel;
+    p.kci = cd->c_in / 64;
+    p.MT = (cd->c_out + 127) / 128;
+    p.T_max = pl.T_max;
+    p.SB = pl.SB;
+    p.per_slot = pl.per_slot;
+    p.smem_bytes = kSmemLimit - 1024;   // usable after aligning the base to 1024
+    p.ncols = pl.ncols;
+}
+
+// Cluster size for a launch: 4 where the K split may reach 4 (so that it can
+// reduce-scatter within the cluster), else 2.  The split is decided on the
+// device from the tile count; G_hint = 1 gives its largest value (sparse
+// launches), the full tile count its exact value (dense launches).
+static int preferred_cluster(const TcArgs &p, int G_hint, int sms)
+{
+    const Sched s = make_sched_for(p.mode, p.T_max, p.MT, p.taps * p.kci, sms, 1, std::max(1, G_hint));
+    return s.S >= 4 ? 4 : 2;
+}
+
+int tc_schedule(const sige_conv_desc *cd, int tiles, int grid, int csize, int32_t *out, int n_out)
+{
+    TcPlan pl;
+    if (!cd || !out || n_out < 1 || tiles < 0 || grid < 1 || csize < 1 || grid % csize != 0 || !plan_layer(cd, pl))
+        return SIGE_ERR_INVALID_ARG;
+    TcArgs p{};
+    plan_args(cd, pl, p);
+    p.num_sms = grid;
+    p.csize = csize;
+    p.pair = csize >= 2;
+    const Sched sc = make_sched_for(p.mode, p.T_max, p.MT, p.taps * p.kci, grid, csize, tiles);
+    const Carve cv = carve(p, sc.T);
+    const int ncols = unit_cols(p, sc.T);
+    const int32_t v[] = {p.mode, sc.T, sc.TB, sc.S, sc.units, split_kind(p, sc, cv), ncols, cv.SA,
+                         (int32_t)(p.SB * cv.stage_b), ncols * 512, p.MT, p.taps * p.kci,
+                         preferred_cluster(p, 1, grid), (int32_t)cv.b_base, (int32_t)p.smem_bytes};
+    const int n = (int)(sizeof(v) / sizeof(v[0]));
+    for (int i = 0; i < n_out; ++i)
+        out[i] = i < n ? v[i] : 0;
+    return SIGE_OK;
+}
+
 size_t tc_workspace_bytes(const sige_conv_desc *cd, int batch, int ntiles)
 {
     (void)batch;
@@ -1625,28 +1692,13 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
     p.k = cp.k; p.s = cp.s; p.pad = cp.pad; p.b = cp.b; p.bin = cp.bin; p.Ho = cp.Ho; p.Wo = cp.Wo;
     p.cap = cp.cap; p.dense = cp.dense; p.tiles_w = cp.tiles_w; p.tiles_total = cp.tiles_total;
     p.silu = cp.silu; p.from_image = cp.from_image; p.to_y = cp.to_y;
-    p.mode = pl.mode;
-    p.taps = cp.k * cp.k;
-    p.kci = cp.Cin / 64;
-    p.MT = (cp.Cout + 127) / 128;
-    p.T_max = pl.T_max;
-    p.SB = pl.SB;
-    p.per_slot = pl.per_slot;
-    p.smem_bytes = kSmemLimit - 1024;   // usable after aligning the base to 1024
-    p.ncols = pl.ncols;
+    plan_args(&cd, pl, p);
     p.num_sms = device_sm_count();
     uint8_t *ws = cp.ws + kWsHeader;
     p.counters = reinterpret_cast<uint32_t *>(ws);
     p.partials = reinterpret_cast<float *>(ws + ((p.num_sms * 4 + 255) / 256) * 256);
 
-    // Cluster size: 4 where the K split may reach 4 (so that it can
-    // reduce-scatter within the cluster), else 2.  The split is decided on the
-    // device from the tile count; the bound below is its value for one tile
-    // (the largest), or the exact value for a dense launch.
-    const int KC = p.taps * p.kci;
-    const int G_hint = cp.dense ? cp.tiles_total * cp.N : 1;
-    const Sched s_hint = make_sched_for(p.mode, p.T_max, p.MT, KC, p.num_sms, 1, std::max(1, G_hint));
-    const int want_c = s_hint.S >= 4 ? 4 : 2;
+    const int want_c = preferred_cluster(p, cp.dense ? cp.tiles_total * cp.N : 1, p.num_sms);
 
     // per device: attribute set, co-resident clusters of 2 and of 4 CTAs (0 =
     // not yet known, -1 = none); concurrent first calls compute the same values

@@ -8,5 +8,6 @@ namespace sige {
 bool tc_supported(const sige_conv_desc *cd, int dtype);
 size_t tc_workspace_bytes(const sige_conv_desc *cd, int batch, int ntiles);
 int launch_conv_tc(const ConvParams &p, cudaStream_t stream);
+int tc_schedule(const sige_conv_desc *cd, int tiles, int grid, int csize, int32_t *out, int n_out);
 
 } // namespace sige

@@ -100,6 +100,14 @@ extern "C" int sige_conv_path(const sige_conv_desc *cd, int32_t dtype)
     return choose_path(cd, dtype);
 }
 
+extern "C" int sige_conv_schedule(const sige_conv_desc *cd, int32_t tiles, int32_t grid, int32_t cluster,
+                                  int32_t *out, int32_t n_out)
+{
+    if (check_layer(cd, SIGE_BF16) != SIGE_OK || !tc_supported(cd, SIGE_BF16))
+        return SIGE_ERR_UNSUPPORTED;
+    return tc_schedule(cd, tiles, grid, cluster, out, n_out);
+}
+
 extern "C" int sige_sparse_conv(const void *blocks, const sige_conv_desc *cd, int32_t dtype, int32_t batch,
                                 const void *weight, const int32_t *count, int32_t capacity,
                                 float *out_blocks, void *workspace, size_t workspace_bytes,

@@ -31,6 +31,11 @@ one that matches the conv path:
 Normalisation layers before the attention (LayerNorm / GroupNorm of the
 transformer block) are not part of this function; they are per-token and would
 be applied to x and the context before it.
+
+Storage precision.  With ``storage=torch.bfloat16`` the projections q, k, v and
+the attention output o (before Wo) are each rounded once to bf16, as a chain
+that stores them between its steps does; everything else stays float64.  With
+``storage=None`` nothing is rounded before the end.
 """
 from __future__ import annotations
 
@@ -80,8 +85,19 @@ def attention_core(q: np.ndarray, k: np.ndarray, v: np.ndarray, heads: int) -> n
     return out
 
 
+def _stored(a: np.ndarray, storage) -> np.ndarray:
+    """`a` rounded once to the storage dtype (bf16: ties to even, straight
+    from double), back in float64; unchanged when storage is None."""
+    if storage is None:
+        return a
+    if storage != torch.bfloat16:
+        raise ValueError("storage must be None or torch.bfloat16")
+    from oracle import bf16_bits_to_f64, round_bf16
+    return bf16_bits_to_f64(round_bf16(a)).reshape(a.shape)
+
+
 def sparse_attention_f64(x_edit, idx: np.ndarray, block: int, wq, wk, wv, wo, bo=None, heads: int = 1,
-                         context=None, residual=None):
+                         context=None, residual=None, storage=None):
     """The active tokens' outputs in float64 (before rounding).
 
     x_edit [N, H, W, C] (edited feature map), wq [C, D], wk [Ck, D], wv [Ck, Dv],
@@ -99,10 +115,10 @@ def sparse_attention_f64(x_edit, idx: np.ndarray, block: int, wq, wk, wv, wo, bo
     for n in range(N):
         seq = x[n].reshape(H * W, C)
         src = seq if ctx is None else ctx[n]
-        k = src @ Wk
-        v = src @ Wv
-        q = seq[tok] @ Wq
-        o = attention_core(q, k, v, heads) @ Wo + b
+        k = _stored(src @ Wk, storage)
+        v = _stored(src @ Wv, storage)
+        q = _stored(seq[tok] @ Wq, storage)
+        o = _stored(attention_core(q, k, v, heads), storage) @ Wo + b
         if res is not None:
             o = o + res[n].reshape(H * W, -1)[tok]
         vals[n] = o
@@ -120,16 +136,29 @@ def _round_to(vals: np.ndarray, dtype: torch.dtype) -> torch.Tensor:
 
 
 def sparse_attention(x_edit, out_cached: torch.Tensor, idx: np.ndarray, block: int, wq, wk, wv, wo, bo=None,
-                     heads: int = 1, context=None, residual=None) -> torch.Tensor:
+                     heads: int = 1, context=None, residual=None, storage=None) -> torch.Tensor:
     """Cached output [N, H, W, Co] with the active tokens recomputed and rounded
     once to its dtype; every other element is the cached one."""
-    tok, vals = sparse_attention_f64(x_edit, idx, block, wq, wk, wv, wo, bo, heads, context, residual)
+    tok, vals = sparse_attention_f64(x_edit, idx, block, wq, wk, wv, wo, bo, heads, context, residual, storage)
     out = out_cached.clone()
     N, H, W, Co = out.shape
     flat = out.view(N, H * W, Co)
     if len(tok):
         flat[:, torch.from_numpy(tok)] = _round_to(vals, out.dtype)
     return out
+
+
+def attention_core_tokens(q, k, v, heads: int, idx: np.ndarray, block: int, H: int, W: int):
+    """The attention step alone on stored projections: q [N, H, W, D] (read at
+    the active tokens), k [N, Lk, D], v [N, Lk, Dv].  Returns (tokens, o) with
+    o [N, len, Dv] in float64 (before rounding)."""
+    Q, K, V = _f64(q), _f64(k), _f64(v)
+    N = Q.shape[0]
+    tok = active_tokens(idx, block, H, W)
+    o = np.empty((N, len(tok), V.shape[2]), dtype=np.float64)
+    for n in range(N):
+        o[n] = attention_core(Q[n].reshape(H * W, -1)[tok], K[n], V[n], heads)
+    return tok, o
 
 
 def dense_attention(x, wq, wk, wv, wo, bo=None, heads: int = 1, context=None, residual=None,

@@ -138,3 +138,45 @@ def test_dense_attention_is_the_full_list():
     cache = torch.zeros((N, H, W, wo.shape[1]), dtype=torch.bfloat16)
     full = att.sparse_attention(x, cache, _all_tiles(H, W, 2), 2, wq, wk, wv, wo, bo, 2)
     assert torch.equal(bits(dense), bits(full))
+
+
+def test_bf16_storage_rounds_q_k_v_and_o_once():
+    # library composition with the same rounding points (q, k, v, o to bf16,
+    # ties to even): element-wise equal to float64 noise except where a value
+    # of o sits on a bf16 rounding boundary (then within one bf16 ulp of o
+    # carried through Wo)
+    import oracle
+    rb = lambda a: oracle.bf16_bits_to_f64(oracle.round_bf16(a)).reshape(np.shape(a))
+    x, wq, wk, wv, wo, bo, _, res = _case(12, H=6, W=6)
+    N, H, W, C = x.shape
+    heads = 4
+    _, got = att.sparse_attention_f64(x, _all_tiles(H, W, 3), 3, wq, wk, wv, wo, bo, heads, residual=res,
+                                      storage=torch.bfloat16)
+    t = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+    seq = x.reshape(N, H * W, C)
+    q, k, v = t(rb(seq @ wq)), t(rb(seq @ wk)), t(rb(seq @ wv))
+    split = lambda a: a.reshape(N, H * W, heads, -1).transpose(1, 2)
+    o = F.scaled_dot_product_attention(split(q), split(k), split(v)).transpose(1, 2).reshape(N, H * W, -1)
+    o = rb(o.numpy())
+    ref = o @ wo + bo + res.reshape(N, H * W, -1)
+    bound = 2.0 ** -8 * (np.abs(o) @ np.abs(wo)) + 1e-12
+    assert np.all(np.abs(got - ref) <= bound)
+    exact = np.abs(got - ref) <= 1e-12 * np.abs(ref).max()
+    assert exact.mean() >= 0.99
+    # and the storage rounding is visible: float64 storage differs
+    _, plain = att.sparse_attention_f64(x, _all_tiles(H, W, 3), 3, wq, wk, wv, wo, bo, heads, residual=res)
+    assert np.abs(plain - got).max() > 1e-6
+
+
+def test_core_on_stored_projections_equals_library():
+    rng = np.random.default_rng(13)
+    N, H, W, D, Dv, Lk, heads = 2, 5, 7, 32, 48, 19, 4
+    q, k, v = rng.normal(size=(N, H, W, D)), rng.normal(size=(N, Lk, D)), rng.normal(size=(N, Lk, Dv))
+    idx = np.array([[0, 0], [2, 4], [4, 6]], dtype=np.int32)
+    tok, o = att.attention_core_tokens(q, k, v, heads, idx, 2, H, W)
+    assert np.array_equal(tok, att.active_tokens(idx, 2, H, W))
+    t = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+    split = lambda a, L: a.reshape(N, L, heads, -1).transpose(1, 2)
+    ref = F.scaled_dot_product_attention(split(t(q).reshape(N, H * W, D), H * W), split(t(k), Lk), split(t(v), Lk))
+    ref = ref.transpose(1, 2).reshape(N, H * W, Dv).numpy()[:, tok]
+    assert np.abs(o - ref).max() <= 1e-12 * np.abs(ref).max()

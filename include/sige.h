@@ -253,6 +253,30 @@ int sige_groupnorm_affine(const void *x, const sige_tensor_desc *xd, int32_t gro
 int sige_restore_tiles(const void *src, void *dst, const sige_tensor_desc *d, int32_t block,
                        const int32_t *idx, const int32_t *count, int32_t capacity, sige_stream_t stream);
 
+/* (8) Attention step with pruned query tokens (nubint.ai review of the SIGE
+ * paper, "Proposed method": attention layers by pruning the query tokens of
+ * unedited regions; mer.dev notes, abstract: attention for Stable Diffusion).
+ * For every token (pixel) under the first min(*count, capacity) tiles of
+ * `idx` (block x block, clipped to the map), per head h:
+ *   o[n][y][x][h*dvh : (h+1)*dvh] = softmax(q_h k_h^T / sqrt(dh)) v_h
+ * over all `keys` keys, dh = qd->c / heads, dvh = dv / heads; float32
+ * arithmetic, one rounding to bf16.  Every other element of o is left as it
+ * is.  The projections before and after are sparse 1x1 convolutions
+ * (sige_conv_fused) on the same tile list.
+ *   q     : device bf16 [N][H][W][D], described by qd (NHWC); read at the tokens
+ *   k     : device bf16 [N][keys][D] (self-attention: the [N][H][W][D] key map)
+ *   v     : device bf16 [N][keys][dv]
+ *   idx, count, capacity, block : the tile list of this resolution (as (1))
+ *   o     : device bf16 [N][H][W][dv], written at the tokens only; must not
+ *           overlap q, k or v
+ * All buffers belong to the caller; nothing is allocated; asynchronous on
+ * `stream`.  Errors: SIGE_ERR_INVALID_ARG (NULL pointer, non-positive size,
+ * D or dv not a multiple of heads), SIGE_ERR_UNSUPPORTED (not bf16 NHWC,
+ * block > 8, dh or dvh > 256), SIGE_ERR_CUDA (launch failure). */
+int sige_attention_core(const void *q, const sige_tensor_desc *qd, const void *k, const void *v, int32_t keys,
+                        int32_t dv, int32_t heads, const int32_t *idx, const int32_t *count, int32_t capacity,
+                        int32_t block, void *o, sige_stream_t stream);
+
 /* ------------------------------------------------------------ utilities */
 
 /* Workspace bytes for sige_sparse_conv / sige_conv_fused / sige_dense_conv

@@ -65,6 +65,7 @@ SIGNATURES = {
     "sige_get_error": (_i32, [_vp, _vp]),
     "sige_conv_path": (_i32, [_CD, _i32]),
     "sige_conv_schedule": (_i32, [_CD, _i32, _i32, _i32, _vp, _i32]),
+    "sige_attention_core": (_i32, [_vp, _TD, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp]),
     "sige_launch_count": (ctypes.c_uint64, []),
     "sige_status_string": (ctypes.c_char_p, [_i32]),
 }
@@ -300,6 +301,57 @@ def sige_get_error(workspace, stream=None) -> int:
 
 def sige_conv_path(cd: ConvDesc, dtype: torch.dtype) -> int:
     return int(lib().sige_conv_path(ctypes.byref(cd), _DT[dtype]))
+
+
+def sige_attention_core(q, k, v, heads: int, idx, count, capacity: int, block: int, o=None, stream=None):
+    """Attention at the tokens under the tile list: q [N, H, W, D] bf16, k
+    [N, Lk, D], v [N, Lk, Dv] (a [N, H, W, *] map is viewed as [N, H*W, *]),
+    o [N, H, W, Dv] written at those tokens only (zeros elsewhere when
+    allocated here)."""
+    N, H, W, D = q.shape
+    kk = k.reshape(N, -1, D)
+    vv = v.reshape(N, kk.shape[1], -1)
+    if o is None:
+        o = torch.zeros((N, H, W, vv.shape[2]), dtype=q.dtype, device=q.device)
+    qd = tensor_desc(q)
+    st = lib().sige_attention_core(_ptr(q), ctypes.byref(qd), _ptr(kk), _ptr(vv), int(kk.shape[1]),
+                                   int(vv.shape[2]), int(heads), _ptr(idx), _ptr(count), int(capacity), int(block),
+                                   _ptr(o), _stream(stream))
+    _check(st, "sige_attention_core")
+    return o
+
+
+def sige_attention_sparse(x, idx, count, capacity: int, block: int, wq, wo, bo, heads: int, k_map, v_map, y,
+                          wk=None, wv=None, residual=None, workspace=None, stream=None):
+    """One attention layer with pruned queries, in place into the cached output
+    ``y`` [N, H, W, Co]: q = x Wq at the tokens under the tile list (sparse 1x1
+    conv), the cached key / value maps ``k_map`` [N, H, W, D] / ``v_map``
+    updated there from x when ``wk`` / ``wv`` are given (self-attention; a
+    cross-attention caller passes the context's key / value sequences
+    [N, Lc, *] and no ``wk`` / ``wv``), the attention step, and
+    y = o Wo + bo (+ residual) at those tokens (sparse 1x1 conv).  Weights
+    are 1x1 conv weights [c_out][1][1][c_in] (the transposed projection
+    matrices).  With caches built from the original map and an edit confined to
+    the listed tiles, the keys and values equal those of the whole edited map."""
+    N, H, W, C = x.shape
+    D, Dv, Co = wq.shape[0], v_map.shape[-1], wo.shape[0]
+    cd_q = conv_desc(1, 1, 0, C, D, block)
+    if workspace is None:
+        need = max(sige_conv_workspace_bytes(conv_desc(1, 1, 0, ci, co, block), N, capacity, 0, 0)
+                   for ci, co in ((C, D), (C, Dv), (Dv, Co)))
+        workspace = zeros_workspace(need, x.device)
+    q = torch.empty((N, H, W, D), dtype=x.dtype, device=x.device)
+    sige_conv_fused(x, wq, None, cd_q, idx, count, capacity, q, workspace=workspace, stream=stream)
+    if wk is not None:
+        sige_conv_fused(x, wk, None, cd_q, idx, count, capacity, k_map, workspace=workspace, stream=stream)
+    if wv is not None:
+        sige_conv_fused(x, wv, None, conv_desc(1, 1, 0, C, Dv, block), idx, count, capacity, v_map,
+                        workspace=workspace, stream=stream)
+    o = torch.empty((N, H, W, Dv), dtype=x.dtype, device=x.device)
+    sige_attention_core(q, k_map, v_map, heads, idx, count, capacity, block, o, stream)
+    sige_conv_fused(o, wo, bo, conv_desc(1, 1, 0, Dv, Co, block), idx, count, capacity, y, residual=residual,
+                    workspace=workspace, stream=stream)
+    return y
 
 
 SCHEDULE_FIELDS = ("layout", "T", "tile_groups", "splits", "units", "split_sum", "unit_cols", "weight_stages",

@@ -169,3 +169,30 @@ def test_restore_tiles_validation(L):
     dn = sige.TensorDesc(1, 32, 32, 16, sige.BF16, sige.NCHW)
     assert call(desc=ctypes.byref(dn)) == sige.ERR_UNSUPPORTED
     assert call(desc=None) == sige.ERR_INVALID_ARG
+
+
+def test_attention_core_validation(L):
+    d = sige.TensorDesc(1, 16, 16, 320, sige.BF16, sige.NHWC)
+    fake = ctypes.c_void_p(0x1000)
+
+    def call(q=fake, desc=ctypes.byref(d), k=fake, v=fake, keys=256, dv=320, heads=8, idx=fake, cnt=fake, cap=16,
+             block=4, o=fake):
+        return L.sige_attention_core(q, desc, k, v, keys, dv, heads, idx, cnt, cap, block, o, None)
+    for kw in ({"q": None}, {"k": None}, {"v": None}, {"o": None}, {"idx": None}, {"cnt": None}, {"desc": None}):
+        assert call(**kw) == sige.ERR_INVALID_ARG, kw
+    assert call(keys=0) == sige.ERR_INVALID_ARG
+    assert call(dv=0) == sige.ERR_INVALID_ARG
+    assert call(heads=0) == sige.ERR_INVALID_ARG
+    assert call(heads=3) == sige.ERR_INVALID_ARG           # 320 not a multiple of 3
+    assert call(dv=324) == sige.ERR_INVALID_ARG            # dv not a multiple of heads
+    assert call(block=0) == sige.ERR_INVALID_ARG
+    assert call(cap=-1) == sige.ERR_INVALID_ARG
+    assert call(block=9) == sige.ERR_UNSUPPORTED           # more than 64 queries per tile
+    assert call(heads=1) == sige.ERR_UNSUPPORTED           # head width 320 > 256
+    df = sige.TensorDesc(1, 16, 16, 320, sige.F32, sige.NHWC)
+    assert call(desc=ctypes.byref(df)) == sige.ERR_UNSUPPORTED
+    dn = sige.TensorDesc(1, 16, 16, 320, sige.BF16, sige.NCHW)
+    assert call(desc=ctypes.byref(dn)) == sige.ERR_UNSUPPORTED
+    big = sige.TensorDesc(1 << 16, 16, 16, 320, sige.BF16, sige.NHWC)
+    assert call(desc=ctypes.byref(big), keys=1 << 16) == sige.ERR_INVALID_ARG   # keys x batch past 32 bits
+    assert call(cap=0) == sige.OK                          # no tiles: no launch

@@ -59,17 +59,48 @@ def load_peaks():
     return {**FALLBACK_PEAKS, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def src_sha(relpaths):
+def strip_c_comments(text: str) -> str:
+    """C / C++ / CUDA source without its comments: each // or /* */ comment
+    becomes one space (string and character literals are left alone), then
+    trailing blanks and empty lines go."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        ch = text[i]
+        if ch in "\"'":
+            j = i + 1
+            while j < n and text[j] != ch and text[j] != "\n":
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+            out.append(" ")
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(ch)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).split("\n"))
+    return "\n".join(ln for ln in lines if ln)
+
+
+def code_sha(relpaths):
+    """Hash of the sources' code (comments and blank lines left out), so that a
+    traffic figure survives a comment edit and not a code edit."""
     h = hashlib.sha256()
     for rp in relpaths:
-        with open(os.path.join(ROOT, rp), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rp), encoding="utf-8") as f:
+            h.update(strip_c_comments(f.read()).encode())
+        h.update(b"\0")
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel):
     """DRAM bytes (read + write) per launch from the committed ncu summary, when
-    it was taken on the current sources of that kernel; else None."""
+    it was taken on the current code of that kernel; else None."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
@@ -78,7 +109,7 @@ def ncu_traffic(kernel):
     if not d:
         return None
     try:
-        if src_sha(d["sources"]) != d["source_sha"]:
+        if code_sha(d["sources"]) != d["code_sha"]:
             return None
     except (OSError, KeyError):
         return None

@@ -33,11 +33,16 @@
 // adds bias and residual and rounds once into the cached output, or writes
 // float32 output blocks.  When the active tiles are too few to fill the GPU,
 // the K loop is split over several CTAs.  The kernel is launched in clusters
-// of two CTAs: a 2-way split of a unit of at most 64 columns is summed through
-// the peer's shared memory (rank 1 sends its partial to rank 0, which adds its
-// own and runs the epilogue); other splits end with the last CTA of a tile
-// group summing the partials from global memory in a fixed order
-// (deterministic either way).
+// of two CTAs, or of four where one tile would split K at least 4 ways (the
+// split is then a power of two dividing 4).  A 2-way split of a unit of at
+// most 64 columns in clusters of two is summed through the peer's shared
+// memory (rank 1 sends its partial to rank 0, which adds its own and runs the
+// epilogue).  A split that divides the cluster size reduce-scatters inside
+// the cluster: member q of the tile group receives column slice q of every
+// member's partial in its freed halo stages, sums them in member order and
+// writes that slice.  Any other split ends with the last CTA of a tile group
+// summing the partials from global memory in a fixed order.  The sums are
+// deterministic in every case.
 //
 // Warp roles (320 threads): warp 0 issues the weight TMA, warp 1 allocates
 // tensor memory and issues the MMAs, warps 2-9 stage the halo and run the
@@ -446,10 +451,11 @@ __device__ __forceinline__ Unit decode_unit(const TcArgs &p, const Sched &s, int
 //   [0, 1024)        mbarriers and control words
 //   [1024, 3072)     tile origins of the current unit (256 x int2)
 //   [4096, ...)      weight stages, 16 KB each, as many as fit (<= 16)
-//   [.., b_base)     pair launches only: the 32 KB receive buffer of the split-K
-//                    partial sent by the cluster peer
+//   [.., b_base)     clusters of two only: the 32 KB receive buffer of the
+//                    split-K partial sent by the cluster peer
 //   [b_base, end)    SB halo stages of T slots each; reused as the epilogue's
-//                    staging buffer once the unit's MMAs are complete
+//                    staging buffer, or as the reduce-scatter's receive area,
+//                    once the unit's MMAs are complete
 
 // Accumulator columns of a unit of T tiles (ROW) or T slots (POS).
 __host__ __device__ inline int unit_cols(const TcArgs &p, int T)

@@ -53,18 +53,28 @@ def test_layer_roofline():
     assert r["bound"] == "alu" and r["roof_us"] == pytest.approx(1.0, rel=1e-3)
 
 
-def test_traffic_dropped_when_sources_change(tmp_path, monkeypatch):
+def test_traffic_dropped_when_code_changes(tmp_path, monkeypatch):
     src = tmp_path / "k.cu"
-    src.write_text("kernel v1\n")
+    src.write_text("// first version\nint f() { return 1; }\n")
     prof = tmp_path / "profiles"
     prof.mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    entry = {"sources": ["k.cu"], "source_sha": bench.src_sha(["k.cu"]), "bytes_per_launch": 1234}
+    entry = {"sources": ["k.cu"], "code_sha": bench.code_sha(["k.cu"]), "bytes_per_launch": 1234}
     (prof / "ncu_traffic.json").write_text(json.dumps({"k_test": entry}))
     assert bench.ncu_traffic("k_test") == 1234.0
     assert bench.ncu_traffic("k_other") is None
-    src.write_text("kernel v2\n")
+    # comments and blank lines do not change the kernel
+    src.write_text("/* reworded */\n\nint f() { return 1; }  // same code\n")
+    assert bench.ncu_traffic("k_test") == 1234.0
+    # code does
+    src.write_text("int f() { return 2; }\n")
     assert bench.ncu_traffic("k_test") is None
     os.remove(src)
     assert bench.ncu_traffic("k_test") is None
 
+
+def test_strip_c_comments():
+    t = ('int a = 1; // one\n/* two\n lines */ int b = 2; char c = \'/\';\n'
+         'const char *s = "// kept /* kept */";\n\n  x = a/*in*/+b;\n')
+    assert bench.strip_c_comments(t) == ('int a = 1;\n  int b = 2; char c = \'/\';\n'
+                                         'const char *s = "// kept /* kept */";\n  x = a +b;')

@@ -2,7 +2,11 @@
 // output (SIGE project page, "Overview": gather the active blocks from the
 // edited activation, stack them along the batch axis, and scatter the output
 // blocks back into F_l(A_original)).  Plus the GroupNorm statistics of the
-// cached original activation, folded into a per-channel affine.
+// cached original activation, folded into a per-channel affine (a cluster of
+// 8 CTAs per image that combine their partial sums through distributed shared
+// memory, or one CTA per (image, group) for the shapes the cluster path does
+// not take), and the restore of listed tiles from a source tensor between
+// sequential edits.
 #include <atomic>
 #include <algorithm>
 

@@ -9,18 +9,22 @@
 // Layout of the work:
 //   phase 1 (every CTA but CTA 0, HBM-bound): stream both inputs once.  The
 //     inputs are cut into chunks (up to 16 KB of each input); a CTA takes
-//     every (number of streaming CTAs)-th chunk and keeps six of them in
+//     every (number of streaming CTAs)-th chunk and keeps seven of them in
 //     flight with bulk asynchronous copies into shared memory, so nearly the
 //     whole input is requested at once.  An element whose |edit - orig| >
-//     threshold marks, at every scale, the tile its pixel falls in.  Downsampling by an integer factor f
-//     followed by b x b tiles is the same as tiles of b*f input pixels, so the
-//     OR-downsample and the tile OR collapse into one flag store per scale.
+//     threshold marks, at every scale, the tile its pixel falls in (with a
+//     pixel radius R, every tile within R pixels of it at that scale).
+//     Downsampling by an integer factor f followed by b x b tiles is the same
+//     as tiles of b*f input pixels, so the OR-downsample and the tile OR
+//     collapse into one flag store per scale.
 //   phase 2 (CTA 0, which takes no part in phase 1): per scale, dilate the
 //     tile flags by `dilate` tiles (equal to dilating the scale's mask by
 //     dilate*b pixels before tiling), compact the active tiles in row-major
-//     order with a block-wide prefix sum, write the (h0, w0) list and the
-//     count, then clear the flags and the arrival counter so the workspace is
-//     ready for the next call.
+//     order, write the (h0, w0) list and the count, then clear the flags and
+//     the arrival counter so the workspace is ready for the next call.  Grids
+//     of at most 32 x 32 tiles take one warp per scale (rows as 32-bit words,
+//     dilation by shifts and shuffles, a warp prefix sum); larger grids use
+//     the block-wide bit-word path.
 //
 // Phase 2 runs once per call on one CTA, so its cost is latency: each of its
 // instructions is fetched cold.  CTA 0 therefore runs it once without storing

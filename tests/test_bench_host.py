@@ -78,3 +78,14 @@ def test_strip_c_comments():
          'const char *s = "// kept /* kept */";\n\n  x = a/*in*/+b;\n')
     assert bench.strip_c_comments(t) == ('int a = 1;\n  int b = 2; char c = \'/\';\n'
                                          'const char *s = "// kept /* kept */";\n  x = a +b;')
+
+
+def test_bench_workload_tiles_from_the_oracle(orc):
+    # the bench's edit (seed 0, 1.2% of the pixels) activates 51 of the 1024
+    # 8x8 tiles after one-tile dilation, as its JSON line reports
+    from spatially_sparse_incremental_b200 import inputs
+    blk = inputs.make_cfg3(0, H=bench.H, W=bench.W, C=bench.C, area=0.012, block=bench.BLOCK)
+    tiles = orc.reduce_mask(blk.x_orig, blk.x_edit, bench.THRESH, [(bench.H, bench.W, bench.BLOCK)], 1)[0]
+    assert len(tiles) == 51
+    edited = orc.pixel_mask(blk.x_orig, blk.x_edit, bench.THRESH).mean()
+    assert abs(edited - 0.012) < 0.002

@@ -17,7 +17,9 @@
  *     allocates no device memory and keeps no state between calls.
  *   - Every call is asynchronous on `stream` (NULL = legacy default stream),
  *     launches exactly one kernel, and returns after enqueueing it.  Only
- *     sige_get_error() synchronises.
+ *     sige_get_error() / sige_get_device_error() synchronise, and
+ *     sige_reduce_mask / sige_reduce_mask_px when the caller asks for the
+ *     counts on the host.
  *   - Host-side checks run before any launch: invalid arguments return
  *     SIGE_ERR_INVALID_ARG, shapes the kernels do not cover return
  *     SIGE_ERR_UNSUPPORTED, a failed launch returns SIGE_ERR_CUDA.  Nothing
@@ -70,7 +72,10 @@ typedef struct {
 /* One convolution layer F_l.  Output size Ho = (H + 2 pad - kernel)/stride + 1.
  * `block` is the output tile edge b; each gathered input block is
  * b_in = (b - 1) * stride + kernel pixels wide, so neighbouring blocks of a
- * 3x3 stride-1 conv overlap by 2 pixels (SIGE project page, "Overview"). */
+ * 3x3 stride-1 conv overlap by 2 pixels (SIGE project page, "Overview").
+ * Kernels and tiles are square (one `kernel`, one `block`): every layer of the
+ * workloads this library serves is, and the pages describe square blocks
+ * only; a k_h x k_w kernel or a b_h x b_w tile has no field here. */
 typedef struct {
     int32_t kernel, stride, pad;
     int32_t c_in, c_out;
@@ -85,6 +90,15 @@ typedef struct {
 
 #define SIGE_MAX_SCALES 8
 #define SIGE_WORKSPACE_HEADER_BYTES 256
+
+/* Which call a workspace is sized for (sige_workspace_bytes). */
+typedef enum {
+    SIGE_CALL_REDUCE_MASK = 0,
+    SIGE_CALL_SPARSE_CONV = 1,
+    SIGE_CALL_CONV_FUSED = 2,
+    SIGE_CALL_DENSE_CONV = 3,
+    SIGE_CALL_RESBLOCK = 4
+} sige_call;
 
 /* ------------------------------------------------------------------ calls */
 
@@ -106,6 +120,11 @@ typedef struct {
  *   counts         : device int32[n_scales], the number of active tiles (may
  *                    exceed the capacity: then only `capacity` pairs are written
  *                    and the device error SIGE_ERR_CAPACITY is recorded)
+ *   host_counts    : host int32[n_scales] or NULL.  When given, the counts are
+ *                    also copied there and the call synchronises `stream`
+ *                    before it returns (an opt-in: the rest of the path reads
+ *                    the counts on the device).  Refused with
+ *                    SIGE_ERR_INVALID_ARG while `stream` is being captured.
  *   workspace      : device, >= sige_reduce_mask_workspace_bytes(), zero-filled
  *                    before its first use; each call leaves it zero-filled
  *                    apart from a recorded device error.  One workspace per
@@ -119,7 +138,8 @@ size_t sige_reduce_mask_workspace_bytes(const sige_tensor_desc *in, int32_t n_sc
 int sige_reduce_mask(const void *a_orig, const void *a_edit, const sige_tensor_desc *in,
                      float threshold, int32_t dilate, int32_t n_scales,
                      const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
-                     void *workspace, size_t workspace_bytes, sige_stream_t stream);
+                     int32_t *host_counts, void *workspace, size_t workspace_bytes,
+                     sige_stream_t stream);
 
 /* (1c) sige_reduce_mask with the dilation in pixels instead of tiles.
  * mer.dev notes on SIGE, section 3.2 "Sparse Engine SIGE": the mask is dilated
@@ -134,7 +154,8 @@ int sige_reduce_mask(const void *a_orig, const void *a_edit, const sige_tensor_d
 int sige_reduce_mask_px(const void *a_orig, const void *a_edit, const sige_tensor_desc *in,
                         float threshold, int32_t radius, int32_t n_scales,
                         const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
-                        void *workspace, size_t workspace_bytes, sige_stream_t stream);
+                        int32_t *host_counts, void *workspace, size_t workspace_bytes,
+                        sige_stream_t stream);
 
 /* (1b) sige_reduce_mask without a caller workspace.  There is no counterpart
  * in the paper: this is a convenience for callers that cannot allocate device
@@ -147,13 +168,19 @@ int sige_reduce_mask_px(const void *a_orig, const void *a_edit, const sige_tenso
  *     enqueued;
  *   - the first call on a device looks the array's address up (once, with
  *     that device current), so make that first call before any stream
- *     capture;
- *   - each call clears the part of the array it uses with an asynchronous
- *     memset on `stream`, then runs the same kernel as sige_reduce_mask;
+ *     capture; the address is kept for the life of the process and does not
+ *     survive a cudaDeviceReset of that device;
+ *   - each call clears the part of the array it uses and sets counts[] to -1
+ *     with two asynchronous memsets on `stream` (not kernels: they are not
+ *     counted by sige_launch_count), then runs the same kernel as
+ *     sige_reduce_mask;
  *   - all calls share the array: calls that overlap on the GPU (other
  *     streams, other threads) race and must be serialised by the caller;
- *   - a list longer than its capacity shows as counts[s] > capacity (there
- *     is no workspace header to read with sige_get_error).
+ *   - there is no workspace header to read with sige_get_error: a list
+ *     longer than its capacity shows as counts[s] > capacity, and a call that
+ *     did not complete on the device (a bounded wait that expired) leaves
+ *     counts[s] < 0;
+ *   - every argument is checked before anything is enqueued.
  * Other arguments as in sige_reduce_mask. */
 int sige_reduce_mask_static(const void *a_orig, const void *a_edit, const sige_tensor_desc *in,
                             float threshold, int32_t dilate, int32_t n_scales,
@@ -285,9 +312,35 @@ int sige_attention_core(const void *q, const sige_tensor_desc *qd, const void *k
 size_t sige_conv_workspace_bytes(const sige_conv_desc *cd, int32_t batch, int32_t capacity,
                                  int32_t out_h, int32_t out_w);
 
+/* Workspace bytes of one call, by sige_call:
+ *   SIGE_CALL_REDUCE_MASK : capacity = the number of tiles over all scale
+ *                           grids (cd is ignored); an upper bound of
+ *                           sige_reduce_mask_workspace_bytes for any split of
+ *                           those tiles into at most SIGE_MAX_SCALES scales
+ *   SIGE_CALL_SPARSE_CONV, SIGE_CALL_CONV_FUSED, SIGE_CALL_DENSE_CONV :
+ *                           this layer, capacity = list capacity (dense: the
+ *                           tiles of the output grid); the same value as
+ *                           sige_conv_workspace_bytes with batch 1
+ *   SIGE_CALL_RESBLOCK    : sige_resblock_fused (cd and capacity ignored)
+ * 0 for an unknown call or invalid sizes. */
+size_t sige_workspace_bytes(int32_t which_call, const sige_conv_desc *cd, int32_t capacity);
+
 /* Synchronise `stream`, return the first device error recorded in the
  * workspace header (SIGE_OK if none) and clear it. */
 int sige_get_error(void *workspace, sige_stream_t stream);
+
+/* The same as sige_get_error: reads (and clears) the device error word in the
+ * workspace header after synchronising `stream`. */
+int sige_get_device_error(void *workspace, sige_stream_t stream);
+
+/* Bound, in SM clock cycles, of the device-side waits that end a call with
+ * SIGE_ERR_TIMEOUT when they expire, for every launch enqueued after this
+ * call, process-wide; 0 restores each kernel's own bound (seconds).  Covered:
+ * the wait of sige_reduce_mask's reducing CTA for the streaming CTAs.  A test
+ * of the failure path sets a bound of a few cycles so that the wait expires,
+ * checks the status and restores 0.  Returns SIGE_ERR_INVALID_ARG for a
+ * negative value. */
+int sige_set_wait_cycles(int64_t cycles);
 
 /* Which conv kernel a call with this layer and dtype runs: 1 = tcgen05 tensor
  * cores, 0 = CUDA cores; negative = a sige_status for an unsupported layer. */

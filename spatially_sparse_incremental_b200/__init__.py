@@ -16,6 +16,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libsige.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_CAPACITY, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5, -6
+CALL_REDUCE_MASK, CALL_SPARSE_CONV, CALL_CONV_FUSED, CALL_DENSE_CONV, CALL_RESBLOCK = 0, 1, 2, 3, 4
 U8, F32, BF16 = 0, 1, 2
 NHWC, NCHW = 0, 1
 WORKSPACE_HEADER = 256
@@ -50,8 +51,8 @@ _vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c
 _TD, _CD, _SD = ctypes.POINTER(TensorDesc), ctypes.POINTER(ConvDesc), ctypes.POINTER(ScaleDesc)
 SIGNATURES = {
     "sige_reduce_mask_workspace_bytes": (_sz, [_TD, _i32, _SD]),
-    "sige_reduce_mask": (_i32, [_vp, _vp, _TD, _f32, _i32, _i32, _SD, _vp, _vp, _vp, _sz, _vp]),
-    "sige_reduce_mask_px": (_i32, [_vp, _vp, _TD, _f32, _i32, _i32, _SD, _vp, _vp, _vp, _sz, _vp]),
+    "sige_reduce_mask": (_i32, [_vp, _vp, _TD, _f32, _i32, _i32, _SD, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "sige_reduce_mask_px": (_i32, [_vp, _vp, _TD, _f32, _i32, _i32, _SD, _vp, _vp, _vp, _vp, _sz, _vp]),
     "sige_reduce_mask_static": (_i32, [_vp, _vp, _TD, _f32, _i32, _i32, _SD, _vp, _vp, _vp]),
     "sige_gather": (_i32, [_vp, _TD, _CD, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _vp]),
     "sige_sparse_conv": (_i32, [_vp, _CD, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _sz, _vp]),
@@ -63,6 +64,9 @@ SIGNATURES = {
     "sige_restore_tiles": (_i32, [_vp, _vp, _TD, _i32, _vp, _vp, _i32, _vp]),
     "sige_conv_workspace_bytes": (_sz, [_CD, _i32, _i32, _i32, _i32]),
     "sige_get_error": (_i32, [_vp, _vp]),
+    "sige_get_device_error": (_i32, [_vp, _vp]),
+    "sige_workspace_bytes": (_sz, [_i32, _CD, _i32]),
+    "sige_set_wait_cycles": (_i32, [ctypes.c_int64]),
     "sige_conv_path": (_i32, [_CD, _i32]),
     "sige_conv_schedule": (_i32, [_CD, _i32, _i32, _i32, _vp, _i32]),
     "sige_attention_core": (_i32, [_vp, _TD, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp]),
@@ -142,11 +146,18 @@ def sige_reduce_mask_workspace_bytes(desc: TensorDesc, scales) -> int:
     return int(lib().sige_reduce_mask_workspace_bytes(ctypes.byref(desc), len(scales), arr))
 
 
+def _host_counts(n, want):
+    return (ctypes.c_int32 * n)() if want else None
+
+
 def sige_reduce_mask(a_orig, a_edit, threshold, scales, dilate=1, layout=NHWC, idx=None, counts=None,
-                     workspace=None, stream=None):
+                     workspace=None, stream=None, host_counts=False):
     """Difference mask -> per-scale active-tile lists.  ``scales`` is a list of
     (h, w, block, capacity).  Returns (idx [sum(capacity), 2] int32, counts
-    [n_scales] int32, workspace); all on the device, nothing synchronised."""
+    [n_scales] int32, workspace); all on the device, nothing synchronised.
+    With ``host_counts=True`` the call also copies the counts to the host
+    (the library synchronises the stream) and returns them as a fourth item,
+    a list of ints."""
     desc = tensor_desc(a_orig, layout)
     arr = (ScaleDesc * len(scales))(*[ScaleDesc(*s) for s in scales])
     dev = a_orig.device
@@ -157,15 +168,18 @@ def sige_reduce_mask(a_orig, a_edit, threshold, scales, dilate=1, layout=NHWC, i
     need = int(lib().sige_reduce_mask_workspace_bytes(ctypes.byref(desc), len(scales), arr))
     if workspace is None:
         workspace = zeros_workspace(need, dev)
+    hc = _host_counts(len(scales), host_counts)
     st = lib().sige_reduce_mask(_ptr(a_orig), _ptr(a_edit), ctypes.byref(desc), float(threshold), int(dilate),
-                                len(scales), arr, _ptr(idx), _ptr(counts), _ptr(workspace),
+                                len(scales), arr, _ptr(idx), _ptr(counts), hc, _ptr(workspace),
                                 workspace.numel(), _stream(stream))
     _check(st, "sige_reduce_mask")
+    if host_counts:
+        return idx, counts, workspace, [int(v) for v in hc]
     return idx, counts, workspace
 
 
 def sige_reduce_mask_px(a_orig, a_edit, threshold, scales, radius=1, layout=NHWC, idx=None, counts=None,
-                        workspace=None, stream=None):
+                        workspace=None, stream=None, host_counts=False):
     """As sige_reduce_mask, with the mask dilated by ``radius`` pixels at each
     scale before tiling (no tile dilation)."""
     desc = tensor_desc(a_orig, layout)
@@ -178,10 +192,13 @@ def sige_reduce_mask_px(a_orig, a_edit, threshold, scales, radius=1, layout=NHWC
     need = int(lib().sige_reduce_mask_workspace_bytes(ctypes.byref(desc), len(scales), arr))
     if workspace is None:
         workspace = zeros_workspace(need, dev)
+    hc = _host_counts(len(scales), host_counts)
     st = lib().sige_reduce_mask_px(_ptr(a_orig), _ptr(a_edit), ctypes.byref(desc), float(threshold), int(radius),
-                                   len(scales), arr, _ptr(idx), _ptr(counts), _ptr(workspace),
+                                   len(scales), arr, _ptr(idx), _ptr(counts), hc, _ptr(workspace),
                                    workspace.numel(), _stream(stream))
     _check(st, "sige_reduce_mask_px")
+    if host_counts:
+        return idx, counts, workspace, [int(v) for v in hc]
     return idx, counts, workspace
 
 
@@ -297,6 +314,21 @@ def sige_conv_workspace_bytes(cd: ConvDesc, batch: int, capacity: int, out_h: in
 
 def sige_get_error(workspace, stream=None) -> int:
     return int(lib().sige_get_error(_ptr(workspace), _stream(stream)))
+
+
+def sige_get_device_error(workspace, stream=None) -> int:
+    return int(lib().sige_get_device_error(_ptr(workspace), _stream(stream)))
+
+
+def sige_workspace_bytes(which_call: int, cd: ConvDesc | None, capacity: int) -> int:
+    return int(lib().sige_workspace_bytes(int(which_call), None if cd is None else ctypes.byref(cd),
+                                          int(capacity)))
+
+
+def sige_set_wait_cycles(cycles: int) -> None:
+    """Bound of the device waits that report SIGE_ERR_TIMEOUT (0: the kernels'
+    own bounds), for launches enqueued from now on, process-wide."""
+    _check(lib().sige_set_wait_cycles(int(cycles)), "sige_set_wait_cycles")
 
 
 def sige_conv_path(cd: ConvDesc, dtype: torch.dtype) -> int:

@@ -74,6 +74,7 @@ struct __align__(16) MaskParams {
     int32_t chunk;       // modes 0, 1: vectors per chunk of each input (multiple of 256)
     int32_t chunks_base, chunks_rem;   // chunks per streaming CTA: base, +1 for the first rem
     int32_t radius;      // pixel dilation at each scale before tiling (0: none)
+    int64_t wait_cycles; // bound of CTA 0's wait for the streaming CTAs, in SM clock cycles
 };
 
 // Copy the parameter block into shared memory, one 16-byte piece per lane of
@@ -602,8 +603,10 @@ __device__ __noinline__ void phase2(const MaskParams &p, const ScaleParams *sc, 
         p.hdr->arrive = 0;
 }
 
-// Bound of CTA 0's wait for the streaming CTAs (about 4 s at 2 GHz); past it
-// the call records SIGE_ERR_TIMEOUT and leaves its workspace as it is.
+// Default bound of CTA 0's wait for the streaming CTAs (about 4 s at 2 GHz);
+// past it the call records SIGE_ERR_TIMEOUT and leaves its workspace as it
+// is.  sige_set_wait_cycles() replaces it for later launches (a test of the
+// failure path shortens it until it expires).
 constexpr long long kMaskWaitCycles = 1ll << 33;
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *ptr)
@@ -641,7 +644,7 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask_reduce(const __grid_const
             const long long t0 = clock64();
             int go = 1;
             while (ld_acquire_u32(&p.hdr->arrive) != want) {
-                if (clock64() - t0 > kMaskWaitCycles) {
+                if (clock64() - t0 > p.wait_cycles) {
                     record_error(p.hdr, SIGE_ERR_TIMEOUT, -1);
                     go = 0;
                     break;
@@ -723,10 +726,11 @@ extern "C" size_t sige_reduce_mask_workspace_bytes(const sige_tensor_desc *in, i
     return kWsHeader + flag_bytes_of(n_scales, scales);
 }
 
-static int reduce_mask_impl(const void *a_orig, const void *a_edit, const sige_tensor_desc *in, float threshold,
-                            int32_t dilate, int32_t radius, int32_t n_scales, const sige_scale_desc *scales,
-                            int32_t *idx, int32_t *counts, void *workspace, size_t workspace_bytes,
-                            sige_stream_t stream)
+// Host-side checks of a mask-reduction call that need no workspace; both
+// entry points run them before anything is enqueued.
+static int validate_mask_args(const void *a_orig, const void *a_edit, const sige_tensor_desc *in, float threshold,
+                              int32_t dilate, int32_t radius, int32_t n_scales, const sige_scale_desc *scales,
+                              const int32_t *idx, const int32_t *counts)
 {
     if (!a_orig || !a_edit || !in || !idx || !counts)
         return SIGE_ERR_INVALID_ARG;
@@ -740,11 +744,50 @@ static int reduce_mask_impl(const void *a_orig, const void *a_edit, const sige_t
         return SIGE_ERR_INVALID_ARG;
     if (!scales_ok(in, n_scales, scales))
         return SIGE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(idx) & 7))
+        return SIGE_ERR_INVALID_ARG;
+    return SIGE_OK;
+}
+
+// The opt-in host copy of the counts: enqueued after the kernel, then the
+// stream is synchronised.  A capturing stream cannot be synchronised, so a
+// request during capture is refused before anything is enqueued.
+static int check_host_counts(const int32_t *host_counts, sige_stream_t stream)
+{
+    if (!host_counts)
+        return SIGE_OK;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing((cudaStream_t)stream, &cs) != cudaSuccess)
+        return SIGE_ERR_CUDA;
+    return cs == cudaStreamCaptureStatusNone ? SIGE_OK : SIGE_ERR_INVALID_ARG;
+}
+
+static int copy_host_counts(int st, int32_t *host_counts, const int32_t *counts, int32_t n_scales,
+                            sige_stream_t stream)
+{
+    if (st != SIGE_OK || !host_counts)
+        return st;
+    if (cudaMemcpyAsync(host_counts, counts, sizeof(int32_t) * (size_t)n_scales, cudaMemcpyDeviceToHost,
+                        (cudaStream_t)stream) != cudaSuccess ||
+        cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)
+        return SIGE_ERR_CUDA;
+    return SIGE_OK;
+}
+
+static int reduce_mask_impl(const void *a_orig, const void *a_edit, const sige_tensor_desc *in, float threshold,
+                            int32_t dilate, int32_t radius, int32_t n_scales, const sige_scale_desc *scales,
+                            int32_t *idx, int32_t *counts, int32_t *host_counts, void *workspace,
+                            size_t workspace_bytes, sige_stream_t stream)
+{
+    int vs = validate_mask_args(a_orig, a_edit, in, threshold, dilate, radius, n_scales, scales, idx, counts);
+    if (vs != SIGE_OK)
+        return vs;
     const size_t need = kWsHeader + flag_bytes_of(n_scales, scales);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15))
         return SIGE_ERR_WORKSPACE;
-    if ((reinterpret_cast<uintptr_t>(idx) & 7))
-        return SIGE_ERR_INVALID_ARG;
+    vs = check_host_counts(host_counts, stream);
+    if (vs != SIGE_OK)
+        return vs;
 
     MaskParams p{};
     p.a = static_cast<const uint8_t *>(a_orig);
@@ -781,6 +824,7 @@ static int reduce_mask_impl(const void *a_orig, const void *a_edit, const sige_t
     p.hdr = static_cast<WsHeader *>(workspace);
     p.flags = static_cast<uint8_t *>(workspace) + kWsHeader;
     p.flag_bytes = foff;
+    p.wait_cycles = wait_cycles_or(kMaskWaitCycles);
 
     const int esz = in->dtype == SIGE_U8 ? 1 : in->dtype == SIGE_BF16 ? 2 : 4;
     const int64_t nelem = (int64_t)in->n * in->h * in->w * in->c;
@@ -833,25 +877,27 @@ static int reduce_mask_impl(const void *a_orig, const void *a_edit, const sige_t
     count_launch();
     if (e != cudaSuccess)
         return SIGE_ERR_CUDA;
-    return launch_check();
+    return copy_host_counts(launch_check(), host_counts, counts, n_scales, stream);
 }
 
 extern "C" int sige_reduce_mask(const void *a_orig, const void *a_edit, const sige_tensor_desc *in,
                                 float threshold, int32_t dilate, int32_t n_scales,
                                 const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
-                                void *workspace, size_t workspace_bytes, sige_stream_t stream)
+                                int32_t *host_counts, void *workspace, size_t workspace_bytes,
+                                sige_stream_t stream)
 {
-    return reduce_mask_impl(a_orig, a_edit, in, threshold, dilate, 0, n_scales, scales, idx, counts, workspace,
-                            workspace_bytes, stream);
+    return reduce_mask_impl(a_orig, a_edit, in, threshold, dilate, 0, n_scales, scales, idx, counts, host_counts,
+                            workspace, workspace_bytes, stream);
 }
 
 extern "C" int sige_reduce_mask_px(const void *a_orig, const void *a_edit, const sige_tensor_desc *in,
                                    float threshold, int32_t radius, int32_t n_scales,
                                    const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
-                                   void *workspace, size_t workspace_bytes, sige_stream_t stream)
+                                   int32_t *host_counts, void *workspace, size_t workspace_bytes,
+                                   sige_stream_t stream)
 {
-    return reduce_mask_impl(a_orig, a_edit, in, threshold, 0, radius, n_scales, scales, idx, counts, workspace,
-                            workspace_bytes, stream);
+    return reduce_mask_impl(a_orig, a_edit, in, threshold, 0, radius, n_scales, scales, idx, counts, host_counts,
+                            workspace, workspace_bytes, stream);
 }
 
 // ------------------------------------------------------------------ variant without a workspace
@@ -870,7 +916,8 @@ constexpr size_t kStaticScratchBytes = 64 * 1024;
 static __device__ __align__(256) uint8_t g_mask_scratch[kStaticScratchBytes];
 
 // The array's name is only a host-side stand-in; its device address is looked
-// up once per device, with that device current.
+// up once per device, with that device current, and kept for the life of the
+// process (it does not survive a cudaDeviceReset of that device).
 static void *static_scratch_address(int &status)
 {
     static std::mutex mu;
@@ -900,19 +947,25 @@ extern "C" int sige_reduce_mask_static(const void *a_orig, const void *a_edit, c
                                        const sige_scale_desc *scales, int32_t *idx, int32_t *counts,
                                        sige_stream_t stream)
 {
-    if (!in || !scales_ok(in, n_scales, scales))
-        return SIGE_ERR_INVALID_ARG;
+    // every argument check first: nothing is enqueued for an invalid call
+    int st = validate_mask_args(a_orig, a_edit, in, threshold, dilate, 0, n_scales, scales, idx, counts);
+    if (st != SIGE_OK)
+        return st;
     const size_t need = kWsHeader + flag_bytes_of(n_scales, scales);
     if (need > kStaticScratchBytes)
         return SIGE_ERR_WORKSPACE;   // more tiles than the built-in scratch holds
-    int st = SIGE_OK;
     void *scratch = static_scratch_address(st);
     if (!scratch)
         return st;
-    // the kernel needs its flags and arrival counter at zero on entry; an
-    // earlier call that failed part-way could have left them otherwise
-    if (cudaMemsetAsync(scratch, 0, need, (cudaStream_t)stream) != cudaSuccess)
+    // The kernel needs its flags and arrival counter at zero on entry (an
+    // earlier call that failed part-way could have left them otherwise).  The
+    // counts start at -1: the kernel overwrites them only when the reduction
+    // completes, so a call that recorded a device error (which no caller can
+    // read here: the header lives in the shared array and the next call clears
+    // it) leaves negative counts behind.
+    if (cudaMemsetAsync(scratch, 0, need, (cudaStream_t)stream) != cudaSuccess ||
+        cudaMemsetAsync(counts, 0xFF, sizeof(int32_t) * (size_t)n_scales, (cudaStream_t)stream) != cudaSuccess)
         return SIGE_ERR_CUDA;
-    return sige_reduce_mask(a_orig, a_edit, in, threshold, dilate, n_scales, scales, idx, counts, scratch, need,
-                            stream);
+    return reduce_mask_impl(a_orig, a_edit, in, threshold, dilate, 0, n_scales, scales, idx, counts, nullptr,
+                            scratch, need, stream);
 }

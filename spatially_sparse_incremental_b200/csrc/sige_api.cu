@@ -9,8 +9,15 @@
 namespace sige {
 
 static std::atomic<uint64_t> g_launches{0};
+static std::atomic<long long> g_wait_cycles{0};   // 0: every kernel keeps its own default
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+long long wait_cycles_or(long long dflt)
+{
+    const long long v = g_wait_cycles.load(std::memory_order_relaxed);
+    return v > 0 ? v : dflt;
+}
 
 int launch_check()
 {
@@ -216,6 +223,41 @@ extern "C" int sige_get_error(void *workspace, sige_stream_t stream)
             return SIGE_ERR_CUDA;
     }
     return h[0];
+}
+
+extern "C" int sige_get_device_error(void *workspace, sige_stream_t stream)
+{
+    return sige_get_error(workspace, stream);
+}
+
+extern "C" int sige_set_wait_cycles(int64_t cycles)
+{
+    if (cycles < 0)
+        return SIGE_ERR_INVALID_ARG;
+    g_wait_cycles.store((long long)cycles, std::memory_order_relaxed);
+    return SIGE_OK;
+}
+
+extern "C" size_t sige_workspace_bytes(int32_t which_call, const sige_conv_desc *cd, int32_t capacity)
+{
+    if (capacity < 0)
+        return 0;
+    switch (which_call) {
+    case SIGE_CALL_REDUCE_MASK:
+        // header + one flag byte per tile of every scale, each scale padded to
+        // 16 bytes (at most SIGE_MAX_SCALES of them)
+        return kWsHeader + (((size_t)capacity + 15) & ~(size_t)15) + 16 * (size_t)SIGE_MAX_SCALES;
+    case SIGE_CALL_SPARSE_CONV:
+    case SIGE_CALL_CONV_FUSED:
+    case SIGE_CALL_DENSE_CONV:
+        if (!cd || cd->block < 1)
+            return 0;
+        return ws_need(cd, 1, capacity);
+    case SIGE_CALL_RESBLOCK:
+        return kWsHeader;
+    default:
+        return 0;
+    }
 }
 
 extern "C" uint64_t sige_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -76,6 +76,9 @@ inline void prefer_max_shared(K kernel)
 }
 void count_launch();
 int device_sm_count();
+// Bound of the device-side waits that sige_set_wait_cycles() may shorten, for
+// launches enqueued from now on: the value set there, or `dflt` when none is.
+long long wait_cycles_or(long long dflt);
 
 // Programmatic dependent launch.  A kernel launched this way may start while
 // the kernel before it in the stream is still running: its CTAs take SMs as

@@ -27,10 +27,22 @@ def _declared():
     return sorted(set(names))
 
 
+# The calls of the hot path's C boundary: the five steps of the layer (mask
+# reduction, gather, block conv, scatter, fused layer) and the workspace /
+# status / device-error utilities around them.
+BOUNDARY = ("sige_reduce_mask", "sige_gather", "sige_sparse_conv", "sige_scatter", "sige_conv_fused",
+            "sige_workspace_bytes", "sige_status_string", "sige_get_device_error")
+
+
 def test_header_declares_the_calls():
     names = _declared()
-    for call in ("sige_reduce_mask", "sige_gather", "sige_sparse_conv", "sige_scatter", "sige_conv_fused"):
-        assert call in names
+    for call in BOUNDARY:
+        assert call in names, call
+
+
+def test_boundary_calls_exported(L):
+    for call in BOUNDARY:
+        assert hasattr(L, call), call
 
 
 def test_every_declared_symbol_is_exported_and_bound(L):
@@ -59,13 +71,14 @@ def test_reduce_mask_validation(L):
     assert need == 256 + 1024 + 1024 + 256 + 256
     fake = ctypes.c_void_p(0x1000)
     ws = ctypes.c_void_p(0x2000)
+    hc = (ctypes.c_int32 * 4)()
     args = lambda **kw: dict(dict(a=fake, b=fake, d=ctypes.byref(d), thr=0.0, dil=1, ns=4, sc=sc,
-                                  idx=fake, cnt=fake, ws=ws, wsb=need, st=None), **kw)
+                                  idx=fake, cnt=fake, hc=None, ws=ws, wsb=need, st=None), **kw)
 
     def call(**kw):
         a = args(**kw)
         return L.sige_reduce_mask(a["a"], a["b"], a["d"], a["thr"], a["dil"], a["ns"], a["sc"], a["idx"],
-                                  a["cnt"], a["ws"], a["wsb"], a["st"])
+                                  a["cnt"], a["hc"], a["ws"], a["wsb"], a["st"])
     assert call(a=None) == sige.ERR_INVALID_ARG
     assert call(idx=None) == sige.ERR_INVALID_ARG
     assert call(thr=-1.0) == sige.ERR_INVALID_ARG
@@ -79,6 +92,56 @@ def test_reduce_mask_validation(L):
     assert call(ns=1, sc=bad) == sige.ERR_INVALID_ARG
     d16 = sige.TensorDesc(1, 16, 16, 3, 7, sige.NHWC)
     assert call(d=ctypes.byref(d16)) == sige.ERR_UNSUPPORTED
+    # with host counts requested, argument errors still come first
+    assert call(a=None, hc=hc) == sige.ERR_INVALID_ARG
+    assert call(wsb=need - 1, hc=hc) == sige.ERR_WORKSPACE
+
+
+def test_reduce_mask_static_checks_before_enqueueing(L):
+    """Every argument is checked before the static entry point touches the
+    device (memsets or the symbol lookup): these calls return the argument
+    error on a host with no GPU at all."""
+    d = sige.TensorDesc(1, 64, 64, 8, sige.F32, sige.NHWC)
+    sc = _scales((64, 64, 8, 64))
+    fake = ctypes.c_void_p(0x1000)
+
+    def call(a=fake, idx=fake, cnt=fake, thr=1e-3, dil=1, desc=ctypes.byref(d), scales=sc, ns=1):
+        return L.sige_reduce_mask_static(a, fake, desc, thr, dil, ns, scales, idx, cnt, None)
+    assert call(a=None) == sige.ERR_INVALID_ARG
+    assert call(idx=None) == sige.ERR_INVALID_ARG
+    assert call(cnt=None) == sige.ERR_INVALID_ARG
+    assert call(idx=ctypes.c_void_p(0x1004)) == sige.ERR_INVALID_ARG      # pairs need 8-byte alignment
+    assert call(thr=float("nan")) == sige.ERR_INVALID_ARG
+    assert call(dil=-1) == sige.ERR_INVALID_ARG
+    assert call(ns=0) == sige.ERR_INVALID_ARG
+    dbad = sige.TensorDesc(1, 64, 64, 8, 7, sige.NHWC)
+    assert call(desc=ctypes.byref(dbad)) == sige.ERR_UNSUPPORTED
+    # more tiles than the 64 KB built-in scratch holds
+    dbig = sige.TensorDesc(1, 4096, 4096, 8, sige.F32, sige.NHWC)
+    assert call(desc=ctypes.byref(dbig), scales=_scales((4096, 4096, 8, 1 << 18))) == sige.ERR_WORKSPACE
+
+
+def test_workspace_bytes_by_call(L):
+    cd = sige.ConvDesc(3, 1, 1, 128, 128, 8)
+    conv = L.sige_conv_workspace_bytes(ctypes.byref(cd), 1, 1024, 0, 0)
+    for which in (sige.CALL_SPARSE_CONV, sige.CALL_CONV_FUSED, sige.CALL_DENSE_CONV):
+        assert sige.sige_workspace_bytes(which, cd, 1024) == conv
+    # the mask bound covers any split of the tiles into scales
+    d = sige.TensorDesc(1, 256, 256, 3, sige.U8, sige.NCHW)
+    sc = _scales((256, 256, 8, 1024), (128, 128, 4, 1024), (64, 64, 4, 256), (32, 32, 2, 256))
+    exact = L.sige_reduce_mask_workspace_bytes(ctypes.byref(d), 4, sc)
+    tiles = 1024 + 1024 + 256 + 256
+    assert sige.sige_workspace_bytes(sige.CALL_REDUCE_MASK, None, tiles) >= exact
+    assert sige.sige_workspace_bytes(sige.CALL_RESBLOCK, None, 0) >= 256
+    assert sige.sige_workspace_bytes(99, cd, 16) == 0
+    assert sige.sige_workspace_bytes(sige.CALL_CONV_FUSED, cd, -1) == 0
+    assert sige.sige_workspace_bytes(sige.CALL_CONV_FUSED, None, 16) == 0
+
+
+def test_wait_cycles_setting(L):
+    assert L.sige_set_wait_cycles(-1) == sige.ERR_INVALID_ARG
+    assert L.sige_set_wait_cycles(1000) == sige.OK
+    assert L.sige_set_wait_cycles(0) == sige.OK
 
 
 def test_conv_validation(L):
@@ -147,7 +210,7 @@ def test_reduce_mask_px_validation(L):
     fake, ws = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000)
 
     def call(radius=1, a=fake, wsb=need, thr=1e-3):
-        return L.sige_reduce_mask_px(a, fake, ctypes.byref(d), thr, radius, 1, sc, fake, fake, ws, wsb, None)
+        return L.sige_reduce_mask_px(a, fake, ctypes.byref(d), thr, radius, 1, sc, fake, fake, None, ws, wsb, None)
     assert call(radius=-1) == sige.ERR_INVALID_ARG
     assert call(a=None) == sige.ERR_INVALID_ARG
     assert call(thr=float("nan")) == sige.ERR_INVALID_ARG

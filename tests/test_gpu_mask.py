@@ -198,3 +198,68 @@ def test_pixel_dilation_cfg3(orc):
         n = int(cnt[0].item())
         assert n == len(ref) and np.array_equal(idx[:n].cpu().numpy(), ref)
         assert sige.sige_get_error(ws) == sige.OK
+
+
+def test_host_counts_equal_device_counts(orc):
+    """The opt-in host copy of the counts (the call synchronises the stream)
+    holds exactly the device counts, for one and for several scales."""
+    blk = inputs.make_cfg3(7)
+    xo, xe = blk.x_orig.to(DEV), blk.x_edit.to(DEV)
+    sc = [(256, 256, 8, 1024), (128, 128, 4, 1024), (64, 64, 2, 1024)]
+    idx, cnt, _, host = sige.sige_reduce_mask(xo, xe, 1e-3, sc, 1, host_counts=True)
+    assert host == cnt.cpu().tolist()
+    ref = orc.reduce_mask(blk.x_orig, blk.x_edit, 1e-3, [s[:3] for s in sc], 1)
+    assert host == [len(r) for r in ref]
+    o, e, _ = inputs.make_cfg2(11)
+    caps = _full_caps(inputs.CFG2_SCALES)
+    _, cnt2, _, host2 = sige.sige_reduce_mask_px(o.to(DEV), e.to(DEV), 0.0, caps, 2, sige.NCHW, host_counts=True)
+    assert host2 == cnt2.cpu().tolist()
+
+
+def test_host_counts_refused_during_capture():
+    """A capturing stream cannot be synchronised: the request is refused
+    before anything is enqueued, and the capture stays valid."""
+    x = torch.zeros((1, 64, 64, 8), dtype=torch.float32, device=DEV)
+    sc = [(64, 64, 8, 64)]
+    ws = sige.zeros_workspace(4096, DEV)
+    sige.sige_reduce_mask(x, x, 0.0, sc, 1, workspace=ws)   # one-time set-up outside the capture
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        with pytest.raises(sige.SigeError) as ei:
+            sige.sige_reduce_mask(x, x, 0.0, sc, 1, workspace=ws, stream=s, host_counts=True)
+        sige.sige_reduce_mask(x, x, 0.0, sc, 1, workspace=ws, stream=s)
+    assert ei.value.status == sige.ERR_INVALID_ARG
+    g.replay()
+    torch.cuda.synchronize()
+
+
+def test_expired_wait_reports_timeout_and_the_next_call_is_exact(orc):
+    """Failure path of the reducing CTA's bounded wait.  With the bound set to
+    one clock cycle it expires while the other CTAs still stream the 33 MB of
+    input: the call returns, the workspace header holds SIGE_ERR_TIMEOUT with
+    the wait site (-1) in its detail word, and no count is written.  With the
+    default bound restored and the workspace zero-filled again, the next call
+    gives the oracle's list bit for bit."""
+    blk = inputs.make_cfg3(2)
+    xo, xe = blk.x_orig.to(DEV), blk.x_edit.to(DEV)
+    sc = [(256, 256, 8, 1024)]
+    ref = orc.reduce_mask(blk.x_orig, blk.x_edit, 1e-3, [(256, 256, 8)], 1)[0]
+    ws = sige.zeros_workspace(sige.sige_reduce_mask_workspace_bytes(sige.tensor_desc(xo), sc), DEV)
+    cnt = torch.full((1,), -9, dtype=torch.int32, device=DEV)
+    try:
+        sige.sige_set_wait_cycles(1)
+        sige.sige_reduce_mask(xo, xe, 1e-3, sc, 1, counts=cnt, workspace=ws)
+        torch.cuda.synchronize()
+    finally:
+        sige.sige_set_wait_cycles(0)
+    head = ws[:8].view(torch.int32).cpu().tolist()
+    assert head == [sige.ERR_TIMEOUT, -1], head
+    assert int(cnt.item()) == -9                       # the reducer wrote nothing
+    assert sige.sige_get_device_error(ws) == sige.ERR_TIMEOUT
+    assert sige.sige_get_device_error(ws) == sige.OK   # read and cleared
+    ws.zero_()
+    got, cnt2, _ = _gpu_lists(blk.x_orig, blk.x_edit, 1e-3, sc, workspace=ws)
+    assert int(cnt2[0]) == len(ref) and np.array_equal(got[0], ref)
+    assert sige.sige_get_device_error(ws) == sige.OK

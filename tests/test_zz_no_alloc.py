@@ -76,3 +76,35 @@ def test_static_scratch_rejects_oversized_requests():
         sige.sige_reduce_mask_static(x, x, 0.0, too_big)
     assert ei.value.status == sige.ERR_WORKSPACE
     assert sige.sige_launch_count() == n0
+
+
+def test_static_scratch_lists_equal_the_oracle(orc):
+    """The allocation-free call's lists against the oracle itself, not only
+    against the workspace entry point."""
+    caps = [(h, w, b, -(-h // b) * -(-w // b)) for (h, w, b) in inputs.CFG2_SCALES]
+    for seed in (21, 22):
+        o, e, _ = inputs.make_cfg2(seed)
+        got, gcnt = _static_call(o.to(DEV), e.to(DEV), 0.0, caps, 1, sige.NCHW)
+        ref = orc.reduce_mask(o, e, 0.0, inputs.CFG2_SCALES, 1, orc.NCHW)
+        for s in range(len(caps)):
+            assert int(gcnt[s]) == len(ref[s]) and np.array_equal(got[s], ref[s]), (seed, s)
+
+
+def test_static_scratch_marks_an_incomplete_call_with_negative_counts():
+    """A call whose reducing CTA gave up (its bounded wait, shortened here to
+    one clock cycle, expired) cannot report through a workspace header, so it
+    leaves counts of -1; the next call, with the default bound, is exact."""
+    blk = inputs.make_cfg3(9)
+    xo, xe = blk.x_orig.to(DEV), blk.x_edit.to(DEV)
+    sc = [(256, 256, 8, 1024)]
+    try:
+        sige.sige_set_wait_cycles(1)
+        _, cnt = sige.sige_reduce_mask_static(xo, xe, 1e-3, sc)
+        torch.cuda.synchronize()
+    finally:
+        sige.sige_set_wait_cycles(0)
+    assert int(cnt.item()) < 0
+    got, gcnt = _static_call(xo, xe, 1e-3, sc, 1, sige.NHWC)
+    ri, rc, _ = sige.sige_reduce_mask(xo, xe, 1e-3, sc, 1)
+    ref, rcnt = _lists(ri, rc, sc)
+    assert np.array_equal(gcnt, rcnt) and np.array_equal(got[0], ref[0])

@@ -4,9 +4,13 @@
 Workload (one step = one pass of the whole hot path over one edit): the
 DDPM-style residual block at 256x256, C=128, bf16 storage / fp32 accumulation,
 with a ~1.2% edit made of 1-3 seeded discs:
-    mask   : difference mask of x_orig vs x_edit -> 8x8 tile list (dilate 1)
-    conv1  : gather(GN1 + SiLU) -> 3x3 conv -> scatter(+bias) into cached y1
-    conv2  : gather(GN2 + SiLU) -> 3x3 conv -> scatter(+bias +x_edit) into cached out
+    mask     : difference mask of x_orig vs x_edit -> 8x8 tile list (dilate 1)
+    resblock : one launch for both layers on the tiles: gather(GN1 + SiLU) ->
+               3x3 conv1 (+bias) -> y1 (into the cached y1, and on chip with a
+               one-pixel ring) -> GN2 + SiLU -> 3x3 conv2 (+bias +x_edit) ->
+               scatter into the cached out
+The same step with the two layers as separate fused-layer launches
+(conv1, conv2) is timed beside it (`unfused_step_us`).
 The caches (y1 and out of the original image, GroupNorm statistics of the
 original) are computed once beforehand by the same library's dense conv, as
 the engine pre-computes the original activations.
@@ -244,13 +248,29 @@ def make_workload(seed, dev, area=0.012):
     mask_ws = sige.zeros_workspace(sige.sige_reduce_mask_workspace_bytes(sige.tensor_desc(d["x_orig"]),
                                                                          [(H, W, BLOCK, cap)]), dev)
     conv_ws = sige.zeros_workspace(sige.sige_conv_workspace_bytes(cd, 1, cap, H, W), dev)
+    rb_ws = sige.zeros_workspace(sige.sige_workspace_bytes(sige.CALL_RESBLOCK, None, cap), dev)
     d.update(cd=cd, cap=cap, gs1=gs1, gh1=gh1, gs2=gs2, gh2=gh2, y1=y1, out=out, idx=idx, cnt=cnt,
-             mask_ws=mask_ws, conv_ws=conv_ws, blk=blk)
+             mask_ws=mask_ws, conv_ws=conv_ws, rb_ws=rb_ws, blk=blk)
     return d
 
 
 def step_calls(d, stream=None):
-    """The three hot-path calls of one step, as closures (for graph capture)."""
+    """The two hot-path calls of one step, as closures (for graph capture)."""
+    import spatially_sparse_incremental_b200 as sige
+
+    def mask():
+        sige.sige_reduce_mask(d["x_orig"], d["x_edit"], THRESH, [(H, W, BLOCK, d["cap"])], 1, idx=d["idx"],
+                              counts=d["cnt"], workspace=d["mask_ws"], stream=stream)
+
+    def resblock():
+        sige.sige_resblock_fused(d["x_edit"], d["w1"], d["b1"], (d["gs1"], d["gh1"]), d["w2"], d["b2"],
+                                 (d["gs2"], d["gh2"]), d["idx"], d["cnt"], d["cap"], d["y1"], d["out"],
+                                 workspace=d["rb_ws"], stream=stream)
+    return {"mask": mask, "resblock": resblock}
+
+
+def unfused_calls(d, stream=None):
+    """The same step with each layer as its own fused-layer launch."""
     import spatially_sparse_incremental_b200 as sige
 
     def mask():
@@ -411,8 +431,7 @@ def measure_extras(dev, flush, stream, peaks, seed, step_graph):
 
     def whole_px():
         mask_px()
-        calls["conv1"]()
-        calls["conv2"]()
+        calls["resblock"]()
     g = capture(whole_px, stream)
     t = time_graph(g, flush, 40, stream)
     out["pixel_dilation_step"] = {"radius_px": 2, "active_tiles": tiles_px, "step_us": float(np.median(t)) * 1e3}
@@ -476,6 +495,19 @@ def conv_work(n_tiles, residual):
     scatter = n_tiles * BLOCK * BLOCK * C * 2 * (2 if residual else 1)
     weights = C * 9 * C * 2 + C * 4
     return 2 * macs, gather + scatter + weights
+
+
+def resblock_work(n_tiles):
+    """Algorithmic FLOPs and bytes of one fused res-block launch: the two convs'
+    MACs on the tiles (the ring of y1 that is recomputed is not counted); the x
+    halo of each tile read once (12 x 12 pixels, which holds the residual), y1
+    and out written at the tile, both weight tensors and the per-channel
+    vectors once."""
+    macs = 2 * n_tiles * BLOCK * BLOCK * C * C * 9
+    halo = n_tiles * (BLOCK + 4) ** 2 * C * 2
+    writes = 2 * n_tiles * BLOCK * BLOCK * C * 2
+    weights = 2 * (C * 9 * C * 2) + 6 * C * 4
+    return 2 * macs, halo + writes + weights
 
 
 def mask_work(n_tiles):
@@ -581,6 +613,13 @@ def run_sige(args):
             fn()
     step_graph = {"step": capture(whole_step, stream)}
     graphs = {nm: capture(fn, stream) for nm, fn in calls.items()}
+    ucalls = unfused_calls(d, stream)
+
+    def whole_unfused():
+        for fn in ucalls.values():
+            fn()
+    ugraph = {"unfused": capture(whole_unfused, stream)}
+    ugraphs = {nm: capture(fn, stream) for nm, fn in ucalls.items()}
     dgraphs = {nm: capture(fn, stream) for nm, fn in dense_calls(d, stream).items()}
     flush = L2Flush(dev)
     stream.synchronize()
@@ -605,9 +644,16 @@ def run_sige(args):
     timed_graph_steps(graphs, flush, args.warmup, stream)
     per, _ = timed_graph_steps(graphs, flush, args.steps, stream)
     kern_ms = {nm: float(np.mean(v)) for nm, v in per.items()}
-    red = max_over_ranks([step_ms] + [kern_ms[k] for k in kern_ms], dev)
-    step_ms = red[0]
-    kern_ms = {k: red[i + 1] for i, k in enumerate(kern_ms)}
+    # the same step with the layers as two separate launches
+    nu = max(10, min(args.steps, 200))
+    timed_graph_steps(ugraph, flush, 3, stream)
+    _, utot = timed_graph_steps(ugraph, flush, nu, stream)
+    uper, _ = timed_graph_steps(ugraphs, flush, nu, stream)
+    unfused_ms = float(np.mean(utot))
+    ukern_ms = {nm: float(np.mean(v)) for nm, v in uper.items()}
+    red = max_over_ranks([step_ms, unfused_ms] + [kern_ms[k] for k in kern_ms], dev)
+    step_ms, unfused_ms = red[0], red[1]
+    kern_ms = {k: red[i + 2] for i, k in enumerate(kern_ms)}
 
     # dense comparison (same launch mode, L2 flushed)
     dper, dtot = timed_graph_steps(dgraphs, flush, max(10, min(args.steps, 50)), stream)
@@ -637,20 +683,17 @@ def run_sige(args):
     e2e_ms = max_over_ranks([e2e_ms], dev)[0]
 
     # roofline of the dominant kernel
-    work = {"mask": ("hbm", None, mask_work(n_tiles)),
-            "conv1": (None,) + conv_work(n_tiles, False),
-            "conv2": (None,) + conv_work(n_tiles, True)}
     dom = max(kern_ms, key=kern_ms.get)
-    kernel_name = {"mask": "k_mask_reduce", "conv1": "conv", "conv2": "conv"}[dom]
+    kernel_name = {"mask": "k_mask_reduce", "resblock": "k_resblock"}[dom]
     if dom == "mask":
-        nbytes = work["mask"][2]
+        nbytes = mask_work(n_tiles)
         ach = nbytes / (kern_ms[dom] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": ach / peaks["hbm_gbs"], "traffic": ncu_traffic("k_mask_reduce"),
                 "kernel": kernel_name, "algorithmic_bytes": nbytes,
                 "peak_source": f"{peaks['source']} hbm_gbs"}
     else:
-        _, flops, nbytes = work[dom]
+        flops, nbytes = resblock_work(n_tiles)
         t_tc = flops / (peaks["bf16_tflops"] * 1e12)
         t_bw = nbytes / (peaks["hbm_gbs"] * 1e9)
         if t_tc >= t_bw:
@@ -661,15 +704,13 @@ def run_sige(args):
             ach = nbytes / (kern_ms[dom] * 1e-3) / 1e9
             roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": ach / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} hbm_gbs"}
-        roof.update(traffic=ncu_traffic("k_conv_tc" if sige.sige_conv_path(d["cd"], torch.bfloat16) == 1
-                                        else "k_conv_simt"), kernel=kernel_name,
-                    algorithmic_bytes=nbytes, algorithmic_flops=flops)
+        roof.update(traffic=ncu_traffic("k_resblock"), kernel=kernel_name, algorithmic_bytes=nbytes,
+                    algorithmic_flops=flops)
     # step roofline: every call at its own bound
-    t_roof = mask_work(n_tiles) / (peaks["hbm_gbs"] * 1e9)
-    for res in (False, True):
-        f, b = conv_work(n_tiles, res)
-        t_roof += max(f / (peaks["bf16_tflops"] * 1e12), b / (peaks["hbm_gbs"] * 1e9))
-    sparse_conv_ms = kern_ms["conv1"] + kern_ms["conv2"]
+    f_rb, b_rb = resblock_work(n_tiles)
+    t_roof = mask_work(n_tiles) / (peaks["hbm_gbs"] * 1e9) + max(f_rb / (peaks["bf16_tflops"] * 1e12),
+                                                                 b_rb / (peaks["hbm_gbs"] * 1e9))
+    sparse_conv_ms = kern_ms["resblock"]
     dense_conv_ms = dense_ms["dense1"] + dense_ms["dense2"]
 
     extras = None
@@ -690,10 +731,12 @@ def run_sige(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "H": H, "W": W, "C": C, "block": BLOCK, "edit_area": 0.012,
                    "active_tiles": n_tiles, "tile_fraction": n_tiles / d["cap"],
-                   "l2": "cold: 256 MiB write then 256 MiB read (clean lines) before every step, untimed", "launch": "one CUDA graph per step (mask + conv1 + conv2); breakdown_us from one graph per call",
+                   "l2": "cold: 256 MiB write then 256 MiB read (clean lines) before every step, untimed", "launch": "one CUDA graph per step (mask + fused res block); breakdown_us from one graph per call",
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
         "step_p50_us": float(np.median(tot)) * 1e3, "step_p90_us": float(np.percentile(tot, 90)) * 1e3,
         "breakdown_us": {k: v * 1e3 for k, v in kern_ms.items()},
+        "unfused_step_us": unfused_ms * 1e3,
+        "unfused_breakdown_us": {k: v * 1e3 for k, v in ukern_ms.items()},
         "dense_conv_us": dense_conv_ms * 1e3, "sparse_conv_us": sparse_conv_ms * 1e3,
         "speedup_vs_dense_conv": dense_conv_ms / sparse_conv_ms,
         "step_roofline_frac": t_roof / (step_ms * 1e-3),
@@ -701,7 +744,7 @@ def run_sige(args):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_ms * 1e3, "unit": "us", "h2d_bytes_per_step": host_in.numel() * host_in.element_size(),
                 "d2h_bytes_per_step": host_out.numel() * host_out.element_size(),
-                "api": "sige_reduce_mask + 2x sige_conv_fused, eager, pinned host buffers"},
+                "api": "sige_reduce_mask + sige_resblock_fused, eager, pinned host buffers"},
         "gpu_launches": sum(launches.values()) * args.steps,
         "clocks": clocks,
         "conv_path": "tcgen05" if sige.sige_conv_path(d["cd"], torch.bfloat16) == 1 else "cuda-core",
@@ -710,11 +753,8 @@ def run_sige(args):
         line.update(extras)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    for g in list(graphs.values()) + list(dgraphs.values()) + list(step_graph.values()):
-        del g
-    graphs.clear()
-    step_graph.clear()
-    dgraphs.clear()
+    for gd in (graphs, dgraphs, step_graph, ugraph, ugraphs):
+        gd.clear()
     if ws > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

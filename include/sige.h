@@ -241,6 +241,48 @@ int sige_conv_fused(const void *x, const sige_tensor_desc *xd, const void *weigh
                     const sige_tensor_desc *yd, void *workspace, size_t workspace_bytes,
                     sige_stream_t stream);
 
+/* (6) The residual block of a diffusion UNet on the active tiles, in one
+ * launch: two chained layers F_l run on the gathered active blocks, each
+ * updating its cached output (SIGE project page, "Overview"; mer.dev notes on
+ * SIGE, section 3 "Method": cached activations reused outside the edit):
+ *   y1  = conv3x3(SiLU(x * gn1_scale + gn1_shift), w1) + b1        -> cached y1
+ *   out = conv3x3(SiLU(y1 * gn2_scale + gn2_shift), w2) + b2 + x   -> cached out
+ * on every in-image pixel of the first min(*count, capacity) tiles of `idx`
+ * (8 x 8, stride 1, zero padding); y1 is rounded to bf16 before GroupNorm2, as
+ * if stored; every other byte of y1 and out is left untouched.  conv2 reads y1
+ * on the tile plus a one-pixel ring, which this call recomputes from x
+ * instead of reading the cache (y1 never goes through memory on its way to
+ * conv2), so the result equals sige_conv_fused for conv1 followed by
+ * sige_conv_fused for conv2 on the same list whenever x differs from the
+ * input the caches were computed from only at pixels whose 3 x 3 window lies
+ * in listed tiles -- true for any list from sige_reduce_mask with dilate >= 1
+ * (or sige_reduce_mask_px with radius >= 1) whose threshold catches every
+ * change.
+ *   x_edit              : device NHWC bf16 [N][H][W][128] (xd), the edited input
+ *   w1, w2              : device bf16 [128][3][3][128] (KRSC)
+ *   b1, b2              : device float32 [128] or NULL (no bias)
+ *   gn1_scale/shift,
+ *   gn2_scale/shift     : device float32 [N][128], GroupNorm folded into an
+ *                         affine (sige_groupnorm_affine of the cached x and y1)
+ *   block               : 8 (the tile edge; others return SIGE_ERR_UNSUPPORTED)
+ *   idx, count, capacity: the tile list (as sige_conv_fused)
+ *   y1, out             : device NHWC bf16, shape of x, holding the caches on
+ *                         entry; must not overlap x or each other
+ *   workspace           : device, >= SIGE_WORKSPACE_HEADER_BYTES (the device
+ *                         error word; see sige_get_device_error), 16-byte
+ *                         aligned
+ * Runs on the tensor cores in clusters of two CTAs; asynchronous on `stream`,
+ * one launch, nothing allocated.  Errors: SIGE_ERR_INVALID_ARG (NULL or
+ * misaligned list, overlapping buffers), SIGE_ERR_UNSUPPORTED (not bf16 NHWC
+ * with 128 channels and 8 x 8 tiles, misaligned tensors), SIGE_ERR_WORKSPACE,
+ * SIGE_ERR_CUDA; on the device a bounded wait that expires records
+ * SIGE_ERR_TIMEOUT. */
+int sige_resblock_fused(const void *x_edit, const sige_tensor_desc *xd, const void *w1, const float *b1,
+                        const float *gn1_scale, const float *gn1_shift, const void *w2, const float *b2,
+                        const float *gn2_scale, const float *gn2_shift, int32_t block, const int32_t *idx,
+                        const int32_t *count, int32_t capacity, void *y1, void *out, void *workspace,
+                        size_t workspace_bytes, sige_stream_t stream);
+
 /* The same layer on every tile of the output: the dense conv that fills the
  * cache F_l(A_original) and the dense baseline the sparse path is compared
  * with.  y is fully written. */

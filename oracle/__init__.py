@@ -62,6 +62,12 @@ def lib():
         L.oracle_sparse_conv.argtypes = conv_common + [i32, vp, i32, vp, vp, i32, vp, vp, vp]
         L.oracle_gather.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp, i32, vp]
         L.oracle_block_conv.argtypes = [vp, i32, i32, vp, i32, i32, i32, i32, i32, vp]
+        L.oracle_conv_transpose_f64.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, i32, i32, i32, i32, i32,
+                                                vp, vp, i32, vp, vp]
+        L.oracle_sparse_conv_transpose.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, i32, i32, i32, i32, i32,
+                                                   i32, vp, i32, vp, vp, i32, vp, vp, vp]
+        L.oracle_spade_conv.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp,
+                                        i32, vp, i32, vp, i32, vp, vp, vp]
         _lib = L
     return _lib
 
@@ -285,3 +291,90 @@ def restore_tiles(src: torch.Tensor, dst: torch.Tensor, block: int, idx: np.ndar
                 if y < H and x < W:
                     out[:, y, x, :] = src[:, y, x, :]
     return out
+
+
+# ------------------------------------------------------- other layer types
+
+def conv_transpose_out_hw(H, W, k=3, stride=2, pad=1, output_padding=1):
+    return (H - 1) * stride - 2 * pad + k + output_padding, (W - 1) * stride - 2 * pad + k + output_padding
+
+
+def conv_transpose_f64(x, w, bias=None, k=3, stride=2, pad=1, output_padding=1, gn=None, silu=False,
+                       residual=None) -> np.ndarray:
+    """Transposed conv (learned upsampling), unrounded float64 [N, Ho, Wo, C_out].
+    ``w`` is [C_out, k, k, C_in]: w[o, r, c, ci] couples input channel ci to
+    output channel o at tap (r, c); input pixel (i, j) feeds output pixel
+    (i*stride - pad + r, j*stride - pad + c)."""
+    x, w = _c(x), _c(w)
+    N, H, W, Cin = x.shape
+    Cout = w.shape[0]
+    assert w.shape == (Cout, k, k, Cin) and w.dtype == x.dtype
+    Ho, Wo = conv_transpose_out_hw(H, W, k, stride, pad, output_padding)
+    b = None if bias is None else _c(bias.float())
+    sc, sh = _gn(gn)
+    r = None if residual is None else _c(residual)
+    z = np.zeros((N, Ho, Wo, Cout), dtype=np.float64)
+    lib().oracle_conv_transpose_f64(_p(x), N, H, W, Cin, _dtype_code(x), _p(w), _p(b), Cout, k, stride, pad,
+                                    output_padding, _p(sc), _p(sh), int(silu), _p(r), _p(z))
+    return z
+
+
+def sparse_conv_transpose(x_edit, w, bias, idx, y_cached, k=3, stride=2, pad=1, output_padding=1, block=4,
+                          gn=None, silu=False, residual=None) -> torch.Tensor:
+    """Tile-masked transposed conv: the cached output, overwritten at the pixels
+    of the listed output tiles (output resolution) by the layer on ``x_edit``."""
+    x, w = _c(x_edit), _c(w)
+    N, H, W, Cin = x.shape
+    Cout = w.shape[0]
+    yc = _c(y_cached)
+    Ho, Wo = conv_transpose_out_hw(H, W, k, stride, pad, output_padding)
+    assert yc.shape == (N, Ho, Wo, Cout) and yc.dtype == x.dtype
+    b = None if bias is None else _c(bias.float())
+    sc, sh = _gn(gn)
+    r = None if residual is None else _c(residual)
+    idx = np.ascontiguousarray(idx, dtype=np.int32).reshape(-1, 2)
+    y = torch.empty_like(yc)
+    lib().oracle_sparse_conv_transpose(_p(x), N, H, W, Cin, _dtype_code(x), _p(w), _p(b), Cout, k, stride, pad,
+                                       output_padding, block, _p(idx), len(idx), _p(sc), _p(sh), int(silu), _p(r),
+                                       _p(yc), _p(y))
+    return y
+
+
+ACT_NONE, ACT_SILU, ACT_LEAKY = 0, 1, 2
+
+
+def spade_conv(x, w, bias, norm, gamma, beta, act=ACT_LEAKY, k=3, stride=1, pad=1, residual=None, idx=None,
+               block=4, y_cached=None, rounded=True):
+    """Conv of a SPADE-style input: act((x * scale + shift) * (1 + gamma) + beta)
+    with (scale, shift) = ``norm`` per (n, channel) and gamma / beta per pixel
+    (NHWC maps of x's shape and dtype).  Dense (idx None) or tile-masked into
+    ``y_cached``; rounded once to x's dtype, or unrounded float64 when
+    ``rounded`` is False (dense only)."""
+    x, w = _c(x), _c(w)
+    N, H, W, Cin = x.shape
+    Cout = w.shape[0]
+    assert w.shape == (Cout, k, k, Cin) and w.dtype == x.dtype
+    g, be = _c(gamma), _c(beta)
+    assert g.shape == x.shape and be.shape == x.shape and g.dtype == x.dtype and be.dtype == x.dtype
+    Ho = (H + 2 * pad - k) // stride + 1
+    Wo = (W + 2 * pad - k) // stride + 1
+    b = None if bias is None else _c(bias.float())
+    sc, sh = _gn(norm)
+    r = None if residual is None else _c(residual)
+    if idx is None and not rounded:
+        z = np.zeros((N, Ho, Wo, Cout), dtype=np.float64)
+        lib().oracle_spade_conv(_p(x), N, H, W, Cin, _dtype_code(x), _p(w), _p(b), Cout, k, stride, pad, _p(sc),
+                                _p(sh), _p(g), _p(be), int(act), _p(r), block, None, 0, None, _p(z), None)
+        return z
+    if idx is None:
+        y = torch.empty((N, Ho, Wo, Cout), dtype=x.dtype)
+        lib().oracle_spade_conv(_p(x), N, H, W, Cin, _dtype_code(x), _p(w), _p(b), Cout, k, stride, pad, _p(sc),
+                                _p(sh), _p(g), _p(be), int(act), _p(r), block, None, 0, None, None, _p(y))
+        return y
+    yc = _c(y_cached)
+    assert yc.shape == (N, Ho, Wo, Cout) and yc.dtype == x.dtype
+    idx = np.ascontiguousarray(idx, dtype=np.int32).reshape(-1, 2)
+    y = torch.empty_like(yc)
+    lib().oracle_spade_conv(_p(x), N, H, W, Cin, _dtype_code(x), _p(w), _p(b), Cout, k, stride, pad, _p(sc),
+                            _p(sh), _p(g), _p(be), int(act), _p(r), block, _p(idx), len(idx), _p(yc), None, _p(y))
+    return y

@@ -460,3 +460,179 @@ void oracle_block_conv(const double *blocks, int nblocks, int Cin, const void *w
                 }
     free(wd);
 }
+
+/* ------------------------------------------ other layer types (GauGAN) */
+
+/* Transposed convolution (the learned upsampling layer of a generator's
+ * decoder; mer.dev notes on SIGE, section 5: GauGAN-style generators beside
+ * the plain convs), written in the textbook scatter form: every input pixel
+ * (i, j) adds W[o][r][c][ci] * X[n][i][j][ci] to output pixel
+ * (i*s - p + r, j*s - p + c), for r, c < k, when that pixel lies in the
+ * Ho x Wo output, Ho = (H - 1)*s - 2p + k + op.  The weight is stored
+ * [C_out][k][k][C_in] like every other layer here: W[o][r][c][ci] is the
+ * coupling of input channel ci to output channel o at tap (r, c).  Optional
+ * per-channel affine + SiLU on the input as in the other layers, bias, and a
+ * residual of the output's shape.  Sums in double; the scatter visits input
+ * pixels row-major and taps (r, c, ci) in order, so each output element is
+ * summed in a fixed order. */
+static void conv_transpose_f64(const void *x, int N, int H, int W, int Cin, int dtype, const void *w,
+                               const float *bias, int Cout, int k, int s, int p, int op, const double *scale,
+                               const double *shift, int silu, const void *residual, double *z)
+{
+    layer_t L;
+    layer_init(&L, N, H, W, Cin, Cout, k, 1, 0, dtype);
+    int Ho = (H - 1) * s - 2 * p + k + op, Wo = (W - 1) * s - 2 * p + k + op;
+    double *xt = transformed_input(&L, x, scale, shift, silu);
+    double *wd = weights_f64(&L, w);
+    size_t nz = (size_t)N * Ho * Wo * Cout;
+    for (size_t i = 0; i < nz; ++i)
+        z[i] = 0.0;
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n)
+        for (int i = 0; i < H; ++i)
+            for (int j = 0; j < W; ++j) {
+                const double *xp = xt + (((size_t)n * H + i) * W + j) * Cin;
+                for (int r = 0; r < k; ++r) {
+                    int y = i * s - p + r;
+                    if (y < 0 || y >= Ho)
+                        continue;
+                    for (int c = 0; c < k; ++c) {
+                        int xo = j * s - p + c;
+                        if (xo < 0 || xo >= Wo)
+                            continue;
+                        double *zp = z + (((size_t)n * Ho + y) * Wo + xo) * Cout;
+                        for (int o = 0; o < Cout; ++o) {
+                            const double *wp = wd + (((size_t)o * k + r) * k + c) * Cin;
+                            double acc = 0.0;
+                            for (int ci = 0; ci < Cin; ++ci)
+                                acc += wp[ci] * xp[ci];
+                            zp[o] += acc;
+                        }
+                    }
+                }
+            }
+    for (int n = 0; n < N; ++n)
+        for (int y = 0; y < Ho; ++y)
+            for (int xo = 0; xo < Wo; ++xo)
+                for (int o = 0; o < Cout; ++o) {
+                    size_t e = (((size_t)n * Ho + y) * Wo + xo) * Cout + o;
+                    if (bias)
+                        z[e] += (double)bias[o];
+                    if (residual)
+                        z[e] += elem_f(residual, dtype, e);
+                }
+    free(xt);
+    free(wd);
+}
+
+void oracle_conv_transpose_f64(const void *x, int N, int H, int W, int Cin, int dtype, const void *w,
+                               const float *bias, int Cout, int k, int s, int p, int op, const double *scale,
+                               const double *shift, int silu, const void *residual, double *z)
+{
+    conv_transpose_f64(x, N, H, W, Cin, dtype, w, bias, Cout, k, s, p, op, scale, shift, silu, residual, z);
+}
+
+/* Tile-masked transposed conv: the cached output, overwritten at the in-image
+ * pixels of the listed output tiles (origins in output pixels, edge `block`)
+ * by the transposed conv of x_edit rounded once to the dtype. */
+void oracle_sparse_conv_transpose(const void *x_edit, int N, int H, int W, int Cin, int dtype, const void *w,
+                                  const float *bias, int Cout, int k, int s, int p, int op, int block,
+                                  const int32_t *idx, int count, const double *scale, const double *shift,
+                                  int silu, const void *residual, const void *y_cached, void *y_out)
+{
+    int Ho = (H - 1) * s - 2 * p + k + op, Wo = (W - 1) * s - 2 * p + k + op;
+    size_t nz = (size_t)N * Ho * Wo * Cout;
+    size_t esz = dtype == O_BF16 ? 2 : 4;
+    double *z = (double *)malloc(nz * sizeof(double));
+    conv_transpose_f64(x_edit, N, H, W, Cin, dtype, w, bias, Cout, k, s, p, op, scale, shift, silu, residual, z);
+    memcpy(y_out, y_cached, nz * esz);
+    for (int n = 0; n < N; ++n)
+        for (int t = 0; t < count; ++t)
+            for (int i = 0; i < block; ++i)
+                for (int j = 0; j < block; ++j) {
+                    int y = idx[2 * t] + i, xo = idx[2 * t + 1] + j;
+                    if (y >= Ho || xo >= Wo)
+                        continue;
+                    for (int o = 0; o < Cout; ++o) {
+                        size_t e = (((size_t)n * Ho + y) * Wo + xo) * Cout + o;
+                        store_out(dtype, y_out, e, z[e]);
+                    }
+                }
+    free(z);
+}
+
+/* SPADE-style input of a GauGAN layer: a parameter-free normalisation whose
+ * per-channel statistics are folded into scale/shift (taken, like GroupNorm
+ * here, from the cached original activation), then modulated per pixel by
+ * maps the generator computes from the segmentation:
+ *   t = act((x * scale[n][c] + shift[n][c]) * (1 + gamma[n][y][x][c]) + beta[n][y][x][c])
+ * with act = identity (0), SiLU (1) or LeakyReLU with slope 0.2 (2), rounded
+ * to bf16 for bf16 layers (the stacked blocks' storage); gamma and beta are
+ * NHWC maps of x's shape and dtype.  The conv that follows is the plain
+ * direct conv above. */
+static double *spade_input(const layer_t *L, const void *x, const double *scale, const double *shift,
+                           const void *gamma, const void *beta, int act)
+{
+    size_t n = (size_t)L->N * L->H * L->W * L->Cin;
+    double *t = (double *)malloc(n * sizeof(double));
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < (long)n; ++i) {
+        int c = (int)(i % L->Cin);
+        int nn = (int)(i / ((size_t)L->H * L->W * L->Cin));
+        double v = elem_f(x, L->dtype, (size_t)i);
+        v = v * scale[(size_t)nn * L->Cin + c] + shift[(size_t)nn * L->Cin + c];
+        v = v * (1.0 + elem_f(gamma, L->dtype, (size_t)i)) + elem_f(beta, L->dtype, (size_t)i);
+        if (act == 1)
+            v = v / (1.0 + exp(-v));
+        else if (act == 2)
+            v = v >= 0.0 ? v : 0.2 * v;
+        if (L->dtype == O_BF16)
+            v = bf16_roundtrip(v);
+        t[i] = v;
+    }
+    return t;
+}
+
+/* Dense conv of the SPADE input, unrounded (z) or, when y != NULL, rounded
+ * once into y; and its tile-masked form when idx != NULL (y_out = y_cached
+ * except at the listed tiles). */
+void oracle_spade_conv(const void *x, int N, int H, int W, int Cin, int dtype, const void *w, const float *bias,
+                       int Cout, int k, int stride, int pad, const double *scale, const double *shift,
+                       const void *gamma, const void *beta, int act, const void *residual, int block,
+                       const int32_t *idx, int count, const void *y_cached, double *z, void *y_out)
+{
+    layer_t L;
+    layer_init(&L, N, H, W, Cin, Cout, k, stride, pad, dtype);
+    double *xt = spade_input(&L, x, scale, shift, gamma, beta, act);
+    double *wd = weights_f64(&L, w);
+    size_t esz = dtype == O_BF16 ? 2 : 4;
+    if (idx && y_out)
+        memcpy(y_out, y_cached, (size_t)N * L.Ho * L.Wo * Cout * esz);
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int n = 0; n < N; ++n)
+        for (int yo = 0; yo < L.Ho; ++yo) {
+            double *acc = (double *)malloc(sizeof(double) * Cout);
+            for (int xo = 0; xo < L.Wo; ++xo) {
+                int listed = 1;
+                if (idx) {
+                    listed = 0;
+                    for (int t = 0; t < count && !listed; ++t)
+                        listed = yo >= idx[2 * t] && yo < idx[2 * t] + block && xo >= idx[2 * t + 1] &&
+                                 xo < idx[2 * t + 1] + block;
+                }
+                if (!listed)
+                    continue;
+                conv_pixel(&L, xt, wd, bias, residual, n, yo, xo, acc);
+                size_t e0 = (((size_t)n * L.Ho + yo) * L.Wo + xo) * Cout;
+                for (int o = 0; o < Cout; ++o) {
+                    if (z)
+                        z[e0 + o] = acc[o];
+                    if (y_out)
+                        store_out(dtype, y_out, e0 + o, acc[o]);
+                }
+            }
+            free(acc);
+        }
+    free(xt);
+    free(wd);
+}

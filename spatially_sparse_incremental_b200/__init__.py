@@ -61,6 +61,8 @@ SIGNATURES = {
                                _vp, _sz, _vp]),
     "sige_dense_conv": (_i32, [_vp, _TD, _vp, _vp, _CD, _vp, _vp, _i32, _vp, _vp, _TD, _vp, _sz, _vp]),
     "sige_groupnorm_affine": (_i32, [_vp, _TD, _i32, _vp, _vp, _f32, _vp, _vp, _vp]),
+    "sige_resblock_fused": (_i32, [_vp, _TD, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp,
+                                   _vp, _vp, _sz, _vp]),
     "sige_restore_tiles": (_i32, [_vp, _vp, _TD, _i32, _vp, _vp, _i32, _vp]),
     "sige_conv_workspace_bytes": (_sz, [_CD, _i32, _i32, _i32, _i32]),
     "sige_get_error": (_i32, [_vp, _vp]),
@@ -282,6 +284,22 @@ def sige_dense_conv(x, weight, bias, cd: ConvDesc, y=None, gn_scale=None, gn_shi
                                ctypes.byref(yd), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "sige_dense_conv")
     return y
+
+
+def sige_resblock_fused(x_edit, w1, b1, gn1, w2, b2, gn2, idx, count, capacity, y1, out, block=8,
+                        workspace=None, stream=None):
+    """The res block on the active tiles in one launch: y1 and out (the caches,
+    NHWC bf16) are updated in place at the listed 8x8 tiles.  ``gn1`` / ``gn2``
+    are (scale, shift) pairs from sige_groupnorm_affine; biases may be None."""
+    xd = tensor_desc(x_edit)
+    if workspace is None:
+        workspace = zeros_workspace(WORKSPACE_HEADER, x_edit.device)
+    st = lib().sige_resblock_fused(_ptr(x_edit), ctypes.byref(xd), _ptr(w1), _ptr(b1), _ptr(gn1[0]), _ptr(gn1[1]),
+                                   _ptr(w2), _ptr(b2), _ptr(gn2[0]), _ptr(gn2[1]), int(block), _ptr(idx),
+                                   _ptr(count), int(capacity), _ptr(y1), _ptr(out), _ptr(workspace),
+                                   workspace.numel(), _stream(stream))
+    _check(st, "sige_resblock_fused")
+    return y1, out
 
 
 def sige_groupnorm_affine(x, groups, gamma, beta, eps=1e-5, scale=None, shift=None, stream=None):

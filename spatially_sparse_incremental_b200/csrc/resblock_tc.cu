@@ -1,0 +1,708 @@
+// The sparse residual block in one launch: GroupNorm1+SiLU -> 3x3 conv1 (+b1)
+// -> GroupNorm2+SiLU -> 3x3 conv2 (+b2 + x) on the active 8x8 tiles, with the
+// intermediate y1 kept on chip.  SIGE project page, "Overview": the layers F_l
+// run on the gathered active blocks one after the other, each scattering into
+// its cached output; mer.dev notes on SIGE, section 3 "Method": the cached
+// activations of the original image are reused everywhere else.
+//
+// Halo recompute.  conv2 on an 8x8 tile reads y1 on the tile plus a one-pixel
+// ring, and y1 there needs x on the tile plus a two-pixel ring.  Each tile's
+// y1 is therefore computed on 10 x 10 pixels (1.56x the MACs of conv1 on the
+// tile alone) from a 12 x 12 halo of x, and never goes through memory on its
+// way to conv2.  Where the ring falls in another active tile this is the value
+// that tile writes; where it falls in an inactive tile, no input of its 3x3
+// window was edited (the list is dilated by at least one pixel beyond every
+// edit), so it is the cached value.  The tile interior of y1 is still written
+// to the cached y1, which stays valid for the next edit.
+//
+// Data path of one tile (one "unit"), on a cluster of two CTAs; CTA r owns
+// output channels [64 r, 64 r + 64) of both convs:
+//   * x halo: one TMA per 64 channels, box (8 channels, 12 x, 12 y, 8 channel
+//     groups) of a 5-d view of the NHWC tensor, zero outside the image (the
+//     conv's padding); shared layout [channel group][12 x 12 pixels][8 ch],
+//     then GroupNorm1 + SiLU in place at in-image pixels;
+//   * conv1 as an implicit GEMM D[pixel][c_out] = X[pixel][K] W1[c_out][K]^T,
+//     K = (64-channel chunk, tap): A = the halo, read as 128 consecutive
+//     "flat" pixels o = 12 yy + xx (pitch 12), the tap (r, c) being an offset
+//     of 12 r + c pixels of the descriptor's start address (rows whose xx >= 10
+//     are discarded); B = W1, 64 output channels x 64 K per TMA stage
+//     (128-byte swizzle); D in tensor memory, one lane per flat pixel;
+//   * epilogue 1: y1 = round_bf16(D + b1), stored to the cached y1 at the tile
+//     interior; t = round_bf16(SiLU(GN2(y1))) (zero outside the image) into the
+//     conv2 input buffer [channel group][10 x 10 pixels][8 ch] of BOTH CTAs
+//     (distributed shared memory), so each holds all 128 channels;
+//   * conv2 the same way on that buffer (pitch 10, rows with j >= 8 discarded);
+//   * epilogue 2: out = round_bf16(D + b2 + x) at the tile's 64 pixels.
+//
+// Warp roles (320 threads): warp 0 streams the weight stages (TMA), warp 1
+// owns tensor memory and issues the MMAs (one elected lane), warps 2-9 load
+// and transform the x halo and run both epilogues (warp w reads tensor-memory
+// lanes 32 (w mod 4) .. +31, and half (w - 2) / 4 of the 64 columns).  The
+// CTA pair walks the units with a stride of the number of pairs; while the
+// epilogue of tile k's conv2 runs, the halo of tile k+1 is already loaded and
+// conv1 of tile k+1 is on the tensor cores.  Every wait is bounded: on
+// expiry the kernel records SIGE_ERR_TIMEOUT (detail = wait site), the roles
+// leave their loops, outstanding copies and MMAs are drained (bounded) and
+// tensor memory is freed.
+#include <algorithm>
+#include <atomic>
+
+#include "tc_ptx.cuh"
+#include "transform.cuh"
+
+namespace sige {
+namespace rb {
+
+constexpr int kThreads = 320;
+constexpr int kEpi = 256;                  // halo / epilogue threads (warps 2-9)
+constexpr int kC = 128;                    // channels of x, y1 and out
+constexpr int kB = 8;                      // output tile edge
+constexpr int kXE = 12;                    // x halo edge (tile + 2-pixel ring)
+constexpr int kXPix = kXE * kXE;           // 144
+constexpr uint32_t kXKc = kXPix * 16;      // bytes of one 8-channel group of the halo
+constexpr uint32_t kXHalf = 8 * kXKc;      // 64 channels of the halo (one TMA)
+constexpr int kYE = 10;                    // conv2 input edge (tile + 1-pixel ring)
+constexpr uint32_t kYKc = kYE * kYE * 16;  // bytes of one 8-channel group of the conv2 input
+constexpr uint32_t kWStage = 64 * 64 * 2;  // 64 output channels x 64 K, bf16
+constexpr int kStages = 20;                // weight ring
+constexpr int kChunks = 18;                // weight stages per conv: 2 channel chunks x 9 taps
+constexpr uint32_t kOffX = 1024;
+constexpr uint32_t kOffY = kOffX + 16 * kXKc;
+constexpr uint32_t kOffW = ((kOffY + 16 * kYKc + 1023) / 1024) * 1024;
+constexpr uint32_t kSmem = kOffW + kStages * kWStage + 1024;   // + alignment of the base
+constexpr uint32_t kTmemCols = 128;        // conv1 accumulator [0, 64), conv2 [64, 128)
+static_assert(kSmem <= 232448, "shared memory");
+static_assert(kOffX % 128 == 0 && kXHalf % 128 == 0 && kOffY % 16 == 0, "TMA destinations");
+
+// mbarriers and control words in [0, 1024)
+constexpr uint32_t kBarWFull = 0, kBarWEmpty = 160, kBarXFull = 320, kBarXReady = 336;
+constexpr uint32_t kBarAcc1Full = 352, kBarAcc1Empty = 360, kBarAcc2Full = 368, kBarAcc2Empty = 376;
+constexpr uint32_t kBarY1tFull = 384, kBarY1tEmpty = 392, kBarDrain = 400;
+constexpr uint32_t kTmemSlot = 512, kAbort = 516;
+
+// wait sites recorded in the error detail on a timeout
+enum : int { kSiteWEmpty = 101, kSiteWFull, kSiteXReady, kSiteAcc1Empty, kSiteAcc2Empty, kSiteY1tFull,
+             kSiteXFull, kSiteAcc1Full, kSiteY1tEmpty, kSiteAcc2Full };
+
+}  // namespace rb
+
+struct RbArgs {
+    const uint8_t *x;           // x_edit, NHWC bf16 [N][H][W][128]
+    const int32_t *idx;         // tile origins (h0, w0)
+    const int32_t *count;
+    const float *b1, *b2;       // [128] or null
+    const float *g1s, *g1h;     // GroupNorm1 affine [N][128]
+    const float *g2s, *g2h;     // GroupNorm2 affine [N][128]
+    uint8_t *y1;                // cached y1, updated at the tile interiors
+    uint8_t *out;               // cached out, updated at the tiles
+    WsHeader *hdr;
+    int32_t N, H, W, cap;
+};
+
+// Four K=16 MMAs of one 64-channel weight stage: A (pixels, no swizzle)
+// advances by a_step (descriptor units of 16 bytes) per step, B (weights,
+// 128-byte swizzle) by 32 bytes; then the commit that frees the stage.  One
+// elected lane issues.
+__device__ __forceinline__ void rb_mma4(uint32_t d_tmem, uint64_t a_desc, uint64_t a_step, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate, uint32_t bar)
+{
+    asm volatile(
+        "{\n .reg .pred p, e, t;\n .reg .b32 l;\n .reg .b64 a1, a2, a3, b1, b2, b3;\n"
+        " elect.sync l|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n setp.eq.b32 t, 0, 0;\n"
+        " add.s64 a1, %1, %5;\n add.s64 a2, a1, %5;\n add.s64 a3, a2, %5;\n"
+        " add.s64 b1, %2, 2;\n add.s64 b2, %2, 4;\n add.s64 b3, %2, 6;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, t;\n"
+        " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "l"(a_step), "r"(bar)
+        : "memory");
+}
+
+// Commit that arrives on the mbarrier at offset `bar` of both CTAs of the pair.
+__device__ __forceinline__ void rb_commit_pair(uint32_t bar)
+{
+    asm volatile(
+        "{\n .reg .pred e;\n .reg .b32 l;\n .reg .b16 m;\n elect.sync l|e, 0xffffffff;\n mov.b16 m, 3;\n"
+        " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n}\n"
+        ::"r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int k = 0; k < 32; ++k)
+        v[k] = __uint_as_float(r[k]);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v)
+{
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_peer_v4(uint32_t addr, uint4 v)
+{
+    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cluster_arrive_rel() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait_acq() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+
+__global__ void __launch_bounds__(rb::kThreads, 1)
+    k_resblock(const __grid_constant__ RbArgs args, const __grid_constant__ CUtensorMap tmx,
+               const __grid_constant__ CUtensorMap tw1, const __grid_constant__ CUtensorMap tw2)
+{
+    using namespace rb;
+    const RbArgs p = args;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
+    const uint32_t sb = smem_u32(smem);
+    auto w_full = [&](int i) { return sb + kBarWFull + 8u * i; };
+    auto w_empty = [&](int i) { return sb + kBarWEmpty + 8u * i; };
+    auto x_full = [&](int h) { return sb + kBarXFull + 8u * h; };
+    auto x_ready = [&](int h) { return sb + kBarXReady + 8u * h; };
+    const uint32_t acc1_full = sb + kBarAcc1Full, acc1_empty = sb + kBarAcc1Empty;
+    const uint32_t acc2_full = sb + kBarAcc2Full, acc2_empty = sb + kBarAcc2Empty;
+    const uint32_t y1t_full = sb + kBarY1tFull, y1t_empty = sb + kBarY1tEmpty, drain = sb + kBarDrain;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kAbort);
+    WsHeader *hdr = p.hdr;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();          // output-channel half of this CTA
+    const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(w_full(i), 1);
+            mbar_init(w_empty(i), 1);
+        }
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(x_full(h), 1);
+            mbar_init(x_ready(h), kEpi);
+        }
+        mbar_init(acc1_full, 1);
+        mbar_init(acc1_empty, kEpi);
+        mbar_init(acc2_full, 1);
+        mbar_init(acc2_empty, kEpi);
+        mbar_init(y1t_full, 2 * kEpi);   // the epilogue threads of both CTAs
+        mbar_init(y1t_empty, 2);         // the conv2 commits of both CTAs
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tw1)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tw2)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmx)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sb + kTmemSlot),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + kTmemSlot);
+    // Both CTAs' barriers are initialised before either side signals the
+    // other: every thread waits on this cluster barrier before its first
+    // access to the peer (and before the final one).
+    cluster_arrive_rel();
+    bool cwaited = false;
+    pdl_trigger();
+
+    if (warp == 0) {
+        // ------------------------------------------------ weight stages (TMA)
+        // The weights do not come from the previous kernel: the first stages
+        // of W1 go out before the wait for it.
+        int s = 0, issued = 0;
+        uint32_t ph = 1;
+        bool ok = true;
+        auto issue = [&](int conv, int j) -> bool {
+            if (!mbar_wait_w(w_empty(s), ph, abort_flag, hdr, kSiteWEmpty))
+                return false;
+            const int kc2 = j / 9, tap = j - kc2 * 9;
+            tma_load_2d_w(sb + kOffW + (uint32_t)s * kWStage, conv ? &tw2 : &tw1, w_full(s), kWStage,
+                          tap * kC + kc2 * 64, (int)rank * 64);
+            ++issued;
+            if (++s == kStages) {
+                s = 0;
+                ph ^= 1;
+            }
+            return true;
+        };
+        const int pre = kStages < kChunks ? kStages : kChunks;
+        for (int j = 0; j < pre && ok; ++j)
+            ok = issue(0, j);
+        pdl_wait();
+        const int units = min(__ldg(p.count), p.cap) * p.N;
+        bool first = true;
+#pragma unroll 1
+        for (int u = pair; u < units && ok; u += npairs) {
+#pragma unroll 1
+            for (int conv = 0; conv < 2 && ok; ++conv)
+#pragma unroll 1
+                for (int j = (first && conv == 0) ? pre : 0; j < kChunks && ok; ++j)
+                    ok = issue(conv, j);
+            first = false;
+        }
+        // every load must land before the CTA may exit: wait for the last
+        // use of each ring slot (a prefetch nothing consumed included)
+#pragma unroll 1
+        for (int k = 1; k <= kStages && k <= issued; ++k) {
+            const int g = issued - k;
+            const int st = g % kStages;
+            const uint32_t par = (uint32_t)(g / kStages) & 1u;
+            const long long t0 = clock64();
+            while (!mbar_try(w_full(st), par) && clock64() - t0 < kWaitCycles) {
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        pdl_wait();
+        const int units = min(__ldg(p.count), p.cap) * p.N;
+        const uint32_t idesc = idesc_bf16(64);          // M = 128 pixels, N = 64 output channels
+        const uint64_t b_desc0 = desc_sw128(sb + kOffW);
+        const uint64_t w_step = kWStage >> 4;
+        int s = 0;
+        uint32_t ph = 0, ait = 0;
+        bool ok = true;
+        cluster_wait_acq();
+        cwaited = true;
+        uint64_t b_cur = b_desc0;
+        // one conv: 2 chunks of 64 input channels x 9 taps, A = the pixel
+        // buffer at `a_base` (pitch `pitch`, 8-channel groups `kc_bytes` apart)
+        auto conv = [&](uint32_t a_base, int pitch, uint32_t kc_bytes, uint32_t d_col, bool wait_x, uint32_t xpar)
+            -> bool {
+            const uint64_t a_step = (2 * kc_bytes) >> 4;
+#pragma unroll 1
+            for (int kc2 = 0; kc2 < 2; ++kc2) {
+                if (wait_x) {
+                    if (!mbar_wait_w(x_ready(kc2), xpar, abort_flag, hdr, kSiteXReady))
+                        return false;
+                    tc_fence_after();
+                }
+                const uint32_t chunk = a_base + (uint32_t)kc2 * 8u * kc_bytes;
+#pragma unroll 1
+                for (int tap = 0; tap < 9; ++tap) {
+                    const int r = tap / 3, c = tap - r * 3;
+                    if (!mbar_wait_w(w_full(s), ph, abort_flag, hdr, kSiteWFull))
+                        return false;
+                    tc_fence_after();
+                    const uint64_t a_desc = desc_plain(chunk + (uint32_t)(pitch * r + c) * 16u, kc_bytes, 128);
+                    rb_mma4(tmem + d_col, a_desc, a_step, b_cur, idesc, (kc2 | tap) ? 1u : 0u, w_empty(s));
+                    ++ait;
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1;
+                        b_cur = b_desc0;
+                    } else {
+                        b_cur += w_step;
+                    }
+                }
+            }
+            return true;
+        };
+        uint32_t k = 0;
+#pragma unroll 1
+        for (int u = pair; u < units && ok; u += npairs, ++k) {
+            // conv1: accumulator [0, 64) free once epilogue 1 of the previous tile has read it
+            if (k > 0 && !mbar_wait_w(acc1_empty, (k - 1) & 1, abort_flag, hdr, kSiteAcc1Empty)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (!conv(sb + kOffX, kXE, kXKc, 0, true, k & 1)) {
+                ok = false;
+                break;
+            }
+            tc_commit_w(acc1_full);
+            // conv2: its input written by both CTAs' epilogue 1
+            if (k > 0 && !mbar_wait_w(acc2_empty, (k - 1) & 1, abort_flag, hdr, kSiteAcc2Empty)) {
+                ok = false;
+                break;
+            }
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(y1t_full, k & 1, abort_flag, hdr, kSiteY1tFull))) {
+                ok = false;
+                break;
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tc_fence_after();
+            if (!conv(sb + kOffY, kYE, kYKc, 64, false, 0)) {
+                ok = false;
+                break;
+            }
+            tc_commit_w(acc2_full);
+            // the conv2 input buffers of both CTAs may be rewritten (none is
+            // after the pair's last tile)
+            if (u + npairs < units)
+                rb_commit_pair(y1t_empty);
+        }
+        // every MMA issued here completes before tensor memory is freed
+        if (ait > 0) {
+            tc_commit_w(drain);
+            const long long t0 = clock64();
+            while (!mbar_try(drain, 0) && clock64() - t0 < kWaitCycles) {
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ x halo + epilogues
+        const int et = threadIdx.x - 64;
+        const int sp = warp & 3;                       // tensor-memory subpartition
+        const int colh = (warp - 2) >> 2;              // columns [32 colh, 32 colh + 32)
+        const int row = sp * 32 + lane;                // accumulator lane = flat pixel
+        const uint32_t t_lane = tmem + ((uint32_t)(sp * 32) << 16);
+        const int cb = (int)rank * 64 + colh * 32;     // first output channel of this thread
+        const int H = p.H, W = p.W;
+        pdl_wait();
+        const int units = min(__ldg(p.count), p.cap) * p.N;
+        bool ok = true, x_pending = false;
+        uint32_t xk = 0;                               // halos loaded so far (phase of x_full / x_ready)
+
+        auto origin = [&](int u, int &h0, int &w0, int &n) {
+            const int2 o = __ldg(reinterpret_cast<const int2 *>(p.idx) + u / p.N);
+            h0 = o.x;
+            w0 = o.y;
+            n = u % p.N;
+        };
+        // Load the x halo of unit u (thread 0 issues both TMAs) and apply
+        // GroupNorm1 + SiLU in place at its in-image pixels.  The halo buffer
+        // is free: conv1 of the previous tile has completed.
+        auto load_x = [&](int u) -> bool {
+            int h0, w0, n;
+            origin(u, h0, w0, n);
+            if (et == 0) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    mbar_expect_tx(x_full(h), kXHalf);
+                    tma_load_5d(sb + kOffX + (uint32_t)h * kXHalf, &tmx, x_full(h), 0, w0 - 2, h0 - 2, h * 8, n);
+                }
+                x_pending = true;
+            }
+            const int kcl = et >> 5;
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                const int ch = (h * 8 + kcl) * 8;
+                float gs[8], gh[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    gs[q] = __ldg(p.g1s + n * kC + ch + q);
+                    gh[q] = __ldg(p.g1h + n * kC + ch + q);
+                }
+                if (!mbar_wait_w(x_full(h), xk & 1, abort_flag, hdr, kSiteXFull))
+                    return false;
+                if (h == 1 && et == 0)
+                    x_pending = false;
+                uint8_t *base = smem + kOffX + h * kXHalf + kcl * kXKc;
+#pragma unroll 1
+                for (int px = lane; px < kXPix; px += 32) {
+                    const int yy = px / kXE, xx = px - yy * kXE;
+                    const int Y = h0 - 2 + yy, X = w0 - 2 + xx;
+                    if (Y >= 0 && Y < H && X >= 0 && X < W) {
+                        uint4 *d = reinterpret_cast<uint4 *>(base + px * 16);
+                        *d = transform16_bf16_reg(*d, gs, gh, true, 1);
+                    }
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(x_ready(h));
+            }
+            ++xk;
+            return true;
+        };
+
+        if (pair < units)
+            ok = load_x(pair);
+        uint32_t k = 0;
+#pragma unroll 1
+        for (int u = pair; u < units && ok; u += npairs, ++k) {
+            int h0, w0, n;
+            origin(u, h0, w0, n);
+            // ------------ epilogue 1: y1 on the 10 x 10 pixels (flat o = 12 yy + xx)
+            {
+                const int yy = row / kXE, xx = row - yy * kXE;
+                const bool valid = yy < kYE && xx < kYE;
+                const int Y = h0 - 1 + yy, X = w0 - 1 + xx;
+                const bool inimg = valid && Y >= 0 && Y < H && X >= 0 && X < W;
+                const bool interior = inimg && yy >= 1 && yy <= kB && xx >= 1 && xx <= kB;
+                float bias[32], gs[32], gh[32];
+#pragma unroll
+                for (int q = 0; q < 32; q += 4) {
+                    const float4 b = p.b1 ? __ldg(reinterpret_cast<const float4 *>(p.b1 + cb + q))
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4 s4 = __ldg(reinterpret_cast<const float4 *>(p.g2s + n * kC + cb + q));
+                    const float4 h4 = __ldg(reinterpret_cast<const float4 *>(p.g2h + n * kC + cb + q));
+                    bias[q] = b.x; bias[q + 1] = b.y; bias[q + 2] = b.z; bias[q + 3] = b.w;
+                    gs[q] = s4.x; gs[q + 1] = s4.y; gs[q + 2] = s4.z; gs[q + 3] = s4.w;
+                    gh[q] = h4.x; gh[q + 1] = h4.y; gh[q + 2] = h4.z; gh[q + 3] = h4.w;
+                }
+                if (!mbar_wait_w(acc1_full, k & 1, abort_flag, hdr, kSiteAcc1Full)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                float v[32];
+                tmem_ld32(t_lane + (uint32_t)(colh * 32), v);
+                uint32_t y1p[16], tp[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    y1p[q] = pack_bf16x2(v[2 * q] + bias[2 * q], v[2 * q + 1] + bias[2 * q + 1]);
+                    float a = __fmaf_rn(bf16_lo(y1p[q]), gs[2 * q], gh[2 * q]);
+                    float b = __fmaf_rn(bf16_hi(y1p[q]), gs[2 * q + 1], gh[2 * q + 1]);
+                    tp[q] = inimg ? pack_bf16x2(silu_f(a), silu_f(b)) : 0u;
+                }
+                if (interior) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.y1 + ((((int64_t)n * H + Y) * W + X) * kC + cb) * 2);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        dst[g] = make_uint4(y1p[4 * g], y1p[4 * g + 1], y1p[4 * g + 2], y1p[4 * g + 3]);
+                }
+                // the accumulator may take the next tile's conv1
+                tc_fence_before();
+                mbar_arrive(acc1_empty);
+                // both CTAs' conv2 of the previous tile have read the buffers
+                if (!cwaited) {
+                    cluster_wait_acq();
+                    cwaited = true;
+                }
+                if (k > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait_cluster(y1t_empty, (k - 1) & 1, abort_flag, hdr,
+                                                                        kSiteY1tEmpty))) {
+                    ok = false;
+                    break;
+                }
+                if (valid) {
+                    const uint32_t pix = (uint32_t)(yy * kYE + xx) * 16u;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        const uint32_t off = sb + kOffY + (uint32_t)(cb / 8 + g) * kYKc + pix;
+                        const uint4 w4 = make_uint4(tp[4 * g], tp[4 * g + 1], tp[4 * g + 2], tp[4 * g + 3]);
+                        st_shared_v4(off, w4);
+                        st_peer_v4(map_peer(off, rank ^ 1u), w4);
+                    }
+                }
+                asm volatile("fence.proxy.async;" ::: "memory");
+                mbar_arrive(y1t_full);
+                mbar_arrive_peer(map_peer(y1t_full, rank ^ 1u));
+            }
+            // ------------ the next tile's halo, while conv2 of this one runs
+            if (u + npairs < units && !load_x(u + npairs)) {
+                ok = false;
+                break;
+            }
+            // ------------ epilogue 2: out on the tile's 8 x 8 pixels (flat o = 10 i + j)
+            {
+                const int i = row / kYE, j = row - i * kYE;
+                const int Y = h0 + i, X = w0 + j;
+                const bool inimg = i < kB && j < kB && Y < H && X < W;
+                const int64_t e = (((int64_t)n * H + Y) * W + X) * kC + cb;
+                uint4 res[4];
+                float bias[32];
+#pragma unroll
+                for (int g = 0; g < 4; ++g)
+                    res[g] = inimg ? __ldg(reinterpret_cast<const uint4 *>(p.x + e * 2) + g) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int q = 0; q < 32; q += 4) {
+                    const float4 b = p.b2 ? __ldg(reinterpret_cast<const float4 *>(p.b2 + cb + q))
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                    bias[q] = b.x; bias[q + 1] = b.y; bias[q + 2] = b.z; bias[q + 3] = b.w;
+                }
+                if (!mbar_wait_w(acc2_full, k & 1, abort_flag, hdr, kSiteAcc2Full)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                float v[32];
+                tmem_ld32(t_lane + 64u + (uint32_t)(colh * 32), v);
+                tc_fence_before();
+                mbar_arrive(acc2_empty);
+                if (inimg) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + e * 2);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        const uint32_t *r = reinterpret_cast<const uint32_t *>(&res[g]);
+                        uint32_t o4[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int c0 = 8 * g + 2 * q;
+                            o4[q] = pack_bf16x2((v[c0] + bias[c0]) + bf16_lo(r[q]),
+                                                (v[c0 + 1] + bias[c0 + 1]) + bf16_hi(r[q]));
+                        }
+                        dst[g] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                    }
+                }
+            }
+        }
+        // a halo copy still in flight (a wait gave up) lands before the exit
+        if (x_pending) {
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                const long long t0 = clock64();
+                while (!mbar_try(x_full(h), xk & 1) && clock64() - t0 < kWaitCycles) {
+                }
+            }
+        }
+    }
+
+    if (!cwaited)
+        cluster_wait_acq();
+    tc_fence_before();
+    __syncthreads();
+    // no CTA leaves while its peer may still write to it
+    cluster_arrive_rel();
+    cluster_wait_acq();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+    }
+}
+
+// ------------------------------------------------------------------ host
+
+static bool encode_weights(CUtensorMap *map, const void *w, PFN_cuTensorMapEncodeTiled_v12000 encode)
+{
+    const cuuint64_t K = 9 * rb::kC;
+    cuuint64_t dims[2] = {K, (cuuint64_t)rb::kC};
+    cuuint64_t strides[1] = {K * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t es[2] = {1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(w), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 5-d view [n][kc][y][x][8 channels] of the NHWC tensor, so that one box
+// lands as [channel group][y][x][8 channels] in shared memory.
+static bool encode_halo(CUtensorMap *map, const void *x, int N, int H, int W,
+                        PFN_cuTensorMapEncodeTiled_v12000 encode)
+{
+    const cuuint64_t C = rb::kC;
+    cuuint64_t dims[5] = {8, (cuuint64_t)W, (cuuint64_t)H, C / 8, (cuuint64_t)N};
+    cuuint64_t strides[4] = {C * 2, (cuuint64_t)W * C * 2, 16, (cuuint64_t)H * W * C * 2};
+    cuuint32_t box[5] = {8, (cuuint32_t)rb::kXE, (cuuint32_t)rb::kXE, 8, 1};
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(x), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bool aligned(const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) == 0; }
+
+static bool overlaps(const void *a, const void *b, size_t n)
+{
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + n && y < x + n;
+}
+
+} // namespace sige
+
+using namespace sige;
+
+extern "C" int sige_resblock_fused(const void *x_edit, const sige_tensor_desc *xd, const void *w1, const float *b1,
+                                   const float *gn1_scale, const float *gn1_shift, const void *w2, const float *b2,
+                                   const float *gn2_scale, const float *gn2_shift, int32_t block,
+                                   const int32_t *idx, const int32_t *count, int32_t capacity, void *y1, void *out,
+                                   void *workspace, size_t workspace_bytes, sige_stream_t stream)
+{
+    if (!x_edit || !xd || !w1 || !w2 || !gn1_scale || !gn1_shift || !gn2_scale || !gn2_shift || !idx || !count ||
+        !y1 || !out || capacity < 0)
+        return SIGE_ERR_INVALID_ARG;
+    if (xd->n < 1 || xd->h < 1 || xd->w < 1 || xd->c < 1 || block < 1)
+        return SIGE_ERR_INVALID_ARG;
+    if (xd->dtype != SIGE_BF16 || xd->layout != SIGE_NHWC || xd->c != rb::kC || block != rb::kB)
+        return SIGE_ERR_UNSUPPORTED;
+    if (!aligned(idx, 8))
+        return SIGE_ERR_INVALID_ARG;
+    if (!aligned(x_edit, 16) || !aligned(w1, 16) || !aligned(w2, 16) || !aligned(y1, 16) || !aligned(out, 16) ||
+        !aligned(gn1_scale, 16) || !aligned(gn1_shift, 16) || !aligned(gn2_scale, 16) || !aligned(gn2_shift, 16) ||
+        !aligned(b1, 16) || !aligned(b2, 16))
+        return SIGE_ERR_UNSUPPORTED;
+    const size_t bytes = (size_t)xd->n * xd->h * xd->w * xd->c * 2;
+    if (overlaps(x_edit, y1, bytes) || overlaps(x_edit, out, bytes) || overlaps(y1, out, bytes))
+        return SIGE_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < kWsHeader || !aligned(workspace, 16))
+        return SIGE_ERR_WORKSPACE;
+    if (capacity == 0)
+        return SIGE_OK;
+    auto encode = get_encode();
+    if (!encode)
+        return SIGE_ERR_CUDA;
+    CUtensorMap tmx, tw1, tw2;
+    if (!encode_halo(&tmx, x_edit, xd->n, xd->h, xd->w, encode) || !encode_weights(&tw1, w1, encode) ||
+        !encode_weights(&tw2, w2, encode))
+        return SIGE_ERR_UNSUPPORTED;
+
+    RbArgs a{};
+    a.x = static_cast<const uint8_t *>(x_edit);
+    a.idx = idx;
+    a.count = count;
+    a.b1 = b1;
+    a.b2 = b2;
+    a.g1s = gn1_scale;
+    a.g1h = gn1_shift;
+    a.g2s = gn2_scale;
+    a.g2h = gn2_shift;
+    a.y1 = static_cast<uint8_t *>(y1);
+    a.out = static_cast<uint8_t *>(out);
+    a.hdr = static_cast<WsHeader *>(workspace);
+    a.N = xd->n;
+    a.H = xd->h;
+    a.W = xd->w;
+    a.cap = capacity;
+
+    // per device: the shared-memory opt-in and the number of co-resident pairs
+    static std::atomic<int> pairs_of[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return SIGE_ERR_CUDA;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.blockDim = dim3(rb::kThreads);
+    cfg.dynamicSmemBytes = rb::kSmem;
+    cfg.stream = (cudaStream_t)stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    int pairs = pairs_of[dev].load(std::memory_order_acquire);
+    if (pairs == 0) {
+        if (cudaFuncSetAttribute(k_resblock, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rb::kSmem) !=
+            cudaSuccess)
+            return SIGE_ERR_CUDA;
+        cfg.gridDim = dim3(2 * (device_sm_count() / 2));
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, k_resblock, &cfg) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            return SIGE_ERR_CUDA;
+        }
+        pairs = n;
+        pairs_of[dev].store(n, std::memory_order_release);
+    }
+    const int64_t units = (int64_t)capacity * xd->n;
+    cfg.gridDim = dim3(2 * (unsigned)std::min<int64_t>(pairs, units));
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_resblock, a, tmx, tw1, tw2);
+    count_launch();
+    if (e != cudaSuccess)
+        return SIGE_ERR_CUDA;
+    return launch_check();
+}

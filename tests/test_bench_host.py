@@ -33,6 +33,19 @@ def test_conv_work_per_tile():
     assert f == 51 * 18_874_368 and b == 51 * 41_984 + weights
 
 
+def test_resblock_work_per_tile():
+    # both convs' MACs on an 8x8 tile (the recomputed ring of y1 is not
+    # counted); the 12x12x128 bf16 halo of x read once (it holds the residual);
+    # y1 and out written at the tile
+    f1, b1 = bench.resblock_work(1)
+    f2, b2 = bench.resblock_work(2)
+    assert f2 - f1 == 2 * 18_874_368
+    assert b2 - b1 == 12 * 12 * 128 * 2 + 2 * 8 * 8 * 128 * 2 == 36_864 + 32_768
+    fixed = 2 * (128 * 9 * 128 * 2) + 6 * 128 * 4       # two weight tensors, biases and GroupNorm affines
+    assert b1 - (b2 - b1) == fixed
+    assert f1 - (f2 - f1) == 0
+
+
 def test_mask_work():
     # both 256x256x128 bf16 activations read once, the list written
     assert bench.mask_work(0) == 2 * 256 * 256 * 128 * 2 + 4 == 33_554_436

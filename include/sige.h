@@ -283,6 +283,39 @@ int sige_resblock_fused(const void *x_edit, const sige_tensor_desc *xd, const vo
                         const int32_t *count, int32_t capacity, void *y1, void *out, void *workspace,
                         size_t workspace_bytes, sige_stream_t stream);
 
+/* Options of the GauGAN-style layers (sige_conv_fused_ext). */
+typedef struct {
+    int32_t transposed;       /* 1: a transposed conv (learned upsampling): input pixel (i, j) feeds
+                                 output pixel (i*stride - pad + r, j*stride - pad + c) through
+                                 weight[o][r][c][ci] */
+    int32_t output_padding;   /* transposed only: extra output rows / columns (< stride); 0 otherwise */
+    const void *spade_gamma;  /* NULL, or device NHWC map of x's shape and dtype */
+    const void *spade_beta;   /* NULL (zero), or a map like spade_gamma; needs spade_gamma */
+    int32_t act;              /* after the input transform: 0 none, 1 SiLU, 2 LeakyReLU(0.2) */
+} sige_layer_ext;
+
+/* (5b) sige_conv_fused for the other layer types of a GauGAN-style generator
+ * (mer.dev notes on SIGE, section 5: the engine serves GauGAN's generator as
+ * well as diffusion UNets): transposed convs and SPADE-style spatially
+ * modulated normalisation.  The conv input is
+ *   t = act((x * gn_scale[n][c] + gn_shift[n][c]) * (1 + gamma[n][y][x][c]) + beta[n][y][x][c])
+ * (each factor only when given), rounded to bf16; the layer is the conv of
+ * `cd` or, with ext->transposed, the transposed conv of kernel, stride and
+ * pad of `cd`, output Ho = (H - 1)*stride - 2*pad + kernel + output_padding;
+ * + bias (+ residual of y's shape), rounded once into y at every in-image
+ * pixel of the listed tiles (tiles at the OUTPUT resolution, origins in
+ * output pixels).  idx == NULL: every tile of the output grid (the dense
+ * layer: the cache of the original, or the dense baseline; count and
+ * capacity ignored).  Runs on the tensor cores: bf16 NHWC, C_in a multiple of
+ * 64; other shapes return SIGE_ERR_UNSUPPORTED.  Arguments otherwise as
+ * sige_conv_fused; the workspace is sized by sige_conv_workspace_bytes of the
+ * same cd. */
+int sige_conv_fused_ext(const void *x, const sige_tensor_desc *xd, const void *weight, const float *bias,
+                        const sige_conv_desc *cd, const sige_layer_ext *ext, const int32_t *idx,
+                        const int32_t *count, int32_t capacity, const float *gn_scale, const float *gn_shift,
+                        const void *residual, void *y, const sige_tensor_desc *yd, void *workspace,
+                        size_t workspace_bytes, sige_stream_t stream);
+
 /* The same layer on every tile of the output: the dense conv that fills the
  * cache F_l(A_original) and the dense baseline the sparse path is compared
  * with.  y is fully written. */

@@ -41,6 +41,14 @@ class ConvDesc(ctypes.Structure):
                 ("c_in", ctypes.c_int32), ("c_out", ctypes.c_int32), ("block", ctypes.c_int32)]
 
 
+class LayerExt(ctypes.Structure):
+    _fields_ = [("transposed", ctypes.c_int32), ("output_padding", ctypes.c_int32),
+                ("spade_gamma", ctypes.c_void_p), ("spade_beta", ctypes.c_void_p), ("act", ctypes.c_int32)]
+
+
+ACT_NONE, ACT_SILU, ACT_LEAKY = 0, 1, 2
+
+
 class ScaleDesc(ctypes.Structure):
     _fields_ = [("h", ctypes.c_int32), ("w", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("capacity", ctypes.c_int32)]
@@ -49,6 +57,7 @@ class ScaleDesc(ctypes.Structure):
 # Every symbol include/sige.h declares, with its ctypes signature.
 _vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
 _TD, _CD, _SD = ctypes.POINTER(TensorDesc), ctypes.POINTER(ConvDesc), ctypes.POINTER(ScaleDesc)
+_LE = ctypes.POINTER(LayerExt)
 SIGNATURES = {
     "sige_reduce_mask_workspace_bytes": (_sz, [_TD, _i32, _SD]),
     "sige_reduce_mask": (_i32, [_vp, _vp, _TD, _f32, _i32, _i32, _SD, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -59,6 +68,8 @@ SIGNATURES = {
     "sige_scatter": (_i32, [_vp, _CD, _vp, _vp, _i32, _vp, _vp, _vp, _TD, _vp]),
     "sige_conv_fused": (_i32, [_vp, _TD, _vp, _vp, _CD, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _vp, _TD,
                                _vp, _sz, _vp]),
+    "sige_conv_fused_ext": (_i32, [_vp, _TD, _vp, _vp, _CD, _LE, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _TD, _vp,
+                                   _sz, _vp]),
     "sige_dense_conv": (_i32, [_vp, _TD, _vp, _vp, _CD, _vp, _vp, _i32, _vp, _vp, _TD, _vp, _sz, _vp]),
     "sige_groupnorm_affine": (_i32, [_vp, _TD, _i32, _vp, _vp, _f32, _vp, _vp, _vp]),
     "sige_resblock_fused": (_i32, [_vp, _TD, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp,
@@ -266,6 +277,35 @@ def sige_conv_fused(x, weight, bias, cd: ConvDesc, idx, count, capacity, y, gn_s
                                _ptr(residual), _ptr(y), ctypes.byref(yd), _ptr(workspace), workspace.numel(),
                                _stream(stream))
     _check(st, "sige_conv_fused")
+    return y
+
+
+def conv_out_hw(cd: ConvDesc, H: int, W: int, transposed=False, output_padding=0):
+    if transposed:
+        return ((H - 1) * cd.stride - 2 * cd.pad + cd.kernel + output_padding,
+                (W - 1) * cd.stride - 2 * cd.pad + cd.kernel + output_padding)
+    return (H + 2 * cd.pad - cd.kernel) // cd.stride + 1, (W + 2 * cd.pad - cd.kernel) // cd.stride + 1
+
+
+def sige_conv_fused_ext(x, weight, bias, cd: ConvDesc, y=None, idx=None, count=None, capacity=0, gn_scale=None,
+                        gn_shift=None, transposed=False, output_padding=0, spade_gamma=None, spade_beta=None,
+                        act=ACT_NONE, residual=None, workspace=None, stream=None):
+    """A GauGAN-style layer (transposed conv and / or SPADE-style modulated
+    input) on the listed tiles of y, or on every tile when ``idx`` is None."""
+    N, H, W, _ = x.shape
+    Ho, Wo = conv_out_hw(cd, H, W, transposed, output_padding)
+    if y is None:
+        y = torch.empty((N, Ho, Wo, cd.c_out), dtype=x.dtype, device=x.device)
+    xd, yd = tensor_desc(x), tensor_desc(y)
+    if workspace is None:
+        workspace = zeros_workspace(sige_conv_workspace_bytes(cd, N, max(capacity, 1), Ho, Wo), x.device)
+    ext = LayerExt(int(bool(transposed)), int(output_padding), None if spade_gamma is None else spade_gamma.data_ptr(),
+                   None if spade_beta is None else spade_beta.data_ptr(), int(act))
+    st = lib().sige_conv_fused_ext(_ptr(x), ctypes.byref(xd), _ptr(weight), _ptr(bias), ctypes.byref(cd),
+                                   ctypes.byref(ext), _ptr(idx), _ptr(count), int(capacity), _ptr(gn_scale),
+                                   _ptr(gn_shift), _ptr(residual), _ptr(y), ctypes.byref(yd), _ptr(workspace),
+                                   workspace.numel(), _stream(stream))
+    _check(st, "sige_conv_fused_ext")
     return y
 
 

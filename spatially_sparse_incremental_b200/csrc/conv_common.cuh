@@ -19,6 +19,14 @@ struct ConvParams {
     // input transform (GroupNorm affine, SiLU)
     const float *gsc, *gsh;
     int32_t silu;
+    // GauGAN-style layers: a per-pixel modulation of the transformed input
+    // (t * (1 + sg) + sb, NHWC maps of the input's shape) and LeakyReLU(0.2)
+    // instead of SiLU; tstride > 0: a transposed conv of that stride, run as a
+    // stride-1 conv over the input with tstride - 1 zeros between pixels
+    // (pad = k - 1 - its padding) and the taps reversed
+    const uint8_t *sg, *sb;
+    int32_t leaky;
+    int32_t tstride;
     const uint8_t *w;  // [Cout][k][k][Cin]
     // destination: float32 output blocks (to_y == 0) or the cached output y
     float *out_blocks;

@@ -93,6 +93,9 @@ struct TcArgs {
     int32_t k, s, pad, b, bin, Ho, Wo;
     int32_t cap, dense, tiles_w, tiles_total;
     int32_t silu, from_image, to_y;
+    const uint8_t *sg, *sb;   // per-pixel modulation maps (NHWC, input shape) or null
+    int32_t leaky;            // LeakyReLU(0.2) after the transform
+    int32_t tstride;          // > 0: transposed conv of this stride (virtual zero-inserted input, taps reversed)
     // schedule / shared-memory plan
     int32_t mode;             // 0 = ROW, 1 = POS, 2 = POS with 8 slots and one MMA per output row
     int32_t taps, kci;        // k*k, C_in / 64
@@ -273,10 +276,54 @@ __device__ __forceinline__ const uint8_t *halo_src(const TcArgs &c, const int2 *
     if (!c.from_image)
         return c.src + (((int64_t)g * c.bin * c.bin + pix) * c.Cin + ch) * 2;
     const int2 o = s_orig[slot];
-    const int y = o.x * c.s - c.pad + hh, x = o.y * c.s - c.pad + ww;
+    int y = o.x * c.s - c.pad + hh, x = o.y * c.s - c.pad + ww;
+    if (c.tstride > 0) {
+        // transposed conv: pixel (y, x) of the virtual input holds x[y / t][x / t]
+        // where both are multiples of t, and zero elsewhere
+        if (y < 0 || x < 0 || y % c.tstride || x % c.tstride)
+            return nullptr;
+        y /= c.tstride;
+        x /= c.tstride;
+    }
     if (y < 0 || y >= c.H || x < 0 || x >= c.W)
         return nullptr;
     return c.src + ((((int64_t)(g % c.N) * c.H + y) * c.W + x) * c.Cin + ch) * 2;
+}
+
+// The input transform of the GauGAN-style layers, for 8 bf16 channels of one
+// pixel whose bytes sit at `off` in the input: GroupNorm-style affine of batch
+// item n (when set), the per-pixel modulation t * (1 + sg) + sb (when set),
+// then SiLU or LeakyReLU(0.2); one rounding to bf16.
+__device__ __noinline__ uint4 transform16_ext(const TcArgs &c, uint4 in, int64_t off, int n, int ch)
+{
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(&in);
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    const uint4 gv = c.sg ? __ldg(reinterpret_cast<const uint4 *>(c.sg + off)) : z;
+    const uint4 bv = c.sb ? __ldg(reinterpret_cast<const uint4 *>(c.sb + off)) : z;
+    const uint32_t *g = reinterpret_cast<const uint32_t *>(&gv);
+    const uint32_t *b = reinterpret_cast<const uint32_t *>(&bv);
+    uint4 out;
+    uint32_t *o = reinterpret_cast<uint32_t *>(&out);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float v[2] = {bf16_lo(w[q]), bf16_hi(w[q])};
+        const float gg[2] = {bf16_lo(g[q]), bf16_hi(g[q])};
+        const float bb[2] = {bf16_lo(b[q]), bf16_hi(b[q])};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int k = ch + 2 * q + e;
+            if (c.gsc)
+                v[e] = __fmaf_rn(v[e], __ldg(c.gsc + (int64_t)n * c.Cin + k), __ldg(c.gsh + (int64_t)n * c.Cin + k));
+            if (c.sg)
+                v[e] = __fmaf_rn(v[e], 1.0f + gg[e], bb[e]);
+            if (c.silu)
+                v[e] = silu_f(v[e]);
+            else if (c.leaky)
+                v[e] = v[e] >= 0.0f ? v[e] : 0.2f * v[e];
+        }
+        o[q] = pack_bf16x2(v[0], v[1]);
+    }
+    return out;
 }
 
 // Fill one B stage: 64 input channels (chunk q) of the halo of every tile of
@@ -311,8 +358,9 @@ __device__ __forceinline__ void fill_b(const TcArgs &c, int T, int tb, int q, in
         }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-    if (c.gsc == nullptr && !c.silu)
+    if (c.gsc == nullptr && !c.silu && !c.sg && !c.leaky)
         return;
+    const bool ext = c.sg != nullptr || c.leaky;
     float gsc[8], gsh[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -330,9 +378,11 @@ __device__ __forceinline__ void fill_b(const TcArgs &c, int T, int tb, int q, in
     int slot = slot0, hh = hh0, ww = ww0;
 #pragma unroll 1
     while (slot < T) {
-        if (halo_src(c, s_orig, T, tb, G, slot, hh, ww, hh * bin + ww, ch)) {
+        if (const uint8_t *src = halo_src(c, s_orig, T, tb, G, slot, hh, ww, hh * bin + ww, ch)) {
             uint4 *d = reinterpret_cast<uint4 *>(stage + b_offset(c, T, slot, hh, ww, kc));
-            if (affine && c.N > 1) {
+            if (ext) {
+                *d = transform16_ext(c, *d, src - c.src, (tb * T + slot) % c.N, ch);
+            } else if (affine && c.N > 1) {
                 const int n = (tb * T + slot) % c.N;
                 *d = transform16(*d, SIGE_BF16, c.gsc + (int64_t)n * c.Cin + ch, c.gsh + (int64_t)n * c.Cin + ch,
                                  c.silu);
@@ -372,21 +422,26 @@ __device__ __forceinline__ void fill_b_slots(const TcArgs &c, int T, int tb, int
         cp_async16(sbase + (uint32_t)lin * 16u, src ? src : c.src, src ? 16u : 0u);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-    if (c.gsc == nullptr && !c.silu)
+    if (c.gsc == nullptr && !c.silu && !c.sg && !c.leaky)
         return;
     const bool affine = c.gsc != nullptr;
+    const bool ext = c.sg != nullptr || c.leaky;
 #pragma unroll 1
     for (int lin = et; lin < total; lin += kProd) {
         const int slot = lin % T, r = lin / T;
         const int kc = r & 7, pix = r >> 3;
         const int hh = pix / bin, ww = pix - hh * bin;
         const int ch = q * 64 + kc * 8;
-        if (!halo_src(c, s_orig, T, tb, G, slot, hh, ww, pix, ch))
+        const uint8_t *src = halo_src(c, s_orig, T, tb, G, slot, hh, ww, pix, ch);
+        if (!src)
             continue;   // zero padding stays zero
         uint4 *d = reinterpret_cast<uint4 *>(stage + (size_t)lin * 16);
-        const int n = affine ? (tb * T + slot) % c.N : 0;
-        *d = transform16(*d, SIGE_BF16, affine ? c.gsc + (int64_t)n * c.Cin + ch : nullptr,
-                         affine ? c.gsh + (int64_t)n * c.Cin + ch : nullptr, c.silu);
+        const int n = (affine || ext) ? (tb * T + slot) % c.N : 0;
+        if (ext)
+            *d = transform16_ext(c, *d, src - c.src, n, ch);
+        else
+            *d = transform16(*d, SIGE_BF16, affine ? c.gsc + (int64_t)n * c.Cin + ch : nullptr,
+                             affine ? c.gsh + (int64_t)n * c.Cin + ch : nullptr, c.silu);
     }
 }
 
@@ -604,8 +659,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     ok = false;
                     break;
                 }
+                // a transposed conv reads its taps in reverse order
+                const int wtap = c.tstride > 0 ? p.taps - 1 - tap : tap;
                 tma_load_2d_w(sbase + cv.a_base + s * kAStageBytes, &tmw, a_full(s), kAStageBytes,
-                              tap * c.Cin + q * 64, y0);
+                              wtap * c.Cin + q * 64, y0);
                 ++issued;
                 if (++s == cv.SA) {
                     s = 0;
@@ -1404,7 +1461,9 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
     // box (8 channels, b_in pixels, 8 channel groups, b_in rows), zero outside.
     CUtensorMap xmap = map;
     int halo_tma = 0;
-    if (pl.mode == 0) {
+    // the TMA halo copies the image as it is: the transposed conv's virtual
+    // input and the per-pixel modulation go through the per-thread copies
+    if (pl.mode == 0 && cp.tstride == 0 && cp.sg == nullptr && !cp.leaky) {
         const cuuint64_t C = (cuuint64_t)cp.Cin;
         cuuint64_t xd[5], xs[4];
         if (cp.from_image) {
@@ -1433,6 +1492,7 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
     p.k = cp.k; p.s = cp.s; p.pad = cp.pad; p.b = cp.b; p.bin = cp.bin; p.Ho = cp.Ho; p.Wo = cp.Wo;
     p.cap = cp.cap; p.dense = cp.dense; p.tiles_w = cp.tiles_w; p.tiles_total = cp.tiles_total;
     p.silu = cp.silu; p.from_image = cp.from_image; p.to_y = cp.to_y;
+    p.sg = cp.sg; p.sb = cp.sb; p.leaky = cp.leaky; p.tstride = cp.tstride;
     plan_args(&cd, pl, p);
     p.num_sms = device_sm_count();
     uint8_t *ws = cp.ws + kWsHeader;

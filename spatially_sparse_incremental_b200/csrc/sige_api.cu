@@ -96,7 +96,12 @@ extern "C" size_t sige_conv_workspace_bytes(const sige_conv_desc *cd, int32_t ba
         return 0;
     const int64_t dense_tiles = (int64_t)((out_h + cd->block - 1) / cd->block) * ((out_w + cd->block - 1) / cd->block);
     const int64_t nt = std::max<int64_t>(capacity, dense_tiles);
-    return ws_need(cd, batch, (int)std::min<int64_t>(nt, INT32_MAX));
+    // the same layer run as a transposed conv plans as a stride-1 conv
+    sige_conv_desc v = *cd;
+    v.stride = 1;
+    v.pad = std::max(0, cd->kernel - 1 - cd->pad);
+    const int n = (int)std::min<int64_t>(nt, INT32_MAX);
+    return std::max(ws_need(cd, batch, n), ws_need(&v, batch, n));
 }
 
 extern "C" int sige_conv_path(const sige_conv_desc *cd, int32_t dtype)
@@ -207,6 +212,77 @@ extern "C" int sige_dense_conv(const void *x, const sige_tensor_desc *xd, const 
     p.tiles_total = ((p.Ho + cd->block - 1) / cd->block) * p.tiles_w;
     p.cap = p.tiles_total;
     return run_conv(p, cd, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+extern "C" int sige_conv_fused_ext(const void *x, const sige_tensor_desc *xd, const void *weight, const float *bias,
+                                   const sige_conv_desc *cd, const sige_layer_ext *ext, const int32_t *idx,
+                                   const int32_t *count, int32_t capacity, const float *gn_scale,
+                                   const float *gn_shift, const void *residual, void *y,
+                                   const sige_tensor_desc *yd, void *workspace, size_t workspace_bytes,
+                                   sige_stream_t stream)
+{
+    if (!x || !xd || !weight || !y || !yd || !cd || !ext)
+        return SIGE_ERR_INVALID_ARG;
+    if ((gn_scale == nullptr) != (gn_shift == nullptr) || (ext->spade_beta && !ext->spade_gamma))
+        return SIGE_ERR_INVALID_ARG;
+    if (idx && (!count || capacity < 0 || (reinterpret_cast<uintptr_t>(idx) & 7)))
+        return SIGE_ERR_INVALID_ARG;
+    if (ext->act < 0 || ext->act > 2 || ext->transposed < 0 || ext->transposed > 1 || ext->output_padding < 0)
+        return SIGE_ERR_INVALID_ARG;
+    int st = check_layer(cd, xd->dtype);
+    if (st != SIGE_OK)
+        return st;
+    if (xd->n < 1 || xd->h < 1 || xd->w < 1 || xd->c != cd->c_in)
+        return SIGE_ERR_INVALID_ARG;
+    // a transposed conv runs as a stride-1 conv over the input with stride - 1
+    // zeros between pixels, padded by k - 1 - pad, with the taps reversed
+    sige_conv_desc vcd = *cd;
+    int Ho, Wo;
+    if (ext->transposed) {
+        if (ext->output_padding >= cd->stride)
+            return SIGE_ERR_INVALID_ARG;
+        vcd.stride = 1;
+        vcd.pad = cd->kernel - 1 - cd->pad;
+        Ho = (xd->h - 1) * cd->stride - 2 * cd->pad + cd->kernel + ext->output_padding;
+        Wo = (xd->w - 1) * cd->stride - 2 * cd->pad + cd->kernel + ext->output_padding;
+    } else {
+        if (ext->output_padding != 0)
+            return SIGE_ERR_INVALID_ARG;
+        Ho = (xd->h + 2 * cd->pad - cd->kernel) / cd->stride + 1;
+        Wo = (xd->w + 2 * cd->pad - cd->kernel) / cd->stride + 1;
+    }
+    if (Ho < 1 || Wo < 1 || yd->n != xd->n || yd->h != Ho || yd->w != Wo || yd->c != cd->c_out)
+        return SIGE_ERR_INVALID_ARG;
+    if (xd->dtype != SIGE_BF16 || xd->layout != SIGE_NHWC || yd->layout != SIGE_NHWC || yd->dtype != xd->dtype ||
+        !tc_supported(&vcd, SIGE_BF16))
+        return SIGE_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(weight) || !aligned16(y) || !aligned16(residual) || !aligned16(bias) ||
+        !aligned16(gn_scale) || !aligned16(gn_shift) || !aligned16(ext->spade_gamma) || !aligned16(ext->spade_beta))
+        return SIGE_ERR_UNSUPPORTED;
+    ConvParams p{};
+    p.src = static_cast<const uint8_t *>(x);
+    p.N = xd->n; p.H = xd->h; p.W = xd->w; p.dtype = xd->dtype;
+    p.gsc = gn_scale; p.gsh = gn_shift;
+    p.silu = ext->act == 1;
+    p.leaky = ext->act == 2;
+    p.sg = static_cast<const uint8_t *>(ext->spade_gamma);
+    p.sb = static_cast<const uint8_t *>(ext->spade_beta);
+    p.tstride = ext->transposed ? cd->stride : 0;
+    p.w = static_cast<const uint8_t *>(weight);
+    p.bias = bias;
+    p.residual = static_cast<const uint8_t *>(residual);
+    p.y = static_cast<uint8_t *>(y);
+    p.Ho = Ho; p.Wo = Wo;
+    p.from_image = 1; p.to_y = 1;
+    if (idx) {
+        p.idx = idx; p.count = count; p.cap = capacity; p.dense = 0;
+    } else {
+        p.dense = 1;
+        p.tiles_w = (Wo + cd->block - 1) / cd->block;
+        p.tiles_total = ((Ho + cd->block - 1) / cd->block) * p.tiles_w;
+        p.cap = p.tiles_total;
+    }
+    return run_conv(p, &vcd, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 extern "C" int sige_get_error(void *workspace, sige_stream_t stream)

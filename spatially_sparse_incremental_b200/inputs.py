@@ -305,3 +305,59 @@ def make_cfg5_layer(seed: int, layer: int, area: float = 0.012, all_edit: bool =
         edit = pool_any(m, 256 // H)
     return make_conv_case(seed + 1000 * (layer + 1), H, W, ci, co, kernel=k, stride=s,
                           pad=k // 2, block=b, edit=edit)
+
+
+# ---------------------------------------------------------------------------
+# GauGAN-style layers beside the plain convs
+# ---------------------------------------------------------------------------
+
+# decoder upsampling layers: (input H, W, C_in, C_out, output tile edge); a
+# 3x3 transposed conv, stride 2, padding 1, output padding 1 doubles H and W
+UPSAMPLE_LAYERS = (
+    (32, 64, 512, 256, 4),
+    (64, 128, 256, 128, 4),
+)
+# SPADE-modulated 3x3 convs: (H, W, C_in, C_out, tile edge)
+SPADE_LAYERS = (
+    (64, 128, 256, 256, 4),
+    (128, 256, 128, 128, 8),
+)
+
+
+def make_upsample_layer(seed: int, layer: int, area: float = 0.012, all_edit: bool = False) -> ConvLayer:
+    """Input at (H, W), output at (2H, 2W).  The edit is drawn at 256x512,
+    placed on the output grid (``meta['edit_out']``) and on the input grid
+    with ``pool_any``; x_edit differs from x_orig inside the input's edit."""
+    H, W, ci, co, b = UPSAMPLE_LAYERS[layer]
+    rng = np.random.default_rng(seed)
+    if all_edit:
+        out_edit = np.ones((2 * H, 2 * W), dtype=bool)
+    else:
+        m = rect_mask(rng, 256, 512, area / 2) | blob_mask(rng, 256, 512, area / 2, 1, 3, ellipse=True)
+        out_edit = pool_any(m, 256 // (2 * H))
+    in_edit = pool_any(out_edit, 2)
+    L = make_conv_case(seed + 7000 * (layer + 1), H, W, ci, co, kernel=3, stride=2, pad=1, block=b, edit=in_edit)
+    L.meta = {"output_padding": 1, "edit_out": out_edit}
+    return L
+
+
+def make_spade_layer(seed: int, layer: int, area: float = 0.012) -> ConvLayer:
+    """A 3x3 conv whose input is modulated per pixel: ``meta`` holds the
+    modulation maps gamma / beta of the original and of the edited image
+    (N(0, 0.3^2), bf16, fresh values inside the edit, as an edited
+    segmentation map changes them there)."""
+    H, W, ci, co, b = SPADE_LAYERS[layer]
+    rng = np.random.default_rng(seed + 9000 * (layer + 1))
+    m = rect_mask(rng, 256, 512, area / 2) | blob_mask(rng, 256, 512, area / 2, 1, 3, ellipse=True)
+    edit = pool_any(m, 256 // H)
+    L = make_conv_case(seed + 8000 * (layer + 1), H, W, ci, co, kernel=3, stride=1, pad=1, block=b, edit=edit)
+    maps = {}
+    for name in ("gamma", "beta"):
+        orig = rng.normal(0.0, 0.3, size=(1, H, W, ci)).astype(np.float32)
+        ed = orig.copy()
+        ys, xs = np.nonzero(edit)
+        ed[:, ys, xs, :] = rng.normal(0.0, 0.3, size=(1, len(ys), ci)).astype(np.float32)
+        maps[name + "_orig"] = _to(orig, torch.bfloat16)
+        maps[name + "_edit"] = _to(ed, torch.bfloat16)
+    L.meta = maps
+    return L

@@ -259,3 +259,60 @@ def test_attention_core_validation(L):
     big = sige.TensorDesc(1 << 16, 16, 16, 320, sige.BF16, sige.NHWC)
     assert call(desc=ctypes.byref(big), keys=1 << 16) == sige.ERR_INVALID_ARG   # keys x batch past 32 bits
     assert call(cap=0) == sige.OK                          # no tiles: no launch
+
+
+def test_resblock_fused_validation(L):
+    xd = sige.TensorDesc(1, 64, 64, 128, sige.BF16, sige.NHWC)
+    fake = ctypes.c_void_p(0x1000)
+    ws = ctypes.c_void_p(0x2000)
+
+    def call(**kw):
+        a = dict(x=fake, xd=ctypes.byref(xd), w1=fake, b1=None, g1s=fake, g1h=fake, w2=fake, b2=None, g2s=fake,
+                 g2h=fake, block=8, idx=fake, cnt=fake, cap=64, y1=ctypes.c_void_p(0x10000000),
+                 out=ctypes.c_void_p(0x20000000), ws=ws, wsb=256, st=None)
+        a.update(kw)
+        return L.sige_resblock_fused(*a.values())
+    assert call(x=None) == sige.ERR_INVALID_ARG
+    assert call(g2h=None) == sige.ERR_INVALID_ARG
+    assert call(cap=-1) == sige.ERR_INVALID_ARG
+    assert call(idx=ctypes.c_void_p(0x1004)) == sige.ERR_INVALID_ARG      # pairs need 8-byte alignment
+    assert call(y1=fake) == sige.ERR_INVALID_ARG                          # y1 overlaps x
+    assert call(block=4) == sige.ERR_UNSUPPORTED
+    xd64 = sige.TensorDesc(1, 64, 64, 64, sige.BF16, sige.NHWC)
+    assert call(xd=ctypes.byref(xd64)) == sige.ERR_UNSUPPORTED
+    xdf = sige.TensorDesc(1, 64, 64, 128, sige.F32, sige.NHWC)
+    assert call(xd=ctypes.byref(xdf)) == sige.ERR_UNSUPPORTED
+    assert call(x=ctypes.c_void_p(0x1008)) == sige.ERR_UNSUPPORTED       # tensors need 16-byte alignment
+    assert call(ws=None) == sige.ERR_WORKSPACE
+    assert call(wsb=255) == sige.ERR_WORKSPACE
+    n0 = sige.sige_launch_count()
+    assert call(cap=0) == sige.OK                                        # nothing to do, no launch
+    assert sige.sige_launch_count() == n0
+
+
+def test_conv_fused_ext_validation(L):
+    xd = sige.TensorDesc(1, 32, 64, 256, sige.BF16, sige.NHWC)
+    cd = sige.ConvDesc(3, 2, 1, 256, 128, 4)
+    yd = sige.TensorDesc(1, 64, 128, 128, sige.BF16, sige.NHWC)        # (32 - 1) * 2 - 2 + 3 + 1 = 64
+    fake = ctypes.c_void_p(0x1000)
+    ws = ctypes.c_void_p(0x2000)
+    wsb = L.sige_conv_workspace_bytes(ctypes.byref(cd), 1, 512, 64, 128)
+
+    def call(transposed=1, op=1, act=0, g=None, b=None, **kw):
+        ext = sige.LayerExt(transposed, op, g, b, act)
+        a = dict(x=fake, xd=ctypes.byref(xd), w=fake, bias=None, cd=ctypes.byref(cd), ext=ctypes.byref(ext),
+                 idx=fake, cnt=fake, cap=512, gs=None, gh=None, res=None, y=fake, yd=ctypes.byref(yd), ws=ws,
+                 wsb=wsb, st=None)
+        a.update(kw)
+        return L.sige_conv_fused_ext(*a.values())
+    assert call(op=2) == sige.ERR_INVALID_ARG            # output padding >= stride
+    assert call(act=3) == sige.ERR_INVALID_ARG
+    assert call(b=0x3000) == sige.ERR_INVALID_ARG       # beta without gamma
+    assert call(ext=None) == sige.ERR_INVALID_ARG
+    assert call(gs=fake) == sige.ERR_INVALID_ARG        # scale without shift
+    assert call(idx=ctypes.c_void_p(0x1004)) == sige.ERR_INVALID_ARG
+    assert call(op=0) == sige.ERR_INVALID_ARG           # then the output would be 63 x 127
+    yd_plain = sige.TensorDesc(1, 16, 32, 128, sige.BF16, sige.NHWC)
+    assert call(transposed=0, op=0, yd=ctypes.byref(yd_plain)) != sige.ERR_INVALID_ARG
+    assert call(g=0x3008) == sige.ERR_UNSUPPORTED       # misaligned modulation map
+    assert call(wsb=16) == sige.ERR_WORKSPACE

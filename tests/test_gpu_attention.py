@@ -89,7 +89,7 @@ def test_attention_core_self(N, H, W, D, Dv, heads, b):
     assert _core_case(100 + H + D + heads + b, N, H, W, D, Dv, heads, b) > 0
 
 
-@pytest.mark.parametrize("Lk,heads", [(77, 8), (33, 1), (1, 2), (300, 4)])
+@pytest.mark.parametrize("Lk,heads", [(77, 8), (33, 2), (1, 2), (300, 4)])
 def test_attention_core_cross(Lk, heads):
     """Keys and values from a context sequence of Lk tokens (not a multiple of
     the 32-key chunk; a single key: weight 1)."""

@@ -3,14 +3,16 @@
 
 Workload (one step = one pass of the whole hot path over one edit): the
 DDPM-style residual block at 256x256, C=128, bf16 storage / fp32 accumulation,
-with a ~1.2% edit made of 1-3 seeded discs:
+with a ~1.2% edit made of 1-3 seeded discs, in ONE launch
+(sige_resblock_step):
     mask     : difference mask of x_orig vs x_edit -> 8x8 tile list (dilate 1)
-    resblock : one launch for both layers on the tiles: gather(GN1 + SiLU) ->
-               3x3 conv1 (+bias) -> y1 (into the cached y1, and on chip with a
-               one-pixel ring) -> GN2 + SiLU -> 3x3 conv2 (+bias +x_edit) ->
-               scatter into the cached out
-The same step with the two layers as separate fused-layer launches
-(conv1, conv2) is timed beside it (`unfused_step_us`).
+    resblock : both layers on the tiles: gather(GN1 + SiLU) -> 3x3 conv1
+               (+bias) -> y1 (into the cached y1, and on chip with a one-pixel
+               ring) -> GN2 + SiLU -> 3x3 conv2 (+bias +x_edit) -> scatter
+               into the cached out
+Timed beside it: the same step as two launches (sige_reduce_mask, then
+sige_resblock_fused: `two_launch_step_us`) and as three (the mask, then each
+layer as its own fused-layer launch: `unfused_step_us`).
 The caches (y1 and out of the original image, GroupNorm statistics of the
 original) are computed once beforehand by the same library's dense conv, as
 the engine pre-computes the original activations.
@@ -249,13 +251,25 @@ def make_workload(seed, dev, area=0.012):
                                                                          [(H, W, BLOCK, cap)]), dev)
     conv_ws = sige.zeros_workspace(sige.sige_conv_workspace_bytes(cd, 1, cap, H, W), dev)
     rb_ws = sige.zeros_workspace(sige.sige_workspace_bytes(sige.CALL_RESBLOCK, None, cap), dev)
+    step_ws = sige.zeros_workspace(sige.sige_resblock_step_workspace_bytes(d["x_orig"], BLOCK), dev)
     d.update(cd=cd, cap=cap, gs1=gs1, gh1=gh1, gs2=gs2, gh2=gh2, y1=y1, out=out, idx=idx, cnt=cnt,
-             mask_ws=mask_ws, conv_ws=conv_ws, rb_ws=rb_ws, blk=blk)
+             mask_ws=mask_ws, conv_ws=conv_ws, rb_ws=rb_ws, step_ws=step_ws, blk=blk)
     return d
 
 
 def step_calls(d, stream=None):
-    """The two hot-path calls of one step, as closures (for graph capture)."""
+    """The step as one call (for graph capture)."""
+    import spatially_sparse_incremental_b200 as sige
+
+    def step():
+        sige.sige_resblock_step(d["x_orig"], d["x_edit"], THRESH, d["w1"], d["b1"], (d["gs1"], d["gh1"]), d["w2"],
+                                d["b2"], (d["gs2"], d["gh2"]), d["y1"], d["out"], d["cap"], idx=d["idx"],
+                                count=d["cnt"], workspace=d["step_ws"], stream=stream)
+    return {"step": step}
+
+
+def two_launch_calls(d, stream=None):
+    """The step as the mask call and the fused res-block call."""
     import spatially_sparse_incremental_b200 as sige
 
     def mask():
@@ -394,7 +408,7 @@ def measure_extras(dev, flush, stream, peaks, seed, step_graph):
         torch.cuda.synchronize()   # the workload is built on the default stream
         calls = step_calls(d, stream)
         with torch.cuda.stream(stream):
-            calls["mask"]()
+            calls["step"]()
         stream.synchronize()
         tiles = int(d["cnt"].item())
 
@@ -419,7 +433,7 @@ def measure_extras(dev, flush, stream, peaks, seed, step_graph):
     # chained 3x3 convs) instead of one tile
     d = make_workload(seed, dev)
     torch.cuda.synchronize()
-    calls = step_calls(d, stream)
+    calls = two_launch_calls(d, stream)
 
     def mask_px():
         sige.sige_reduce_mask_px(d["x_orig"], d["x_edit"], THRESH, [(H, W, BLOCK, d["cap"])], 2, idx=d["idx"],
@@ -597,6 +611,17 @@ def resblock_work(n_tiles):
     return 2 * macs, halo + writes + weights
 
 
+def step_work(n_tiles):
+    """Algorithmic FLOPs and bytes of the one-launch step: both inputs read
+    once by the mask (the halo of x_edit is read again from L2, not counted),
+    the list written, y1 and out written at the tiles, both weight tensors and
+    the per-channel vectors once; the two convs' MACs on the tiles."""
+    flops, _ = resblock_work(n_tiles)
+    writes = 2 * n_tiles * BLOCK * BLOCK * C * 2
+    weights = 2 * (C * 9 * C * 2) + 6 * C * 4
+    return flops, mask_work(n_tiles) + writes + weights
+
+
 def mask_work(n_tiles):
     return 2 * H * W * C * 2 + n_tiles * 8 + 4
 
@@ -759,7 +784,13 @@ def run_sige(args):
         for fn in calls.values():
             fn()
     step_graph = {"step": capture(whole_step, stream)}
-    graphs = {nm: capture(fn, stream) for nm, fn in calls.items()}
+    tcalls = two_launch_calls(d, stream)
+
+    def whole_two():
+        for fn in tcalls.values():
+            fn()
+    tgraph = {"two": capture(whole_two, stream)}
+    graphs = {nm: capture(fn, stream) for nm, fn in tcalls.items()}
     ucalls = unfused_calls(d, stream)
 
     def whole_unfused():
@@ -786,21 +817,24 @@ def run_sige(args):
     barrier()
     clocks = sampler.stop()
     step_ms = float(np.mean(tot))
-    # per-call breakdown: each call in a graph of its own (so each number also
-    # carries one graph launch), same L2 flush before every step
-    timed_graph_steps(graphs, flush, args.warmup, stream)
-    per, _ = timed_graph_steps(graphs, flush, args.steps, stream)
-    kern_ms = {nm: float(np.mean(v)) for nm, v in per.items()}
-    # the same step with the layers as two separate launches
+    # the step as two launches, and each of them in a graph of its own (so
+    # each number also carries one graph launch), same L2 flush before every step
     nu = max(10, min(args.steps, 200))
+    timed_graph_steps(tgraph, flush, 3, stream)
+    _, ttot = timed_graph_steps(tgraph, flush, nu, stream)
+    two_ms = float(np.mean(ttot))
+    timed_graph_steps(graphs, flush, 3, stream)
+    per, _ = timed_graph_steps(graphs, flush, nu, stream)
+    kern_ms = {nm: float(np.mean(v)) for nm, v in per.items()}
+    # the same step with the layers as separate launches
     timed_graph_steps(ugraph, flush, 3, stream)
     _, utot = timed_graph_steps(ugraph, flush, nu, stream)
     uper, _ = timed_graph_steps(ugraphs, flush, nu, stream)
     unfused_ms = float(np.mean(utot))
     ukern_ms = {nm: float(np.mean(v)) for nm, v in uper.items()}
-    red = max_over_ranks([step_ms, unfused_ms] + [kern_ms[k] for k in kern_ms], dev)
-    step_ms, unfused_ms = red[0], red[1]
-    kern_ms = {k: red[i + 2] for i, k in enumerate(kern_ms)}
+    red = max_over_ranks([step_ms, unfused_ms, two_ms] + [kern_ms[k] for k in kern_ms], dev)
+    step_ms, unfused_ms, two_ms = red[0], red[1], red[2]
+    kern_ms = {k: red[i + 3] for i, k in enumerate(kern_ms)}
 
     # dense comparison (same launch mode, L2 flushed)
     dper, dtot = timed_graph_steps(dgraphs, flush, max(10, min(args.steps, 50)), stream)
@@ -829,34 +863,29 @@ def run_sige(args):
     e2e_ms = float(np.mean(e2e_times))
     e2e_ms = max_over_ranks([e2e_ms], dev)[0]
 
-    # roofline of the dominant kernel
-    dom = max(kern_ms, key=kern_ms.get)
-    kernel_name = {"mask": "k_mask_reduce", "resblock": "k_resblock"}[dom]
-    if dom == "mask":
-        nbytes = mask_work(n_tiles)
-        ach = nbytes / (kern_ms[dom] * 1e-3) / 1e9
+    # roofline of the step's one kernel: the two inputs streamed once, the
+    # list, y1 and out written at the tiles, the weights read once; the convs'
+    # MACs on the tiles.  It is bound by the bytes.
+    flops, nbytes = step_work(n_tiles)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    t_bw = nbytes / (peaks["hbm_gbs"] * 1e9)
+    if t_bw >= t_tc:
+        ach = nbytes / (step_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / peaks["hbm_gbs"], "traffic": ncu_traffic("k_mask_reduce"),
-                "kernel": kernel_name, "algorithmic_bytes": nbytes,
-                "peak_source": f"{peaks['source']} hbm_gbs"}
+                "frac": ach / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} hbm_gbs"}
     else:
-        flops, nbytes = resblock_work(n_tiles)
-        t_tc = flops / (peaks["bf16_tflops"] * 1e12)
-        t_bw = nbytes / (peaks["hbm_gbs"] * 1e9)
-        if t_tc >= t_bw:
-            ach = flops / (kern_ms[dom] * 1e-3) / 1e12
-            roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": ach / peaks["bf16_tflops"], "peak_source": f"{peaks['source']} bf16_tflops (burst)"}
-        else:
-            ach = nbytes / (kern_ms[dom] * 1e-3) / 1e9
-            roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": ach / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} hbm_gbs"}
-        roof.update(traffic=ncu_traffic("k_resblock"), kernel=kernel_name, algorithmic_bytes=nbytes,
-                    algorithmic_flops=flops)
-    # step roofline: every call at its own bound
+        ach = flops / (step_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"], "peak_source": f"{peaks['source']} bf16_tflops (burst)"}
+    roof.update(traffic=ncu_traffic("k_resblock_step"), kernel="k_resblock<step>", algorithmic_bytes=nbytes,
+                algorithmic_flops=flops, duration_us=step_ms * 1e3,
+                tensor_frac=(flops / (step_ms * 1e-3) / 1e12) / peaks["bf16_tflops"])
+    # the fused res block of the two-launch step against its own roofline
     f_rb, b_rb = resblock_work(n_tiles)
-    t_roof = mask_work(n_tiles) / (peaks["hbm_gbs"] * 1e9) + max(f_rb / (peaks["bf16_tflops"] * 1e12),
-                                                                 b_rb / (peaks["hbm_gbs"] * 1e9))
+    t_rb = max(f_rb / (peaks["bf16_tflops"] * 1e12), b_rb / (peaks["hbm_gbs"] * 1e9))
+    resblock_roof = {"kernel": "k_resblock", "roof_us": t_rb * 1e6, "us": kern_ms["resblock"] * 1e3,
+                     "frac": t_rb / (kern_ms["resblock"] * 1e-3)}
+    t_roof = max(t_tc, t_bw)
     sparse_conv_ms = kern_ms["resblock"]
     dense_conv_ms = dense_ms["dense1"] + dense_ms["dense2"]
 
@@ -894,10 +923,12 @@ def run_sige(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "H": H, "W": W, "C": C, "block": BLOCK, "edit_area": 0.012,
                    "active_tiles": n_tiles, "tile_fraction": n_tiles / d["cap"],
-                   "l2": "cold: 256 MiB write then 256 MiB read (clean lines) before every step, untimed", "launch": "one CUDA graph per step (mask + fused res block); breakdown_us from one graph per call",
+                   "l2": "cold: 256 MiB write then 256 MiB read (clean lines) before every step, untimed", "launch": "one CUDA graph per step holding the one-launch step kernel; breakdown_us: the two-launch form, one graph per call",
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
         "step_p50_us": float(np.median(tot)) * 1e3, "step_p90_us": float(np.percentile(tot, 90)) * 1e3,
+        "two_launch_step_us": two_ms * 1e3,
         "breakdown_us": {k: v * 1e3 for k, v in kern_ms.items()},
+        "resblock_roofline": resblock_roof,
         "unfused_step_us": unfused_ms * 1e3,
         "unfused_breakdown_us": {k: v * 1e3 for k, v in ukern_ms.items()},
         "dense_conv_us": dense_conv_ms * 1e3, "sparse_conv_us": sparse_conv_ms * 1e3,
@@ -907,7 +938,7 @@ def run_sige(args):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_ms * 1e3, "unit": "us", "h2d_bytes_per_step": host_in.numel() * host_in.element_size(),
                 "d2h_bytes_per_step": host_out.numel() * host_out.element_size(),
-                "api": "sige_reduce_mask + sige_resblock_fused, eager, pinned host buffers"},
+                "api": "sige_resblock_step, eager, pinned host buffers"},
         "gpu_launches": sum(launches.values()) * args.steps,
         "clocks": clocks,
         "conv_path": "tcgen05" if sige.sige_conv_path(d["cd"], torch.bfloat16) == 1 else "cuda-core",
@@ -916,7 +947,7 @@ def run_sige(args):
         line.update(extras)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    for gd in (graphs, dgraphs, step_graph, ugraph, ugraphs):
+    for gd in (graphs, dgraphs, step_graph, ugraph, ugraphs, tgraph):
         gd.clear()
     if ws > 1:
         torch.distributed.barrier()

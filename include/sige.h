@@ -316,6 +316,39 @@ int sige_conv_fused_ext(const void *x, const sige_tensor_desc *xd, const void *w
                         const void *residual, void *y, const sige_tensor_desc *yd, void *workspace,
                         size_t workspace_bytes, sige_stream_t stream);
 
+/* (6b) The whole step of an edit for one residual block, in ONE launch: the
+ * difference mask of x_orig vs x_edit, its 8 x 8 tiles dilated by `dilate`
+ * tiles and compacted in row-major order (as sige_reduce_mask with one
+ * scale at full resolution), then sige_resblock_fused on that list (mer.dev
+ * notes on SIGE, sections 3 and 3.2; SIGE project page, "Overview").  Every
+ * CTA of the launch streams its share of the two inputs and marks tile
+ * flags; after a grid-wide barrier each CTA derives the list itself, so no
+ * second launch and no host round trip separate the mask from the convs.
+ *   x_orig, x_edit : device NHWC bf16 [N][H][W][128] (xd); the mask is
+ *                    OR-ed over the batch
+ *   threshold      : a pixel is edited when some channel differs by more
+ *                    (strict >), the difference taken in float32
+ *   idx, count     : OUTPUTS: the list (int32 pairs, capacity entries) and
+ *                    its length (which may exceed capacity: then only
+ *                    capacity tiles are listed and processed, and the device
+ *                    error SIGE_ERR_CAPACITY is recorded)
+ *   workspace      : device, >= sige_resblock_step_workspace_bytes(xd, block),
+ *                    zero-filled before its first use; each call leaves it
+ *                    zero-filled apart from a recorded device error.  One
+ *                    workspace per stream: calls sharing one must not overlap.
+ * Other arguments as sige_resblock_fused.  The launch keeps every CTA
+ * resident at once (one pair of CTAs per two SMs); if other work holds SMs so
+ * that some CTAs cannot start, the grid barrier's bounded wait (about 1 s)
+ * expires and records SIGE_ERR_TIMEOUT instead of hanging.  At most 64 units
+ * (tiles x batch) per CTA pair: larger capacities return
+ * SIGE_ERR_UNSUPPORTED, as do tile grids beyond 16384 tiles. */
+size_t sige_resblock_step_workspace_bytes(const sige_tensor_desc *xd, int32_t block);
+int sige_resblock_step(const void *x_orig, const void *x_edit, const sige_tensor_desc *xd, float threshold,
+                       int32_t dilate, const void *w1, const float *b1, const float *gn1_scale,
+                       const float *gn1_shift, const void *w2, const float *b2, const float *gn2_scale,
+                       const float *gn2_shift, int32_t block, int32_t *idx, int32_t *count, int32_t capacity,
+                       void *y1, void *out, void *workspace, size_t workspace_bytes, sige_stream_t stream);
+
 /* The same layer on every tile of the output: the dense conv that fills the
  * cache F_l(A_original) and the dense baseline the sparse path is compared
  * with.  y is fully written. */

@@ -68,6 +68,9 @@ SIGNATURES = {
     "sige_scatter": (_i32, [_vp, _CD, _vp, _vp, _i32, _vp, _vp, _vp, _TD, _vp]),
     "sige_conv_fused": (_i32, [_vp, _TD, _vp, _vp, _CD, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _vp, _TD,
                                _vp, _sz, _vp]),
+    "sige_resblock_step_workspace_bytes": (_sz, [_TD, _i32]),
+    "sige_resblock_step": (_i32, [_vp, _vp, _TD, _f32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
+                                  _i32, _vp, _vp, _vp, _sz, _vp]),
     "sige_conv_fused_ext": (_i32, [_vp, _TD, _vp, _vp, _CD, _LE, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _TD, _vp,
                                    _sz, _vp]),
     "sige_dense_conv": (_i32, [_vp, _TD, _vp, _vp, _CD, _vp, _vp, _i32, _vp, _vp, _TD, _vp, _sz, _vp]),
@@ -340,6 +343,31 @@ def sige_resblock_fused(x_edit, w1, b1, gn1, w2, b2, gn2, idx, count, capacity, 
                                    workspace.numel(), _stream(stream))
     _check(st, "sige_resblock_fused")
     return y1, out
+
+
+def sige_resblock_step_workspace_bytes(x, block=8) -> int:
+    xd = tensor_desc(x)
+    return int(lib().sige_resblock_step_workspace_bytes(ctypes.byref(xd), int(block)))
+
+
+def sige_resblock_step(x_orig, x_edit, threshold, w1, b1, gn1, w2, b2, gn2, y1, out, capacity, dilate=1, block=8,
+                       idx=None, count=None, workspace=None, stream=None):
+    """Mask, tile list and the fused res block in one launch.  Returns (idx,
+    count) on the device; y1 and out are updated in place."""
+    xd = tensor_desc(x_edit)
+    dev = x_edit.device
+    if idx is None:
+        idx = torch.empty((max(int(capacity), 1), 2), dtype=torch.int32, device=dev)
+    if count is None:
+        count = torch.empty(1, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = zeros_workspace(sige_resblock_step_workspace_bytes(x_edit, block), dev)
+    st = lib().sige_resblock_step(_ptr(x_orig), _ptr(x_edit), ctypes.byref(xd), float(threshold), int(dilate),
+                                  _ptr(w1), _ptr(b1), _ptr(gn1[0]), _ptr(gn1[1]), _ptr(w2), _ptr(b2), _ptr(gn2[0]),
+                                  _ptr(gn2[1]), int(block), _ptr(idx), _ptr(count), int(capacity), _ptr(y1),
+                                  _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "sige_resblock_step")
+    return idx, count
 
 
 def sige_groupnorm_affine(x, groups, gamma, beta, eps=1e-5, scale=None, shift=None, stream=None):

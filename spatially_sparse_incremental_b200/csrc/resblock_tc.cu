@@ -78,11 +78,13 @@ static_assert(kOffX % 128 == 0 && kXHalf % 128 == 0 && kOffY % 16 == 0, "TMA des
 constexpr uint32_t kBarWFull = 0, kBarWEmpty = 160, kBarXFull = 320, kBarXReady = 336;
 constexpr uint32_t kBarAcc1Full = 352, kBarAcc1Empty = 360, kBarAcc2Full = 368, kBarAcc2Empty = 376;
 constexpr uint32_t kBarY1tFull = 384, kBarY1tEmpty = 392, kBarDrain = 400;
-constexpr uint32_t kTmemSlot = 512, kAbort = 516;
+constexpr uint32_t kTmemSlot = 416, kAbort = 420, kUnits = 448;   // kUnits: the step's unit table (int2)
+constexpr int kMaxUnits = 64;              // units one CTA pair takes in the step (tile origins at kUnits)
+constexpr int kMaxTiles = 16384;           // tile grid of the step's mask (flags staged in the halo buffer)
 
 // wait sites recorded in the error detail on a timeout
 enum : int { kSiteWEmpty = 101, kSiteWFull, kSiteXReady, kSiteAcc1Empty, kSiteAcc2Empty, kSiteY1tFull,
-             kSiteXFull, kSiteAcc1Full, kSiteY1tEmpty, kSiteAcc2Full };
+             kSiteXFull, kSiteAcc1Full, kSiteY1tEmpty, kSiteAcc2Full, kSiteGrid };
 
 }  // namespace rb
 
@@ -97,6 +99,14 @@ struct RbArgs {
     uint8_t *out;               // cached out, updated at the tiles
     WsHeader *hdr;
     int32_t N, H, W, cap;
+    // the one-launch step: the tile list is made here from x_orig vs x (the
+    // list and its count are then outputs: idx / count)
+    const uint8_t *xo;          // x_orig, NHWC bf16 like x
+    float thr;                  // difference threshold (strict >)
+    int32_t dilate;             // tile dilation
+    int32_t th, tw;             // tile grid
+    uint8_t *flags;             // [th * tw] tile flags in the workspace, zero on entry and exit
+    uint32_t *ctr;              // [2] grid-barrier arrivals and departures in the workspace header
 };
 
 // Four K=16 MMAs of one 64-channel weight stage: A (pixels, no swizzle)
@@ -163,6 +173,189 @@ __device__ __forceinline__ void st_peer_v4(uint32_t addr, uint4 v)
 __device__ __forceinline__ void cluster_arrive_rel() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait_acq() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
 
+
+// ------------------------------------------------------------------ step mode
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *ptr)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+// Some bf16 of 16 bytes differ by more than thr (the difference taken in float32).
+__device__ __forceinline__ bool rb_exceeds(uint4 a, uint4 b, float thr)
+{
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+    bool r = false;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        r |= fabsf(bf16_lo(bw[q]) - bf16_lo(aw[q])) > thr || fabsf(bf16_hi(bw[q]) - bf16_hi(aw[q])) > thr;
+    return r;
+}
+
+// Phases of the one-launch step before the res block, run by every thread of
+// every CTA (mer.dev notes on SIGE, sections 3 and 3.2: difference mask,
+// dilation, tile selection; SIGE project page, "Overview": active block
+// indices):
+//   A. this CTA's contiguous share of x_orig and x_edit, 16-byte loads, eight
+//      in flight per input and thread; a pixel some channel of which differs
+//      by more than thr marks its 8x8 tile in the workspace flags;
+//   B. grid barrier (bounded): every CTA arrives once, all wait for all;
+//   C. the flags (dilated by `dilate` tiles, clipped) compacted in row-major
+//      order -- every CTA computes the same list; CTA 0 writes it and its
+//      count out, each pair keeps the origins of its own units (units
+//      u = pair + j * npairs, tile u / N); the last CTA to finish reading the
+//      flags zeroes them and the two counters for the next call.
+// Returns the number of units, min(count, cap) * N.
+__device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, volatile int *abort_flag, int pair,
+                                            int npairs)
+{
+    using namespace rb;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int H = p.H, W = p.W, tw = p.tw, nt = p.th * p.tw;
+    // ---- A: difference mask -> tile flags
+    bool wrote = false;
+    {
+        const int64_t nvec = (int64_t)p.N * H * W * (kC / 8);
+        const int64_t per = (nvec + gridDim.x - 1) / gridDim.x;
+        const int64_t v0 = (int64_t)blockIdx.x * per, v1 = min(nvec, v0 + per);
+        int last = -1;
+#pragma unroll 1
+        for (int64_t base = v0 + tid; base < v1; base += 8 * kThreads) {
+            uint4 a[8], b[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int64_t v = base + (int64_t)k * kThreads;
+                a[k] = b[k] = make_uint4(0, 0, 0, 0);
+                if (v < v1) {
+                    a[k] = __ldg(reinterpret_cast<const uint4 *>(p.xo) + v);
+                    b[k] = __ldg(reinterpret_cast<const uint4 *>(p.x) + v);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                if (((a[k].x ^ b[k].x) | (a[k].y ^ b[k].y) | (a[k].z ^ b[k].z) | (a[k].w ^ b[k].w)) &&
+                    rb_exceeds(a[k], b[k], p.thr)) {
+                    const int64_t pix = (base + (int64_t)k * kThreads) >> 4;   // 16 vectors per pixel
+                    const int64_t hw = pix % ((int64_t)H * W);
+                    const int y = (int)(hw / W), x = (int)(hw - (int64_t)y * W);
+                    const int t = (y >> 3) * tw + (x >> 3);
+                    if (t != last) {
+                        p.flags[t] = 1;
+                        last = t;
+                        wrote = true;
+                    }
+                }
+            }
+        }
+    }
+    // ---- B: grid barrier; the fence (cumulative, after the CTA barrier)
+    // publishes every thread's flags before this CTA's arrival
+    const bool any = __syncthreads_or(wrote);
+    volatile int *s_ok = reinterpret_cast<volatile int *>(smem + kAbort + 8);
+    if (tid == 0) {
+        if (any)
+            __threadfence();
+        atomicAdd(p.ctr, 1u);
+        const long long t0 = clock64();
+        int ok = 1;
+        while (ld_acquire_gpu(p.ctr) < gridDim.x) {
+            if (clock64() - t0 > kWaitCycles) {
+                record_error(p.hdr, SIGE_ERR_TIMEOUT, kSiteGrid);
+                ok = 0;
+                break;
+            }
+            __nanosleep(64);
+        }
+        *s_ok = ok;
+    }
+    __syncthreads();
+    const bool ok = *s_ok != 0;
+    // ---- C: flags -> shared, dilate, compact
+    uint8_t *s_flag = smem + kOffX;                 // halo buffer, unused until the first halo
+    uint8_t *s_act = s_flag + kMaxTiles;
+    int *s_wsum = reinterpret_cast<int *>(smem + kOffY);
+    int2 *s_units = reinterpret_cast<int2 *>(smem + kUnits);
+    if (ok) {
+        for (int i = tid; i < nt; i += kThreads)
+            s_flag[i] = __ldcg(p.flags + i);
+    }
+    __syncthreads();
+    const int seg = (nt + kThreads - 1) / kThreads;
+    const int t0 = min(nt, tid * seg), t1 = min(nt, t0 + seg);
+    const int D = p.dilate;
+    int cnt = 0;
+    for (int t = t0; t < t1; ++t) {
+        int act = 0;
+        if (ok) {
+            const int ty = t / tw, tx = t - ty * tw;
+            for (int dy = max(0, ty - D); dy <= min(p.th - 1, ty + D) && !act; ++dy)
+                for (int dx = max(0, tx - D); dx <= min(tw - 1, tx + D) && !act; ++dx)
+                    act = s_flag[dy * tw + dx];
+        }
+        s_act[t] = (uint8_t)act;
+        cnt += act;
+    }
+    // exclusive scan of the per-thread counts in thread order (= tile order)
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o)
+            incl += v;
+    }
+    if (lane == 31)
+        s_wsum[wid] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int w = 0; w < kThreads / 32; ++w) {
+        const int v = s_wsum[w];
+        before += w < wid ? v : 0;
+        total += v;
+    }
+    int pos = before + incl - cnt;
+    const int n_list = min(total, p.cap);
+    for (int t = t0; t < t1; ++t) {
+        if (!s_act[t])
+            continue;
+        const int2 org = make_int2((t / tw) * kB, (t - (t / tw) * tw) * kB);
+        if (pos < n_list) {
+            if (blockIdx.x == 0)
+                reinterpret_cast<int2 *>(const_cast<int32_t *>(p.idx))[pos] = org;
+            for (int n = 0; n < p.N; ++n) {
+                const int u = pos * p.N + n;
+                if (u % npairs == pair && u / npairs < kMaxUnits)
+                    s_units[u / npairs] = org;
+            }
+        }
+        ++pos;
+    }
+    if (blockIdx.x == 0 && tid == 0) {
+        *const_cast<int32_t *>(p.count) = ok ? total : 0;
+        if (total > p.cap)
+            record_error(p.hdr, SIGE_ERR_CAPACITY, 0);
+    }
+    __syncthreads();
+    // every CTA has its copy of the flags: the last one out clears them and
+    // the counters for the next call
+    if (tid == 0) {
+        __threadfence();
+        if (atomicAdd(p.ctr + 1, 1u) == gridDim.x - 1) {
+            for (int i = 0; i < nt; i += 16)
+                *reinterpret_cast<uint4 *>(p.flags + i) = make_uint4(0, 0, 0, 0);
+            p.ctr[0] = 0;
+            p.ctr[1] = 0;
+            __threadfence();
+        }
+    }
+    __syncthreads();
+    if (!ok)
+        *abort_flag = 1;
+    return ok ? n_list * p.N : 0;
+}
+
+template <bool kStep>
 __global__ void __launch_bounds__(rb::kThreads, 1)
     k_resblock(const __grid_constant__ RbArgs args, const __grid_constant__ CUtensorMap tmx,
                const __grid_constant__ CUtensorMap tw1, const __grid_constant__ CUtensorMap tw2)
@@ -226,14 +419,15 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
     bool cwaited = false;
     pdl_trigger();
 
-    if (warp == 0) {
-        // ------------------------------------------------ weight stages (TMA)
-        // The weights do not come from the previous kernel: the first stages
-        // of W1 go out before the wait for it.
-        int s = 0, issued = 0;
-        uint32_t ph = 1;
-        bool ok = true;
-        auto issue = [&](int conv, int j) -> bool {
+    // ---------------------------------------------------- weight stages (TMA)
+    // The weights do not come from the previous kernel: the first stages of W1
+    // go out before the wait for it (and, in the step, while the difference
+    // mask streams).
+    int s = 0, issued = 0;
+    uint32_t ph = 1;
+    bool ok = true;
+    const int pre = kStages < kChunks ? kStages : kChunks;
+    auto issue = [&](int conv, int j) -> bool {
             if (!mbar_wait_w(w_empty(s), ph, abort_flag, hdr, kSiteWEmpty))
                 return false;
             const int kc2 = j / 9, tap = j - kc2 * 9;
@@ -245,12 +439,19 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                 ph ^= 1;
             }
             return true;
-        };
-        const int pre = kStages < kChunks ? kStages : kChunks;
+    };
+    if (warp == 0) {
         for (int j = 0; j < pre && ok; ++j)
             ok = issue(0, j);
-        pdl_wait();
-        const int units = min(__ldg(p.count), p.cap) * p.N;
+    }
+    pdl_wait();
+    int units;
+    if constexpr (kStep)
+        units = rb_step_list(p, smem, abort_flag, pair, npairs);
+    else
+        units = min(__ldg(p.count), p.cap) * p.N;
+
+    if (warp == 0) {
         bool first = true;
 #pragma unroll 1
         for (int u = pair; u < units && ok; u += npairs) {
@@ -275,14 +476,12 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        pdl_wait();
-        const int units = min(__ldg(p.count), p.cap) * p.N;
         const uint32_t idesc = idesc_bf16(64);          // M = 128 pixels, N = 64 output channels
         const uint64_t b_desc0 = desc_sw128(sb + kOffW);
         const uint64_t w_step = kWStage >> 4;
-        int s = 0;
-        uint32_t ph = 0, ait = 0;
-        bool ok = true;
+        s = 0;
+        ph = 0;
+        uint32_t ait = 0;
         cluster_wait_acq();
         cwaited = true;
         uint64_t b_cur = b_desc0;
@@ -371,13 +570,15 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
         const uint32_t t_lane = tmem + ((uint32_t)(sp * 32) << 16);
         const int cb = (int)rank * 64 + colh * 32;     // first output channel of this thread
         const int H = p.H, W = p.W;
-        pdl_wait();
-        const int units = min(__ldg(p.count), p.cap) * p.N;
-        bool ok = true, x_pending = false;
+        bool x_pending = false;
         uint32_t xk = 0;                               // halos loaded so far (phase of x_full / x_ready)
 
         auto origin = [&](int u, int &h0, int &w0, int &n) {
-            const int2 o = __ldg(reinterpret_cast<const int2 *>(p.idx) + u / p.N);
+            int2 o;
+            if constexpr (kStep)
+                o = reinterpret_cast<const int2 *>(smem + kUnits)[(u - pair) / npairs];
+            else
+                o = __ldg(reinterpret_cast<const int2 *>(p.idx) + u / p.N);
             h0 = o.x;
             w0 = o.y;
             n = u % p.N;
@@ -610,15 +811,36 @@ static bool overlaps(const void *a, const void *b, size_t n)
     return x < y + n && y < x + n;
 }
 
-} // namespace sige
+// Shared-memory opt-in and co-resident pairs of a kernel instance, per device.
+template <bool kStep>
+static int rb_pairs(int dev, cudaLaunchConfig_t &cfg)
+{
+    static std::atomic<int> pairs_of[64];
+    int pairs = pairs_of[dev].load(std::memory_order_acquire);
+    if (pairs == 0) {
+        if (cudaFuncSetAttribute(k_resblock<kStep>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rb::kSmem) !=
+            cudaSuccess)
+            return -1;
+        cfg.gridDim = dim3(2 * (device_sm_count() / 2));
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, k_resblock<kStep>, &cfg) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            return -1;
+        }
+        pairs = n;
+        pairs_of[dev].store(n, std::memory_order_release);
+    }
+    return pairs;
+}
 
-using namespace sige;
-
-extern "C" int sige_resblock_fused(const void *x_edit, const sige_tensor_desc *xd, const void *w1, const float *b1,
-                                   const float *gn1_scale, const float *gn1_shift, const void *w2, const float *b2,
-                                   const float *gn2_scale, const float *gn2_shift, int32_t block,
-                                   const int32_t *idx, const int32_t *count, int32_t capacity, void *y1, void *out,
-                                   void *workspace, size_t workspace_bytes, sige_stream_t stream)
+// Checks shared by both entry points; fills the tensor maps and the
+// argument block.
+static int rb_prepare(const void *x_edit, const sige_tensor_desc *xd, const void *w1, const float *b1,
+                      const float *gn1_scale, const float *gn1_shift, const void *w2, const float *b2,
+                      const float *gn2_scale, const float *gn2_shift, int32_t block, const int32_t *idx,
+                      const int32_t *count, int32_t capacity, void *y1, void *out, void *workspace,
+                      size_t workspace_bytes, size_t ws_need, bool maps, RbArgs &a, CUtensorMap &tmx,
+                      CUtensorMap &tw1, CUtensorMap &tw2)
 {
     if (!x_edit || !xd || !w1 || !w2 || !gn1_scale || !gn1_shift || !gn2_scale || !gn2_shift || !idx || !count ||
         !y1 || !out || capacity < 0)
@@ -636,19 +858,17 @@ extern "C" int sige_resblock_fused(const void *x_edit, const sige_tensor_desc *x
     const size_t bytes = (size_t)xd->n * xd->h * xd->w * xd->c * 2;
     if (overlaps(x_edit, y1, bytes) || overlaps(x_edit, out, bytes) || overlaps(y1, out, bytes))
         return SIGE_ERR_INVALID_ARG;
-    if (!workspace || workspace_bytes < kWsHeader || !aligned(workspace, 16))
+    if (!workspace || workspace_bytes < ws_need || !aligned(workspace, 16))
         return SIGE_ERR_WORKSPACE;
-    if (capacity == 0)
-        return SIGE_OK;
-    auto encode = get_encode();
-    if (!encode)
-        return SIGE_ERR_CUDA;
-    CUtensorMap tmx, tw1, tw2;
-    if (!encode_halo(&tmx, x_edit, xd->n, xd->h, xd->w, encode) || !encode_weights(&tw1, w1, encode) ||
-        !encode_weights(&tw2, w2, encode))
-        return SIGE_ERR_UNSUPPORTED;
-
-    RbArgs a{};
+    if (maps) {
+        auto encode = get_encode();
+        if (!encode)
+            return SIGE_ERR_CUDA;
+        if (!encode_halo(&tmx, x_edit, xd->n, xd->h, xd->w, encode) || !encode_weights(&tw1, w1, encode) ||
+            !encode_weights(&tw2, w2, encode))
+            return SIGE_ERR_UNSUPPORTED;
+    }
+    a = RbArgs{};
     a.x = static_cast<const uint8_t *>(x_edit);
     a.idx = idx;
     a.count = count;
@@ -665,9 +885,13 @@ extern "C" int sige_resblock_fused(const void *x_edit, const sige_tensor_desc *x
     a.H = xd->h;
     a.W = xd->w;
     a.cap = capacity;
+    return SIGE_OK;
+}
 
-    // per device: the shared-memory opt-in and the number of co-resident pairs
-    static std::atomic<int> pairs_of[64];
+template <bool kStep>
+static int rb_launch(const RbArgs &a, const CUtensorMap &tmx, const CUtensorMap &tw1, const CUtensorMap &tw2,
+                     int64_t units_max, sige_stream_t stream)
+{
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return SIGE_ERR_CUDA;
@@ -684,25 +908,99 @@ extern "C" int sige_resblock_fused(const void *x_edit, const sige_tensor_desc *x
     cfg.stream = (cudaStream_t)stream;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    int pairs = pairs_of[dev].load(std::memory_order_acquire);
-    if (pairs == 0) {
-        if (cudaFuncSetAttribute(k_resblock, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rb::kSmem) !=
-            cudaSuccess)
-            return SIGE_ERR_CUDA;
-        cfg.gridDim = dim3(2 * (device_sm_count() / 2));
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, k_resblock, &cfg) != cudaSuccess || n < 1) {
-            cudaGetLastError();
-            return SIGE_ERR_CUDA;
-        }
-        pairs = n;
-        pairs_of[dev].store(n, std::memory_order_release);
+    const int pairs = rb_pairs<kStep>(dev, cfg);
+    if (pairs < 1)
+        return SIGE_ERR_CUDA;
+    // the step's grid barrier needs every CTA resident at once: as many pairs
+    // as fit (and every unit a pair takes must fit its table); the list call
+    // launches no more pairs than there can be units
+    int64_t g = pairs;
+    if (kStep) {
+        if (units_max > (int64_t)rb::kMaxUnits * pairs)
+            return SIGE_ERR_UNSUPPORTED;
+    } else {
+        g = std::min<int64_t>(pairs, units_max);
     }
-    const int64_t units = (int64_t)capacity * xd->n;
-    cfg.gridDim = dim3(2 * (unsigned)std::min<int64_t>(pairs, units));
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_resblock, a, tmx, tw1, tw2);
+    cfg.gridDim = dim3(2 * (unsigned)g);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_resblock<kStep>, a, tmx, tw1, tw2);
     count_launch();
     if (e != cudaSuccess)
         return SIGE_ERR_CUDA;
     return launch_check();
+}
+
+size_t rb_step_workspace_bytes(int32_t tiles)
+{
+    return kWsHeader + (((size_t)std::max(tiles, 0) + 15) & ~(size_t)15);
+}
+
+} // namespace sige
+
+using namespace sige;
+
+extern "C" int sige_resblock_fused(const void *x_edit, const sige_tensor_desc *xd, const void *w1, const float *b1,
+                                   const float *gn1_scale, const float *gn1_shift, const void *w2, const float *b2,
+                                   const float *gn2_scale, const float *gn2_shift, int32_t block,
+                                   const int32_t *idx, const int32_t *count, int32_t capacity, void *y1, void *out,
+                                   void *workspace, size_t workspace_bytes, sige_stream_t stream)
+{
+    RbArgs a;
+    CUtensorMap tmx, tw1, tw2;
+    const int st = rb_prepare(x_edit, xd, w1, b1, gn1_scale, gn1_shift, w2, b2, gn2_scale, gn2_shift, block, idx,
+                              count, capacity, y1, out, workspace, workspace_bytes, kWsHeader, capacity > 0, a, tmx,
+                              tw1, tw2);
+    if (st != SIGE_OK || capacity == 0)
+        return st;
+    return rb_launch<false>(a, tmx, tw1, tw2, (int64_t)capacity * xd->n, stream);
+}
+
+extern "C" size_t sige_resblock_step_workspace_bytes(const sige_tensor_desc *xd, int32_t block)
+{
+    if (!xd || xd->h < 1 || xd->w < 1 || block < 1)
+        return 0;
+    const int64_t tiles = (int64_t)((xd->h + block - 1) / block) * ((xd->w + block - 1) / block);
+    return tiles > INT32_MAX ? 0 : rb_step_workspace_bytes((int32_t)tiles);
+}
+
+extern "C" int sige_resblock_step(const void *x_orig, const void *x_edit, const sige_tensor_desc *xd, float threshold,
+                                  int32_t dilate, const void *w1, const float *b1, const float *gn1_scale,
+                                  const float *gn1_shift, const void *w2, const float *b2, const float *gn2_scale,
+                                  const float *gn2_shift, int32_t block, int32_t *idx, int32_t *count,
+                                  int32_t capacity, void *y1, void *out, void *workspace, size_t workspace_bytes,
+                                  sige_stream_t stream)
+{
+    if (!x_orig || !(threshold >= 0.0f) || dilate < 0)
+        return SIGE_ERR_INVALID_ARG;
+    if (!xd || xd->h < 1 || xd->w < 1 || block != rb::kB)
+        return !xd || xd->h < 1 || xd->w < 1 || block < 1 ? SIGE_ERR_INVALID_ARG : SIGE_ERR_UNSUPPORTED;
+    const int th = (xd->h + block - 1) / block, tw = (xd->w + block - 1) / block;
+    if ((int64_t)th * tw > rb::kMaxTiles)
+        return SIGE_ERR_UNSUPPORTED;
+    RbArgs a;
+    CUtensorMap tmx, tw1, tw2;
+    const int st = rb_prepare(x_edit, xd, w1, b1, gn1_scale, gn1_shift, w2, b2, gn2_scale, gn2_shift, block, idx,
+                              count, capacity, y1, out, workspace, workspace_bytes,
+                              rb_step_workspace_bytes(th * tw), false, a, tmx, tw1, tw2);
+    if (st != SIGE_OK)
+        return st;
+    const size_t bytes = (size_t)xd->n * xd->h * xd->w * xd->c * 2;
+    if (!aligned(x_orig, 16))
+        return SIGE_ERR_UNSUPPORTED;
+    if (overlaps(x_orig, y1, bytes) || overlaps(x_orig, out, bytes))
+        return SIGE_ERR_INVALID_ARG;
+    auto encode = get_encode();
+    if (!encode)
+        return SIGE_ERR_CUDA;
+    if (!encode_halo(&tmx, x_edit, xd->n, xd->h, xd->w, encode) || !encode_weights(&tw1, w1, encode) ||
+        !encode_weights(&tw2, w2, encode))
+        return SIGE_ERR_UNSUPPORTED;
+    a.xo = static_cast<const uint8_t *>(x_orig);
+    a.thr = threshold;
+    a.dilate = dilate;
+    a.th = th;
+    a.tw = tw;
+    WsHeader *h = static_cast<WsHeader *>(workspace);
+    a.ctr = &h->arrive;
+    a.flags = static_cast<uint8_t *>(workspace) + kWsHeader;
+    return rb_launch<true>(a, tmx, tw1, tw2, (int64_t)capacity * xd->n, stream);
 }

@@ -316,3 +316,26 @@ def test_conv_fused_ext_validation(L):
     assert call(transposed=0, op=0, yd=ctypes.byref(yd_plain)) != sige.ERR_INVALID_ARG
     assert call(g=0x3008) == sige.ERR_UNSUPPORTED       # misaligned modulation map
     assert call(wsb=16) == sige.ERR_WORKSPACE
+
+
+def test_resblock_step_validation(L):
+    xd = sige.TensorDesc(1, 64, 64, 128, sige.BF16, sige.NHWC)
+    need = L.sige_resblock_step_workspace_bytes(ctypes.byref(xd), 8)
+    assert need == 256 + 64                      # header + one flag byte per 8x8 tile
+    fake = ctypes.c_void_p(0x1000)
+    ws = ctypes.c_void_p(0x2000)
+
+    def call(**kw):
+        a = dict(xo=ctypes.c_void_p(0x30000000), x=fake, xd=ctypes.byref(xd), thr=1e-3, dil=1, w1=fake, b1=None,
+                 g1s=fake, g1h=fake, w2=fake, b2=None, g2s=fake, g2h=fake, block=8, idx=fake, cnt=fake, cap=64,
+                 y1=ctypes.c_void_p(0x10000000), out=ctypes.c_void_p(0x20000000), ws=ws, wsb=need, st=None)
+        a.update(kw)
+        return L.sige_resblock_step(*a.values())
+    assert call(xo=None) == sige.ERR_INVALID_ARG
+    assert call(thr=-1.0) == sige.ERR_INVALID_ARG
+    assert call(thr=float("nan")) == sige.ERR_INVALID_ARG
+    assert call(dil=-1) == sige.ERR_INVALID_ARG
+    assert call(block=4) == sige.ERR_UNSUPPORTED
+    assert call(wsb=need - 1) == sige.ERR_WORKSPACE
+    assert call(y1=ctypes.c_void_p(0x30000000)) == sige.ERR_INVALID_ARG     # y1 overlaps x_orig
+    assert call(xo=ctypes.c_void_p(0x30000008)) == sige.ERR_UNSUPPORTED     # x_orig needs 16-byte alignment

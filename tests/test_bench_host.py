@@ -46,6 +46,15 @@ def test_resblock_work_per_tile():
     assert f1 - (f2 - f1) == 0
 
 
+def test_step_work():
+    # the one-launch step: both inputs once, y1 and out at the tiles, both
+    # weight tensors, and the list; the MACs of both convs on the tiles
+    f, b = bench.step_work(51)
+    assert f == 51 * 2 * 18_874_368
+    fixed = 2 * (128 * 9 * 128 * 2) + 6 * 128 * 4
+    assert b == 33_554_436 + 51 * 8 + 51 * 2 * 16_384 + fixed
+
+
 def test_mask_work():
     # both 256x256x128 bf16 activations read once, the list written
     assert bench.mask_work(0) == 2 * 256 * 256 * 128 * 2 + 4 == 33_554_436

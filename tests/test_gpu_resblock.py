@@ -165,3 +165,76 @@ def test_fused_resblock_argument_checks():
     with pytest.raises(sige.SigeError) as ei:         # 64 channels: not this kernel's shape
         sige.sige_resblock_fused(x, w, None, g, w, None, g, idx, cnt, 16, x.clone(), x.clone())
     assert ei.value.status == sige.ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------------ one-launch step
+
+def _step(blk, xo, xe, cap, ws=None, thr=1e-3):
+    cd, (w1, b1, w2, b2), gn1, gn2, y1c, outc = _caches(blk, xo)
+    y1, out = y1c.clone(), outc.clone()
+    if ws is None:
+        ws = sige.zeros_workspace(sige.sige_resblock_step_workspace_bytes(xe), DEV)
+    idx, cnt = sige.sige_resblock_step(xo, xe, thr, w1, b1, gn1, w2, b2, gn2, y1, out, cap, workspace=ws)
+    torch.cuda.synchronize()
+    return idx, cnt, ws, y1, out, y1c, outc
+
+
+@pytest.mark.parametrize("H,W,area,seed,N", [(64, 64, 0.05, 40, 1), (256, 256, 0.012, 40, 1),
+                                             (256, 256, 0.20, 41, 1), (68, 60, 0.08, 3, 1), (64, 64, 0.04, 50, 2)])
+def test_step_vs_oracle(orc, H, W, area, seed, N):
+    blk = inputs.make_cfg3(seed, H=H, W=W, area=area)
+    x_orig, x_edit = blk.x_orig, blk.x_edit
+    if N == 2:
+        c = inputs.make_cfg3(seed + 1, H=H, W=W, area=area)
+        x_orig, x_edit = torch.cat([x_orig, c.x_orig]), torch.cat([x_edit, c.x_edit])
+    b = blk.block
+    cap = -(-H // b) * -(-W // b)
+    xo, xe = x_orig.to(DEV), x_edit.to(DEV)
+    idx, cnt, ws, y1, out, y1c, outc = _step(blk, xo, xe, cap)
+    n = int(cnt[0].item())
+    ref_idx = orc.reduce_mask(x_orig, x_edit, 1e-3, [(H, W, b)], 1)[0]
+    assert n == len(ref_idx) and np.array_equal(idx[:n].cpu().numpy(), ref_idx)
+    midx, mcnt, _ = sige.sige_reduce_mask(xo, xe, 1e-3, [(H, W, b, cap)], 1)
+    assert int(mcnt[0].item()) == n and torch.equal(midx[:n].cpu(), idx[:n].cpu())
+    assert int(ws.count_nonzero().item()) == 0, "the workspace must be left zero-filled"
+    _check(orc, blk, x_orig, x_edit, ref_idx, y1, out, y1c, outc)
+
+
+def test_step_twice_on_one_workspace(orc):
+    """The second call finds the workspace as the first left it (zero) and
+    gives its own edit's list and outputs."""
+    a = inputs.make_cfg3(60, H=128, W=128, area=0.02)
+    c = inputs.make_cfg3(61, H=128, W=128, area=0.05)
+    cap = 256
+    ws = sige.zeros_workspace(sige.sige_resblock_step_workspace_bytes(a.x_orig), DEV)
+    for blk in (a, c, a):
+        xo, xe = blk.x_orig.to(DEV), blk.x_edit.to(DEV)
+        idx, cnt, _, y1, out, y1c, outc = _step(blk, xo, xe, cap, ws=ws)
+        n = int(cnt[0].item())
+        ref_idx = orc.reduce_mask(blk.x_orig, blk.x_edit, 1e-3, [(128, 128, 8)], 1)[0]
+        assert np.array_equal(idx[:n].cpu().numpy(), ref_idx)
+        _check(orc, blk, blk.x_orig, blk.x_edit, ref_idx, y1, out, y1c, outc)
+    assert sige.sige_get_device_error(ws) == sige.OK
+
+
+def test_step_capacity_overflow_truncates_and_reports(orc):
+    blk = inputs.make_cfg3(62, H=64, W=64, area=0.08)
+    xo, xe = blk.x_orig.to(DEV), blk.x_edit.to(DEV)
+    ref_idx = orc.reduce_mask(blk.x_orig, blk.x_edit, 1e-3, [(64, 64, 8)], 1)[0]
+    cap = len(ref_idx) // 2
+    assert cap >= 1
+    idx, cnt, ws, y1, out, y1c, outc = _step(blk, xo, xe, cap)
+    assert int(cnt[0].item()) == len(ref_idx)
+    assert np.array_equal(idx[:cap].cpu().numpy(), ref_idx[:cap])
+    assert sige.sige_get_device_error(ws) == sige.ERR_CAPACITY
+    # the first `cap` tiles are processed, nothing else
+    _check(orc, blk, blk.x_orig, blk.x_edit, ref_idx[:cap], y1, out, y1c, outc)
+
+
+def test_step_without_an_edit_writes_nothing():
+    blk = inputs.make_cfg3(63, H=64, W=64, area=0.05)
+    xo = blk.x_orig.to(DEV)
+    idx, cnt, ws, y1, out, y1c, outc = _step(blk, xo, xo.clone(), 64)
+    assert int(cnt[0].item()) == 0
+    assert torch.equal(bits(y1.cpu()), bits(y1c.cpu())) and torch.equal(bits(out.cpu()), bits(outc.cpu()))
+    assert int(ws.count_nonzero().item()) == 0

@@ -157,6 +157,31 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
         v[k] = __uint_as_float(r[k]);
 }
 
+// SiLU v * sigmoid(v) with sigmoid(v) = (1 + tanh(v / 2)) / 2: one special-
+// function instruction per element (tanh.approx.f32, absolute error of the
+// tanh about 2^-11) instead of an exponential and a division, which halves
+// the work of the special-function units that bound the halo transform and
+// epilogue 1; the value is rounded to bf16 (8 significant bits) right after.
+__device__ __forceinline__ float rb_silu(float v)
+{
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * v));
+    return v * __fmaf_rn(0.5f, t, 0.5f);
+}
+
+// GroupNorm affine + SiLU of 8 bf16 channels (parameters in registers).
+__device__ __forceinline__ uint4 rb_gn_silu16(uint4 in, const float (&sc)[8], const float (&sh)[8])
+{
+    uint4 out;
+    uint32_t *o = reinterpret_cast<uint32_t *>(&out);
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(&in);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        o[q] = pack_bf16x2(rb_silu(__fmaf_rn(bf16_lo(w[q]), sc[2 * q], sh[2 * q])),
+                           rb_silu(__fmaf_rn(bf16_hi(w[q]), sc[2 * q + 1], sh[2 * q + 1])));
+    return out;
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v)
 {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
@@ -446,10 +471,14 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
     }
     pdl_wait();
     int units;
-    if constexpr (kStep)
+    int2 org0 = make_int2(0, 0);   // list mode: the pair's first tile origin, read beside the count
+    if constexpr (kStep) {
         units = rb_step_list(p, smem, abort_flag, pair, npairs);
-    else
+    } else {
+        if (warp >= 2 && pair < p.cap * p.N)
+            org0 = __ldg(reinterpret_cast<const int2 *>(p.idx) + pair / p.N);
         units = min(__ldg(p.count), p.cap) * p.N;
+    }
 
     if (warp == 0) {
         bool first = true;
@@ -503,7 +532,6 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                     const int r = tap / 3, c = tap - r * 3;
                     if (!mbar_wait_w(w_full(s), ph, abort_flag, hdr, kSiteWFull))
                         return false;
-                    tc_fence_after();
                     const uint64_t a_desc = desc_plain(chunk + (uint32_t)(pitch * r + c) * 16u, kc_bytes, 128);
                     rb_mma4(tmem + d_col, a_desc, a_step, b_cur, idesc, (kc2 | tap) ? 1u : 0u, w_empty(s));
                     ++ait;
@@ -578,7 +606,7 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
             if constexpr (kStep)
                 o = reinterpret_cast<const int2 *>(smem + kUnits)[(u - pair) / npairs];
             else
-                o = __ldg(reinterpret_cast<const int2 *>(p.idx) + u / p.N);
+                o = u == pair ? org0 : __ldg(reinterpret_cast<const int2 *>(p.idx) + u / p.N);
             h0 = o.x;
             w0 = o.y;
             n = u % p.N;
@@ -618,7 +646,7 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                     const int Y = h0 - 2 + yy, X = w0 - 2 + xx;
                     if (Y >= 0 && Y < H && X >= 0 && X < W) {
                         uint4 *d = reinterpret_cast<uint4 *>(base + px * 16);
-                        *d = transform16_bf16_reg(*d, gs, gh, true, 1);
+                        *d = rb_gn_silu16(*d, gs, gh);
                     }
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -666,13 +694,7 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                     y1p[q] = pack_bf16x2(v[2 * q] + bias[2 * q], v[2 * q + 1] + bias[2 * q + 1]);
                     float a = __fmaf_rn(bf16_lo(y1p[q]), gs[2 * q], gh[2 * q]);
                     float b = __fmaf_rn(bf16_hi(y1p[q]), gs[2 * q + 1], gh[2 * q + 1]);
-                    tp[q] = inimg ? pack_bf16x2(silu_f(a), silu_f(b)) : 0u;
-                }
-                if (interior) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.y1 + ((((int64_t)n * H + Y) * W + X) * kC + cb) * 2);
-#pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        dst[g] = make_uint4(y1p[4 * g], y1p[4 * g + 1], y1p[4 * g + 2], y1p[4 * g + 3]);
+                    tp[q] = inimg ? pack_bf16x2(rb_silu(a), rb_silu(b)) : 0u;
                 }
                 // the accumulator may take the next tile's conv1
                 tc_fence_before();
@@ -697,9 +719,18 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                         st_peer_v4(map_peer(off, rank ^ 1u), w4);
                     }
                 }
-                asm volatile("fence.proxy.async;" ::: "memory");
+                // the conv2 inputs of both CTAs, written through the generic
+                // proxy, are read next by the tensor cores (async proxy)
+                asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
                 mbar_arrive(y1t_full);
                 mbar_arrive_peer(map_peer(y1t_full, rank ^ 1u));
+                // the cached y1 at the tile interior, off the path to conv2
+                if (interior) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.y1 + ((((int64_t)n * H + Y) * W + X) * kC + cb) * 2);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        dst[g] = make_uint4(y1p[4 * g], y1p[4 * g + 1], y1p[4 * g + 2], y1p[4 * g + 3]);
+                }
             }
             // ------------ the next tile's halo, while conv2 of this one runs
             if (u + npairs < units && !load_x(u + npairs)) {

@@ -12,7 +12,7 @@ sige_conv_fused_ext on the tensor cores:
     SiLU, normalisation statistics of the original (instance norm), against
     ``oracle.spade_conv``;
   * bf16 bar per element (max(2e-2 RMS, one bf16 ulp) of the rounded oracle),
-    plain 2e-2 RMS against the unrounded value, every byte outside the tiles
+    max(2e-2 RMS, half an ulp) against the unrounded value, every byte outside the tiles
     untouched, an every-tile list equal to the dense layer.
 """
 import numpy as np
@@ -21,7 +21,7 @@ import torch
 
 import spatially_sparse_incremental_b200 as sige
 from spatially_sparse_incremental_b200 import inputs
-from helpers import assert_close, bits, rel_err, tile_cover
+from helpers import assert_close, assert_close_unrounded, bits, rel_err, tile_cover
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -46,7 +46,7 @@ def test_transposed_conv_sparse_vs_oracle(orc, layer):
     y = sige.sige_conv_fused_ext(xo, w, bias, cd, transposed=True, output_padding=op)
     torch.cuda.synchronize()
     dense_ref = orc.conv_transpose_f64(L.x_orig, L.weight, L.bias)
-    assert rel_err(y.cpu(), torch.from_numpy(dense_ref)) <= 2e-2
+    assert_close_unrounded(y.cpu(), dense_ref, what="dense transposed conv vs unrounded")
     cache = y.clone()
     # tiles at the output resolution, from the output-resolution edit
     idx = orc.reduce_scale(L.meta["edit_out"].astype(np.uint8), Ho, Wo, b, 1)
@@ -59,8 +59,8 @@ def test_transposed_conv_sparse_vs_oracle(orc, layer):
     assert_close(y.cpu(), ref, torch.bfloat16, what="transposed conv")
     cov = tile_cover(idx, b, N, Ho, Wo, co)
     assert torch.equal(bits(y.cpu()[~cov]), bits(cache.cpu()[~cov]))
-    r64 = torch.from_numpy(orc.conv_transpose_f64(L.x_edit, L.weight, L.bias))
-    assert rel_err(y.cpu(), r64, cov) <= 2e-2
+    r64 = orc.conv_transpose_f64(L.x_edit, L.weight, L.bias)
+    assert_close_unrounded(y.cpu(), r64, cov, what="sparse transposed conv vs unrounded")
 
 
 def test_transposed_conv_with_groupnorm_silu_residual(orc):
@@ -114,9 +114,8 @@ def test_spade_conv_sparse_vs_oracle(orc, layer, act):
     assert_close(y.cpu(), ref, torch.bfloat16, what="sparse SPADE conv")
     cov = tile_cover(idx, b, N, H, W, co)
     assert torch.equal(bits(y.cpu()[~cov]), bits(cache.cpu()[~cov]))
-    r64 = torch.from_numpy(orc.spade_conv(L.x_edit, L.weight, L.bias, norm, m["gamma_edit"], m["beta_edit"],
-                                          act=act, rounded=False))
-    assert rel_err(y.cpu(), r64, cov) <= 2e-2
+    r64 = orc.spade_conv(L.x_edit, L.weight, L.bias, norm, m["gamma_edit"], m["beta_edit"], act=act, rounded=False)
+    assert_close_unrounded(y.cpu(), r64, cov, what="sparse SPADE conv vs unrounded")
 
 
 def test_ext_layer_checks():

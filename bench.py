@@ -476,6 +476,10 @@ def measure_extras(dev, flush, stream, peaks, seed, step_graph):
                                                            peaks, spade=True)))
         except Exception as e:
             rows.append({"name": name, "error": str(e)[:200]})
+    try:
+        out["attention"] = attention_timing(seed, dev, flush, stream, peaks)
+    except Exception as e:
+        out["attention"] = {"error": str(e)[:200]}
     # edit-area sweeps of the SD-latent and GauGAN-shaped layers: active tiles,
     # sparse and dense time and the roofline fraction at every area
     sweeps = []
@@ -534,6 +538,44 @@ def layer_timing(L, bits, dev, flush, stream, peaks, reps=30, dense_us=None):
     return {"active_tiles": tiles, "tiles_total": cap, "sparse_us": t_sp, "dense_us": t_de,
             "speedup": t_de / t_sp, "path": "tcgen05" if sige.sige_conv_path(cd, L.x_orig.dtype) == 1 else "cuda-core",
             "roofline": roof}
+
+
+def attention_timing(seed, dev, flush, stream, peaks, H_=64, W_=64, C_=320, heads=8, block=4, area=0.012, reps=20):
+    """The SD-latent self-attention step with pruned queries: the tokens under
+    the 4x4-tile list of a 1.2% edit (one rectangle plus discs at 64x64) attend
+    to all 4096 keys; 8 heads of 40.  Sparse = sige_attention_core at those
+    tokens; dense = the same call with every tile listed."""
+    import spatially_sparse_incremental_b200 as sige
+    from spatially_sparse_incremental_b200 import inputs
+    L = inputs.make_cfg4_layer(seed, 0, area=area)            # the 64x64 C320 map and its edit
+    q = L.x_edit.to(dev)
+    g = torch.Generator().manual_seed(seed)
+    k = torch.randn((1, H_ * W_, C_), generator=g).to(torch.bfloat16).to(dev)
+    v = torch.randn((1, H_ * W_, C_), generator=g).to(torch.bfloat16).to(dev)
+    cap = (H_ // block) * (W_ // block)
+    idx, cnt, _ = sige.sige_reduce_mask(L.x_orig.to(dev), q, 1e-3, [(H_, W_, block, cap)], 1)
+    every = torch.tensor([(h, w) for h in range(0, H_, block) for w in range(0, W_, block)], dtype=torch.int32,
+                         device=dev)
+    call = torch.tensor([cap], dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+    tiles = int(cnt.item())
+    o = torch.zeros((1, H_, W_, C_), dtype=torch.bfloat16, device=dev)
+    g_sp = capture(lambda: sige.sige_attention_core(q, k, v, heads, idx, cnt, cap, block, o, stream), stream)
+    g_de = capture(lambda: sige.sige_attention_core(q, k, v, heads, every, call, cap, block, o, stream), stream)
+    t_sp = float(np.median(time_graph(g_sp, flush, reps, stream))) * 1e3
+    t_de = float(np.median(time_graph(g_de, flush, max(3, reps // 4), stream))) * 1e3
+    del g_sp, g_de
+    m_tok = tiles * block * block
+    flops = 2.0 * m_tok * H_ * W_ * (C_ + C_)
+    nbytes = H_ * W_ * (C_ + C_) * 2 + m_tok * (C_ + C_) * 2
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_alu = flops / (FP32_ALU_TFLOPS * 1e12)
+    return {"name": f"SD latent {H_}x{W_} C{C_} self-attention, {heads} heads, b{block}, {area:.1%} edit",
+            "active_tiles": tiles, "query_tokens": m_tok, "keys": H_ * W_, "sparse_us": t_sp, "dense_us": t_de,
+            "speedup": t_de / t_sp, "path": "cuda-core (fp32 online softmax)",
+            "roofline": {"bound": "tensor", "flops": flops, "bytes": nbytes, "roof_us": t_tensor * 1e6,
+                         "frac": t_tensor / (t_sp * 1e-6),
+                         "alu_roof_us": t_alu * 1e6, "alu_frac": t_alu / (t_sp * 1e-6)}}
 
 
 def ext_layer_timing(L, dev, flush, stream, peaks, transposed=False, spade=False, reps=20):

@@ -105,8 +105,8 @@ struct RbArgs {
     float thr;                  // difference threshold (strict >)
     int32_t dilate;             // tile dilation
     int32_t th, tw;             // tile grid
-    uint8_t *flags;             // [th * tw] tile flags in the workspace, zero on entry and exit
-    uint32_t *ctr;              // [2] grid-barrier arrivals and departures in the workspace header
+    uint32_t *flags;            // [th * tw] tile flags in the workspace: the epoch of the call that set them
+    unsigned long long *ctr;    // grid-barrier arrivals in the workspace header (only grows)
 };
 
 // Four K=16 MMAs of one 64-channel weight stage: A (pixels, no swizzle)
@@ -219,19 +219,26 @@ __device__ __forceinline__ bool rb_exceeds(uint4 a, uint4 b, float thr)
     return r;
 }
 
-// Phases of the one-launch step before the res block, run by every thread of
-// every CTA (mer.dev notes on SIGE, sections 3 and 3.2: difference mask,
-// dilation, tile selection; SIGE project page, "Overview": active block
-// indices):
-//   A. this CTA's contiguous share of x_orig and x_edit, 16-byte loads, eight
-//      in flight per input and thread; a pixel some channel of which differs
-//      by more than thr marks its 8x8 tile in the workspace flags;
-//   B. grid barrier (bounded): every CTA arrives once, all wait for all;
-//   C. the flags (dilated by `dilate` tiles, clipped) compacted in row-major
-//      order -- every CTA computes the same list; CTA 0 writes it and its
-//      count out, each pair keeps the origins of its own units (units
-//      u = pair + j * npairs, tile u / N); the last CTA to finish reading the
-//      flags zeroes them and the two counters for the next call.
+// Phases of the one-launch step before the res block (mer.dev notes on SIGE,
+// sections 3 and 3.2: difference mask, dilation, tile selection; SIGE project
+// page, "Overview": active block indices):
+//   A. warps 1-9 of every CTA stream this CTA's contiguous share of x_orig and
+//      x_edit (16-byte loads, eight in flight per input and thread) while warp
+//      0 issues the first weight stages; a pixel some channel of which differs
+//      by more than thr marks its 8x8 tile: the tile's 32-bit flag is set to
+//      this call's epoch;
+//   B. grid barrier (bounded): every CTA adds one arrival to a 64-bit counter
+//      in the workspace header that only grows, and waits until it reaches
+//      (generation + 1) * CTAs;
+//   C. every CTA reads the flags once (16-byte loads), takes as active the
+//      tiles whose flag equals the epoch, dilates by `dilate` tiles (clipped),
+//      and compacts them in row-major order -- every CTA computes the same
+//      list; CTA 0 writes it and its count out, each pair keeps the origins of
+//      its own units (u = pair + j * npairs, tile u / N).
+// The generation is the counter's value at entry divided by the number of
+// CTAs (every CTA of every call arrives exactly once, so the counter moves by
+// exactly that much per call) and the epoch is generation + 1: flags of
+// earlier calls never equal it, so nothing is cleared between calls.
 // Returns the number of units, min(count, cap) * N.
 __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, volatile int *abort_flag, int pair,
                                             int npairs)
@@ -239,19 +246,29 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
     using namespace rb;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int H = p.H, W = p.W, tw = p.tw, nt = p.th * p.tw;
-    // ---- A: difference mask -> tile flags
+    volatile uint32_t *s_epoch = reinterpret_cast<volatile uint32_t *>(smem + kAbort + 8);
+    volatile int *s_ok = reinterpret_cast<volatile int *>(smem + kAbort + 12);
+    if (tid == 0) {
+        unsigned long long c0;
+        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(c0) : "l"(p.ctr) : "memory");
+        *s_epoch = (uint32_t)(c0 / gridDim.x) + 1u;
+    }
+    __syncthreads();
+    const uint32_t epoch = *s_epoch;
+    // ---- A: difference mask -> tile flags (warps 1-9)
     bool wrote = false;
-    {
+    if (wid >= 1) {
+        const int st = tid - 32, nst = kThreads - 32;
         const int64_t nvec = (int64_t)p.N * H * W * (kC / 8);
         const int64_t per = (nvec + gridDim.x - 1) / gridDim.x;
         const int64_t v0 = (int64_t)blockIdx.x * per, v1 = min(nvec, v0 + per);
         int last = -1;
 #pragma unroll 1
-        for (int64_t base = v0 + tid; base < v1; base += 8 * kThreads) {
+        for (int64_t base = v0 + st; base < v1; base += 8 * nst) {
             uint4 a[8], b[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const int64_t v = base + (int64_t)k * kThreads;
+                const int64_t v = base + (int64_t)k * nst;
                 a[k] = b[k] = make_uint4(0, 0, 0, 0);
                 if (v < v1) {
                     a[k] = __ldg(reinterpret_cast<const uint4 *>(p.xo) + v);
@@ -262,12 +279,12 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
             for (int k = 0; k < 8; ++k) {
                 if (((a[k].x ^ b[k].x) | (a[k].y ^ b[k].y) | (a[k].z ^ b[k].z) | (a[k].w ^ b[k].w)) &&
                     rb_exceeds(a[k], b[k], p.thr)) {
-                    const int64_t pix = (base + (int64_t)k * kThreads) >> 4;   // 16 vectors per pixel
+                    const int64_t pix = (base + (int64_t)k * nst) >> 4;   // 16 vectors per pixel
                     const int64_t hw = pix % ((int64_t)H * W);
                     const int y = (int)(hw / W), x = (int)(hw - (int64_t)y * W);
                     const int t = (y >> 3) * tw + (x >> 3);
                     if (t != last) {
-                        p.flags[t] = 1;
+                        p.flags[t] = epoch;
                         last = t;
                         wrote = true;
                     }
@@ -278,33 +295,40 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
     // ---- B: grid barrier; the fence (cumulative, after the CTA barrier)
     // publishes every thread's flags before this CTA's arrival
     const bool any = __syncthreads_or(wrote);
-    volatile int *s_ok = reinterpret_cast<volatile int *>(smem + kAbort + 8);
     if (tid == 0) {
         if (any)
             __threadfence();
-        atomicAdd(p.ctr, 1u);
+        const unsigned long long target = (unsigned long long)epoch * gridDim.x;
+        atomicAdd(p.ctr, 1ull);
         const long long t0 = clock64();
         int ok = 1;
-        while (ld_acquire_gpu(p.ctr) < gridDim.x) {
+        while (true) {
+            unsigned long long v;
+            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p.ctr) : "memory");
+            if (v >= target)
+                break;
             if (clock64() - t0 > kWaitCycles) {
                 record_error(p.hdr, SIGE_ERR_TIMEOUT, kSiteGrid);
                 ok = 0;
                 break;
             }
-            __nanosleep(64);
+            __nanosleep(32);
         }
         *s_ok = ok;
     }
     __syncthreads();
     const bool ok = *s_ok != 0;
-    // ---- C: flags -> shared, dilate, compact
+    // ---- C: flags -> shared (one round of 16-byte loads), dilate, compact
     uint8_t *s_flag = smem + kOffX;                 // halo buffer, unused until the first halo
     uint8_t *s_act = s_flag + kMaxTiles;
     int *s_wsum = reinterpret_cast<int *>(smem + kOffY);
     int2 *s_units = reinterpret_cast<int2 *>(smem + kUnits);
-    if (ok) {
-        for (int i = tid; i < nt; i += kThreads)
-            s_flag[i] = __ldcg(p.flags + i);
+    for (int i = tid * 4; i < nt; i += kThreads * 4) {
+        const uint4 f = ok ? __ldcg(reinterpret_cast<const uint4 *>(p.flags + i)) : make_uint4(0, 0, 0, 0);
+        s_flag[i] = f.x == epoch;
+        s_flag[i + 1] = f.y == epoch;
+        s_flag[i + 2] = f.z == epoch;
+        s_flag[i + 3] = f.w == epoch;
     }
     __syncthreads();
     const int seg = (nt + kThreads - 1) / kThreads;
@@ -312,13 +336,11 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
     const int D = p.dilate;
     int cnt = 0;
     for (int t = t0; t < t1; ++t) {
+        const int ty = t / tw, tx = t - ty * tw;
         int act = 0;
-        if (ok) {
-            const int ty = t / tw, tx = t - ty * tw;
-            for (int dy = max(0, ty - D); dy <= min(p.th - 1, ty + D) && !act; ++dy)
-                for (int dx = max(0, tx - D); dx <= min(tw - 1, tx + D) && !act; ++dx)
-                    act = s_flag[dy * tw + dx];
-        }
+        for (int dy = max(0, ty - D); dy <= min(p.th - 1, ty + D) && !act; ++dy)
+            for (int dx = max(0, tx - D); dx <= min(tw - 1, tx + D) && !act; ++dx)
+                act = s_flag[dy * tw + dx];
         s_act[t] = (uint8_t)act;
         cnt += act;
     }
@@ -357,22 +379,9 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
         ++pos;
     }
     if (blockIdx.x == 0 && tid == 0) {
-        *const_cast<int32_t *>(p.count) = ok ? total : 0;
+        *const_cast<int32_t *>(p.count) = total;
         if (total > p.cap)
             record_error(p.hdr, SIGE_ERR_CAPACITY, 0);
-    }
-    __syncthreads();
-    // every CTA has its copy of the flags: the last one out clears them and
-    // the counters for the next call
-    if (tid == 0) {
-        __threadfence();
-        if (atomicAdd(p.ctr + 1, 1u) == gridDim.x - 1) {
-            for (int i = 0; i < nt; i += 16)
-                *reinterpret_cast<uint4 *>(p.flags + i) = make_uint4(0, 0, 0, 0);
-            p.ctr[0] = 0;
-            p.ctr[1] = 0;
-            __threadfence();
-        }
     }
     __syncthreads();
     if (!ok)
@@ -626,15 +635,24 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                 x_pending = true;
             }
             const int kcl = et >> 5;
-#pragma unroll 1
+            // both halves' GroupNorm parameters before the first wait
+            float gsa[2][8], gha[2][8];
+#pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int ch = (h * 8 + kcl) * 8;
-                float gs[8], gh[8];
+                const float4 s0 = __ldg(reinterpret_cast<const float4 *>(p.g1s + n * kC + ch));
+                const float4 s1 = __ldg(reinterpret_cast<const float4 *>(p.g1s + n * kC + ch + 4));
+                const float4 h0v = __ldg(reinterpret_cast<const float4 *>(p.g1h + n * kC + ch));
+                const float4 h1v = __ldg(reinterpret_cast<const float4 *>(p.g1h + n * kC + ch + 4));
+                gsa[h][0] = s0.x; gsa[h][1] = s0.y; gsa[h][2] = s0.z; gsa[h][3] = s0.w;
+                gsa[h][4] = s1.x; gsa[h][5] = s1.y; gsa[h][6] = s1.z; gsa[h][7] = s1.w;
+                gha[h][0] = h0v.x; gha[h][1] = h0v.y; gha[h][2] = h0v.z; gha[h][3] = h0v.w;
+                gha[h][4] = h1v.x; gha[h][5] = h1v.y; gha[h][6] = h1v.z; gha[h][7] = h1v.w;
+            }
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    gs[q] = __ldg(p.g1s + n * kC + ch + q);
-                    gh[q] = __ldg(p.g1h + n * kC + ch + q);
-                }
+            for (int h = 0; h < 2; ++h) {
+                const float (&gs)[8] = gsa[h];
+                const float (&gh)[8] = gha[h];
                 if (!mbar_wait_w(x_full(h), xk & 1, abort_flag, hdr, kSiteXFull))
                     return false;
                 if (h == 1 && et == 0)
@@ -962,7 +980,7 @@ static int rb_launch(const RbArgs &a, const CUtensorMap &tmx, const CUtensorMap 
 
 size_t rb_step_workspace_bytes(int32_t tiles)
 {
-    return kWsHeader + (((size_t)std::max(tiles, 0) + 15) & ~(size_t)15);
+    return kWsHeader + (((size_t)std::max(tiles, 0) * 4 + 15) & ~(size_t)15);
 }
 
 } // namespace sige
@@ -1030,8 +1048,8 @@ extern "C" int sige_resblock_step(const void *x_orig, const void *x_edit, const 
     a.dilate = dilate;
     a.th = th;
     a.tw = tw;
-    WsHeader *h = static_cast<WsHeader *>(workspace);
-    a.ctr = &h->arrive;
-    a.flags = static_cast<uint8_t *>(workspace) + kWsHeader;
+    // the arrival counter: 8 bytes at offset 16 of the header
+    a.ctr = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + 16);
+    a.flags = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kWsHeader);
     return rb_launch<true>(a, tmx, tw1, tw2, (int64_t)capacity * xd->n, stream);
 }

@@ -321,7 +321,7 @@ def test_conv_fused_ext_validation(L):
 def test_resblock_step_validation(L):
     xd = sige.TensorDesc(1, 64, 64, 128, sige.BF16, sige.NHWC)
     need = L.sige_resblock_step_workspace_bytes(ctypes.byref(xd), 8)
-    assert need == 256 + 64                      # header + one flag byte per 8x8 tile
+    assert need == 256 + 64 * 4                  # header + one 32-bit flag per 8x8 tile
     fake = ctypes.c_void_p(0x1000)
     ws = ctypes.c_void_p(0x2000)
 

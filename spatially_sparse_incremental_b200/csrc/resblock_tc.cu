@@ -17,10 +17,11 @@
 //
 // Data path of one tile (one "unit"), on a cluster of two CTAs; CTA r owns
 // output channels [64 r, 64 r + 64) of both convs:
-//   * x halo: one TMA per 64 channels, box (8 channels, 12 x, 12 y, 8 channel
-//     groups) of a 5-d view of the NHWC tensor, zero outside the image (the
-//     conv's padding); shared layout [channel group][12 x 12 pixels][8 ch],
-//     then GroupNorm1 + SiLU in place at in-image pixels;
+//   * x halo: one TMA per 64 channels, box (64 channels, 12 x, 12 y) of the
+//     NHWC tensor, landing pixel-major (128-byte rows, zero outside the
+//     image); GroupNorm1 + SiLU then writes it as the conv's input,
+//     [channel group][12 x 12 pixels][8 ch], zero outside the image (the
+//     conv's padding);
 //   * conv1 as an implicit GEMM D[pixel][c_out] = X[pixel][K] W1[c_out][K]^T,
 //     K = (64-channel chunk, tap): A = the halo, read as 128 consecutive
 //     "flat" pixels o = 12 yy + xx (pitch 12), the tap (r, c) being an offset
@@ -59,20 +60,25 @@ constexpr int kC = 128;                    // channels of x, y1 and out
 constexpr int kB = 8;                      // output tile edge
 constexpr int kXE = 12;                    // x halo edge (tile + 2-pixel ring)
 constexpr int kXPix = kXE * kXE;           // 144
-constexpr uint32_t kXKc = kXPix * 16;      // bytes of one 8-channel group of the halo
-constexpr uint32_t kXHalf = 8 * kXKc;      // 64 channels of the halo (one TMA)
+// bytes of one 8-channel group of the conv1 input: 144 pixels and one of
+// padding, so that the groups start 16 bytes apart modulo 128 and the
+// transform's scattered 16-byte writes of 8 groups fall in 8 bank groups
+constexpr uint32_t kXKc = (kXPix + 1) * 16;
+constexpr uint32_t kXHalf = 8 * kXKc;      // 64 channels of the conv1 input
+constexpr uint32_t kSHalf = kXPix * 128;   // 64 channels of the raw halo, pixel-major (one TMA)
 constexpr int kYE = 10;                    // conv2 input edge (tile + 1-pixel ring)
 constexpr uint32_t kYKc = kYE * kYE * 16;  // bytes of one 8-channel group of the conv2 input
 constexpr uint32_t kWStage = 64 * 64 * 2;  // 64 output channels x 64 K, bf16
-constexpr int kStages = 20;                // weight ring
+constexpr int kStages = 15;                // weight ring
 constexpr int kChunks = 18;                // weight stages per conv: 2 channel chunks x 9 taps
 constexpr uint32_t kOffX = 1024;
-constexpr uint32_t kOffY = kOffX + 16 * kXKc;
-constexpr uint32_t kOffW = ((kOffY + 16 * kYKc + 1023) / 1024) * 1024;
+constexpr uint32_t kOffS = kOffX + 16 * kXKc;                       // raw halo, two halves
+constexpr uint32_t kOffY = kOffS + 2 * kSHalf;
+constexpr uint32_t kOffW = ((kOffY + 16 * kYKc + 1023) / 1024 + 1) * 1024;   // (+1 KB: garbage-row reads of conv2)
 constexpr uint32_t kSmem = kOffW + kStages * kWStage + 1024;   // + alignment of the base
 constexpr uint32_t kTmemCols = 128;        // conv1 accumulator [0, 64), conv2 [64, 128)
 static_assert(kSmem <= 232448, "shared memory");
-static_assert(kOffX % 128 == 0 && kXHalf % 128 == 0 && kOffY % 16 == 0, "TMA destinations");
+static_assert(kOffS % 128 == 0 && kSHalf % 128 == 0 && kOffY % 16 == 0, "TMA destinations");
 
 // mbarriers and control words in [0, 1024)
 constexpr uint32_t kBarWFull = 0, kBarWEmpty = 160, kBarXFull = 320, kBarXReady = 336;
@@ -180,6 +186,15 @@ __device__ __forceinline__ uint4 rb_gn_silu16(uint4 in, const float (&sc)[8], co
         o[q] = pack_bf16x2(rb_silu(__fmaf_rn(bf16_lo(w[q]), sc[2 * q], sh[2 * q])),
                            rb_silu(__fmaf_rn(bf16_hi(w[q]), sc[2 * q + 1], sh[2 * q + 1])));
     return out;
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1, int c2,
+                                            int c3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v)
@@ -629,12 +644,15 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
             if (et == 0) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    mbar_expect_tx(x_full(h), kXHalf);
-                    tma_load_5d(sb + kOffX + (uint32_t)h * kXHalf, &tmx, x_full(h), 0, w0 - 2, h0 - 2, h * 8, n);
+                    mbar_expect_tx(x_full(h), kSHalf);
+                    tma_load_4d(sb + kOffS + (uint32_t)h * kSHalf, &tmx, x_full(h), h * 64, w0 - 2, h0 - 2, n);
                 }
                 x_pending = true;
             }
-            const int kcl = et >> 5;
+            // thread: channel group kcl of each half, pixels 4 m + (lane >> 3)
+            // of warp (et >> 5)'s share; a warp reads 4 raw pixels (512
+            // contiguous bytes) and writes 8 groups x 4 pixels
+            const int kcl = et & 7, pq = (et >> 3) & 3, ew = et >> 5;
             // both halves' GroupNorm parameters before the first wait
             float gsa[2][8], gha[2][8];
 #pragma unroll
@@ -657,15 +675,16 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                     return false;
                 if (h == 1 && et == 0)
                     x_pending = false;
-                uint8_t *base = smem + kOffX + h * kXHalf + kcl * kXKc;
+                const uint8_t *raw = smem + kOffS + h * kSHalf + kcl * 16;
+                uint8_t *dst = smem + kOffX + (h * 8 + kcl) * kXKc;
 #pragma unroll 1
-                for (int px = lane; px < kXPix; px += 32) {
+                for (int px = 4 * ew + pq; px < kXPix; px += 32) {
                     const int yy = px / kXE, xx = px - yy * kXE;
                     const int Y = h0 - 2 + yy, X = w0 - 2 + xx;
-                    if (Y >= 0 && Y < H && X >= 0 && X < W) {
-                        uint4 *d = reinterpret_cast<uint4 *>(base + px * 16);
-                        *d = rb_gn_silu16(*d, gs, gh);
-                    }
+                    uint4 v = make_uint4(0, 0, 0, 0);   // outside the image: the conv's zero padding
+                    if (Y >= 0 && Y < H && X >= 0 && X < W)
+                        v = rb_gn_silu16(*reinterpret_cast<const uint4 *>(raw + px * 128), gs, gh);
+                    *reinterpret_cast<uint4 *>(dst + px * 16) = v;
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 mbar_arrive(x_ready(h));
@@ -837,17 +856,18 @@ static bool encode_weights(CUtensorMap *map, const void *w, PFN_cuTensorMapEncod
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 5-d view [n][kc][y][x][8 channels] of the NHWC tensor, so that one box
-// lands as [channel group][y][x][8 channels] in shared memory.
+// The NHWC tensor as a 4-d map [n][y][x][c]; a box of 64 channels x 12 x 12
+// pixels lands pixel-major (128-byte rows) in shared memory, zero outside the
+// image.
 static bool encode_halo(CUtensorMap *map, const void *x, int N, int H, int W,
                         PFN_cuTensorMapEncodeTiled_v12000 encode)
 {
     const cuuint64_t C = rb::kC;
-    cuuint64_t dims[5] = {8, (cuuint64_t)W, (cuuint64_t)H, C / 8, (cuuint64_t)N};
-    cuuint64_t strides[4] = {C * 2, (cuuint64_t)W * C * 2, 16, (cuuint64_t)H * W * C * 2};
-    cuuint32_t box[5] = {8, (cuuint32_t)rb::kXE, (cuuint32_t)rb::kXE, 8, 1};
-    cuuint32_t es[5] = {1, 1, 1, 1, 1};
-    return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(x), dims, strides, box, es,
+    cuuint64_t dims[4] = {C, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)N};
+    cuuint64_t strides[3] = {C * 2, (cuuint64_t)W * C * 2, (cuuint64_t)H * W * C * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)rb::kXE, (cuuint32_t)rb::kXE, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(x), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

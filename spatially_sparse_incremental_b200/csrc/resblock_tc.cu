@@ -65,7 +65,7 @@ constexpr int kXPix = kXE * kXE;           // 144
 // transform's scattered 16-byte writes of 8 groups fall in 8 bank groups
 constexpr uint32_t kXKc = (kXPix + 1) * 16;
 constexpr uint32_t kXHalf = 8 * kXKc;      // 64 channels of the conv1 input
-constexpr uint32_t kSHalf = kXPix * 128;   // 64 channels of the raw halo, pixel-major (one TMA)
+constexpr uint32_t kSHalf = kXPix * 128;   // 64 channels of the raw halo (the TMA box holds both, pixel-major)
 constexpr int kYE = 10;                    // conv2 input edge (tile + 1-pixel ring)
 constexpr uint32_t kYKc = kYE * kYE * 16;  // bytes of one 8-channel group of the conv2 input
 constexpr uint32_t kWStage = 64 * 64 * 2;  // 64 output channels x 64 K, bf16
@@ -83,14 +83,14 @@ static_assert(kOffS % 128 == 0 && kSHalf % 128 == 0 && kOffY % 16 == 0, "TMA des
 // mbarriers and control words in [0, 1024)
 constexpr uint32_t kBarWFull = 0, kBarWEmpty = 160, kBarXFull = 320, kBarXReady = 336;
 constexpr uint32_t kBarAcc1Full = 352, kBarAcc1Empty = 360, kBarAcc2Full = 368, kBarAcc2Empty = 376;
-constexpr uint32_t kBarY1tFull = 384, kBarY1tEmpty = 392, kBarDrain = 400;
+constexpr uint32_t kBarY1tFull = 384, kBarY1tEmpty = 392, kBarDrain = 400, kBarY1tLocal = 408;
 constexpr uint32_t kTmemSlot = 416, kAbort = 420, kUnits = 448;   // kUnits: the step's unit table (int2)
 constexpr int kMaxUnits = 64;              // units one CTA pair takes in the step (tile origins at kUnits)
 constexpr int kMaxTiles = 16384;           // tile grid of the step's mask (flags staged in the halo buffer)
 
 // wait sites recorded in the error detail on a timeout
 enum : int { kSiteWEmpty = 101, kSiteWFull, kSiteXReady, kSiteAcc1Empty, kSiteAcc2Empty, kSiteY1tFull,
-             kSiteXFull, kSiteAcc1Full, kSiteY1tEmpty, kSiteAcc2Full, kSiteGrid };
+             kSiteXFull, kSiteAcc1Full, kSiteY1tEmpty, kSiteAcc2Full, kSiteGrid, kSiteY1tLocal };
 
 }  // namespace rb
 
@@ -278,23 +278,31 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
         const int64_t per = (nvec + gridDim.x - 1) / gridDim.x;
         const int64_t v0 = (int64_t)blockIdx.x * per, v1 = min(nvec, v0 + per);
         int last = -1;
+        // Rolling loads: slot k holds vector base + k * nst; right after it is
+        // compared, the slot is refilled with the vector one round later, so
+        // the memory system always has about eight loads per input and thread
+        // in flight instead of draining between rounds.
+        uint4 a[8], b[8];
+        const uint4 *xo4 = reinterpret_cast<const uint4 *>(p.xo), *xe4 = reinterpret_cast<const uint4 *>(p.x);
+        const uint4 z4 = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int64_t v = v0 + st + (int64_t)k * nst;
+            a[k] = v < v1 ? __ldg(xo4 + v) : z4;
+            b[k] = v < v1 ? __ldg(xe4 + v) : z4;
+        }
 #pragma unroll 1
         for (int64_t base = v0 + st; base < v1; base += 8 * nst) {
-            uint4 a[8], b[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const int64_t v = base + (int64_t)k * nst;
-                a[k] = b[k] = make_uint4(0, 0, 0, 0);
-                if (v < v1) {
-                    a[k] = __ldg(reinterpret_cast<const uint4 *>(p.xo) + v);
-                    b[k] = __ldg(reinterpret_cast<const uint4 *>(p.x) + v);
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                if (((a[k].x ^ b[k].x) | (a[k].y ^ b[k].y) | (a[k].z ^ b[k].z) | (a[k].w ^ b[k].w)) &&
-                    rb_exceeds(a[k], b[k], p.thr)) {
-                    const int64_t pix = (base + (int64_t)k * nst) >> 4;   // 16 vectors per pixel
+                const bool differs = ((a[k].x ^ b[k].x) | (a[k].y ^ b[k].y) | (a[k].z ^ b[k].z) | (a[k].w ^ b[k].w)) &&
+                                     rb_exceeds(a[k], b[k], p.thr);
+                const int64_t vn = v + 8 * (int64_t)nst;
+                a[k] = vn < v1 ? __ldg(xo4 + vn) : z4;
+                b[k] = vn < v1 ? __ldg(xe4 + vn) : z4;
+                if (differs) {
+                    const int64_t pix = v >> 4;   // 16 vectors per pixel
                     const int64_t hw = pix % ((int64_t)H * W);
                     const int y = (int)(hw / W), x = (int)(hw - (int64_t)y * W);
                     const int t = (y >> 3) * tw + (x >> 3);
@@ -346,52 +354,141 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
         s_flag[i + 3] = f.w == epoch;
     }
     __syncthreads();
-    const int seg = (nt + kThreads - 1) / kThreads;
-    const int t0 = min(nt, tid * seg), t1 = min(nt, t0 + seg);
     const int D = p.dilate;
-    int cnt = 0;
-    for (int t = t0; t < t1; ++t) {
-        const int ty = t / tw, tx = t - ty * tw;
-        int act = 0;
-        for (int dy = max(0, ty - D); dy <= min(p.th - 1, ty + D) && !act; ++dy)
-            for (int dx = max(0, tx - D); dx <= min(tw - 1, tx + D) && !act; ++dx)
-                act = s_flag[dy * tw + dx];
-        s_act[t] = (uint8_t)act;
-        cnt += act;
-    }
-    // exclusive scan of the per-thread counts in thread order (= tile order)
-    int incl = cnt;
+    int total = 0, n_list = 0;
+    if (p.th <= 64 && tw <= 64) {
+        // rows of tiles as 64-bit words: warp 0 dilates (shifts across a row,
+        // shuffles across rows) and counts; rows y and y + 32 sit in lane y
+        uint64_t *s_row = reinterpret_cast<uint64_t *>(smem + kOffY);      // [64] dilated rows
+        int *s_pre = reinterpret_cast<int *>(smem + kOffY + 512);          // [65] row prefix, [64] = total
+        if (wid == 0) {
+            const uint64_t full = tw == 64 ? ~0ull : ((1ull << tw) - 1);
+            uint64_t h[2];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o)
-            incl += v;
-    }
-    if (lane == 31)
-        s_wsum[wid] = incl;
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int w = 0; w < kThreads / 32; ++w) {
-        const int v = s_wsum[w];
-        before += w < wid ? v : 0;
-        total += v;
-    }
-    int pos = before + incl - cnt;
-    const int n_list = min(total, p.cap);
-    for (int t = t0; t < t1; ++t) {
-        if (!s_act[t])
-            continue;
-        const int2 org = make_int2((t / tw) * kB, (t - (t / tw) * tw) * kB);
-        if (pos < n_list) {
-            if (blockIdx.x == 0)
-                reinterpret_cast<int2 *>(const_cast<int32_t *>(p.idx))[pos] = org;
-            for (int n = 0; n < p.N; ++n) {
-                const int u = pos * p.N + n;
-                if (u % npairs == pair && u / npairs < kMaxUnits)
-                    s_units[u / npairs] = org;
+            for (int r = 0; r < 2; ++r) {
+                const int y = lane + 32 * r;
+                uint64_t m = 0;
+                if (y < p.th)
+                    for (int x = 0; x < tw; ++x)
+                        m |= (uint64_t)s_flag[y * tw + x] << x;
+                uint64_t hd = m;
+                for (int k = 1; k <= D && k < 64; ++k)
+                    hd |= (m << k) | (m >> k);
+                h[r] = hd & full;
+            }
+            uint64_t d[2] = {0, 0};
+            for (int dy = -D; dy <= D; ++dy) {
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int yy = lane + 32 * r + dy;
+                    const int src = yy & 31;
+                    const uint64_t v0 = __shfl_sync(0xFFFFFFFFu, h[0], src);
+                    const uint64_t v1 = __shfl_sync(0xFFFFFFFFu, h[1], src);
+                    if (yy >= 0 && yy < p.th)
+                        d[r] |= (yy >> 5) ? v1 : v0;
+                }
+            }
+            int c[2];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                if (lane + 32 * r >= p.th)
+                    d[r] = 0;
+                c[r] = __popcll(d[r]);
+            }
+            // row-order prefix: rows 0..31, then 32..63
+            int run = 0;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                int incl = c[r];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                    if (lane >= o)
+                        incl += v;
+                }
+                s_row[lane + 32 * r] = d[r];
+                s_pre[lane + 32 * r] = run + incl - c[r];
+                run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+            }
+            if (lane == 0)
+                s_pre[64] = run;
+        }
+        __syncthreads();
+        total = s_pre[64];
+        n_list = min(total, p.cap);
+        // CTA 0 writes the list: thread y takes row y
+        if (blockIdx.x == 0 && tid < p.th) {
+            uint64_t m = s_row[tid];
+            int pos = s_pre[tid];
+            while (m && pos < n_list) {
+                const int x = __ffsll((long long)m) - 1;
+                m &= m - 1;
+                reinterpret_cast<int2 *>(const_cast<int32_t *>(p.idx))[pos++] = make_int2(tid * kB, x * kB);
             }
         }
-        ++pos;
+        // this pair's units u = pair + j * npairs: the (u / N)-th active tile
+        if (tid < kMaxUnits) {
+            const int u = pair + tid * npairs;
+            if (u < n_list * p.N) {
+                const int pos = u / p.N;
+                int y = 0;
+                while (y + 1 < p.th && s_pre[y + 1] <= pos)
+                    ++y;
+                uint64_t m = s_row[y];
+                for (int r = pos - s_pre[y]; r > 0; --r)
+                    m &= m - 1;
+                const int x = __ffsll((long long)m) - 1;
+                s_units[tid] = make_int2(y * kB, x * kB);
+            }
+        }
+    } else {
+        // larger grids: one pass per thread over a contiguous run of tiles
+        const int seg = (nt + kThreads - 1) / kThreads;
+        const int t0 = min(nt, tid * seg), t1 = min(nt, t0 + seg);
+        int cnt = 0;
+        for (int t = t0; t < t1; ++t) {
+            const int ty = t / tw, tx = t - ty * tw;
+            int act = 0;
+            for (int dy = max(0, ty - D); dy <= min(p.th - 1, ty + D) && !act; ++dy)
+                for (int dx = max(0, tx - D); dx <= min(tw - 1, tx + D) && !act; ++dx)
+                    act = s_flag[dy * tw + dx];
+            s_act[t] = (uint8_t)act;
+            cnt += act;
+        }
+        // exclusive scan of the per-thread counts in thread order (= tile order)
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o)
+                incl += v;
+        }
+        if (lane == 31)
+            s_wsum[wid] = incl;
+        __syncthreads();
+        int before = 0;
+        for (int w = 0; w < kThreads / 32; ++w) {
+            const int v = s_wsum[w];
+            before += w < wid ? v : 0;
+            total += v;
+        }
+        int pos = before + incl - cnt;
+        n_list = min(total, p.cap);
+        for (int t = t0; t < t1; ++t) {
+            if (!s_act[t])
+                continue;
+            const int2 org = make_int2((t / tw) * kB, (t - (t / tw) * tw) * kB);
+            if (pos < n_list) {
+                if (blockIdx.x == 0)
+                    reinterpret_cast<int2 *>(const_cast<int32_t *>(p.idx))[pos] = org;
+                for (int n = 0; n < p.N; ++n) {
+                    const int u = pos * p.N + n;
+                    if (u % npairs == pair && u / npairs < kMaxUnits)
+                        s_units[u / npairs] = org;
+                }
+            }
+            ++pos;
+        }
     }
     if (blockIdx.x == 0 && tid == 0) {
         *const_cast<int32_t *>(p.count) = total;
@@ -422,6 +519,7 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
     const uint32_t acc1_full = sb + kBarAcc1Full, acc1_empty = sb + kBarAcc1Empty;
     const uint32_t acc2_full = sb + kBarAcc2Full, acc2_empty = sb + kBarAcc2Empty;
     const uint32_t y1t_full = sb + kBarY1tFull, y1t_empty = sb + kBarY1tEmpty, drain = sb + kBarDrain;
+    const uint32_t y1t_local = sb + kBarY1tLocal;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kAbort);
     WsHeader *hdr = p.hdr;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -441,8 +539,9 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
         mbar_init(acc1_empty, kEpi);
         mbar_init(acc2_full, 1);
         mbar_init(acc2_empty, kEpi);
-        mbar_init(y1t_full, 2 * kEpi);   // the epilogue threads of both CTAs
+        mbar_init(y1t_full, 1);          // this CTA's half written + the peer's half copied in (tx bytes)
         mbar_init(y1t_empty, 2);         // the conv2 commits of both CTAs
+        mbar_init(y1t_local, kEpi);      // every epilogue thread has written its part of this CTA's half
         mbar_init(drain, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -642,11 +741,8 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
             int h0, w0, n;
             origin(u, h0, w0, n);
             if (et == 0) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    mbar_expect_tx(x_full(h), kSHalf);
-                    tma_load_4d(sb + kOffS + (uint32_t)h * kSHalf, &tmx, x_full(h), h * 64, w0 - 2, h0 - 2, n);
-                }
+                mbar_expect_tx(x_full(0), 2 * kSHalf);
+                tma_load_4d(sb + kOffS, &tmx, x_full(0), 0, w0 - 2, h0 - 2, n);
                 x_pending = true;
             }
             // thread: channel group kcl of each half, pixels 4 m + (lane >> 3)
@@ -671,11 +767,11 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
             for (int h = 0; h < 2; ++h) {
                 const float (&gs)[8] = gsa[h];
                 const float (&gh)[8] = gha[h];
-                if (!mbar_wait_w(x_full(h), xk & 1, abort_flag, hdr, kSiteXFull))
+                if (h == 0 && !mbar_wait_w(x_full(0), xk & 1, abort_flag, hdr, kSiteXFull))
                     return false;
-                if (h == 1 && et == 0)
+                if (et == 0)
                     x_pending = false;
-                const uint8_t *raw = smem + kOffS + h * kSHalf + kcl * 16;
+                const uint8_t *raw = smem + kOffS + h * 128 + kcl * 16;
                 uint8_t *dst = smem + kOffX + (h * 8 + kcl) * kXKc;
 #pragma unroll 1
                 for (int px = 4 * ew + pq; px < kXPix; px += 32) {
@@ -683,7 +779,7 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                     const int Y = h0 - 2 + yy, X = w0 - 2 + xx;
                     uint4 v = make_uint4(0, 0, 0, 0);   // outside the image: the conv's zero padding
                     if (Y >= 0 && Y < H && X >= 0 && X < W)
-                        v = rb_gn_silu16(*reinterpret_cast<const uint4 *>(raw + px * 128), gs, gh);
+                        v = rb_gn_silu16(*reinterpret_cast<const uint4 *>(raw + px * 256), gs, gh);
                     *reinterpret_cast<uint4 *>(dst + px * 16) = v;
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -749,18 +845,31 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                 if (valid) {
                     const uint32_t pix = (uint32_t)(yy * kYE + xx) * 16u;
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        const uint32_t off = sb + kOffY + (uint32_t)(cb / 8 + g) * kYKc + pix;
-                        const uint4 w4 = make_uint4(tp[4 * g], tp[4 * g + 1], tp[4 * g + 2], tp[4 * g + 3]);
-                        st_shared_v4(off, w4);
-                        st_peer_v4(map_peer(off, rank ^ 1u), w4);
+                    for (int g = 0; g < 4; ++g)
+                        st_shared_v4(sb + kOffY + (uint32_t)(cb / 8 + g) * kYKc + pix,
+                                     make_uint4(tp[4 * g], tp[4 * g + 1], tp[4 * g + 2], tp[4 * g + 3]));
+                }
+                // written through the generic proxy, read next by the tensor
+                // cores and the bulk copy (async proxy)
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(y1t_local);
+                if (et == 0) {
+                    // once the whole half is written: one bulk copy of it (this
+                    // CTA's 8 channel groups, 12800 bytes) into the peer's
+                    // buffer, completing on the peer's y1t_full; here, the
+                    // local half is ready and the peer's copy is expected
+                    if (!mbar_wait(y1t_local, k & 1, abort_flag, hdr, kSiteY1tLocal)) {
+                        ok = false;
+                    } else {
+                        const uint32_t src = sb + kOffY + rank * 8u * kYKc;
+                        asm volatile(
+                            "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                            ::"r"(map_peer(src, rank ^ 1u)), "r"(src), "r"(8u * kYKc),
+                            "r"(map_peer(y1t_full, rank ^ 1u))
+                            : "memory");
+                        mbar_expect_tx(y1t_full, 8u * kYKc);
                     }
                 }
-                // the conv2 inputs of both CTAs, written through the generic
-                // proxy, are read next by the tensor cores (async proxy)
-                asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
-                mbar_arrive(y1t_full);
-                mbar_arrive_peer(map_peer(y1t_full, rank ^ 1u));
                 // the cached y1 at the tile interior, off the path to conv2
                 if (interior) {
                     uint4 *dst = reinterpret_cast<uint4 *>(p.y1 + ((((int64_t)n * H + Y) * W + X) * kC + cb) * 2);
@@ -819,11 +928,8 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
         }
         // a halo copy still in flight (a wait gave up) lands before the exit
         if (x_pending) {
-#pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
-                const long long t0 = clock64();
-                while (!mbar_try(x_full(h), xk & 1) && clock64() - t0 < kWaitCycles) {
-                }
+            const long long t0 = clock64();
+            while (!mbar_try(x_full(0), xk & 1) && clock64() - t0 < kWaitCycles) {
             }
         }
     }
@@ -856,16 +962,16 @@ static bool encode_weights(CUtensorMap *map, const void *w, PFN_cuTensorMapEncod
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The NHWC tensor as a 4-d map [n][y][x][c]; a box of 64 channels x 12 x 12
-// pixels lands pixel-major (128-byte rows) in shared memory, zero outside the
-// image.
+// The NHWC tensor as a 4-d map [n][y][x][c]; a box of all 128 channels x 12 x
+// 12 pixels lands pixel-major (256-byte rows) in shared memory, zero outside
+// the image.
 static bool encode_halo(CUtensorMap *map, const void *x, int N, int H, int W,
                         PFN_cuTensorMapEncodeTiled_v12000 encode)
 {
     const cuuint64_t C = rb::kC;
     cuuint64_t dims[4] = {C, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)N};
     cuuint64_t strides[3] = {C * 2, (cuuint64_t)W * C * 2, (cuuint64_t)H * W * C * 2};
-    cuuint32_t box[4] = {64, (cuuint32_t)rb::kXE, (cuuint32_t)rb::kXE, 1};
+    cuuint32_t box[4] = {(cuuint32_t)C, (cuuint32_t)rb::kXE, (cuuint32_t)rb::kXE, 1};
     cuuint32_t es[4] = {1, 1, 1, 1};
     return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(x), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,

@@ -10,4 +10,8 @@ size_t tc_workspace_bytes(const sige_conv_desc *cd, int batch, int ntiles);
 int launch_conv_tc(const ConvParams &p, cudaStream_t stream);
 int tc_schedule(const sige_conv_desc *cd, int tiles, int grid, int csize, int32_t *out, int n_out);
 
+// 3x3 stride-1 layers on 8x8 tiles (pixels as the MMA's M, C_out as N).
+bool conv8_supported(const sige_conv_desc *cd, int dtype);
+int launch_conv8(const ConvParams &p, cudaStream_t stream);
+
 } // namespace sige

@@ -80,8 +80,12 @@ static int run_conv(ConvParams &p, const sige_conv_desc *cd, void *ws, size_t ws
         return SIGE_ERR_WORKSPACE;
     if (ntiles == 0)
         return SIGE_OK;
-    if (choose_path(cd, p.dtype) == 1)
+    if (choose_path(cd, p.dtype) == 1) {
+        // image to image, no GauGAN extension: the 8x8-tile kernel when it fits
+        if (conv8_supported(cd, p.dtype) && p.from_image && p.to_y && !p.tstride && !p.sg && !p.leaky)
+            return launch_conv8(p, st);
         return launch_conv_tc(p, st);
+    }
     return launch_conv_simt(p, st);
 }
 

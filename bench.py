@@ -417,8 +417,12 @@ def measure_extras(dev, flush, stream, peaks, seed, step_graph):
                 fn()
         g = capture(whole, stream)
         t = time_graph(g, flush, 40, stream)
-        sweep.append({"area": area, "active_tiles": tiles, "step_us": float(np.median(t)) * 1e3,
-                      "p90_us": float(np.percentile(t, 90)) * 1e3})
+        fl, by = step_work(tiles)
+        t_roof = max(fl / (peaks["bf16_tflops"] * 1e12), by / (peaks["hbm_gbs"] * 1e9))
+        med = float(np.median(t)) * 1e-3
+        sweep.append({"area": area, "active_tiles": tiles, "step_us": med * 1e6,
+                      "p90_us": float(np.percentile(t, 90)) * 1e3, "roof_us": t_roof * 1e6, "frac": t_roof / med,
+                      "tensor_frac": fl / med / 1e12 / peaks["bf16_tflops"]})
         del g, d
     x = np.array([r["active_tiles"] for r in sweep], dtype=np.float64)
     y = np.array([r["step_us"] for r in sweep], dtype=np.float64)
@@ -930,6 +934,14 @@ def run_sige(args):
     t_roof = max(t_tc, t_bw)
     sparse_conv_ms = kern_ms["resblock"]
     dense_conv_ms = dense_ms["dense1"] + dense_ms["dense2"]
+    # the dense conv of the layer (GroupNorm + SiLU in, bias out) against the
+    # tensor roofline: 2 * 256 * 256 * 128 * 128 * 9 FLOPs per conv
+    dflops = 2.0 * H * W * C * C * 9
+    dense_roof = {"flops_per_conv": dflops, "us": {k: v * 1e3 for k, v in dense_ms.items()},
+                  "tflops": {k: dflops / (v * 1e-3) / 1e12 for k, v in dense_ms.items()},
+                  "frac": {k: dflops / (v * 1e-3) / 1e12 / peaks["bf16_tflops"] for k, v in dense_ms.items()},
+                  "peak_tflops": peaks["bf16_tflops"], "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                  "l2": "cold (flushed before every call)"}
 
     extras = None
     if not args.no_extras:
@@ -973,7 +985,8 @@ def run_sige(args):
         "resblock_roofline": resblock_roof,
         "unfused_step_us": unfused_ms * 1e3,
         "unfused_breakdown_us": {k: v * 1e3 for k, v in ukern_ms.items()},
-        "dense_conv_us": dense_conv_ms * 1e3, "sparse_conv_us": sparse_conv_ms * 1e3,
+        "dense_conv_us": dense_conv_ms * 1e3, "dense_conv_roofline": dense_roof,
+        "sparse_conv_us": sparse_conv_ms * 1e3,
         "speedup_vs_dense_conv": dense_conv_ms / sparse_conv_ms,
         "step_roofline_frac": t_roof / (step_ms * 1e-3),
         "roofline": roof,

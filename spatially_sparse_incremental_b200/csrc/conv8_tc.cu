@@ -3,7 +3,7 @@
 // +residual) in one launch (SIGE project page, "Overview": gather the active
 // blocks with their halo, run F_l on them, scatter into the cached output).
 // Used for every bf16 layer with a 3x3 kernel, stride 1, pad 1, 8x8 tiles,
-// C_in a multiple of 64 and C_out a multiple of 16 up to 256 -- sparse (a
+// C_in a multiple of 64 and C_out a multiple of 32 up to 256 -- sparse (a
 // tile list) and dense (every tile: the cache of the original and the dense
 // baseline).
 //
@@ -22,14 +22,18 @@
 //     swizzle; D in tensor memory, lane = pixel row, column = output channel;
 //   * per 64-channel chunk the halo comes by one TMA of 128-byte pixel rows
 //     (64 channels x 10 x 34 rows of a strip, or 64 x 10 x 10 per tile, zero
-//     outside the image) into a staging buffer; warps 2-5 apply the GroupNorm
-//     affine + SiLU (one tanh per element) and write the A layout, into the
-//     other of two A buffers while the MMAs of the previous chunk run;
-//   * warps 6-9 run the epilogue from the other tensor-memory buffer while
+//     outside the image) into a staging buffer; warps 2-9 apply the GroupNorm
+//     affine + SiLU (one f16x2 tanh per two elements) and write the A layout,
+//     into the other of two A buffers while the MMAs of the previous chunk run;
+//   * warps 10-13 run the epilogue from the other tensor-memory buffer while
 //     the next unit's MMAs run: + bias (+ residual), one rounding to bf16,
-//     16-byte stores of each pixel's channels into the cached output.
-// Warp roles (320 threads): 0 weight TMA, 1 tensor memory + MMA issue (one
-// elected lane), 2-5 halo TMA + transform, 6-9 epilogue.  CTAs are
+//     16-byte stores of each pixel's channels into the cached output;
+//   * every CTA on the device wants the same weight stages at about the same
+//     time; each CTA takes the nine taps of a chunk starting at tap
+//     (CTA index mod 9), so that the requests spread over nine stages' lines
+//     of the L2 instead of one.
+// Warp roles (448 threads): 0 weight TMA, 1 tensor memory + MMA issue (one
+// elected lane), 2-9 halo TMA + transform, 10-13 epilogue.  CTAs are
 // persistent (one per SM) and take units with a stride of the grid.  Every
 // wait is bounded; on expiry the kernel records SIGE_ERR_TIMEOUT (detail =
 // wait site), the roles leave their loops, copies and MMAs in flight are
@@ -44,9 +48,9 @@
 namespace sige {
 namespace c8 {
 
-constexpr int kThreads = 320;
-constexpr int kHaloT = 128;                  // warps 2-5
-constexpr int kEpiT = 128;                   // warps 6-9
+constexpr int kThreads = 448;
+constexpr int kHaloT = 256;                  // warps 2-9
+constexpr int kEpiT = 128;                   // warps 10-13
 constexpr int kRows = 36;                    // A-buffer halo rows (a strip's 34, or 2 x 18 per tile pair)
 constexpr int kCols = 10;
 constexpr int kPix = kRows * kCols;          // 360
@@ -87,31 +91,32 @@ struct C8Args {
     int32_t dbuf;               // 1: two accumulator pairs (double-buffered units)
 };
 
-__device__ __forceinline__ float c8_silu(float v)
+// SiLU of two values from their halves u = v / 2: v sigmoid(v) =
+// u + u tanh(u), both tanh in one tanh.approx.f16x2 (u rounded to f16, the
+// tanh's absolute error about 2^-11), the rest in f32.
+__device__ __forceinline__ uint32_t c8_silu2(float ua, float ub)
 {
-    float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * v));
-    return v * __fmaf_rn(0.5f, t, 0.5f);
+    uint32_t h, t;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(ub), "f"(ua));   // ua in the low half
+    asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(h));
+    float ta, tb;
+    asm("{\n .reg .f16 l, h;\n mov.b32 {l, h}, %2;\n cvt.f32.f16 %0, l;\n cvt.f32.f16 %1, h;\n}\n"
+        : "=f"(ta), "=f"(tb) : "r"(t));
+    return pack_bf16x2(__fmaf_rn(ua, ta, ua), __fmaf_rn(ub, tb, ub));
 }
 
-__device__ __forceinline__ uint4 c8_transform(uint4 in, const float (&sc)[8], const float (&sh)[8], bool affine,
-                                              int silu)
+// GroupNorm affine (sc, sh; identity when absent) and SiLU of 8 bf16
+// channels.  With SiLU the affine arrives pre-halved (u = v / 2).
+__device__ __forceinline__ uint4 c8_transform(uint4 in, const float (&sc)[8], const float (&sh)[8], int silu)
 {
     uint4 out;
     uint32_t *o = reinterpret_cast<uint32_t *>(&out);
     const uint32_t *w = reinterpret_cast<const uint32_t *>(&in);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        float a = bf16_lo(w[q]), b = bf16_hi(w[q]);
-        if (affine) {
-            a = __fmaf_rn(a, sc[2 * q], sh[2 * q]);
-            b = __fmaf_rn(b, sc[2 * q + 1], sh[2 * q + 1]);
-        }
-        if (silu) {
-            a = c8_silu(a);
-            b = c8_silu(b);
-        }
-        o[q] = pack_bf16x2(a, b);
+        const float a = __fmaf_rn(bf16_lo(w[q]), sc[2 * q], sh[2 * q]);
+        const float b = __fmaf_rn(bf16_hi(w[q]), sc[2 * q + 1], sh[2 * q + 1]);
+        o[q] = silu ? c8_silu2(a, b) : pack_bf16x2(a, b);
     }
     return out;
 }
@@ -309,8 +314,9 @@ __global__ void __launch_bounds__(c8::kThreads, 1)
         // go out before the wait for it
         const int per_unit = kch * 9;
         const int pre = min(S, per_unit);
+        const int rot = (int)(blockIdx.x % 9);          // first tap of every chunk
         for (int j = 0; j < pre && ok; ++j)
-            ok = issue(j / 9, j % 9);
+            ok = issue(j / 9, (j % 9 + rot) % 9);
         pdl_wait();
         const int units = p.dense ? ((p.th + 3) / 4) * p.tw * p.N : (min(__ldg(p.count), p.cap) * p.N + 1) / 2;
         bool first = true;
@@ -318,7 +324,7 @@ __global__ void __launch_bounds__(c8::kThreads, 1)
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
 #pragma unroll 1
             for (int j = first ? pre : 0; j < per_unit && ok; ++j)
-                ok = issue(j / 9, j % 9);
+                ok = issue(j / 9, (j % 9 + rot) % 9);
             first = false;
         }
 #pragma unroll 1
@@ -341,6 +347,7 @@ __global__ void __launch_bounds__(c8::kThreads, 1)
         const uint64_t a_step = (2 * kKc) >> 4;
         // accumulator 1's A rows: 16 halo rows on in a strip, 18 for a tile pair
         const uint64_t a1_off = (uint64_t)(((p.dense ? 16 : 18) * kCols * 16) >> 4);
+        const int rot = (int)(blockIdx.x % 9);          // the weight producer's tap order
         int s = 0;
         uint32_t ph = 0, ait = 0, qit = 0;
         bool ok = true;
@@ -375,7 +382,8 @@ __global__ void __launch_bounds__(c8::kThreads, 1)
                 const uint32_t abase = sb + kOffA + (uint32_t)ab * kABuf;
 #pragma unroll 1
                 for (int tap = 0; tap < 9; ++tap) {
-                    const int r = tap / 3, c = tap - r * 3;
+                    const int tr = tap + rot < 9 ? tap + rot : tap + rot - 9;
+                    const int r = tr / 3, c = tr - r * 3;
                     if (!mbar_wait_w(w_full(s), ph, abort_flag, hdr, kSiteWFull)) {
                         ok = false;
                         break;
@@ -410,10 +418,11 @@ __global__ void __launch_bounds__(c8::kThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp < 6) {
+    } else if (warp < 10) {
         // ------------------------------------------------ halo: TMA + transform
-        const int ht = threadIdx.x - 64;                 // 0..127
-        const int kcl = ht & 7, pq = ht >> 3;            // channel group; pixel phase 0..15
+        const int ht = threadIdx.x - 64;                 // 0..255
+        const int kcl = ht & 7, pq = ht >> 3;            // channel group; pixel phase 0..31
+        constexpr int kPhases = kHaloT / 8;
         pdl_wait();
         const int units = p.dense ? ((p.th + 3) / 4) * p.tw * p.N : (min(__ldg(p.count), p.cap) * p.N + 1) / 2;
         const bool affine = p.gsc != nullptr;
@@ -444,14 +453,16 @@ __global__ void __launch_bounds__(c8::kThreads, 1)
                     pending = true;
                 }
                 // GroupNorm parameters of this thread's 8 channels, per item
+                // (halved for the SiLU's u = v / 2)
                 float sc0[8], sh0[8], sc1[8], sh1[8];
                 const int ch = q * 64 + kcl * 8;
+                const float hs = p.silu ? 0.5f : 1.0f;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    sc0[e] = affine ? __ldg(p.gsc + (int64_t)g.n0 * p.Cin + ch + e) : 1.0f;
-                    sh0[e] = affine ? __ldg(p.gsh + (int64_t)g.n0 * p.Cin + ch + e) : 0.0f;
-                    sc1[e] = affine ? __ldg(p.gsc + (int64_t)g.n1 * p.Cin + ch + e) : 1.0f;
-                    sh1[e] = affine ? __ldg(p.gsh + (int64_t)g.n1 * p.Cin + ch + e) : 0.0f;
+                    sc0[e] = hs * (affine ? __ldg(p.gsc + (int64_t)g.n0 * p.Cin + ch + e) : 1.0f);
+                    sh0[e] = hs * (affine ? __ldg(p.gsh + (int64_t)g.n0 * p.Cin + ch + e) : 0.0f);
+                    sc1[e] = hs * (affine ? __ldg(p.gsc + (int64_t)g.n1 * p.Cin + ch + e) : 1.0f);
+                    sh1[e] = hs * (affine ? __ldg(p.gsh + (int64_t)g.n1 * p.Cin + ch + e) : 0.0f);
                 }
                 // the A buffer is free (the MMAs of the chunk before last read it)
                 const int ab = (int)(qit & 1);
@@ -479,7 +490,7 @@ __global__ void __launch_bounds__(c8::kThreads, 1)
                     const int row_off = second ? 18 : 0;
                     const int oy = (second ? g.y1 : g.y0) - 1, ox = (second ? g.x1 : g.x0) - 1;
 #pragma unroll 1
-                    for (int i = pq; i < npx; i += 16) {
+                    for (int i = pq; i < npx; i += kPhases) {
                         const int hr = i / kCols, hc = i - hr * kCols;
                         const int Y = oy + hr, X = ox + hc;
                         const int px = (row_off + hr) * kCols + hc;
@@ -487,8 +498,7 @@ __global__ void __launch_bounds__(c8::kThreads, 1)
                         if (Y >= 0 && Y < p.H && X >= 0 && X < p.W) {
                             v = *reinterpret_cast<const uint4 *>(stg + px * 128);
                             if (affine || p.silu)
-                                v = second ? c8_transform(v, sc1, sh1, affine, p.silu)
-                                           : c8_transform(v, sc0, sh0, affine, p.silu);
+                                v = second ? c8_transform(v, sc1, sh1, p.silu) : c8_transform(v, sc0, sh0, p.silu);
                         }
                         *reinterpret_cast<uint4 *>(dst + px * 16) = v;
                     }
@@ -528,7 +538,7 @@ __global__ void __launch_bounds__(c8::kThreads, 1)
                 const int rows = a ? g.rows1 : g.rows0;
                 const int n = a ? g.n1 : g.n0;
                 const int Y = (a ? g.y1 : g.y0) + oi, X = (a ? g.x1 : g.x0) + oj;
-                const bool valid = rows > 0 && oi < (p.dense ? 16 : 8) && oi < rows && X < p.W;
+                const bool valid = rows > 0 && oi < (p.dense ? 16 : 8) && oi < rows && Y >= 0 && X >= 0 && X < p.W;
                 const int64_t e = ((((int64_t)n * p.H + Y) * p.W + X) * p.Cout);
                 const uint32_t tcol = (uint32_t)((buf * 2 + a) * NC);
                 // both accumulators of a strip exist; a tile pair may have one
@@ -545,10 +555,13 @@ __global__ void __launch_bounds__(c8::kThreads, 1)
                                                   : nullptr;
 #pragma unroll
                     for (int g8 = 0; g8 < 4; ++g8) {
-                        float bb[8];
-#pragma unroll
-                        for (int t = 0; t < 8; ++t)
-                            bb[t] = p.bias ? __ldg(p.bias + c0 + 8 * g8 + t) : 0.0f;
+                        float bb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        if (p.bias) {
+                            const float4 b0 = __ldg(reinterpret_cast<const float4 *>(p.bias + c0 + 8 * g8));
+                            const float4 b1 = __ldg(reinterpret_cast<const float4 *>(p.bias + c0 + 8 * g8 + 4));
+                            bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w;
+                            bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
+                        }
                         uint4 rr = res ? __ldg(res + g8) : make_uint4(0, 0, 0, 0);
                         const uint32_t *rw = reinterpret_cast<const uint32_t *>(&rr);
                         uint32_t o[4];
@@ -581,7 +594,7 @@ __global__ void __launch_bounds__(c8::kThreads, 1)
 bool conv8_supported(const sige_conv_desc *cd, int dtype)
 {
     return cd && dtype == SIGE_BF16 && cd->kernel == 3 && cd->stride == 1 && cd->pad == 1 && cd->block == 8 &&
-           cd->c_in >= 64 && cd->c_in % 64 == 0 && cd->c_out >= 16 && cd->c_out <= c8::kMaxN && cd->c_out % 16 == 0;
+           cd->c_in >= 64 && cd->c_in % 64 == 0 && cd->c_out >= 32 && cd->c_out <= c8::kMaxN && cd->c_out % 32 == 0;
 }
 
 static bool c8_encode_halo(CUtensorMap *map, const void *x, int N, int H, int W, int C, int rows,

@@ -68,9 +68,11 @@ constexpr uint32_t kXHalf = 8 * kXKc;      // 64 channels of the conv1 input
 constexpr uint32_t kSHalf = kXPix * 128;   // 64 channels of the raw halo (the TMA box holds both, pixel-major)
 constexpr int kYE = 10;                    // conv2 input edge (tile + 1-pixel ring)
 constexpr uint32_t kYKc = kYE * kYE * 16;  // bytes of one 8-channel group of the conv2 input
-constexpr uint32_t kWStage = 64 * 64 * 2;  // 64 output channels x 64 K, bf16
-constexpr int kStages = 15;                // weight ring
-constexpr int kChunks = 18;                // weight stages per conv: 2 channel chunks x 9 taps
+constexpr uint32_t kWTap = 64 * 64 * 2;    // one tap: 64 output channels x 64 K, bf16
+constexpr int kTapsPerStage = 3;           // one kernel row: a weight stage is ONE TMA of 24 KB
+constexpr uint32_t kWStage = kTapsPerStage * kWTap;
+constexpr int kStages = 5;                 // weight ring
+constexpr int kChunks = 6;                 // weight stages per conv: 2 channel halves x 3 kernel rows
 constexpr uint32_t kOffX = 1024;
 constexpr uint32_t kOffS = kOffX + 16 * kXKc;                       // raw halo, two halves
 constexpr uint32_t kOffY = kOffS + 2 * kSHalf;
@@ -87,10 +89,20 @@ constexpr uint32_t kBarY1tFull = 384, kBarY1tEmpty = 392, kBarDrain = 400, kBarY
 constexpr uint32_t kTmemSlot = 416, kAbort = 420, kUnits = 448;   // kUnits: the step's unit table (int2)
 constexpr int kMaxUnits = 64;              // units one CTA pair takes in the step (tile origins at kUnits)
 constexpr int kMaxTiles = 16384;           // tile grid of the step's mask (flags staged in the halo buffer)
+// the step's difference stream: a ring of kRing slots, each a chunk of x_orig
+// and the same chunk of x_edit (kRingVec 16-byte vectors each), filled by
+// bulk copies in the halo / conv2-input region before the first halo
+constexpr int kRing = 2;
+constexpr int kRingVec = 1536;
+constexpr uint32_t kRingBytes = kRingVec * 16;
+constexpr uint32_t kOffRing = kOffX;
+constexpr uint32_t kBarRingFull = 960, kBarRingEmpty = 992;
+static_assert(kOffRing + 2 * kRing * kRingBytes <= kOffW && kRingVec % 256 == 0, "ring");
+static_assert(kUnits + 8 * kMaxUnits <= kBarRingFull, "control words");
 
 // wait sites recorded in the error detail on a timeout
 enum : int { kSiteWEmpty = 101, kSiteWFull, kSiteXReady, kSiteAcc1Empty, kSiteAcc2Empty, kSiteY1tFull,
-             kSiteXFull, kSiteAcc1Full, kSiteY1tEmpty, kSiteAcc2Full, kSiteGrid, kSiteY1tLocal };
+             kSiteXFull, kSiteAcc1Full, kSiteY1tEmpty, kSiteAcc2Full, kSiteGrid, kSiteY1tLocal, kSiteRing };
 
 }  // namespace rb
 
@@ -136,6 +148,35 @@ __device__ __forceinline__ void rb_mma4(uint32_t d_tmem, uint64_t a_desc, uint64
         : "memory");
 }
 
+// Four K=16 MMAs (A advances by a_step, B by 32 bytes), no commit.
+__device__ __forceinline__ void rb_mma4_nc(uint32_t d_tmem, uint64_t a_desc, uint64_t a_step, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n .reg .pred p, e, t;\n .reg .b32 l;\n .reg .b64 a1, a2, a3, b1, b2, b3;\n"
+        " elect.sync l|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n setp.eq.b32 t, 0, 0;\n"
+        " add.s64 a1, %1, %5;\n add.s64 a2, a1, %5;\n add.s64 a3, a2, %5;\n"
+        " add.s64 b1, %2, 2;\n add.s64 b2, %2, 4;\n add.s64 b3, %2, 6;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, t;\n}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "l"(a_step)
+        : "memory");
+}
+
+// expect_tx on `bar` and one 4-d tile load completing on it, from one lane.
+__device__ __forceinline__ void rb_tma4_w(uint32_t dst, const CUtensorMap *map, uint32_t bar, uint32_t bytes, int c0,
+                                          int c1, int c2, int c3)
+{
+    asm volatile(
+        "{\n .reg .pred e;\n .reg .b32 l;\n elect.sync l|e, 0xffffffff;\n"
+        " @e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%2], %3;\n"
+        " @e cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%4, %5, %6, %7}], [%2];\n}\n"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(bytes), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
 // Commit that arrives on the mbarrier at offset `bar` of both CTAs of the pair.
 __device__ __forceinline__ void rb_commit_pair(uint32_t bar)
 {
@@ -163,19 +204,24 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
         v[k] = __uint_as_float(r[k]);
 }
 
-// SiLU v * sigmoid(v) with sigmoid(v) = (1 + tanh(v / 2)) / 2: one special-
-// function instruction per element (tanh.approx.f32, absolute error of the
-// tanh about 2^-11) instead of an exponential and a division, which halves
-// the work of the special-function units that bound the halo transform and
-// epilogue 1; the value is rounded to bf16 (8 significant bits) right after.
-__device__ __forceinline__ float rb_silu(float v)
+// SiLU of two values from their halves u = v / 2 (the GroupNorm affine is
+// pre-scaled by 1/2): v sigmoid(v) = v (1 + tanh(v / 2)) / 2 = u + u tanh(u).
+// Both tanh in one special-function instruction (tanh.approx.f16x2; u rounded
+// to f16 first, the tanh's absolute error about 2^-11, like the f32 form), the
+// rest in f32, one rounding to bf16 at the end.  The special-function units
+// bound the halo transform and epilogue 1; this halves their work.
+__device__ __forceinline__ uint32_t rb_silu2(float ua, float ub)
 {
-    float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * v));
-    return v * __fmaf_rn(0.5f, t, 0.5f);
+    uint32_t h, t;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(ub), "f"(ua));   // ua in the low half
+    asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(h));
+    float ta, tb;
+    asm("{\n .reg .f16 l, h;\n mov.b32 {l, h}, %2;\n cvt.f32.f16 %0, l;\n cvt.f32.f16 %1, h;\n}\n"
+        : "=f"(ta), "=f"(tb) : "r"(t));
+    return pack_bf16x2(__fmaf_rn(ua, ta, ua), __fmaf_rn(ub, tb, ub));
 }
 
-// GroupNorm affine + SiLU of 8 bf16 channels (parameters in registers).
+// GroupNorm affine (pre-halved, in registers) + SiLU of 8 bf16 channels.
 __device__ __forceinline__ uint4 rb_gn_silu16(uint4 in, const float (&sc)[8], const float (&sh)[8])
 {
     uint4 out;
@@ -183,8 +229,8 @@ __device__ __forceinline__ uint4 rb_gn_silu16(uint4 in, const float (&sc)[8], co
     const uint32_t *w = reinterpret_cast<const uint32_t *>(&in);
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-        o[q] = pack_bf16x2(rb_silu(__fmaf_rn(bf16_lo(w[q]), sc[2 * q], sh[2 * q])),
-                           rb_silu(__fmaf_rn(bf16_hi(w[q]), sc[2 * q + 1], sh[2 * q + 1])));
+        o[q] = rb_silu2(__fmaf_rn(bf16_lo(w[q]), sc[2 * q], sh[2 * q]),
+                        __fmaf_rn(bf16_hi(w[q]), sc[2 * q + 1], sh[2 * q + 1]));
     return out;
 }
 
@@ -223,6 +269,24 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *ptr)
     return v;
 }
 
+// Bits 0..7 of x to bits 0, 4, .., 28.
+__device__ __forceinline__ uint32_t rb_spread4(uint32_t x)
+{
+    x &= 0xFFu;
+    x = (x | (x << 12)) & 0x000F000Fu;
+    x = (x | (x << 6)) & 0x03030303u;
+    return (x | (x << 3)) & 0x11111111u;
+}
+
+// Bulk copy of `bytes` (a multiple of 16) from global memory into this CTA's
+// shared memory, completing on the mbarrier `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
 // Some bf16 of 16 bytes differ by more than thr (the difference taken in float32).
 __device__ __forceinline__ bool rb_exceeds(uint4 a, uint4 b, float thr)
 {
@@ -237,23 +301,27 @@ __device__ __forceinline__ bool rb_exceeds(uint4 a, uint4 b, float thr)
 // Phases of the one-launch step before the res block (mer.dev notes on SIGE,
 // sections 3 and 3.2: difference mask, dilation, tile selection; SIGE project
 // page, "Overview": active block indices):
-//   A. warps 1-9 of every CTA stream this CTA's contiguous share of x_orig and
-//      x_edit (16-byte loads, eight in flight per input and thread) while warp
-//      0 issues the first weight stages; a pixel some channel of which differs
-//      by more than thr marks its 8x8 tile: the tile's 32-bit flag is set to
-//      this call's epoch;
+//   A. every CTA streams its contiguous share of x_orig and x_edit through a
+//      ring of kRing shared-memory slots: one lane of warp 1 fills a slot with
+//      two bulk copies (the same kRingVec 16-byte vectors of both inputs),
+//      warps 2-9 compare it and release it, while warp 0 issues the first
+//      weight stages; a pixel some channel of which differs by more than thr
+//      marks its 8x8 tile: the tile's 32-bit flag is set to this call's epoch;
 //   B. grid barrier (bounded): every CTA adds one arrival to a 64-bit counter
 //      in the workspace header that only grows, and waits until it reaches
 //      (generation + 1) * CTAs;
-//   C. every CTA reads the flags once (16-byte loads), takes as active the
-//      tiles whose flag equals the epoch, dilates by `dilate` tiles (clipped),
-//      and compacts them in row-major order -- every CTA computes the same
-//      list; CTA 0 writes it and its count out, each pair keeps the origins of
-//      its own units (u = pair + j * npairs, tile u / N).
+//   C. every CTA reads the flags once (16-byte loads) into a bitmap (one
+//      ballot per flag position), takes as active the tiles whose flag equals
+//      the epoch, dilates by `dilate` tiles (clipped) on 64-bit row words, and
+//      compacts them in row-major order -- every CTA computes the same list;
+//      CTA 0 writes it and its count out, each pair finds the origins of its
+//      own units (u = pair + j * npairs, tile u / N) by a binary search of the
+//      row prefix and a bit select.
 // The generation is the counter's value at entry divided by the number of
 // CTAs (every CTA of every call arrives exactly once, so the counter moves by
-// exactly that much per call) and the epoch is generation + 1: flags of
-// earlier calls never equal it, so nothing is cleared between calls.
+// exactly that much per call) and the epoch is the generation modulo
+// 2^32 - 1, plus 1: flags of the last 2^32 - 2 calls never equal it and 0 (a
+// flag never set) never does, so nothing is cleared between calls.
 // Returns the number of units, min(count, cap) * N.
 __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, volatile int *abort_flag, int pair,
                                             int npairs)
@@ -261,57 +329,86 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
     using namespace rb;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int H = p.H, W = p.W, tw = p.tw, nt = p.th * p.tw;
-    volatile uint32_t *s_epoch = reinterpret_cast<volatile uint32_t *>(smem + kAbort + 8);
     volatile int *s_ok = reinterpret_cast<volatile int *>(smem + kAbort + 12);
-    if (tid == 0) {
-        unsigned long long c0;
+    // Every warp reads the counter itself, before this CTA's arrival: fewer
+    // than gridDim.x arrivals of this call can precede the read, so all warps
+    // of all CTAs find the same generation (and no warp waits for another to
+    // start streaming).
+    unsigned long long c0 = 0;
+    if (lane == 0)
         asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(c0) : "l"(p.ctr) : "memory");
-        *s_epoch = (uint32_t)(c0 / gridDim.x) + 1u;
-    }
-    __syncthreads();
-    const uint32_t epoch = *s_epoch;
-    // ---- A: difference mask -> tile flags (warps 1-9)
+    c0 = __shfl_sync(0xFFFFFFFFu, c0, 0);
+    const unsigned long long gen = c0 / gridDim.x;
+    const unsigned long long target = (gen + 1) * gridDim.x;   // the counter value that ends the grid barrier
+    const uint32_t epoch = (uint32_t)(gen % 0xFFFFFFFFull) + 1u; // never 0, the value of an unset flag
+    // ---- A: difference mask -> tile flags
     bool wrote = false;
-    if (wid >= 1) {
-        const int st = tid - 32, nst = kThreads - 32;
+    {
         const int64_t nvec = (int64_t)p.N * H * W * (kC / 8);
         const int64_t per = (nvec + gridDim.x - 1) / gridDim.x;
-        const int64_t v0 = (int64_t)blockIdx.x * per, v1 = min(nvec, v0 + per);
-        int last = -1;
-        // Rolling loads: slot k holds vector base + k * nst; right after it is
-        // compared, the slot is refilled with the vector one round later, so
-        // the memory system always has about eight loads per input and thread
-        // in flight instead of draining between rounds.
-        uint4 a[8], b[8];
-        const uint4 *xo4 = reinterpret_cast<const uint4 *>(p.xo), *xe4 = reinterpret_cast<const uint4 *>(p.x);
-        const uint4 z4 = make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int64_t v = v0 + st + (int64_t)k * nst;
-            a[k] = v < v1 ? __ldg(xo4 + v) : z4;
-            b[k] = v < v1 ? __ldg(xe4 + v) : z4;
-        }
-#pragma unroll 1
-        for (int64_t base = v0 + st; base < v1; base += 8 * nst) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int64_t v = base + (int64_t)k * nst;
-                const bool differs = ((a[k].x ^ b[k].x) | (a[k].y ^ b[k].y) | (a[k].z ^ b[k].z) | (a[k].w ^ b[k].w)) &&
-                                     rb_exceeds(a[k], b[k], p.thr);
-                const int64_t vn = v + 8 * (int64_t)nst;
-                a[k] = vn < v1 ? __ldg(xo4 + vn) : z4;
-                b[k] = vn < v1 ? __ldg(xe4 + vn) : z4;
-                if (differs) {
-                    const int64_t pix = v >> 4;   // 16 vectors per pixel
-                    const int64_t hw = pix % ((int64_t)H * W);
-                    const int y = (int)(hw / W), x = (int)(hw - (int64_t)y * W);
-                    const int t = (y >> 3) * tw + (x >> 3);
-                    if (t != last) {
-                        p.flags[t] = epoch;
-                        last = t;
-                        wrote = true;
+        const int64_t v0 = min(nvec, (int64_t)blockIdx.x * per), v1 = min(nvec, v0 + per);
+        const int nchunks = (int)((v1 - v0 + kRingVec - 1) / kRingVec);
+        const uint32_t sb = smem_u32(smem);
+        auto ring_full = [&](int i) { return sb + kBarRingFull + 8u * i; };
+        auto ring_empty = [&](int i) { return sb + kBarRingEmpty + 8u * i; };
+        if (wid == 1) {
+            // one lane fills the ring: per slot, the chunk of both inputs
+            if (lane == 0) {
+                int issued = 0;
+                for (int c = 0; c < nchunks; ++c) {
+                    const int sl = c % kRing;
+                    if (c >= kRing && !mbar_wait(ring_empty(sl), (uint32_t)((c / kRing) - 1) & 1u, abort_flag, p.hdr,
+                                                 kSiteRing))
+                        break;
+                    const int64_t a = v0 + (int64_t)c * kRingVec;
+                    const uint32_t bytes = (uint32_t)min((int64_t)kRingVec, v1 - a) * 16u;
+                    const uint32_t dst = sb + kOffRing + (uint32_t)sl * 2u * kRingBytes;
+                    mbar_expect_tx(ring_full(sl), 2u * bytes);
+                    bulk_load(dst, p.xo + a * 16, bytes, ring_full(sl));
+                    bulk_load(dst + kRingBytes, p.x + a * 16, bytes, ring_full(sl));
+                    ++issued;
+                }
+                // every copy lands before the region is reused (bounded)
+                for (int c = max(0, issued - kRing); c < issued; ++c) {
+                    const long long t0 = clock64();
+                    while (!mbar_try(ring_full(c % kRing), (uint32_t)(c / kRing) & 1u) && clock64() - t0 < kWaitCycles) {
                     }
                 }
+            }
+            __syncwarp();
+        } else if (wid >= 2) {
+            // warps 2-9 compare; a warp releases a slot once its lanes read it
+            const int ct = tid - 64;
+            int last = -1;
+            for (int c = 0; c < nchunks; ++c) {
+                const int sl = c % kRing;
+                if (!mbar_wait_w(ring_full(sl), (uint32_t)(c / kRing) & 1u, abort_flag, p.hdr, kSiteRing))
+                    break;
+                const int64_t a = v0 + (int64_t)c * kRingVec;
+                const int n = (int)min((int64_t)kRingVec, v1 - a);
+                const uint4 *so = reinterpret_cast<const uint4 *>(smem + kOffRing + (uint32_t)sl * 2u * kRingBytes);
+                const uint4 *se = so + kRingVec;
+#pragma unroll
+                for (int k = 0; k < kRingVec / kEpi; ++k) {
+                    const int i = k * kEpi + ct;
+                    if (i < n) {
+                        const uint4 va = so[i], vb = se[i];
+                        if (((va.x ^ vb.x) | (va.y ^ vb.y) | (va.z ^ vb.z) | (va.w ^ vb.w)) && rb_exceeds(va, vb, p.thr)) {
+                            const int64_t pix = (a + i) >> 4;   // 16 vectors per pixel
+                            const int64_t hw = pix % ((int64_t)H * W);
+                            const int y = (int)(hw / W), x = (int)(hw - (int64_t)y * W);
+                            const int t = (y >> 3) * tw + (x >> 3);
+                            if (t != last) {
+                                p.flags[t] = epoch;
+                                last = t;
+                                wrote = true;
+                            }
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(ring_empty(sl));
             }
         }
     }
@@ -321,7 +418,6 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
     if (tid == 0) {
         if (any)
             __threadfence();
-        const unsigned long long target = (unsigned long long)epoch * gridDim.x;
         atomicAdd(p.ctr, 1ull);
         const long long t0 = clock64();
         int ok = 1;
@@ -341,19 +437,11 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
     }
     __syncthreads();
     const bool ok = *s_ok != 0;
-    // ---- C: flags -> shared (one round of 16-byte loads), dilate, compact
-    uint8_t *s_flag = smem + kOffX;                 // halo buffer, unused until the first halo
+    // ---- C: flags -> bits, dilate, compact
+    uint8_t *s_flag = smem + kOffX;                 // ring / halo region, unused until the first halo
     uint8_t *s_act = s_flag + kMaxTiles;
     int *s_wsum = reinterpret_cast<int *>(smem + kOffY);
     int2 *s_units = reinterpret_cast<int2 *>(smem + kUnits);
-    for (int i = tid * 4; i < nt; i += kThreads * 4) {
-        const uint4 f = ok ? __ldcg(reinterpret_cast<const uint4 *>(p.flags + i)) : make_uint4(0, 0, 0, 0);
-        s_flag[i] = f.x == epoch;
-        s_flag[i + 1] = f.y == epoch;
-        s_flag[i + 2] = f.z == epoch;
-        s_flag[i + 3] = f.w == epoch;
-    }
-    __syncthreads();
     const int D = p.dilate;
     int total = 0, n_list = 0;
     if (p.th <= 64 && tw <= 64) {
@@ -361,6 +449,25 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
         // shuffles across rows) and counts; rows y and y + 32 sit in lane y
         uint64_t *s_row = reinterpret_cast<uint64_t *>(smem + kOffY);      // [64] dilated rows
         int *s_pre = reinterpret_cast<int *>(smem + kOffY + 512);          // [65] row prefix, [64] = total
+        uint32_t *s_bits = reinterpret_cast<uint32_t *>(smem + kOffY + 1024);   // [128] flags, 32 tiles a word
+        // One round of 16-byte loads: a warp reads 128 consecutive flags (4 a
+        // lane) and four ballots (one per position in the vector) give the
+        // four bitmap words of that range.
+        const int nwords = (nt + 31) >> 5;
+        for (int base = wid * 128; base < nt; base += kThreads * 4) {
+            const int i = base + 4 * lane;
+            const uint4 f = (ok && i < nt) ? __ldcg(reinterpret_cast<const uint4 *>(p.flags + i))
+                                           : make_uint4(0, 0, 0, 0);
+            const uint32_t b0 = __ballot_sync(0xFFFFFFFFu, f.x == epoch), b1 = __ballot_sync(0xFFFFFFFFu, f.y == epoch);
+            const uint32_t b2 = __ballot_sync(0xFFFFFFFFu, f.z == epoch), b3 = __ballot_sync(0xFFFFFFFFu, f.w == epoch);
+            if (lane < 4) {
+                // flag base + 32 lane + 4 m + k is bit 8 lane + m of ballot k
+                const int sh = 8 * lane;
+                s_bits[(base >> 5) + lane] = rb_spread4(b0 >> sh) | (rb_spread4(b1 >> sh) << 1) |
+                                             (rb_spread4(b2 >> sh) << 2) | (rb_spread4(b3 >> sh) << 3);
+            }
+        }
+        __syncthreads();
         if (wid == 0) {
             const uint64_t full = tw == 64 ? ~0ull : ((1ull << tw) - 1);
             uint64_t h[2];
@@ -368,9 +475,13 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
             for (int r = 0; r < 2; ++r) {
                 const int y = lane + 32 * r;
                 uint64_t m = 0;
-                if (y < p.th)
-                    for (int x = 0; x < tw; ++x)
-                        m |= (uint64_t)s_flag[y * tw + x] << x;
+                if (y < p.th) {
+                    // bits [y tw, y tw + tw) of the bitmap
+                    const int st = y * tw, w0 = st >> 5, sh = st & 31;
+                    const uint64_t lo = (uint64_t)s_bits[w0] | ((uint64_t)(w0 + 1 < nwords ? s_bits[w0 + 1] : 0u) << 32);
+                    const uint64_t hi = w0 + 2 < nwords ? s_bits[w0 + 2] : 0u;
+                    m = ((lo >> sh) | (sh ? hi << (64 - sh) : 0ull)) & full;
+                }
                 uint64_t hd = m;
                 for (int k = 1; k <= D && k < 64; ++k)
                     hd |= (m << k) | (m >> k);
@@ -431,18 +542,41 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
             const int u = pair + tid * npairs;
             if (u < n_list * p.N) {
                 const int pos = u / p.N;
-                int y = 0;
-                while (y + 1 < p.th && s_pre[y + 1] <= pos)
-                    ++y;
-                uint64_t m = s_row[y];
-                for (int r = pos - s_pre[y]; r > 0; --r)
-                    m &= m - 1;
-                const int x = __ffsll((long long)m) - 1;
-                s_units[tid] = make_int2(y * kB, x * kB);
+                // the last row whose prefix is <= pos, then the (pos - prefix)-th
+                // set bit of that row
+                int lo = 0, hi = p.th - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (s_pre[mid] <= pos)
+                        lo = mid;
+                    else
+                        hi = mid - 1;
+                }
+                uint64_t m = s_row[lo];
+                int r = pos - s_pre[lo], x = 0;
+#pragma unroll
+                for (int w = 32; w > 0; w >>= 1) {
+                    const int c = __popcll(m & ((1ull << w) - 1));
+                    if (r >= c) {
+                        r -= c;
+                        m >>= w;
+                        x += w;
+                    }
+                }
+                s_units[tid] = make_int2(lo * kB, x * kB);
             }
         }
     } else {
-        // larger grids: one pass per thread over a contiguous run of tiles
+        // larger grids: flags to bytes, then one pass per thread over a
+        // contiguous run of tiles
+        for (int i = tid * 4; i < nt; i += kThreads * 4) {
+            const uint4 f = ok ? __ldcg(reinterpret_cast<const uint4 *>(p.flags + i)) : make_uint4(0, 0, 0, 0);
+            s_flag[i] = f.x == epoch;
+            s_flag[i + 1] = f.y == epoch;
+            s_flag[i + 2] = f.z == epoch;
+            s_flag[i + 3] = f.w == epoch;
+        }
+        __syncthreads();
         const int seg = (nt + kThreads - 1) / kThreads;
         const int t0 = min(nt, tid * seg), t1 = min(nt, t0 + seg);
         int cnt = 0;
@@ -543,6 +677,12 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
         mbar_init(y1t_empty, 2);         // the conv2 commits of both CTAs
         mbar_init(y1t_local, kEpi);      // every epilogue thread has written its part of this CTA's half
         mbar_init(drain, 1);
+        if constexpr (kStep) {
+            for (int i = 0; i < kRing; ++i) {
+                mbar_init(sb + kBarRingFull + 8u * i, 1);
+                mbar_init(sb + kBarRingEmpty + 8u * i, kEpi / 32);   // one arrival per comparing warp
+            }
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -575,12 +715,14 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
     uint32_t ph = 1;
     bool ok = true;
     const int pre = kStages < kChunks ? kStages : kChunks;
+    // stage j of a conv: channel half j / 3, kernel row j % 3 (its three
+    // taps), this CTA's 64 output channels: one 24 KB box
     auto issue = [&](int conv, int j) -> bool {
             if (!mbar_wait_w(w_empty(s), ph, abort_flag, hdr, kSiteWEmpty))
                 return false;
-            const int kc2 = j / 9, tap = j - kc2 * 9;
-            tma_load_2d_w(sb + kOffW + (uint32_t)s * kWStage, conv ? &tw2 : &tw1, w_full(s), kWStage,
-                          tap * kC + kc2 * 64, (int)rank * 64);
+            const int half = j / 3, row = j - half * 3;
+            rb_tma4_w(sb + kOffW + (uint32_t)s * kWStage, conv ? &tw2 : &tw1, w_full(s), kWStage, 0, (int)rank * 64,
+                      row * 3, half);
             ++issued;
             if (++s == kStages) {
                 s = 0;
@@ -651,12 +793,18 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                 }
                 const uint32_t chunk = a_base + (uint32_t)kc2 * 8u * kc_bytes;
 #pragma unroll 1
-                for (int tap = 0; tap < 9; ++tap) {
-                    const int r = tap / 3, c = tap - r * 3;
+                for (int r = 0; r < 3; ++r) {
                     if (!mbar_wait_w(w_full(s), ph, abort_flag, hdr, kSiteWFull))
                         return false;
-                    const uint64_t a_desc = desc_plain(chunk + (uint32_t)(pitch * r + c) * 16u, kc_bytes, 128);
-                    rb_mma4(tmem + d_col, a_desc, a_step, b_cur, idesc, (kc2 | tap) ? 1u : 0u, w_empty(s));
+                    // the kernel row's three taps (r, c): A shifted by pitch r + c
+                    // pixels, B the stage's c-th 8 KB tile
+#pragma unroll
+                    for (int c = 0; c < 3; ++c) {
+                        const uint64_t a_desc = desc_plain(chunk + (uint32_t)(pitch * r + c) * 16u, kc_bytes, 128);
+                        rb_mma4_nc(tmem + d_col, a_desc, a_step, b_cur + (uint64_t)(c * (kWTap >> 4)), idesc,
+                                   (kc2 | r | c) ? 1u : 0u);
+                    }
+                    tc_commit_w(w_empty(s));
                     ++ait;
                     if (++s == kStages) {
                         s = 0;
@@ -762,6 +910,11 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                 gsa[h][4] = s1.x; gsa[h][5] = s1.y; gsa[h][6] = s1.z; gsa[h][7] = s1.w;
                 gha[h][0] = h0v.x; gha[h][1] = h0v.y; gha[h][2] = h0v.z; gha[h][3] = h0v.w;
                 gha[h][4] = h1v.x; gha[h][5] = h1v.y; gha[h][6] = h1v.z; gha[h][7] = h1v.w;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    gsa[h][e] *= 0.5f;
+                    gha[h][e] *= 0.5f;
+                }
             }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -811,8 +964,9 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                     const float4 s4 = __ldg(reinterpret_cast<const float4 *>(p.g2s + n * kC + cb + q));
                     const float4 h4 = __ldg(reinterpret_cast<const float4 *>(p.g2h + n * kC + cb + q));
                     bias[q] = b.x; bias[q + 1] = b.y; bias[q + 2] = b.z; bias[q + 3] = b.w;
-                    gs[q] = s4.x; gs[q + 1] = s4.y; gs[q + 2] = s4.z; gs[q + 3] = s4.w;
-                    gh[q] = h4.x; gh[q + 1] = h4.y; gh[q + 2] = h4.z; gh[q + 3] = h4.w;
+                    // halved for the SiLU's u = v / 2
+                    gs[q] = 0.5f * s4.x; gs[q + 1] = 0.5f * s4.y; gs[q + 2] = 0.5f * s4.z; gs[q + 3] = 0.5f * s4.w;
+                    gh[q] = 0.5f * h4.x; gh[q + 1] = 0.5f * h4.y; gh[q + 2] = 0.5f * h4.z; gh[q + 3] = 0.5f * h4.w;
                 }
                 if (!mbar_wait_w(acc1_full, k & 1, abort_flag, hdr, kSiteAcc1Full)) {
                     ok = false;
@@ -827,7 +981,7 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                     y1p[q] = pack_bf16x2(v[2 * q] + bias[2 * q], v[2 * q + 1] + bias[2 * q + 1]);
                     float a = __fmaf_rn(bf16_lo(y1p[q]), gs[2 * q], gh[2 * q]);
                     float b = __fmaf_rn(bf16_hi(y1p[q]), gs[2 * q + 1], gh[2 * q + 1]);
-                    tp[q] = inimg ? pack_bf16x2(rb_silu(a), rb_silu(b)) : 0u;
+                    tp[q] = inimg ? rb_silu2(a, b) : 0u;
                 }
                 // the accumulator may take the next tile's conv1
                 tc_fence_before();
@@ -950,14 +1104,17 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
 
 // ------------------------------------------------------------------ host
 
+// Weights [c_out][3][3][c_in] as a 4-d map (64 input channels, c_out, tap,
+// channel half) with strides 2304 / 256 / 128 bytes: a box of 64 output
+// channels x 3 taps of one half lands as three 8 KB K-major tiles with the
+// 128-byte swizzle, one TMA per weight stage.
 static bool encode_weights(CUtensorMap *map, const void *w, PFN_cuTensorMapEncodeTiled_v12000 encode)
 {
-    const cuuint64_t K = 9 * rb::kC;
-    cuuint64_t dims[2] = {K, (cuuint64_t)rb::kC};
-    cuuint64_t strides[1] = {K * 2};
-    cuuint32_t box[2] = {64, 64};
-    cuuint32_t es[2] = {1, 1};
-    return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(w), dims, strides, box, es,
+    cuuint64_t dims[4] = {64, (cuuint64_t)rb::kC, 9, 2};
+    cuuint64_t strides[3] = {(cuuint64_t)9 * rb::kC * 2, (cuuint64_t)rb::kC * 2, 128};
+    cuuint32_t box[4] = {64, 64, (cuuint32_t)rb::kTapsPerStage, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(w), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -339,3 +339,44 @@ def test_fused_cuda_core_bf16(orc):
     # C_in = 32 is below the tensor-core kernel's 64-channel chunk
     L = inputs.make_conv_case(28, 24, 24, 32, 32, dtype=torch.bfloat16, block=4, area=0.08, gn=True)
     _fused_vs_oracle(orc, L, _tiles(orc, L), residual=True)
+
+
+# ------------------------------------------------------------------ 3x3 layers on 8x8 tiles
+
+@pytest.mark.parametrize("H,W,ci,co,N,gn,res", [
+    (40, 24, 64, 64, 1, True, False),     # last strip of 8 rows: its second accumulator idles
+    (56, 40, 192, 256, 2, True, True),    # C_out 256: one accumulator pair, three K chunks, batch 2
+    (48, 48, 128, 96, 1, False, False),   # C_out 96, no input transform
+    (30, 26, 64, 32, 2, True, True),      # ragged map, C_out 32
+])
+def test_conv8_dense(orc, H, W, ci, co, N, gn, res):
+    """Every tile of the map: strips of four 8x8 tiles share each weight stage."""
+    L = inputs.make_conv_case(60 + H + co, H, W, ci, co, dtype=torch.bfloat16, block=8, gn=gn, N=N)
+    g, gs, gh = _gn(orc, L)
+    r = random_cache((N, H, W, co), torch.bfloat16, 3) if res else None
+    every = np.array([(h, w) for h in range(0, H, 8) for w in range(0, W, 8)], np.int32)
+    ref = orc.sparse_conv(L.x_orig, L.weight, L.bias, every, torch.zeros((N, H, W, co), dtype=torch.bfloat16),
+                          3, 1, 1, 8, gn=g, silu=gn, residual=r)
+    cd = sige.conv_desc(3, 1, 1, ci, co, 8)
+    y = sige.sige_dense_conv(L.x_orig.to(DEV), L.weight.to(DEV), L.bias.to(DEV), cd, gn_scale=gs, gn_shift=gh,
+                             silu=gn, residual=None if r is None else r.to(DEV))
+    torch.cuda.synchronize()
+    assert_close(y.cpu(), ref, torch.bfloat16)
+
+
+@pytest.mark.parametrize("H,W,ci,co,N,area", [
+    (64, 64, 256, 256, 1, 0.05),          # C_out 256, four K chunks
+    (40, 56, 64, 32, 2, 0.08),            # batch 2: tile pairs across items
+    (24, 24, 128, 160, 1, 0.02),          # C_out 160 (not a power of two)
+])
+def test_conv8_sparse(orc, H, W, ci, co, N, area):
+    L = inputs.make_conv_case(70 + H + co, H, W, ci, co, dtype=torch.bfloat16, block=8, area=area, gn=True, N=N)
+    _fused_vs_oracle(orc, L, _tiles(orc, L), residual=True, seed=4)
+
+
+@pytest.mark.parametrize("ntiles", [1, 3])
+def test_conv8_odd_tile_count(orc, ntiles):
+    """An odd number of listed items: the last unit holds a single tile."""
+    L = inputs.make_conv_case(80 + ntiles, 32, 32, 64, 64, dtype=torch.bfloat16, block=8, gn=True)
+    idx = np.array([(8, 8), (24, 0), (0, 24)][:ntiles], np.int32)
+    _fused_vs_oracle(orc, L, idx, residual=True, seed=6)

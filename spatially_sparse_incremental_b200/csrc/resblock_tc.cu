@@ -77,13 +77,22 @@ constexpr uint32_t kOffX = 1024;
 constexpr uint32_t kOffS = kOffX + 16 * kXKc;                       // raw halo, two halves
 constexpr uint32_t kOffY = kOffS + 2 * kSHalf;
 constexpr uint32_t kOffW = ((kOffY + 16 * kYKc + 1023) / 1024 + 1) * 1024;   // (+1 KB: garbage-row reads of conv2)
-constexpr uint32_t kSmem = kOffW + kStages * kWStage + 1024;   // + alignment of the base
+// Per-unit parameter tables, two buffers (unit k uses buffer k & 1), filled
+// by warp 0 from global memory ahead of the unit; floats: [0, 128) GroupNorm1
+// scale / 2 and [128, 256) shift / 2 (all input channels of the unit's batch
+// item), [256, 320) GroupNorm2 scale / 2 and [320, 384) shift / 2, [384, 448)
+// b1, [448, 512) b2 (this CTA's 64 output channels).  The halving folds the
+// SiLU's u = v / 2 into the affine.
+constexpr uint32_t kOffP = kOffW + kStages * kWStage;
+constexpr uint32_t kParBytes = 512 * 4;
+constexpr uint32_t kSmem = kOffP + 2 * kParBytes + 1024;   // + alignment of the base
 constexpr uint32_t kTmemCols = 128;        // conv1 accumulator [0, 64), conv2 [64, 128)
 static_assert(kSmem <= 232448, "shared memory");
 static_assert(kOffS % 128 == 0 && kSHalf % 128 == 0 && kOffY % 16 == 0, "TMA destinations");
 
 // mbarriers and control words in [0, 1024)
 constexpr uint32_t kBarWFull = 0, kBarWEmpty = 160, kBarXFull = 320, kBarXReady = 336;
+constexpr uint32_t kBarParFull = 40, kBarParEmpty = 56;   // [2] each (after the 5 weight-stage barriers)
 constexpr uint32_t kBarAcc1Full = 352, kBarAcc1Empty = 360, kBarAcc2Full = 368, kBarAcc2Empty = 376;
 constexpr uint32_t kBarY1tFull = 384, kBarY1tEmpty = 392, kBarDrain = 400, kBarY1tLocal = 408;
 constexpr uint32_t kTmemSlot = 416, kAbort = 420, kUnits = 448;   // kUnits: the step's unit table (int2)
@@ -102,7 +111,8 @@ static_assert(kUnits + 8 * kMaxUnits <= kBarRingFull, "control words");
 
 // wait sites recorded in the error detail on a timeout
 enum : int { kSiteWEmpty = 101, kSiteWFull, kSiteXReady, kSiteAcc1Empty, kSiteAcc2Empty, kSiteY1tFull,
-             kSiteXFull, kSiteAcc1Full, kSiteY1tEmpty, kSiteAcc2Full, kSiteGrid, kSiteY1tLocal, kSiteRing };
+             kSiteXFull, kSiteAcc1Full, kSiteY1tEmpty, kSiteAcc2Full, kSiteGrid, kSiteY1tLocal, kSiteRing,
+             kSiteParFull, kSiteParEmpty };
 
 }  // namespace rb
 
@@ -116,6 +126,7 @@ struct RbArgs {
     uint8_t *y1;                // cached y1, updated at the tile interiors
     uint8_t *out;               // cached out, updated at the tiles
     WsHeader *hdr;
+    const uint8_t *w1, *w2;     // the weights (L2 prefetch; the stages come by TMA)
     int32_t N, H, W, cap;
     // the one-launch step: the tile list is made here from x_orig vs x (the
     // list and its count are then outputs: idx / count)
@@ -201,6 +212,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int k = 0; k < 32; ++k)
+        v[k] = __uint_as_float(r[k]);
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8])
+{
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
         v[k] = __uint_as_float(r[k]);
 }
 
@@ -445,10 +468,9 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
     const int D = p.dilate;
     int total = 0, n_list = 0;
     if (p.th <= 64 && tw <= 64) {
-        // rows of tiles as 64-bit words: warp 0 dilates (shifts across a row,
-        // shuffles across rows) and counts; rows y and y + 32 sit in lane y
+        // rows of tiles as 64-bit words (grids of up to 64 x 64 tiles)
         uint64_t *s_row = reinterpret_cast<uint64_t *>(smem + kOffY);      // [64] dilated rows
-        int *s_pre = reinterpret_cast<int *>(smem + kOffY + 512);          // [65] row prefix, [64] = total
+        int *s_pre = reinterpret_cast<int *>(smem + kOffY + 512);          // [65] row prefix, [th] = total
         uint32_t *s_bits = reinterpret_cast<uint32_t *>(smem + kOffY + 1024);   // [128] flags, 32 tiles a word
         // One round of 16-byte loads: a warp reads 128 consecutive flags (4 a
         // lane) and four ballots (one per position in the vector) give the
@@ -468,64 +490,41 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
             }
         }
         __syncthreads();
-        if (wid == 0) {
-            const uint64_t full = tw == 64 ? ~0ull : ((1ull << tw) - 1);
-            uint64_t h[2];
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int y = lane + 32 * r;
-                uint64_t m = 0;
-                if (y < p.th) {
-                    // bits [y tw, y tw + tw) of the bitmap
-                    const int st = y * tw, w0 = st >> 5, sh = st & 31;
-                    const uint64_t lo = (uint64_t)s_bits[w0] | ((uint64_t)(w0 + 1 < nwords ? s_bits[w0 + 1] : 0u) << 32);
-                    const uint64_t hi = w0 + 2 < nwords ? s_bits[w0 + 2] : 0u;
-                    m = ((lo >> sh) | (sh ? hi << (64 - sh) : 0ull)) & full;
-                }
-                uint64_t hd = m;
-                for (int k = 1; k <= D && k < 64; ++k)
-                    hd |= (m << k) | (m >> k);
-                h[r] = hd & full;
-            }
-            uint64_t d[2] = {0, 0};
-            for (int dy = -D; dy <= D; ++dy) {
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const int yy = lane + 32 * r + dy;
-                    const int src = yy & 31;
-                    const uint64_t v0 = __shfl_sync(0xFFFFFFFFu, h[0], src);
-                    const uint64_t v1 = __shfl_sync(0xFFFFFFFFu, h[1], src);
-                    if (yy >= 0 && yy < p.th)
-                        d[r] |= (yy >> 5) ? v1 : v0;
-                }
-            }
-            int c[2];
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                if (lane + 32 * r >= p.th)
-                    d[r] = 0;
-                c[r] = __popcll(d[r]);
-            }
-            // row-order prefix: rows 0..31, then 32..63
-            int run = 0;
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                int incl = c[r];
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-                    if (lane >= o)
-                        incl += v;
-                }
-                s_row[lane + 32 * r] = d[r];
-                s_pre[lane + 32 * r] = run + incl - c[r];
-                run += __shfl_sync(0xFFFFFFFFu, incl, 31);
-            }
-            if (lane == 0)
-                s_pre[64] = run;
+        // Thread y < th: row y of the bitmap, dilated across the row; then the
+        // OR of rows y - D .. y + D and its count; then the exclusive prefix of
+        // the counts (independent loads).  Short dependency chains on many
+        // threads: a chain of shuffles in one warp was measured at several us.
+        uint64_t *s_h = reinterpret_cast<uint64_t *>(smem + kOffY + 1536);   // [64] rows dilated across
+        int *s_cnt = reinterpret_cast<int *>(smem + kOffY + 2048);          // [64] active tiles per row
+        const uint64_t full = tw == 64 ? ~0ull : ((1ull << tw) - 1);
+        if (tid < p.th) {
+            // bits [y tw, y tw + tw) of the bitmap
+            const int st = tid * tw, w0 = st >> 5, sh = st & 31;
+            const uint64_t lo = (uint64_t)s_bits[w0] | ((uint64_t)(w0 + 1 < nwords ? s_bits[w0 + 1] : 0u) << 32);
+            const uint64_t hi = w0 + 2 < nwords ? s_bits[w0 + 2] : 0u;
+            const uint64_t m = ((lo >> sh) | (sh ? hi << (64 - sh) : 0ull)) & full;
+            uint64_t hd = m;
+            for (int k = 1; k <= D && k < 64; ++k)
+                hd |= (m << k) | (m >> k);
+            s_h[tid] = hd & full;
         }
         __syncthreads();
-        total = s_pre[64];
+        if (tid < p.th) {
+            uint64_t d = 0;
+            for (int yy = max(0, tid - D); yy <= min(p.th - 1, tid + D); ++yy)
+                d |= s_h[yy];
+            s_row[tid] = d;
+            s_cnt[tid] = __popcll(d);
+        }
+        __syncthreads();
+        if (tid <= p.th) {
+            int pre = 0;
+            for (int i = 0; i < tid; ++i)
+                pre += s_cnt[i];
+            s_pre[tid] = pre;                                             // s_pre[th]: the total
+        }
+        __syncthreads();
+        total = s_pre[p.th];
         n_list = min(total, p.cap);
         // CTA 0 writes the list: thread y takes row y
         if (blockIdx.x == 0 && tid < p.th) {
@@ -654,6 +653,8 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
     const uint32_t acc2_full = sb + kBarAcc2Full, acc2_empty = sb + kBarAcc2Empty;
     const uint32_t y1t_full = sb + kBarY1tFull, y1t_empty = sb + kBarY1tEmpty, drain = sb + kBarDrain;
     const uint32_t y1t_local = sb + kBarY1tLocal;
+    auto par_full = [&](int b) { return sb + kBarParFull + 8u * b; };
+    auto par_empty = [&](int b) { return sb + kBarParEmpty + 8u * b; };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kAbort);
     WsHeader *hdr = p.hdr;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -677,6 +678,10 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
         mbar_init(y1t_empty, 2);         // the conv2 commits of both CTAs
         mbar_init(y1t_local, kEpi);      // every epilogue thread has written its part of this CTA's half
         mbar_init(drain, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(par_full(b), 1);
+            mbar_init(par_empty(b), kEpi);
+        }
         if constexpr (kStep) {
             for (int i = 0; i < kRing; ++i) {
                 mbar_init(sb + kBarRingFull + 8u * i, 1);
@@ -733,8 +738,51 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
     if (warp == 0) {
         for (int j = 0; j < pre && ok; ++j)
             ok = issue(0, j);
+    } else if (warp == 1 && lane == 0) {
+        // Both weight tensors into the L2 (4 KB slices over the grid): every
+        // CTA with a tile reads all of them, the first reads of a line after
+        // a cold start would otherwise each wait for the DRAM.
+        constexpr int kSlice = 4096, kSlices = (int)(9 * kC * kC * 2 / kSlice);   // per tensor
+        for (int q = (int)blockIdx.x; q < 2 * kSlices; q += (int)gridDim.x) {
+            const uint8_t *src = (q < kSlices ? p.w1 : p.w2) + (size_t)(q % kSlices) * kSlice;
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
+                         "r"(kSlice) : "memory");
+        }
     }
     pdl_wait();
+    // Parameter table of this pair's unit k (batch item (pair + k npairs) mod
+    // N) into buffer k & 1, by warp 0; the first one (two for a batch) while
+    // the difference streams / the list is read.
+    auto load_params = [&](int k) {
+        const int n = (pair + k * npairs) % p.N;
+        float *tab = reinterpret_cast<float *>(smem + kOffP + (uint32_t)(k & 1) * kParBytes);
+        const int c_half = (int)rank * 64;
+        for (int i = lane; i < 128; i += 32) {
+            const int f = 4 * i;
+            float4 v;
+            if (f < 256) {
+                const float *src = (f < 128 ? p.g1s : p.g1h) + n * kC + (f & 127);
+                v = __ldg(reinterpret_cast<const float4 *>(src));
+                v = make_float4(0.5f * v.x, 0.5f * v.y, 0.5f * v.z, 0.5f * v.w);
+            } else if (f < 384) {
+                const float *src = (f < 320 ? p.g2s : p.g2h) + n * kC + c_half + (f & 63);
+                v = __ldg(reinterpret_cast<const float4 *>(src));
+                v = make_float4(0.5f * v.x, 0.5f * v.y, 0.5f * v.z, 0.5f * v.w);
+            } else {
+                const float *b = f < 448 ? p.b1 : p.b2;
+                v = b ? __ldg(reinterpret_cast<const float4 *>(b + c_half + (f & 63))) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            reinterpret_cast<float4 *>(tab)[i] = v;
+        }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(par_full(k & 1));
+    };
+    if (warp == 0) {
+        load_params(0);
+        if (p.N > 1)
+            load_params(1);
+    }
     int units;
     int2 org0 = make_int2(0, 0);   // list mode: the pair's first tile origin, read beside the count
     if constexpr (kStep) {
@@ -748,7 +796,15 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
     if (warp == 0) {
         bool first = true;
 #pragma unroll 1
-        for (int u = pair; u < units && ok; u += npairs) {
+        for (int u = pair, k = 0; u < units && ok; u += npairs, ++k) {
+            // the parameter buffer of unit k, once unit k - 2's epilogues are done with it
+            if (p.N > 1 && k >= 2) {
+                if (!mbar_wait_w(par_empty(k & 1), (uint32_t)((k >> 1) - 1) & 1u, abort_flag, hdr, kSiteParEmpty)) {
+                    ok = false;
+                    break;
+                }
+                load_params(k);
+            }
 #pragma unroll 1
             for (int conv = 0; conv < 2 && ok; ++conv)
 #pragma unroll 1
@@ -897,24 +953,23 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
             // of warp (et >> 5)'s share; a warp reads 4 raw pixels (512
             // contiguous bytes) and writes 8 groups x 4 pixels
             const int kcl = et & 7, pq = (et >> 3) & 3, ew = et >> 5;
-            // both halves' GroupNorm parameters before the first wait
+            // both halves' GroupNorm1 parameters (halved) from this unit's table
+            const int pb = p.N > 1 ? (int)(xk & 1) : 0;
+            if (!mbar_wait_w(par_full(pb), p.N > 1 ? (xk >> 1) & 1u : 0u, abort_flag, hdr, kSiteParFull))
+                return false;
+            const float *tab = reinterpret_cast<const float *>(smem + kOffP + (uint32_t)pb * kParBytes);
             float gsa[2][8], gha[2][8];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int ch = (h * 8 + kcl) * 8;
-                const float4 s0 = __ldg(reinterpret_cast<const float4 *>(p.g1s + n * kC + ch));
-                const float4 s1 = __ldg(reinterpret_cast<const float4 *>(p.g1s + n * kC + ch + 4));
-                const float4 h0v = __ldg(reinterpret_cast<const float4 *>(p.g1h + n * kC + ch));
-                const float4 h1v = __ldg(reinterpret_cast<const float4 *>(p.g1h + n * kC + ch + 4));
+                const float4 s0 = *reinterpret_cast<const float4 *>(tab + ch);
+                const float4 s1 = *reinterpret_cast<const float4 *>(tab + ch + 4);
+                const float4 h0v = *reinterpret_cast<const float4 *>(tab + 128 + ch);
+                const float4 h1v = *reinterpret_cast<const float4 *>(tab + 128 + ch + 4);
                 gsa[h][0] = s0.x; gsa[h][1] = s0.y; gsa[h][2] = s0.z; gsa[h][3] = s0.w;
                 gsa[h][4] = s1.x; gsa[h][5] = s1.y; gsa[h][6] = s1.z; gsa[h][7] = s1.w;
                 gha[h][0] = h0v.x; gha[h][1] = h0v.y; gha[h][2] = h0v.z; gha[h][3] = h0v.w;
                 gha[h][4] = h1v.x; gha[h][5] = h1v.y; gha[h][6] = h1v.z; gha[h][7] = h1v.w;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    gsa[h][e] *= 0.5f;
-                    gha[h][e] *= 0.5f;
-                }
             }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -926,7 +981,7 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                     x_pending = false;
                 const uint8_t *raw = smem + kOffS + h * 128 + kcl * 16;
                 uint8_t *dst = smem + kOffX + (h * 8 + kcl) * kXKc;
-#pragma unroll 1
+#pragma unroll 2
                 for (int px = 4 * ew + pq; px < kXPix; px += 32) {
                     const int yy = px / kXE, xx = px - yy * kXE;
                     const int Y = h0 - 2 + yy, X = w0 - 2 + xx;
@@ -949,6 +1004,9 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
         for (int u = pair; u < units && ok; u += npairs, ++k) {
             int h0, w0, n;
             origin(u, h0, w0, n);
+            // this unit's parameter table (waited for by load_x)
+            const int pb = p.N > 1 ? (int)(k & 1) : 0;
+            const float *tab = reinterpret_cast<const float *>(smem + kOffP + (uint32_t)pb * kParBytes);
             // ------------ epilogue 1: y1 on the 10 x 10 pixels (flat o = 12 yy + xx)
             {
                 const int yy = row / kXE, xx = row - yy * kXE;
@@ -956,36 +1014,11 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                 const int Y = h0 - 1 + yy, X = w0 - 1 + xx;
                 const bool inimg = valid && Y >= 0 && Y < H && X >= 0 && X < W;
                 const bool interior = inimg && yy >= 1 && yy <= kB && xx >= 1 && xx <= kB;
-                float bias[32], gs[32], gh[32];
-#pragma unroll
-                for (int q = 0; q < 32; q += 4) {
-                    const float4 b = p.b1 ? __ldg(reinterpret_cast<const float4 *>(p.b1 + cb + q))
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
-                    const float4 s4 = __ldg(reinterpret_cast<const float4 *>(p.g2s + n * kC + cb + q));
-                    const float4 h4 = __ldg(reinterpret_cast<const float4 *>(p.g2h + n * kC + cb + q));
-                    bias[q] = b.x; bias[q + 1] = b.y; bias[q + 2] = b.z; bias[q + 3] = b.w;
-                    // halved for the SiLU's u = v / 2
-                    gs[q] = 0.5f * s4.x; gs[q + 1] = 0.5f * s4.y; gs[q + 2] = 0.5f * s4.z; gs[q + 3] = 0.5f * s4.w;
-                    gh[q] = 0.5f * h4.x; gh[q + 1] = 0.5f * h4.y; gh[q + 2] = 0.5f * h4.z; gh[q + 3] = 0.5f * h4.w;
-                }
                 if (!mbar_wait_w(acc1_full, k & 1, abort_flag, hdr, kSiteAcc1Full)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                float v[32];
-                tmem_ld32(t_lane + (uint32_t)(colh * 32), v);
-                uint32_t y1p[16], tp[16];
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    y1p[q] = pack_bf16x2(v[2 * q] + bias[2 * q], v[2 * q + 1] + bias[2 * q + 1]);
-                    float a = __fmaf_rn(bf16_lo(y1p[q]), gs[2 * q], gh[2 * q]);
-                    float b = __fmaf_rn(bf16_hi(y1p[q]), gs[2 * q + 1], gh[2 * q + 1]);
-                    tp[q] = inimg ? rb_silu2(a, b) : 0u;
-                }
-                // the accumulator may take the next tile's conv1
-                tc_fence_before();
-                mbar_arrive(acc1_empty);
                 // both CTAs' conv2 of the previous tile have read the buffers
                 if (!cwaited) {
                     cluster_wait_acq();
@@ -996,13 +1029,45 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                     ok = false;
                     break;
                 }
-                if (valid) {
-                    const uint32_t pix = (uint32_t)(yy * kYE + xx) * 16u;
+                const uint32_t pix = (uint32_t)(yy * kYE + xx) * 16u;
+                uint4 *y1dst = reinterpret_cast<uint4 *>(p.y1 + ((((int64_t)n * H + Y) * W + X) * kC + cb) * 2);
+                // Eight channels a pass in a rolled loop: this code runs once per
+                // tile, and code executed for the first time in a launch is
+                // fetched at a few bytes per clock, so its size is latency.
+#pragma unroll 1
+                for (int g = 0; g < 4; ++g) {
+                    const int c0 = cb + 8 * g;
+                    float v[8];
+                    tmem_ld8(t_lane + (uint32_t)(colh * 32 + 8 * g), v);
+                    const int cl = c0 - (int)rank * 64;          // channel within this CTA's half
+                    const float4 s0 = *reinterpret_cast<const float4 *>(tab + 256 + cl);
+                    const float4 s1 = *reinterpret_cast<const float4 *>(tab + 256 + cl + 4);
+                    const float4 q0 = *reinterpret_cast<const float4 *>(tab + 320 + cl);
+                    const float4 q1 = *reinterpret_cast<const float4 *>(tab + 320 + cl + 4);
+                    const float4 b0 = *reinterpret_cast<const float4 *>(tab + 384 + cl);
+                    const float4 b1v = *reinterpret_cast<const float4 *>(tab + 384 + cl + 4);
+                    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1v.x, b1v.y, b1v.z, b1v.w};
+                    const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+                    const float hh[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                    uint32_t y1p[4], tp[4];
 #pragma unroll
-                    for (int g = 0; g < 4; ++g)
+                    for (int q = 0; q < 4; ++q) {
+                        y1p[q] = pack_bf16x2(v[2 * q] + bb[2 * q], v[2 * q + 1] + bb[2 * q + 1]);
+                        // GroupNorm2 (halved: u = v / 2 for the SiLU)
+                        const float ua = __fmaf_rn(bf16_lo(y1p[q]), ss[2 * q], hh[2 * q]);
+                        const float ub = __fmaf_rn(bf16_hi(y1p[q]), ss[2 * q + 1], hh[2 * q + 1]);
+                        tp[q] = inimg ? rb_silu2(ua, ub) : 0u;
+                    }
+                    if (valid)
                         st_shared_v4(sb + kOffY + (uint32_t)(cb / 8 + g) * kYKc + pix,
-                                     make_uint4(tp[4 * g], tp[4 * g + 1], tp[4 * g + 2], tp[4 * g + 3]));
+                                     make_uint4(tp[0], tp[1], tp[2], tp[3]));
+                    // the cached y1 at the tile interior
+                    if (interior)
+                        y1dst[g] = make_uint4(y1p[0], y1p[1], y1p[2], y1p[3]);
                 }
+                // the accumulator may take the next tile's conv1
+                tc_fence_before();
+                mbar_arrive(acc1_empty);
                 // written through the generic proxy, read next by the tensor
                 // cores and the bulk copy (async proxy)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -1024,13 +1089,6 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                         mbar_expect_tx(y1t_full, 8u * kYKc);
                     }
                 }
-                // the cached y1 at the tile interior, off the path to conv2
-                if (interior) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.y1 + ((((int64_t)n * H + Y) * W + X) * kC + cb) * 2);
-#pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        dst[g] = make_uint4(y1p[4 * g], y1p[4 * g + 1], y1p[4 * g + 2], y1p[4 * g + 3]);
-                }
             }
             // ------------ the next tile's halo, while conv2 of this one runs
             if (u + npairs < units && !load_x(u + npairs)) {
@@ -1050,8 +1108,7 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                     res[g] = inimg ? __ldg(reinterpret_cast<const uint4 *>(p.x + e * 2) + g) : make_uint4(0, 0, 0, 0);
 #pragma unroll
                 for (int q = 0; q < 32; q += 4) {
-                    const float4 b = p.b2 ? __ldg(reinterpret_cast<const float4 *>(p.b2 + cb + q))
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4 b = *reinterpret_cast<const float4 *>(tab + 448 + (cb - (int)rank * 64) + q);
                     bias[q] = b.x; bias[q + 1] = b.y; bias[q + 2] = b.z; bias[q + 3] = b.w;
                 }
                 if (!mbar_wait_w(acc2_full, k & 1, abort_flag, hdr, kSiteAcc2Full)) {
@@ -1078,6 +1135,9 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                         dst[g] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
                     }
                 }
+                // this unit's parameter table may take unit k + 2's
+                if (p.N > 1)
+                    mbar_arrive(par_empty(pb));
             }
         }
         // a halo copy still in flight (a wait gave up) lands before the exit
@@ -1213,6 +1273,8 @@ static int rb_prepare(const void *x_edit, const sige_tensor_desc *xd, const void
     a.y1 = static_cast<uint8_t *>(y1);
     a.out = static_cast<uint8_t *>(out);
     a.hdr = static_cast<WsHeader *>(workspace);
+    a.w1 = static_cast<const uint8_t *>(w1);
+    a.w2 = static_cast<const uint8_t *>(w2);
     a.N = xd->n;
     a.H = xd->h;
     a.W = xd->w;

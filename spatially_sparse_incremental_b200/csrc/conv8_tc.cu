@@ -23,7 +23,7 @@
 //   * per 64-channel chunk the halo comes by one TMA of 128-byte pixel rows
 //     (64 channels x 10 x 34 rows of a strip, or 64 x 10 x 10 per tile, zero
 //     outside the image) into a staging buffer; warps 2-9 apply the GroupNorm
-//     affine + SiLU (one f16x2 tanh per two elements) and write the A layout,
+//     affine + SiLU (one tanh per element) and write the A layout,
 //     into the other of two A buffers while the MMAs of the previous chunk run;
 //   * warps 10-13 run the epilogue from the other tensor-memory buffer while
 //     the next unit's MMAs run: + bias (+ residual), one rounding to bf16,
@@ -92,16 +92,14 @@ struct C8Args {
 };
 
 // SiLU of two values from their halves u = v / 2: v sigmoid(v) =
-// u + u tanh(u), both tanh in one tanh.approx.f16x2 (u rounded to f16, the
-// tanh's absolute error about 2^-11), the rest in f32.
+// u + u tanh(u), one tanh.approx.f32 (absolute error about 2^-11) and one
+// FMA per element (the f16x2 tanh has the same element rate on the
+// special-function pipe and adds conversions at half rate).
 __device__ __forceinline__ uint32_t c8_silu2(float ua, float ub)
 {
-    uint32_t h, t;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(ub), "f"(ua));   // ua in the low half
-    asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(h));
     float ta, tb;
-    asm("{\n .reg .f16 l, h;\n mov.b32 {l, h}, %2;\n cvt.f32.f16 %0, l;\n cvt.f32.f16 %1, h;\n}\n"
-        : "=f"(ta), "=f"(tb) : "r"(t));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(ta) : "f"(ua));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(tb) : "f"(ub));
     return pack_bf16x2(__fmaf_rn(ua, ta, ua), __fmaf_rn(ub, tb, ub));
 }
 

@@ -93,6 +93,7 @@ static_assert(kOffS % 128 == 0 && kSHalf % 128 == 0 && kOffY % 16 == 0, "TMA des
 // mbarriers and control words in [0, 1024)
 constexpr uint32_t kBarWFull = 0, kBarWEmpty = 160, kBarXFull = 320, kBarXReady = 336;
 constexpr uint32_t kBarParFull = 40, kBarParEmpty = 56;   // [2] each (after the 5 weight-stage barriers)
+constexpr uint32_t kBarEpiSync = 72;                       // the 256 halo / epilogue threads meet (bounded)
 constexpr uint32_t kBarAcc1Full = 352, kBarAcc1Empty = 360, kBarAcc2Full = 368, kBarAcc2Empty = 376;
 constexpr uint32_t kBarY1tFull = 384, kBarY1tEmpty = 392, kBarDrain = 400, kBarY1tLocal = 408;
 constexpr uint32_t kTmemSlot = 416, kAbort = 420, kUnits = 448;   // kUnits: the step's unit table (int2)
@@ -101,18 +102,19 @@ constexpr int kMaxTiles = 16384;           // tile grid of the step's mask (flag
 // the step's difference stream: a ring of kRing slots, each a chunk of x_orig
 // and the same chunk of x_edit (kRingVec 16-byte vectors each), filled by
 // bulk copies in the halo / conv2-input region before the first halo
-constexpr int kRing = 2;
-constexpr int kRingVec = 1536;
+constexpr int kRing = 3;
+constexpr int kRingVec = 1024;
 constexpr uint32_t kRingBytes = kRingVec * 16;
 constexpr uint32_t kOffRing = kOffX;
 constexpr uint32_t kBarRingFull = 960, kBarRingEmpty = 992;
+constexpr uint32_t kRingTag = 80;          // [kRing] int: the chunk each ring slot holds (-1: the stream is done)
 static_assert(kOffRing + 2 * kRing * kRingBytes <= kOffW && kRingVec % 256 == 0, "ring");
 static_assert(kUnits + 8 * kMaxUnits <= kBarRingFull, "control words");
 
 // wait sites recorded in the error detail on a timeout
 enum : int { kSiteWEmpty = 101, kSiteWFull, kSiteXReady, kSiteAcc1Empty, kSiteAcc2Empty, kSiteY1tFull,
              kSiteXFull, kSiteAcc1Full, kSiteY1tEmpty, kSiteAcc2Full, kSiteGrid, kSiteY1tLocal, kSiteRing,
-             kSiteParFull, kSiteParEmpty };
+             kSiteParFull, kSiteParEmpty, kSiteEpiSync };
 
 }  // namespace rb
 
@@ -136,6 +138,7 @@ struct RbArgs {
     int32_t th, tw;             // tile grid
     uint32_t *flags;            // [th * tw] tile flags in the workspace: the epoch of the call that set them
     unsigned long long *ctr;    // grid-barrier arrivals in the workspace header (only grows)
+    unsigned long long *chunk_ctr;   // difference-stream chunks handed out (workspace header, only grows)
 };
 
 // Four K=16 MMAs of one 64-channel weight stage: A (pixels, no swizzle)
@@ -228,19 +231,17 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8])
 }
 
 // SiLU of two values from their halves u = v / 2 (the GroupNorm affine is
-// pre-scaled by 1/2): v sigmoid(v) = v (1 + tanh(v / 2)) / 2 = u + u tanh(u).
-// Both tanh in one special-function instruction (tanh.approx.f16x2; u rounded
-// to f16 first, the tanh's absolute error about 2^-11, like the f32 form), the
-// rest in f32, one rounding to bf16 at the end.  The special-function units
-// bound the halo transform and epilogue 1; this halves their work.
+// pre-scaled by 1/2): v sigmoid(v) = v (1 + tanh(v / 2)) / 2 = u + u tanh(u),
+// one special-function instruction (tanh.approx.f32, absolute error about
+// 2^-11) and one FMA per element, one rounding to bf16 at the end.  The
+// special-function pipe (16 results per clock and SM, the same for the f16x2
+// form, which adds conversions at half rate) bounds the halo transform and
+// epilogue 1.
 __device__ __forceinline__ uint32_t rb_silu2(float ua, float ub)
 {
-    uint32_t h, t;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(ub), "f"(ua));   // ua in the low half
-    asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(h));
     float ta, tb;
-    asm("{\n .reg .f16 l, h;\n mov.b32 {l, h}, %2;\n cvt.f32.f16 %0, l;\n cvt.f32.f16 %1, h;\n}\n"
-        : "=f"(ta), "=f"(tb) : "r"(t));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(ta) : "f"(ua));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(tb) : "f"(ub));
     return pack_bf16x2(__fmaf_rn(ua, ta, ua), __fmaf_rn(ub, tb, ub));
 }
 
@@ -270,6 +271,26 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v)
 {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
+}
+
+// A staged 8x8 tile (64 pixels x this CTA's 64 channels, 16-byte chunk c of
+// pixel r at chunk c ^ (r & 7)) to the NHWC tensor `dst` at (n, h0.., w0..,
+// 64 rank..): thread et of 256 moves chunks et and et + 256, eight threads per
+// pixel, so a warp stores four pixels' 128 contiguous bytes at a time.
+__device__ __forceinline__ void rb_copy_out(uint32_t stage, uint8_t *dst, int n, int h0, int w0, int H, int W,
+                                            int rank, int et)
+{
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+        const int idx = et + 256 * pass, r = idx >> 3, c = idx & 7;
+        const int Y = h0 + (r >> 3), X = w0 + (r & 7);
+        uint4 v;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                     : "r"(stage + (uint32_t)(r * 128) + ((uint32_t)(c ^ (r & 7)) << 4)));
+        if (Y < H && X < W)
+            *reinterpret_cast<uint4 *>(dst + ((((int64_t)n * H + Y) * W + X) * 128 + rank * 64 + c * 8) * 2) = v;
+    }
 }
 
 __device__ __forceinline__ void st_peer_v4(uint32_t addr, uint4 v)
@@ -368,31 +389,54 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
     bool wrote = false;
     {
         const int64_t nvec = (int64_t)p.N * H * W * (kC / 8);
-        const int64_t per = (nvec + gridDim.x - 1) / gridDim.x;
-        const int64_t v0 = min(nvec, (int64_t)blockIdx.x * per), v1 = min(nvec, v0 + per);
-        const int nchunks = (int)((v1 - v0 + kRingVec - 1) / kRingVec);
+        const int nchunks = (int)((nvec + kRingVec - 1) / kRingVec);
+        // chunks are handed out by a counter in the workspace that only grows:
+        // each call takes exactly nchunks + gridDim.x values from it (every
+        // CTA stops at its first index past the end), so this call's first
+        // value is gen * (nchunks + gridDim.x)
+        const unsigned long long cbase = gen * (unsigned long long)(nchunks + (int)gridDim.x);
         const uint32_t sb = smem_u32(smem);
         auto ring_full = [&](int i) { return sb + kBarRingFull + 8u * i; };
         auto ring_empty = [&](int i) { return sb + kBarRingEmpty + 8u * i; };
+        volatile int *s_tag = reinterpret_cast<volatile int *>(smem + kRingTag);   // chunk of each slot, -1: none
         if (wid == 1) {
-            // one lane fills the ring: per slot, the chunk of both inputs
+            // one lane fills the ring: per slot, one chunk of both inputs
             if (lane == 0) {
-                int issued = 0;
-                for (int c = 0; c < nchunks; ++c) {
+                auto grab = [&]() -> int {
+                    const long long j = (long long)(atomicAdd(p.chunk_ctr, 1ull) - cbase);
+                    return j >= 0 && j < nchunks ? (int)j : -1;
+                };
+                int issued = 0, next = grab();
+                bool stopped = false;
+                for (int c = 0;; ++c) {
                     const int sl = c % kRing;
                     if (c >= kRing && !mbar_wait(ring_empty(sl), (uint32_t)((c / kRing) - 1) & 1u, abort_flag, p.hdr,
-                                                 kSiteRing))
+                                                 kSiteRing)) {
+                        while (next >= 0)   // keep the count exact: claim the rest
+                            next = grab();
                         break;
-                    const int64_t a = v0 + (int64_t)c * kRingVec;
-                    const uint32_t bytes = (uint32_t)min((int64_t)kRingVec, v1 - a) * 16u;
+                    }
+                    const int j = next;
+                    s_tag[sl] = j;
+                    if (j < 0) {
+                        mbar_arrive(ring_full(sl));   // the comparing warps stop at this slot
+                        stopped = true;
+                        break;
+                    }
+                    const int64_t a = (int64_t)j * kRingVec;
+                    const uint32_t bytes = (uint32_t)min((int64_t)kRingVec, nvec - a) * 16u;
                     const uint32_t dst = sb + kOffRing + (uint32_t)sl * 2u * kRingBytes;
                     mbar_expect_tx(ring_full(sl), 2u * bytes);
                     bulk_load(dst, p.xo + a * 16, bytes, ring_full(sl));
                     bulk_load(dst + kRingBytes, p.x + a * 16, bytes, ring_full(sl));
                     ++issued;
+                    next = grab();   // the next index while these copies are in flight
                 }
-                // every copy lands before the region is reused (bounded)
-                for (int c = max(0, issued - kRing); c < issued; ++c) {
+                // every copy lands before the region is reused (bounded); the
+                // copy that shared its slot with the stop mark is complete (its
+                // slot was released before the mark) and its phase parity has
+                // been passed twice, so it is not waited for
+                for (int c = max(0, issued - kRing + (stopped ? 1 : 0)); c < issued; ++c) {
                     const long long t0 = clock64();
                     while (!mbar_try(ring_full(c % kRing), (uint32_t)(c / kRing) & 1u) && clock64() - t0 < kWaitCycles) {
                     }
@@ -403,12 +447,15 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
             // warps 2-9 compare; a warp releases a slot once its lanes read it
             const int ct = tid - 64;
             int last = -1;
-            for (int c = 0; c < nchunks; ++c) {
+            for (int c = 0;; ++c) {
                 const int sl = c % kRing;
                 if (!mbar_wait_w(ring_full(sl), (uint32_t)(c / kRing) & 1u, abort_flag, p.hdr, kSiteRing))
                     break;
-                const int64_t a = v0 + (int64_t)c * kRingVec;
-                const int n = (int)min((int64_t)kRingVec, v1 - a);
+                const int j = s_tag[sl];
+                if (j < 0)
+                    break;
+                const int64_t a = (int64_t)j * kRingVec;
+                const int n = (int)min((int64_t)kRingVec, nvec - a);
                 const uint4 *so = reinterpret_cast<const uint4 *>(smem + kOffRing + (uint32_t)sl * 2u * kRingBytes);
                 const uint4 *se = so + kRingVec;
 #pragma unroll
@@ -454,6 +501,8 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
                 ok = 0;
                 break;
             }
+            // back off: 148 pollers spinning on the counter's line can starve
+            // the last arrivals (a call without this pause timed out here)
             __nanosleep(32);
         }
         *s_ok = ok;
@@ -682,6 +731,7 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
             mbar_init(par_full(b), 1);
             mbar_init(par_empty(b), kEpi);
         }
+        mbar_init(sb + kBarEpiSync, kEpi);
         if constexpr (kStep) {
             for (int i = 0; i < kRing; ++i) {
                 mbar_init(sb + kBarRingFull + 8u * i, 1);
@@ -757,7 +807,8 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
         const int n = (pair + k * npairs) % p.N;
         float *tab = reinterpret_cast<float *>(smem + kOffP + (uint32_t)(k & 1) * kParBytes);
         const int c_half = (int)rank * 64;
-        for (int i = lane; i < 128; i += 32) {
+#pragma unroll
+        for (int i = lane; i < 128; i += 32) {   // four independent loads per lane
             const int f = 4 * i;
             float4 v;
             if (f < 256) {
@@ -876,33 +927,38 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
         uint32_t k = 0;
 #pragma unroll 1
         for (int u = pair; u < units && ok; u += npairs, ++k) {
-            // conv1: accumulator [0, 64) free once epilogue 1 of the previous tile has read it
-            if (k > 0 && !mbar_wait_w(acc1_empty, (k - 1) & 1, abort_flag, hdr, kSiteAcc1Empty)) {
-                ok = false;
-                break;
+            // conv1, then conv2 through ONE copy of the issue code (code run
+            // for the first time in a launch is fetched slowly)
+#pragma unroll 1
+            for (int cv = 0; cv < 2; ++cv) {
+                if (cv == 0) {
+                    // accumulator [0, 64) free once epilogue 1 of the previous tile has read it
+                    if (k > 0 && !mbar_wait_w(acc1_empty, (k - 1) & 1, abort_flag, hdr, kSiteAcc1Empty)) {
+                        ok = false;
+                        break;
+                    }
+                } else {
+                    // conv2: its input written by both CTAs' epilogue 1
+                    if (k > 0 && !mbar_wait_w(acc2_empty, (k - 1) & 1, abort_flag, hdr, kSiteAcc2Empty)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(y1t_full, k & 1, abort_flag, hdr, kSiteY1tFull))) {
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                }
+                tc_fence_after();
+                if (!conv(cv ? sb + kOffY : sb + kOffX, cv ? kYE : kXE, cv ? kYKc : kXKc, cv ? 64u : 0u, cv == 0,
+                          k & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_commit_w(cv ? acc2_full : acc1_full);
             }
-            tc_fence_after();
-            if (!conv(sb + kOffX, kXE, kXKc, 0, true, k & 1)) {
-                ok = false;
+            if (!ok)
                 break;
-            }
-            tc_commit_w(acc1_full);
-            // conv2: its input written by both CTAs' epilogue 1
-            if (k > 0 && !mbar_wait_w(acc2_empty, (k - 1) & 1, abort_flag, hdr, kSiteAcc2Empty)) {
-                ok = false;
-                break;
-            }
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(y1t_full, k & 1, abort_flag, hdr, kSiteY1tFull))) {
-                ok = false;
-                break;
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            tc_fence_after();
-            if (!conv(sb + kOffY, kYE, kYKc, 64, false, 0)) {
-                ok = false;
-                break;
-            }
-            tc_commit_w(acc2_full);
             // the conv2 input buffers of both CTAs may be rewritten (none is
             // after the pair's last tile)
             if (u + npairs < units)
@@ -927,6 +983,15 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
         const int H = p.H, W = p.W;
         bool x_pending = false;
         uint32_t xk = 0;                               // halos loaded so far (phase of x_full / x_ready)
+        // The 256 threads meet on an mbarrier (bounded wait, unlike a named
+        // barrier, so a thread that left on an error cannot hang the rest).
+        uint32_t esync = 0;
+        auto epi_sync = [&]() -> bool {
+            mbar_arrive(sb + kBarEpiSync);
+            const bool r = mbar_wait_w(sb + kBarEpiSync, esync & 1u, abort_flag, hdr, kSiteEpiSync);
+            ++esync;
+            return r;
+        };
 
         auto origin = [&](int u, int &h0, int &w0, int &n) {
             int2 o;
@@ -1014,6 +1079,19 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                 const int Y = h0 - 1 + yy, X = w0 - 1 + xx;
                 const bool inimg = valid && Y >= 0 && Y < H && X >= 0 && X < W;
                 const bool interior = inimg && yy >= 1 && yy <= kB && xx >= 1 && xx <= kB;
+                // this thread's 32 channels of b1 and GroupNorm2 (halved) from the
+                // unit's table, before the wait
+                const int cl0 = colh * 32;
+                float bias[32], gs[32], gh[32];
+#pragma unroll
+                for (int q = 0; q < 32; q += 4) {
+                    const float4 s4 = *reinterpret_cast<const float4 *>(tab + 256 + cl0 + q);
+                    const float4 h4 = *reinterpret_cast<const float4 *>(tab + 320 + cl0 + q);
+                    const float4 b4 = *reinterpret_cast<const float4 *>(tab + 384 + cl0 + q);
+                    gs[q] = s4.x; gs[q + 1] = s4.y; gs[q + 2] = s4.z; gs[q + 3] = s4.w;
+                    gh[q] = h4.x; gh[q + 1] = h4.y; gh[q + 2] = h4.z; gh[q + 3] = h4.w;
+                    bias[q] = b4.x; bias[q + 1] = b4.y; bias[q + 2] = b4.z; bias[q + 3] = b4.w;
+                }
                 if (!mbar_wait_w(acc1_full, k & 1, abort_flag, hdr, kSiteAcc1Full)) {
                     ok = false;
                     break;
@@ -1030,40 +1108,33 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                     break;
                 }
                 const uint32_t pix = (uint32_t)(yy * kYE + xx) * 16u;
-                uint4 *y1dst = reinterpret_cast<uint4 *>(p.y1 + ((((int64_t)n * H + Y) * W + X) * kC + cb) * 2);
-                // Eight channels a pass in a rolled loop: this code runs once per
-                // tile, and code executed for the first time in a launch is
-                // fetched at a few bytes per clock, so its size is latency.
-#pragma unroll 1
+                // the tile interior of y1 goes through a staging tile in the
+                // conv1 input buffer (free once conv1 is complete): 64 pixels x
+                // 128 bytes, 16-byte chunk c of pixel r at chunk c ^ (r & 7)
+                const uint32_t y1s = sb + kOffX + (uint32_t)(((yy - 1) * kB + (xx - 1)) * 128);
+                const uint32_t y1s_sw = (uint32_t)((yy - 1) * kB + (xx - 1)) & 7u;
+                float v[32];
+                tmem_ld32(t_lane + (uint32_t)cl0, v);
+                // all 32 columns in straight-line code: four independent groups
+                // keep the special-function pipe busy
+#pragma unroll
                 for (int g = 0; g < 4; ++g) {
-                    const int c0 = cb + 8 * g;
-                    float v[8];
-                    tmem_ld8(t_lane + (uint32_t)(colh * 32 + 8 * g), v);
-                    const int cl = c0 - (int)rank * 64;          // channel within this CTA's half
-                    const float4 s0 = *reinterpret_cast<const float4 *>(tab + 256 + cl);
-                    const float4 s1 = *reinterpret_cast<const float4 *>(tab + 256 + cl + 4);
-                    const float4 q0 = *reinterpret_cast<const float4 *>(tab + 320 + cl);
-                    const float4 q1 = *reinterpret_cast<const float4 *>(tab + 320 + cl + 4);
-                    const float4 b0 = *reinterpret_cast<const float4 *>(tab + 384 + cl);
-                    const float4 b1v = *reinterpret_cast<const float4 *>(tab + 384 + cl + 4);
-                    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1v.x, b1v.y, b1v.z, b1v.w};
-                    const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-                    const float hh[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
                     uint32_t y1p[4], tp[4];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        y1p[q] = pack_bf16x2(v[2 * q] + bb[2 * q], v[2 * q + 1] + bb[2 * q + 1]);
+                        const int c = 8 * g + 2 * q;
+                        y1p[q] = pack_bf16x2(v[c] + bias[c], v[c + 1] + bias[c + 1]);
                         // GroupNorm2 (halved: u = v / 2 for the SiLU)
-                        const float ua = __fmaf_rn(bf16_lo(y1p[q]), ss[2 * q], hh[2 * q]);
-                        const float ub = __fmaf_rn(bf16_hi(y1p[q]), ss[2 * q + 1], hh[2 * q + 1]);
+                        const float ua = __fmaf_rn(bf16_lo(y1p[q]), gs[c], gh[c]);
+                        const float ub = __fmaf_rn(bf16_hi(y1p[q]), gs[c + 1], gh[c + 1]);
                         tp[q] = inimg ? rb_silu2(ua, ub) : 0u;
                     }
                     if (valid)
                         st_shared_v4(sb + kOffY + (uint32_t)(cb / 8 + g) * kYKc + pix,
                                      make_uint4(tp[0], tp[1], tp[2], tp[3]));
-                    // the cached y1 at the tile interior
                     if (interior)
-                        y1dst[g] = make_uint4(y1p[0], y1p[1], y1p[2], y1p[3]);
+                        st_shared_v4(y1s + ((((uint32_t)(colh * 4 + g)) ^ y1s_sw) << 4),
+                                     make_uint4(y1p[0], y1p[1], y1p[2], y1p[3]));
                 }
                 // the accumulator may take the next tile's conv1
                 tc_fence_before();
@@ -1089,8 +1160,21 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                         mbar_expect_tx(y1t_full, 8u * kYKc);
                     }
                 }
+                // the staged y1 interior to the cached y1, coalesced: a warp
+                // writes four pixels' 128 contiguous bytes per instruction
+                ok = __all_sync(0xFFFFFFFFu, ok);   // thread 0's wait, warp-uniform
+                if (!ok || !epi_sync()) {
+                    ok = false;
+                    break;
+                }
+                rb_copy_out(sb + kOffX, p.y1, n, h0, w0, H, W, (int)rank, et);
             }
             // ------------ the next tile's halo, while conv2 of this one runs
+            // every thread has copied the staged y1 out of the conv1 input buffer
+            if (u + npairs < units && !epi_sync()) {
+                ok = false;
+                break;
+            }
             if (u + npairs < units && !load_x(u + npairs)) {
                 ok = false;
                 break;
@@ -1120,20 +1204,35 @@ __global__ void __launch_bounds__(rb::kThreads, 1)
                 tmem_ld32(t_lane + 64u + (uint32_t)(colh * 32), v);
                 tc_fence_before();
                 mbar_arrive(acc2_empty);
+                // out through a staging tile in this CTA's half of the conv2
+                // input buffer (conv2 is complete; the peer writes only the
+                // other half), then coalesced stores
+                const uint32_t os = sb + kOffY + rank * 8u * kYKc;
                 if (inimg) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + e * 2);
+                    const uint32_t r = (uint32_t)(i * kB + j);
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
-                        const uint32_t *r = reinterpret_cast<const uint32_t *>(&res[g]);
+                        const uint32_t *rr = reinterpret_cast<const uint32_t *>(&res[g]);
                         uint32_t o4[4];
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const int c0 = 8 * g + 2 * q;
-                            o4[q] = pack_bf16x2((v[c0] + bias[c0]) + bf16_lo(r[q]),
-                                                (v[c0 + 1] + bias[c0 + 1]) + bf16_hi(r[q]));
+                            o4[q] = pack_bf16x2((v[c0] + bias[c0]) + bf16_lo(rr[q]),
+                                                (v[c0 + 1] + bias[c0 + 1]) + bf16_hi(rr[q]));
                         }
-                        dst[g] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                        st_shared_v4(os + r * 128u + ((((uint32_t)(colh * 4 + g)) ^ (r & 7u)) << 4),
+                                     make_uint4(o4[0], o4[1], o4[2], o4[3]));
                     }
+                }
+                if (!epi_sync()) {
+                    ok = false;
+                    break;
+                }
+                rb_copy_out(os, p.out, n, h0, w0, H, W, (int)rank, et);
+                // the staging half may take the next tile's conv2 input
+                if (u + npairs < units && !epi_sync()) {
+                    ok = false;
+                    break;
                 }
                 // this unit's parameter table may take unit k + 2's
                 if (p.N > 1)
@@ -1395,6 +1494,7 @@ extern "C" int sige_resblock_step(const void *x_orig, const void *x_edit, const 
     a.tw = tw;
     // the arrival counter: 8 bytes at offset 16 of the header
     a.ctr = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + 16);
+    a.chunk_ctr = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + 24);
     a.flags = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kWsHeader);
     return rb_launch<true>(a, tmx, tw1, tw2, (int64_t)capacity * xd->n, stream);
 }

@@ -334,12 +334,16 @@ int sige_conv_fused_ext(const void *x, const sige_tensor_desc *xd, const void *w
  *                    error SIGE_ERR_CAPACITY is recorded)
  *   workspace      : device, >= sige_resblock_step_workspace_bytes(xd, block),
  *                    zero-filled before its first use and not written by the
- *                    caller afterwards: the header holds the error word and a
+ *                    caller afterwards: the header holds the error word, a
  *                    grid-barrier counter that only grows (the call's
- *                    generation), and each tile flag holds the generation of
- *                    the call that last set it, so no call has to clear
- *                    anything for the next.  One workspace per device and
- *                    stream: calls sharing one must not overlap.
+ *                    generation) and a counter that hands out the chunks of
+ *                    the difference stream (it also only grows, by a fixed
+ *                    amount per call), and each tile flag holds the
+ *                    generation of the call that last set it, so no call has
+ *                    to clear anything for the next.  After a call that
+ *                    recorded SIGE_ERR_TIMEOUT, zero the workspace again.
+ *                    One workspace per device and stream: calls sharing one
+ *                    must not overlap.
  * Other arguments as sige_resblock_fused.  The launch keeps every CTA
  * resident at once (one pair of CTAs per two SMs); if other work holds SMs so
  * that some CTAs cannot start, the grid barrier's bounded wait (about 1 s)

@@ -501,8 +501,7 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
                 ok = 0;
                 break;
             }
-            // back off: 148 pollers spinning on the counter's line can starve
-            // the last arrivals (a call without this pause timed out here)
+            // a short pause between polls of the counter's line
             __nanosleep(32);
         }
         *s_ok = ok;

@@ -452,7 +452,10 @@ int sige_get_device_error(void *workspace, sige_stream_t stream);
 /* Bound, in SM clock cycles, of the device-side waits that end a call with
  * SIGE_ERR_TIMEOUT when they expire, for every launch enqueued after this
  * call, process-wide; 0 restores each kernel's own bound (seconds).  Covered:
- * the wait of sige_reduce_mask's reducing CTA for the streaming CTAs.  A test
+ * the wait of sige_reduce_mask's reducing CTA for the streaming CTAs, and the
+ * grid barrier of sige_resblock_step (on expiry every CTA takes no tile, the
+ * outputs are left as they were and the workspace stays consistent for the
+ * next call; the error detail is the wait site, 111).  A test
  * of the failure path sets a bound of a few cycles so that the wait expires,
  * checks the status and restores 0.  Returns SIGE_ERR_INVALID_ARG for a
  * negative value. */

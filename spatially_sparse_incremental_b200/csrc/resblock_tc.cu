@@ -139,6 +139,7 @@ struct RbArgs {
     uint32_t *flags;            // [th * tw] tile flags in the workspace: the epoch of the call that set them
     unsigned long long *ctr;    // grid-barrier arrivals in the workspace header (only grows)
     unsigned long long *chunk_ctr;   // difference-stream chunks handed out (workspace header, only grows)
+    long long grid_wait;        // bound of the grid barrier's wait, in clocks (sige_set_wait_cycles, else ~1 s)
 };
 
 // Four K=16 MMAs of one 64-channel weight stage: A (pixels, no swizzle)
@@ -496,7 +497,7 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
             asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p.ctr) : "memory");
             if (v >= target)
                 break;
-            if (clock64() - t0 > kWaitCycles) {
+            if (clock64() - t0 > p.grid_wait) {
                 record_error(p.hdr, SIGE_ERR_TIMEOUT, kSiteGrid);
                 ok = 0;
                 break;
@@ -1494,6 +1495,7 @@ extern "C" int sige_resblock_step(const void *x_orig, const void *x_edit, const 
     // the arrival counter: 8 bytes at offset 16 of the header
     a.ctr = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + 16);
     a.chunk_ctr = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + 24);
+    a.grid_wait = wait_cycles_or(kWaitCycles);
     a.flags = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kWsHeader);
     return rb_launch<true>(a, tmx, tw1, tw2, (int64_t)capacity * xd->n, stream);
 }

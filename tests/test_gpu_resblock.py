@@ -245,3 +245,29 @@ def test_step_without_an_edit_writes_nothing():
     idx, cnt, ws, y1, out, y1c, outc = _step(blk, xo, xo.clone(), 64)
     assert int(cnt[0].item()) == 0
     assert torch.equal(bits(y1.cpu()), bits(y1c.cpu())) and torch.equal(bits(out.cpu()), bits(outc.cpu()))
+
+
+def test_step_grid_barrier_timeout_reports_and_the_next_call_is_exact(orc):
+    """The failure path of the one-launch step, the allowed way: a wait bound of
+    a few cycles makes the grid barrier give up (nothing faults, nothing
+    hangs).  The call returns, records SIGE_ERR_TIMEOUT with the barrier's
+    wait site (its outputs are then unspecified: the last CTA to arrive still
+    sees the barrier complete), and the next call with the default bound, on
+    the same workspace, is exact."""
+    blk = inputs.make_cfg3(64, H=64, W=64, area=0.05)
+    xo, xe = blk.x_orig.to(DEV), blk.x_edit.to(DEV)
+    ws = sige.zeros_workspace(sige.sige_resblock_step_workspace_bytes(xe), DEV)
+    sige.sige_set_wait_cycles(16)
+    try:
+        idx, cnt, _, y1, out, y1c, outc = _step(blk, xo, xe, 64, ws=ws)
+    finally:
+        sige.sige_set_wait_cycles(0)
+    detail = int(ws[4:8].cpu().view(torch.int32)[0].item())
+    assert sige.sige_get_device_error(ws) == sige.ERR_TIMEOUT
+    assert detail == 111                                     # the grid barrier
+    idx, cnt, _, y1, out, y1c, outc = _step(blk, xo, xe, 64, ws=ws)
+    n = int(cnt[0].item())
+    ref_idx = orc.reduce_mask(blk.x_orig, blk.x_edit, 1e-3, [(64, 64, 8)], 1)[0]
+    assert n == len(ref_idx) and np.array_equal(idx[:n].cpu().numpy(), ref_idx)
+    assert sige.sige_get_device_error(ws) == sige.OK
+    _check(orc, blk, blk.x_orig, blk.x_edit, ref_idx, y1, out, y1c, outc)

@@ -484,6 +484,10 @@ def measure_extras(dev, flush, stream, peaks, seed, step_graph):
         out["attention"] = attention_timing(seed, dev, flush, stream, peaks)
     except Exception as e:
         out["attention"] = {"error": str(e)[:200]}
+    try:
+        out["gather_scatter"] = gather_scatter_timing(seed, dev, flush, stream, peaks)
+    except Exception as e:
+        out["gather_scatter"] = {"error": str(e)[:200]}
     # edit-area sweeps of the SD-latent and GauGAN-shaped layers: active tiles,
     # sparse and dense time and the roofline fraction at every area
     sweeps = []
@@ -505,6 +509,41 @@ def measure_extras(dev, flush, stream, peaks, seed, step_graph):
     out["layer_sweeps"] = srows
     out["layers"] = rows
     return out
+
+
+def gather_scatter_timing(seed, dev, flush, stream, peaks, reps=30):
+    """The unfused calls on the headline workload's tile list: the gather of
+    conv1's 10x10 halos (GroupNorm1 + SiLU applied, bf16 blocks out) and the
+    scatter of conv2's float32 blocks (+ bias + residual, bf16 into the cached
+    output); each against the HBM roofline of its own bytes (halo pixels read
+    once per tile, blocks written / read, outputs and residual)."""
+    import spatially_sparse_incremental_b200 as sige
+    d = make_workload(seed, dev)
+    torch.cuda.synchronize()
+    n = int(d["cnt"].item())
+    cd = d["cd"]
+    b_in = (cd.block - 1) * cd.stride + cd.kernel
+    blocks = torch.empty((max(d["cap"], 1), 1, b_in, b_in, C), dtype=torch.bfloat16, device=dev)
+    oblk = torch.randn((max(d["cap"], 1), 1, BLOCK, BLOCK, C), generator=torch.Generator().manual_seed(seed)).to(dev)
+    y = d["out"].clone()
+
+    def gather():
+        sige.sige_gather(d["x_edit"], cd, d["idx"], d["cnt"], d["cap"], d["gs1"], d["gh1"], silu=True, blocks=blocks,
+                         stream=stream)
+
+    def scatter():
+        sige.sige_scatter(oblk, cd, d["idx"], d["cnt"], d["cap"], y, bias=d["b2"], residual=d["x_edit"],
+                          stream=stream)
+    res = {"active_tiles": n}
+    for name, fn, nbytes in (("gather", gather, 2 * n * b_in * b_in * C * 2),
+                             ("scatter", scatter, n * BLOCK * BLOCK * C * (4 + 2 + 2))):
+        g = capture(fn, stream)
+        t = time_graph(g, flush, reps, stream)
+        us = float(np.median(t)) * 1e3
+        res[name] = {"us": us, "bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9,
+                     "frac": nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"]}
+        del g
+    return res
 
 
 def layer_timing(L, bits, dev, flush, stream, peaks, reps=30, dense_us=None):

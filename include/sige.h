@@ -403,8 +403,8 @@ int sige_restore_tiles(const void *src, void *dst, const sige_tensor_desc *d, in
  * `idx` (block x block, clipped to the map), per head h:
  *   o[n][y][x][h*dvh : (h+1)*dvh] = softmax(q_h k_h^T / sqrt(dh)) v_h
  * over all `keys` keys, dh = qd->c / heads, dvh = dv / heads; float32
- * arithmetic, one rounding to bf16.  Every other element of o is left as it
- * is.  The projections before and after are sparse 1x1 convolutions
+ * accumulation, one rounding of o to bf16.  Every other element of o is left
+ * as it is.  The projections before and after are sparse 1x1 convolutions
  * (sige_conv_fused) on the same tile list.
  *   q     : device bf16 [N][H][W][D], described by qd (NHWC); read at the tokens
  *   k     : device bf16 [N][keys][D] (self-attention: the [N][H][W][D] key map)
@@ -412,6 +412,15 @@ int sige_restore_tiles(const void *src, void *dst, const sige_tensor_desc *d, in
  *   idx, count, capacity, block : the tile list of this resolution (as (1))
  *   o     : device bf16 [N][H][W][dv], written at the tokens only; must not
  *           overlap q, k or v
+ * Two kernels (sige_attention_path tells which one a layer gets):
+ *   tensor cores, for dh and dvh multiples of 8 up to 64 and 16-byte aligned
+ *     buffers: 128 query slots x 128-key chunks, S = q k^T and O += P v by
+ *     tcgen05.mma, P = exp(S - running max) rounded to bf16 for the second
+ *     product; the keys of a block are split over up to 8 CTAs of a cluster
+ *     when the list is short, the partial rows merged in distributed shared
+ *     memory.  A device-side wait that expires (a fault elsewhere) leaves the
+ *     rows of that block unwritten;
+ *   CUDA cores otherwise: fp32 scores and weights.
  * All buffers belong to the caller; nothing is allocated; asynchronous on
  * `stream`.  Errors: SIGE_ERR_INVALID_ARG (NULL pointer, non-positive size,
  * D or dv not a multiple of heads), SIGE_ERR_UNSUPPORTED (not bf16 NHWC,
@@ -419,6 +428,12 @@ int sige_restore_tiles(const void *src, void *dst, const sige_tensor_desc *d, in
 int sige_attention_core(const void *q, const sige_tensor_desc *qd, const void *k, const void *v, int32_t keys,
                         int32_t dv, int32_t heads, const int32_t *idx, const int32_t *count, int32_t capacity,
                         int32_t block, void *o, sige_stream_t stream);
+
+/* Which kernel sige_attention_core runs for queries described by qd, value
+ * width dv and `heads` heads (16-byte aligned buffers): 1 = tcgen05 tensor
+ * cores, 0 = CUDA cores; SIGE_ERR_INVALID_ARG / SIGE_ERR_UNSUPPORTED as that
+ * call would return them.  Host only. */
+int sige_attention_path(const sige_tensor_desc *qd, int32_t dv, int32_t heads);
 
 /* ------------------------------------------------------------ utilities */
 

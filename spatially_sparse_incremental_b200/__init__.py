@@ -86,6 +86,7 @@ SIGNATURES = {
     "sige_conv_path": (_i32, [_CD, _i32]),
     "sige_conv_schedule": (_i32, [_CD, _i32, _i32, _i32, _vp, _i32]),
     "sige_attention_core": (_i32, [_vp, _TD, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp]),
+    "sige_attention_path": (_i32, [_TD, _i32, _i32]),
     "sige_launch_count": (ctypes.c_uint64, []),
     "sige_status_string": (ctypes.c_char_p, [_i32]),
 }
@@ -419,6 +420,14 @@ def sige_set_wait_cycles(cycles: int) -> None:
 
 def sige_conv_path(cd: ConvDesc, dtype: torch.dtype) -> int:
     return int(lib().sige_conv_path(ctypes.byref(cd), _DT[dtype]))
+
+
+def sige_attention_path(q, dv: int, heads: int) -> int:
+    """Which kernel sige_attention_core runs for queries like ``q`` (an NHWC
+    tensor), value width dv and this head count: 1 = tcgen05 tensor cores,
+    0 = CUDA cores; negative = a sige_status."""
+    qd = tensor_desc(q)
+    return int(lib().sige_attention_path(ctypes.byref(qd), int(dv), int(heads)))
 
 
 def sige_attention_core(q, k, v, heads: int, idx, count, capacity: int, block: int, o=None, stream=None):

@@ -201,6 +201,10 @@ extern "C" int sige_attention_core(const void *q, const sige_tensor_desc *qd, co
         return SIGE_ERR_UNSUPPORTED;
     if (capacity == 0)
         return SIGE_OK;
+    const int tc = attention_core_tc(q, k, v, o, idx, count, qd->n, qd->h, qd->w, qd->c, dv, keys, heads, block,
+                                     capacity, (cudaStream_t)stream);
+    if (tc != 1)
+        return tc;
     AttnParams p{};
     p.q = static_cast<const __nv_bfloat16 *>(q);
     p.k = static_cast<const __nv_bfloat16 *>(k);
@@ -230,4 +234,15 @@ extern "C" int sige_attention_core(const void *q, const sige_tensor_desc *qd, co
     k_attention<<<grid, kAttnThreads, smem, (cudaStream_t)stream>>>(p);
     count_launch();
     return launch_check();
+}
+
+extern "C" int sige_attention_path(const sige_tensor_desc *qd, int32_t dv, int32_t heads)
+{
+    if (!qd || dv < 1 || heads < 1 || qd->c < 1)
+        return SIGE_ERR_INVALID_ARG;
+    if (qd->c % heads || dv % heads)
+        return SIGE_ERR_INVALID_ARG;
+    if (qd->dtype != SIGE_BF16 || qd->layout != SIGE_NHWC || qd->c / heads > kAttnMaxHead || dv / heads > kAttnMaxHead)
+        return SIGE_ERR_UNSUPPORTED;
+    return attention_tc_scope(qd->c / heads, dv / heads) ? 1 : 0;
 }

@@ -79,6 +79,12 @@ int device_sm_count();
 // Bound of the device-side waits that sige_set_wait_cycles() may shorten, for
 // launches enqueued from now on: the value set there, or `dflt` when none is.
 long long wait_cycles_or(long long dflt);
+// The tensor-core attention step (attention_tc.cu): a sige_status, or 1 when
+// the call is outside that kernel's scope and the CUDA-core kernel runs it.
+int attention_core_tc(const void *q, const void *k, const void *v, void *o, const int32_t *idx, const int32_t *count,
+                      int N, int H, int W, int D, int Dv, int Lk, int heads, int b, int cap, cudaStream_t stream);
+// Head widths that kernel takes (with 16-byte aligned buffers).
+bool attention_tc_scope(int dh, int dvh);
 
 // Programmatic dependent launch.  A kernel launched this way may start while
 // the kernel before it in the stream is still running: its CTAs take SMs as

@@ -339,3 +339,17 @@ def test_resblock_step_validation(L):
     assert call(wsb=need - 1) == sige.ERR_WORKSPACE
     assert call(y1=ctypes.c_void_p(0x30000000)) == sige.ERR_INVALID_ARG     # y1 overlaps x_orig
     assert call(xo=ctypes.c_void_p(0x30000008)) == sige.ERR_UNSUPPORTED     # x_orig needs 16-byte alignment
+
+
+def test_attention_path_selection(L):
+    """Heads of width 8..64 in steps of 8 take the tensor-core kernel; wider
+    heads or widths that are not multiples of 8, the CUDA-core one."""
+    import torch
+    q = lambda c: torch.empty((1, 8, 8, c), dtype=torch.bfloat16)
+    assert sige.sige_attention_path(q(320), 320, 8) == 1      # heads of 40
+    assert sige.sige_attention_path(q(64), 32, 1) == 1        # 64 / 32
+    assert sige.sige_attention_path(q(32), 32, 4) == 1        # heads of 8
+    assert sige.sige_attention_path(q(256), 256, 2) == 0      # heads of 128
+    assert sige.sige_attention_path(q(60), 60, 2) == 0        # heads of 30
+    assert sige.sige_attention_path(q(320), 320, 3) == sige.ERR_INVALID_ARG
+    assert sige.sige_attention_path(torch.empty((1, 8, 8, 64)), 64, 1) == sige.ERR_UNSUPPORTED   # float32

@@ -377,6 +377,7 @@ def time_graph(g, flush, reps, stream, warm=False):
 
 
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # FMA lanes x 2 x max SM clock
+SFU_TEXP = 148 * 16 * 1.965e9 / 1e12                 # exp2 results per second (1e12): 16 per SM and clock
 
 
 def layer_roofline(macs, nbytes, dtype_bits, peaks, us):
@@ -611,14 +612,19 @@ def attention_timing(seed, dev, flush, stream, peaks, H_=64, W_=64, C_=320, head
     m_tok = tiles * block * block
     flops = 2.0 * m_tok * H_ * W_ * (C_ + C_)
     nbytes = H_ * W_ * (C_ + C_) * 2 + m_tok * (C_ + C_) * 2
+    exps = float(m_tok) * H_ * W_ * heads                      # one exponential per (query, key, head)
     t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
-    t_alu = flops / (FP32_ALU_TFLOPS * 1e12)
+    t_sfu = exps / (SFU_TEXP * 1e12)
+    t_de_sfu = float(H_ * W_) * H_ * W_ * heads / (SFU_TEXP * 1e12)
+    path = sige.sige_attention_path(q, C_, heads)
     return {"name": f"SD latent {H_}x{W_} C{C_} self-attention, {heads} heads, b{block}, {area:.1%} edit",
             "active_tiles": tiles, "query_tokens": m_tok, "keys": H_ * W_, "sparse_us": t_sp, "dense_us": t_de,
-            "speedup": t_de / t_sp, "path": "cuda-core (fp32 online softmax)",
-            "roofline": {"bound": "tensor", "flops": flops, "bytes": nbytes, "roof_us": t_tensor * 1e6,
-                         "frac": t_tensor / (t_sp * 1e-6),
-                         "alu_roof_us": t_alu * 1e6, "alu_frac": t_alu / (t_sp * 1e-6)}}
+            "speedup": t_de / t_sp,
+            "path": "tcgen05 (QK^T and PV on tensor cores, P bf16 in tensor memory)" if path == 1
+                    else "cuda-core (fp32 online softmax)",
+            "roofline": {"bound": "sfu", "exps": exps, "roof_us": t_sfu * 1e6, "frac": t_sfu / (t_sp * 1e-6),
+                         "dense_frac": t_de_sfu / (t_de * 1e-6),
+                         "tensor_roof_us": t_tensor * 1e6, "flops": flops, "bytes": nbytes}}
 
 
 def ext_layer_timing(L, dev, flush, stream, peaks, transposed=False, spade=False, reps=20):

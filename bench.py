@@ -520,8 +520,10 @@ def gather_scatter_timing(seed, dev, flush, stream, peaks, reps=30):
     once per tile, blocks written / read, outputs and residual)."""
     import spatially_sparse_incremental_b200 as sige
     d = make_workload(seed, dev)
+    two_launch_calls(d)["mask"]()            # the step's tile list
     torch.cuda.synchronize()
     n = int(d["cnt"].item())
+    assert n > 0, "the headline edit lists no tile"
     cd = d["cd"]
     b_in = (cd.block - 1) * cd.stride + cd.kernel
     blocks = torch.empty((max(d["cap"], 1), 1, b_in, b_in, C), dtype=torch.bfloat16, device=dev)

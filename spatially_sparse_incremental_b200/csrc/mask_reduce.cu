@@ -8,10 +8,13 @@
 //
 // Layout of the work:
 //   phase 1 (every CTA but CTA 0, HBM-bound): stream both inputs once.  The
-//     inputs are cut into chunks (up to 16 KB of each input); a CTA takes
-//     every (number of streaming CTAs)-th chunk and keeps seven of them in
-//     flight with bulk asynchronous copies into shared memory, so nearly the
-//     whole input is requested at once.  An element whose |edit - orig| >
+//     inputs are cut into chunks (up to 16 KB of each input); every streaming
+//     CTA keeps four in flight with bulk asynchronous copies into shared
+//     memory.  The first four of each CTA are fixed (chunk worker + k *
+//     workers); the rest are handed out by a counter in the workspace header,
+//     one at a time as a stage frees, so CTAs whose copies land late take
+//     fewer chunks and all finish together (with a fixed split the last CTA
+//     finished ~4 us after the median one).  An element whose |edit - orig| >
 //     threshold marks, at every scale, the tile its pixel falls in (with a
 //     pixel radius R, every tile within R pixels of it at that scale).
 //     Downsampling by an integer factor f followed by b x b tiles is the same
@@ -72,7 +75,7 @@ struct __align__(16) MaskParams {
     int32_t pow2;        // vpp, H and W are powers of two: index math by shifts
     int32_t log_vpp, log_w, log_epv;
     int32_t chunk;       // modes 0, 1: vectors per chunk of each input (multiple of 256)
-    int32_t chunks_base, chunks_rem;   // chunks per streaming CTA: base, +1 for the first rem
+    int32_t nchunks;     // modes 0, 1: chunks of each input
     int32_t radius;      // pixel dilation at each scale before tiling (0: none)
     int64_t wait_cycles; // bound of CTA 0's wait for the streaming CTAs, in SM clock cycles
 };
@@ -216,9 +219,9 @@ __device__ __noinline__ bool scalar_pass(const MaskParams &p, const ScaleParams 
     return wrote;
 }
 
-constexpr int kMaskStages = 7;          // chunks in flight per streaming CTA
+constexpr int kMaskStages = 4;          // chunks in flight per streaming CTA
 constexpr int kMaskChunkMax = 1024;     // vectors (16 KB) per chunk and input
-constexpr size_t kMaskStreamSmem = (size_t)kMaskStages * 2 * kMaskChunkMax * 16;   // 224 KB
+constexpr size_t kMaskStreamSmem = (size_t)kMaskStages * 2 * kMaskChunkMax * 16;   // 128 KB
 constexpr long long kMaskCopyWait = 1ll << 31;   // bound of one chunk wait (about 1 s)
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
@@ -247,15 +250,11 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
     return true;
 }
 
-// Chunk i of this CTA (global chunk worker + i * nworkers) of both inputs into
-// stage i % kMaskStages; one thread issues it.
-__device__ __forceinline__ void issue_chunk(const MaskParams &p, uint8_t *stages, uint64_t *full, int worker,
-                                            int nworkers, int64_t i)
+// Chunk c of both inputs into stage st; one thread issues it.
+__device__ __forceinline__ void issue_chunk(const MaskParams &p, uint8_t *stages, uint64_t *full, int64_t c, int st)
 {
-    const int64_t c = worker + i * nworkers;
     const int64_t v0 = c * p.chunk;
     const uint32_t bytes = (uint32_t)(min((int64_t)p.chunk, p.nwork - v0) * 16);
-    const int st = (int)(i % kMaskStages);
     uint8_t *da = stages + (size_t)st * 2 * kMaskChunkMax * 16;
     uint8_t *db = da + (size_t)kMaskChunkMax * 16;
     const uint32_t bar = smem_addr(&full[st]);
@@ -270,38 +269,63 @@ __device__ __forceinline__ void issue_chunk(const MaskParams &p, uint8_t *stages
                  : "memory");
 }
 
-__device__ __forceinline__ int64_t chunks_of(const MaskParams &p, int worker, int nworkers)
+__device__ __forceinline__ int64_t chunk_count(const MaskParams &p) { return p.nchunks; }
+
+// The fixed first round of a streaming CTA (one thread; barriers
+// initialised): chunk worker + k * nworkers into stage k, -1 past the end.
+__device__ __forceinline__ void issue_first_chunks(const MaskParams &p, uint8_t *stages, uint64_t *full,
+                                                   int64_t *s_chunk, int worker, int nworkers)
 {
-    return p.chunks_base + (worker < p.chunks_rem ? 1 : 0);
+    const int64_t n = chunk_count(p);
+    for (int k = 0; k < kMaskStages; ++k) {
+        const int64_t c = worker + (int64_t)k * nworkers;
+        s_chunk[k] = c < n ? c : -1;
+        if (c < n)
+            issue_chunk(p, stages, full, c, k);
+    }
 }
 
-// The first copies of a streaming CTA (one thread; barriers initialised).
-__device__ __forceinline__ void issue_first_chunks(const MaskParams &p, uint8_t *stages, uint64_t *full, int worker,
-                                                   int nworkers)
+// Every streaming CTA takes from the work counter until a take returns a
+// chunk past the end, so a call makes exactly (chunks - dyn0) + workers takes
+// when dyn0 < chunks, none otherwise.  CTA 0 subtracts that number after the
+// last arrival instead of storing 0: a take still on its way to memory then
+// cannot leave the counter non-zero for the next call (subtraction and
+// addition commute), and the streaming CTAs need no fence for it.
+__device__ __forceinline__ void release_work_counter(const MaskParams &p, int nworkers)
 {
-    const int64_t mine = chunks_of(p, worker, nworkers);
-    for (int64_t i = 0; i < min(mine, (int64_t)kMaskStages); ++i)
-        issue_chunk(p, stages, full, worker, nworkers, i);
+    const int64_t n = chunk_count(p), dyn0 = (int64_t)kMaskStages * nworkers;
+    if (p.mode != 2 && dyn0 < n)
+        atomicSub(&p.hdr->next, (uint32_t)(n - dyn0 + nworkers));
 }
 
-// Stream this CTA's chunks through the stage ring and compare them.  The first
-// kMaskStages chunks were issued by issue_first_chunks.
+// Stream chunks through the stage ring and compare them: stage i mod 4 holds
+// chunk s_chunk[i mod 4] (-1: none; chunks are taken in increasing order, so
+// the first empty stage ends the stream).  Thread 0 refills a stage from the
+// counter once every thread is done with it, and asks for the index of the
+// refill after that right away, so the counter's round trip overlaps a
+// chunk's comparison.
 // Bitwise-equal 16-byte vectors cannot differ by more than a non-negative
 // threshold, so only vectors whose bytes differ get the exact float32 test.  Returns
 // whether this thread stored a flag; *ok turns false if a copy never landed
 // (then every copy still in flight has been waited for, boundedly).
 __device__ __forceinline__ bool phase1_bulk(const MaskParams &p, const MaskParams &sp, uint8_t *stages,
-                                            uint64_t *full, int worker, int nworkers, bool *ok)
+                                            uint64_t *full, int64_t *s_chunk, int nworkers, bool *ok)
 {
-    const int64_t mine = chunks_of(p, worker, nworkers);
+    const int64_t n = chunk_count(p), dyn0 = (int64_t)kMaskStages * nworkers;
+    int64_t pend = n;
+    if (threadIdx.x == 0 && dyn0 < n)
+        pend = dyn0 + (int64_t)atomicAdd(&p.hdr->next, 1u);
     bool wrote = false;
     *ok = true;
     int64_t i = 0;
-    for (; i < mine; ++i) {
+    for (;; ++i) {
         const int st = (int)(i % kMaskStages);
+        const int64_t c = s_chunk[st];
+        if (c < 0)
+            break;
         const bool landed = mbar_wait_bounded(smem_addr(&full[st]), (uint32_t)((i / kMaskStages) & 1));
         if (landed) {
-            const int64_t v0 = (worker + i * nworkers) * (int64_t)p.chunk;
+            const int64_t v0 = c * (int64_t)p.chunk;
             const int nv = (int)min((int64_t)p.chunk, p.nwork - v0);
             const uint4 *sa = reinterpret_cast<const uint4 *>(stages + (size_t)st * 2 * kMaskChunkMax * 16);
             const uint4 *sb = sa + kMaskChunkMax;
@@ -317,18 +341,28 @@ __device__ __forceinline__ bool phase1_bulk(const MaskParams &p, const MaskParam
                 }
             }
         }
-        // every thread is done with the stage before it is refilled
+        // every thread is done with the stage (and has read s_chunk) before
+        // it is refilled; the refill's s_chunk entry is read S iterations on,
+        // after at least one more of these barriers
         if (!__syncthreads_and(landed)) {
             *ok = false;
             break;
         }
-        if (threadIdx.x == 0 && i + kMaskStages < mine)
-            issue_chunk(p, stages, full, worker, nworkers, i + kMaskStages);
+        if (threadIdx.x == 0) {
+            if (pend < n) {
+                s_chunk[st] = pend;
+                issue_chunk(p, stages, full, pend, st);
+                pend = dyn0 + (int64_t)atomicAdd(&p.hdr->next, 1u);
+            } else {
+                s_chunk[st] = -1;
+            }
+        }
     }
     if (!*ok && threadIdx.x == 0) {
         // no copy may still be writing this CTA's shared memory when it exits
-        for (int64_t k = i; k < min(mine, i + kMaskStages); ++k)
-            mbar_wait_bounded(smem_addr(&full[k % kMaskStages]), (uint32_t)((k / kMaskStages) & 1));
+        for (int64_t k = i; k < i + kMaskStages; ++k)
+            if (s_chunk[k % kMaskStages] >= 0)
+                mbar_wait_bounded(smem_addr(&full[k % kMaskStages]), (uint32_t)((k / kMaskStages) & 1));
     }
     return wrote;
 }
@@ -486,8 +520,10 @@ __device__ __noinline__ void phase2(const MaskParams &p, const ScaleParams *sc, 
         const int warp = threadIdx.x >> 5;
         if (warp < p.n_scales)
             scale_small(p, sc[warp], warp, commit, reinterpret_cast<uint8_t *>(sdil) + warp * 1024);
-        if (commit && threadIdx.x == 0)
+        if (commit && threadIdx.x == 0) {
             p.hdr->arrive = 0;
+            release_work_counter(p, gridDim.x - 1);
+        }
         return;
     }
     const int n_scales = p.n_scales, D = p.dilate;
@@ -599,8 +635,10 @@ __device__ __noinline__ void phase2(const MaskParams &p, const ScaleParams *sc, 
 #pragma unroll 1
     for (int k = threadIdx.x; k < p.flag_bytes / 16; k += blockDim.x)
         reinterpret_cast<uint4 *>(p.flags)[k] = z;
-    if (threadIdx.x == 0)
+    if (threadIdx.x == 0) {
         p.hdr->arrive = 0;
+        release_work_counter(p, gridDim.x - 1);
+    }
 }
 
 // Default bound of CTA 0's wait for the streaming CTAs (about 4 s at 2 GHz);
@@ -621,6 +659,7 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask_reduce(const __grid_const
     extern __shared__ __align__(128) uint8_t dyn[];
     __shared__ MaskParams s_p;
     __shared__ __align__(8) uint64_t full[kMaskStages];
+    __shared__ int64_t s_chunk[kMaskStages];
     __shared__ int s_go;
     pdl_trigger();
     pdl_wait();   // the inputs, lists and workspace may come from the kernel before
@@ -629,7 +668,7 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask_reduce(const __grid_const
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&full[i])));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         if (blockIdx.x != 0 && p.mode != 2)
-            issue_first_chunks(p, dyn, full, blockIdx.x - 1, gridDim.x - 1);
+            issue_first_chunks(p, dyn, full, s_chunk, blockIdx.x - 1, gridDim.x - 1);
     }
     if (threadIdx.x < 32)
         copy_params(&s_p, p);
@@ -639,22 +678,30 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask_reduce(const __grid_const
         uint32_t *sbits = reinterpret_cast<uint32_t *>(dyn);
         uint32_t *sdil = sbits + kMaxWords;
         phase2(s_p, s_sc, false, sbits, sdil);
-        if (threadIdx.x == 0) {
+        // lane 0 of each warp polls the arrival counter, so the last arrival
+        // is seen within an eighth of a load round trip; the first to see it
+        // (or the first to give up) tells the others through shared memory
+        if (threadIdx.x == 0)
+            s_go = -1;
+        __syncthreads();
+        if ((threadIdx.x & 31) == 0) {
+            volatile int *go = &s_go;
             const uint32_t want = gridDim.x - 1;
             const long long t0 = clock64();
-            int go = 1;
-            while (ld_acquire_u32(&p.hdr->arrive) != want) {
-                if (clock64() - t0 > p.wait_cycles) {
-                    record_error(p.hdr, SIGE_ERR_TIMEOUT, -1);
-                    go = 0;
+            while (*go < 0) {
+                if (ld_acquire_u32(&p.hdr->arrive) == want) {
+                    *go = 1;
                     break;
                 }
-                __nanosleep(32);
+                if (clock64() - t0 > p.wait_cycles) {
+                    if (atomicCAS(&s_go, -1, 0) == -1)
+                        record_error(p.hdr, SIGE_ERR_TIMEOUT, -1);
+                    break;
+                }
             }
-            s_go = go;
         }
         __syncthreads();
-        if (s_go)
+        if (s_go == 1)
             phase2(s_p, s_sc, true, sbits, sdil);
         return;
     }
@@ -662,7 +709,7 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask_reduce(const __grid_const
     if (p.mode == 2)
         wrote = scalar_pass(s_p, s_sc, blockIdx.x - 1, gridDim.x - 1);
     else
-        wrote = phase1_bulk(p, s_p, dyn, full, blockIdx.x - 1, gridDim.x - 1, &ok);
+        wrote = phase1_bulk(p, s_p, dyn, full, s_chunk, gridDim.x - 1, &ok);
     if (!ok && threadIdx.x == 0)
         record_error(p.hdr, SIGE_ERR_TIMEOUT, -2);
     // The barrier orders every thread's flag stores before thread 0's fence,
@@ -858,9 +905,8 @@ static int reduce_mask_impl(const void *a_orig, const void *a_edit, const sige_t
         chunk = std::max<int64_t>(256, std::min<int64_t>(kMaskChunkMax, chunk));
         p.chunk = (int32_t)chunk;
         const int64_t nchunks = (p.nwork + chunk - 1) / chunk;
+        p.nchunks = (int32_t)nchunks;
         grid = 1 + (int)std::min<int64_t>(nchunks, workers_max);
-        p.chunks_base = (int32_t)(nchunks / (grid - 1));
-        p.chunks_rem = (int32_t)(nchunks % (grid - 1));
         smem = std::max(kMaskStreamSmem, 2 * kMaxWords * sizeof(uint32_t));
     }
     static std::atomic<int> attr_done[64];

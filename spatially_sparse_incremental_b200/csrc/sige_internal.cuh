@@ -20,7 +20,8 @@ struct WsHeader {
     int32_t error;        // first device error (a sige_status), 0 = none
     int32_t detail;       // call-specific detail of that error
     uint32_t arrive;      // "last CTA" arrival counter (self-resetting)
-    uint32_t pad[61];
+    uint32_t next;        // work counter of the mask's difference stream (self-resetting)
+    uint32_t pad[60];
 };
 static_assert(sizeof(WsHeader) == kWsHeader, "header size");
 

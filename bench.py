@@ -1069,12 +1069,43 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the area sweep, warm-L2 step and per-layer rows")
+    ap.add_argument("--row", choices=["attention", "gather_scatter", "mask"],
+                    help="time one component alone on one GPU and print its JSON (no headline line); "
+                         "a small, self-contained run for profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.row:
+        return run_row(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_sige(args)
+
+
+def run_row(args):
+    """One component of the extras, alone: the SD-latent attention step, the
+    unfused gather and scatter, or the mask reduction (its own graph, L2
+    flushed before each launch)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    stream = torch.cuda.Stream(device=dev)
+    flush = L2Flush(dev)
+    with torch.cuda.stream(stream):
+        if args.row == "attention":
+            r = attention_timing(args.seed, dev, flush, stream, peaks, reps=max(3, args.steps))
+        elif args.row == "gather_scatter":
+            r = gather_scatter_timing(args.seed, dev, flush, stream, peaks, reps=max(3, args.steps))
+        else:
+            d = make_workload(args.seed, dev)
+            g = capture(two_launch_calls(d, stream)["mask"], stream)
+            t = time_graph(g, flush, max(3, args.steps), stream)
+            us = float(np.median(t)) * 1e3
+            nbytes = 2 * d["x_orig"].numel() * d["x_orig"].element_size()
+            r = {"mask_us": us, "bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9,
+                 "frac": nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], "note": "graph time, launch included"}
+    print(json.dumps({"row": args.row, **r}))
+    return 0
 
 
 if __name__ == "__main__":

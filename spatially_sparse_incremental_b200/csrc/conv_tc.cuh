@@ -14,4 +14,8 @@ int tc_schedule(const sige_conv_desc *cd, int tiles, int grid, int csize, int32_
 bool conv8_supported(const sige_conv_desc *cd, int dtype);
 int launch_conv8(const ConvParams &p, cudaStream_t stream);
 
+// 1x1 stride-1 layers on any tile size (a GEMM over the gathered pixels).
+bool conv1x1_supported(const sige_conv_desc *cd, int dtype);
+int launch_conv1x1(const ConvParams &p, cudaStream_t stream);
+
 } // namespace sige

@@ -55,10 +55,11 @@ static int check_layer(const sige_conv_desc *cd, int dtype)
     return SIGE_OK;
 }
 
-// 1 = tensor-core kernel, 0 = CUDA-core kernel.
+// 1 = a tensor-core kernel runs the fused and dense calls of this layer,
+// 0 = the CUDA-core kernel.
 static int choose_path(const sige_conv_desc *cd, int dtype)
 {
-    return tc_supported(cd, dtype) ? 1 : 0;
+    return tc_supported(cd, dtype) || conv1x1_supported(cd, dtype) ? 1 : 0;
 }
 
 static size_t ws_need(const sige_conv_desc *cd, int batch, int ntiles)
@@ -80,9 +81,13 @@ static int run_conv(ConvParams &p, const sige_conv_desc *cd, void *ws, size_t ws
         return SIGE_ERR_WORKSPACE;
     if (ntiles == 0)
         return SIGE_OK;
-    if (choose_path(cd, p.dtype) == 1) {
-        // image to image, no GauGAN extension: the 8x8-tile kernel when it fits
-        if (conv8_supported(cd, p.dtype) && p.from_image && p.to_y && !p.tstride && !p.sg && !p.leaky)
+    // image to image, no GauGAN extension: the 8x8-tile kernel or the 1x1
+    // GEMM when they fit
+    const bool plain = p.from_image && p.to_y && !p.tstride && !p.sg && !p.leaky;
+    if (plain && conv1x1_supported(cd, p.dtype))
+        return launch_conv1x1(p, st);
+    if (tc_supported(cd, p.dtype)) {
+        if (plain && conv8_supported(cd, p.dtype))
             return launch_conv8(p, st);
         return launch_conv_tc(p, st);
     }

@@ -380,3 +380,51 @@ def test_conv8_odd_tile_count(orc, ntiles):
     L = inputs.make_conv_case(80 + ntiles, 32, 32, 64, 64, dtype=torch.bfloat16, block=8, gn=True)
     idx = np.array([(8, 8), (24, 0), (0, 24)][:ntiles], np.int32)
     _fused_vs_oracle(orc, L, idx, residual=True, seed=6)
+
+
+# ------------------------------------------------------------------ 1x1 layers (GEMM over gathered pixels)
+
+@pytest.mark.parametrize("H,W,ci,co,b,N,gn,res,area", [
+    (64, 128, 512, 256, 4, 1, False, False, 0.012),   # the GauGAN 1x1 layer's shape: two output-channel units
+    (36, 28, 128, 48, 4, 2, True, True, 0.08),        # ragged map, batch 2, C_out 48, GN + SiLU, residual
+    (32, 32, 64, 128, 8, 1, True, False, 0.05),       # 8x8 tiles: two per unit
+    (20, 20, 192, 64, 1, 1, False, True, 0.1),        # one-pixel tiles: 128 per unit
+    (30, 26, 64, 16, 3, 1, True, True, 0.1),          # 3x3 tiles: 14 per unit, two padding slots
+])
+def test_conv1x1_sparse(orc, H, W, ci, co, b, N, gn, res, area):
+    L = inputs.make_conv_case(90 + H + co + b, H, W, ci, co, dtype=torch.bfloat16, kernel=1, stride=1, pad=0,
+                              block=b, area=area, gn=gn, N=N)
+    assert sige.sige_conv_path(sige.conv_desc(1, 1, 0, ci, co, b), torch.bfloat16) == 1
+    _fused_vs_oracle(orc, L, _tiles(orc, L), residual=res, seed=7)
+
+
+@pytest.mark.parametrize("H,W,ci,co,b,N,gn,res", [
+    (64, 64, 256, 128, 4, 1, True, True),
+    (30, 26, 128, 256, 8, 2, False, False),
+])
+def test_conv1x1_dense(orc, H, W, ci, co, b, N, gn, res):
+    """Every tile of the map through sige_dense_conv (the same kernel)."""
+    L = inputs.make_conv_case(95 + H + co, H, W, ci, co, dtype=torch.bfloat16, kernel=1, stride=1, pad=0, block=b,
+                              gn=gn, N=N)
+    g, gs, gh = _gn(orc, L)
+    r = random_cache((N, H, W, co), torch.bfloat16, 5) if res else None
+    every = np.array([(h, w) for h in range(0, H, b) for w in range(0, W, b)], np.int32)
+    ref = orc.sparse_conv(L.x_orig, L.weight, L.bias, every, torch.zeros((N, H, W, co), dtype=torch.bfloat16),
+                          1, 1, 0, b, gn=g, silu=gn, residual=r)
+    cd = sige.conv_desc(1, 1, 0, ci, co, b)
+    y = sige.sige_dense_conv(L.x_orig.to(DEV), L.weight.to(DEV), L.bias.to(DEV), cd, gn_scale=gs, gn_shift=gh,
+                             silu=gn, residual=None if r is None else r.to(DEV))
+    torch.cuda.synchronize()
+    assert_close(y.cpu(), ref, torch.bfloat16)
+
+
+def test_conv1x1_empty_list_writes_nothing(orc):
+    L = inputs.make_conv_case(98, 16, 16, 64, 64, dtype=torch.bfloat16, kernel=1, stride=1, pad=0, block=4)
+    cache = random_cache((1, 16, 16, 64), torch.bfloat16, 8)
+    cd = sige.conv_desc(1, 1, 0, 64, 64, 4)
+    di = torch.zeros((16, 2), dtype=torch.int32, device=DEV)
+    dc = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y = cache.to(DEV)
+    sige.sige_conv_fused(L.x_edit.to(DEV), L.weight.to(DEV), L.bias.to(DEV), cd, di, dc, 16, y)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(y.cpu()), bits(cache))

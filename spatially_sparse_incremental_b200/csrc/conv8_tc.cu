@@ -62,6 +62,7 @@ constexpr uint32_t kOffA = 1024;
 constexpr uint32_t kOffS = kOffA + 2 * kABuf;
 constexpr uint32_t kOffW = ((kOffS + kStageS + 1023) / 1024) * 1024;
 constexpr uint32_t kSmemLimit = 232448;
+constexpr uint32_t kEpiBias = kMaxN * 4;    // per epilogue warp: a copy of the bias
 constexpr int kMaxStages = 8;
 // control words
 constexpr uint32_t kBarWFull = 0, kBarWEmpty = 64, kBarSFull = 128, kBarSEmpty = 136, kBarAFull = 144,
@@ -517,7 +518,16 @@ __global__ void __launch_bounds__(c8::kThreads, 1)
         const int row = sp * 32 + lane;                  // accumulator row
         const int oi = row >> 3, oj = row & 7;           // output row / column within the accumulator
         const uint32_t t_lane = tmem + ((uint32_t)(sp * 32) << 16);
+        // this warp's copy of the bias: a global load per 32 columns would sit
+        // behind the tensor-memory wait (a memory clobber) and cost a round
+        // trip each time
+        const float4 *bsm = reinterpret_cast<const float4 *>(smem + kOffW + (uint32_t)p.stages * p.stage_bytes +
+                                                             (uint32_t)(warp - 10) * kEpiBias);
         pdl_wait();
+        for (int c = lane * 4; c < NC; c += 128)
+            const_cast<float4 *>(bsm)[c / 4] =
+                p.bias ? __ldg(reinterpret_cast<const float4 *>(p.bias + c)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        __syncwarp();
         const int units = p.dense ? ((p.th + 3) / 4) * p.tw * p.N : (min(__ldg(p.count), p.cap) * p.N + 1) / 2;
         bool ok = true;
         uint32_t k = 0;
@@ -544,23 +554,25 @@ __global__ void __launch_bounds__(c8::kThreads, 1)
                     continue;
 #pragma unroll 1
                 for (int c0 = 0; c0 < NC; c0 += 32) {
+                    // the slice's residual is requested before the tensor-memory
+                    // load, so that its round trip overlaps the load and wait
+                    const uint4 *res = p.residual && valid
+                                           ? reinterpret_cast<const uint4 *>(p.residual + (e + c0) * 2)
+                                           : nullptr;
+                    uint4 rq[4];
+#pragma unroll
+                    for (int g8 = 0; g8 < 4; ++g8)
+                        rq[g8] = res ? __ldg(res + g8) : make_uint4(0, 0, 0, 0);
                     float v[32];
                     c8_tmem_ld32(t_lane + tcol + (uint32_t)c0, v);
                     if (!valid)
                         continue;
                     uint4 *dst = reinterpret_cast<uint4 *>(p.y + (e + c0) * 2);
-                    const uint4 *res = p.residual ? reinterpret_cast<const uint4 *>(p.residual + (e + c0) * 2)
-                                                  : nullptr;
 #pragma unroll
                     for (int g8 = 0; g8 < 4; ++g8) {
-                        float bb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                        if (p.bias) {
-                            const float4 b0 = __ldg(reinterpret_cast<const float4 *>(p.bias + c0 + 8 * g8));
-                            const float4 b1 = __ldg(reinterpret_cast<const float4 *>(p.bias + c0 + 8 * g8 + 4));
-                            bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w;
-                            bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
-                        }
-                        uint4 rr = res ? __ldg(res + g8) : make_uint4(0, 0, 0, 0);
+                        const float4 b0 = bsm[(c0 + 8 * g8) / 4], b1 = bsm[(c0 + 8 * g8) / 4 + 1];
+                        const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                        const uint4 rr = rq[g8];
                         const uint32_t *rw = reinterpret_cast<const uint32_t *>(&rr);
                         uint32_t o[4];
 #pragma unroll
@@ -649,7 +661,7 @@ int launch_conv8(const ConvParams &cp, cudaStream_t stream)
     a.tw = (cp.Wo + 7) / 8;
     a.silu = cp.silu;
     a.stage_bytes = (uint32_t)cp.Cout * 128u;
-    const uint32_t room = kSmemLimit - 1024 - kOffW;
+    const uint32_t room = kSmemLimit - 1024 - kOffW - 4 * kEpiBias;
     a.stages = (int)std::min<uint32_t>(kMaxStages, room / a.stage_bytes);
     if (a.stages < 2)
         return SIGE_ERR_UNSUPPORTED;
@@ -659,7 +671,7 @@ int launch_conv8(const ConvParams &cp, cudaStream_t stream)
     while (tc < (a.dbuf ? 2 * cols : cols))
         tc <<= 1;
     a.tmem_cols = tc;
-    const size_t smem = kOffW + (size_t)a.stages * a.stage_bytes + 1024;
+    const size_t smem = kOffW + (size_t)a.stages * a.stage_bytes + 4 * kEpiBias + 1024;
     static std::atomic<int> attr_set[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)

@@ -6,14 +6,18 @@
 // 1x1 conv needs no halo, so the gather is a row gather.)
 //
 // A unit is 128 pixel slots (slot s = pixel s mod b^2 of the (tile, batch
-// item) pair s / b^2, 128 / b^2 pairs per unit; clipped pixels and slots past
-// the list are zero rows that are not written) times up to 128 output
-// channels:
-//   * warps 4..7, one slot per thread, copy their pixel's 64-channel chunks
-//     with cp.async straight into the 128-byte-swizzled K-major A layout (row
-//     = slot, 128 bytes = 64 channels; zero fill outside the map), seven of
-//     eight stages in flight (a 512-channel unit is requested at once), apply GroupNorm + SiLU in place when asked, then run the
-//     epilogue from tensor memory (bias, residual, bf16);
+// item) pair s / b^2, 128 / b^2 pairs per unit; rows of clipped pixels are
+// zero, slots past the list are computed and not written) times up to 128
+// output channels:
+//   * A, for b = 4 or 8: warp 2 loads one TMA box of 64 channels x b x b
+//     pixels per (tile, item) and chunk, which lands as that pair's b^2 rows
+//     of the 128-byte-swizzled K-major A layout (row = slot, 128 bytes = 64
+//     channels; zero outside the map); other tile sizes: warps 4..7, one slot
+//     per thread, copy their pixel's chunks with cp.async straight into the
+//     same layout, seven of eight stages in flight;
+//   * warps 4..7 apply GroupNorm + SiLU to their row in place when asked, hand
+//     the stage to the MMAs, and run the epilogue from tensor memory (bias,
+//     residual, bf16);
 //   * warp 0 loads the weights [C_out][C_in] by TMA (64 channels x the unit's
 //     output channels per stage, 128-byte swizzle), four stages;
 //   * warp 1 issues D += A W^T (M 128 slots, N the unit's output channels,
@@ -39,11 +43,12 @@ constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffW = kOffA + kAStages * kABytes;
 constexpr uint32_t kOffBias = kOffW + kWStages * kWBytes;  // per rows warp: the unit's bias (kMaxNT floats)
 constexpr uint32_t kOffBar = kOffBias + 4 * kMaxNT * 4;
-constexpr uint32_t kBarAFull = 0, kBarAEmpty = kBarAFull + 8 * kAStages, kBarWFull = kBarAEmpty + 8 * kAStages,
-                   kBarWEmpty = kBarWFull + 8 * kWStages, kBarAccFull = kBarWEmpty + 8 * kWStages,
-                   kBarAccEmpty = kBarAccFull + 8, kTmemSlot = kBarAccEmpty + 8, kAbort = kTmemSlot + 4;
-static_assert(kAbort + 4 <= 256, "barrier block");
-constexpr uint32_t kSmem = kOffBar + 256 + 1024;          // + alignment slack
+constexpr uint32_t kBarAFull = 0, kBarAEmpty = kBarAFull + 8 * kAStages, kBarALand = kBarAEmpty + 8 * kAStages,
+                   kBarWFull = kBarALand + 8 * kAStages, kBarWEmpty = kBarWFull + 8 * kWStages,
+                   kBarAccFull = kBarWEmpty + 8 * kWStages, kBarAccEmpty = kBarAccFull + 8,
+                   kTmemSlot = kBarAccEmpty + 8, kAbort = kTmemSlot + 4;
+static_assert(kAbort + 4 <= 512, "barrier block");
+constexpr uint32_t kSmem = kOffBar + 512 + 1024;          // + alignment slack
 
 enum : int { kSiteWEmpty = 301, kSiteWFull, kSiteAFull, kSiteAEmpty, kSiteAccFull, kSiteAccEmpty };
 
@@ -61,7 +66,16 @@ struct Args {
     uint8_t *y;                // NHWC bf16 [N][H][W][Cout]
     WsHeader *hdr;
     uint32_t tmem_cols;
+    int32_t tma_a;             // A by one TMA per (tile, chunk) (b^2 rows fill whole 1 KB swizzle atoms)
 };
+
+__device__ __forceinline__ void tma4(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1, int c2, int c3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
 {
@@ -99,7 +113,8 @@ __device__ __forceinline__ void mma_w(uint32_t d, uint64_t a, uint64_t b, uint32
 using namespace g1;
 
 __global__ void __launch_bounds__(g1::kThreads, 1)
-    k_conv1x1(const __grid_constant__ g1::Args p, const __grid_constant__ CUtensorMap tw)
+    k_conv1x1(const __grid_constant__ g1::Args p, const __grid_constant__ CUtensorMap tw,
+              const __grid_constant__ CUtensorMap tx)
 {
     extern __shared__ __align__(1024) uint8_t g1_raw[];
     const uint32_t raw = smem_u32(g1_raw);
@@ -111,6 +126,7 @@ __global__ void __launch_bounds__(g1::kThreads, 1)
     WsHeader *hdr = p.hdr;
     auto a_full = [&](int i) { return bar + kBarAFull + 8u * i; };
     auto a_empty = [&](int i) { return bar + kBarAEmpty + 8u * i; };
+    auto a_land = [&](int i) { return bar + kBarALand + 8u * i; };
     auto w_full = [&](int i) { return bar + kBarWFull + 8u * i; };
     auto w_empty = [&](int i) { return bar + kBarWEmpty + 8u * i; };
 
@@ -125,6 +141,7 @@ __global__ void __launch_bounds__(g1::kThreads, 1)
         for (int i = 0; i < kAStages; ++i) {
             mbar_init(a_full(i), kRows);
             mbar_init(a_empty(i), 1);
+            mbar_init(a_land(i), 1);
         }
         for (int i = 0; i < kWStages; ++i) {
             mbar_init(w_full(i), 1);
@@ -135,8 +152,11 @@ __global__ void __launch_bounds__(g1::kThreads, 1)
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0 && lane == 0)
+    if (warp == 0 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tw)) : "memory");
+        if (p.tma_a)
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tx)) : "memory");
+    }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(bar + kTmemSlot),
                      "r"(p.tmem_cols));
@@ -189,6 +209,46 @@ __global__ void __launch_bounds__(g1::kThreads, 1)
             }
             if (ok)
                 tc_commit_w(bar + kBarAccFull);
+        }
+    } else if (warp == 2 && p.tma_a) {
+        // ---- A by TMA: per chunk, one box of 64 channels x b x b pixels per
+        // (tile, item) of the unit (lane q: pair q), landing as that pair's b^2
+        // swizzled rows; zero outside the map.  Rows of pairs past the list
+        // stay as they are: their outputs are not written.
+        int ia = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
+            const int blk = u / p.ntn;
+            const int64_t T = (int64_t)blk * tpb + lane;
+            const bool tv = lane < tpb && T < items;
+            int n = 0, h0 = 0, w0 = 0;
+            if (tv) {
+                const int t = (int)(T / p.N);
+                n = (int)(T - (int64_t)t * p.N);
+                if (p.dense) {
+                    h0 = (t / p.tiles_w) * p.b;
+                    w0 = (t % p.tiles_w) * p.b;
+                } else {
+                    const int2 o = __ldg(reinterpret_cast<const int2 *>(p.idx) + t);
+                    h0 = o.x;
+                    w0 = o.y;
+                }
+            }
+            const uint32_t bytes = (uint32_t)__popc(__ballot_sync(0xFFFFFFFFu, tv)) * (uint32_t)bb * 128u;
+            for (int kc = 0; kc < kcn; ++kc) {
+                const int g = ia + kc, st = g % kAStages;
+                if (g >= kAStages &&
+                    !mbar_wait_w(a_empty(st), ((g / kAStages) - 1) & 1, abort_flag, hdr, kSiteAEmpty)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0)
+                    mbar_expect_tx(a_land(st), bytes);
+                __syncwarp();
+                if (tv)
+                    tma4(sb + kOffA + st * kABytes + (uint32_t)(lane * bb) * 128u, &tx, a_land(st), kc * 64, w0, h0, n);
+            }
+            ia += kcn;
         }
     } else if (warp >= 4) {
         // ---- pixel rows (A) and the epilogue; thread = slot r = TMEM lane r
@@ -247,14 +307,42 @@ __global__ void __launch_bounds__(g1::kThreads, 1)
                                  : "memory");
                 __syncwarp();
             }
-            for (int j = 0; j < kAStages - 1; ++j) {
+            for (int j = 0; !p.tma_a && j < kAStages - 1; ++j) {
                 if (j < kcn && !issue(j)) {
                     ok = false;
                     break;
                 }
                 cp_async_commit();
             }
-            for (int kc = 0; ok && kc < kcn; ++kc) {
+            for (int kc = 0; p.tma_a && ok && kc < kcn; ++kc) {
+                // A landed by TMA: GroupNorm + SiLU of this row in place when
+                // asked, then hand the stage to the MMAs
+                const int g = ia + kc, st = g % kAStages;
+                if (!mbar_wait_w(a_land(st), (g / kAStages) & 1, abort_flag, hdr, kSiteAFull)) {
+                    ok = false;
+                    break;
+                }
+                if (transform && valid) {
+                    const uint32_t row = sb + kOffA + st * kABytes + (uint32_t)r * 128u;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t a = row + ((uint32_t)(c ^ (r & 7)) << 4);
+                        uint4 v;
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                     : "r"(a));
+                        const int c0 = kc * 64 + c * 8;
+                        v = transform16(v, SIGE_BF16, affine ? p.gsc + (int64_t)n * p.Cin + c0 : nullptr,
+                                        affine ? p.gsh + (int64_t)n * p.Cin + c0 : nullptr, p.silu);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y),
+                                     "r"(v.z), "r"(v.w)
+                                     : "memory");
+                    }
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(a_full(st));
+            }
+            for (int kc = 0; !p.tma_a && ok && kc < kcn; ++kc) {
                 // chunk kc first (its group is the oldest of the seven in
                 // flight), then the refill of the stage the MMAs of chunk kc - 1
                 // release: chunk kc never waits for an MMA
@@ -395,6 +483,24 @@ int launch_conv1x1(const ConvParams &cp, cudaStream_t stream)
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return SIGE_ERR_UNSUPPORTED;
+    // the input [N][H][W][C_in] as a 4-d map: a box of 64 channels x b x b
+    // pixels of one item lands as the tile's b^2 rows of 128 bytes, 128-byte
+    // swizzle, zero outside the map.  Used when b^2 rows fill whole 1 KB
+    // swizzle atoms (b = 4 or 8), so that every box starts on an atom.
+    CUtensorMap tx = tw;
+    a.tma_a = 0;
+    if ((cp.b * cp.b) % 8 == 0) {
+        cuuint64_t xd[4] = {(cuuint64_t)cp.Cin, (cuuint64_t)cp.W, (cuuint64_t)cp.H, (cuuint64_t)cp.N};
+        cuuint64_t xs[3] = {(cuuint64_t)cp.Cin * 2, (cuuint64_t)cp.W * cp.Cin * 2, (cuuint64_t)cp.H * cp.W * cp.Cin * 2};
+        cuuint32_t xb[4] = {64, (cuuint32_t)cp.b, (cuuint32_t)cp.b, 1};
+        cuuint32_t xe[4] = {1, 1, 1, 1};
+        if (encode(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint8_t *>(cp.src), xd, xs, xb, xe,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+            a.tma_a = 1;
+        else
+            tx = tw;
+    }
     static std::atomic<int> attr_set[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
@@ -412,7 +518,7 @@ int launch_conv1x1(const ConvParams &cp, cudaStream_t stream)
     if (units_max > INT32_MAX)
         return SIGE_ERR_INVALID_ARG;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(units_max, device_sm_count()));
-    if (launch_pdl(k_conv1x1, dim3(grid), dim3(g1::kThreads), g1::kSmem, stream, a, tw) != cudaSuccess)
+    if (launch_pdl(k_conv1x1, dim3(grid), dim3(g1::kThreads), g1::kSmem, stream, a, tw, tx) != cudaSuccess)
         return SIGE_ERR_CUDA;
     count_launch();
     return launch_check();

@@ -456,31 +456,7 @@ def measure_extras(dev, flush, stream, peaks, seed, step_graph):
     out["pixel_dilation_step"] = {"radius_px": 2, "active_tiles": tiles_px, "step_us": float(np.median(t)) * 1e3}
     del g, d
 
-    layers = [("fp32 64x64 C64 3x3 b4", inputs.make_cfg1(seed), 32)]
-    for i, (h, w, c, b) in enumerate(inputs.CFG4_LAYERS):
-        layers.append((f"SD latent {h}x{w} C{c} 3x3 b{b}", inputs.make_cfg4_layer(seed, i), 16))
-    for i, (h, w, ci, co, k, st, b) in enumerate(inputs.CFG5_LAYERS):
-        layers.append((f"GauGAN {h}x{w} {ci}->{co} {k}x{k} s{st} b{b}", inputs.make_cfg5_layer(seed, i), 16))
-    rows = []
-    for name, L, bits in layers:
-        try:
-            rows.append(dict(name=name, **layer_timing(L, bits, dev, flush, stream, peaks)))
-        except Exception as e:   # a failing row is reported, not fatal to the headline line
-            rows.append({"name": name, "error": str(e)[:200]})
-    for i, (h, w, ci, co, b) in enumerate(inputs.UPSAMPLE_LAYERS):
-        name = f"GauGAN upsample {h}x{w}->{2 * h}x{2 * w} {ci}->{co} 3x3 transposed s2 b{b}"
-        try:
-            rows.append(dict(name=name, **ext_layer_timing(inputs.make_upsample_layer(seed, i), dev, flush, stream,
-                                                           peaks, transposed=True)))
-        except Exception as e:
-            rows.append({"name": name, "error": str(e)[:200]})
-    for i, (h, w, ci, co, b) in enumerate(inputs.SPADE_LAYERS):
-        name = f"GauGAN SPADE {h}x{w} {ci}->{co} 3x3 b{b} LeakyReLU"
-        try:
-            rows.append(dict(name=name, **ext_layer_timing(inputs.make_spade_layer(seed, i), dev, flush, stream,
-                                                           peaks, spade=True)))
-        except Exception as e:
-            rows.append({"name": name, "error": str(e)[:200]})
+    rows = layer_rows(seed, dev, flush, stream, peaks)
     try:
         out["attention"] = attention_timing(seed, dev, flush, stream, peaks)
     except Exception as e:
@@ -510,6 +486,38 @@ def measure_extras(dev, flush, stream, peaks, seed, step_graph):
     out["layer_sweeps"] = srows
     out["layers"] = rows
     return out
+
+
+def layer_rows(seed, dev, flush, stream, peaks):
+    """Every per-layer workload at its default edit: one fused call, sparse
+    and dense, each in its own CUDA graph with L2 flushed."""
+    from spatially_sparse_incremental_b200 import inputs
+    layers = [("fp32 64x64 C64 3x3 b4", inputs.make_cfg1(seed), 32)]
+    for i, (h, w, c, b) in enumerate(inputs.CFG4_LAYERS):
+        layers.append((f"SD latent {h}x{w} C{c} 3x3 b{b}", inputs.make_cfg4_layer(seed, i), 16))
+    for i, (h, w, ci, co, k, st, b) in enumerate(inputs.CFG5_LAYERS):
+        layers.append((f"GauGAN {h}x{w} {ci}->{co} {k}x{k} s{st} b{b}", inputs.make_cfg5_layer(seed, i), 16))
+    rows = []
+    for name, L, bits in layers:
+        try:
+            rows.append(dict(name=name, **layer_timing(L, bits, dev, flush, stream, peaks)))
+        except Exception as e:   # a failing row is reported, not fatal to the headline line
+            rows.append({"name": name, "error": str(e)[:200]})
+    for i, (h, w, ci, co, b) in enumerate(inputs.UPSAMPLE_LAYERS):
+        name = f"GauGAN upsample {h}x{w}->{2 * h}x{2 * w} {ci}->{co} 3x3 transposed s2 b{b}"
+        try:
+            rows.append(dict(name=name, **ext_layer_timing(inputs.make_upsample_layer(seed, i), dev, flush, stream,
+                                                           peaks, transposed=True)))
+        except Exception as e:
+            rows.append({"name": name, "error": str(e)[:200]})
+    for i, (h, w, ci, co, b) in enumerate(inputs.SPADE_LAYERS):
+        name = f"GauGAN SPADE {h}x{w} {ci}->{co} 3x3 b{b} LeakyReLU"
+        try:
+            rows.append(dict(name=name, **ext_layer_timing(inputs.make_spade_layer(seed, i), dev, flush, stream,
+                                                           peaks, spade=True)))
+        except Exception as e:
+            rows.append({"name": name, "error": str(e)[:200]})
+    return rows
 
 
 def gather_scatter_timing(seed, dev, flush, stream, peaks, reps=30):
@@ -1069,7 +1077,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the area sweep, warm-L2 step and per-layer rows")
-    ap.add_argument("--row", choices=["attention", "gather_scatter", "mask"],
+    ap.add_argument("--row", choices=["attention", "gather_scatter", "mask", "layers"],
                     help="time one component alone on one GPU and print its JSON (no headline line); "
                          "a small, self-contained run for profiling")
     args = ap.parse_args()
@@ -1094,6 +1102,8 @@ def run_row(args):
     with torch.cuda.stream(stream):
         if args.row == "attention":
             r = attention_timing(args.seed, dev, flush, stream, peaks, reps=max(3, args.steps))
+        elif args.row == "layers":
+            r = {"layers": layer_rows(args.seed, dev, flush, stream, peaks)}
         elif args.row == "gather_scatter":
             r = gather_scatter_timing(args.seed, dev, flush, stream, peaks, reps=max(3, args.steps))
         else:

@@ -14,8 +14,10 @@ int tc_schedule(const sige_conv_desc *cd, int tiles, int grid, int csize, int32_
 bool conv8_supported(const sige_conv_desc *cd, int dtype);
 int launch_conv8(const ConvParams &p, cudaStream_t stream);
 
-// 1x1 stride-1 layers on any tile size (a GEMM over the gathered pixels).
-bool conv1x1_supported(const sige_conv_desc *cd, int dtype);
-int launch_conv1x1(const ConvParams &p, cudaStream_t stream);
+// 1x1 and 3x3 "same" stride-1 layers on any tile size: a GEMM over the
+// tiles' pixels, one tap-shifted copy of the tile per K chunk, K split across
+// a cluster when the units are few.
+bool tile_gemm_supported(const sige_conv_desc *cd, int dtype);
+int launch_tile_gemm(const ConvParams &p, cudaStream_t stream);
 
 } // namespace sige

@@ -59,7 +59,7 @@ static int check_layer(const sige_conv_desc *cd, int dtype)
 // 0 = the CUDA-core kernel.
 static int choose_path(const sige_conv_desc *cd, int dtype)
 {
-    return tc_supported(cd, dtype) || conv1x1_supported(cd, dtype) ? 1 : 0;
+    return tc_supported(cd, dtype) || tile_gemm_supported(cd, dtype) ? 1 : 0;
 }
 
 static size_t ws_need(const sige_conv_desc *cd, int batch, int ntiles)
@@ -84,13 +84,12 @@ static int run_conv(ConvParams &p, const sige_conv_desc *cd, void *ws, size_t ws
     // image to image, no GauGAN extension: the 8x8-tile kernel or the 1x1
     // GEMM when they fit
     const bool plain = p.from_image && p.to_y && !p.tstride && !p.sg && !p.leaky;
-    if (plain && conv1x1_supported(cd, p.dtype))
-        return launch_conv1x1(p, st);
-    if (tc_supported(cd, p.dtype)) {
-        if (plain && conv8_supported(cd, p.dtype))
-            return launch_conv8(p, st);
+    if (plain && conv8_supported(cd, p.dtype))
+        return launch_conv8(p, st);
+    if (plain && tile_gemm_supported(cd, p.dtype))
+        return launch_tile_gemm(p, st);
+    if (tc_supported(cd, p.dtype))
         return launch_conv_tc(p, st);
-    }
     return launch_conv_simt(p, st);
 }
 

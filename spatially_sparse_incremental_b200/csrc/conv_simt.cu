@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(kSimtThreads) k_conv_simt(const __grid_constan
 constexpr int kS16Threads = 256;
 constexpr int kS16Cout = 64;            // output channels per unit
 constexpr int kS16WStride = kS16Cout + 4;   // weight row stride (floats): 16-byte aligned, fewer bank conflicts
-constexpr int kS16SmemFloats = 16384;   // 64 KB
+constexpr int kS16SmemFloats = 24576;   // 96 KB: two CTAs per SM, fewer channel chunks
 
 __global__ void __launch_bounds__(kS16Threads, 1) k_conv_simt16(const __grid_constant__ ConvParams p)
 {
@@ -315,21 +315,29 @@ __global__ void __launch_bounds__(kS16Threads, 1) k_conv_simt16(const __grid_con
             // (converted on the way): kStageBatch rows in flight per warp.
             const int nrow = kS16Cout * taps;
             if (p.dtype == SIGE_F32) {
+                // (row = col * taps + tap, stepped without a division: the
+                // issue loop, not the copies, bounded this staging)
                 const float *wg = reinterpret_cast<const float *>(p.w);
+                int col = warp / taps, tap = warp - col * taps;
 #pragma unroll 1
                 for (int row = warp; row < nrow; row += nwarp) {
-                    const int col = row / taps, tap = row - col * taps;
                     const int o2 = cog * kS16Cout + col;
+                    const float *src = wg + ((int64_t)o2 * taps + tap) * p.Cin + ci0;
+                    float *dst = sw + tap * cc * kS16WStride + col;
 #pragma unroll 1
                     for (int ci = lane; ci < cc; ci += 32) {
-                        float *dst = sw + (tap * cc + ci) * kS16WStride + col;
                         if (o2 < p.Cout)
                             asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
-                                             static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-                                         "l"(wg + ((int64_t)o2 * taps + tap) * p.Cin + ci0 + ci)
+                                             static_cast<uint32_t>(__cvta_generic_to_shared(dst + ci * kS16WStride))),
+                                         "l"(src + ci)
                                          : "memory");
                         else
-                            *dst = 0.0f;
+                            dst[ci * kS16WStride] = 0.0f;
+                    }
+                    tap += nwarp;
+                    while (tap >= taps) {
+                        tap -= taps;
+                        ++col;
                     }
                 }
             } else
@@ -440,7 +448,7 @@ static int pow2_ceil(int v)
 static int launch_conv_simt16(ConvParams p, cudaStream_t stream)
 {
     const int npix = p.bin * p.bin, taps = p.k * p.k;
-    // one chunk of channels: halo block + weights, within 64 KB (the K-group
+    // one chunk of channels: halo block + weights, within 96 KB (the K-group
     // sums of the end reuse the same space)
     const int per_ci = npix + taps * kS16WStride;
     p.ci_chunk = std::min(p.Cin, (kS16SmemFloats - 4) / per_ci);

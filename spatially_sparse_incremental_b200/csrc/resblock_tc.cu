@@ -118,6 +118,29 @@ enum : int { kSiteWEmpty = 101, kSiteWFull, kSiteXReady, kSiteAcc1Empty, kSiteAc
 
 }  // namespace rb
 
+// Division of 32-bit values by a divisor fixed for the launch: a multiply-high
+// and two shifts (Granlund and Montgomery, "Division by invariant integers
+// using multiplication", 1994, the unsigned case), for the difference stream's
+// pixel -> (row, column) mapping.
+struct UDiv {
+    uint32_t m, s1, s2;
+};
+
+static inline UDiv udiv_make(uint32_t d)   // 1 <= d <= 2^31
+{
+    uint32_t l = 0;
+    while (l < 32 && (1ull << l) < d)
+        ++l;                                   // ceil(log2 d)
+    const uint64_t m = ((((uint64_t)1 << l) - d) << 32) / d + 1;
+    return UDiv{(uint32_t)m, l < 1 ? l : 1u, l > 1 ? l - 1 : 0u};
+}
+
+__device__ __forceinline__ uint32_t udiv(uint32_t n, UDiv f)
+{
+    const uint32_t t = __umulhi(n, f.m);
+    return (t + ((n - t) >> f.s1)) >> f.s2;
+}
+
 struct RbArgs {
     const uint8_t *x;           // x_edit, NHWC bf16 [N][H][W][128]
     const int32_t *idx;         // tile origins (h0, w0)
@@ -140,6 +163,8 @@ struct RbArgs {
     unsigned long long *ctr;    // grid-barrier arrivals in the workspace header (only grows)
     unsigned long long *chunk_ctr;   // difference-stream chunks handed out (workspace header, only grows)
     long long grid_wait;        // bound of the grid barrier's wait, in clocks (sige_set_wait_cycles, else ~1 s)
+    UDiv div_hw, div_w;         // by H * W and by W, when every pixel index fits 32 bits (fast_px)
+    int32_t fast_px;
 };
 
 // Four K=16 MMAs of one 64-channel weight stage: A (pixels, no swizzle)
@@ -465,9 +490,19 @@ __device__ __forceinline__ int rb_step_list(const RbArgs &p, uint8_t *smem, vola
                     if (i < n) {
                         const uint4 va = so[i], vb = se[i];
                         if (((va.x ^ vb.x) | (va.y ^ vb.y) | (va.z ^ vb.z) | (va.w ^ vb.w)) && rb_exceeds(va, vb, p.thr)) {
-                            const int64_t pix = (a + i) >> 4;   // 16 vectors per pixel
-                            const int64_t hw = pix % ((int64_t)H * W);
-                            const int y = (int)(hw / W), x = (int)(hw - (int64_t)y * W);
+                            int y, x;
+                            if (p.fast_px) {
+                                const uint32_t pix = (uint32_t)((a + i) >> 4);   // 16 vectors per pixel
+                                const uint32_t hw = pix - udiv(pix, p.div_hw) * ((uint32_t)H * (uint32_t)W);
+                                const uint32_t yq = udiv(hw, p.div_w);
+                                y = (int)yq;
+                                x = (int)(hw - yq * (uint32_t)W);
+                            } else {
+                                const int64_t pix = (a + i) >> 4;
+                                const int64_t hw = pix % ((int64_t)H * W);
+                                y = (int)(hw / W);
+                                x = (int)(hw - (int64_t)y * W);
+                            }
                             const int t = (y >> 3) * tw + (x >> 3);
                             if (t != last) {
                                 p.flags[t] = epoch;
@@ -1497,5 +1532,11 @@ extern "C" int sige_resblock_step(const void *x_orig, const void *x_edit, const 
     a.chunk_ctr = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + 24);
     a.grid_wait = wait_cycles_or(kWaitCycles);
     a.flags = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kWsHeader);
+    const uint64_t pixels = (uint64_t)xd->n * xd->h * xd->w;
+    a.fast_px = pixels <= 0xFFFFFFFFull && (uint64_t)xd->h * xd->w <= (1ull << 31) ? 1 : 0;
+    if (a.fast_px) {
+        a.div_hw = udiv_make((uint32_t)(xd->h * xd->w));
+        a.div_w = udiv_make((uint32_t)xd->w);
+    }
     return rb_launch<true>(a, tmx, tw1, tw2, (int64_t)capacity * xd->n, stream);
 }

@@ -108,6 +108,7 @@ struct TcArgs {
     int32_t num_sms;
     int32_t halo_tma;         // 1: ROW-mode halo rows come by TMA (tmx), 0: per-thread cp.async
     int32_t pair;             // 1: launched in clusters (of csize CTAs)
+    UDiv dN, dbin, db;        // division by N, bin and b in the per-element loops
     int32_t csize;            // CTAs per cluster (1: no clusters).  csize 2: a 2-way K split of
                               // a unit of <= 64 columns is summed through the peer's shared
                               // memory; other splits that divide csize reduce-scatter within
@@ -129,6 +130,7 @@ __device__ __forceinline__ void tile_origin_a(const TcArgs &a, int t, int &h0, i
 // ------------------------------------------------------------------ schedule
 
 struct Sched {
+    UDiv dT;    // division by T
     int T;      // tiles per unit (POS: slots, multiple of 16)
     int TB;     // tile groups
     int S;      // K splits
@@ -149,6 +151,7 @@ __host__ __device__ inline Sched make_sched_for(int mode, int T_max, int MT, int
     else
         s.T = min(T_max, ((want + 15) / 16) * 16);
     s.TB = (G + s.T - 1) / s.T;
+    s.dT = udiv_make((uint32_t)s.T);
     // split K only where each split keeps a long K loop: below that the extra
     // round trip of the partial sums costs more than the shorter loop saves
     s.S = max(1, min(num_sms / max(1, s.TB * MT), min(KC / 8, kMaxSplit)));
@@ -265,6 +268,12 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 
+// Batch item of stacked item g (tile-major, item-minor).
+__device__ __forceinline__ int item_of(const TcArgs &c, int g)
+{
+    return c.N == 1 ? 0 : g - (int)udiv((uint32_t)g, c.dN) * c.N;
+}
+
 // Source of one 16-byte halo chunk, or nullptr where the conv's zero padding
 // (or a tile past the list) applies.
 __device__ __forceinline__ const uint8_t *halo_src(const TcArgs &c, const int2 *s_orig, int T, int tb, int G, int slot,
@@ -287,7 +296,7 @@ __device__ __forceinline__ const uint8_t *halo_src(const TcArgs &c, const int2 *
     }
     if (y < 0 || y >= c.H || x < 0 || x >= c.W)
         return nullptr;
-    return c.src + ((((int64_t)(g % c.N) * c.H + y) * c.W + x) * c.Cin + ch) * 2;
+    return c.src + ((((int64_t)item_of(c, g) * c.H + y) * c.W + x) * c.Cin + ch) * 2;
 }
 
 // The input transform of the GauGAN-style layers, for 8 bf16 channels of one
@@ -381,9 +390,9 @@ __device__ __forceinline__ void fill_b(const TcArgs &c, int T, int tb, int q, in
         if (const uint8_t *src = halo_src(c, s_orig, T, tb, G, slot, hh, ww, hh * bin + ww, ch)) {
             uint4 *d = reinterpret_cast<uint4 *>(stage + b_offset(c, T, slot, hh, ww, kc));
             if (ext) {
-                *d = transform16_ext(c, *d, src - c.src, (tb * T + slot) % c.N, ch);
+                *d = transform16_ext(c, *d, src - c.src, item_of(c, tb * T + slot), ch);
             } else if (affine && c.N > 1) {
-                const int n = (tb * T + slot) % c.N;
+                const int n = item_of(c, tb * T + slot);
                 *d = transform16(*d, SIGE_BF16, c.gsc + (int64_t)n * c.Cin + ch, c.gsh + (int64_t)n * c.Cin + ch,
                                  c.silu);
             } else {
@@ -407,17 +416,17 @@ __device__ __forceinline__ void fill_b(const TcArgs &c, int T, int tb, int q, in
 // writes 512 contiguous bytes of shared memory (no bank conflicts) and reads
 // 64 contiguous bytes from each of 8 tiles.  Then the GroupNorm affine and
 // SiLU are applied in place, in the same order.
-__device__ __forceinline__ void fill_b_slots(const TcArgs &c, int T, int tb, int q, int G, uint8_t *stage, int et,
-                                             const int2 *s_orig)
+__device__ __forceinline__ void fill_b_slots(const TcArgs &c, int T, UDiv dT, int tb, int q, int G, uint8_t *stage,
+                                             int et, const int2 *s_orig)
 {
     const int bin = c.bin;
     const int total = bin * bin * 8 * T;
     const uint32_t sbase = smem_u32(stage);
 #pragma unroll 1
     for (int lin = et; lin < total; lin += kProd) {
-        const int slot = lin % T, r = lin / T;
+        const int r = (int)udiv((uint32_t)lin, dT), slot = lin - r * T;
         const int kc = r & 7, pix = r >> 3;
-        const int hh = pix / bin, ww = pix - hh * bin;
+        const int hh = (int)udiv((uint32_t)pix, c.dbin), ww = pix - hh * bin;
         const uint8_t *src = halo_src(c, s_orig, T, tb, G, slot, hh, ww, pix, q * 64 + kc * 8);
         cp_async16(sbase + (uint32_t)lin * 16u, src ? src : c.src, src ? 16u : 0u);
     }
@@ -428,15 +437,15 @@ __device__ __forceinline__ void fill_b_slots(const TcArgs &c, int T, int tb, int
     const bool ext = c.sg != nullptr || c.leaky;
 #pragma unroll 1
     for (int lin = et; lin < total; lin += kProd) {
-        const int slot = lin % T, r = lin / T;
+        const int r = (int)udiv((uint32_t)lin, dT), slot = lin - r * T;
         const int kc = r & 7, pix = r >> 3;
-        const int hh = pix / bin, ww = pix - hh * bin;
+        const int hh = (int)udiv((uint32_t)pix, c.dbin), ww = pix - hh * bin;
         const int ch = q * 64 + kc * 8;
         const uint8_t *src = halo_src(c, s_orig, T, tb, G, slot, hh, ww, pix, ch);
         if (!src)
             continue;   // zero padding stays zero
         uint4 *d = reinterpret_cast<uint4 *>(stage + (size_t)lin * 16);
-        const int n = (affine || ext) ? (tb * T + slot) % c.N : 0;
+        const int n = (affine || ext) ? item_of(c, tb * T + slot) : 0;
         if (ext)
             *d = transform16_ext(c, *d, src - c.src, n, ch);
         else
@@ -478,7 +487,7 @@ __device__ __forceinline__ void transform_b(const TcArgs &c, int T, int tb, int 
         if (halo_src(c, s_orig, T, tb, G, slot, hh, ww, hh * bin + ww, ch)) {
             uint4 *d = reinterpret_cast<uint4 *>(stage + b_offset(c, T, slot, hh, ww, kc));
             if (affine && c.N > 1) {
-                const int n = (tb * T + slot) % c.N;
+                const int n = item_of(c, tb * T + slot);
                 *d = transform16(*d, SIGE_BF16, c.gsc + (int64_t)n * c.Cin + ch, c.gsh + (int64_t)n * c.Cin + ch,
                                  c.silu);
             } else {
@@ -502,18 +511,19 @@ __device__ __forceinline__ void transform_b(const TcArgs &c, int T, int tb, int 
 // Pixel of accumulator column `col`: returns the flat element index of its
 // first channel `co0` in the destination, or -1 when the column is not a
 // pixel to write (past the list, outside the image).
-__device__ __forceinline__ int64_t col_target(const TcArgs &c, const int2 *s_orig, int T, int tb, int G, int col,
-                                              int co0)
+__device__ __forceinline__ int64_t col_target(const TcArgs &c, const int2 *s_orig, const Sched &sc, int tb, int G,
+                                              int col, int co0)
 {
+    const int T = sc.T;
     int slot, i, j;
     if (c.mode == 0) {
         slot = col >> 6;
         i = (col >> 3) & 7;
         j = col & 7;
     } else {
-        const int pos = col / T;
+        const int pos = (int)udiv((uint32_t)col, sc.dT);
         slot = col - pos * T;
-        i = pos / c.b;
+        i = (int)udiv((uint32_t)pos, c.db);
         j = pos - i * c.b;
     }
     const int g = tb * T + slot;
@@ -524,7 +534,7 @@ __device__ __forceinline__ int64_t col_target(const TcArgs &c, const int2 *s_ori
         const int yo = o.x + i, xo = o.y + j;
         if (yo >= c.Ho || xo >= c.Wo)
             return -1;
-        return (((int64_t)(g % c.N) * c.Ho + yo) * c.Wo + xo) * c.Cout + co0;
+        return (((int64_t)item_of(c, g) * c.Ho + yo) * c.Wo + xo) * c.Cout + co0;
     }
     return (((int64_t)g * c.b + i) * c.b + j) * c.Cout + co0;
 }
@@ -869,8 +879,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint32_t rsit = 0;  // reduce-scatter units done (phase of rs_ready / rs_full)
         // output vectors: 8 bf16 channels (16 per 128-channel column) or 4 floats (32)
         const int vpc = (c.to_y && c.dtype == SIGE_BF16) ? 16 : 32;
+        const int lvpc = vpc == 16 ? 4 : 5;   // log2 vpc
         const int cpv = 128 / vpc;          // channels per vector
-        const int cg = et % vpc;            // this thread's vector within a column (fixed)
+        const int cg = et & (vpc - 1);      // this thread's vector within a column (fixed)
         float * const stage_d = reinterpret_cast<float *>(smem + cv.b_base);
         const int stage_cols = min(512, (int)((p.SB * cv.stage_b) / 512) & ~15);
         uint32_t bit = 0, uit = 0;
@@ -888,7 +899,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int2 o = s_orig[slot];
                 const int x1 = c.from_image ? o.y * c.s - c.pad : 0;
                 const int y0 = c.from_image ? o.x * c.s - c.pad : 0;
-                const int n = c.from_image ? gg % c.N : gg;
+                const int n = c.from_image ? item_of(c, gg) : gg;
                 tma_load_5d(st + b_offset(c, sc.T, slot, 0, 0, 0), &tmx, bl, 0, x1, q * 8, y0, n);
             }
         };
@@ -912,7 +923,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int g = un.tb * sc.T + slot;
                 int h0 = 0, w0 = 0;
                 if (g < G && (c.from_image || c.to_y))
-                    tile_origin_a(c, g / c.N, h0, w0);
+                    tile_origin_a(c, c.N == 1 ? g : (int)udiv((uint32_t)g, c.dN), h0, w0);
                 s_orig[slot] = make_int2(h0, w0);
             }
             asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -941,7 +952,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         if (p.mode == 0)
                             fill_b(c, sc.T, un.tb, q, G, stage, et, s_orig);
                         else
-                            fill_b_slots(c, sc.T, un.tb, q, G, stage, et, s_orig);
+                            fill_b_slots(c, sc.T, sc.dT, un.tb, q, G, stage, et, s_orig);
                     }
                     fence_async_smem();
                     mbar_arrive(b_full(sb));
@@ -976,7 +987,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int it = et + k * kProd;
-                e_pre[k] = (it < ncols * vpc && write_ok) ? col_target(c, s_orig, sc.T, un.tb, G, it / vpc, co0) : -1;
+                e_pre[k] = (it < ncols * vpc && write_ok) ? col_target(c, s_orig, sc, un.tb, G, (it >> lvpc), co0) : -1;
                 rr_pre[k] = make_uint4(0, 0, 0, 0);
                 if (pre && e_pre[k] >= 0)
                     rr_pre[k] = __ldg(reinterpret_cast<const uint4 *>(c.residual + e_pre[k] * (c.dtype == SIGE_BF16 ? 2 : 4)));
@@ -1037,7 +1048,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             e[k] = e_pre[k];
                             rr[k] = rr_pre[k];
                         } else {
-                            e[k] = (it < ncols * vpc && write_ok) ? col_target(c, s_orig, sc.T, un.tb, G, it / vpc, co0)
+                            e[k] = (it < ncols * vpc && write_ok) ? col_target(c, s_orig, sc, un.tb, G, (it >> lvpc), co0)
                                                                   : -1;
                             rr[k] = make_uint4(0, 0, 0, 0);
                         }
@@ -1048,7 +1059,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     for (int k = 0; k < 4; ++k) {
                         if (e[k] < 0)
                             continue;
-                        const int col = (it0 + k * kProd) / vpc;
+                        const int col = (it0 + k * kProd) >> lvpc;
                         float v[8];
                         const float4 *src = reinterpret_cast<const float4 *>(red + col * 128 + cg * cpv);
                         const float4 lo = src[0];
@@ -1137,7 +1148,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     for (int k = 0; k < 4; ++k) {
                         const int it = it0 + k * kProd;
                         e[k] = (it < w * vpc && write_ok)
-                                   ? col_target(c, s_orig, sc.T, un.tb, G, (int)me * w + it / vpc, co0) : -1;
+                                   ? col_target(c, s_orig, sc, un.tb, G, (int)me * w + (it >> lvpc), co0) : -1;
                         rr[k] = make_uint4(0, 0, 0, 0);
                         if (e[k] >= 0 && c.residual && c.to_y)
                             rr[k] = __ldg(reinterpret_cast<const uint4 *>(c.residual + e[k] * (c.dtype == SIGE_BF16 ? 2 : 4)));
@@ -1146,7 +1157,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     for (int k = 0; k < 4; ++k) {
                         if (e[k] < 0)
                             continue;
-                        const int col = (it0 + k * kProd) / vpc;
+                        const int col = (it0 + k * kProd) >> lvpc;
                         float v[8];
 #pragma unroll
                         for (int m = 0; m < 8; ++m)
@@ -1184,7 +1195,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                 continue;
                             }
                             e[k] = (it < cc_n * vpc && write_ok)
-                                       ? col_target(c, s_orig, sc.T, un.tb, G, c0 + it / vpc, co0) : -1;
+                                       ? col_target(c, s_orig, sc, un.tb, G, c0 + (it >> lvpc), co0) : -1;
                             rr[k] = make_uint4(0, 0, 0, 0);
                             if (e[k] >= 0 && c.residual && c.to_y)
                                 rr[k] = __ldg(reinterpret_cast<const uint4 *>(c.residual + e[k] * (c.dtype == SIGE_BF16 ? 2 : 4)));
@@ -1193,7 +1204,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         for (int k = 0; k < 4; ++k) {
                             if (e[k] < 0)
                                 continue;
-                            const int col = (it0 + k * kProd) / vpc;
+                            const int col = (it0 + k * kProd) >> lvpc;
                             float v[8];
                             const float4 *src = reinterpret_cast<const float4 *>(stage_d + col * 128 + cg * cpv);
                             const float4 lo = src[0];
@@ -1240,7 +1251,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         for (int k = 0; k < 4; ++k) {
                             const int it = it0 + k * kProd;
                             e[k] = (it < ncols * vpc && write_ok)
-                                       ? col_target(c, s_orig, sc.T, un.tb, G, it / vpc, co0) : -1;
+                                       ? col_target(c, s_orig, sc, un.tb, G, (it >> lvpc), co0) : -1;
                             rr[k] = make_uint4(0, 0, 0, 0);
                             if (e[k] >= 0 && c.residual && c.to_y)
                                 rr[k] = __ldg(reinterpret_cast<const uint4 *>(c.residual + e[k] * (c.dtype == SIGE_BF16 ? 2 : 4)));
@@ -1254,7 +1265,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             for (int k = 0; k < 4; ++k) {
                                 if (e[k] < 0)
                                     continue;
-                                const int col = (it0 + k * kProd) / vpc;
+                                const int col = (it0 + k * kProd) >> lvpc;
                                 const float4 *src = reinterpret_cast<const float4 *>(
                                     base + ((size_t)s2 * p.ncols + col) * 128 + cg * cpv);
                                 const float4 lo = __ldcg(src);
@@ -1490,6 +1501,9 @@ int launch_conv_tc(const ConvParams &cp, cudaStream_t stream)
     p.residual = cp.residual; p.y = cp.y; p.out_blocks = cp.out_blocks; p.ws = cp.ws;
     p.N = cp.N; p.H = cp.H; p.W = cp.W; p.Cin = cp.Cin; p.Cout = cp.Cout; p.dtype = cp.dtype;
     p.k = cp.k; p.s = cp.s; p.pad = cp.pad; p.b = cp.b; p.bin = cp.bin; p.Ho = cp.Ho; p.Wo = cp.Wo;
+    p.dN = udiv_make((uint32_t)std::max(1, cp.N));
+    p.dbin = udiv_make((uint32_t)std::max(1, cp.bin));
+    p.db = udiv_make((uint32_t)std::max(1, cp.b));
     p.cap = cp.cap; p.dense = cp.dense; p.tiles_w = cp.tiles_w; p.tiles_total = cp.tiles_total;
     p.silu = cp.silu; p.from_image = cp.from_image; p.to_y = cp.to_y;
     p.sg = cp.sg; p.sb = cp.sb; p.leaky = cp.leaky; p.tstride = cp.tstride;

@@ -118,29 +118,6 @@ enum : int { kSiteWEmpty = 101, kSiteWFull, kSiteXReady, kSiteAcc1Empty, kSiteAc
 
 }  // namespace rb
 
-// Division of 32-bit values by a divisor fixed for the launch: a multiply-high
-// and two shifts (Granlund and Montgomery, "Division by invariant integers
-// using multiplication", 1994, the unsigned case), for the difference stream's
-// pixel -> (row, column) mapping.
-struct UDiv {
-    uint32_t m, s1, s2;
-};
-
-static inline UDiv udiv_make(uint32_t d)   // 1 <= d <= 2^31
-{
-    uint32_t l = 0;
-    while (l < 32 && (1ull << l) < d)
-        ++l;                                   // ceil(log2 d)
-    const uint64_t m = ((((uint64_t)1 << l) - d) << 32) / d + 1;
-    return UDiv{(uint32_t)m, l < 1 ? l : 1u, l > 1 ? l - 1 : 0u};
-}
-
-__device__ __forceinline__ uint32_t udiv(uint32_t n, UDiv f)
-{
-    const uint32_t t = __umulhi(n, f.m);
-    return (t + ((n - t) >> f.s1)) >> f.s2;
-}
-
 struct RbArgs {
     const uint8_t *x;           // x_edit, NHWC bf16 [N][H][W][128]
     const int32_t *idx;         // tile origins (h0, w0)

@@ -114,4 +114,28 @@ inline cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
 }
 
+// Division of 32-bit values by a divisor fixed for a launch (or a unit): a
+// multiply-high and two shifts (Granlund and Montgomery, "Division by
+// invariant integers using multiplication", 1994, the unsigned case).  Exact
+// for every n < 2^32 and 1 <= d <= 2^31.  A runtime division in a per-element
+// loop costs tens of instructions; this costs four.
+struct UDiv {
+    uint32_t m, s1, s2;
+};
+
+__host__ __device__ inline UDiv udiv_make(uint32_t d)
+{
+    uint32_t l = 0;                                  // ceil(log2 d)
+    while (l < 32 && (1ull << l) < d)
+        ++l;
+    const uint64_t m = ((((uint64_t)1 << l) - d) << 32) / d + 1;
+    return UDiv{(uint32_t)m, l < 1 ? l : 1u, l > 1 ? l - 1 : 0u};
+}
+
+__device__ __forceinline__ uint32_t udiv(uint32_t n, UDiv f)
+{
+    const uint32_t t = __umulhi(n, f.m);
+    return (t + ((n - t) >> f.s1)) >> f.s2;
+}
+
 } // namespace sige

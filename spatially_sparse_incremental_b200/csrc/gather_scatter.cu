@@ -28,6 +28,8 @@ struct GatherParams {
     int32_t silu;
     uint8_t *blocks;
     int32_t vpp;  // 16-byte vectors per pixel
+    int32_t fast; // every vector index fits 32 bits: decompose it by the divisors below
+    UDiv dvpp, dbin, dN;
 };
 
 __global__ void __launch_bounds__(256) k_gather(const __grid_constant__ GatherParams p)
@@ -39,14 +41,31 @@ __global__ void __launch_bounds__(256) k_gather(const __grid_constant__ GatherPa
     const int epv = 16 / esz;
     for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
          v += (int64_t)gridDim.x * blockDim.x) {
-        const int cv = (int)(v % p.vpp);
-        int64_t pix = v / p.vpp;
-        const int ww = (int)(pix % p.bin);
-        pix /= p.bin;
-        const int hh = (int)(pix % p.bin);
-        pix /= p.bin;
-        const int n = (int)(pix % p.N);
-        const int t = (int)(pix / p.N);
+        int cv, ww, hh, n, t;
+        if (p.fast) {
+            // (multiply-high divisions: a 64-bit division per index bounded this loop)
+            uint32_t r = (uint32_t)v, q = udiv(r, p.dvpp);
+            cv = (int)(r - q * (uint32_t)p.vpp);
+            r = q;
+            q = udiv(r, p.dbin);
+            ww = (int)(r - q * (uint32_t)p.bin);
+            r = q;
+            q = udiv(r, p.dbin);
+            hh = (int)(r - q * (uint32_t)p.bin);
+            r = q;
+            q = p.N == 1 ? r : udiv(r, p.dN);
+            n = (int)(r - q * (uint32_t)p.N);
+            t = (int)q;
+        } else {
+            cv = (int)(v % p.vpp);
+            int64_t pix = v / p.vpp;
+            ww = (int)(pix % p.bin);
+            pix /= p.bin;
+            hh = (int)(pix % p.bin);
+            pix /= p.bin;
+            n = (int)(pix % p.N);
+            t = (int)(pix / p.N);
+        }
         const int2 o = __ldg(reinterpret_cast<const int2 *>(p.idx) + t);
         const int y = o.x * p.s - p.pad + hh, x = o.y * p.s - p.pad + ww;
         uint4 out = make_uint4(0, 0, 0, 0);
@@ -71,6 +90,8 @@ struct ScatterParams {
     const float *bias;
     const uint8_t *residual;
     uint8_t *y;
+    int32_t fast; // every vector index fits 32 bits: decompose it by the divisors below
+    UDiv dc4n, db, dN;
 };
 
 __global__ void __launch_bounds__(256) k_scatter(const __grid_constant__ ScatterParams p)
@@ -80,14 +101,30 @@ __global__ void __launch_bounds__(256) k_scatter(const __grid_constant__ Scatter
     const int64_t total = ntile * p.N * p.b * p.b * c4n;
     for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
          v += (int64_t)gridDim.x * blockDim.x) {
-        const int c4 = (int)(v % c4n);
-        int64_t pix = v / c4n;
-        const int j = (int)(pix % p.b);
-        pix /= p.b;
-        const int i = (int)(pix % p.b);
-        pix /= p.b;
-        const int n = (int)(pix % p.N);
-        const int t = (int)(pix / p.N);
+        int c4, j, i, n, t;
+        if (p.fast) {
+            uint32_t r = (uint32_t)v, q = udiv(r, p.dc4n);
+            c4 = (int)(r - q * (uint32_t)c4n);
+            r = q;
+            q = udiv(r, p.db);
+            j = (int)(r - q * (uint32_t)p.b);
+            r = q;
+            q = udiv(r, p.db);
+            i = (int)(r - q * (uint32_t)p.b);
+            r = q;
+            q = p.N == 1 ? r : udiv(r, p.dN);
+            n = (int)(r - q * (uint32_t)p.N);
+            t = (int)q;
+        } else {
+            c4 = (int)(v % c4n);
+            int64_t pix = v / c4n;
+            j = (int)(pix % p.b);
+            pix /= p.b;
+            i = (int)(pix % p.b);
+            pix /= p.b;
+            n = (int)(pix % p.N);
+            t = (int)(pix / p.N);
+        }
         const int2 o = __ldg(reinterpret_cast<const int2 *>(p.idx) + t);
         const int yo = o.x + i, xo = o.y + j;
         if (yo >= p.Ho || xo >= p.Wo)
@@ -387,6 +424,10 @@ extern "C" int sige_gather(const void *x, const sige_tensor_desc *xd, const sige
     p.blocks = static_cast<uint8_t *>(blocks);
     p.vpp = xd->c * esz / 16;
     const int64_t work = (int64_t)capacity * p.N * p.bin * p.bin * p.vpp;
+    p.fast = work <= 0xFFFFFFFFll ? 1 : 0;
+    p.dvpp = udiv_make((uint32_t)p.vpp);
+    p.dbin = udiv_make((uint32_t)p.bin);
+    p.dN = udiv_make((uint32_t)p.N);
     prefer_max_shared(k_gather);
     k_gather<<<grid_for(work, 256), 256, 0, (cudaStream_t)stream>>>(p);
     count_launch();
@@ -417,6 +458,10 @@ extern "C" int sige_scatter(const float *out_blocks, const sige_conv_desc *cd, c
     p.residual = static_cast<const uint8_t *>(residual);
     p.y = static_cast<uint8_t *>(y);
     const int64_t work = (int64_t)capacity * p.N * p.b * p.b * (p.Co / 4);
+    p.fast = work <= 0xFFFFFFFFll ? 1 : 0;
+    p.dc4n = udiv_make((uint32_t)(p.Co / 4));
+    p.db = udiv_make((uint32_t)p.b);
+    p.dN = udiv_make((uint32_t)p.N);
     prefer_max_shared(k_scatter);
     k_scatter<<<grid_for(work, 256), 256, 0, (cudaStream_t)stream>>>(p);
     count_launch();

@@ -396,6 +396,31 @@ int sige_groupnorm_affine(const void *x, const sige_tensor_desc *xd, int32_t gro
 int sige_restore_tiles(const void *src, void *dst, const sige_tensor_desc *d, int32_t block,
                        const int32_t *idx, const int32_t *count, int32_t capacity, sige_stream_t stream);
 
+/* (7b) Incremental read-back of a layer's output to the host.  SIGE project
+ * page, "Overview": only the active blocks are recomputed and scattered into
+ * the cached output, so a host copy of that output, current before the edit,
+ * differs from the new output only at the listed tiles.  This copies, for
+ * every in-image pixel of the tiles listed in idx[0 .. min(count, capacity)),
+ *   host_y[n][h0+i][w0+j][:] = y[n][h0+i][w0+j][:]     (i, j < block)
+ * and leaves every other byte of host_y as it is: the device packs the tiles
+ * (and a copy of the count and the list) into `staging`; one device-to-host
+ * copy brings the count and the list, a second one the packed tiles of that
+ * count, and the host places their rows.  Synchronous: it waits for `stream`
+ * twice and returns once host_y is complete.
+ *   y           : device NHWC (u8, f32 or bf16), C * element size a multiple
+ *                 of 16 bytes, 16-byte aligned
+ *   host_y      : host memory of y's shape (pinned or pageable)
+ *   staging     : device scratch of sige_download_tiles_bytes(...) bytes,
+ *                 16-byte aligned
+ *   host_staging: host scratch of the same size (pinned, so that the copies
+ *                 are asynchronous DMA)
+ * Returns SIGE_OK, SIGE_ERR_INVALID_ARG (null or inconsistent arguments),
+ * SIGE_ERR_UNSUPPORTED (layout, dtype or alignment) or SIGE_ERR_CUDA. */
+size_t sige_download_tiles_bytes(const sige_tensor_desc *yd, int32_t block, int32_t capacity);
+int sige_download_tiles(const void *y, const sige_tensor_desc *yd, int32_t block, const int32_t *idx,
+                        const int32_t *count, int32_t capacity, void *staging, void *host_staging, void *host_y,
+                        sige_stream_t stream);
+
 /* (8) Attention step with pruned query tokens (nubint.ai review of the SIGE
  * paper, "Proposed method": attention layers by pruning the query tokens of
  * unedited regions; mer.dev notes, abstract: attention for Stable Diffusion).

@@ -78,6 +78,8 @@ SIGNATURES = {
     "sige_resblock_fused": (_i32, [_vp, _TD, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp,
                                    _vp, _vp, _sz, _vp]),
     "sige_restore_tiles": (_i32, [_vp, _vp, _TD, _i32, _vp, _vp, _i32, _vp]),
+    "sige_download_tiles_bytes": (_sz, [_TD, _i32, _i32]),
+    "sige_download_tiles": (_i32, [_vp, _TD, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp]),
     "sige_conv_workspace_bytes": (_sz, [_CD, _i32, _i32, _i32, _i32]),
     "sige_get_error": (_i32, [_vp, _vp]),
     "sige_get_device_error": (_i32, [_vp, _vp]),
@@ -393,6 +395,34 @@ def sige_restore_tiles(src, dst, block, idx, count, capacity, stream=None):
                                   int(capacity), _stream(stream))
     _check(st, "sige_restore_tiles")
     return dst
+
+
+def sige_download_tiles_bytes(y, block, capacity) -> int:
+    d = tensor_desc(y)
+    return int(lib().sige_download_tiles_bytes(ctypes.byref(d), int(block), int(capacity)))
+
+
+def sige_download_tiles(y, block, idx, count, capacity, host_y, staging=None, host_staging=None, stream=None):
+    """host_y[n, h0+i, w0+j, :] = y[n, h0+i, w0+j, :] for the listed tiles of the
+    device tensor y (in-image pixels, i, j < block); every other element of the
+    host tensor host_y is left as it is.  Returns once host_y is complete."""
+    if tuple(host_y.shape) != tuple(y.shape) or host_y.dtype != y.dtype or host_y.device.type != "cpu":
+        raise ValueError("host_y must be a host tensor of y's shape and dtype")
+    if not host_y.is_contiguous():
+        raise ValueError("host_y must be contiguous")
+    nbytes = sige_download_tiles_bytes(y, block, capacity)
+    if staging is None:
+        staging = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=y.device)
+    if host_staging is None:
+        host_staging = torch.empty(max(nbytes, 16), dtype=torch.uint8).pin_memory()
+    if staging.numel() * staging.element_size() < nbytes or host_staging.numel() * host_staging.element_size() < nbytes:
+        raise ValueError("staging buffers smaller than sige_download_tiles_bytes")
+    d = tensor_desc(y)
+    st = lib().sige_download_tiles(_ptr(y), ctypes.byref(d), int(block), _ptr(idx), _ptr(count), int(capacity),
+                                   _ptr(staging), ctypes.c_void_p(host_staging.data_ptr()),
+                                   ctypes.c_void_p(host_y.data_ptr()), _stream(stream))
+    _check(st, "sige_download_tiles")
+    return host_y
 
 
 def sige_conv_workspace_bytes(cd: ConvDesc, batch: int, capacity: int, out_h: int, out_w: int) -> int:

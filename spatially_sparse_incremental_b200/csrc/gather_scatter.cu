@@ -9,6 +9,7 @@
 // sequential edits.
 #include <atomic>
 #include <algorithm>
+#include <cstring>
 
 #include "sige_internal.cuh"
 #include "transform.cuh"
@@ -540,4 +541,127 @@ extern "C" int sige_restore_tiles(const void *src, void *dst, const sige_tensor_
     k_restore<<<grid_for(work, 256), 256, 0, (cudaStream_t)stream>>>(p);
     count_launch();
     return launch_check();
+}
+
+// ------------------------------------------------------------------ tile read-back
+
+// Staging layout: [0, 16) the count; [16, 16 + 8 cap) the list; then, 16-byte
+// aligned, the packed tiles [tile][n][i][j][C] (b x b pixels each).
+static inline size_t dl_tiles_offset(int32_t capacity) { return (16 + (size_t)capacity * 8 + 15) & ~(size_t)15; }
+
+struct PackParams {
+    const uint8_t *y;
+    int32_t N, H, W, vpp, b;    // vpp: 16-byte vectors per pixel
+    const int32_t *idx, *count;
+    int32_t cap;
+    uint8_t *staging;
+    size_t tiles_off;
+    UDiv dvpp, db, dN;
+};
+
+__global__ void __launch_bounds__(256) k_pack_tiles(const __grid_constant__ PackParams p)
+{
+    const int ntile = max(0, min(__ldg(p.count), p.cap));
+    if (blockIdx.x == 0) {
+        if (threadIdx.x == 0)
+            *reinterpret_cast<int32_t *>(p.staging) = ntile;
+        for (int t = threadIdx.x; t < ntile; t += blockDim.x)
+            reinterpret_cast<int2 *>(p.staging + 16)[t] = __ldg(reinterpret_cast<const int2 *>(p.idx) + t);
+    }
+    const uint32_t total = (uint32_t)ntile * (uint32_t)p.N * (uint32_t)(p.b * p.b) * (uint32_t)p.vpp;
+    uint4 *dst = reinterpret_cast<uint4 *>(p.staging + p.tiles_off);
+    for (uint32_t v = blockIdx.x * blockDim.x + threadIdx.x; v < total; v += gridDim.x * blockDim.x) {
+        uint32_t q = udiv(v, p.dvpp);
+        const uint32_t cv = v - q * (uint32_t)p.vpp;
+        uint32_t r = q;
+        q = udiv(r, p.db);
+        const int j = (int)(r - q * (uint32_t)p.b);
+        r = q;
+        q = udiv(r, p.db);
+        const int i = (int)(r - q * (uint32_t)p.b);
+        r = q;
+        q = p.N == 1 ? r : udiv(r, p.dN);
+        const int n = (int)(r - q * (uint32_t)p.N);
+        const int2 o = __ldg(reinterpret_cast<const int2 *>(p.idx) + q);
+        const int yy = o.x + i, xx = o.y + j;
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (yy < p.H && xx < p.W)
+            val = ld_nc16(p.y + ((((int64_t)n * p.H + yy) * p.W + xx) * p.vpp + cv) * 16);
+        dst[v] = val;
+    }
+}
+
+static int dl_esz(int dtype) { return dtype == SIGE_U8 ? 1 : dtype == SIGE_BF16 ? 2 : dtype == SIGE_F32 ? 4 : 0; }
+
+extern "C" size_t sige_download_tiles_bytes(const sige_tensor_desc *yd, int32_t block, int32_t capacity)
+{
+    if (!yd || block < 1 || capacity < 0 || yd->n < 1 || yd->c < 1 || !dl_esz(yd->dtype))
+        return 0;
+    const size_t tile = (size_t)yd->n * block * block * yd->c * dl_esz(yd->dtype);
+    return dl_tiles_offset(capacity) + (size_t)capacity * tile;
+}
+
+extern "C" int sige_download_tiles(const void *y, const sige_tensor_desc *yd, int32_t block, const int32_t *idx,
+                                   const int32_t *count, int32_t capacity, void *staging, void *host_staging,
+                                   void *host_y, sige_stream_t stream)
+{
+    if (!y || !yd || !idx || !count || !staging || !host_staging || !host_y || block < 1 || capacity < 0)
+        return SIGE_ERR_INVALID_ARG;
+    if (yd->n < 1 || yd->h < 1 || yd->w < 1 || yd->c < 1)
+        return SIGE_ERR_INVALID_ARG;
+    const int esz = dl_esz(yd->dtype);
+    if (yd->layout != SIGE_NHWC || !esz || ((size_t)yd->c * esz) % 16 ||
+        ((reinterpret_cast<uintptr_t>(y) | reinterpret_cast<uintptr_t>(staging)) & 15))
+        return SIGE_ERR_UNSUPPORTED;
+    if (capacity == 0)
+        return SIGE_OK;
+    const size_t px_bytes = (size_t)yd->c * esz;
+    const size_t tile_bytes = (size_t)yd->n * block * block * px_bytes;
+    const int64_t vec_total = (int64_t)capacity * yd->n * block * block * (int64_t)(px_bytes / 16);
+    if (vec_total > 0xFFFFFFFFll)
+        return SIGE_ERR_UNSUPPORTED;
+    PackParams p{};
+    p.y = static_cast<const uint8_t *>(y);
+    p.N = yd->n; p.H = yd->h; p.W = yd->w;
+    p.vpp = (int32_t)(px_bytes / 16);
+    p.b = block;
+    p.idx = idx; p.count = count; p.cap = capacity;
+    p.staging = static_cast<uint8_t *>(staging);
+    p.tiles_off = dl_tiles_offset(capacity);
+    p.dvpp = udiv_make((uint32_t)p.vpp);
+    p.db = udiv_make((uint32_t)block);
+    p.dN = udiv_make((uint32_t)p.N);
+    const cudaStream_t st = (cudaStream_t)stream;
+    k_pack_tiles<<<grid_for(vec_total, 256), 256, 0, st>>>(p);
+    count_launch();
+    int rc = launch_check();
+    if (rc != SIGE_OK)
+        return rc;
+    // the count and the list, then the packed tiles of that count
+    uint8_t *hs = static_cast<uint8_t *>(host_staging);
+    if (cudaMemcpyAsync(hs, staging, 16 + (size_t)capacity * 8, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return SIGE_ERR_CUDA;
+    const int n = std::max(0, std::min(*reinterpret_cast<const int32_t *>(hs), capacity));
+    if (n == 0)
+        return SIGE_OK;
+    if (cudaMemcpyAsync(hs + p.tiles_off, p.staging + p.tiles_off, (size_t)n * tile_bytes, cudaMemcpyDeviceToHost,
+                        st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return SIGE_ERR_CUDA;
+    // place the rows (clipped at the map's edges)
+    const int2 *list = reinterpret_cast<const int2 *>(hs + 16);
+    uint8_t *out = static_cast<uint8_t *>(host_y);
+    for (int t = 0; t < n; ++t) {
+        const int h0 = list[t].x, w0 = list[t].y;
+        if (h0 < 0 || w0 < 0 || h0 >= yd->h || w0 >= yd->w)
+            continue;
+        const int rows = std::min(block, yd->h - h0), cols = std::min(block, yd->w - w0);
+        for (int nn = 0; nn < yd->n; ++nn)
+            for (int i = 0; i < rows; ++i)
+                memcpy(out + ((((size_t)nn * yd->h + h0 + i) * yd->w + w0) * px_bytes),
+                       hs + p.tiles_off + (size_t)t * tile_bytes + (((size_t)nn * block + i) * block) * px_bytes,
+                       (size_t)cols * px_bytes);
+    }
+    return SIGE_OK;
 }

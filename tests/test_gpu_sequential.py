@@ -42,6 +42,39 @@ def test_restore_tiles_vs_oracle(orc, dtype, C, N, H, W, b):
     assert torch.equal(bits(d.cpu()), bits(want))
 
 
+@pytest.mark.parametrize("dtype,C,N,H,W,b,frac,over", [
+    (torch.bfloat16, 128, 1, 64, 64, 8, 0.3, False), (torch.float32, 64, 2, 30, 26, 4, 0.3, False),
+    (torch.uint8, 16, 1, 33, 35, 4, 0.5, False), (torch.bfloat16, 8, 2, 17, 19, 2, 0.2, True),
+    (torch.bfloat16, 64, 1, 16, 16, 8, 0.0, False)])
+def test_download_tiles_vs_oracle(orc, dtype, C, N, H, W, b, frac, over):
+    """The listed tiles of a device tensor into a host copy (the incremental
+    read-back): the host tensor must equal the oracle's tile restore from the
+    device values, byte for byte; ragged edge tiles, batch 2, an empty list,
+    and a count above the capacity (only the first capacity pairs count)."""
+    g = torch.Generator().manual_seed(C * 11 + W)
+    if dtype == torch.uint8:
+        y = torch.randint(0, 256, (N, H, W, C), generator=g, dtype=torch.uint8)
+        host = torch.randint(0, 256, (N, H, W, C), generator=g, dtype=torch.uint8)
+    else:
+        y = torch.randn((N, H, W, C), generator=g).to(dtype)
+        host = torch.randn((N, H, W, C), generator=g).to(dtype)
+    th, tw = -(-H // b), -(-W // b)
+    rng = np.random.default_rng(C + H)
+    tiles = np.array([(i * b, j * b) for i in range(th) for j in range(tw) if rng.random() < frac],
+                     np.int32).reshape(-1, 2)
+    cap = th * tw
+    if over and len(tiles) > 2:
+        cap = len(tiles) - 2                                # the device count exceeds the capacity
+    idx = torch.zeros((max(cap, len(tiles)), 2), dtype=torch.int32)
+    idx[:len(tiles)] = torch.from_numpy(tiles)
+    cnt = torch.tensor([len(tiles)], dtype=torch.int32)
+    used = tiles[:min(len(tiles), cap)]
+    want = orc.restore_tiles(y, host.clone(), b, used)
+    host_y = host.clone().pin_memory()
+    sige.sige_download_tiles(y.to(DEV), b, idx.to(DEV), cnt.to(DEV), cap, host_y)
+    assert torch.equal(bits(host_y), bits(want))
+
+
 def _apply(xo, xe, blk, cd, cap, y1, out, gs1, gh1, gs2, gh2, w, dev_ws=None):
     idx, cnt, _ = sige.sige_reduce_mask(xo, xe, 1e-3, [(xo.shape[1], xo.shape[2], blk.block, cap)], 1)
     sige.sige_conv_fused(xe, w["w1"], w["b1"], cd, idx, cnt, cap, y1, gs1, gh1, silu=True)

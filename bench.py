@@ -488,7 +488,7 @@ def measure_extras(dev, flush, stream, peaks, seed, step_graph):
     return out
 
 
-def layer_rows(seed, dev, flush, stream, peaks):
+def layer_rows(seed, dev, flush, stream, peaks, reps=30):
     """Every per-layer workload at its default edit: one fused call, sparse
     and dense, each in its own CUDA graph with L2 flushed."""
     from spatially_sparse_incremental_b200 import inputs
@@ -500,21 +500,21 @@ def layer_rows(seed, dev, flush, stream, peaks):
     rows = []
     for name, L, bits in layers:
         try:
-            rows.append(dict(name=name, **layer_timing(L, bits, dev, flush, stream, peaks)))
+            rows.append(dict(name=name, **layer_timing(L, bits, dev, flush, stream, peaks, reps=reps)))
         except Exception as e:   # a failing row is reported, not fatal to the headline line
             rows.append({"name": name, "error": str(e)[:200]})
     for i, (h, w, ci, co, b) in enumerate(inputs.UPSAMPLE_LAYERS):
         name = f"GauGAN upsample {h}x{w}->{2 * h}x{2 * w} {ci}->{co} 3x3 transposed s2 b{b}"
         try:
             rows.append(dict(name=name, **ext_layer_timing(inputs.make_upsample_layer(seed, i), dev, flush, stream,
-                                                           peaks, transposed=True)))
+                                                           peaks, transposed=True, reps=min(20, reps))))
         except Exception as e:
             rows.append({"name": name, "error": str(e)[:200]})
     for i, (h, w, ci, co, b) in enumerate(inputs.SPADE_LAYERS):
         name = f"GauGAN SPADE {h}x{w} {ci}->{co} 3x3 b{b} LeakyReLU"
         try:
             rows.append(dict(name=name, **ext_layer_timing(inputs.make_spade_layer(seed, i), dev, flush, stream,
-                                                           peaks, spade=True)))
+                                                           peaks, spade=True, reps=min(20, reps))))
         except Exception as e:
             rows.append({"name": name, "error": str(e)[:200]})
     return rows
@@ -1115,7 +1115,7 @@ def run_row(args):
         if args.row == "attention":
             r = attention_timing(args.seed, dev, flush, stream, peaks, reps=max(3, args.steps))
         elif args.row == "layers":
-            r = {"layers": layer_rows(args.seed, dev, flush, stream, peaks)}
+            r = {"layers": layer_rows(args.seed, dev, flush, stream, peaks, reps=max(3, args.steps))}
         elif args.row == "gather_scatter":
             r = gather_scatter_timing(args.seed, dev, flush, stream, peaks, reps=max(3, args.steps))
         else:

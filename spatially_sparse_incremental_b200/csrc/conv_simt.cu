@@ -1,8 +1,8 @@
 // Layer F_l on the CUDA cores (float32 arithmetic): the path for float32
 // layers, and for bf16 layers the tensor-core kernel does not cover.
 //
-// Tiles of at most 16 pixels (b <= 4) run k_conv_simt16: a unit of 64 output
-// channels x 16 pixel slots, 4 K groups of 64 threads each holding a
+// Tiles of at most 16 pixels (b <= 4) run k_conv_simt16: a unit of 32 output
+// channels x 16 pixel slots, 8 K groups of 32 threads each holding a
 // 4-channel x 4-pixel block of accumulators, weights and halo staged per
 // input-channel chunk in shared memory (float32: asynchronous 4-byte copies),
 // the K groups summed in a fixed order at the end.  Larger tiles run
@@ -218,14 +218,17 @@ __global__ void __launch_bounds__(kSimtThreads) k_conv_simt(const __grid_constan
     }
 }
 
-// Tiles of at most 16 pixels (b <= 4): register-blocked.  A unit is 64 output
-// channels x 16 pixel slots of one tile; its 256 threads form 4 K groups (input
-// channel ci of a chunk goes to group ci % 4) of 64 threads, and each thread
+// Tiles of at most 16 pixels (b <= 4): register-blocked.  A unit is 32 output
+// channels x 16 pixel slots of one tile; its 256 threads form 8 K groups (input
+// channel ci of a chunk goes to group ci % 8) of 32 threads, and each thread
 // holds a 4-channel x 4-pixel block of accumulators, so one 16-byte weight read
 // and four input reads feed 16 FMAs.  The K groups are summed in a fixed order
 // through shared memory at the end.
 constexpr int kS16Threads = 256;
-constexpr int kS16Cout = 64;            // output channels per unit
+constexpr int kS16Cout = 32;            // output channels per unit (fewer per unit: more CTAs on few tiles)
+constexpr int kS16Cq = kS16Cout / 4;    // 4-channel groups of a unit
+constexpr int kS16Kg = kS16Threads / (kS16Cq * 4);   // K groups (a K group: kS16Cq x 4 pixel groups of threads)
+static_assert(kS16Kg * kS16Cq * 4 == kS16Threads && kS16Kg * 16 * kS16Cout <= 4096, "unit shape");
 constexpr int kS16WStride = kS16Cout + 4;   // weight row stride (floats): 16-byte aligned, fewer bank conflicts
 constexpr int kS16SmemFloats = 24576;   // 96 KB: two CTAs per SM, fewer channel chunks
 
@@ -238,7 +241,7 @@ __global__ void __launch_bounds__(kS16Threads, 1) k_conv_simt16(const __grid_con
     float *sw = s16 + ((npix * cmax + 3) & ~3);                 // [tap][cc][kS16WStride]
     float *red = s16;                                           // [K group][16 px][64 co], after the last chunk
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = kS16Threads / 32;
-    const int kg = tid >> 6, cq = tid & 15, pq = (tid >> 4) & 3;
+    const int kg = tid / (kS16Cq * 4), cq = tid % kS16Cq, pq = (tid / kS16Cq) & 3;
     const int ntiles = p.dense ? p.tiles_total : min(__ldg(p.count), p.cap);
     const int ncog = (p.Cout + kS16Cout - 1) / kS16Cout;
     const int units = ntiles * p.N * ncog;
@@ -394,7 +397,7 @@ __global__ void __launch_bounds__(kS16Threads, 1) k_conv_simt16(const __grid_con
                     const float *x3 = sx + (pix0[3] + r * p.bin + c) * cc;
                     const float *wr = sw + (r * p.k + c) * cc * kS16WStride + cq * 4;
 #pragma unroll 2
-                    for (int ci = kg; ci < cc; ci += 4) {
+                    for (int ci = kg; ci < cc; ci += kS16Kg) {
                         const float4 w4 = *reinterpret_cast<const float4 *>(wr + ci * kS16WStride);
                         const float xv[4] = {x0[ci], x1[ci], x2[ci], x3[ci]};
                         const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
@@ -414,15 +417,15 @@ __global__ void __launch_bounds__(kS16Threads, 1) k_conv_simt16(const __grid_con
                 make_float4(acc[0][j], acc[1][j], acc[2][j], acc[3][j]);
         __syncthreads();
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int oi = tid + kS16Threads * m;       // [16 px][64 co]
+        for (int m = 0; m < (16 * kS16Cout + kS16Threads - 1) / kS16Threads; ++m) {
+            const int oi = tid + kS16Threads * m;       // [16 px][kS16Cout co]
             const int col = oi & (kS16Cout - 1), px = oi / kS16Cout;
             const int o = cog * kS16Cout + col;
             if (px >= npx || o >= p.Cout)
                 continue;
             float a = 0.0f;
 #pragma unroll
-            for (int g = 0; g < 4; ++g)
+            for (int g = 0; g < kS16Kg; ++g)
                 a += red[(g * 16 + px) * kS16Cout + col];
             const int i = px / p.b, j = px % p.b;
             if (p.to_y) {

@@ -1,8 +1,8 @@
 // Layer F_l on the CUDA cores (float32 arithmetic): the path for float32
 // layers, and for bf16 layers the tensor-core kernel does not cover.
 //
-// Tiles of at most 16 pixels (b <= 4) run k_conv_simt16: a unit of 32 output
-// channels x 16 pixel slots, 8 K groups of 32 threads each holding a
+// Tiles of at most 16 pixels (b <= 4) run k_conv_simt16: a unit of 16 output
+// channels x 16 pixel slots, 16 K groups of 16 threads each holding a
 // 4-channel x 4-pixel block of accumulators, weights and halo staged per
 // input-channel chunk in shared memory (float32: asynchronous 4-byte copies),
 // the K groups summed in a fixed order at the end.  Larger tiles run
@@ -218,14 +218,14 @@ __global__ void __launch_bounds__(kSimtThreads) k_conv_simt(const __grid_constan
     }
 }
 
-// Tiles of at most 16 pixels (b <= 4): register-blocked.  A unit is 32 output
-// channels x 16 pixel slots of one tile; its 256 threads form 8 K groups (input
-// channel ci of a chunk goes to group ci % 8) of 32 threads, and each thread
+// Tiles of at most 16 pixels (b <= 4): register-blocked.  A unit is 16 output
+// channels x 16 pixel slots of one tile; its 256 threads form 16 K groups (input
+// channel ci of a chunk goes to group ci % 16) of 16 threads, and each thread
 // holds a 4-channel x 4-pixel block of accumulators, so one 16-byte weight read
 // and four input reads feed 16 FMAs.  The K groups are summed in a fixed order
 // through shared memory at the end.
 constexpr int kS16Threads = 256;
-constexpr int kS16Cout = 32;            // output channels per unit (fewer per unit: more CTAs on few tiles)
+constexpr int kS16Cout = 16;            // output channels per unit (fewer per unit: more CTAs on few tiles)
 constexpr int kS16Cq = kS16Cout / 4;    // 4-channel groups of a unit
 constexpr int kS16Kg = kS16Threads / (kS16Cq * 4);   // K groups (a K group: kS16Cq x 4 pixel groups of threads)
 static_assert(kS16Kg * kS16Cq * 4 == kS16Threads && kS16Kg * 16 * kS16Cout <= 4096, "unit shape");

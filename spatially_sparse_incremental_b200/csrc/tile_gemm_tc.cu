@@ -87,8 +87,9 @@ struct Args {
     const int32_t *idx;        // sparse: tile origins (h0, w0)
     const int32_t *count;
     int32_t cap, dense, tiles_w, tiles_total;
-    int32_t N, H, W, Cin, Cout, b;
-    int32_t k, pad;            // kernel size and padding (stride 1, output size = input size)
+    int32_t N, H, W, Cin, Cout, b;   // H, W: the input map
+    int32_t k, pad, s;         // kernel size, padding, stride
+    int32_t Ho, Wo;            // the output map
     int32_t nt, ntn;           // output channels per unit, units along C_out
     const float *gsc, *gsh;    // GroupNorm affine [N][Cin] (or null)
     int32_t silu;
@@ -391,7 +392,7 @@ __global__ void __launch_bounds__(tg::kThreads, 1)
                 __syncwarp();
                 if (tv)
                     tma4(sb + kOffA + st * kABytes + (uint32_t)(lane * bb) * 128u, &tx, a_land(st), tp.cc * 64,
-                         w0 + tp.dc, h0 + tp.dr, n);
+                         w0 * p.s + tp.dc, h0 * p.s + tp.dr, n);
             }
             ia += nck;
         }
@@ -429,13 +430,13 @@ __global__ void __launch_bounds__(tg::kThreads, 1)
                 const int sl = r % bb;
                 yy = h0 + sl / p.b;
                 xx = w0 + sl % p.b;
-                valid = h0 >= 0 && w0 >= 0 && yy < p.H && xx < p.W;
+                valid = h0 >= 0 && w0 >= 0 && yy < p.Ho && xx < p.Wo;
             }
-            const int64_t pix = ((int64_t)n * p.H + yy) * p.W + xx;
+            const int64_t pix = ((int64_t)n * p.Ho + yy) * p.Wo + xx;
             // the slot's pixel shifted by a chunk's tap; false outside the map
             // (a zero row: the conv's padding)
             auto tap_in = [&](const TapPos &t, int64_t &ipix) -> bool {
-                const int yi = yy + t.dr, xi = xx + t.dc;
+                const int yi = yy * p.s + t.dr, xi = xx * p.s + t.dc;
                 ipix = ((int64_t)n * p.H + yi) * p.W + xi;
                 return valid && yi >= 0 && yi < p.H && xi >= 0 && xi < p.W;
             };
@@ -659,15 +660,17 @@ __global__ void __launch_bounds__(tg::kThreads, 1)
 
 bool tile_gemm_supported(const sige_conv_desc *cd, int dtype)
 {
-    if (!cd || dtype != SIGE_BF16 || cd->stride != 1 || cd->block < 1 || cd->block * cd->block > tg::kRows ||
+    if (!cd || dtype != SIGE_BF16 || cd->stride < 1 || cd->stride > 2 || cd->block < 1 ||
+        cd->block * cd->block > tg::kRows ||
         cd->c_in < 64 || cd->c_in % 64 || cd->c_out < 16 || cd->c_out % 16)
         return false;
     if ((long long)cd->kernel * cd->kernel * cd->c_in >= (1ll << 31))
         return false;
-    // 1x1 (any tile size), or 3x3 "same" (padding 1) on 4x4 or 8x8 tiles,
-    // whose shifted boxes the TMA fills (the CUDA-core copies of other tile
-    // sizes cannot keep a 3x3 layer's K loop fed)
-    return (cd->kernel == 1 && cd->pad == 0) ||
+    // 1x1 stride 1 (any tile size), or 3x3 padding 1, stride 1 or 2, on 4x4
+    // or 8x8 tiles, whose tap-shifted (and strided) boxes the TMA fills (the
+    // CUDA-core copies of other tile sizes cannot keep a 3x3 layer's K loop
+    // fed)
+    return (cd->kernel == 1 && cd->pad == 0 && cd->stride == 1) ||
            (cd->kernel == 3 && cd->pad == 1 && (cd->block * cd->block) % 8 == 0);
 }
 
@@ -687,6 +690,9 @@ int launch_tile_gemm(const ConvParams &cp, cudaStream_t stream)
     a.N = cp.N;
     a.H = cp.H;
     a.W = cp.W;
+    a.s = cp.s;
+    a.Ho = cp.Ho;
+    a.Wo = cp.Wo;
     a.Cin = cp.Cin;
     a.Cout = cp.Cout;
     a.b = cp.b;
@@ -735,8 +741,9 @@ int launch_tile_gemm(const ConvParams &cp, cudaStream_t stream)
     if ((cp.b * cp.b) % 8 == 0) {
         cuuint64_t xd[4] = {(cuuint64_t)cp.Cin, (cuuint64_t)cp.W, (cuuint64_t)cp.H, (cuuint64_t)cp.N};
         cuuint64_t xs[3] = {(cuuint64_t)cp.Cin * 2, (cuuint64_t)cp.W * cp.Cin * 2, (cuuint64_t)cp.H * cp.W * cp.Cin * 2};
-        cuuint32_t xb[4] = {64, (cuuint32_t)cp.b, (cuuint32_t)cp.b, 1};
-        cuuint32_t xe[4] = {1, 1, 1, 1};
+        // (stride s: a box of b s pixels per side read every s-th pixel, b per side)
+        cuuint32_t xb[4] = {64, (cuuint32_t)(cp.b * cp.s), (cuuint32_t)(cp.b * cp.s), 1};
+        cuuint32_t xe[4] = {1, (cuuint32_t)cp.s, (cuuint32_t)cp.s, 1};
         if (encode(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint8_t *>(cp.src), xd, xs, xb, xe,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)

@@ -437,6 +437,20 @@ def test_tile_gemm_3x3_sparse(orc, H, W, ci, co, b, N, gn, res, area):
     _fused_vs_oracle(orc, L, _tiles(orc, L), residual=res, seed=9)
 
 
+@pytest.mark.parametrize("H,W,ci,co,b,N,gn,res,area", [
+    (64, 64, 64, 64, 4, 1, False, False, 0.05),      # stride 2: strided TMA boxes, 9 K chunks
+    (33, 29, 128, 80, 4, 2, True, True, 0.15),       # odd input map, batch 2, C_out 80, GN + SiLU, residual
+    (40, 48, 64, 32, 8, 1, True, False, 0.2),        # 8x8 output tiles (16x16 strided boxes)
+])
+def test_tile_gemm_3x3_stride2(orc, H, W, ci, co, b, N, gn, res, area):
+    """3x3 stride-2 layers on the tile GEMM: tap (dr, dc) of output tile
+    (h0, w0) reads every other input pixel from (2 h0 + dr - 1, 2 w0 + dc - 1)."""
+    L = inputs.make_conv_case(130 + H + co + b, H, W, ci, co, dtype=torch.bfloat16, stride=2, block=b, area=area,
+                              gn=gn, N=N)
+    assert sige.sige_conv_path(sige.conv_desc(3, 2, 1, ci, co, b), torch.bfloat16) == 1
+    _fused_vs_oracle(orc, L, _tiles(orc, L), residual=res, seed=11)
+
+
 @pytest.mark.parametrize("H,W,ci,co,b,N", [(28, 36, 64, 64, 4, 1), (18, 14, 128, 48, 2, 2)])
 def test_tile_gemm_3x3_dense(orc, H, W, ci, co, b, N):
     L = inputs.make_conv_case(120 + H + co, H, W, ci, co, dtype=torch.bfloat16, block=b, gn=True, N=N)

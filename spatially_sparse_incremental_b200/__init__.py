@@ -277,7 +277,8 @@ def sige_conv_fused(x, weight, bias, cd: ConvDesc, idx, count, capacity, y, gn_s
                     silu=False, residual=None, workspace=None, stream=None):
     xd, yd = tensor_desc(x), tensor_desc(y)
     if workspace is None:
-        workspace = zeros_workspace(sige_conv_workspace_bytes(cd, x.shape[0], capacity, 0, 0), x.device)
+        workspace = zeros_workspace(sige_conv_workspace_bytes(cd, x.shape[0], capacity, y.shape[1], y.shape[2]),
+                                    x.device)
     st = lib().sige_conv_fused(_ptr(x), ctypes.byref(xd), _ptr(weight), _ptr(bias), ctypes.byref(cd), _ptr(idx),
                                _ptr(count), int(capacity), _ptr(gn_scale), _ptr(gn_shift), int(bool(silu)),
                                _ptr(residual), _ptr(y), ctypes.byref(yd), _ptr(workspace), workspace.numel(),

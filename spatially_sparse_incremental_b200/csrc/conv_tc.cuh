@@ -19,5 +19,10 @@ int launch_conv8(const ConvParams &p, cudaStream_t stream);
 // a cluster when the units are few.
 bool tile_gemm_supported(const sige_conv_desc *cd, int dtype);
 int launch_tile_gemm(const ConvParams &p, cudaStream_t stream);
+// A 3x3 layer with an input transform: the transform of the pixels its tiles
+// read, once, into `scratch` (tile_gemm_scratch_bytes), then the tile GEMM on
+// that copy without a transform.
+size_t tile_gemm_scratch_bytes(const sige_conv_desc *cd, int batch, int in_h, int in_w);
+int launch_tile_gemm_pre(const ConvParams &p, uint8_t *scratch, cudaStream_t stream);
 
 } // namespace sige

@@ -86,11 +86,17 @@ static int run_conv(ConvParams &p, const sige_conv_desc *cd, void *ws, size_t ws
     const bool plain = p.from_image && p.to_y && !p.tstride && !p.sg && !p.leaky;
     if (plain && conv8_supported(cd, p.dtype))
         return launch_conv8(p, st);
-    // (a 3x3 layer with an input transform stays on the general kernel, which
-    // transforms each halo pixel once, where the tile GEMM would transform
-    // every tap's copy: measured 1.7-3.9x slower)
-    if (plain && tile_gemm_supported(cd, p.dtype) && (cd->kernel == 1 || (!p.gsc && !p.silu)))
-        return launch_tile_gemm(p, st);
+    if (plain && tile_gemm_supported(cd, p.dtype)) {
+        if (cd->kernel == 1 || (!p.gsc && !p.silu))
+            return launch_tile_gemm(p, st);
+        // a 3x3 layer with an input transform: the transform once per pixel
+        // into a scratch copy in the workspace (transforming every tap's copy
+        // of a row measured 1.7-3.9x slower than the general kernel), when the
+        // workspace was sized by sige_conv_workspace_bytes
+        const size_t base = (ws_need(cd, p.N, ntiles) + 255) & ~(size_t)255;
+        if (ws_bytes >= base + tile_gemm_scratch_bytes(cd, p.N, p.H, p.W))
+            return launch_tile_gemm_pre(p, p.ws + base, st);
+    }
     if (tc_supported(cd, p.dtype))
         return launch_conv_tc(p, st);
     return launch_conv_simt(p, st);
@@ -112,7 +118,12 @@ extern "C" size_t sige_conv_workspace_bytes(const sige_conv_desc *cd, int32_t ba
     v.stride = 1;
     v.pad = std::max(0, cd->kernel - 1 - cd->pad);
     const int n = (int)std::min<int64_t>(nt, INT32_MAX);
-    return std::max(ws_need(cd, batch, n), ws_need(&v, batch, n));
+    size_t need = std::max(ws_need(cd, batch, n), ws_need(&v, batch, n));
+    // the tile GEMM's scratch copy of a transformed input (3x3 layers)
+    if (tile_gemm_supported(cd, SIGE_BF16) && cd->kernel == 3)
+        need = ((ws_need(cd, batch, n) + 255) & ~(size_t)255) +
+               tile_gemm_scratch_bytes(cd, batch, out_h * cd->stride + cd->kernel, out_w * cd->stride + cd->kernel);
+    return std::max(need, std::max(ws_need(cd, batch, n), ws_need(&v, batch, n)));
 }
 
 extern "C" int sige_conv_path(const sige_conv_desc *cd, int32_t dtype)

@@ -656,6 +656,68 @@ __global__ void __launch_bounds__(tg::kThreads, 1)
     cluster_wait();
 }
 
+// ------------------------------------------------------------------ input transform pre-pass
+
+// For a 3x3 layer with an input transform (GroupNorm affine, SiLU): the
+// transform of every input pixel the listed tiles' taps read (the halo of
+// each tile, or the whole map for a dense call) is written once into a
+// scratch copy of the input, which the GEMM then reads untransformed, instead
+// of transforming each tap's copy of a row (nine times the work).  Pixels of
+// overlapping halos are written with the same value by every tile that
+// covers them.
+struct PreArgs {
+    const uint8_t *x;          // NHWC bf16 [N][H][W][Cin]
+    uint8_t *xt;               // the scratch copy, same layout
+    const int32_t *idx, *count;
+    int32_t cap, dense;
+    int32_t N, H, W, Cin, b, s, pad, hb;   // hb: halo side (b - 1) s + 3
+    const float *gsc, *gsh;
+    int32_t silu;
+    UDiv dvpp, dhb, dN, dW, dH;
+};
+
+__global__ void __launch_bounds__(256) k_tile_pretransform(const __grid_constant__ PreArgs p)
+{
+    pdl_wait();
+    const uint32_t vpp = (uint32_t)(p.Cin / 8);
+    const uint32_t per_tile = (uint32_t)(p.hb * p.hb) * vpp;
+    const uint32_t total = p.dense ? (uint32_t)p.N * (uint32_t)p.H * (uint32_t)p.W * vpp
+                                   : (uint32_t)max(0, min(__ldg(p.count), p.cap)) * (uint32_t)p.N * per_tile;
+    for (uint32_t v = blockIdx.x * blockDim.x + threadIdx.x; v < total; v += gridDim.x * blockDim.x) {
+        uint32_t q = udiv(v, p.dvpp);
+        const uint32_t cv = v - q * vpp;
+        int n, y, x;
+        if (p.dense) {
+            const uint32_t r = q;                               // pixel n H W + y W + x
+            q = udiv(r, p.dW);
+            x = (int)(r - q * (uint32_t)p.W);
+            const uint32_t q2 = udiv(q, p.dH);
+            y = (int)(q - q2 * (uint32_t)p.H);
+            n = (int)q2;
+        } else {
+            uint32_t r = q;
+            q = udiv(r, p.dhb);
+            const int ww = (int)(r - q * (uint32_t)p.hb);
+            r = q;
+            q = udiv(r, p.dhb);
+            const int hh = (int)(r - q * (uint32_t)p.hb);
+            r = q;
+            q = p.N == 1 ? r : udiv(r, p.dN);
+            n = (int)(r - q * (uint32_t)p.N);
+            const int2 o = __ldg(reinterpret_cast<const int2 *>(p.idx) + q);
+            y = o.x * p.s - p.pad + hh;
+            x = o.y * p.s - p.pad + ww;
+            if (y < 0 || y >= p.H || x < 0 || x >= p.W)
+                continue;
+        }
+        const int64_t e = (((int64_t)n * p.H + y) * p.W + x) * p.Cin + (int64_t)cv * 8;
+        const uint4 in = ld_nc16(p.x + e * 2);
+        reinterpret_cast<uint4 *>(p.xt)[e / 8] =
+            transform16(in, SIGE_BF16, p.gsc ? p.gsc + (int64_t)n * p.Cin + cv * 8 : nullptr,
+                        p.gsc ? p.gsh + (int64_t)n * p.Cin + cv * 8 : nullptr, p.silu);
+    }
+}
+
 // ------------------------------------------------------------------ host
 
 bool tile_gemm_supported(const sige_conv_desc *cd, int dtype)
@@ -795,6 +857,57 @@ int launch_tile_gemm(const ConvParams &cp, cudaStream_t stream)
         return SIGE_ERR_CUDA;
     count_launch();
     return launch_check();
+}
+
+size_t tile_gemm_scratch_bytes(const sige_conv_desc *cd, int batch, int in_h, int in_w)
+{
+    if (!cd || cd->kernel != 3)
+        return 0;
+    return ((size_t)batch * in_h * in_w * cd->c_in * 2 + 255) & ~(size_t)255;
+}
+
+int launch_tile_gemm_pre(const ConvParams &cp, uint8_t *scratch, cudaStream_t stream)
+{
+    PreArgs a{};
+    a.x = cp.src;
+    a.xt = scratch;
+    a.idx = cp.idx;
+    a.count = cp.count;
+    a.cap = cp.cap;
+    a.dense = cp.dense;
+    a.N = cp.N;
+    a.H = cp.H;
+    a.W = cp.W;
+    a.Cin = cp.Cin;
+    a.b = cp.b;
+    a.s = cp.s;
+    a.pad = cp.pad;
+    a.hb = (cp.b - 1) * cp.s + cp.k;
+    a.gsc = cp.gsc;
+    a.gsh = cp.gsh;
+    a.silu = cp.silu;
+    a.dvpp = udiv_make((uint32_t)(cp.Cin / 8));
+    a.dhb = udiv_make((uint32_t)a.hb);
+    a.dN = udiv_make((uint32_t)cp.N);
+    a.dW = udiv_make((uint32_t)cp.W);
+    a.dH = udiv_make((uint32_t)cp.H);
+    const int64_t work = cp.dense ? (int64_t)cp.N * cp.H * cp.W * (cp.Cin / 8)
+                                  : (int64_t)cp.cap * cp.N * a.hb * a.hb * (cp.Cin / 8);
+    if (work > 0xFFFFFFFFll)
+        return SIGE_ERR_UNSUPPORTED;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, (int64_t)device_sm_count() * 8));
+    if (launch_pdl(k_tile_pretransform, dim3(grid), dim3(256), 0, stream, a) != cudaSuccess)
+        return SIGE_ERR_CUDA;
+    count_launch();
+    int rc = launch_check();
+    if (rc != SIGE_OK)
+        return rc;
+    ConvParams g = cp;
+    g.src = scratch;
+    g.gsc = nullptr;
+    g.gsh = nullptr;
+    g.silu = 0;
+    return launch_tile_gemm(g, stream);
 }
 
 } // namespace sige

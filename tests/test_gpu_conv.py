@@ -423,7 +423,7 @@ def test_conv1x1_dense(orc, H, W, ci, co, b, N, gn, res):
     (24, 20, 128, 320, 4, 1, False, False, 0.1),      # C_out 320: five units of 64 output channels
     (64, 64, 320, 320, 4, 1, False, True, 0.012),     # the SD-latent layer's shape (K split 4)
     (24, 24, 64, 48, 8, 1, False, True, 0.1),         # 8x8 tiles with a C_out the 8x8 kernel does not take
-    (30, 26, 64, 48, 4, 2, True, True, 0.1),          # GN + SiLU: the general kernel
+    (30, 26, 64, 48, 4, 2, True, True, 0.1),          # GN + SiLU: transformed once into a scratch copy
     (20, 18, 64, 64, 2, 1, True, True, 0.1),          # 2x2, 1x1 and 3x3 tiles: the general tile kernel
     (12, 10, 128, 32, 1, 2, False, True, 0.2),
     (21, 19, 64, 16, 3, 1, True, False, 0.15),
@@ -432,8 +432,9 @@ def test_tile_gemm_3x3_sparse(orc, H, W, ci, co, b, N, gn, res, area):
     """3x3 stride-1 layers on 4x4 tiles (and 8x8 ones outside the 8x8
     kernel's range) without an input transform: the tile GEMM, one shifted TMA
     box of the tile's pixels per tap (zero outside the map), K split across a
-    cluster when the units are few; other tile sizes, and layers with GN +
-    SiLU, on the general kernel."""
+    cluster when the units are few (with GN + SiLU: the transform once per
+    input pixel into a scratch copy first); other tile sizes on the general
+    kernel."""
     L = inputs.make_conv_case(110 + H + co + b, H, W, ci, co, dtype=torch.bfloat16, block=b, area=area, gn=gn, N=N)
     assert sige.sige_conv_path(sige.conv_desc(3, 1, 1, ci, co, b), torch.bfloat16) == 1
     _fused_vs_oracle(orc, L, _tiles(orc, L), residual=res, seed=9)
@@ -443,7 +444,7 @@ def test_tile_gemm_3x3_sparse(orc, H, W, ci, co, b, N, gn, res, area):
     (64, 64, 64, 64, 4, 1, False, False, 0.05),      # stride 2: strided TMA boxes, 9 K chunks
     (33, 29, 128, 80, 4, 2, False, True, 0.15),      # odd input map, batch 2, C_out 80, residual
     (40, 48, 64, 32, 8, 1, False, False, 0.2),       # 8x8 output tiles (16x16 strided boxes)
-    (33, 29, 128, 80, 4, 2, True, True, 0.15),       # GN + SiLU: the general kernel
+    (33, 29, 128, 80, 4, 2, True, True, 0.15),       # GN + SiLU: transformed once into a scratch copy
 ])
 def test_tile_gemm_3x3_stride2(orc, H, W, ci, co, b, N, gn, res, area):
     """3x3 stride-2 layers on the tile GEMM: tap (dr, dc) of output tile

@@ -464,7 +464,11 @@ int sige_attention_path(const sige_tensor_desc *qd, int32_t dv, int32_t heads);
 
 /* Workspace bytes for sige_sparse_conv / sige_conv_fused / sige_dense_conv
  * with this layer, batch and list capacity (capacity is ignored for the dense
- * call, which uses the full tile grid of an output of `out_h` x `out_w`). */
+ * call, which uses the full tile grid of an output of `out_h` x `out_w`).
+ * With the output dimensions given (> 0), the size also covers a scratch copy
+ * of the input for 3x3 layers that the tile GEMM can run: a fused or dense
+ * call with GroupNorm / SiLU then transforms each input pixel once into it;
+ * with a smaller workspace such a call runs on the general kernel. */
 size_t sige_conv_workspace_bytes(const sige_conv_desc *cd, int32_t batch, int32_t capacity,
                                  int32_t out_h, int32_t out_w);
 

@@ -119,8 +119,9 @@ extern "C" size_t sige_conv_workspace_bytes(const sige_conv_desc *cd, int32_t ba
     v.pad = std::max(0, cd->kernel - 1 - cd->pad);
     const int n = (int)std::min<int64_t>(nt, INT32_MAX);
     size_t need = std::max(ws_need(cd, batch, n), ws_need(&v, batch, n));
-    // the tile GEMM's scratch copy of a transformed input (3x3 layers)
-    if (tile_gemm_supported(cd, SIGE_BF16) && cd->kernel == 3)
+    // the tile GEMM's scratch copy of a transformed input (3x3 layers; sized
+    // from the output dimensions, so only when they are given)
+    if (tile_gemm_supported(cd, SIGE_BF16) && cd->kernel == 3 && out_h > 0 && out_w > 0)
         need = ((ws_need(cd, batch, n) + 255) & ~(size_t)255) +
                tile_gemm_scratch_bytes(cd, batch, out_h * cd->stride + cd->kernel, out_w * cd->stride + cd->kernel);
     return std::max(need, std::max(ws_need(cd, batch, n), ws_need(&v, batch, n)));

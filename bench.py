@@ -503,6 +503,16 @@ def layer_rows(seed, dev, flush, stream, peaks, reps=30):
             rows.append(dict(name=name, **layer_timing(L, bits, dev, flush, stream, peaks, reps=reps)))
         except Exception as e:   # a failing row is reported, not fatal to the headline line
             rows.append({"name": name, "error": str(e)[:200]})
+    # the 4x4-tile 3x3 layers with GroupNorm + SiLU on the input (a U-Net res block's convs)
+    gn_layers = [(f"SD latent {h}x{w} C{c} 3x3 b{b}, GN+SiLU", inputs.make_cfg4_layer(seed, i))
+                 for i, (h, w, c, b) in enumerate(inputs.CFG4_LAYERS) if b == 4]
+    gn_layers += [(f"GauGAN {h}x{w} {ci}->{co} {k}x{k} s{st} b{b}, GN+SiLU", inputs.make_cfg5_layer(seed, i))
+                  for i, (h, w, ci, co, k, st, b) in enumerate(inputs.CFG5_LAYERS) if b == 4 and k == 3]
+    for name, L in gn_layers:
+        try:
+            rows.append(dict(name=name, **layer_timing(L, 16, dev, flush, stream, peaks, reps=reps, gn=True)))
+        except Exception as e:
+            rows.append({"name": name, "error": str(e)[:200]})
     for i, (h, w, ci, co, b) in enumerate(inputs.UPSAMPLE_LAYERS):
         name = f"GauGAN upsample {h}x{w}->{2 * h}x{2 * w} {ci}->{co} 3x3 transposed s2 b{b}"
         try:
@@ -557,13 +567,22 @@ def gather_scatter_timing(seed, dev, flush, stream, peaks, reps=30):
     return res
 
 
-def layer_timing(L, bits, dev, flush, stream, peaks, reps=30, dense_us=None):
+def layer_timing(L, bits, dev, flush, stream, peaks, reps=30, dense_us=None, gn=False):
+    """One layer, sparse (its tile list at the layer's edit) and dense, each one
+    call in its own graph with L2 flushed; gn: with a GroupNorm-style affine
+    (seeded per-channel scale / shift) and SiLU on the input, as in a
+    diffusion U-Net's res-block convs."""
     import spatially_sparse_incremental_b200 as sige
     xo, xe = L.x_orig.to(dev), L.x_edit.to(dev)
     wt, bias = L.weight.to(dev), L.bias.to(dev)
     N, Hi, Wi, ci = xo.shape
     co, k, st, b = wt.shape[0], L.kernel, L.stride, L.block
     cd = sige.conv_desc(k, st, L.pad, ci, co, b)
+    gs = gh = None
+    if gn:
+        g = torch.Generator().manual_seed(ci * 7 + co)
+        gs = (1.0 + 0.3 * torch.randn((N, ci), generator=g)).float().to(dev)
+        gh = (0.1 * torch.randn((N, ci), generator=g)).float().to(dev)
     y0 = sige.sige_dense_conv(xo, wt, bias, cd)
     Ho, Wo = y0.shape[1], y0.shape[2]
     cap = -(-Ho // b) * -(-Wo // b)
@@ -574,11 +593,12 @@ def layer_timing(L, bits, dev, flush, stream, peaks, reps=30, dense_us=None):
     y = y0.clone()
     ws = sige.zeros_workspace(sige.sige_conv_workspace_bytes(cd, N, cap, Ho, Wo), dev)
     yd = torch.empty_like(y0)
-    g_sp = capture(lambda: sige.sige_conv_fused(xe, wt, bias, cd, idx, cnt, cap, y, workspace=ws, stream=stream),
-                   stream)
+    g_sp = capture(lambda: sige.sige_conv_fused(xe, wt, bias, cd, idx, cnt, cap, y, gs, gh, silu=gn, workspace=ws,
+                                                stream=stream), stream)
     t_sp = float(np.median(time_graph(g_sp, flush, reps, stream))) * 1e3
     if dense_us is None:
-        g_de = capture(lambda: sige.sige_dense_conv(xe, wt, bias, cd, y=yd, workspace=ws, stream=stream), stream)
+        g_de = capture(lambda: sige.sige_dense_conv(xe, wt, bias, cd, y=yd, gn_scale=gs, gn_shift=gh, silu=gn,
+                                                    workspace=ws, stream=stream), stream)
         t_de = float(np.median(time_graph(g_de, flush, reps, stream))) * 1e3
         del g_de
     else:

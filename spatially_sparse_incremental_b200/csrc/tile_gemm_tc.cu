@@ -658,7 +658,8 @@ __global__ void __launch_bounds__(tg::kThreads, 1)
 
 // ------------------------------------------------------------------ input transform pre-pass
 
-// For a 3x3 layer with an input transform (GroupNorm affine, SiLU): the
+// For a 3x3 layer with an input transform (GroupNorm affine, SiLU, or the
+// GauGAN-style per-pixel modulation and LeakyReLU): the
 // transform of every input pixel the listed tiles' taps read (the halo of
 // each tile, or the whole map for a dense call) is written once into a
 // scratch copy of the input, which the GEMM then reads untransformed, instead
@@ -673,6 +674,8 @@ struct PreArgs {
     int32_t N, H, W, Cin, b, s, pad, hb;   // hb: halo side (b - 1) s + 3
     const float *gsc, *gsh;
     int32_t silu;
+    const uint8_t *sg, *sb;    // per-pixel modulation maps (input shape, NHWC bf16) or null
+    int32_t leaky;             // LeakyReLU(0.2) instead of SiLU
     UDiv dvpp, dhb, dN, dW, dH;
 };
 
@@ -712,9 +715,17 @@ __global__ void __launch_bounds__(256) k_tile_pretransform(const __grid_constant
         }
         const int64_t e = (((int64_t)n * p.H + y) * p.W + x) * p.Cin + (int64_t)cv * 8;
         const uint4 in = ld_nc16(p.x + e * 2);
-        reinterpret_cast<uint4 *>(p.xt)[e / 8] =
-            transform16(in, SIGE_BF16, p.gsc ? p.gsc + (int64_t)n * p.Cin + cv * 8 : nullptr,
-                        p.gsc ? p.gsh + (int64_t)n * p.Cin + cv * 8 : nullptr, p.silu);
+        const float *sc = p.gsc ? p.gsc + (int64_t)n * p.Cin + cv * 8 : nullptr;
+        const float *sh = p.gsc ? p.gsh + (int64_t)n * p.Cin + cv * 8 : nullptr;
+        uint4 out;
+        if (p.sg || p.leaky) {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            out = transform16_mod(in, sc, sh, p.sg != nullptr, p.sg ? ld_nc16(p.sg + e * 2) : z,
+                                  p.sb ? ld_nc16(p.sb + e * 2) : z, p.silu, p.leaky);
+        } else {
+            out = transform16(in, SIGE_BF16, sc, sh, p.silu);
+        }
+        reinterpret_cast<uint4 *>(p.xt)[e / 8] = out;
     }
 }
 
@@ -886,6 +897,9 @@ int launch_tile_gemm_pre(const ConvParams &cp, uint8_t *scratch, cudaStream_t st
     a.gsc = cp.gsc;
     a.gsh = cp.gsh;
     a.silu = cp.silu;
+    a.sg = cp.sg;
+    a.sb = cp.sb;
+    a.leaky = cp.leaky;
     a.dvpp = udiv_make((uint32_t)(cp.Cin / 8));
     a.dhb = udiv_make((uint32_t)a.hb);
     a.dN = udiv_make((uint32_t)cp.N);
@@ -907,6 +921,9 @@ int launch_tile_gemm_pre(const ConvParams &cp, uint8_t *scratch, cudaStream_t st
     g.gsc = nullptr;
     g.gsh = nullptr;
     g.silu = 0;
+    g.sg = nullptr;
+    g.sb = nullptr;
+    g.leaky = 0;
     return launch_tile_gemm(g, stream);
 }
 

@@ -64,6 +64,39 @@ __device__ __forceinline__ uint4 transform16_bf16_reg(uint4 in, const float (&sc
     return out;
 }
 
+// The GauGAN-style input transform of 8 bf16 channels of one pixel: the
+// GroupNorm-style affine (when sc), the per-pixel modulation t * (1 + g) + b
+// with g, b the same 8 channels of the modulation maps at that pixel (when
+// mod), then SiLU or LeakyReLU(0.2); one rounding to bf16.
+__device__ __forceinline__ uint4 transform16_mod(uint4 in, const float *sc, const float *sh, bool mod, uint4 g,
+                                                 uint4 b, int silu, int leaky)
+{
+    uint4 out;
+    uint32_t *o = reinterpret_cast<uint32_t *>(&out);
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(&in);
+    const uint32_t *gw = reinterpret_cast<const uint32_t *>(&g);
+    const uint32_t *bw = reinterpret_cast<const uint32_t *>(&b);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float v[2] = {bf16_lo(w[q]), bf16_hi(w[q])};
+        const float gg[2] = {bf16_lo(gw[q]), bf16_hi(gw[q])};
+        const float bb[2] = {bf16_lo(bw[q]), bf16_hi(bw[q])};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            if (sc)
+                v[e] = __fmaf_rn(v[e], __ldg(sc + 2 * q + e), __ldg(sh + 2 * q + e));
+            if (mod)
+                v[e] = __fmaf_rn(v[e], 1.0f + gg[e], bb[e]);
+            if (silu)
+                v[e] = silu_f(v[e]);
+            else if (leaky)
+                v[e] = v[e] >= 0.0f ? v[e] : 0.2f * v[e];
+        }
+        o[q] = pack_bf16x2(v[0], v[1]);
+    }
+    return out;
+}
+
 __device__ __forceinline__ float load_elem(const uint8_t *base, int64_t e, int dtype)
 {
     if (dtype == SIGE_BF16)

@@ -17,7 +17,7 @@ int launch_conv8(const ConvParams &p, cudaStream_t stream);
 // 1x1 and 3x3 "same" stride-1 layers on any tile size: a GEMM over the
 // tiles' pixels, one tap-shifted copy of the tile per K chunk, K split across
 // a cluster when the units are few.
-bool tile_gemm_supported(const sige_conv_desc *cd, int dtype);
+bool tile_gemm_supported(const sige_conv_desc *cd, int dtype, bool dense);
 int launch_tile_gemm(const ConvParams &p, cudaStream_t stream);
 // A 3x3 layer with an input transform: the transform of the pixels its tiles
 // read, once, into `scratch` (tile_gemm_scratch_bytes), then the tile GEMM on

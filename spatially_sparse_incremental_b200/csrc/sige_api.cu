@@ -59,7 +59,7 @@ static int check_layer(const sige_conv_desc *cd, int dtype)
 // 0 = the CUDA-core kernel.
 static int choose_path(const sige_conv_desc *cd, int dtype)
 {
-    return tc_supported(cd, dtype) || tile_gemm_supported(cd, dtype) ? 1 : 0;
+    return tc_supported(cd, dtype) || tile_gemm_supported(cd, dtype, false) ? 1 : 0;
 }
 
 static size_t ws_need(const sige_conv_desc *cd, int batch, int ntiles)
@@ -87,7 +87,7 @@ static int run_conv(ConvParams &p, const sige_conv_desc *cd, void *ws, size_t ws
     const bool plain = image && !p.sg && !p.leaky;
     if (plain && conv8_supported(cd, p.dtype))
         return launch_conv8(p, st);
-    if (image && tile_gemm_supported(cd, p.dtype)) {
+    if (image && tile_gemm_supported(cd, p.dtype, p.dense != 0)) {
         if (plain && (cd->kernel == 1 || (!p.gsc && !p.silu)))
             return launch_tile_gemm(p, st);
         // a 3x3 layer with an input transform: the transform once per pixel
@@ -122,7 +122,7 @@ extern "C" size_t sige_conv_workspace_bytes(const sige_conv_desc *cd, int32_t ba
     size_t need = std::max(ws_need(cd, batch, n), ws_need(&v, batch, n));
     // the tile GEMM's scratch copy of a transformed input (3x3 layers; sized
     // from the output dimensions, so only when they are given)
-    if (tile_gemm_supported(cd, SIGE_BF16) && cd->kernel == 3 && out_h > 0 && out_w > 0)
+    if (tile_gemm_supported(cd, SIGE_BF16, true) && cd->kernel == 3 && out_h > 0 && out_w > 0)
         need = ((ws_need(cd, batch, n) + 255) & ~(size_t)255) +
                tile_gemm_scratch_bytes(cd, batch, out_h * cd->stride + cd->kernel, out_w * cd->stride + cd->kernel);
     return std::max(need, std::max(ws_need(cd, batch, n), ws_need(&v, batch, n)));

@@ -731,7 +731,7 @@ __global__ void __launch_bounds__(256) k_tile_pretransform(const __grid_constant
 
 // ------------------------------------------------------------------ host
 
-bool tile_gemm_supported(const sige_conv_desc *cd, int dtype)
+bool tile_gemm_supported(const sige_conv_desc *cd, int dtype, bool dense)
 {
     if (!cd || dtype != SIGE_BF16 || cd->stride < 1 || cd->stride > 2 || cd->block < 1 ||
         cd->block * cd->block > tg::kRows ||
@@ -740,11 +740,12 @@ bool tile_gemm_supported(const sige_conv_desc *cd, int dtype)
     if ((long long)cd->kernel * cd->kernel * cd->c_in >= (1ll << 31))
         return false;
     // 1x1 stride 1 (any tile size), or 3x3 padding 1, stride 1 or 2, on 4x4
-    // or 8x8 tiles, whose tap-shifted (and strided) boxes the TMA fills (the
-    // CUDA-core copies of other tile sizes cannot keep a 3x3 layer's K loop
-    // fed)
+    // or 8x8 tiles, whose tap-shifted (and strided) boxes the TMA fills.  On
+    // other tile sizes the rows are copied per thread: a dense call (every
+    // tile, many units) still gains (2.1x on the 1x1 / 2x2-tile layers), a
+    // sparse one of few tiles measured no better than the general kernel.
     return (cd->kernel == 1 && cd->pad == 0 && cd->stride == 1) ||
-           (cd->kernel == 3 && cd->pad == 1 && (cd->block * cd->block) % 8 == 0);
+           (cd->kernel == 3 && cd->pad == 1 && (dense || (cd->block * cd->block) % 8 == 0));
 }
 
 int launch_tile_gemm(const ConvParams &cp, cudaStream_t stream)

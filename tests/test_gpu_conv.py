@@ -456,8 +456,12 @@ def test_tile_gemm_3x3_stride2(orc, H, W, ci, co, b, N, gn, res, area):
 
 
 @pytest.mark.parametrize("H,W,ci,co,b,N,gn", [(28, 36, 64, 64, 4, 1, False), (30, 26, 128, 80, 4, 2, False),
-                                               (18, 14, 128, 48, 2, 2, True)])
+                                               (18, 14, 128, 48, 2, 2, True), (13, 11, 64, 32, 1, 1, False),
+                                               (20, 17, 64, 48, 3, 2, False)])
 def test_tile_gemm_3x3_dense(orc, H, W, ci, co, b, N, gn):
+    """Every tile through sige_dense_conv: the tile GEMM (TMA boxes for 4x4
+    tiles, per-thread row copies for 1x1, 2x2 and 3x3 tiles; GN + SiLU through
+    the transform pre-pass)."""
     L = inputs.make_conv_case(120 + H + co, H, W, ci, co, dtype=torch.bfloat16, block=b, gn=gn, N=N)
     g, gs, gh = _gn(orc, L)
     r = random_cache((N, H, W, co), torch.bfloat16, 5)

@@ -82,20 +82,24 @@ static int run_conv(ConvParams &p, const sige_conv_desc *cd, void *ws, size_t ws
     if (ntiles == 0)
         return SIGE_OK;
     // image to image: the 8x8-tile kernel (no GauGAN extension) or the tile
-    // GEMM when they fit
-    const bool image = p.from_image && p.to_y && !p.tstride;
-    const bool plain = image && !p.sg && !p.leaky;
+    // GEMM when they fit (a transposed conv with an input transform: the
+    // general kernel)
+    const bool image = p.from_image && p.to_y;
+    const bool plain = image && !p.tstride && !p.sg && !p.leaky;
+    const bool xform = p.gsc || p.silu || p.sg || p.leaky;
     if (plain && conv8_supported(cd, p.dtype))
         return launch_conv8(p, st);
     if (image && tile_gemm_supported(cd, p.dtype, p.dense != 0)) {
-        if (plain && (cd->kernel == 1 || (!p.gsc && !p.silu)))
+        // no transform (transposed convs included: rows copied per thread),
+        // or a 1x1 layer's GroupNorm / SiLU applied in the GEMM
+        if (!xform || (plain && cd->kernel == 1))
             return launch_tile_gemm(p, st);
         // a 3x3 layer with an input transform: the transform once per pixel
         // into a scratch copy in the workspace (transforming every tap's copy
         // of a row measured 1.7-3.9x slower than the general kernel), when the
         // workspace was sized by sige_conv_workspace_bytes
         const size_t base = (ws_need(cd, p.N, ntiles) + 255) & ~(size_t)255;
-        if (cd->kernel == 3 && ws_bytes >= base + tile_gemm_scratch_bytes(cd, p.N, p.H, p.W))
+        if (!p.tstride && cd->kernel == 3 && ws_bytes >= base + tile_gemm_scratch_bytes(cd, p.N, p.H, p.W))
             return launch_tile_gemm_pre(p, p.ws + base, st);
     }
     if (tc_supported(cd, p.dtype))

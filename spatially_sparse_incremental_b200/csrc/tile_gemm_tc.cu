@@ -89,6 +89,8 @@ struct Args {
     int32_t cap, dense, tiles_w, tiles_total;
     int32_t N, H, W, Cin, Cout, b;   // H, W: the input map
     int32_t k, pad, s;         // kernel size, padding, stride
+    int32_t tstride;           // > 0: a transposed conv run as a stride-1 conv over the input with
+                               // tstride - 1 zeros between pixels, taps reversed (rows copied per thread)
     int32_t Ho, Wo;            // the output map
     int32_t nt, ntn;           // output channels per unit, units along C_out
     const float *gsc, *gsh;    // GroupNorm affine [N][Cin] (or null)
@@ -315,14 +317,17 @@ __global__ void __launch_bounds__(tg::kThreads, 1)
         bool ok = true;
         for (int u = u_first; ok && u < units; u += u_step) {
             const int nt = u % p.ntn;
-            for (int q = c_lo; q < c_hi; ++q, ++it) {
+            TapPos tp = tap_at(c_lo, kcin, p.k, p.pad);
+            for (int q = c_lo; q < c_hi; ++q, ++it, tap_next(tp, kcin, p.k, p.pad)) {
                 const int st = it % kWStages;
                 if (it >= kWStages &&
                     !mbar_wait_w(w_empty(st), ((it / kWStages) & 1) ^ 1, abort_flag, hdr, kSiteWEmpty)) {
                     ok = false;
                     break;
                 }
-                tma_load_2d_w(sb + kOffW + st * kWBytes, &tw, w_full(st), bytes, q * 64, nt * p.nt);
+                // (a transposed conv reads its taps in reverse order)
+                const int wq = p.tstride ? (p.k * p.k - 1 - ((tp.dr + p.pad) * p.k + tp.dc + p.pad)) * kcin + tp.cc : q;
+                tma_load_2d_w(sb + kOffW + st * kWBytes, &tw, w_full(st), bytes, wq * 64, nt * p.nt);
             }
         }
         cluster_wait();
@@ -436,7 +441,24 @@ __global__ void __launch_bounds__(tg::kThreads, 1)
             // the slot's pixel shifted by a chunk's tap; false outside the map
             // (a zero row: the conv's padding)
             auto tap_in = [&](const TapPos &t, int64_t &ipix) -> bool {
-                const int yi = yy * p.s + t.dr, xi = xx * p.s + t.dc;
+                int yi = yy * p.s + t.dr, xi = xx * p.s + t.dc;
+                if (p.tstride > 0) {
+                    // the virtual input holds x[y / t][x / t] where both are
+                    // multiples of t, zero elsewhere
+                    if (yi < 0 || xi < 0)
+                        return false;
+                    if (p.tstride == 2) {
+                        if ((yi | xi) & 1)
+                            return false;
+                        yi >>= 1;
+                        xi >>= 1;
+                    } else {
+                        if (yi % p.tstride || xi % p.tstride)
+                            return false;
+                        yi /= p.tstride;
+                        xi /= p.tstride;
+                    }
+                }
                 ipix = ((int64_t)n * p.H + yi) * p.W + xi;
                 return valid && yi >= 0 && yi < p.H && xi >= 0 && xi < p.W;
             };
@@ -768,6 +790,7 @@ int launch_tile_gemm(const ConvParams &cp, cudaStream_t stream)
     a.H = cp.H;
     a.W = cp.W;
     a.s = cp.s;
+    a.tstride = cp.tstride;
     a.Ho = cp.Ho;
     a.Wo = cp.Wo;
     a.Cin = cp.Cin;
@@ -815,7 +838,7 @@ int launch_tile_gemm(const ConvParams &cp, cudaStream_t stream)
     // or 8), so that every box starts on an atom.
     CUtensorMap tx = tw;
     a.tma_a = 0;
-    if ((cp.b * cp.b) % 8 == 0) {
+    if ((cp.b * cp.b) % 8 == 0 && cp.tstride == 0) {
         cuuint64_t xd[4] = {(cuuint64_t)cp.Cin, (cuuint64_t)cp.W, (cuuint64_t)cp.H, (cuuint64_t)cp.N};
         cuuint64_t xs[3] = {(cuuint64_t)cp.Cin * 2, (cuuint64_t)cp.W * cp.Cin * 2, (cuuint64_t)cp.H * cp.W * cp.Cin * 2};
         // (stride s: a box of b s pixels per side read every s-th pixel, b per side)

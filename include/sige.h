@@ -508,9 +508,11 @@ int sige_set_wait_cycles(int64_t cycles);
 /* Which conv kernel the fused and dense calls (sige_conv_fused,
  * sige_dense_conv) of this layer and dtype run: 1 = tcgen05 tensor cores (the
  * general tile kernel, the 8x8-tile 3x3 kernel, or the tile GEMM for bf16
- * layers with C_in % 64 == 0 and C_out % 16 == 0 that are 1x1 stride 1 on any
- * tile size, or 3x3 pad 1 stride 1 or 2 on 4x4 / 8x8 tiles without an input
- * transform), 0 = CUDA cores; negative = a
+ * layers with C_in % 64 == 0 and C_out % 16 == 0 that are 1x1 stride 1, or
+ * 3x3 pad 1 stride 1 or 2 on 4x4 / 8x8 tiles (any tile size for a dense call,
+ * one-pixel tiles too for a sparse one; an input transform through a
+ * pre-pass into the workspace when sige_conv_workspace_bytes sized it with
+ * the output dimensions)), 0 = CUDA cores; negative = a
  * sige_status for an unsupported layer.  sige_sparse_conv (stacked blocks)
  * takes the general tile kernel or the CUDA cores. */
 int sige_conv_path(const sige_conv_desc *cd, int32_t dtype);

@@ -745,7 +745,18 @@ __global__ void __launch_bounds__(256) k_tile_pretransform(const __grid_constant
             out = transform16_mod(in, sc, sh, p.sg != nullptr, p.sg ? ld_nc16(p.sg + e * 2) : z,
                                   p.sb ? ld_nc16(p.sb + e * 2) : z, p.silu, p.leaky);
         } else {
-            out = transform16(in, SIGE_BF16, sc, sh, p.silu);
+            // the 8 channels' scale and shift by four 16-byte loads (8 scalar
+            // loads each throttled the memory pipe)
+            float gsc8[8], gsh8[8];
+            if (sc) {
+                const float4 a0 = __ldg(reinterpret_cast<const float4 *>(sc)), a1 = __ldg(reinterpret_cast<const float4 *>(sc) + 1);
+                const float4 b0 = __ldg(reinterpret_cast<const float4 *>(sh)), b1 = __ldg(reinterpret_cast<const float4 *>(sh) + 1);
+                gsc8[0] = a0.x; gsc8[1] = a0.y; gsc8[2] = a0.z; gsc8[3] = a0.w;
+                gsc8[4] = a1.x; gsc8[5] = a1.y; gsc8[6] = a1.z; gsc8[7] = a1.w;
+                gsh8[0] = b0.x; gsh8[1] = b0.y; gsh8[2] = b0.z; gsh8[3] = b0.w;
+                gsh8[4] = b1.x; gsh8[5] = b1.y; gsh8[6] = b1.z; gsh8[7] = b1.w;
+            }
+            out = transform16_bf16_reg(in, gsc8, gsh8, sc != nullptr, p.silu);
         }
         reinterpret_cast<uint4 *>(p.xt)[e / 8] = out;
     }
@@ -936,7 +947,10 @@ int launch_tile_gemm_pre(const ConvParams &cp, uint8_t *scratch, cudaStream_t st
                                   : (int64_t)cp.cap * cp.N * a.hb * a.hb * (cp.Cin / 8);
     if (work > 0xFFFFFFFFll)
         return SIGE_ERR_UNSUPPORTED;
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, (int64_t)device_sm_count() * 8));
+    // (a sparse call's grid is sized for the capacity; its tiles are read on
+    // the device, usually far fewer)
+    const int grid = (int)std::max<int64_t>(
+        1, std::min<int64_t>((work + 255) / 256, (int64_t)device_sm_count() * (cp.dense ? 8 : 2)));
     if (launch_pdl(k_tile_pretransform, dim3(grid), dim3(256), 0, stream, a) != cudaSuccess)
         return SIGE_ERR_CUDA;
     count_launch();
